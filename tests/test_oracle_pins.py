@@ -1,0 +1,411 @@
+"""Pins of the CPU oracle to facts that do not come from the oracle itself.
+
+Each test checks the oracle against something the reviewed pages or mathematics
+fix: hand-worked values (tests/golden), closed forms of the Load Imbalance Score
+(R&Q Definition 1), library routines computing the same thing by another route
+(numpy lexsort / stable argsort / bincount, scipy softmax, torch fp64 matmuls),
+invariants, and a brute-force dense-masked evaluation. A plausible slip in the
+oracle (dropped bias, wrong tie-break, missing renormalisation, unstable
+permutation, transposed weight, missing SiLU or up factor, shared branch lost,
+wrong LIS formula) fails at least one of them; test_oracle_mutations.py plants
+such slips in a copy of the oracle and checks exactly that.
+"""
+import math
+import os
+from fractions import Fraction
+
+import numpy as np
+import pytest
+import scipy.special
+import torch
+
+import oracle as O
+import workloads as W
+
+pytestmark = pytest.mark.filterwarnings("ignore::DeprecationWarning")
+
+
+def _golden(path):
+    rows = []
+    with open(path) as fh:
+        for line in fh:
+            line = line.strip()
+            if not line or line.startswith("#"):
+                continue
+            rows.append([c.strip() for c in line.split("|")])
+    return rows
+
+
+def _t64(a, dtype):
+    return torch.from_numpy(np.asarray(W.as_f32(a, dtype), dtype=np.float64))
+
+
+# ------------------------------------------------------------------------- LIS
+
+def test_lis_golden_cases(golden_dir):
+    for name, m, k, routing, counts, mx, am, lis in _golden(os.path.join(golden_dir, "lis_cases.txt")):
+        m, k = int(m), int(k)
+        idx = np.array([[int(e) for e in tok.split(",")] for tok in routing.split(";")], dtype=np.int32)
+        assert idx.shape[1] == k, name
+        r = O.histogram_lis(idx, m)
+        assert r["counts"].tolist() == [int(c) for c in counts.split(",")], name
+        assert r["max_count"] == int(mx) and r["argmax"] == int(am), name
+        assert r["lis"] == float(Fraction(lis)), name
+
+
+def _favouring_logits(T, m, k, pick):
+    """Logits where token t's slot s clearly prefers expert pick(t, s)."""
+    lg = np.zeros((T, m), dtype=np.float32)
+    for t in range(T):
+        for s in range(k):
+            lg[t, pick(t, s)] = np.float32(10.0 - s)
+    return lg
+
+
+def test_lis_balanced_construction_is_one():
+    # (t*k + s) mod m with T*k divisible by m gives every expert T*k/m tasks -> LIS = 1
+    T, m, k = 64, 8, 2
+    idx, _ = O.topk_softmax(_favouring_logits(T, m, k, lambda t, s: (t * k + s) % m), k, False)
+    r = O.histogram_lis(idx, m)
+    assert set(r["counts"].tolist()) == {T * k // m}
+    assert r["lis"] == 1.0
+
+
+def test_lis_all_tokens_same_experts_is_maximum():
+    T, m, k = 50, 16, 4
+    idx, _ = O.topk_softmax(_favouring_logits(T, m, k, lambda t, s: 3 + s), k, False)
+    r = O.histogram_lis(idx, m)
+    assert r["lis"] == m / k  # the largest value: n_j <= T
+    assert r["argmax"] == 3
+
+
+@pytest.mark.parametrize("c", [1, 7, 33, 64])
+def test_lis_constructed_max_count(c):
+    T, m, k = 64, 8, 1
+    # the first c tokens go to expert 5, the rest spread round-robin over the other 7
+    others = [e for e in range(m) if e != 5]
+    pick = lambda t, s: 5 if t < c else others[t % len(others)]
+    idx, _ = O.topk_softmax(_favouring_logits(T, m, k, pick), k, False)
+    counts = np.bincount(idx.ravel(), minlength=m)
+    r = O.histogram_lis(idx, m)
+    assert r["lis"] == m * counts.max() / (T * k)
+    if c > (T - c) / 7 + 1:
+        assert r["argmax"] == 5 and r["max_count"] == c
+
+
+def test_lis_bounds_and_counts_random():
+    rng = np.random.default_rng(0)
+    for _ in range(20):
+        T, m = int(rng.integers(1, 300)), int(rng.integers(2, 40))
+        k = int(rng.integers(1, m + 1))
+        lg = rng.standard_normal((T, m)).astype(np.float32)
+        idx, _ = O.topk_softmax(lg, k, False)
+        r = O.histogram_lis(idx, m)
+        np.testing.assert_array_equal(r["counts"], np.bincount(idx.ravel(), minlength=m))
+        np.testing.assert_array_equal(r["offsets"], np.concatenate([[0], np.cumsum(r["counts"])]))
+        assert r["counts"].sum() == T * k
+        assert 1.0 - 1e-12 <= r["lis"] <= m / k + 1e-12
+
+
+def test_histogram_rejects_out_of_range_ids():
+    with pytest.raises(ValueError):
+        O.histogram_lis(np.array([[0], [4]], dtype=np.int32), 4)
+    with pytest.raises(ValueError):
+        O.histogram_lis(np.array([[-1], [1]], dtype=np.int32), 4)
+
+
+# --------------------------------------------------------------- top-k, softmax
+
+def _parse_logit(s):
+    return np.float32(math.log(float(s[3:]))) if s.startswith("ln:") else np.float32(float(s))
+
+
+def test_topk_golden(golden_dir):
+    for name, k, rn, logits, idx, wts in _golden(os.path.join(golden_dir, "topk_cases.txt")):
+        lg = np.array([[_parse_logit(v) for v in logits.split(",")]], dtype=np.float32)
+        i, w = O.topk_softmax(lg, int(k), bool(int(rn)))
+        assert i[0].tolist() == [int(v) for v in idx.split(",")], name
+        np.testing.assert_allclose(w[0], [float(Fraction(v)) for v in wts.split(",")], rtol=1e-6, err_msg=name)
+
+
+def test_topk_matches_lexsort_with_many_ties():
+    rng = np.random.default_rng(1)
+    for m in (2, 7, 8, 64, 128):
+        T = 200
+        lg = (rng.integers(-3, 4, size=(T, m)) * 0.5).astype(np.float32)  # heavy ties
+        for k in sorted({1, 2, min(6, m), m}):
+            idx, _ = O.topk_softmax(lg, k, False)
+            for t in range(T):
+                order = np.lexsort((np.arange(m), -lg[t].astype(np.float64)))
+                assert idx[t].tolist() == order[:k].tolist()
+
+
+def test_constant_logits_pick_first_k():
+    idx, w = O.topk_softmax(np.zeros((3, 9), np.float32), 4, False)
+    assert idx.tolist() == [[0, 1, 2, 3]] * 3
+    np.testing.assert_allclose(w, 1.0 / 9.0, rtol=1e-15)
+
+
+@pytest.mark.parametrize("renorm", [False, True])
+def test_gate_weights_vs_scipy_softmax(renorm):
+    rng = np.random.default_rng(2)
+    lg = (rng.standard_normal((300, 64)) * 3).astype(np.float32)
+    idx, w = O.topk_softmax(lg, 6, renorm)
+    p = scipy.special.softmax(lg.astype(np.float64), axis=1)
+    sel = np.take_along_axis(p, idx.astype(np.int64), axis=1)
+    if renorm:
+        sel = sel / sel.sum(axis=1, keepdims=True)
+        np.testing.assert_allclose(w.sum(axis=1), 1.0, rtol=1e-14)
+    np.testing.assert_allclose(w, sel, rtol=1e-12)
+
+
+def test_top1_weight_closed_form():
+    rng = np.random.default_rng(3)
+    lg = rng.standard_normal((100, 16)).astype(np.float32)
+    idx, w = O.topk_softmax(lg, 1, False)
+    for t in range(100):
+        e = idx[t, 0]
+        others = np.delete(lg[t].astype(np.float64), e)
+        assert w[t, 0] == pytest.approx(1.0 / (1.0 + np.exp(others - lg[t, e]).sum()), rel=1e-13)
+
+
+# -------------------------------------------------------------------- router
+
+@pytest.mark.parametrize("dtype", [W.F32, W.BF16])
+def test_router_logits_vs_torch_fp64(dtype):
+    cfg = W.small_moe(T=33, d=96, f=32, m=12, k=2, dtype=dtype, zipf_s=1.0)
+    inp = W.make_moe_inputs(cfg, weights=False)
+    got = O.router_logits(inp["x"], inp["w_router"], inp["bias"])
+    ref = (_t64(inp["x"], dtype) @ _t64(inp["w_router"], dtype).T + torch.from_numpy(
+        inp["bias"].astype(np.float64))).float().numpy()
+    # both are fp64 sums rounded once to fp32; summation order may move a tie by one ulp
+    np.testing.assert_array_max_ulp(got, ref, maxulp=1)
+    assert (got == ref).mean() > 0.99
+    assert np.any(inp["bias"] != 0)
+
+
+def test_zipf_bias_shape():
+    b = W.zipf_bias(16, 1.1, 0.5, seed=123)
+    r = np.sort(-b)  # ranks 1..m in increasing -bias order
+    np.testing.assert_allclose(r, [0.5 * 1.1 * math.log(i) for i in range(1, 17)], rtol=1e-6)
+    assert len(set(np.argsort(-b).tolist())) == 16
+
+
+# --------------------------------------------------------------- permutation
+
+def test_permutation_is_stable_argsort_by_expert():
+    rng = np.random.default_rng(4)
+    for m, k in ((8, 2), (128, 1), (64, 6), (3, 3)):
+        T = 257
+        lg = rng.standard_normal((T, m)).astype(np.float32)
+        idx, _ = O.topk_softmax(lg, k, False)
+        r = O.histogram_lis(idx, m)
+        perm, inv = O.permutation(idx, m, r["offsets"])
+        np.testing.assert_array_equal(perm, np.argsort(idx.ravel(), kind="stable"))
+        np.testing.assert_array_equal(perm[inv], np.arange(T * k))
+        np.testing.assert_array_equal(inv[perm], np.arange(T * k))
+        flat = idx.ravel()
+        for e in range(m):
+            seg = perm[r["offsets"][e]:r["offsets"][e + 1]]
+            assert np.all(flat[seg] == e)
+            assert np.all(np.diff(seg) > 0)
+
+
+# ----------------------------------------------------------------- expert FFN
+
+def _torch_ffn(x, wg, wu, wd, act):
+    a = x @ wg.T
+    h = torch.nn.functional.silu(a) * (x @ wu.T) if act == W.SWIGLU else torch.relu(a)
+    return h @ wd.T
+
+
+@pytest.mark.parametrize("act", [W.SWIGLU, W.RELU])
+@pytest.mark.parametrize("dtype", [W.F32, W.BF16])
+def test_single_expert_is_textbook_ffn(act, dtype):
+    # m = 1, k = 1: the layer is one dense FFN with weight 1
+    cfg = W.small_moe(T=9, d=64, f=80, m=1, k=1, act=act, dtype=dtype, zipf_s=0.0)
+    inp = W.make_moe_inputs(cfg)
+    r = O.layer_forward(cfg, inp)
+    assert np.all(r["idx"] == 0) and np.allclose(r["w"], 1.0)
+    t = lambda key: _t64(inp[key], dtype)
+    ref = _torch_ffn(t("x"), t("w_gate")[0], t("w_up")[0] if act == W.SWIGLU else None, t("w_down")[0], act)
+    np.testing.assert_allclose(r["out"], ref.numpy(), rtol=1e-10, atol=1e-12)
+
+
+@pytest.mark.parametrize("shared", [0, 2])
+@pytest.mark.parametrize("act", [W.SWIGLU, W.RELU])
+def test_dense_masked_equals_sparse(shared, act):
+    cfg = W.small_moe(T=12, d=32, f=48, m=6, k=2, act=act, dtype=W.BF16, zipf_s=1.0, n_shared=shared,
+                      f_shared=40 if shared else 0)
+    inp = W.make_moe_inputs(cfg)
+    r = O.layer_forward(cfg, inp)
+    np.testing.assert_allclose(O.dense_masked(cfg, inp, r["idx"], r["w"]), r["out"], rtol=1e-12, atol=1e-14)
+
+
+def test_full_mixture_when_k_equals_m():
+    cfg = W.small_moe(T=7, d=48, f=40, m=4, k=4, act=W.SWIGLU, dtype=W.BF16, zipf_s=1.0, renorm=True)
+    inp = W.make_moe_inputs(cfg)
+    r = O.layer_forward(cfg, inp)
+    t = lambda key: _t64(inp[key], W.BF16)
+    p = torch.softmax(torch.from_numpy(r["logits"].astype(np.float64)), dim=1)
+    ref = sum(p[:, e:e + 1] * _torch_ffn(t("x"), t("w_gate")[e], t("w_up")[e], t("w_down")[e], W.SWIGLU)
+              for e in range(4))
+    np.testing.assert_allclose(r["out"], ref.numpy(), rtol=1e-10, atol=1e-12)
+
+
+def test_identical_experts_with_renorm_ignore_routing():
+    cfg = W.small_moe(T=10, d=32, f=24, m=5, k=3, act=W.SWIGLU, dtype=W.F32, zipf_s=1.0, renorm=True)
+    inp = W.make_moe_inputs(cfg)
+    for key in ("w_gate", "w_up", "w_down"):
+        inp[key][:] = inp[key][0:1]
+    r = O.layer_forward(cfg, inp)
+    t = lambda key: _t64(inp[key], W.F32)
+    ref = _torch_ffn(t("x"), t("w_gate")[0], t("w_up")[0], t("w_down")[0], W.SWIGLU)
+    np.testing.assert_allclose(r["out"], ref.numpy(), rtol=1e-10, atol=1e-12)
+
+
+def test_shared_experts_add_plain_ffns():
+    cfg = W.small_moe(T=6, d=32, f=24, m=4, k=2, act=W.SWIGLU, dtype=W.BF16, zipf_s=1.0, n_shared=2,
+                      f_shared=16)
+    inp = W.make_moe_inputs(cfg)
+    with_sh = O.layer_forward(cfg, inp)
+    cfg0 = W.small_moe(T=6, d=32, f=24, m=4, k=2, act=W.SWIGLU, dtype=W.BF16, zipf_s=1.0)
+    no_sh = O.layer_forward(cfg0, {k: v for k, v in inp.items() if not k.startswith("ws_")})
+    t = lambda key: _t64(inp[key], W.BF16)
+    shared = sum(_torch_ffn(t("x"), t("ws_gate")[s], t("ws_up")[s], t("ws_down")[s], W.SWIGLU) for s in range(2))
+    np.testing.assert_allclose(with_sh["out"] - no_sh["out"], shared.numpy(), rtol=1e-9, atol=1e-11)
+
+
+def test_sampled_tokens_match_full_output():
+    cfg = W.small_moe(T=20, d=32, f=24, m=4, k=2, act=W.RELU, dtype=W.BF16)
+    inp = W.make_moe_inputs(cfg)
+    r = O.layer_forward(cfg, inp)
+    tok = np.array([19, 0, 7, 7], np.int32)
+    np.testing.assert_array_equal(O.moe_output(cfg, inp, r["idx"], r["w"], tokens=tok), r["out"][tok])
+
+
+# -------------------------------------------------------------- atomic experts
+
+def _small_atomic(T=3, d=64, Nr=16, Nc=12, K=8, act=W.ACT_SILU):
+    return W.AtomicWorkload("atomic_small", 91, T=T, d=d, Nr=Nr, Nc=Nc, K=K, act=act)
+
+
+def test_atomic_logprobs_vs_torch():
+    cfg = _small_atomic()
+    inp = W.make_atomic_inputs(cfg)
+    lr, lc = O.atomic_logprobs(inp["x"], inp["w_row"], inp["w_col"])
+    x = _t64(inp["x"], W.BF16)
+    rr = torch.log_softmax(x @ _t64(inp["w_row"], W.BF16).T, dim=1).float().numpy()
+    rc = torch.log_softmax(x @ _t64(inp["w_col"], W.BF16).T, dim=1).float().numpy()
+    np.testing.assert_array_max_ulp(lr, rr, maxulp=1)
+    np.testing.assert_array_max_ulp(lc, rc, maxulp=1)
+
+
+def _lexsort_topk(lr, lc, K):
+    S = (lr[:, None] + lc[None, :]).astype(np.float32).ravel()  # fp32 sums, row-major flat id
+    order = np.lexsort((np.arange(S.size), -S.astype(np.float64)))
+    return order[:K], S
+
+
+def test_atomic_select_vs_lexsort():
+    rng = np.random.default_rng(5)
+    for trial in range(6):
+        Nr, Nc, K = 9, 13, 10
+        lr = (rng.integers(-4, 1, size=(2, Nr)) * 0.25).astype(np.float32)  # many ties
+        lc = (rng.integers(-4, 1, size=(2, Nc)) * 0.25).astype(np.float32)
+        if trial % 2:
+            lr += rng.standard_normal((2, Nr)).astype(np.float32)
+        idx, g = O.atomic_select(lr, lc, K)
+        for t in range(2):
+            order, S = _lexsort_topk(lr[t], lc[t], K)
+            assert idx[t].tolist() == order.tolist()
+            np.testing.assert_allclose(g[t], scipy.special.softmax(S[order].astype(np.float64)), rtol=1e-12)
+
+
+def test_atomic_gates_are_renormalised_product_of_factors():
+    # OmniMoE Eq. 8: p(i,j|x) ~ p_r(i|x) p_c(j|x); softmax over the selected
+    # S = log p_r + log p_c is the product renormalised over the selection.
+    cfg = _small_atomic(T=2, Nr=32, Nc=32, K=16)
+    inp = W.make_atomic_inputs(cfg, experts=False)
+    lr, lc = O.atomic_logprobs(inp["x"], inp["w_row"], inp["w_col"])
+    idx, g = O.atomic_select(lr, lc, cfg.K)
+    for t in range(2):
+        pr, pc = np.exp(lr[t].astype(np.float64)), np.exp(lc[t].astype(np.float64))
+        prod = pr[idx[t] // cfg.Nc] * pc[idx[t] % cfg.Nc]
+        np.testing.assert_allclose(g[t], prod / prod.sum(), rtol=2e-6)  # S is rounded to fp32
+        assert np.all(np.diff(g[t]) <= 0)
+
+
+@pytest.mark.parametrize("act", [W.ACT_SILU, W.ACT_SIGMOID])
+def test_atomic_output_vs_torch(act):
+    cfg = _small_atomic(act=act)
+    inp = W.make_atomic_inputs(cfg)
+    lr, lc = O.atomic_logprobs(inp["x"], inp["w_row"], inp["w_col"])
+    idx, g = O.atomic_select(lr, lc, cfg.K)
+    out = O.atomic_output(inp["x"], inp["w_in"], inp["w_out"], idx, g, act)
+    x = _t64(inp["x"], W.BF16)
+    wi, wo = _t64(inp["w_in"], W.BF16), _t64(inp["w_out"], W.BF16)
+    z = (x[:, None, :] * wi[torch.from_numpy(idx.astype(np.int64))]).sum(-1)
+    a = torch.nn.functional.silu(z) if act == W.ACT_SILU else torch.sigmoid(z)
+    ref = ((torch.from_numpy(g) * a)[:, :, None] * wo[torch.from_numpy(idx.astype(np.int64))]).sum(1)
+    np.testing.assert_allclose(out, ref.numpy(), rtol=1e-10, atol=1e-12)
+
+
+# ---------------------------------------- exactness of the grid top-K candidate method
+
+def grid_topk_threshold_method(lr, lc, K):
+    """The selection method the GPU kernel uses (restated here in plain Python):
+    candidates = top-K rows x top-K cols (each by value desc, index asc); tau =
+    the K-th best candidate score; every pair scoring above tau lies inside the
+    candidate block, so the answer is those plus the first (in flat-id order)
+    pairs of the whole grid that score exactly tau."""
+    Nr, Nc = len(lr), len(lc)
+    rows = sorted(range(Nr), key=lambda i: (-float(lr[i]), i))[:min(K, Nr)]
+    cols = sorted(range(Nc), key=lambda j: (-float(lc[j]), j))[:min(K, Nc)]
+    cand = sorted(((np.float32(lr[i]) + np.float32(lc[j]), i * Nc + j) for i in rows for j in cols),
+                  key=lambda p: (-float(p[0]), p[1]))
+    tau = cand[K - 1][0]
+    above = [p for p in cand if p[0] > tau]
+    need, tied = K - len(above), []
+    for q in range(Nr * Nc):
+        if len(tied) == need:
+            break
+        s = np.float32(lr[q // Nc]) + np.float32(lc[q % Nc])
+        if s == tau:
+            tied.append((s, q))
+    return [q for _, q in sorted(above + tied, key=lambda p: (-float(p[0]), p[1]))]
+
+
+def _collapse_case():
+    # rows 1 and 2 beat row 0 by less than half an ulp of the sum, so all three
+    # sums with column 0 round to the same fp32 value; flat id then decides.
+    lr = np.array([-1.0, np.nextafter(np.float32(-1.0), np.float32(0)),
+                   np.nextafter(np.float32(-1.0), np.float32(0)), -50.0], np.float32)
+    lc = np.array([-8.0, -100.0, -100.0, -100.0], np.float32)
+    return lr, lc
+
+
+def test_grid_topk_method_exact_on_adversarial_grids():
+    rng = np.random.default_rng(6)
+    cases = [_collapse_case(), (np.zeros(8, np.float32), np.zeros(8, np.float32))]
+    for _ in range(40):
+        Nr, Nc = int(rng.integers(1, 12)), int(rng.integers(1, 12))
+        q = rng.choice([0.25, 1e-7, 0.0])
+        lr = (rng.integers(-3, 1, Nr) * q + rng.standard_normal(Nr) * (q == 1e-7) * 1e-7 - 5).astype(np.float32)
+        lc = (rng.integers(-3, 1, Nc) * q - 7).astype(np.float32)
+        cases.append((lr, lc))
+    for lr, lc in cases:
+        for K in sorted({1, 2, min(5, lr.size * lc.size), lr.size * lc.size}):
+            idx, _ = O.atomic_select(lr[None], lc[None], K)
+            assert grid_topk_threshold_method(lr, lc, K) == idx[0].tolist()
+
+
+def test_plain_candidate_block_is_not_always_exact():
+    # Selecting only inside top-K rows x top-K cols misses (0, 0) here: the
+    # rounding of the fp32 sums ties it with rows 1 and 2, and it has the lowest id.
+    lr, lc = _collapse_case()
+    K = 2
+    idx, _ = O.atomic_select(lr[None], lc[None], K)
+    assert idx[0].tolist() == [0, 4]
+    rows = sorted(range(4), key=lambda i: (-float(lr[i]), i))[:K]
+    assert 0 not in rows
