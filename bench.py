@@ -1,0 +1,464 @@
+#!/usr/bin/env python
+"""Benchmark of the sparse-MoE layer forward (moe_layer_forward) on B200s.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--config NAME] [--impl ours|reference]
+
+One step = one moe_layer_forward (router -> top-k -> histogram/LIS/ranks ->
+permutation -> grouped expert GEMMs -> combine) over one batch of T tokens held
+in device memory. Multi-GPU runs (torchrun, one process per GPU) are data
+parallel: every rank holds the same expert weights and its own token batch, no
+collective touches the data path (weak scaling); the timing barrier and the
+max-over-ranks reduction are the only collectives.
+
+Prints ONE JSON line on rank 0. `value` = tokens/s of the whole job from CUDA
+events on the launching stream (L2 flushed between steps, outside the timed
+events); `e2e` = the same metric through the C-ABI call with the batch copied
+from pinned host memory and the output copied back inside the timed region;
+`roofline` = the dominant kernel's algorithmic bytes or flops per launch over its
+event-timed duration against the measured peaks; `cpu_baseline` = the CPU oracle
+timed on a bounded sample of the same workload on this host's cores.
+`--impl reference` times that oracle alone (the only other code path that exists).
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import hashlib
+import json
+import math
+import os
+import statistics
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+
+import workloads as W  # noqa: E402
+
+METRIC = "MoE-layer tokens/sec at 1 B200; grouped-GEMM TFLOPS and HBM GB/s as % of peak"
+UNIT = "tokens/s"
+STAGES = ["router", "topk", "histogram_lis_ranks", "permute", "expert_up", "expert_down", "combine"]
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+L2_FLUSH_BYTES = 256 << 20
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--config", default="switch", choices=[k for k, v in W.CONFIGS.items()
+                                                           if isinstance(v, W.MoEWorkload)])
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--cpu-seconds", type=float, default=12.0, help="CPU-oracle baseline budget (rank 0, N=1)")
+    ap.add_argument("--no-cpu-baseline", action="store_true", help="skip the CPU-oracle leg (for profiling runs)")
+    return ap.parse_args()
+
+
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as fh:
+            p = json.load(fh)
+        return {k: float(p[k]) for k in FALLBACK_PEAKS}, "measured"
+    except Exception:
+        return dict(FALLBACK_PEAKS), "fallback"
+
+
+def workload_config(cfg) -> dict:
+    return {"workload": cfg.name, "tokens": cfg.T, "d_model": cfg.d, "d_ff": cfg.f, "experts": cfg.m, "top_k": cfg.k,
+            "shared_experts": cfg.n_shared, "d_ff_shared": cfg.f_shared,
+            "ffn": "swiglu" if cfg.act == W.SWIGLU else "relu", "renormalised_gates": bool(cfg.renorm),
+            "router_bias_zipf_s": cfg.zipf_s, "description": cfg.note}
+
+
+# ------------------------------------------------------------------ CPU oracle baseline
+
+def cpu_oracle_sample(cfg, inp, budget_s: float):
+    """Time the oracle's full layer forward on the first n tokens, n sized to ~budget_s."""
+    import oracle as O
+
+    threads = os.cpu_count() or 1
+
+    def run(n):
+        sub = dict(inp)
+        sub["x"] = np.ascontiguousarray(inp["x"][:n])
+        t0 = time.perf_counter()
+        O.layer_forward(cfg, sub, nthreads=threads)
+        return time.perf_counter() - t0
+
+    n = 1
+    dt = run(n)
+    while dt < budget_s / 8 and n < cfg.T:
+        n = min(cfg.T, n * 4)
+        dt = run(n)
+    if dt < budget_s / 2 and n < cfg.T:
+        n = min(cfg.T, max(n + 1, int(n * budget_s / max(dt, 1e-6) * 0.8)))
+        dt = run(n)
+    return {"value": n / dt, "unit": UNIT, "cores": threads, "kind": "oracle", "seconds": round(dt, 3),
+            "sample": f"first {n} of {cfg.T} tokens of the {cfg.name} workload; every step of the layer "
+                      f"(router, top-k, histogram/LIS, permutation, expert FFNs, combine) in fp64 C, "
+                      f"{threads} threads over tokens"}
+
+
+def reference_arm(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    import oracle as O
+
+    cfg = W.CONFIGS[args.config]
+    inp = W.make_moe_inputs(cfg)
+    threads = os.cpu_count() or 1
+    per_step_budget = max(0.2, min(20.0, 150.0 / (args.steps + args.warmup)))
+    # size the sample so one step takes about per_step_budget seconds
+    n, dt = 1, 0.0
+    while True:
+        sub = dict(inp)
+        sub["x"] = np.ascontiguousarray(inp["x"][:n])
+        t0 = time.perf_counter()
+        O.layer_forward(cfg, sub, nthreads=threads)
+        dt = time.perf_counter() - t0
+        if dt >= per_step_budget / 4 or n >= cfg.T:
+            break
+        n = min(cfg.T, n * 4)
+    n = max(1, min(cfg.T, int(n * per_step_budget / max(dt, 1e-9)))) if n < cfg.T else n
+    sub = dict(inp)
+    sub["x"] = np.ascontiguousarray(inp["x"][:n])
+    for _ in range(args.warmup):
+        O.layer_forward(cfg, sub, nthreads=threads)
+    times = []
+    for _ in range(args.steps):
+        t0 = time.perf_counter()
+        O.layer_forward(cfg, sub, nthreads=threads)
+        times.append(time.perf_counter() - t0)
+    sec = sum(times) / len(times)
+    value = n / sec
+    sample = (f"first {n} of {cfg.T} tokens of the {cfg.name} workload per step; every step of the layer in fp64 C "
+              f"on {threads} host threads")
+    line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": sec * 1e3, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic (seeded generator)", "impl": "reference",
+            "config": dict(workload_config(cfg), parallelism="host threads", l2="n/a (CPU)"),
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": threads, "kind": "oracle", "sample": sample},
+            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ------------------------------------------------------------------ clocks (NVML, sampled during timing)
+
+REASONS = {0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap", 0x8: "hw_slowdown",
+           0x10: "sync_boost", 0x20: "sw_thermal_slowdown", 0x40: "hw_thermal_slowdown",
+           0x80: "hw_power_brake_slowdown", 0x100: "display_clock_setting"}
+
+
+class ClockSampler:
+    def __init__(self, device_index: int):
+        self.samples, self.masks, self.err = [], 0, None
+        self.h = None
+        try:
+            import pynvml
+            import torch
+
+            pynvml.nvmlInit()
+            self.nv = pynvml
+            try:
+                uuid = "GPU-" + str(torch.cuda.get_device_properties(device_index).uuid)
+                self.h = pynvml.nvmlDeviceGetHandleByUUID(uuid)
+            except Exception:
+                self.h = pynvml.nvmlDeviceGetHandleByIndex(device_index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+        except Exception as e:  # no NVML: report why
+            self.err = f"nvml unavailable: {e}"
+        self._stop = threading.Event()
+        self._t = None
+
+    def _one(self):
+        nv = self.nv
+        self.samples.append(nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM))
+        try:
+            self.masks |= nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+        except AttributeError:
+            self.masks |= nv.nvmlDeviceGetCurrentClocksThrottleReasons(self.h)
+
+    def _loop(self):
+        while not self._stop.is_set():
+            try:
+                self._one()
+            except Exception as e:
+                self.err = str(e)
+                return
+            time.sleep(0.004)
+
+    def start(self):
+        if self.h is not None:
+            self._t = threading.Thread(target=self._loop, daemon=True)
+            self._t.start()
+
+    def stop(self):
+        if self._t is not None:
+            self._stop.set()
+            self._t.join()
+            if not self.samples:
+                self._one()
+
+    def report(self):
+        if self.h is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "note": self.err}
+        reasons = sorted(name for bit, name in REASONS.items() if self.masks & bit and name != "gpu_idle")
+        return {"sm_mhz": float(statistics.median(self.samples)) if self.samples else None,
+                "sm_max_mhz": float(self.max_mhz), "reasons": reasons, "samples": len(self.samples)}
+
+
+# ------------------------------------------------------------------ algorithmic cost model
+
+def stage_costs(cfg, active: int, ksplit: int):
+    """Algorithmic flops and bytes per launch of each stage (operands read once,
+    results written once; weights of ACTIVE experts only)."""
+    es = 4 if cfg.dtype == W.F32 else 2
+    T, d, f, m, k = cfg.T, cfg.d, cfg.f, cfg.m, cfg.k
+    Tk = T * k
+    mats = 2 if cfg.act == W.SWIGLU else 1
+    nsh, fsh = cfg.n_shared, cfg.f_shared
+    c = {}
+    c["router"] = (2.0 * T * d * m, T * d * es + m * d * es + T * m * 4)
+    c["topk"] = (0.0, T * m * 4 + Tk * 8)
+    c["histogram_lis_ranks"] = (0.0, Tk * 4 + Tk * 8 + (m + 1) * 8)
+    c["permute"] = (0.0, Tk * 4 + T * d * es + Tk * d * es)
+    c["expert_up"] = (2.0 * mats * f * d * Tk + 2.0 * mats * fsh * d * T * nsh,
+                      active * mats * f * d * es + nsh * mats * fsh * d * es + Tk * d * es + (T * d * es if nsh else 0)
+                      + Tk * f * es + nsh * T * fsh * es)
+    c["expert_down"] = (2.0 * d * f * Tk + 2.0 * d * fsh * T * nsh,
+                        active * d * f * es + nsh * d * fsh * es + Tk * f * es + nsh * T * fsh * es
+                        + ksplit * Tk * d * 4 + nsh * T * d * 4)
+    c["combine"] = (0.0, ksplit * Tk * d * 4 + nsh * T * d * 4 + Tk * 4 + T * d * es)
+    layer_flops = 2.0 * T * d * m + c["expert_up"][0] + c["expert_down"][0]
+    layer_bytes = (m * d + active * (mats + 1) * f * d + nsh * (mats + 1) * fsh * d) * es + 2 * T * d * es
+    return c, layer_flops, layer_bytes
+
+
+def source_hash() -> str:
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "sparse_mixture_experts_08_b200", "csrc")
+    for name in sorted(os.listdir(csrc)):
+        with open(os.path.join(csrc, name), "rb") as fh:
+            h.update(name.encode() + fh.read())
+    return h.hexdigest()[:16]
+
+
+def traffic_for(workload: str, stage: str):
+    """dram bytes per launch from a committed ncu capture, if it matches the current source."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    try:
+        with open(path) as fh:
+            t = json.load(fh)
+        e = t[workload][stage]
+        return e["dram_bytes_per_launch"] if e.get("source_hash") == source_hash() else None
+    except Exception:
+        return None
+
+
+# ------------------------------------------------------------------ our arm
+
+def ours(args):
+    import torch
+    import torch.distributed as dist
+
+    import sparse_mixture_experts_08_b200 as moe
+
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world != args.gpus:
+        raise SystemExit(f"--gpus {args.gpus} needs {args.gpus} ranks (torchrun), found WORLD_SIZE={world}")
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=180), device_id=dev)
+
+    cfg = W.CONFIGS[args.config]
+    inp = W.make_moe_inputs(cfg, replicate=0)  # expert weights: identical on every rank
+    if rank:
+        inp["x"] = W.normal(cfg.seed(rank), W.STREAM["x"], (cfg.T, cfg.d), 1.0, cfg.dtype)
+
+    def to_dev(a):
+        if a.dtype == np.uint16:
+            return torch.from_numpy(a.view(np.int16)).to(dev).view(torch.bfloat16)
+        return torch.from_numpy(a).to(dev)
+
+    d_in = {k: to_dev(v) for k, v in inp.items()}
+    c = moe.make_config(cfg.T, cfg.d, cfg.f, cfg.m, cfg.k, cfg.n_shared, cfg.f_shared, cfg.dtype, cfg.act,
+                        cfg.renorm)
+    ws = moe.workspace(c, device=dev)
+    tdt = torch.float32 if cfg.dtype == W.F32 else torch.bfloat16
+    out = torch.empty((cfg.T, cfg.d), dtype=tdt, device=dev)
+    counts = torch.empty(cfg.m, dtype=torch.int32, device=dev)
+    lis = moe.lis_buffer(dev)
+    s = torch.cuda.Stream(device=dev)
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+
+    def fwd(x=None, o=None):
+        moe.moe_layer_forward(c, d_in["x"] if x is None else x, d_in["w_router"], d_in["bias"], d_in["w_gate"],
+                              d_in.get("w_up"), d_in["w_down"], d_in.get("ws_gate"), d_in.get("ws_up"),
+                              d_in.get("ws_down"), out if o is None else o, ws, counts_out=counts, lis_out=lis,
+                              stream=s)
+
+    with torch.cuda.stream(s):
+        n0 = moe.moe_launch_count()
+        fwd()
+        launches_per_step = moe.moe_launch_count() - n0
+        for _ in range(max(args.warmup, 3)):
+            flush.zero_()
+            fwd()
+    torch.cuda.synchronize(dev)
+    st = moe.moe_read_device_status(ws, stream=s)
+    if st != moe.OK:
+        raise RuntimeError(f"device status after warm-up: {moe.moe_status_string(st)}")
+    cnt = counts.cpu().numpy()
+    active = int((cnt > 0).sum())
+    max_count, argmax, lis_v = moe.unpack_lis(lis)
+    ent = cnt[cnt > 0] / cnt.sum()
+    entropy = float(-(ent * np.log(ent)).sum())
+
+    # ---- timed region: K steps, CUDA events on the launching stream, L2 flushed between steps
+    K = args.steps
+    ev_s = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
+    ev_e = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
+    ev_stage = [[torch.cuda.Event(enable_timing=True) for _ in range(8)] for _ in range(K)]
+    sampler = ClockSampler(local)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize(dev)
+    sampler.start()
+    with torch.cuda.stream(s):
+        for i in range(K):
+            flush.zero_()
+            moe.moe_set_stage_events(ev_stage[i])
+            ev_s[i].record(s)
+            fwd()
+            ev_e[i].record(s)
+    torch.cuda.synchronize(dev)
+    if world > 1:
+        dist.barrier()
+    sampler.stop()
+    moe.moe_set_stage_events([])
+    step_ms = [ev_s[i].elapsed_time(ev_e[i]) for i in range(K)]
+    stage_ms = {name: sum(ev_stage[i][j].elapsed_time(ev_stage[i][j + 1]) for i in range(K)) / K
+                for j, name in enumerate(STAGES)}
+    ms_local = sum(step_ms) / K
+    st = moe.moe_read_device_status(ws, stream=s)
+    if st != moe.OK:
+        raise RuntimeError(f"device status after the timed steps: {moe.moe_status_string(st)}")
+
+    # ---- end to end through the C ABI: pinned host batch in, result out, every step
+    x_host = torch.from_numpy(inp["x"].view(np.int16) if inp["x"].dtype == np.uint16 else inp["x"]).pin_memory()
+    out_host = torch.empty(out.shape, dtype=torch.int16 if tdt == torch.bfloat16 else torch.float32).pin_memory()
+    x_dev = torch.empty_like(d_in["x"])
+    xd_raw = x_dev.view(torch.int16) if tdt == torch.bfloat16 else x_dev
+    out_raw = out.view(torch.int16) if tdt == torch.bfloat16 else out
+    Ke = max(3, min(K, 100))
+    e_s = [torch.cuda.Event(enable_timing=True) for _ in range(Ke)]
+    e_e = [torch.cuda.Event(enable_timing=True) for _ in range(Ke)]
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize(dev)
+    with torch.cuda.stream(s):
+        for i in range(Ke):
+            flush.zero_()
+            e_s[i].record(s)
+            xd_raw.copy_(x_host, non_blocking=True)
+            fwd(x=x_dev)
+            out_host.copy_(out_raw, non_blocking=True)
+            e_e[i].record(s)
+    torch.cuda.synchronize(dev)
+    if world > 1:
+        dist.barrier()
+    e2e_local = sum(e_s[i].elapsed_time(e_e[i]) for i in range(Ke)) / Ke
+    h2d = x_host.numel() * x_host.element_size()
+    d2h = out_host.numel() * out_host.element_size()
+
+    # ---- max over ranks
+    t = torch.tensor([ms_local, e2e_local], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    ms, e2e_ms = float(t[0]), float(t[1])
+
+    pk, pk_src = peaks()
+    plan_ksplit = 1
+    if cfg.dtype == W.BF16 and cfg.n_shared == 0:
+        # the library's static down-projection split (mirrors its planner; only affects the byte count)
+        avg = cfg.T * cfg.k / cfg.m
+        bn = 16
+        while bn < 256 and bn < avg:
+            bn <<= 1
+        tiles = min(cfg.m, cfg.T * cfg.k) * ((cfg.d + 127) // 128) * max(1, math.ceil(avg / bn))
+        if tiles < 4 * 148:
+            kb = (cfg.f + 63) // 64
+            ks = min(16, -(-4 * 148 // tiles), kb)
+            kbps = -(-kb // ks)
+            plan_ksplit = -(-kb // kbps)
+    costs, layer_flops, layer_bytes = stage_costs(cfg, active, plan_ksplit)
+    dom = max(STAGES, key=lambda n: stage_ms[n])
+    fl, by = costs[dom]
+    sec = stage_ms[dom] * 1e-3
+    long_step = K * ms > 1000.0
+    tensor_peak = pk["bf16_tflops_sustained"] if long_step else pk["bf16_tflops"]
+    ridge = tensor_peak * 1e12 / (pk["hbm_gbs"] * 1e9)
+    if fl > 0 and fl / by > ridge and cfg.dtype == W.BF16:
+        roof = {"bound": "tensor", "achieved": fl / sec / 1e12, "peak": tensor_peak, "unit": "TFLOP/s"}
+        roof["peak_source"] = f"{pk_src} bf16 ({'sustained' if long_step else 'burst'})"
+    else:
+        roof = {"bound": "hbm", "achieved": by / sec / 1e9, "peak": pk["hbm_gbs"], "unit": "GB/s",
+                "peak_source": f"{pk_src} hbm copy"}
+    roof["frac"] = roof["achieved"] / roof["peak"]
+    roof["traffic"] = traffic_for(cfg.name, dom)
+    roof["kernel"] = dom
+    roof["algorithmic_bytes"] = by
+    roof["algorithmic_flops"] = fl
+    roof["duration_us"] = stage_ms[dom] * 1e3
+    t_layer = max(layer_flops / (tensor_peak * 1e12), layer_bytes / (pk["hbm_gbs"] * 1e9))
+
+    line = {"metric": METRIC, "value": world * cfg.T / (ms * 1e-3), "unit": UNIT, "n_gpus": world, "steps": K,
+            "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16" if cfg.dtype == W.BF16 else "f32",
+            "data": "synthetic (seeded generator; x ~ N(0,1), weights ~ N(0, 1/sqrt(fan_in)), Zipf router bias)",
+            "config": dict(workload_config(cfg), parallelism=f"data-parallel token batches x{world} (weak scaling)",
+                           l2=f"flushed between steps ({L2_FLUSH_BYTES >> 20} MiB write, outside the timed events)",
+                           launch="eager C-ABI call per step"),
+            "roofline": roof,
+            "layer_roofline": {"time_us": t_layer * 1e6, "frac": t_layer / (ms * 1e-3),
+                               "flops": layer_flops, "bytes": layer_bytes},
+            "stages_us": {k: v * 1e3 for k, v in stage_ms.items()},
+            "routing": {"lis": lis_v, "max_count": max_count, "heavy_hitter": argmax, "active_experts": active,
+                        "reuse_ratio": cfg.T * cfg.k / max(active, 1), "load_entropy": entropy},
+            "e2e": {"value": world * cfg.T / (e2e_ms * 1e-3), "unit": UNIT, "h2d_bytes_per_step": h2d,
+                    "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
+            "gpu_launches": K * launches_per_step, "launches_per_step": launches_per_step,
+            "clocks": sampler.report()}
+    if world > 1:
+        dist.barrier()
+    if rank == 0:
+        if world == 1 and not args.no_cpu_baseline:
+            line["cpu_baseline"] = cpu_oracle_sample(cfg, inp, args.cpu_seconds)
+        else:
+            line["cpu_baseline"] = None
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.destroy_process_group()
+    return 0
+
+
+def main():
+    args = parse()
+    if args.impl == "reference":
+        return reference_arm(args)
+    return ours(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,223 @@
+/*
+ * moe.h - C ABI of libmoe.so: the forward pass of one sparse Mixture-of-Experts
+ * layer on an NVIDIA B200 (sm_100a).
+ *
+ * What the layer computes (the reviewed pages, cited by title and section):
+ *  - Token-choice top-k routing over m experts; R&Q ("A Replicate-and-Quantize
+ *    Strategy for Plug-and-Play Load Balancing of Sparse Mixture-of-Experts
+ *    LLMs") applies to top-1, top-2 and shared-expert routing ("If this is
+ *    right"), and its Definition 1 counts n_j, the tokens routed to expert j.
+ *  - The Load Imbalance Score LIS = m * max_j n_j / (n k) (R&Q, Definition 1;
+ *    1 is perfectly balanced, larger is more skewed).
+ *  - Expert-centric scheduling: (token, expert) tasks are sorted into one
+ *    contiguous group per active expert and each group runs as a grouped GEMM
+ *    (OmniMoE, "An Efficient MoE by Orchestrating Atomic Experts at Scale",
+ *    "What carries the argument" and Fig. 3).
+ *  - SwiGLU experts with W_gate, W_up, W_down and a SiLU gate (FloE, "On-the-Fly
+ *    MoE Inference on Memory-constrained GPU", "What carries the argument";
+ *    OmniMoE Sec. 2.1), or Switch-style two-matrix ReLU experts.
+ *  - Always-on shared experts added with weight 1 (OmniMoE's shared dense MLP
+ *    branch; R&Q's shared-expert routing).
+ *  - The atomic-expert variant: a Cartesian Product Router (OmniMoE Sec. 2.2,
+ *    Eq. 8), exact top-K over the implicit grid (OmniMoE App. A) and atomic
+ *    experts sigma(x w_in^T) w_out (OmniMoE Eq. 4).
+ *
+ * Conventions for every call:
+ *  - Pointers named x, w_*, out, ... are DEVICE pointers owned by the caller;
+ *    config structs and scalar out-parameters (bytes, moe_status_t*) are HOST
+ *    pointers. The library allocates no device memory; scratch comes from the
+ *    caller's workspace `ws` of `ws_bytes` bytes (size it with
+ *    moe_workspace_size / moe_atomic_workspace_size, zero it once before first
+ *    use: its first 4 bytes hold the device status word).
+ *  - Layouts are row-major with nn.Linear [out, in] weights:
+ *      x [T, d]; w_router [m, d]; bias [m] fp32;
+ *      w_gate, w_up [m, f, d]; w_down [m, d, f];   (ReLU experts: w_gate = W1, w_up = NULL, w_down = W2)
+ *      ws_gate, ws_up [n_shared, f_shared, d]; ws_down [n_shared, d, f_shared];
+ *      topk_idx [T, k] int32; topk_w [T, k] fp32; logits [T, m] fp32;
+ *      counts [m] int32; offsets [m + 1] int32; perm, inv_perm [T k] int32;
+ *      x_perm [T k, d]; y_perm [T k, d] fp32; out [T, d] in the config dtype.
+ *    Element type of x / weights / x_perm / out is cfg->dtype (fp32 or bf16).
+ *  - Alignment: every device pointer must be 16-byte aligned; d, f and f_shared
+ *    must be multiples of 8.
+ *  - Calls are asynchronous on `stream` (a cudaStream_t; NULL = legacy default
+ *    stream), never synchronise the host, and may be captured in a CUDA graph.
+ *  - Errors: arguments are checked on the host before any launch
+ *    (MOE_ERR_INVALID_ARG, MOE_ERR_UNSUPPORTED, MOE_ERR_WORKSPACE); a failed
+ *    launch returns MOE_ERR_CUDA. Errors found on the device (an expert id
+ *    outside [0, m): MOE_ERR_DEVICE_INDEX, and no write is issued for it; a
+ *    bounded wait inside a kernel that ran out: MOE_ERR_TIMEOUT) are recorded
+ *    in the status word of `ws` and read with moe_read_device_status.
+ *  - Only sm_100 devices are supported (MOE_ERR_UNSUPPORTED elsewhere); there
+ *    is no fallback path.
+ */
+#ifndef MOE_H_
+#define MOE_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#if defined(__GNUC__)
+#define MOE_API __attribute__((visibility("default")))
+#else
+#define MOE_API
+#endif
+
+typedef struct CUstream_st* moe_stream_t; /* identical to cudaStream_t */
+
+typedef enum {
+  MOE_OK = 0,
+  MOE_ERR_INVALID_ARG = 1,
+  MOE_ERR_UNSUPPORTED = 2,
+  MOE_ERR_WORKSPACE = 3,
+  MOE_ERR_CUDA = 4,
+  MOE_ERR_TIMEOUT = 5,
+  MOE_ERR_DEVICE_INDEX = 6
+} moe_status_t;
+
+typedef enum { MOE_F32 = 0, MOE_BF16 = 1 } moe_dtype_t;
+typedef enum { MOE_SWIGLU = 0, MOE_RELU = 1 } moe_act_t;
+typedef enum { MOE_ATOMIC_SILU = 0, MOE_ATOMIC_SIGMOID = 1 } moe_atomic_act_t;
+
+/* One coarse-expert layer. T = tokens (the pages' n), d = d_model, f = d_ff of a
+ * routed expert, m = routed experts (1..1024), k = experts per token (1..min(m, 32)),
+ * n_shared / f_shared = always-on shared experts (0..8) and their d_ff.
+ * renormalize != 0 divides the k gate weights by their sum. */
+typedef struct {
+  int32_t T, d, f, m, k, n_shared, f_shared;
+  int32_t dtype;       /* moe_dtype_t */
+  int32_t act;         /* moe_act_t */
+  int32_t renormalize; /* 0 or 1 */
+} moe_config_t;
+
+/* Load diagnostics of one layer call (device memory, 16 bytes). */
+typedef struct {
+  int32_t max_count;     /* max_j n_j */
+  int32_t argmax_expert; /* lowest j attaining it: the heavy hitter (R&Q Alg. 1) */
+  double lis;            /* m * max_j n_j / (T k), one correctly rounded fp64 division */
+} moe_lis_t;
+
+/* Atomic-expert layer: N = Nr * Nc experts on a grid, K selected per token
+ * (1..64), Nr and Nc in 64..1024 and multiples of 8; dtype must be MOE_BF16. */
+typedef struct {
+  int32_t T, d, Nr, Nc, K;
+  int32_t act;   /* moe_atomic_act_t */
+  int32_t dtype; /* moe_dtype_t */
+} moe_atomic_config_t;
+
+/* Workspace bytes needed by every call below for this config (the maximum over
+ * them, i.e. what moe_layer_forward needs). bytes: host out-parameter. */
+MOE_API moe_status_t moe_workspace_size(const moe_config_t* cfg, size_t* bytes);
+MOE_API moe_status_t moe_atomic_workspace_size(const moe_atomic_config_t* cfg, size_t* bytes);
+
+/* Router (R&Q's token-choice routing). logits = x w_router^T + bias (fp32,
+ * fp32 accumulation; bias may be NULL), or logits_in verbatim when given (then x,
+ * w_router and bias are ignored). top-k by (logit desc, expert index asc);
+ * p = softmax over all m logits; topk_w[t,s] = p[idx] (or renormalised over the
+ * k when cfg->renormalize). logits_out (nullable) receives the logits used. */
+MOE_API moe_status_t moe_route(const moe_config_t* cfg, const void* x, const void* w_router, const float* bias,
+                       const float* logits_in, float* logits_out, int32_t* topk_idx, float* topk_w, void* ws,
+                       size_t ws_bytes, moe_stream_t stream);
+
+/* Per-expert histogram n_j, segment offsets (exclusive prefix sum, m + 1
+ * entries) and LIS (R&Q Definition 1). counts, offsets and lis are device
+ * pointers; lis may be NULL. An id outside [0, m) sets MOE_ERR_DEVICE_INDEX in
+ * the status word and nothing is written. */
+MOE_API moe_status_t moe_histogram_lis(const moe_config_t* cfg, const int32_t* topk_idx, int32_t* counts, int32_t* offsets,
+                               moe_lis_t* lis, void* ws, size_t ws_bytes, moe_stream_t stream);
+
+/* Expert-centric permutation (OmniMoE Fig. 3). Task q = t k + s goes to
+ * position pos = offsets[e] + (number of earlier tasks q' < q with the same
+ * expert e): segments are contiguous and ordered by task id. Writes
+ * perm[pos] = q, inv_perm[q] = pos and x_perm[pos, :] = x[q / k, :]. A task
+ * whose id or position falls outside the segment given by `offsets` sets
+ * MOE_ERR_DEVICE_INDEX and is not written. */
+MOE_API moe_status_t moe_permute(const moe_config_t* cfg, const void* x, const int32_t* topk_idx, const int32_t* offsets,
+                         void* x_perm, int32_t* perm, int32_t* inv_perm, void* ws, size_t ws_bytes,
+                         moe_stream_t stream);
+
+/* Grouped expert FFN over the segments of x_perm (rows offsets[e]..offsets[e+1]
+ * belong to expert e): y_perm[pos] = task_w[perm[pos]] * FFN_e(x_perm[pos]) with
+ * FFN_e the SwiGLU (or ReLU) expert; task_w == NULL means weight 1 (perm is then
+ * ignored). bf16 runs on the tcgen05 tensor cores (bf16 operands, fp32
+ * accumulation, the hidden activation h rounded to bf16 between the two GEMMs);
+ * fp32 runs on the CUDA cores in fp32. */
+MOE_API moe_status_t moe_grouped_ffn(const moe_config_t* cfg, const void* x_perm, const int32_t* offsets,
+                             const void* w_gate, const void* w_up, const void* w_down, const float* task_w,
+                             const int32_t* perm, float* y_perm, void* ws, size_t ws_bytes, moe_stream_t stream);
+
+/* Shared experts: y_shared[s, t, :] = FFN_s(x[t, :]) for s < cfg->n_shared,
+ * y_shared fp32 [n_shared, T, d]. */
+MOE_API moe_status_t moe_shared_ffn(const moe_config_t* cfg, const void* x, const void* ws_gate, const void* ws_up,
+                            const void* ws_down, float* y_shared, void* ws, size_t ws_bytes, moe_stream_t stream);
+
+/* Combine: out[t] = sum_{s<k} y_perm[inv_perm[t k + s]] + sum_{s<n_shared}
+ * y_shared[s, t] (y_shared may be NULL), summed in fp32 in that order and rounded
+ * to cfg->dtype. */
+MOE_API moe_status_t moe_combine(const moe_config_t* cfg, const float* y_perm, const int32_t* inv_perm,
+                         const float* y_shared, void* out, moe_stream_t stream);
+
+/* The whole layer in one call, on one stream with no host synchronisation:
+ * route -> histogram/LIS -> permute -> grouped FFN (+ shared experts) -> combine.
+ * Optional device outputs (each may be NULL): logits_out [T, m], topk_idx_out,
+ * topk_w_out [T, k], counts_out [m], lis_out. w_up / ws_up are NULL for ReLU;
+ * ws_* are NULL when n_shared == 0. */
+MOE_API moe_status_t moe_layer_forward(const moe_config_t* cfg, const void* x, const void* w_router, const float* bias,
+                               const void* w_gate, const void* w_up, const void* w_down, const void* ws_gate,
+                               const void* ws_up, const void* ws_down, void* out, float* logits_out,
+                               int32_t* topk_idx_out, float* topk_w_out, int32_t* counts_out, moe_lis_t* lis_out,
+                               void* ws, size_t ws_bytes, moe_stream_t stream);
+
+/* Cartesian Product Router (OmniMoE Sec. 2.2, Eq. 8; App. A): lr = log_softmax(x
+ * w_row^T), lc = log_softmax(x w_col^T) (fp32); expert (i, j) with flat id
+ * i Nc + j scores S = fl32(lr_i + lc_j); idx_out [T, K] = the exact top-K of all
+ * Nr Nc scores by (S desc, id asc), g_out [T, K] = softmax of the selected S.
+ * row_logp_out [T, Nr] and col_logp_out [T, Nc] are optional (nullable). */
+MOE_API moe_status_t moe_atomic_route(const moe_atomic_config_t* cfg, const void* x, const void* w_row, const void* w_col,
+                              float* row_logp_out, float* col_logp_out, int32_t* idx_out, float* g_out, void* ws,
+                              size_t ws_bytes, moe_stream_t stream);
+
+/* Atomic experts (OmniMoE Eq. 4, Dynamic Expert Assembly): out[t] = sum_s
+ * g[t,s] act(x_t . w_in[idx[t,s]]) w_out[idx[t,s]], act = SiLU or sigmoid;
+ * w_in, w_out [Nr Nc, d] bf16; out [T, d] bf16. */
+MOE_API moe_status_t moe_atomic_experts(const moe_atomic_config_t* cfg, const void* x, const void* w_in, const void* w_out,
+                                const int32_t* idx, const float* g, void* out, void* ws, size_t ws_bytes,
+                                moe_stream_t stream);
+
+/* moe_atomic_route followed by moe_atomic_experts. idx_out, g_out nullable. */
+MOE_API moe_status_t moe_atomic_forward(const moe_atomic_config_t* cfg, const void* x, const void* w_row, const void* w_col,
+                                const void* w_in, const void* w_out, void* out, int32_t* idx_out, float* g_out,
+                                void* ws, size_t ws_bytes, moe_stream_t stream);
+
+/* Synchronises `stream`, reads the status word of `ws` into *out (host) and
+ * clears it. Returns MOE_ERR_CUDA if the synchronisation or copy fails. */
+MOE_API moe_status_t moe_read_device_status(void* ws, moe_stream_t stream, moe_status_t* out);
+
+/* Static string for a status code. */
+MOE_API const char* moe_status_string(moe_status_t status);
+
+/* Test hook: the time limit, in nanoseconds, of every bounded wait inside the
+ * tensor-core kernels launched after this call (0 restores the default of 2 s).
+ * Not thread-safe; meant for fault-injection tests. */
+MOE_API moe_status_t moe_debug_set_wait_limit_ns(uint64_t ns);
+
+/* Profiling hook: when n > 0, every later moe_layer_forward records the n
+ * cudaEvent_t handles in `events` (host array, caller-owned events) on its
+ * stream at its stage boundaries, in order: 0 start, 1 router logits, 2 top-k,
+ * 3 histogram/LIS/ranks, 4 row permutation, 5 up projection, 6 down projection,
+ * 7 combine (n <= 8; extra stages are not recorded). n = 0 turns it off. The
+ * array is copied. Process-wide and not thread-safe; meant for benchmarks. */
+MOE_API moe_status_t moe_set_stage_events(void* const* events, int n);
+
+/* Number of kernels this library launched since the process started (host
+ * counter; for benchmarks that report their launch count). */
+MOE_API uint64_t moe_launch_count(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MOE_H_ */

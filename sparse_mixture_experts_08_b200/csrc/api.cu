@@ -1,0 +1,718 @@
+// libmoe C ABI: argument checks, workspace layout and launch orchestration.
+// Every entry point validates on the host before launching anything, launches
+// asynchronously on the caller's stream, allocates nothing and never blocks the
+// host (except moe_read_device_status, which exists to do exactly that).
+#include <algorithm>
+#include <atomic>
+#include <cstring>
+#include <initializer_list>
+
+#include "common.cuh"
+
+namespace moe {
+
+static std::atomic<uint64_t> g_launches{0};
+void count_launch(int n) { g_launches += (uint64_t)n; }
+
+int num_sms() {
+  static int cache[64] = {0};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 148;
+  if (!cache[dev]) {
+    int n = 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) n = 148;
+    cache[dev] = n;
+  }
+  return cache[dev];
+}
+
+static unsigned long long g_wait_limit_ns = 2000ull * 1000 * 1000;
+static cudaEvent_t g_stage_events[8];
+static int g_n_stage_events = 0;
+
+static moe_status_t mark_stage(int i, cudaStream_t s) {
+  if (i < g_n_stage_events) return cudaEventRecord(g_stage_events[i], s) == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+  return MOE_OK;
+}
+constexpr int PLAN_SMS = 148;  // B200 SM count used for static planning (split-K, tile sizes)
+
+static moe_status_t check_device() {
+  static int ok_cache[64] = {0};  // 0 unknown, 1 ok, 2 unsupported
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return MOE_ERR_CUDA;
+  if (!ok_cache[dev]) {
+    int major = 0, minor = 0;
+    if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess)
+      return MOE_ERR_CUDA;
+    ok_cache[dev] = (major == 10 && minor == 0) ? 1 : 2;
+  }
+  return ok_cache[dev] == 1 ? MOE_OK : MOE_ERR_UNSUPPORTED;
+}
+
+static bool aligned16(const void* p) { return ((uintptr_t)p & 15u) == 0; }
+static size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
+
+// ------------------------------------------------------------------ planning
+struct Plan {
+  int es;          // element size of x / weights
+  int bn_up, bn_down;
+  int ksplit;      // down-projection K split (1 when shared experts are present)
+  int kbps;        // k-blocks per split of the routed down projection
+};
+
+static int kblocks(int K) { return (K + 63) / 64; }
+
+static Plan make_plan(const moe_config_t& c) {
+  Plan p;
+  p.es = c.dtype == MOE_F32 ? 4 : 2;
+  const double avg = (double)c.T * c.k / c.m;
+  p.bn_up = tc_pick_bn(c.act == MOE_SWIGLU ? EPI_SWIGLU : EPI_RELU, avg);
+  p.bn_down = tc_pick_bn(EPI_DOWN, avg);
+  p.ksplit = 1;
+  p.kbps = kblocks(c.f);
+  if (c.dtype == MOE_BF16 && c.n_shared == 0) {
+    const long long active = std::min<long long>(c.m, (long long)c.T * c.k);
+    const long long nt = std::max<long long>(1, (long long)((avg + p.bn_down - 1) / p.bn_down));
+    const long long tiles = active * ((c.d + 127) / 128) * nt;
+    const long long want = 4LL * PLAN_SMS;
+    if (tiles < want) {
+      int ks = (int)std::min<long long>((want + tiles - 1) / tiles, 16);
+      ks = std::min(ks, kblocks(c.f));
+      const int kbps = (kblocks(c.f) + ks - 1) / ks;
+      p.ksplit = (kblocks(c.f) + kbps - 1) / kbps;  // no empty split
+      p.kbps = kbps;
+    }
+  }
+  return p;
+}
+
+struct Layout {
+  size_t status, logits, idx, w, counts, offsets, lis, perm, inv_perm, x_perm, h, h_sh, y, y_sh, total;
+};
+
+static Layout make_layout(const moe_config_t& c, const Plan& p) {
+  Layout L;
+  size_t off = 0;
+  auto take = [&](size_t bytes) {
+    const size_t o = off;
+    off += align256(bytes);
+    return o;
+  };
+  const size_t Tk = (size_t)c.T * c.k;
+  const size_t T = (size_t)c.T;
+  L.status = take(256);
+  L.logits = take(T * c.m * 4);
+  L.idx = take(Tk * 4);
+  L.w = take(Tk * 4);
+  L.counts = take((size_t)c.m * 4);
+  L.offsets = take((size_t)(c.m + 1) * 4);
+  L.lis = take(sizeof(moe_lis_t));
+  L.perm = take(Tk * 4);
+  L.inv_perm = take(Tk * 4);
+  L.x_perm = take(Tk * c.d * p.es);
+  L.h = take(Tk * c.f * p.es);
+  L.h_sh = take((size_t)c.n_shared * T * std::max(c.f_shared, 0) * p.es);
+  L.y = take((size_t)p.ksplit * Tk * c.d * 4);
+  L.y_sh = take((size_t)p.ksplit * c.n_shared * T * c.d * 4);
+  L.total = off;
+  return L;
+}
+
+template <typename Tp>
+static Tp* at(void* ws, size_t off) {
+  return reinterpret_cast<Tp*>(reinterpret_cast<char*>(ws) + off);
+}
+
+static moe_status_t check_cfg(const moe_config_t* c) {
+  if (!c) return MOE_ERR_INVALID_ARG;
+  if (c->T < 1 || c->d < 8 || c->f < 8 || c->m < 1 || c->k < 1) return MOE_ERR_INVALID_ARG;
+  if (c->k > c->m) return MOE_ERR_INVALID_ARG;
+  if (c->dtype != MOE_F32 && c->dtype != MOE_BF16) return MOE_ERR_INVALID_ARG;
+  if (c->act != MOE_SWIGLU && c->act != MOE_RELU) return MOE_ERR_INVALID_ARG;
+  if (c->renormalize != 0 && c->renormalize != 1) return MOE_ERR_INVALID_ARG;
+  if (c->n_shared < 0 || (c->n_shared > 0 && c->f_shared < 8)) return MOE_ERR_INVALID_ARG;
+  if (c->d % 8 || c->f % 8 || (c->n_shared && c->f_shared % 8)) return MOE_ERR_UNSUPPORTED;
+  if (c->m > 1024 || c->k > 32 || c->n_shared > 8) return MOE_ERR_UNSUPPORTED;
+  if ((long long)c->T * c->k >= (1LL << 31) / 2) return MOE_ERR_UNSUPPORTED;
+  if (c->m + c->n_shared > tc_max_groups()) return MOE_ERR_UNSUPPORTED;
+  return MOE_OK;
+}
+
+static moe_status_t check_ws(const moe_config_t& c, void* ws, size_t ws_bytes, size_t need) {
+  (void)c;
+  if (!ws || ((uintptr_t)ws & 255u)) return MOE_ERR_INVALID_ARG;
+  if (ws_bytes < need) return MOE_ERR_WORKSPACE;
+  return MOE_OK;
+}
+
+static moe_status_t cuda_status(cudaError_t e) { return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA; }
+
+#define MOE_TRY(expr)                          \
+  do {                                         \
+    const moe_status_t st_ = (expr);           \
+    if (st_ != MOE_OK) return st_;             \
+  } while (0)
+#define MOE_CUDA(expr) MOE_TRY(cuda_status(expr))
+
+// ------------------------------------------------------------------ building blocks
+
+static moe_status_t run_router(const moe_config_t& c, const void* x, const void* w_r, const float* bias, float* logits,
+                               int* status, cudaStream_t s) {
+  if (c.dtype == MOE_F32) return cuda_status(launch_simt_logits(MOE_F32, c.T, c.d, c.m, x, w_r, bias, logits, s));
+  // logits^T = W_r . x^T on the tensor cores: one group, features = experts.
+  GemmParams p;
+  std::memset(&p, 0, sizeof(p));
+  GemmClass& g = p.cls[0];
+  g.n_groups = 1;
+  g.R = c.m;
+  g.K = c.d;
+  g.ksplit = 1;
+  g.kb_per_split = kblocks(c.d);
+  g.const_rows = c.T;
+  g.out = logits;
+  g.out_ld = c.m;
+  g.bias = bias;
+  p.n_classes = 1;
+  p.status = status;
+  p.wait_limit_ns = g_wait_limit_ns;
+  int bn = 128;
+  const long long mt = (c.m + 127) / 128;
+  while (bn > 16 && mt * ((c.T + bn - 1) / bn) < PLAN_SMS) bn >>= 1;
+  TcMaps maps;
+  std::memset(&maps, 0, sizeof(maps));
+  maps.a0[0] = {w_r, c.m, c.d};
+  maps.a1[0] = maps.a0[0];
+  maps.b[0] = {x, c.T, c.d};
+  const long long tiles = mt * ((c.T + bn - 1) / bn);
+  const int ctas = (int)std::min<long long>(tiles, num_sms());
+  return cuda_status(launch_tc_gemm(EPI_LOGITS, bn, maps, p, ctas, s));
+}
+
+struct FfnIo {
+  // routed class (may be absent: n_routed_groups == 0)
+  int n_routed;           // groups (experts) of the routed class
+  const int32_t* offsets; // device
+  const void* x_perm;     // [rows, d]
+  long long routed_rows;  // rows of x_perm / h / y (T k)
+  const void *w_gate, *w_up, *w_down;
+  void* h;
+  float* y;
+  const float* task_w;
+  const int32_t* perm;
+  // shared class
+  int n_shared;
+  const void* x;          // [T, d]
+  const void *ws_gate, *ws_up, *ws_down;
+  void* h_sh;             // [n_shared T, f_shared]
+  float* y_sh;            // [n_shared T, d]
+};
+
+static void fill_common(GemmParams& p, int* status) {
+  p.status = status;
+  p.wait_limit_ns = g_wait_limit_ns;
+}
+
+static moe_status_t run_ffn(const moe_config_t& c, const Plan& pl, const FfnIo& io, int ksplit, int kbps, int* status,
+                            cudaStream_t s, bool stage_marks = false) {
+  const bool swiglu = c.act == MOE_SWIGLU;
+  const bool tc = c.dtype == MOE_BF16;
+  // ---- up projection (+ activation): h = act(x W_gate^T [, x W_up^T])
+  GemmParams up;
+  std::memset(&up, 0, sizeof(up));
+  fill_common(up, status);
+  TcMaps mu;
+  std::memset(&mu, 0, sizeof(mu));
+  int ncls = 0;
+  if (io.n_routed > 0) {
+    GemmClass& g = up.cls[ncls];
+    g.n_groups = io.n_routed;
+    g.R = c.f;
+    g.K = c.d;
+    g.ksplit = 1;
+    g.kb_per_split = kblocks(c.d);
+    g.seg_off = io.offsets;
+    g.max_row = (int)io.routed_rows;
+    g.out = io.h;
+    g.out_ld = c.f;
+    g.a0 = io.w_gate;
+    g.a1 = swiglu ? io.w_up : nullptr;
+    g.b = io.x_perm;
+    g.a_ld = c.d;
+    g.b_ld = c.d;
+    mu.a0[ncls] = {io.w_gate, (long long)io.n_routed * c.f, c.d};
+    mu.a1[ncls] = {swiglu ? io.w_up : io.w_gate, (long long)io.n_routed * c.f, c.d};
+    mu.b[ncls] = {io.x_perm, io.routed_rows, c.d};
+    ++ncls;
+  }
+  if (io.n_shared > 0) {
+    GemmClass& g = up.cls[ncls];
+    g.n_groups = io.n_shared;
+    g.R = c.f_shared;
+    g.K = c.d;
+    g.ksplit = 1;
+    g.kb_per_split = kblocks(c.d);
+    g.const_rows = c.T;
+    g.b_group_stride = 0;
+    g.out_group_stride = c.T;
+    g.out = io.h_sh;
+    g.out_ld = c.f_shared;
+    g.a0 = io.ws_gate;
+    g.a1 = swiglu ? io.ws_up : nullptr;
+    g.b = io.x;
+    g.a_ld = c.d;
+    g.b_ld = c.d;
+    mu.a0[ncls] = {io.ws_gate, (long long)io.n_shared * c.f_shared, c.d};
+    mu.a1[ncls] = {swiglu ? io.ws_up : io.ws_gate, (long long)io.n_shared * c.f_shared, c.d};
+    mu.b[ncls] = {io.x, c.T, c.d};
+    ++ncls;
+  }
+  if (ncls == 0) return MOE_OK;
+  up.n_classes = ncls;
+  const int epi_up = swiglu ? EPI_SWIGLU : EPI_RELU;
+  if (tc)
+    MOE_CUDA(launch_tc_gemm(epi_up, pl.bn_up, mu, up, num_sms(), s));
+  else
+    MOE_CUDA(launch_simt_gemm(epi_up, c.dtype, up, (int)std::min<long long>(io.routed_rows, 1LL << 30), s));
+  if (stage_marks) MOE_TRY(mark_stage(5, s));
+
+  // ---- down projection: y = w * (h W_down^T), K split into `ksplit` partial outputs
+  GemmParams dn;
+  std::memset(&dn, 0, sizeof(dn));
+  fill_common(dn, status);
+  TcMaps md;
+  std::memset(&md, 0, sizeof(md));
+  ncls = 0;
+  if (io.n_routed > 0) {
+    GemmClass& g = dn.cls[ncls];
+    g.n_groups = io.n_routed;
+    g.R = c.d;
+    g.K = c.f;
+    g.ksplit = ksplit;
+    g.kb_per_split = kbps;
+    g.seg_off = io.offsets;
+    g.max_row = (int)io.routed_rows;
+    g.out = io.y;
+    g.out_ld = c.d;
+    g.out_split_stride = io.routed_rows * c.d;
+    g.task_w = io.task_w;
+    g.perm = io.perm;
+    g.a0 = io.w_down;
+    g.b = io.h;
+    g.a_ld = c.f;
+    g.b_ld = c.f;
+    md.a0[ncls] = {io.w_down, (long long)io.n_routed * c.d, c.f};
+    md.a1[ncls] = md.a0[ncls];
+    md.b[ncls] = {io.h, io.routed_rows, c.f};
+    ++ncls;
+  }
+  if (io.n_shared > 0) {
+    GemmClass& g = dn.cls[ncls];
+    g.n_groups = io.n_shared;
+    g.R = c.d;
+    g.K = c.f_shared;
+    g.ksplit = 1;
+    g.kb_per_split = kblocks(c.f_shared);
+    g.const_rows = c.T;
+    g.b_group_stride = c.T;
+    g.out_group_stride = c.T;
+    g.out = io.y_sh;
+    g.out_ld = c.d;
+    g.a0 = io.ws_down;
+    g.b = io.h_sh;
+    g.a_ld = c.f_shared;
+    g.b_ld = c.f_shared;
+    md.a0[ncls] = {io.ws_down, (long long)io.n_shared * c.d, c.f_shared};
+    md.a1[ncls] = md.a0[ncls];
+    md.b[ncls] = {io.h_sh, (long long)io.n_shared * c.T, c.f_shared};
+    ++ncls;
+  }
+  dn.n_classes = ncls;
+  if (tc)
+    return cuda_status(launch_tc_gemm(EPI_DOWN, pl.bn_down, md, dn, num_sms(), s));
+  return cuda_status(launch_simt_gemm(EPI_DOWN, c.dtype, dn, (int)std::min<long long>(io.routed_rows, 1LL << 30), s));
+}
+
+}  // namespace moe
+
+using namespace moe;
+
+// ====================================================================== C ABI
+extern "C" {
+
+moe_status_t moe_workspace_size(const moe_config_t* cfg, size_t* bytes) {
+  MOE_TRY(check_cfg(cfg));
+  if (!bytes) return MOE_ERR_INVALID_ARG;
+  *bytes = make_layout(*cfg, make_plan(*cfg)).total;
+  return MOE_OK;
+}
+
+moe_status_t moe_route(const moe_config_t* cfg, const void* x, const void* w_router, const float* bias,
+                       const float* logits_in, float* logits_out, int32_t* topk_idx, float* topk_w, void* ws,
+                       size_t ws_bytes, moe_stream_t stream) {
+  MOE_TRY(check_cfg(cfg));
+  const moe_config_t& c = *cfg;
+  const Layout L = make_layout(c, make_plan(c));
+  if (!topk_idx || !topk_w) return MOE_ERR_INVALID_ARG;
+  if (!logits_in && (!x || !w_router)) return MOE_ERR_INVALID_ARG;
+  for (const void* p : std::initializer_list<const void*>{x, w_router, (const void*)bias, (const void*)logits_in, (const void*)logits_out,
+                        (const void*)topk_idx, (const void*)topk_w})
+    if (p && !aligned16(p)) return MOE_ERR_INVALID_ARG;
+  MOE_TRY(check_ws(c, ws, ws_bytes, L.logits + align256((size_t)c.T * c.m * 4)));
+  MOE_TRY(check_device());
+  cudaStream_t s = (cudaStream_t)stream;
+  int* status = at<int>(ws, L.status);
+  const float* lg = logits_in;
+  if (!lg) {
+    float* dst = logits_out ? logits_out : at<float>(ws, L.logits);
+    MOE_TRY(run_router(c, x, w_router, bias, dst, status, s));
+    lg = dst;
+  } else if (logits_out && logits_out != logits_in) {
+    MOE_CUDA(cudaMemcpyAsync(logits_out, logits_in, (size_t)c.T * c.m * 4, cudaMemcpyDeviceToDevice, s));
+  }
+  return cuda_status(launch_topk_softmax(c.T, c.m, c.k, c.renormalize, lg, topk_idx, topk_w, s));
+}
+
+moe_status_t moe_histogram_lis(const moe_config_t* cfg, const int32_t* topk_idx, int32_t* counts, int32_t* offsets,
+                               moe_lis_t* lis, void* ws, size_t ws_bytes, moe_stream_t stream) {
+  MOE_TRY(check_cfg(cfg));
+  const moe_config_t& c = *cfg;
+  if (!topk_idx || !counts || !offsets) return MOE_ERR_INVALID_ARG;
+  for (const void* p : std::initializer_list<const void*>{(const void*)topk_idx, (const void*)counts, (const void*)offsets, (const void*)lis})
+    if (p && !aligned16(p)) return MOE_ERR_INVALID_ARG;
+  const Layout L = make_layout(c, make_plan(c));
+  MOE_TRY(check_ws(c, ws, ws_bytes, L.status + 256));
+  MOE_TRY(check_device());
+  return cuda_status(launch_route_index(1, c.T, c.k, c.m, topk_idx, counts, offsets, lis, nullptr, nullptr,
+                                        at<int>(ws, L.status), (cudaStream_t)stream));
+}
+
+moe_status_t moe_permute(const moe_config_t* cfg, const void* x, const int32_t* topk_idx, const int32_t* offsets,
+                         void* x_perm, int32_t* perm, int32_t* inv_perm, void* ws, size_t ws_bytes,
+                         moe_stream_t stream) {
+  MOE_TRY(check_cfg(cfg));
+  const moe_config_t& c = *cfg;
+  if (!x || !topk_idx || !offsets || !x_perm || !perm || !inv_perm) return MOE_ERR_INVALID_ARG;
+  for (const void* p : std::initializer_list<const void*>{x, (const void*)topk_idx, (const void*)offsets, (const void*)x_perm, (const void*)perm,
+                        (const void*)inv_perm})
+    if (!aligned16(p)) return MOE_ERR_INVALID_ARG;
+  const Layout L = make_layout(c, make_plan(c));
+  MOE_TRY(check_ws(c, ws, ws_bytes, L.status + 256));
+  MOE_TRY(check_device());
+  cudaStream_t s = (cudaStream_t)stream;
+  const long long Tk = (long long)c.T * c.k;
+  // Positions not covered by a valid task keep -1, so the row copy skips them.
+  MOE_CUDA(cudaMemsetAsync(perm, 0xFF, (size_t)Tk * 4, s));
+  MOE_CUDA(launch_route_index(2, c.T, c.k, c.m, topk_idx, nullptr, const_cast<int32_t*>(offsets), nullptr, perm,
+                              inv_perm, at<int>(ws, L.status), s));
+  return cuda_status(launch_permute_rows(c.dtype, (int)Tk, c.k, c.d, x, perm, x_perm, s));
+}
+
+moe_status_t moe_grouped_ffn(const moe_config_t* cfg, const void* x_perm, const int32_t* offsets, const void* w_gate,
+                             const void* w_up, const void* w_down, const float* task_w, const int32_t* perm,
+                             float* y_perm, void* ws, size_t ws_bytes, moe_stream_t stream) {
+  MOE_TRY(check_cfg(cfg));
+  const moe_config_t& c = *cfg;
+  if (!x_perm || !offsets || !w_gate || !w_down || !y_perm) return MOE_ERR_INVALID_ARG;
+  if (c.act == MOE_SWIGLU && !w_up) return MOE_ERR_INVALID_ARG;
+  if (task_w && !perm) return MOE_ERR_INVALID_ARG;
+  for (const void* p : std::initializer_list<const void*>{x_perm, (const void*)offsets, w_gate, w_up, w_down, (const void*)task_w, (const void*)perm,
+                        (const void*)y_perm})
+    if (p && !aligned16(p)) return MOE_ERR_INVALID_ARG;
+  const Plan pl = make_plan(c);
+  const Layout L = make_layout(c, pl);
+  MOE_TRY(check_ws(c, ws, ws_bytes, L.h + align256((size_t)c.T * c.k * c.f * pl.es)));
+  MOE_TRY(check_device());
+  FfnIo io;
+  std::memset(&io, 0, sizeof(io));
+  io.n_routed = c.m;
+  io.offsets = offsets;
+  io.x_perm = x_perm;
+  io.routed_rows = (long long)c.T * c.k;
+  io.w_gate = w_gate;
+  io.w_up = w_up;
+  io.w_down = w_down;
+  io.h = at<void>(ws, L.h);
+  io.y = y_perm;
+  io.task_w = task_w;
+  io.perm = perm;
+  return run_ffn(c, pl, io, 1, kblocks(c.f), at<int>(ws, L.status), (cudaStream_t)stream);
+}
+
+moe_status_t moe_shared_ffn(const moe_config_t* cfg, const void* x, const void* ws_gate, const void* ws_up,
+                            const void* ws_down, float* y_shared, void* ws, size_t ws_bytes, moe_stream_t stream) {
+  MOE_TRY(check_cfg(cfg));
+  const moe_config_t& c = *cfg;
+  if (c.n_shared == 0) return MOE_OK;
+  if (!x || !ws_gate || !ws_down || !y_shared) return MOE_ERR_INVALID_ARG;
+  if (c.act == MOE_SWIGLU && !ws_up) return MOE_ERR_INVALID_ARG;
+  for (const void* p : std::initializer_list<const void*>{x, ws_gate, ws_up, ws_down, (const void*)y_shared})
+    if (p && !aligned16(p)) return MOE_ERR_INVALID_ARG;
+  const Plan pl = make_plan(c);
+  const Layout L = make_layout(c, pl);
+  MOE_TRY(check_ws(c, ws, ws_bytes, L.h_sh + align256((size_t)c.n_shared * c.T * c.f_shared * pl.es)));
+  MOE_TRY(check_device());
+  FfnIo io;
+  std::memset(&io, 0, sizeof(io));
+  io.n_shared = c.n_shared;
+  io.x = x;
+  io.ws_gate = ws_gate;
+  io.ws_up = ws_up;
+  io.ws_down = ws_down;
+  io.h_sh = at<void>(ws, L.h_sh);
+  io.y_sh = y_shared;
+  return run_ffn(c, pl, io, 1, kblocks(c.f), at<int>(ws, L.status), (cudaStream_t)stream);
+}
+
+moe_status_t moe_combine(const moe_config_t* cfg, const float* y_perm, const int32_t* inv_perm, const float* y_shared,
+                         void* out, moe_stream_t stream) {
+  MOE_TRY(check_cfg(cfg));
+  const moe_config_t& c = *cfg;
+  if (!y_perm || !inv_perm || !out) return MOE_ERR_INVALID_ARG;
+  for (const void* p : std::initializer_list<const void*>{(const void*)y_perm, (const void*)inv_perm, (const void*)y_shared, (const void*)out})
+    if (p && !aligned16(p)) return MOE_ERR_INVALID_ARG;
+  MOE_TRY(check_device());
+  return cuda_status(launch_combine(c.dtype, c.T, c.d, c.k, 1, y_perm, 0, inv_perm, c.n_shared, y_shared, 0, out,
+                                    (cudaStream_t)stream));
+}
+
+moe_status_t moe_layer_forward(const moe_config_t* cfg, const void* x, const void* w_router, const float* bias,
+                               const void* w_gate, const void* w_up, const void* w_down, const void* ws_gate,
+                               const void* ws_up, const void* ws_down, void* out, float* logits_out,
+                               int32_t* topk_idx_out, float* topk_w_out, int32_t* counts_out, moe_lis_t* lis_out,
+                               void* ws, size_t ws_bytes, moe_stream_t stream) {
+  MOE_TRY(check_cfg(cfg));
+  const moe_config_t& c = *cfg;
+  if (!x || !w_router || !w_gate || !w_down || !out) return MOE_ERR_INVALID_ARG;
+  if (c.act == MOE_SWIGLU && !w_up) return MOE_ERR_INVALID_ARG;
+  if (c.n_shared > 0 && (!ws_gate || !ws_down || (c.act == MOE_SWIGLU && !ws_up))) return MOE_ERR_INVALID_ARG;
+  for (const void* p : std::initializer_list<const void*>{x, w_router, (const void*)bias, w_gate, w_up, w_down, ws_gate, ws_up, ws_down, out,
+                        (const void*)logits_out, (const void*)topk_idx_out, (const void*)topk_w_out,
+                        (const void*)counts_out, (const void*)lis_out})
+    if (p && !aligned16(p)) return MOE_ERR_INVALID_ARG;
+  const Plan pl = make_plan(c);
+  const Layout L = make_layout(c, pl);
+  MOE_TRY(check_ws(c, ws, ws_bytes, L.total));
+  MOE_TRY(check_device());
+  cudaStream_t s = (cudaStream_t)stream;
+  int* status = at<int>(ws, L.status);
+  float* logits = logits_out ? logits_out : at<float>(ws, L.logits);
+  int32_t* idx = topk_idx_out ? topk_idx_out : at<int32_t>(ws, L.idx);
+  float* w = topk_w_out ? topk_w_out : at<float>(ws, L.w);
+  int32_t* counts = counts_out ? counts_out : at<int32_t>(ws, L.counts);
+  moe_lis_t* lis = lis_out ? lis_out : at<moe_lis_t>(ws, L.lis);
+  int32_t* offsets = at<int32_t>(ws, L.offsets);
+  int32_t* perm = at<int32_t>(ws, L.perm);
+  int32_t* inv_perm = at<int32_t>(ws, L.inv_perm);
+  const long long Tk = (long long)c.T * c.k;
+
+  MOE_TRY(mark_stage(0, s));
+  MOE_TRY(run_router(c, x, w_router, bias, logits, status, s));
+  MOE_TRY(mark_stage(1, s));
+  MOE_CUDA(launch_topk_softmax(c.T, c.m, c.k, c.renormalize, logits, idx, w, s));
+  MOE_TRY(mark_stage(2, s));
+  MOE_CUDA(launch_route_index(3, c.T, c.k, c.m, idx, counts, offsets, lis, perm, inv_perm, status, s));
+  MOE_TRY(mark_stage(3, s));
+  MOE_CUDA(launch_permute_rows(c.dtype, (int)Tk, c.k, c.d, x, perm, at<void>(ws, L.x_perm), s));
+  MOE_TRY(mark_stage(4, s));
+  FfnIo io;
+  std::memset(&io, 0, sizeof(io));
+  io.n_routed = c.m;
+  io.offsets = offsets;
+  io.x_perm = at<void>(ws, L.x_perm);
+  io.routed_rows = Tk;
+  io.w_gate = w_gate;
+  io.w_up = w_up;
+  io.w_down = w_down;
+  io.h = at<void>(ws, L.h);
+  io.y = at<float>(ws, L.y);
+  io.task_w = w;
+  io.perm = perm;
+  io.n_shared = c.n_shared;
+  io.x = x;
+  io.ws_gate = ws_gate;
+  io.ws_up = ws_up;
+  io.ws_down = ws_down;
+  io.h_sh = at<void>(ws, L.h_sh);
+  io.y_sh = at<float>(ws, L.y_sh);
+  MOE_TRY(run_ffn(c, pl, io, pl.ksplit, pl.kbps, status, s, true));
+  MOE_TRY(mark_stage(6, s));
+  MOE_CUDA(launch_combine(c.dtype, c.T, c.d, c.k, pl.ksplit, io.y, Tk * c.d, inv_perm, c.n_shared, io.y_sh,
+                          (long long)c.n_shared * c.T * c.d, out, s));
+  return mark_stage(7, s);
+}
+
+// ------------------------------------------------------------------ atomic experts
+static moe_status_t check_atomic_cfg(const moe_atomic_config_t* c) {
+  if (!c) return MOE_ERR_INVALID_ARG;
+  if (c->T < 1 || c->d < 8 || c->Nr < 1 || c->Nc < 1 || c->K < 1) return MOE_ERR_INVALID_ARG;
+  if (c->act != MOE_ATOMIC_SILU && c->act != MOE_ATOMIC_SIGMOID) return MOE_ERR_INVALID_ARG;
+  if (c->dtype != MOE_BF16) return MOE_ERR_UNSUPPORTED;
+  if ((long long)c->K > (long long)c->Nr * c->Nc) return MOE_ERR_INVALID_ARG;
+  if (c->d % 8 || c->Nr % 8 || c->Nc % 8 || c->Nr < 64 || c->Nc < 64 || c->Nr > 1024 || c->Nc > 1024 || c->K > 64)
+    return MOE_ERR_UNSUPPORTED;
+  if (c->T > 65535) return MOE_ERR_UNSUPPORTED;
+  return MOE_OK;
+}
+
+struct AtomicPlan {
+  int ksplit, kbps;
+  size_t status, zr, zc, idx, g, coef, total;
+};
+
+static AtomicPlan make_atomic_plan(const moe_atomic_config_t& c) {
+  AtomicPlan p;
+  const long long tiles = (long long)((c.Nr + 127) / 128 + (c.Nc + 127) / 128) * ((c.T + 15) / 16);
+  int ks = (int)std::min<long long>(16, std::max<long long>(1, (PLAN_SMS + tiles - 1) / tiles));
+  ks = std::min(ks, kblocks(c.d));
+  p.kbps = (kblocks(c.d) + ks - 1) / ks;
+  p.ksplit = (kblocks(c.d) + p.kbps - 1) / p.kbps;
+  size_t off = 0;
+  auto take = [&](size_t bytes) {
+    const size_t o = off;
+    off += align256(bytes);
+    return o;
+  };
+  p.status = take(256);
+  p.zr = take((size_t)p.ksplit * c.T * c.Nr * 4);
+  p.zc = take((size_t)p.ksplit * c.T * c.Nc * 4);
+  p.idx = take((size_t)c.T * c.K * 4);
+  p.g = take((size_t)c.T * c.K * 4);
+  p.coef = take((size_t)c.T * c.K * 4);
+  p.total = off;
+  return p;
+}
+
+moe_status_t moe_atomic_workspace_size(const moe_atomic_config_t* cfg, size_t* bytes) {
+  MOE_TRY(check_atomic_cfg(cfg));
+  if (!bytes) return MOE_ERR_INVALID_ARG;
+  *bytes = make_atomic_plan(*cfg).total;
+  return MOE_OK;
+}
+
+static moe_status_t atomic_route_impl(const moe_atomic_config_t& c, const AtomicPlan& P, const void* x,
+                                      const void* w_row, const void* w_col, float* lr_out, float* lc_out,
+                                      int32_t* idx, float* g, void* ws, cudaStream_t s) {
+  int* status = at<int>(ws, P.status);
+  float* zr = at<float>(ws, P.zr);
+  float* zc = at<float>(ws, P.zc);
+  GemmParams p;
+  std::memset(&p, 0, sizeof(p));
+  fill_common(p, status);
+  p.n_classes = 2;
+  TcMaps maps;
+  std::memset(&maps, 0, sizeof(maps));
+  for (int side = 0; side < 2; ++side) {
+    GemmClass& gc = p.cls[side];
+    const int n = side ? c.Nc : c.Nr;
+    gc.n_groups = 1;
+    gc.R = n;
+    gc.K = c.d;
+    gc.ksplit = P.ksplit;
+    gc.kb_per_split = P.kbps;
+    gc.const_rows = c.T;
+    gc.out = side ? zc : zr;
+    gc.out_ld = n;
+    gc.out_split_stride = (long long)c.T * n;
+    maps.a0[side] = {side ? w_col : w_row, n, c.d};
+    maps.a1[side] = maps.a0[side];
+    maps.b[side] = {x, c.T, c.d};
+  }
+  const int bn = c.T <= 16 ? 16 : c.T <= 32 ? 32 : c.T <= 64 ? 64 : 128;
+  MOE_CUDA(launch_tc_gemm(EPI_LOGITS, bn, maps, p, num_sms(), s));
+  return cuda_status(launch_atomic_select(c.T, c.Nr, c.Nc, c.K, P.ksplit, zr, (long long)c.T * c.Nr, zc,
+                                          (long long)c.T * c.Nc, lr_out, lc_out, idx, g, status, s));
+}
+
+moe_status_t moe_atomic_route(const moe_atomic_config_t* cfg, const void* x, const void* w_row, const void* w_col,
+                              float* row_logp_out, float* col_logp_out, int32_t* idx_out, float* g_out, void* ws,
+                              size_t ws_bytes, moe_stream_t stream) {
+  MOE_TRY(check_atomic_cfg(cfg));
+  const moe_atomic_config_t& c = *cfg;
+  if (!x || !w_row || !w_col || !idx_out || !g_out) return MOE_ERR_INVALID_ARG;
+  for (const void* p : std::initializer_list<const void*>{x, w_row, w_col, (const void*)row_logp_out, (const void*)col_logp_out, (const void*)idx_out,
+                        (const void*)g_out})
+    if (p && !aligned16(p)) return MOE_ERR_INVALID_ARG;
+  const AtomicPlan P = make_atomic_plan(c);
+  if (!ws || ((uintptr_t)ws & 255u)) return MOE_ERR_INVALID_ARG;
+  if (ws_bytes < P.total) return MOE_ERR_WORKSPACE;
+  MOE_TRY(check_device());
+  return atomic_route_impl(c, P, x, w_row, w_col, row_logp_out, col_logp_out, idx_out, g_out, ws,
+                           (cudaStream_t)stream);
+}
+
+moe_status_t moe_atomic_experts(const moe_atomic_config_t* cfg, const void* x, const void* w_in, const void* w_out,
+                                const int32_t* idx, const float* g, void* out, void* ws, size_t ws_bytes,
+                                moe_stream_t stream) {
+  MOE_TRY(check_atomic_cfg(cfg));
+  const moe_atomic_config_t& c = *cfg;
+  if (!x || !w_in || !w_out || !idx || !g || !out) return MOE_ERR_INVALID_ARG;
+  for (const void* p : std::initializer_list<const void*>{x, w_in, w_out, (const void*)idx, (const void*)g, out})
+    if (!aligned16(p)) return MOE_ERR_INVALID_ARG;
+  const AtomicPlan P = make_atomic_plan(c);
+  if (!ws || ((uintptr_t)ws & 255u)) return MOE_ERR_INVALID_ARG;
+  if (ws_bytes < P.total) return MOE_ERR_WORKSPACE;
+  MOE_TRY(check_device());
+  return cuda_status(launch_atomic_experts(c.T, c.d, c.K, c.act, x, w_in, w_out, idx, g, at<float>(ws, P.coef), out,
+                                           (long long)c.Nr * c.Nc, at<int>(ws, P.status), (cudaStream_t)stream));
+}
+
+moe_status_t moe_atomic_forward(const moe_atomic_config_t* cfg, const void* x, const void* w_row, const void* w_col,
+                                const void* w_in, const void* w_out, void* out, int32_t* idx_out, float* g_out,
+                                void* ws, size_t ws_bytes, moe_stream_t stream) {
+  MOE_TRY(check_atomic_cfg(cfg));
+  const moe_atomic_config_t& c = *cfg;
+  if (!x || !w_row || !w_col || !w_in || !w_out || !out) return MOE_ERR_INVALID_ARG;
+  for (const void* p : std::initializer_list<const void*>{x, w_row, w_col, w_in, w_out, out, (const void*)idx_out, (const void*)g_out})
+    if (p && !aligned16(p)) return MOE_ERR_INVALID_ARG;
+  const AtomicPlan P = make_atomic_plan(c);
+  if (!ws || ((uintptr_t)ws & 255u)) return MOE_ERR_INVALID_ARG;
+  if (ws_bytes < P.total) return MOE_ERR_WORKSPACE;
+  MOE_TRY(check_device());
+  cudaStream_t s = (cudaStream_t)stream;
+  int32_t* idx = idx_out ? idx_out : at<int32_t>(ws, P.idx);
+  float* g = g_out ? g_out : at<float>(ws, P.g);
+  MOE_TRY(atomic_route_impl(c, P, x, w_row, w_col, nullptr, nullptr, idx, g, ws, s));
+  return cuda_status(launch_atomic_experts(c.T, c.d, c.K, c.act, x, w_in, w_out, idx, g, at<float>(ws, P.coef), out,
+                                           (long long)c.Nr * c.Nc, at<int>(ws, P.status), s));
+}
+
+// ------------------------------------------------------------------ status helpers
+moe_status_t moe_read_device_status(void* ws, moe_stream_t stream, moe_status_t* out) {
+  if (!ws || !out) return MOE_ERR_INVALID_ARG;
+  if (cudaStreamSynchronize((cudaStream_t)stream) != cudaSuccess) return MOE_ERR_CUDA;
+  int v = 0;
+  if (cudaMemcpy(&v, ws, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess) return MOE_ERR_CUDA;
+  if (cudaMemset(ws, 0, sizeof(int)) != cudaSuccess) return MOE_ERR_CUDA;
+  *out = (moe_status_t)v;
+  return MOE_OK;
+}
+
+const char* moe_status_string(moe_status_t s) {
+  switch (s) {
+    case MOE_OK: return "ok";
+    case MOE_ERR_INVALID_ARG: return "invalid argument";
+    case MOE_ERR_UNSUPPORTED: return "unsupported configuration or device";
+    case MOE_ERR_WORKSPACE: return "workspace too small";
+    case MOE_ERR_CUDA: return "CUDA error";
+    case MOE_ERR_TIMEOUT: return "device wait timed out";
+    case MOE_ERR_DEVICE_INDEX: return "expert index or position out of range (device)";
+  }
+  return "unknown status";
+}
+
+moe_status_t moe_debug_set_wait_limit_ns(uint64_t ns) {
+  g_wait_limit_ns = ns ? (unsigned long long)ns : 2000ull * 1000 * 1000;
+  return MOE_OK;
+}
+
+moe_status_t moe_set_stage_events(void* const* events, int n) {
+  if (n < 0 || (n > 0 && !events)) return MOE_ERR_INVALID_ARG;
+  g_n_stage_events = std::min(n, 8);
+  for (int i = 0; i < g_n_stage_events; ++i) g_stage_events[i] = (cudaEvent_t)events[i];
+  return MOE_OK;
+}
+
+uint64_t moe_launch_count(void) { return g_launches.load(); }
+
+}  // extern "C"

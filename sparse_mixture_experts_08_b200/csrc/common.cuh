@@ -1,0 +1,110 @@
+// Shared device helpers and internal launch interfaces of libmoe (sm_100a only).
+#pragma once
+
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "../../include/moe.h"
+
+namespace moe {
+
+// Record the first device-side error in the status word (later errors keep it).
+__device__ __forceinline__ void set_status(int* status, int code) {
+  if (status) atomicCAS(status, 0, code);
+}
+
+__device__ __forceinline__ float bf16_bits_to_f32(uint16_t b) { return __uint_as_float(((uint32_t)b) << 16); }
+
+__device__ __forceinline__ uint64_t globaltimer_ns() {
+  uint64_t t;
+  asm volatile("mov.u64 %0, %globaltimer;" : "=l"(t));
+  return t;
+}
+
+// ---------------------------------------------------------------- internal API
+// Every launcher returns cudaSuccess or the launch error; arguments were checked
+// by the C-ABI layer before.
+
+enum Epi { EPI_LOGITS = 0, EPI_SWIGLU = 1, EPI_RELU = 2, EPI_DOWN = 3 };
+
+// One class of problems for the grouped GEMM  out = epi(A_g . B_rows^T):
+// A_g = rows [g*R, g*R + R) of a K-major weight matrix, B rows = one segment.
+struct GemmClass {
+  int n_groups;
+  int R;                     // output features per group (rows of A per group)
+  int K;                     // reduction length
+  int ksplit;                // K is cut into ksplit contiguous ranges (partial outputs)
+  int kb_per_split;          // 64-wide k-blocks per range
+  const int* seg_off;        // device [n_groups + 1]: B/out rows of group g (nullable)
+  int max_row;               // seg_off entries and perm values must lie in [0, max_row]
+  int const_rows;            // rows per group when seg_off == nullptr
+  int b_group_stride;        // B row start of group g when seg_off == nullptr
+  int out_group_stride;      // out row start of group g when seg_off == nullptr
+  void* out;                 // fp32 (LOGITS, DOWN) or the activation dtype (SWIGLU, RELU)
+  long long out_ld;          // elements between output rows
+  long long out_split_stride;// elements between k-split partial outputs
+  const float* bias;         // LOGITS: bias[feature] (nullable)
+  const float* task_w;       // DOWN: row weight task_w[perm[row]] (nullable = 1)
+  const int* perm;
+  // SIMT path only (fp32 / bf16 element pointers, row-major)
+  const void* a0;            // [n_groups * R, K]
+  const void* a1;            // second matrix (SwiGLU up) or nullptr
+  const void* b;             // [rows, K]
+  long long a_ld, b_ld;      // elements between rows
+};
+
+struct GemmParams {
+  GemmClass cls[2];
+  int n_classes;
+  int* status;
+  unsigned long long wait_limit_ns;
+};
+
+// Tensor-core grouped GEMM (bf16 in, fp32 accumulate). Tensor maps are built
+// from the pointers in `maps` (see tc_gemm.cu). mats = 2 for SwiGLU.
+struct TcOperand {
+  const void* ptr;     // bf16 [rows, K] row-major
+  long long rows;
+  long long K;
+};
+struct TcMaps {
+  TcOperand a0[2], a1[2], b[2];
+};
+cudaError_t launch_tc_gemm(int epi, int bn, const TcMaps& maps, const GemmParams& p, int num_ctas,
+                           cudaStream_t s);
+int tc_pick_bn(int epi, double avg_rows_per_group);
+int tc_max_groups();
+
+// SIMT grouped linear (fp32 or bf16 inputs, fp32 math), same GemmParams.
+cudaError_t launch_simt_gemm(int epi, int dtype, const GemmParams& p, int max_rows_per_group, cudaStream_t s);
+
+// Routing
+cudaError_t launch_simt_logits(int dtype, int T, int d, int m, const void* x, const void* w_r, const float* bias,
+                               float* logits, cudaStream_t s);
+cudaError_t launch_topk_softmax(int T, int m, int k, int renorm, const float* logits, int32_t* idx, float* w,
+                                cudaStream_t s);
+// mode bit 1: histogram (counts, offsets, lis from idx); bit 2: ranks (perm, inv_perm from offsets)
+cudaError_t launch_route_index(int mode, int T, int k, int m, const int32_t* idx, int32_t* counts, int32_t* offsets,
+                               moe_lis_t* lis, int32_t* perm, int32_t* inv_perm, int* status, cudaStream_t s);
+cudaError_t launch_permute_rows(int dtype, int Tk, int k, int d, const void* x, const int32_t* perm, void* x_perm,
+                                cudaStream_t s);
+cudaError_t launch_combine(int dtype, int T, int d, int k, int ksplit, const float* y_perm, long long y_split_stride,
+                           const int32_t* inv_perm, int n_shared, const float* y_shared, long long ysh_split_stride,
+                           void* out, cudaStream_t s);
+cudaError_t launch_reduce_splits(long long n, int ksplit, const float* in, long long split_stride, float* out,
+                                 cudaStream_t s);
+
+// Atomic experts
+cudaError_t launch_atomic_select(int T, int Nr, int Nc, int K, int ksplit, const float* zr, long long zr_split,
+                                 const float* zc, long long zc_split, float* lr_out, float* lc_out, int32_t* idx,
+                                 float* g, int* status, cudaStream_t s);
+cudaError_t launch_atomic_experts(int T, int d, int K, int act, const void* x, const void* w_in, const void* w_out,
+                                  const int32_t* idx, const float* g, float* coef, void* out, long long n_experts,
+                                  int* status, cudaStream_t s);
+
+int num_sms();
+void count_launch(int n = 1);
+
+}  // namespace moe

@@ -1,0 +1,555 @@
+// Grouped GEMM on the 5th-generation tensor cores (tcgen05 + TMEM + TMA), sm_100a.
+//
+// Expert-centric scheduling (OmniMoE, "What carries the argument" and Fig. 3):
+// once the (token, expert) tasks sit in one contiguous segment per expert, every
+// expert's work is a dense GEMM over its segment, and all experts run in ONE
+// persistent launch. The segment boundaries live only in device memory (the
+// offsets written by the histogram kernel), so the tile schedule is built on the
+// device: each CTA reads the per-group row counts, forms the tile prefix sum in
+// shared memory and walks tiles blockIdx.x, blockIdx.x + gridDim.x, ...
+//
+// Orientation ("swap-AB"): the weight matrix is the MMA's A operand (M = 128
+// output features per tile) and the segment's activation rows are the B operand
+// (N = BN rows, 16..256), so short segments (decode: a few tokens per expert;
+// Switch: ~64) waste no 128-row M tile. The MMA's N is chosen per tile as the
+// segment rows left, rounded up to 16. Both operands are K-major (nn.Linear
+// weights [out, in] and row-major activations), staged by TMA with the 128-byte
+// swizzle. One tile = the full K loop (or one of `ksplit` K ranges).
+//
+// Warp roles (192 threads): warp 0 = TMA producer, warp 1 = MMA issuer (and TMEM
+// owner), warps 2..5 = epilogue (TMEM -> registers -> activation -> global).
+// The accumulator is double-buffered in TMEM when it fits (2 x mats x BN <= 512
+// columns) so the epilogue of tile i overlaps the MMAs of tile i + 1.
+//
+// Every wait on an mbarrier is bounded in time (globaltimer); on expiry the kernel
+// records MOE_ERR_TIMEOUT in the status word, the other roles stop, outstanding
+// TMA copies and MMAs are drained (again with a bound) and TMEM is freed.
+#include <algorithm>
+#include <cstdio>
+
+#include "common.cuh"
+
+namespace moe {
+
+constexpr int TC_BM = 128;
+constexpr int TC_BK = 64;  // bf16 elements of one 128-byte swizzle row
+constexpr int TC_THREADS = 192;
+constexpr int TC_MAX_GROUPS = 1040;
+constexpr int TC_SMEM_BUDGET = 200 * 1024;
+constexpr unsigned long long TC_DRAIN_LIMIT_NS = 200ull * 1000 * 1000;
+
+int tc_max_groups() { return TC_MAX_GROUPS; }
+
+template <int BN, int MATS>
+struct TcShape {
+  static constexpr int A_BYTES = TC_BM * TC_BK * 2;    // 16 KB
+  static constexpr int B_BYTES = BN * TC_BK * 2;       // BN * 128 B
+  static constexpr int STAGE_BYTES = MATS * A_BYTES + B_BYTES;
+  static constexpr int STAGES_RAW = TC_SMEM_BUDGET / STAGE_BYTES;
+  static constexpr int STAGES = STAGES_RAW > 8 ? 8 : STAGES_RAW;
+  static constexpr int ACC_COLS = MATS * BN;
+  static constexpr int NUM_ACC = (2 * ACC_COLS <= 512) ? 2 : 1;
+  static constexpr int TMEM_NEED = NUM_ACC * ACC_COLS;
+  static constexpr int TMEM_COLS = TMEM_NEED <= 32 ? 32 : TMEM_NEED <= 64 ? 64 : TMEM_NEED <= 128 ? 128
+                                   : TMEM_NEED <= 256 ? 256 : 512;
+  static constexpr int DYN_SMEM = STAGES * STAGE_BYTES + 1024;  // + alignment slack
+  static_assert(STAGES >= 2, "pipeline needs at least two stages");
+  static_assert(TMEM_NEED <= 512, "accumulators exceed TMEM");
+  static_assert(BN % 16 == 0 && BN >= 16 && BN <= 256, "MMA N range");
+};
+
+// ------------------------------------------------------------------ PTX wrappers
+__device__ __forceinline__ uint32_t smem_u32(const void* p) { return (uint32_t)__cvta_generic_to_shared(p); }
+
+__device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count) : "memory");
+}
+__device__ __forceinline__ void fence_mbar_init() { asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory"); }
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes) : "memory");
+}
+__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+__device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}\n"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
+// Bounded wait: true when the phase with `parity` completed; false when the time
+// limit ran out or another role already aborted.
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, unsigned long long limit_ns,
+                                          const volatile int* abort_flag) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = globaltimer_ns();
+  while (true) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if (*abort_flag) return false;
+    if (globaltimer_ns() - t0 > limit_ns) return false;
+  }
+}
+
+__device__ __forceinline__ void tma_load_2d(const CUtensorMap* map, uint64_t* bar, void* dst, int x, int y) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4}], [%2];"
+      ::"r"(smem_u32(dst)), "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(x), "r"(y)
+      : "memory");
+}
+__device__ __forceinline__ void tma_prefetch_desc(const CUtensorMap* map) {
+  asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
+}
+
+__device__ __forceinline__ void tmem_alloc(uint32_t* dst, uint32_t ncols) {
+  asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(dst)), "r"(ncols)
+               : "memory");
+}
+__device__ __forceinline__ void tmem_relinquish() {
+  asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void tmem_dealloc(uint32_t taddr, uint32_t ncols) {
+  asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols) : "memory");
+}
+__device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
+
+// D(tmem) (+)= A(smem desc) * B(smem desc)^T, kind::f16 (bf16 operands, fp32 accumulator)
+__device__ __forceinline__ void umma_bf16(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                          uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}\n" ::"r"(d_tmem),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+// Arrive on `bar` once every tcgen05.mma issued so far by this thread completed.
+__device__ __forceinline__ void umma_commit(uint64_t* bar) {
+  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(smem_u32(bar))
+               : "memory");
+}
+
+__device__ __forceinline__ void tmem_ld_x16(uint32_t taddr, uint32_t* r) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+      : "r"(taddr));
+}
+__device__ __forceinline__ void tmem_ld_wait() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
+
+// Shared-memory matrix descriptor: K-major operand, 128-byte swizzle, rows of
+// 128 B, 8-row core groups 1024 B apart (SBO), descriptor version 1 (sm_100).
+__device__ __forceinline__ uint64_t sdesc_sw128(uint32_t saddr) {
+  uint64_t d = 0;
+  d |= (uint64_t)((saddr & 0x3FFFF) >> 4);
+  d |= (uint64_t)(16 >> 4) << 16;    // leading byte offset (unused for swizzled K-major)
+  d |= (uint64_t)(1024 >> 4) << 32;  // stride byte offset
+  d |= (uint64_t)1 << 46;            // version
+  d |= (uint64_t)2 << 61;            // SWIZZLE_128B
+  return d;
+}
+
+// Instruction descriptor, kind::f16: D fp32, A and B bf16, both K-major.
+__device__ __forceinline__ uint32_t idesc_bf16(int M, int N) {
+  return (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
+}
+
+// ------------------------------------------------------------------ tile schedule
+struct TileInfo {
+  int cls, g, mt, ks, nt, rows_in_tile, b_row, out_row, a_row, kb0, kb1;
+};
+
+struct SchedSmem {
+  int tile_start[TC_MAX_GROUPS + 1];
+  int rows[TC_MAX_GROUPS];
+  int brow[TC_MAX_GROUPS];
+};
+
+template <int BN>
+__device__ __forceinline__ void decode_tile(const GemmParams& p, const SchedSmem& s, int G, int w, TileInfo& ti) {
+  int lo = 0, hi = G - 1;  // largest gi with tile_start[gi] <= w
+  while (lo < hi) {
+    int mid = (lo + hi + 1) >> 1;
+    if (s.tile_start[mid] <= w) lo = mid; else hi = mid - 1;
+  }
+  const int gi = lo;
+  const int G0 = p.cls[0].n_groups;
+  ti.cls = gi < G0 ? 0 : 1;
+  ti.g = gi - (ti.cls ? G0 : 0);
+  const GemmClass& c = p.cls[ti.cls];
+  const int rows = s.rows[gi];
+  const int NT = (rows + BN - 1) / BN;
+  const int local = w - s.tile_start[gi];
+  ti.nt = local % NT;
+  const int rest = local / NT;
+  ti.ks = rest % c.ksplit;
+  ti.mt = rest / c.ksplit;
+  ti.rows_in_tile = min(BN, rows - ti.nt * BN);
+  ti.b_row = s.brow[gi] + ti.nt * BN;
+  ti.out_row = (c.seg_off ? s.brow[gi] : ti.g * c.out_group_stride) + ti.nt * BN;
+  ti.a_row = ti.g * c.R + ti.mt * TC_BM;
+  const int KB = (c.K + TC_BK - 1) / TC_BK;
+  ti.kb0 = ti.ks * c.kb_per_split;
+  ti.kb1 = min(KB, ti.kb0 + c.kb_per_split);
+}
+
+template <int EPI>
+__device__ __forceinline__ void store_out(const GemmClass& c, const TileInfo& ti, int feature, int j, float v0,
+                                          float v1) {
+  const long long row = (long long)ti.out_row + j;
+  if (EPI == EPI_LOGITS) {
+    float* o = reinterpret_cast<float*>(c.out) + (long long)ti.ks * c.out_split_stride;
+    o[row * c.out_ld + feature] = v0 + (c.bias ? c.bias[feature] : 0.f);
+  } else if (EPI == EPI_SWIGLU) {
+    const float h = v0 / (1.f + __expf(-v0)) * v1;
+    reinterpret_cast<__nv_bfloat16*>(c.out)[row * c.out_ld + feature] = __float2bfloat16_rn(h);
+  } else if (EPI == EPI_RELU) {
+    reinterpret_cast<__nv_bfloat16*>(c.out)[row * c.out_ld + feature] = __float2bfloat16_rn(fmaxf(v0, 0.f));
+  } else {  // EPI_DOWN
+    float wgt = 1.f;
+    if (c.task_w) {
+      const int q = c.perm[row];
+      wgt = (q >= 0 && q < c.max_row) ? c.task_w[q] : 0.f;
+    }
+    float* o = reinterpret_cast<float*>(c.out) + (long long)ti.ks * c.out_split_stride;
+    o[row * c.out_ld + feature] = v0 * wgt;
+  }
+}
+
+template <int BN, int MATS, int EPI>
+__global__ void __launch_bounds__(TC_THREADS, 1)
+    tc_grouped_gemm_kernel(const __grid_constant__ CUtensorMap tA0_0, const __grid_constant__ CUtensorMap tA1_0,
+                           const __grid_constant__ CUtensorMap tB_0, const __grid_constant__ CUtensorMap tA0_1,
+                           const __grid_constant__ CUtensorMap tA1_1, const __grid_constant__ CUtensorMap tB_1,
+                           const __grid_constant__ GemmParams p) {
+  using S = TcShape<BN, MATS>;
+  constexpr int STAGES = S::STAGES;
+
+  __shared__ SchedSmem sched;
+  __shared__ __align__(8) uint64_t full_bar[STAGES], empty_bar[STAGES], accf_bar[2], acce_bar[2], drain_bar;
+  __shared__ uint32_t tmem_base_s;
+  __shared__ int abort_s;
+  __shared__ int total_tiles_s;
+  extern __shared__ uint8_t dyn_smem[];
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t smem_base = (smem_u32(dyn_smem) + 1023u) & ~1023u;
+  uint8_t* smem_gen = dyn_smem + (smem_base - smem_u32(dyn_smem));
+  const int G0 = p.cls[0].n_groups;
+  const int G = G0 + (p.n_classes > 1 ? p.cls[1].n_groups : 0);
+  volatile int* abort_flag = &abort_s;
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < STAGES; ++i) {
+      mbar_init(&full_bar[i], 1);
+      mbar_init(&empty_bar[i], 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&accf_bar[i], 1);
+      mbar_init(&acce_bar[i], 4);
+    }
+    mbar_init(&drain_bar, 1);
+    abort_s = 0;
+    fence_mbar_init();
+    tma_prefetch_desc(&tA0_0);
+    tma_prefetch_desc(&tB_0);
+  }
+  if (warp == 1) {
+    tmem_alloc(&tmem_base_s, S::TMEM_COLS);
+    tmem_relinquish();
+  }
+  // Tile schedule from the device-resident segment sizes.
+  if (warp == 0) {
+    const int per = (G + 31) / 32;
+    const int lo = lane * per, hi = min(G, lo + per);
+    int local = 0;
+    for (int gi = lo; gi < hi; ++gi) {
+      const int cl = gi < G0 ? 0 : 1;
+      const int g = gi - (cl ? G0 : 0);
+      const GemmClass& c = p.cls[cl];
+      int rows, brow;
+      if (c.seg_off) {
+        const int a = c.seg_off[g], b = c.seg_off[g + 1];
+        rows = b - a;
+        brow = a;
+        if (a < 0 || b < a || b > c.max_row) {
+          set_status(p.status, MOE_ERR_DEVICE_INDEX);
+          rows = 0;
+          brow = 0;
+        }
+      } else {
+        rows = c.const_rows;
+        brow = g * c.b_group_stride;
+      }
+      sched.rows[gi] = rows;
+      sched.brow[gi] = brow;
+      const int MT = (c.R + TC_BM - 1) / TC_BM;
+      local += MT * c.ksplit * ((rows + BN - 1) / BN);
+      sched.tile_start[gi + 1] = local;
+    }
+    int incl = local;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+      const int v = __shfl_up_sync(0xffffffffu, incl, off);
+      if (lane >= off) incl += v;
+    }
+    const int excl = incl - local;
+    for (int gi = lo; gi < hi; ++gi) sched.tile_start[gi + 1] += excl;
+    if (lane == 0) sched.tile_start[0] = 0;
+    // An earlier kernel of this layer flagged a device error: its index tables
+    // cannot be trusted, so this launch does no work.
+    const int prior = p.status ? *reinterpret_cast<volatile int*>(p.status) : 0;
+    if (lane == 31) total_tiles_s = prior ? 0 : incl;
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = tmem_base_s;
+  const int total = total_tiles_s;
+  const unsigned long long lim = p.wait_limit_ns;
+
+  if (warp == 0 && lane == 0) {
+    // ---------------------------------------------------------------- producer
+    int stage = 0;
+    uint32_t phase = 0;
+    int last_parity[STAGES];
+#pragma unroll
+    for (int i = 0; i < STAGES; ++i) last_parity[i] = -1;
+    bool ok = true;
+    for (int w = blockIdx.x; w < total && ok; w += gridDim.x) {
+      TileInfo ti;
+      decode_tile<BN>(p, sched, G, w, ti);
+      const CUtensorMap* mA0 = ti.cls ? &tA0_1 : &tA0_0;
+      const CUtensorMap* mA1 = ti.cls ? &tA1_1 : &tA1_0;
+      const CUtensorMap* mB = ti.cls ? &tB_1 : &tB_0;
+      for (int kb = ti.kb0; kb < ti.kb1; ++kb) {
+        if (!mbar_wait(&empty_bar[stage], phase ^ 1u, lim, abort_flag)) {
+          ok = false;
+          break;
+        }
+        uint8_t* st = smem_gen + stage * S::STAGE_BYTES;
+        mbar_arrive_expect_tx(&full_bar[stage], S::STAGE_BYTES);
+        tma_load_2d(mA0, &full_bar[stage], st, kb * TC_BK, ti.a_row);
+        if (MATS == 2) tma_load_2d(mA1, &full_bar[stage], st + S::A_BYTES, kb * TC_BK, ti.a_row);
+        tma_load_2d(mB, &full_bar[stage], st + MATS * S::A_BYTES, kb * TC_BK, ti.b_row);
+        last_parity[stage] = (int)phase;
+        if (++stage == STAGES) {
+          stage = 0;
+          phase ^= 1u;
+        }
+      }
+    }
+    if (!ok) {
+      set_status(p.status, MOE_ERR_TIMEOUT);
+      abort_s = 1;
+    }
+    // Drain: every issued copy must land before the CTA may exit.
+    for (int i = 0; i < STAGES; ++i)
+      if (last_parity[i] >= 0) {
+        const volatile int never = 0;
+        if (!mbar_wait(&full_bar[i], (uint32_t)last_parity[i], TC_DRAIN_LIMIT_NS, &never))
+          set_status(p.status, MOE_ERR_TIMEOUT);
+      }
+  } else if (warp == 1 && lane == 0) {
+    // ---------------------------------------------------------------- MMA issuer
+    int stage = 0;
+    uint32_t phase = 0;
+    int acc = 0;
+    uint32_t acc_phase = 0;
+    bool ok = true;
+    for (int w = blockIdx.x; w < total && ok; w += gridDim.x) {
+      TileInfo ti;
+      decode_tile<BN>(p, sched, G, w, ti);
+      if (!mbar_wait(&acce_bar[acc], acc_phase ^ 1u, lim, abort_flag)) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      const uint32_t d_tmem = tmem_base + (uint32_t)(acc * S::ACC_COLS);
+      const int n_inst = max(16, (ti.rows_in_tile + 15) & ~15);
+      const uint32_t idesc = idesc_bf16(TC_BM, n_inst);
+      for (int kb = ti.kb0; kb < ti.kb1; ++kb) {
+        if (!mbar_wait(&full_bar[stage], phase, lim, abort_flag)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t st = smem_base + stage * S::STAGE_BYTES;
+        const uint64_t da0 = sdesc_sw128(st);
+        const uint64_t da1 = sdesc_sw128(st + S::A_BYTES);
+        const uint64_t db = sdesc_sw128(st + MATS * S::A_BYTES);
+#pragma unroll
+        for (int kk = 0; kk < TC_BK / 16; ++kk) {
+          const uint32_t accum = (kb > ti.kb0 || kk > 0) ? 1u : 0u;
+          // advance 16 bf16 (32 B) along K inside the swizzle atom: +2 in the >>4 address field
+          umma_bf16(d_tmem, da0 + 2 * kk, db + 2 * kk, idesc, accum);
+          if (MATS == 2) umma_bf16(d_tmem + BN, da1 + 2 * kk, db + 2 * kk, idesc, accum);
+        }
+        umma_commit(&empty_bar[stage]);
+        if (++stage == STAGES) {
+          stage = 0;
+          phase ^= 1u;
+        }
+      }
+      if (!ok) break;
+      umma_commit(&accf_bar[acc]);
+      if (++acc == S::NUM_ACC) {
+        acc = 0;
+        acc_phase ^= 1u;
+      }
+    }
+    if (!ok) {
+      set_status(p.status, MOE_ERR_TIMEOUT);
+      abort_s = 1;
+    }
+    umma_commit(&drain_bar);
+    const volatile int never = 0;
+    if (!mbar_wait(&drain_bar, 0, TC_DRAIN_LIMIT_NS, &never)) set_status(p.status, MOE_ERR_TIMEOUT);
+  } else if (warp >= 2) {
+    // ---------------------------------------------------------------- epilogue
+    const int q = warp & 3;  // TMEM lane quarter this warp may access
+    int acc = 0;
+    uint32_t acc_phase = 0;
+    for (int w = blockIdx.x; w < total; w += gridDim.x) {
+      TileInfo ti;
+      decode_tile<BN>(p, sched, G, w, ti);
+      const bool got = mbar_wait(&accf_bar[acc], acc_phase, lim, abort_flag);
+      if (!got) {
+        set_status(p.status, MOE_ERR_TIMEOUT);
+        abort_s = 1;
+        break;
+      }
+      tc_fence_after();
+      const GemmClass& c = p.cls[ti.cls];
+      const int feature = ti.mt * TC_BM + q * 32 + lane;
+      const bool fvalid = feature < c.R;
+      const bool has_k = ti.kb1 > ti.kb0;  // an empty K range leaves the accumulator unwritten
+      const uint32_t t_row = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * S::ACC_COLS);
+      for (int c0 = 0; c0 < ti.rows_in_tile; c0 += 16) {
+        uint32_t r0[16], r1[16];
+        tmem_ld_x16(t_row + c0, r0);
+        if (MATS == 2) tmem_ld_x16(t_row + BN + c0, r1);
+        tmem_ld_wait();
+        if (fvalid) {
+          const int jn = min(16, ti.rows_in_tile - c0);
+#pragma unroll
+          for (int j = 0; j < 16; ++j)
+            if (j < jn)
+              store_out<EPI>(c, ti, feature, c0 + j, has_k ? __uint_as_float(r0[j]) : 0.f,
+                             (MATS == 2 && has_k) ? __uint_as_float(r1[j]) : 0.f);
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&acce_bar[acc]);
+      if (++acc == S::NUM_ACC) {
+        acc = 0;
+        acc_phase ^= 1u;
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, S::TMEM_COLS);
+  }
+}
+
+// ------------------------------------------------------------------ host side
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+static EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  if (!fn) {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(ptr);
+  }
+  return fn;
+}
+
+// bf16 [rows, K] row-major, box = 64 (K) x box_rows, 128-byte swizzle; out-of-range
+// elements read as zero.
+static bool make_map(CUtensorMap* m, const TcOperand& op, int box_rows) {
+  EncodeTiledFn enc = encode_fn();
+  if (!enc || !op.ptr || op.rows <= 0 || op.K <= 0) return false;
+  cuuint64_t dims[2] = {(cuuint64_t)op.K, (cuuint64_t)op.rows};
+  cuuint64_t strides[1] = {(cuuint64_t)op.K * 2};
+  cuuint32_t box[2] = {(cuuint32_t)TC_BK, (cuuint32_t)box_rows};
+  cuuint32_t es[2] = {1, 1};
+  CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(op.ptr), dims, strides, box, es,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+template <int BN, int MATS, int EPI>
+static cudaError_t launch_impl(const TcMaps& maps, const GemmParams& p, int num_ctas, cudaStream_t s) {
+  using S = TcShape<BN, MATS>;
+  CUtensorMap m[6];
+  const int nc = p.n_classes;
+  for (int c = 0; c < 2; ++c) {
+    const int src = c < nc ? c : 0;
+    if (!make_map(&m[3 * c + 0], maps.a0[src], TC_BM)) return cudaErrorInvalidValue;
+    const TcOperand& a1 = MATS == 2 ? maps.a1[src] : maps.a0[src];
+    if (!make_map(&m[3 * c + 1], a1, TC_BM)) return cudaErrorInvalidValue;
+    if (!make_map(&m[3 * c + 2], maps.b[src], BN)) return cudaErrorInvalidValue;
+  }
+  auto kern = tc_grouped_gemm_kernel<BN, MATS, EPI>;
+  static bool attr_set = false;
+  if (!attr_set) {
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, S::DYN_SMEM);
+    if (e != cudaSuccess) return e;
+    attr_set = true;
+  }
+  kern<<<num_ctas, TC_THREADS, S::DYN_SMEM, s>>>(m[0], m[1], m[2], m[3], m[4], m[5], p);
+  count_launch();
+  return cudaGetLastError();
+}
+
+int tc_pick_bn(int epi, double avg) {
+  const int cap = (epi == EPI_SWIGLU || epi == EPI_LOGITS) ? 128 : 256;
+  int bn = 16;
+  while (bn < cap && bn < avg) bn <<= 1;
+  return bn;
+}
+
+cudaError_t launch_tc_gemm(int epi, int bn, const TcMaps& maps, const GemmParams& p, int num_ctas,
+                           cudaStream_t s) {
+#define MOE_TC_CASE(EPI_, MATS_, BN_) \
+  if (epi == EPI_ && bn == BN_) return launch_impl<BN_, MATS_, EPI_>(maps, p, num_ctas, s);
+  MOE_TC_CASE(EPI_LOGITS, 1, 16)
+  MOE_TC_CASE(EPI_LOGITS, 1, 32)
+  MOE_TC_CASE(EPI_LOGITS, 1, 64)
+  MOE_TC_CASE(EPI_LOGITS, 1, 128)
+  MOE_TC_CASE(EPI_SWIGLU, 2, 16)
+  MOE_TC_CASE(EPI_SWIGLU, 2, 32)
+  MOE_TC_CASE(EPI_SWIGLU, 2, 64)
+  MOE_TC_CASE(EPI_SWIGLU, 2, 128)
+  MOE_TC_CASE(EPI_RELU, 1, 16)
+  MOE_TC_CASE(EPI_RELU, 1, 32)
+  MOE_TC_CASE(EPI_RELU, 1, 64)
+  MOE_TC_CASE(EPI_RELU, 1, 128)
+  MOE_TC_CASE(EPI_RELU, 1, 256)
+  MOE_TC_CASE(EPI_DOWN, 1, 16)
+  MOE_TC_CASE(EPI_DOWN, 1, 32)
+  MOE_TC_CASE(EPI_DOWN, 1, 64)
+  MOE_TC_CASE(EPI_DOWN, 1, 128)
+  MOE_TC_CASE(EPI_DOWN, 1, 256)
+#undef MOE_TC_CASE
+  return cudaErrorInvalidValue;
+}
+
+}  // namespace moe

@@ -1,0 +1,136 @@
+"""The C ABI without a GPU: the library loads, exports every symbol that
+include/moe.h declares, and rejects bad arguments on the host with the
+documented status codes before touching the device."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import sparse_mixture_experts_08_b200 as moe
+from sparse_mixture_experts_08_b200.moe import MoEAtomicConfig, MoEConfig
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _declared():
+    with open(os.path.join(ROOT, "include", "moe.h")) as fh:
+        text = fh.read()
+    return sorted(set(re.findall(r"MOE_API\s+[\w\s\*]+?\b(moe_\w+)\s*\(", text)))
+
+
+def test_header_declares_the_binding_exports():
+    assert _declared() == sorted(moe.moe.EXPORTS)
+
+
+def test_library_exports_every_declared_symbol():
+    lib = moe.moe.lib()
+    for name in _declared():
+        assert hasattr(lib, name), name
+
+
+def test_struct_layouts_match_header():
+    assert ctypes.sizeof(MoEConfig) == 40
+    assert ctypes.sizeof(MoEAtomicConfig) == 28
+    assert moe.moe.LIS_BYTES == 16
+
+
+def test_status_strings():
+    lib = moe.moe.lib()
+    for code in range(7):
+        assert moe.moe_status_string(code)
+    assert moe.moe_status_string(99) == "unknown status"
+
+
+def _ws_size(**kw):
+    base = dict(T=64, d=128, f=256, m=8, k=2, n_shared=0, f_shared=0, dtype=moe.F32, act=moe.SWIGLU, renormalize=0)
+    base.update(kw)
+    c = MoEConfig(**base)
+    n = ctypes.c_size_t(0)
+    return moe.moe.lib().moe_workspace_size(ctypes.byref(c), ctypes.byref(n)), n.value
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(T=0), moe.ERR_INVALID_ARG),        # LIS undefined for an empty batch
+    (dict(k=9), moe.ERR_INVALID_ARG),        # k > m
+    (dict(k=0), moe.ERR_INVALID_ARG),
+    (dict(dtype=7), moe.ERR_INVALID_ARG),
+    (dict(act=5), moe.ERR_INVALID_ARG),
+    (dict(renormalize=2), moe.ERR_INVALID_ARG),
+    (dict(d=100), moe.ERR_UNSUPPORTED),      # d % 8
+    (dict(f=12), moe.ERR_UNSUPPORTED),
+    (dict(m=2048, k=2), moe.ERR_UNSUPPORTED),
+    (dict(m=64, k=33), moe.ERR_UNSUPPORTED),
+    (dict(n_shared=1, f_shared=0), moe.ERR_INVALID_ARG),
+    (dict(n_shared=9, f_shared=64), moe.ERR_UNSUPPORTED),
+])
+def test_config_validation(kw, code):
+    rc, _ = _ws_size(**kw)
+    assert rc == code
+
+
+def test_workspace_size_grows_with_tokens():
+    rc1, a = _ws_size(T=64)
+    rc2, b = _ws_size(T=640)
+    assert rc1 == rc2 == moe.OK and b > a > 0
+    assert moe.moe.lib().moe_workspace_size(None, None) == moe.ERR_INVALID_ARG
+
+
+def _fake(addr):
+    return ctypes.c_void_p(addr)
+
+
+def test_calls_reject_bad_pointers_and_small_workspace_before_launch():
+    lib = moe.moe.lib()
+    c = MoEConfig(64, 128, 256, 8, 2, 0, 0, moe.BF16, moe.SWIGLU, 0)
+    ok_ws = _fake(1 << 20)
+    a = _fake(1 << 24)
+    # missing outputs
+    assert lib.moe_route(ctypes.byref(c), a, a, None, None, None, None, None, ok_ws, 1 << 30, None) == \
+        moe.ERR_INVALID_ARG
+    # misaligned pointer
+    assert lib.moe_route(ctypes.byref(c), _fake((1 << 24) + 4), a, None, None, None, a, a, ok_ws, 1 << 30, None) == \
+        moe.ERR_INVALID_ARG
+    # workspace too small / misaligned
+    assert lib.moe_route(ctypes.byref(c), a, a, None, None, None, a, a, ok_ws, 16, None) == moe.ERR_WORKSPACE
+    assert lib.moe_layer_forward(ctypes.byref(c), a, a, None, a, a, a, None, None, None, a, None, None, None, None,
+                                 None, _fake((1 << 20) + 16), 1 << 30, None) == moe.ERR_INVALID_ARG
+    assert lib.moe_layer_forward(ctypes.byref(c), a, a, None, a, a, a, None, None, None, a, None, None, None, None,
+                                 None, ok_ws, 1024, None) == moe.ERR_WORKSPACE
+    # SwiGLU needs w_up
+    assert lib.moe_grouped_ffn(ctypes.byref(c), a, a, a, None, a, None, None, a, ok_ws, 1 << 30, None) == \
+        moe.ERR_INVALID_ARG
+    # task weights need perm
+    assert lib.moe_grouped_ffn(ctypes.byref(c), a, a, a, a, a, a, None, a, ok_ws, 1 << 30, None) == \
+        moe.ERR_INVALID_ARG
+    assert lib.moe_permute(ctypes.byref(c), a, a, None, a, a, a, ok_ws, 1 << 30, None) == moe.ERR_INVALID_ARG
+    assert lib.moe_combine(ctypes.byref(c), a, None, None, a, None) == moe.ERR_INVALID_ARG
+    assert lib.moe_read_device_status(None, None, None) == moe.ERR_INVALID_ARG
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(K=65), moe.ERR_UNSUPPORTED),
+    (dict(Nr=32), moe.ERR_UNSUPPORTED),
+    (dict(Nc=2048), moe.ERR_UNSUPPORTED),
+    (dict(dtype=moe.F32), moe.ERR_UNSUPPORTED),
+    (dict(act=3), moe.ERR_INVALID_ARG),
+    (dict(T=0), moe.ERR_INVALID_ARG),
+])
+def test_atomic_config_validation(kw, code):
+    base = dict(T=16, d=4096, Nr=512, Nc=512, K=64, act=moe.ATOMIC_SILU, dtype=moe.BF16)
+    base.update(kw)
+    c = MoEAtomicConfig(**base)
+    n = ctypes.c_size_t(0)
+    assert moe.moe.lib().moe_atomic_workspace_size(ctypes.byref(c), ctypes.byref(n)) == code
+
+
+def test_atomic_workspace_size_ok():
+    c = MoEAtomicConfig(16, 4096, 512, 512, 64, moe.ATOMIC_SILU, moe.BF16)
+    assert moe.moe_atomic_workspace_size(c) > 0
+
+
+def test_debug_wait_limit_hook():
+    lib = moe.moe.lib()
+    assert lib.moe_debug_set_wait_limit_ns(5) == moe.OK
+    assert lib.moe_debug_set_wait_limit_ns(0) == moe.OK
+    assert moe.moe_launch_count() >= 0

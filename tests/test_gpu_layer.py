@@ -1,0 +1,171 @@
+"""End-to-end parity of moe_layer_forward (the call the benchmark times) on every
+workload at full size, plus the atomic-expert variant.
+
+All tokens: top-k ids, counts, max/argmax and LIS bit-exact against the oracle
+deciding on the GPU's own fp32 logits. Outputs: every token for the small
+workloads; for the large ones a sample the oracle can evaluate token by token
+(always the first and last token and tokens of the most and least loaded
+experts), within the per-token relative tolerance.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle as O
+import sparse_mixture_experts_08_b200 as moe
+import workloads as W
+from gpu_helpers import (GATE_RTOL, TOL, device_inputs, host, layer_forward, out_f64, require_gpu, sample_tokens,
+                         token_rel_err)
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(autouse=True, scope="module")
+def _gpu():
+    require_gpu()
+
+
+def _check_layer(cfg, inp, n_sample):
+    d_in = device_inputs(inp)
+    r = layer_forward(cfg, d_in)
+    assert moe.moe_read_device_status(r["ws"]) == moe.OK
+    lg, idx, w, counts = host(r["logits"]), host(r["idx"]), host(r["w"]), host(r["counts"])
+    # integer parity on the GPU's logits (whole batch)
+    oidx, ow = O.topk_softmax(lg, cfg.k, cfg.renorm)
+    np.testing.assert_array_equal(idx, oidx)
+    np.testing.assert_allclose(w, ow, rtol=GATE_RTOL, atol=1e-12)
+    ref = O.histogram_lis(oidx, cfg.m)
+    np.testing.assert_array_equal(counts, ref["counts"])
+    mx, am, lis = moe.unpack_lis(r["lis"])
+    assert (mx, am, lis) == (ref["max_count"], ref["argmax"], ref["lis"])
+    # float parity
+    toks = np.arange(cfg.T, dtype=np.int32) if n_sample >= cfg.T else sample_tokens(oidx, ref["counts"], cfg.T,
+                                                                                    n_sample)
+    exp = O.moe_output(cfg, inp, oidx, ow, tokens=toks)
+    got = out_f64(r["out"])[toks]
+    err = token_rel_err(got, exp)
+    assert err <= TOL[cfg.dtype], f"max per-token relative error {err:.3e}"
+    assert np.all(np.isfinite(out_f64(r["out"])))
+    return ref, err
+
+
+def test_tiny_fp32_all_tokens():
+    cfg = W.CONFIGS["tiny"]
+    _check_layer(cfg, W.make_moe_inputs(cfg), n_sample=cfg.T)
+
+
+def test_tiny_fp32_renormalised_and_shared():
+    cfg = W.small_moe(T=64, d=128, f=256, m=8, k=2, dtype=W.F32, zipf_s=1.2, renorm=True, n_shared=1, f_shared=64,
+                      index=71)
+    _check_layer(cfg, W.make_moe_inputs(cfg), n_sample=cfg.T)
+
+
+def test_switch_full_size():
+    cfg = W.CONFIGS["switch"]
+    ref, _ = _check_layer(cfg, W.make_moe_inputs(cfg), n_sample=48)
+    assert 2.0 <= ref["lis"] <= 4.0
+
+
+def test_mixtral_full_size():
+    cfg = W.CONFIGS["mixtral"]
+    _check_layer(cfg, W.make_moe_inputs(cfg), n_sample=12)
+
+
+def test_dsv2lite_full_size():
+    cfg = W.CONFIGS["dsv2lite"]
+    ref, _ = _check_layer(cfg, W.make_moe_inputs(cfg), n_sample=24)
+    assert 3.5 <= ref["lis"] <= 4.5
+
+
+def test_decode_all_tokens():
+    cfg = W.CONFIGS["decode"]
+    _check_layer(cfg, W.make_moe_inputs(cfg), n_sample=cfg.T)
+
+
+@pytest.mark.parametrize("case", ["one_hot", "T1", "ragged_small", "relu_many_experts"])
+def test_layer_edge_cases(case):
+    if case == "one_hot":  # every token's top-1 is the same expert (huge bias)
+        cfg = W.small_moe(T=300, d=256, f=192, m=16, k=2, dtype=W.BF16, zipf_s=0.0, index=72)
+        inp = W.make_moe_inputs(cfg)
+        inp["bias"][:] = 0.0
+        inp["bias"][11] = 1000.0
+    elif case == "T1":
+        cfg = W.small_moe(T=1, d=1024, f=512, m=8, k=2, dtype=W.BF16, zipf_s=0.8, renorm=True, index=73)
+        inp = W.make_moe_inputs(cfg)
+    elif case == "ragged_small":
+        cfg = W.small_moe(T=77, d=136, f=200, m=12, k=3, dtype=W.BF16, zipf_s=1.5, n_shared=1, f_shared=72,
+                          index=74)
+        inp = W.make_moe_inputs(cfg)
+    else:
+        cfg = W.small_moe(T=1500, d=128, f=320, m=256, k=2, act=W.RELU, dtype=W.BF16, zipf_s=1.0, index=75)
+        inp = W.make_moe_inputs(cfg)
+    ref, _ = _check_layer(cfg, inp, n_sample=min(cfg.T, 64))
+    if case == "one_hot":  # expert 11 holds every token: LIS reaches its maximum m / k
+        assert ref["counts"][11] == cfg.T and ref["lis"] == cfg.m / cfg.k
+
+
+def test_workspace_reuse_is_stable():
+    cfg = W.small_moe(T=257, d=256, f=384, m=8, k=2, dtype=W.BF16, zipf_s=1.0, index=76)
+    d_in = device_inputs(W.make_moe_inputs(cfg))
+    r1 = layer_forward(cfg, d_in)
+    r2 = layer_forward(cfg, d_in, ws=r1["ws"])
+    torch.cuda.synchronize()
+    assert torch.equal(r1["out"], r2["out"])  # deterministic: no atomics on float data
+
+
+# ------------------------------------------------------------------ atomic experts
+
+def _atomic(cfg, inp):
+    c = moe.make_atomic_config(cfg.T, cfg.d, cfg.Nr, cfg.Nc, cfg.K, cfg.act)
+    ws = moe.workspace(c)
+    d_in = device_inputs(inp)
+    lr = torch.empty((cfg.T, cfg.Nr), dtype=torch.float32, device="cuda")
+    lc = torch.empty((cfg.T, cfg.Nc), dtype=torch.float32, device="cuda")
+    idx = torch.empty((cfg.T, cfg.K), dtype=torch.int32, device="cuda")
+    g = torch.empty((cfg.T, cfg.K), dtype=torch.float32, device="cuda")
+    moe.moe_atomic_route(c, d_in["x"], d_in["w_row"], d_in["w_col"], lr, lc, idx, g, ws)
+    out = torch.empty((cfg.T, cfg.d), dtype=torch.bfloat16, device="cuda")
+    moe.moe_atomic_experts(c, d_in["x"], d_in["w_in"], d_in["w_out"], idx, g, out, ws)
+    out2 = torch.empty_like(out)
+    moe.moe_atomic_forward(c, d_in["x"], d_in["w_row"], d_in["w_col"], d_in["w_in"], d_in["w_out"], out2, ws)
+    assert moe.moe_read_device_status(ws) == moe.OK
+    return host(lr), host(lc), host(idx), host(g), out, out2
+
+
+@pytest.mark.parametrize("full", [False, True])
+def test_atomic_layer(full):
+    if full:
+        cfg = W.CONFIGS["atomic"]
+    else:
+        cfg = W.AtomicWorkload("atomic_small", 92, T=5, d=256, Nr=64, Nc=128, K=16, act=W.ACT_SIGMOID)
+    inp = W.make_atomic_inputs(cfg)
+    lr, lc, idx, g, out, out2 = _atomic(cfg, inp)
+    olr, olc = O.atomic_logprobs(inp["x"], inp["w_row"], inp["w_col"])
+    np.testing.assert_allclose(lr, olr, rtol=0, atol=2e-4)
+    np.testing.assert_allclose(lc, olc, rtol=0, atol=2e-4)
+    oidx, og = O.atomic_select(lr, lc, cfg.K)  # oracle selects on the GPU's own log-probabilities
+    np.testing.assert_array_equal(idx, oidx)
+    np.testing.assert_allclose(g, og, rtol=GATE_RTOL * 4, atol=1e-9)
+    exp = O.atomic_output(inp["x"], inp["w_in"], inp["w_out"], oidx, og, cfg.act)
+    assert token_rel_err(out_f64(out), exp) <= TOL[W.BF16]
+    torch.cuda.synchronize()
+    assert torch.equal(out, out2)
+
+
+def test_atomic_select_ties_and_rounding_collapse():
+    # Row/column weights built so many grid scores tie exactly: x = e_0 and integer-valued
+    # logits; the exact top-K must follow (S desc, flat id asc).
+    cfg = W.AtomicWorkload("atomic_ties", 93, T=2, d=64, Nr=64, Nc=64, K=64, act=W.ACT_SILU)
+    inp = W.make_atomic_inputs(cfg)
+    x = np.zeros((2, 64), np.uint16)
+    x[:, 0] = 0x3F80  # bf16 1.0
+    inp["x"] = x
+    rng = np.random.default_rng(5)
+    for key in ("w_row", "w_col"):
+        vals = rng.integers(0, 3, size=64).astype(np.float32)  # 0, 1, 2 -> heavy ties
+        wr = np.zeros((64, 64), np.uint16)
+        wr[:, 0] = (vals.view(np.uint32) >> 16).astype(np.uint16)
+        inp[key] = wr
+    lr, lc, idx, g, out, _ = _atomic(cfg, inp)
+    oidx, og = O.atomic_select(lr, lc, cfg.K)
+    np.testing.assert_array_equal(idx, oidx)
