@@ -330,6 +330,10 @@ def ours(args):
     ev_s = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
     ev_e = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
     ev_stage = [[torch.cuda.Event(enable_timing=True) for _ in range(8)] for _ in range(K)]
+    with torch.cuda.stream(s):  # torch creates the CUDA events on first record
+        for evs in ev_stage:
+            for e in evs:
+                e.record(s)
     sampler = ClockSampler(local)
     if world > 1:
         dist.barrier()

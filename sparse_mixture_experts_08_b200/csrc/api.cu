@@ -34,7 +34,8 @@ static moe_status_t mark_stage(int i, cudaStream_t s) {
   if (i < g_n_stage_events) return cudaEventRecord(g_stage_events[i], s) == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
   return MOE_OK;
 }
-constexpr int PLAN_SMS = 148;  // B200 SM count used for static planning (split-K, tile sizes)
+constexpr int PLAN_SMS = 148;
+  // B200 SM count used for static planning (split-K, tile sizes)
 
 static moe_status_t check_device() {
   static int ok_cache[64] = {0};  // 0 unknown, 1 ok, 2 unsupported
@@ -88,7 +89,7 @@ static Plan make_plan(const moe_config_t& c) {
 }
 
 struct Layout {
-  size_t status, logits, idx, w, counts, offsets, lis, perm, inv_perm, x_perm, h, h_sh, y, y_sh, total;
+  size_t status, logits, idx, w, counts, offsets, lis, perm, inv_perm, w_perm, x_perm, h, h_sh, y, y_sh, total;
 };
 
 static Layout make_layout(const moe_config_t& c, const Plan& p) {
@@ -110,6 +111,7 @@ static Layout make_layout(const moe_config_t& c, const Plan& p) {
   L.lis = take(sizeof(moe_lis_t));
   L.perm = take(Tk * 4);
   L.inv_perm = take(Tk * 4);
+  L.w_perm = take(Tk * 4);
   L.x_perm = take(Tk * c.d * p.es);
   L.h = take(Tk * c.f * p.es);
   L.h_sh = take((size_t)c.n_shared * T * std::max(c.f_shared, 0) * p.es);
@@ -159,7 +161,9 @@ static moe_status_t cuda_status(cudaError_t e) { return e == cudaSuccess ? MOE_O
 
 static moe_status_t run_router(const moe_config_t& c, const void* x, const void* w_r, const float* bias, float* logits,
                                int* status, cudaStream_t s) {
-  if (c.dtype == MOE_F32) return cuda_status(launch_simt_logits(MOE_F32, c.T, c.d, c.m, x, w_r, bias, logits, s));
+  // fp32 layers, and batches too small to fill the tensor cores (decode), use CUDA cores.
+  if (c.dtype == MOE_F32 || c.T <= 64)
+    return cuda_status(launch_simt_logits(c.dtype, c.T, c.d, c.m, x, w_r, bias, logits, s));
   // logits^T = W_r . x^T on the tensor cores: one group, features = experts.
   GemmParams p;
   std::memset(&p, 0, sizeof(p));
@@ -176,9 +180,11 @@ static moe_status_t run_router(const moe_config_t& c, const void* x, const void*
   p.n_classes = 1;
   p.status = status;
   p.wait_limit_ns = g_wait_limit_ns;
-  int bn = 128;
+  // Smallest token tile that still covers the batch in one wave of CTAs (each tile
+  // re-reads all of W_r from L2, so fewer, larger tiles are cheaper).
   const long long mt = (c.m + 127) / 128;
-  while (bn > 16 && mt * ((c.T + bn - 1) / bn) < PLAN_SMS) bn >>= 1;
+  int bn = 16;
+  while (bn < 128 && mt * ((c.T + bn - 1) / bn) > PLAN_SMS) bn <<= 1;
   TcMaps maps;
   std::memset(&maps, 0, sizeof(maps));
   maps.a0[0] = {w_r, c.m, c.d};
@@ -200,6 +206,8 @@ struct FfnIo {
   float* y;
   const float* task_w;
   const int32_t* perm;
+  const float* row_w;     // task_w already gathered into segment order (nullable)
+  void* out_k1;           // top-1 layers: the down projection writes the layer output directly
   // shared class
   int n_shared;
   const void* x;          // [T, d]
@@ -292,10 +300,12 @@ static moe_status_t run_ffn(const moe_config_t& c, const Plan& pl, const FfnIo& 
     g.kb_per_split = kbps;
     g.seg_off = io.offsets;
     g.max_row = (int)io.routed_rows;
-    g.out = io.y;
+    g.out = io.out_k1 ? io.out_k1 : io.y;
+    g.scatter_k1 = io.out_k1 ? 1 : 0;
     g.out_ld = c.d;
     g.out_split_stride = io.routed_rows * c.d;
     g.task_w = io.task_w;
+    g.row_w = io.row_w;
     g.perm = io.perm;
     g.a0 = io.w_down;
     g.b = io.h;
@@ -383,7 +393,7 @@ moe_status_t moe_histogram_lis(const moe_config_t* cfg, const int32_t* topk_idx,
   const Layout L = make_layout(c, make_plan(c));
   MOE_TRY(check_ws(c, ws, ws_bytes, L.status + 256));
   MOE_TRY(check_device());
-  return cuda_status(launch_route_index(1, c.T, c.k, c.m, topk_idx, counts, offsets, lis, nullptr, nullptr,
+  return cuda_status(launch_route_index(1, c.T, c.k, c.m, topk_idx, counts, offsets, lis, nullptr,
                                         at<int>(ws, L.status), (cudaStream_t)stream));
 }
 
@@ -403,9 +413,10 @@ moe_status_t moe_permute(const moe_config_t* cfg, const void* x, const int32_t* 
   const long long Tk = (long long)c.T * c.k;
   // Positions not covered by a valid task keep -1, so the row copy skips them.
   MOE_CUDA(cudaMemsetAsync(perm, 0xFF, (size_t)Tk * 4, s));
-  MOE_CUDA(launch_route_index(2, c.T, c.k, c.m, topk_idx, nullptr, const_cast<int32_t*>(offsets), nullptr, perm,
-                              inv_perm, at<int>(ws, L.status), s));
-  return cuda_status(launch_permute_rows(c.dtype, (int)Tk, c.k, c.d, x, perm, x_perm, s));
+  MOE_CUDA(cudaMemsetAsync(inv_perm, 0xFF, (size_t)Tk * 4, s));
+  MOE_CUDA(launch_route_index(2, c.T, c.k, c.m, topk_idx, nullptr, const_cast<int32_t*>(offsets), nullptr, inv_perm,
+                              at<int>(ws, L.status), s));
+  return cuda_status(launch_permute_rows(c.dtype, (int)Tk, c.k, c.d, x, inv_perm, nullptr, perm, nullptr, x_perm, s));
 }
 
 moe_status_t moe_grouped_ffn(const moe_config_t* cfg, const void* x_perm, const int32_t* offsets, const void* w_gate,
@@ -511,9 +522,10 @@ moe_status_t moe_layer_forward(const moe_config_t* cfg, const void* x, const voi
   MOE_TRY(mark_stage(1, s));
   MOE_CUDA(launch_topk_softmax(c.T, c.m, c.k, c.renormalize, logits, idx, w, s));
   MOE_TRY(mark_stage(2, s));
-  MOE_CUDA(launch_route_index(3, c.T, c.k, c.m, idx, counts, offsets, lis, perm, inv_perm, status, s));
+  float* w_perm = at<float>(ws, L.w_perm);
+  MOE_CUDA(launch_route_index(3, c.T, c.k, c.m, idx, counts, offsets, lis, inv_perm, status, s));
   MOE_TRY(mark_stage(3, s));
-  MOE_CUDA(launch_permute_rows(c.dtype, (int)Tk, c.k, c.d, x, perm, at<void>(ws, L.x_perm), s));
+  MOE_CUDA(launch_permute_rows(c.dtype, (int)Tk, c.k, c.d, x, inv_perm, w, perm, w_perm, at<void>(ws, L.x_perm), s));
   MOE_TRY(mark_stage(4, s));
   FfnIo io;
   std::memset(&io, 0, sizeof(io));
@@ -527,6 +539,7 @@ moe_status_t moe_layer_forward(const moe_config_t* cfg, const void* x, const voi
   io.h = at<void>(ws, L.h);
   io.y = at<float>(ws, L.y);
   io.task_w = w;
+  io.row_w = w_perm;
   io.perm = perm;
   io.n_shared = c.n_shared;
   io.x = x;
@@ -535,10 +548,16 @@ moe_status_t moe_layer_forward(const moe_config_t* cfg, const void* x, const voi
   io.ws_down = ws_down;
   io.h_sh = at<void>(ws, L.h_sh);
   io.y_sh = at<float>(ws, L.y_sh);
+  // Top-1 routing without shared experts: each token has exactly one weighted
+  // expert output, so the down projection's epilogue scatters it straight into
+  // `out` and the combine kernel (and the fp32 y_perm round trip) disappears.
+  const bool fuse_combine = c.k == 1 && c.n_shared == 0 && pl.ksplit == 1 && c.dtype == MOE_BF16;
+  io.out_k1 = fuse_combine ? out : nullptr;
   MOE_TRY(run_ffn(c, pl, io, pl.ksplit, pl.kbps, status, s, true));
   MOE_TRY(mark_stage(6, s));
-  MOE_CUDA(launch_combine(c.dtype, c.T, c.d, c.k, pl.ksplit, io.y, Tk * c.d, inv_perm, c.n_shared, io.y_sh,
-                          (long long)c.n_shared * c.T * c.d, out, s));
+  if (!fuse_combine)
+    MOE_CUDA(launch_combine(c.dtype, c.T, c.d, c.k, pl.ksplit, io.y, Tk * c.d, inv_perm, c.n_shared, io.y_sh,
+                            (long long)c.n_shared * c.T * c.d, out, s));
   return mark_stage(7, s);
 }
 

@@ -46,8 +46,10 @@ struct GemmClass {
   long long out_ld;          // elements between output rows
   long long out_split_stride;// elements between k-split partial outputs
   const float* bias;         // LOGITS: bias[feature] (nullable)
+  const float* row_w;        // DOWN: weight of output row `row` (nullable; preferred over task_w)
   const float* task_w;       // DOWN: row weight task_w[perm[row]] (nullable = 1)
   const int* perm;
+  int scatter_k1;            // DOWN with top-1 routing: write bf16 out[perm[row]] (combine fused)
   // SIMT path only (fp32 / bf16 element pointers, row-major)
   const void* a0;            // [n_groups * R, K]
   const void* a1;            // second matrix (SwiGLU up) or nullptr
@@ -85,11 +87,11 @@ cudaError_t launch_simt_logits(int dtype, int T, int d, int m, const void* x, co
                                float* logits, cudaStream_t s);
 cudaError_t launch_topk_softmax(int T, int m, int k, int renorm, const float* logits, int32_t* idx, float* w,
                                 cudaStream_t s);
-// mode bit 1: histogram (counts, offsets, lis from idx); bit 2: ranks (perm, inv_perm from offsets)
+// mode bit 1: histogram (counts, offsets, lis from idx); bit 2: inv_perm (stable positions from offsets)
 cudaError_t launch_route_index(int mode, int T, int k, int m, const int32_t* idx, int32_t* counts, int32_t* offsets,
-                               moe_lis_t* lis, int32_t* perm, int32_t* inv_perm, int* status, cudaStream_t s);
-cudaError_t launch_permute_rows(int dtype, int Tk, int k, int d, const void* x, const int32_t* perm, void* x_perm,
-                                cudaStream_t s);
+                               moe_lis_t* lis, int32_t* inv_perm, int* status, cudaStream_t s);
+cudaError_t launch_permute_rows(int dtype, int Tk, int k, int d, const void* x, const int32_t* inv_perm,
+                                const float* task_w, int32_t* perm, float* w_perm, void* x_perm, cudaStream_t s);
 cudaError_t launch_combine(int dtype, int T, int d, int k, int ksplit, const float* y_perm, long long y_split_stride,
                            const int32_t* inv_perm, int n_shared, const float* y_shared, long long ysh_split_stride,
                            void* out, cudaStream_t s);

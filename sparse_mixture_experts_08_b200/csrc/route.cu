@@ -121,51 +121,84 @@ cudaError_t launch_topk_softmax(int T, int m, int k, int renorm, const float* lo
 }
 
 // ------------------------------------------------ histogram, offsets, LIS, ranks
-// One block of 1024 threads (the routing tables are tiny: T k ids).
-// mode & 1: n_e = #{q : idx[q] = e} (shared-memory atomics), offsets = exclusive
-//           scan, max / lowest argmax, LIS = m max / (T k) (R&Q Definition 1).
-// mode & 2: stable rank of each task inside its expert's segment, chunk by chunk
-//           of 1024 tasks: rank within the warp from __match_any_sync, rank of the
-//           warp among the chunk's warps from a [32][m] count table scanned per
-//           expert, plus the expert's running cursor from earlier chunks. Then
-//           pos = offsets[e] + rank; perm[pos] = q; inv_perm[q] = pos.
+// One block of 1024 threads (the routing tables are tiny: T k ids). Warp w owns
+// the contiguous task range [w L, (w + 1) L), L = ceil(T k / 32), walked 32 tasks
+// at a time in increasing task id.
+//  pass 1: per-warp counts wc[w][e] (peer groups from __match_any_sync; each warp
+//          writes only its own row, so no atomics).
+//  scan:   per expert, exclusive prefix over warps -> wc[w][e] = tasks of e in
+//          warps before w; the total is n_e.
+// mode & 1: offsets = exclusive scan of n_e, max / lowest argmax, and
+//           LIS = m max / (T k) (R&Q Definition 1).
+// mode & 2: pass 2 re-walks each warp's range in the same order:
+//           pos = offsets[e] + wc[w][e] + (rank among the sub-chunk's peers), then
+//           wc[w][e] += peers: the stable counting-sort position, inv_perm[q] = pos
+//           (its inverse perm[pos] = q is scattered by the many-block row copy, so
+//           this one-SM kernel issues only coalesced stores).
 // Any id outside [0, m) (or, with given offsets, a position outside its segment)
 // sets MOE_ERR_DEVICE_INDEX and nothing further is written.
+constexpr int RI_MAX_REG = 16;  // sub-chunks per warp kept in registers between the passes
+
 __global__ void __launch_bounds__(RI_THREADS, 1)
     route_index_kernel(int mode, int T, int k, int m, const int32_t* __restrict__ idx, int32_t* __restrict__ counts,
-                       int32_t* __restrict__ offsets, moe_lis_t* __restrict__ lis, int32_t* __restrict__ perm,
-                       int32_t* __restrict__ inv_perm, int* status) {
+                       int32_t* __restrict__ offsets, moe_lis_t* __restrict__ lis, int32_t* __restrict__ inv_perm,
+                       int* status) {
   extern __shared__ int sm[];
-  int* cnt = sm;             // [m]
-  int* off = cnt + m;        // [m + 1]
-  int* cur = off + m + 1;    // [m]
-  int* tab = cur + m;        // [32][m]
+  int* wc = sm;             // [32][m]
+  int* off = wc + 32 * m;   // [m + 1]
   __shared__ int bad;
   __shared__ int wsum[32], wmax[32], warg[32];
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int nw = blockDim.x >> 5;
   const int Tk = T * k;
+  const int L = (Tk + nw - 1) / nw;
+  const int lo = min(Tk, warp * L), hi = min(Tk, lo + L);
+  const unsigned lt = (1u << lane) - 1u;
   if (tid == 0) bad = 0;
-  for (int e = tid; e < m; e += blockDim.x) {
-    cnt[e] = 0;
-    cur[e] = 0;
-  }
-  for (int i = tid; i < nw * m; i += blockDim.x) tab[i] = 0;
+  for (int i = tid; i < nw * m; i += blockDim.x) wc[i] = 0;
   __syncthreads();
-  for (int q = tid; q < Tk; q += blockDim.x) {
-    const int e = idx[q];
-    if (e < 0 || e >= m)
+  // All of this warp's ids (up to RI_MAX_REG sub-chunks) are loaded up front so the
+  // loads overlap; longer ranges reload the rest in the loops below.
+  int ev[RI_MAX_REG];
+#pragma unroll
+  for (int r = 0; r < RI_MAX_REG; ++r) {
+    const int q = lo + r * 32 + lane;
+    ev[r] = q < hi ? idx[q] : -1;
+  }
+  for (int base = lo, r = 0; base < hi; base += 32, ++r) {
+    const int q = base + lane;
+    int e = -1;
+    if (r < RI_MAX_REG) {
+#pragma unroll
+      for (int rr = 0; rr < RI_MAX_REG; ++rr)
+        if (rr == r) e = ev[rr];
+    } else {
+      e = q < hi ? idx[q] : -1;
+    }
+    if (q < hi && (e < 0 || e >= m)) {
       bad = 1;
-    else if (mode & 1)
-      atomicAdd(&cnt[e], 1);
+      e = -2;
+    }
+    const unsigned peers = __match_any_sync(FULL, e);
+    if (e >= 0 && lane == __ffs(peers) - 1) wc[warp * m + e] += __popc(peers);
   }
   __syncthreads();
   if (bad) {
     if (tid == 0) set_status(status, MOE_ERR_DEVICE_INDEX);
     return;
   }
+  for (int e = tid; e < m; e += blockDim.x) {
+    int run = 0;
+    for (int w = 0; w < nw; ++w) {
+      const int t = wc[w * m + e];
+      wc[w * m + e] = run;
+      run += t;
+    }
+    off[e] = run;  // n_e for now
+  }
+  __syncthreads();
   if (mode & 1) {
-    const int c = tid < m ? cnt[tid] : 0;
+    const int c = tid < m ? off[tid] : 0;
     int incl = c;
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
@@ -188,14 +221,14 @@ __global__ void __launch_bounds__(RI_THREADS, 1)
     }
     __syncthreads();
     if (warp == 0) {
-      int ws = lane < nw ? wsum[lane] : 0;
+      const int ws = lane < nw ? wsum[lane] : 0;
       int wi = ws;
 #pragma unroll
       for (int o = 1; o < 32; o <<= 1) {
         const int v = __shfl_up_sync(FULL, wi, o);
         if (lane >= o) wi += v;
       }
-      wsum[lane] = wi - ws;  // exclusive prefix of the warp totals
+      wsum[lane] = wi - ws;
       int bv = lane < nw ? wmax[lane] : -1, ba = lane < nw ? warg[lane] : 0x7fffffff;
 #pragma unroll
       for (int o = 16; o; o >>= 1) {
@@ -227,50 +260,42 @@ __global__ void __launch_bounds__(RI_THREADS, 1)
       lis->lis = (double)((long long)m * wmax[0]) / (double)((long long)T * k);
     }
   } else {
+    __syncthreads();
     for (int e = tid; e <= m; e += blockDim.x) off[e] = offsets[e];
   }
   __syncthreads();
   if (!(mode & 2)) return;
-  for (int base = 0; base < Tk; base += blockDim.x) {
-    const int q = base + tid;
-    const bool valid = q < Tk;
-    const int e = valid ? idx[q] : -1;
-    const unsigned peers = __match_any_sync(FULL, e);
-    const int rank = __popc(peers & ((1u << lane) - 1u));
-    const int leader = __ffs(peers) - 1;
-    if (valid && lane == leader) tab[warp * m + e] = __popc(peers);
-    __syncthreads();
-    for (int ee = tid; ee < m; ee += blockDim.x) {
-      int run = cur[ee];
-      for (int w = 0; w < nw; ++w) {
-        const int t = tab[w * m + ee];
-        if (t) {
-          tab[w * m + ee] = run;
-          run += t;
-        }
-      }
-      cur[ee] = run;
+  for (int base = lo, r = 0; base < hi; base += 32, ++r) {
+    const int q = base + lane;
+    int e = -1;
+    if (r < RI_MAX_REG) {
+#pragma unroll
+      for (int rr = 0; rr < RI_MAX_REG; ++rr)
+        if (rr == r) e = ev[rr];
+    } else {
+      e = q < hi ? idx[q] : -1;
     }
-    __syncthreads();
-    if (valid) {
-      const int pos = off[e] + tab[warp * m + e] + rank;
+    const unsigned peers = __match_any_sync(FULL, e);
+    const int leader = __ffs(peers) - 1;
+    const int b = e >= 0 ? wc[warp * m + e] : 0;
+    __syncwarp();
+    if (e >= 0) {
+      const int pos = off[e] + b + __popc(peers & lt);
       if (pos >= 0 && pos >= off[e] && pos < off[e + 1] && pos < Tk) {
-        perm[pos] = q;
-        inv_perm[q] = pos;
+        inv_perm[q] = pos;  // coalesced; the scattered perm[pos] is written by the row copy
       } else {
         set_status(status, MOE_ERR_DEVICE_INDEX);
       }
+      if (lane == leader) wc[warp * m + e] = b + __popc(peers);
     }
-    __syncthreads();
-    if (valid && lane == leader) tab[warp * m + e] = 0;
-    __syncthreads();
+    __syncwarp();
   }
 }
 
-size_t route_index_smem(int m) { return sizeof(int) * ((size_t)3 * m + 1 + (size_t)32 * m); }
+size_t route_index_smem(int m) { return sizeof(int) * ((size_t)33 * m + 1); }
 
 cudaError_t launch_route_index(int mode, int T, int k, int m, const int32_t* idx, int32_t* counts, int32_t* offsets,
-                               moe_lis_t* lis, int32_t* perm, int32_t* inv_perm, int* status, cudaStream_t s) {
+                               moe_lis_t* lis, int32_t* inv_perm, int* status, cudaStream_t s) {
   const size_t smem = route_index_smem(m);
   static size_t attr = 0;
   if (smem > 48 * 1024 && smem > attr) {
@@ -278,31 +303,40 @@ cudaError_t launch_route_index(int mode, int T, int k, int m, const int32_t* idx
     if (e != cudaSuccess) return e;
     attr = smem;
   }
-  route_index_kernel<<<1, RI_THREADS, smem, s>>>(mode, T, k, m, idx, counts, offsets, lis, perm, inv_perm, status);
+  route_index_kernel<<<1, RI_THREADS, smem, s>>>(mode, T, k, m, idx, counts, offsets, lis, inv_perm, status);
   count_launch();
   return cudaGetLastError();
 }
 
 // ------------------------------------------------------------------ permute rows
-// x_perm[pos, :] = x[perm[pos] / k, :]; one warp per row, 16-byte vectors.
+// Walks the tasks q in order (one warp each): pos = inv_perm[q];
+// x_perm[pos, :] = x[q / k, :] with 16-byte vectors; perm[pos] = q; and, when
+// given, w_perm[pos] = task_w[q] (the gate weight in segment order, read by the
+// down-projection epilogue).
 __global__ void permute_rows_kernel(int Tk, int k, int chunks, const int4* __restrict__ x,
-                                    const int32_t* __restrict__ perm, int4* __restrict__ x_perm) {
+                                    const int32_t* __restrict__ inv_perm, const float* __restrict__ task_w,
+                                    int32_t* __restrict__ perm, float* __restrict__ w_perm, int4* __restrict__ x_perm) {
   const int lane = threadIdx.x & 31;
   const long long warps = (long long)gridDim.x * (blockDim.x >> 5);
-  for (long long pos = (long long)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); pos < Tk; pos += warps) {
-    const int q = perm[pos];
-    if (q < 0 || q >= Tk) continue;
-    const int4* src = x + (long long)(q / k) * chunks;
-    int4* dst = x_perm + pos * chunks;
+  for (long long q = (long long)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); q < Tk; q += warps) {
+    const int pos = inv_perm[q];
+    if (pos < 0 || pos >= Tk) continue;
+    if (lane == 0) {
+      perm[pos] = (int32_t)q;
+      if (w_perm) w_perm[pos] = task_w[q];
+    }
+    const int4* src = x + (q / k) * chunks;
+    int4* dst = x_perm + (long long)pos * chunks;
     for (int c = lane; c < chunks; c += 32) dst[c] = src[c];
   }
 }
 
-cudaError_t launch_permute_rows(int dtype, int Tk, int k, int d, const void* x, const int32_t* perm, void* x_perm,
-                                cudaStream_t s) {
+cudaError_t launch_permute_rows(int dtype, int Tk, int k, int d, const void* x, const int32_t* inv_perm,
+                                const float* task_w, int32_t* perm, float* w_perm, void* x_perm, cudaStream_t s) {
   const int chunks = d * (dtype == MOE_F32 ? 4 : 2) / 16;
   const int blocks = std::max(1, std::min((Tk + 7) / 8, num_sms() * 8));
-  permute_rows_kernel<<<blocks, 256, 0, s>>>(Tk, k, chunks, (const int4*)x, perm, (int4*)x_perm);
+  permute_rows_kernel<<<blocks, 256, 0, s>>>(Tk, k, chunks, (const int4*)x, inv_perm, task_w, perm, w_perm,
+                                             (int4*)x_perm);
   count_launch();
   return cudaGetLastError();
 }

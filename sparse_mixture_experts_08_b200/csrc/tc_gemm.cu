@@ -200,24 +200,45 @@ __device__ __forceinline__ void decode_tile(const GemmParams& p, const SchedSmem
   ti.kb1 = min(KB, ti.kb0 + c.kb_per_split);
 }
 
+// Per-row epilogue data for a chunk of 16 output rows, loaded once per warp (lane
+// l < 16 handles row c0 + l) and broadcast with shuffles: the gate weight of the
+// row's task and, for the fused top-1 combine, the destination token.
+struct RowAux {
+  float w;
+  int dst;
+};
+
+template <int EPI>
+__device__ __forceinline__ RowAux load_row_aux(const GemmClass& c, const TileInfo& ti, int j) {
+  RowAux a{1.f, -1};
+  if (EPI != EPI_DOWN || j >= ti.rows_in_tile) return a;
+  const long long row = (long long)ti.out_row + j;
+  if (c.row_w) a.w = c.row_w[row];
+  if ((c.task_w && !c.row_w) || c.scatter_k1) {
+    const int q = c.perm[row];
+    const bool ok = q >= 0 && q < c.max_row;
+    if (c.task_w && !c.row_w) a.w = ok ? c.task_w[q] : 0.f;
+    a.dst = ok ? q : -1;
+  }
+  return a;
+}
+
 template <int EPI>
 __device__ __forceinline__ void store_out(const GemmClass& c, const TileInfo& ti, int feature, int j, float v0,
-                                          float v1) {
+                                          float v1, float bias, float wgt, int dst) {
   const long long row = (long long)ti.out_row + j;
   if (EPI == EPI_LOGITS) {
     float* o = reinterpret_cast<float*>(c.out) + (long long)ti.ks * c.out_split_stride;
-    o[row * c.out_ld + feature] = v0 + (c.bias ? c.bias[feature] : 0.f);
+    o[row * c.out_ld + feature] = v0 + bias;
   } else if (EPI == EPI_SWIGLU) {
     const float h = v0 / (1.f + __expf(-v0)) * v1;
     reinterpret_cast<__nv_bfloat16*>(c.out)[row * c.out_ld + feature] = __float2bfloat16_rn(h);
   } else if (EPI == EPI_RELU) {
     reinterpret_cast<__nv_bfloat16*>(c.out)[row * c.out_ld + feature] = __float2bfloat16_rn(fmaxf(v0, 0.f));
+  } else if (c.scatter_k1) {  // EPI_DOWN, combine fused: one task per token
+    if (dst >= 0)
+      reinterpret_cast<__nv_bfloat16*>(c.out)[(long long)dst * c.out_ld + feature] = __float2bfloat16_rn(v0 * wgt);
   } else {  // EPI_DOWN
-    float wgt = 1.f;
-    if (c.task_w) {
-      const int q = c.perm[row];
-      wgt = (q >= 0 && q < c.max_row) ? c.task_w[q] : 0.f;
-    }
     float* o = reinterpret_cast<float*>(c.out) + (long long)ti.ks * c.out_split_stride;
     o[row * c.out_ld + feature] = v0 * wgt;
   }
@@ -234,6 +255,8 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
 
   __shared__ SchedSmem sched;
   __shared__ __align__(8) uint64_t full_bar[STAGES], empty_bar[STAGES], accf_bar[2], acce_bar[2], drain_bar;
+  __shared__ float aux_w[4][EPI == EPI_DOWN ? BN : 1];  // per epilogue warp: row weights of the tile
+  __shared__ int aux_d[4][EPI == EPI_DOWN ? BN : 1];    // and destination tokens (fused top-1 combine)
   __shared__ uint32_t tmem_base_s;
   __shared__ int abort_s;
   __shared__ int total_tiles_s;
@@ -420,6 +443,22 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
     for (int w = blockIdx.x; w < total; w += gridDim.x) {
       TileInfo ti;
       decode_tile<BN>(p, sched, G, w, ti);
+      const GemmClass& c = p.cls[ti.cls];
+      const int feature = ti.mt * TC_BM + q * 32 + lane;
+      const bool fvalid = feature < c.R;
+      const bool has_k = ti.kb1 > ti.kb0;  // an empty K range leaves the accumulator unwritten
+      const float bias = (EPI == EPI_LOGITS && c.bias && fvalid) ? c.bias[feature] : 0.f;
+      // Row data of the whole tile (gate weight, destination token), fetched into this
+      // warp's shared-memory slice before waiting for the accumulator so the loads
+      // overlap the MMAs; the chunk loop below then reads it with broadcasts.
+      if (EPI == EPI_DOWN) {
+        for (int j = lane; j < BN; j += 32) {
+          const RowAux a = load_row_aux<EPI>(c, ti, j);
+          aux_w[q][j] = a.w;
+          aux_d[q][j] = a.dst;
+        }
+        __syncwarp();
+      }
       const bool got = mbar_wait(&accf_bar[acc], acc_phase, lim, abort_flag);
       if (!got) {
         set_status(p.status, MOE_ERR_TIMEOUT);
@@ -427,23 +466,21 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
         break;
       }
       tc_fence_after();
-      const GemmClass& c = p.cls[ti.cls];
-      const int feature = ti.mt * TC_BM + q * 32 + lane;
-      const bool fvalid = feature < c.R;
-      const bool has_k = ti.kb1 > ti.kb0;  // an empty K range leaves the accumulator unwritten
       const uint32_t t_row = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * S::ACC_COLS);
+#pragma unroll 1
       for (int c0 = 0; c0 < ti.rows_in_tile; c0 += 16) {
         uint32_t r0[16], r1[16];
         tmem_ld_x16(t_row + c0, r0);
         if (MATS == 2) tmem_ld_x16(t_row + BN + c0, r1);
         tmem_ld_wait();
+        const int jn = min(16, ti.rows_in_tile - c0);
         if (fvalid) {
-          const int jn = min(16, ti.rows_in_tile - c0);
 #pragma unroll
           for (int j = 0; j < 16; ++j)
             if (j < jn)
               store_out<EPI>(c, ti, feature, c0 + j, has_k ? __uint_as_float(r0[j]) : 0.f,
-                             (MATS == 2 && has_k) ? __uint_as_float(r1[j]) : 0.f);
+                             (MATS == 2 && has_k) ? __uint_as_float(r1[j]) : 0.f, bias,
+                             EPI == EPI_DOWN ? aux_w[q][c0 + j] : 1.f, EPI == EPI_DOWN ? aux_d[q][c0 + j] : -1);
         }
       }
       tc_fence_before();
@@ -519,10 +556,14 @@ static cudaError_t launch_impl(const TcMaps& maps, const GemmParams& p, int num_
   return cudaGetLastError();
 }
 
+// Token rows per tile: about twice the mean segment, so most experts' segments fit
+// one tile and each weight tile is streamed once (every extra row tile of a segment
+// re-reads the expert's weights), capped by TMEM (two SwiGLU accumulators of BN
+// columns, double-buffered, must fit 512 columns).
 int tc_pick_bn(int epi, double avg) {
   const int cap = (epi == EPI_SWIGLU || epi == EPI_LOGITS) ? 128 : 256;
   int bn = 16;
-  while (bn < cap && bn < avg) bn <<= 1;
+  while (bn < cap && bn < 2.0 * avg) bn <<= 1;
   return bn;
 }
 
