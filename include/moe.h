@@ -192,6 +192,25 @@ MOE_API moe_status_t moe_atomic_forward(const moe_atomic_config_t* cfg, const vo
                                 const void* w_in, const void* w_out, void* out, int32_t* idx_out, float* g_out,
                                 void* ws, size_t ws_bytes, moe_stream_t stream);
 
+/* moe_route without a workspace, for callers that cannot allocate device memory:
+ * code running while a CUDA graph is captured (cudaMalloc is not allowed then),
+ * plugins that only see the tensors a host framework hands them, or request paths
+ * that must not allocate. (The reviewed pages have no counterpart: this is a
+ * deployment convenience, not part of the method.) Same arguments and results as
+ * moe_route, except that the status word and - when neither logits_in nor
+ * logits_out is given - the router logits live in an 8 MiB array compiled into
+ * the library, held on every GPU that loads it until the process exits. It
+ * allocates nothing. Limits: T * m <= 2,097,088 when the logits go to that
+ * array, else MOE_ERR_WORKSPACE is returned before any launch. The status word
+ * is cleared at the start of each call and, when device_status_out (device
+ * pointer, nullable) is given, copied there at the end (0 = ok, else a
+ * moe_status_t). All calls on a device share the array: calls whose work overlaps
+ * on the GPU race on it, so order them on one stream. The first call on each
+ * device looks up the array's address; make it before any stream capture. */
+MOE_API moe_status_t moe_route_static(const moe_config_t* cfg, const void* x, const void* w_router, const float* bias,
+                                      const float* logits_in, float* logits_out, int32_t* topk_idx, float* topk_w,
+                                      int32_t* device_status_out, moe_stream_t stream);
+
 /* Synchronises `stream`, reads the status word of `ws` into *out (host) and
  * clears it. Returns MOE_ERR_CUDA if the synchronisation or copy fails. */
 MOE_API moe_status_t moe_read_device_status(void* ws, moe_stream_t stream, moe_status_t* out);

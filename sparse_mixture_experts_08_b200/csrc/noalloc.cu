@@ -1,0 +1,142 @@
+// moe_route_static: the router (logits -> top-k -> gate weights) for callers that
+// cannot hand the library a workspace.
+//
+// Some callers have no way to obtain device memory for scratch: code that runs
+// while a CUDA graph is being captured (cudaMalloc is not allowed then), plugins
+// that only ever see the tensors a host framework gives them, or serving loops
+// that forbid allocation on the request path. moe_route needs scratch for the
+// intermediate router logits (when the caller does not want them) and for the
+// device status word; this entry point keeps both in a fixed array compiled into
+// the library instead, and allocates nothing.
+//
+// Limits and sharing:
+//  - The array holds MOE_STATIC_SCRATCH_BYTES (8 MiB) on every GPU that loads the
+//    library, for the life of the process: the status word plus at most
+//    (8 MiB - 256 B) / 4 router logits, i.e. T * m <= 2,097,088 when neither
+//    logits_in nor logits_out is given. Larger calls are rejected with
+//    MOE_ERR_WORKSPACE before anything is launched.
+//  - All calls on a device share the one array and it keeps whatever the last
+//    call left in it; the status word is cleared at the start of every call.
+//    Calls whose work overlaps on the GPU (different streams without ordering
+//    between them) race on the array: order them on one stream.
+//  - The first call on each device looks up the array's device address with
+//    cudaGetSymbolAddress (with that device current); make that first call
+//    before starting any stream capture.
+#include <algorithm>
+#include <cstring>
+#include <initializer_list>
+
+#include "common.cuh"
+
+namespace moe {
+
+constexpr size_t MOE_STATIC_SCRATCH_BYTES = 8u << 20;
+constexpr size_t STATIC_STATUS_BYTES = 256;  // status word, padded so the logits stay 256-byte aligned
+
+static __device__ __align__(256) unsigned char g_static_scratch[MOE_STATIC_SCRATCH_BYTES];
+
+namespace {
+
+constexpr int MAX_DEVICES = 64;
+unsigned char* g_scratch_ptr[MAX_DEVICES] = {nullptr};
+
+// Device address of g_static_scratch on the current device (looked up once per
+// device). In host code the array's name is only a host-side handle.
+moe_status_t scratch_address(unsigned char** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= MAX_DEVICES) return MOE_ERR_CUDA;
+  if (!g_scratch_ptr[dev]) {
+    void* ptr = nullptr;
+    if (cudaGetSymbolAddress(&ptr, g_static_scratch) != cudaSuccess || !ptr) return MOE_ERR_CUDA;
+    g_scratch_ptr[dev] = static_cast<unsigned char*>(ptr);
+  }
+  *out = g_scratch_ptr[dev];
+  return MOE_OK;
+}
+
+moe_status_t device_is_sm100() {
+  int dev = 0, major = 0, minor = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return MOE_ERR_CUDA;
+  if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess)
+    return MOE_ERR_CUDA;
+  return (major == 10 && minor == 0) ? MOE_OK : MOE_ERR_UNSUPPORTED;
+}
+
+bool aligned16(const void* p) { return ((uintptr_t)p & 15u) == 0; }
+
+}  // namespace
+}  // namespace moe
+
+using namespace moe;
+
+extern "C" MOE_API moe_status_t moe_route_static(const moe_config_t* cfg, const void* x, const void* w_router,
+                                                 const float* bias, const float* logits_in, float* logits_out,
+                                                 int32_t* topk_idx, float* topk_w, int32_t* device_status_out,
+                                                 moe_stream_t stream) {
+  size_t unused = 0;
+  const moe_status_t cfg_ok = moe_workspace_size(cfg, &unused);  // full config validation
+  if (cfg_ok != MOE_OK) return cfg_ok;
+  const moe_config_t& c = *cfg;
+  if (!topk_idx || !topk_w) return MOE_ERR_INVALID_ARG;
+  if (!logits_in && (!x || !w_router)) return MOE_ERR_INVALID_ARG;
+  for (const void* p : std::initializer_list<const void*>{x, w_router, bias, logits_in, logits_out, topk_idx, topk_w})
+    if (p && !aligned16(p)) return MOE_ERR_INVALID_ARG;
+  if (device_status_out && ((uintptr_t)device_status_out & 3u)) return MOE_ERR_INVALID_ARG;
+  const size_t logits_bytes = (size_t)c.T * c.m * sizeof(float);
+  const bool need_logits_scratch = !logits_in && !logits_out;
+  if (need_logits_scratch && logits_bytes > MOE_STATIC_SCRATCH_BYTES - STATIC_STATUS_BYTES) return MOE_ERR_WORKSPACE;
+  moe_status_t st = device_is_sm100();
+  if (st != MOE_OK) return st;
+  unsigned char* scratch = nullptr;
+  if ((st = scratch_address(&scratch)) != MOE_OK) return st;
+
+  cudaStream_t s = (cudaStream_t)stream;
+  int* status = reinterpret_cast<int*>(scratch);
+  if (cudaMemsetAsync(status, 0, sizeof(int), s) != cudaSuccess) return MOE_ERR_CUDA;
+  const float* lg = logits_in;
+  if (!lg) {
+    float* dst = logits_out ? logits_out : reinterpret_cast<float*>(scratch + STATIC_STATUS_BYTES);
+    cudaError_t e;
+    if (c.dtype == MOE_F32 || c.T <= 64) {
+      e = launch_simt_logits(c.dtype, c.T, c.d, c.m, x, w_router, bias, dst, s);
+    } else {
+      // logits^T = W_r . x^T on the tensor cores, one token tile per CTA in one wave
+      GemmParams p;
+      std::memset(&p, 0, sizeof(p));
+      GemmClass& g = p.cls[0];
+      g.n_groups = 1;
+      g.R = c.m;
+      g.K = c.d;
+      g.ksplit = 1;
+      g.kb_per_split = (c.d + 63) / 64;
+      g.const_rows = c.T;
+      g.out = dst;
+      g.out_ld = c.m;
+      g.bias = bias;
+      p.n_classes = 1;
+      p.status = status;
+      p.wait_limit_ns = 2000ull * 1000 * 1000;
+      const long long mt = (c.m + 127) / 128;
+      int bn = 16;
+      while (bn < 128 && mt * ((c.T + bn - 1) / bn) > 148) bn <<= 1;
+      TcMaps maps;
+      std::memset(&maps, 0, sizeof(maps));
+      maps.a0[0] = {w_router, c.m, c.d};
+      maps.a1[0] = maps.a0[0];
+      maps.b[0] = {x, c.T, c.d};
+      const long long tiles = mt * ((c.T + bn - 1) / bn);
+      e = launch_tc_gemm(EPI_LOGITS, bn, maps, p, (int)std::min<long long>(tiles, num_sms()), s);
+    }
+    if (e != cudaSuccess) return MOE_ERR_CUDA;
+    lg = dst;
+  } else if (logits_out && logits_out != logits_in) {
+    if (cudaMemcpyAsync(logits_out, logits_in, logits_bytes, cudaMemcpyDeviceToDevice, s) != cudaSuccess)
+      return MOE_ERR_CUDA;
+  }
+  if (launch_topk_softmax(c.T, c.m, c.k, c.renormalize, lg, topk_idx, topk_w, s) != cudaSuccess) return MOE_ERR_CUDA;
+  if (device_status_out &&
+      cudaMemcpyAsync(device_status_out, status, sizeof(int32_t), cudaMemcpyDeviceToDevice, s) != cudaSuccess)
+    return MOE_ERR_CUDA;
+  return MOE_OK;
+}

@@ -30,7 +30,7 @@ STATUS_NAMES = {0: "MOE_OK", 1: "MOE_ERR_INVALID_ARG", 2: "MOE_ERR_UNSUPPORTED",
 EXPORTS = ["moe_workspace_size", "moe_atomic_workspace_size", "moe_route", "moe_histogram_lis", "moe_permute",
            "moe_grouped_ffn", "moe_shared_ffn", "moe_combine", "moe_layer_forward", "moe_atomic_route",
            "moe_atomic_experts", "moe_atomic_forward", "moe_read_device_status", "moe_status_string",
-           "moe_debug_set_wait_limit_ns", "moe_set_stage_events", "moe_launch_count"]
+           "moe_debug_set_wait_limit_ns", "moe_set_stage_events", "moe_launch_count", "moe_route_static"]
 
 
 class MoEConfig(ctypes.Structure):
@@ -79,6 +79,7 @@ def lib() -> ctypes.CDLL:
             "moe_read_device_status": [P, P, P],
             "moe_debug_set_wait_limit_ns": [ctypes.c_uint64],
             "moe_set_stage_events": [P, ctypes.c_int],
+            "moe_route_static": [P, P, P, P, P, P, P, P, P, P],
         }
         for name, args in sig.items():
             fn = getattr(L, name)
@@ -141,6 +142,14 @@ def moe_route(cfg, x, w_router, bias, logits_in, logits_out, topk_idx, topk_w, w
     _check("moe_route", lib().moe_route(ctypes.byref(cfg), _p(x), _p(w_router), _p(bias), _p(logits_in),
                                         _p(logits_out), _p(topk_idx), _p(topk_w), _p(ws), ws.numel(),
                                         _stream(stream)))
+
+
+def moe_route_static(cfg, x, w_router, bias, logits_in, logits_out, topk_idx, topk_w, device_status_out=None,
+                     stream=None):
+    """moe_route without a workspace (scratch compiled into the library; see include/moe.h)."""
+    _check("moe_route_static", lib().moe_route_static(ctypes.byref(cfg), _p(x), _p(w_router), _p(bias),
+                                                      _p(logits_in), _p(logits_out), _p(topk_idx), _p(topk_w),
+                                                      _p(device_status_out), _stream(stream)))
 
 
 def moe_histogram_lis(cfg, topk_idx, counts, offsets, lis, ws, stream=None):
