@@ -134,7 +134,9 @@ MOE_API moe_status_t moe_histogram_lis(const moe_config_t* cfg, const int32_t* t
  * expert e): segments are contiguous and ordered by task id. Writes
  * perm[pos] = q, inv_perm[q] = pos and x_perm[pos, :] = x[q / k, :]. A task
  * whose id or position falls outside the segment given by `offsets` sets
- * MOE_ERR_DEVICE_INDEX and is not written. */
+ * MOE_ERR_DEVICE_INDEX; such a task keeps inv_perm[q] = -1 and its perm / x_perm
+ * rows are not written (an id outside [0, m) anywhere leaves every inv_perm entry
+ * at -1 and writes no perm or x_perm row). */
 MOE_API moe_status_t moe_permute(const moe_config_t* cfg, const void* x, const int32_t* topk_idx, const int32_t* offsets,
                          void* x_perm, int32_t* perm, int32_t* inv_perm, void* ws, size_t ws_bytes,
                          moe_stream_t stream);
@@ -227,8 +229,10 @@ MOE_API moe_status_t moe_debug_set_wait_limit_ns(uint64_t ns);
  * cudaEvent_t handles in `events` (host array, caller-owned events) on its
  * stream at its stage boundaries, in order: 0 start, 1 router logits, 2 top-k,
  * 3 histogram/LIS/ranks, 4 row permutation, 5 up projection, 6 down projection,
- * 7 combine (n <= 8; extra stages are not recorded). n = 0 turns it off. The
- * array is copied. Process-wide and not thread-safe; meant for benchmarks. */
+ * 7 combine (n <= 8; extra stages are not recorded). A NULL entry skips that
+ * boundary (a recorded event between two kernels stops the second one from
+ * starting early, so record only the boundaries you time). n = 0 turns it off.
+ * The array is copied. Process-wide and not thread-safe; meant for benchmarks. */
 MOE_API moe_status_t moe_set_stage_events(void* const* events, int n);
 
 /* Number of kernels this library launched since the process started (host

@@ -31,7 +31,8 @@ static cudaEvent_t g_stage_events[8];
 static int g_n_stage_events = 0;
 
 static moe_status_t mark_stage(int i, cudaStream_t s) {
-  if (i < g_n_stage_events) return cudaEventRecord(g_stage_events[i], s) == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+  if (i < g_n_stage_events && g_stage_events[i])
+    return cudaEventRecord(g_stage_events[i], s) == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
   return MOE_OK;
 }
 constexpr int PLAN_SMS = 148;
@@ -89,7 +90,7 @@ static Plan make_plan(const moe_config_t& c) {
 }
 
 struct Layout {
-  size_t status, logits, idx, w, counts, offsets, lis, perm, inv_perm, w_perm, x_perm, h, h_sh, y, y_sh, total;
+  size_t status, logits, idx, w, counts, offsets, lis, perm, inv_perm, w_perm, start, x_perm, h, h_sh, y, y_sh, total;
 };
 
 static Layout make_layout(const moe_config_t& c, const Plan& p) {
@@ -112,6 +113,7 @@ static Layout make_layout(const moe_config_t& c, const Plan& p) {
   L.perm = take(Tk * 4);
   L.inv_perm = take(Tk * 4);
   L.w_perm = take(Tk * 4);
+  L.start = take((size_t)8192 * 4);  // [R][m] range starts of the stable sort, R * (m + 1) <= 8192
   L.x_perm = take(Tk * c.d * p.es);
   L.h = take(Tk * c.f * p.es);
   L.h_sh = take((size_t)c.n_shared * T * std::max(c.f_shared, 0) * p.es);
@@ -391,9 +393,9 @@ moe_status_t moe_histogram_lis(const moe_config_t* cfg, const int32_t* topk_idx,
   for (const void* p : std::initializer_list<const void*>{(const void*)topk_idx, (const void*)counts, (const void*)offsets, (const void*)lis})
     if (p && !aligned16(p)) return MOE_ERR_INVALID_ARG;
   const Layout L = make_layout(c, make_plan(c));
-  MOE_TRY(check_ws(c, ws, ws_bytes, L.status + 256));
+  MOE_TRY(check_ws(c, ws, ws_bytes, L.start + (size_t)8192 * 4));
   MOE_TRY(check_device());
-  return cuda_status(launch_route_index(1, c.T, c.k, c.m, topk_idx, counts, offsets, lis, nullptr,
+  return cuda_status(launch_route_index(1, c.T, c.k, c.m, topk_idx, counts, offsets, lis, at<int32_t>(ws, L.start),
                                         at<int>(ws, L.status), (cudaStream_t)stream));
 }
 
@@ -407,16 +409,18 @@ moe_status_t moe_permute(const moe_config_t* cfg, const void* x, const int32_t* 
                         (const void*)inv_perm})
     if (!aligned16(p)) return MOE_ERR_INVALID_ARG;
   const Layout L = make_layout(c, make_plan(c));
-  MOE_TRY(check_ws(c, ws, ws_bytes, L.status + 256));
+  MOE_TRY(check_ws(c, ws, ws_bytes, L.start + (size_t)8192 * 4));
   MOE_TRY(check_device());
   cudaStream_t s = (cudaStream_t)stream;
   const long long Tk = (long long)c.T * c.k;
-  // Positions not covered by a valid task keep -1, so the row copy skips them.
-  MOE_CUDA(cudaMemsetAsync(perm, 0xFF, (size_t)Tk * 4, s));
+  // Tasks that get no valid position keep inv_perm = -1, so the row copy skips them.
   MOE_CUDA(cudaMemsetAsync(inv_perm, 0xFF, (size_t)Tk * 4, s));
-  MOE_CUDA(launch_route_index(2, c.T, c.k, c.m, topk_idx, nullptr, const_cast<int32_t*>(offsets), nullptr, inv_perm,
-                              at<int>(ws, L.status), s));
-  return cuda_status(launch_permute_rows(c.dtype, (int)Tk, c.k, c.d, x, inv_perm, nullptr, perm, nullptr, x_perm, s));
+  int32_t* start = at<int32_t>(ws, L.start);
+  int* status = at<int>(ws, L.status);
+  MOE_CUDA(launch_route_index(2, c.T, c.k, c.m, topk_idx, nullptr, const_cast<int32_t*>(offsets), nullptr, start,
+                              status, s));
+  MOE_CUDA(launch_rank(c.T, c.k, c.m, topk_idx, offsets, start, nullptr, perm, inv_perm, nullptr, status, s));
+  return cuda_status(launch_permute_rows(c.dtype, (int)Tk, c.k, c.d, x, inv_perm, x_perm, s));
 }
 
 moe_status_t moe_grouped_ffn(const moe_config_t* cfg, const void* x_perm, const int32_t* offsets, const void* w_gate,
@@ -523,9 +527,11 @@ moe_status_t moe_layer_forward(const moe_config_t* cfg, const void* x, const voi
   MOE_CUDA(launch_topk_softmax(c.T, c.m, c.k, c.renormalize, logits, idx, w, s));
   MOE_TRY(mark_stage(2, s));
   float* w_perm = at<float>(ws, L.w_perm);
-  MOE_CUDA(launch_route_index(3, c.T, c.k, c.m, idx, counts, offsets, lis, inv_perm, status, s));
+  int32_t* start = at<int32_t>(ws, L.start);
+  MOE_CUDA(launch_route_index(1, c.T, c.k, c.m, idx, counts, offsets, lis, start, status, s));
+  MOE_CUDA(launch_rank(c.T, c.k, c.m, idx, offsets, start, w, perm, inv_perm, w_perm, status, s));
   MOE_TRY(mark_stage(3, s));
-  MOE_CUDA(launch_permute_rows(c.dtype, (int)Tk, c.k, c.d, x, inv_perm, w, perm, w_perm, at<void>(ws, L.x_perm), s));
+  MOE_CUDA(launch_permute_rows(c.dtype, (int)Tk, c.k, c.d, x, inv_perm, at<void>(ws, L.x_perm), s));
   MOE_TRY(mark_stage(4, s));
   FfnIo io;
   std::memset(&io, 0, sizeof(io));

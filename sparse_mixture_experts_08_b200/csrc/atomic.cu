@@ -94,6 +94,8 @@ __global__ void __launch_bounds__(SEL_THREADS, 1)
   __shared__ int warp_cnt[32];
   __shared__ int found_s;
   const int t = blockIdx.x, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  pdl_launch_dependents();
+  pdl_wait();
 
   // 1. sum the split-K partials, log-softmax of rows and of columns (fp32 values,
   //    max and log-sum-exp formed in fp64).
@@ -200,7 +202,7 @@ __global__ void __launch_bounds__(SEL_THREADS, 1)
 cudaError_t launch_atomic_select(int T, int Nr, int Nc, int K, int ksplit, const float* zr, long long zr_split,
                                  const float* zc, long long zc_split, float* lr_out, float* lc_out, int32_t* idx,
                                  float* g, int* status, cudaStream_t s) {
-  atomic_select_kernel<<<T, SEL_THREADS, 0, s>>>(T, Nr, Nc, K, ksplit, zr, zr_split, zc, zc_split, lr_out, lc_out, idx,
+  launch_k(atomic_select_kernel, T, SEL_THREADS, 0, s, T, Nr, Nc, K, ksplit, zr, zr_split, zc, zc_split, lr_out, lc_out, idx,
                                                  g, status);
   count_launch();
   return cudaGetLastError();
@@ -213,6 +215,8 @@ __global__ void atomic_coef_kernel(int T, int d, int K, int act, const uint4* __
                                    const uint4* __restrict__ w_in, const int32_t* __restrict__ idx,
                                    const float* __restrict__ g, float* __restrict__ coef, long long n_experts,
                                    int* status) {
+  pdl_launch_dependents();
+  pdl_wait();
   const int lane = threadIdx.x & 31;
   const long long task = (long long)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
   if (task >= (long long)T * K) return;
@@ -252,6 +256,8 @@ __global__ void atomic_coef_kernel(int T, int d, int K, int act, const uint4* __
 __global__ void atomic_assemble_kernel(int T, int d, int K, const uint4* __restrict__ w_out,
                                        const int32_t* __restrict__ idx, const float* __restrict__ coef,
                                        uint4* __restrict__ out, long long n_experts) {
+  pdl_launch_dependents();
+  pdl_wait();
   const int chunks = d / 8;
   const long long item = (long long)blockIdx.x * blockDim.x + threadIdx.x;
   if (item >= (long long)T * chunks) return;
@@ -282,13 +288,13 @@ cudaError_t launch_atomic_experts(int T, int d, int K, int act, const void* x, c
                                   const int32_t* idx, const float* g, float* coef, void* out, long long n_experts,
                                   int* status, cudaStream_t s) {
   const long long tasks = (long long)T * K;
-  atomic_coef_kernel<<<(unsigned)((tasks + 7) / 8), 256, 0, s>>>(T, d, K, act, (const uint4*)x, (const uint4*)w_in,
+  launch_k(atomic_coef_kernel, (unsigned)((tasks + 7) / 8), 256, 0, s, T, d, K, act, (const uint4*)x, (const uint4*)w_in,
                                                                  idx, g, coef, n_experts, status);
   count_launch();
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   const long long items = (long long)T * (d / 8);
-  atomic_assemble_kernel<<<(unsigned)((items + 63) / 64), 64, 0, s>>>(T, d, K, (const uint4*)w_out, idx, coef,
+  launch_k(atomic_assemble_kernel, (unsigned)((items + 63) / 64), 64, 0, s, T, d, K, (const uint4*)w_out, idx, coef,
                                                                       (uint4*)out, n_experts);
   count_launch();
   return cudaGetLastError();

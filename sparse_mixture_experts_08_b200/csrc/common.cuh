@@ -23,6 +23,30 @@ __device__ __forceinline__ uint64_t globaltimer_ns() {
   return t;
 }
 
+// ---------------------------------------------------------------- dependent launch
+// Every kernel of the layer is launched with programmatic stream serialization:
+// it tells the hardware at entry that its successor may be scheduled
+// (launch_dependents), and waits for its predecessor's completion (and memory)
+// right before reading that predecessor's outputs. The successor's launch and
+// prologue then overlap this kernel's tail instead of following it.
+__device__ __forceinline__ void pdl_launch_dependents() { asm volatile("griddepcontrol.launch_dependents;" :::); }
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
+template <typename... KArgs, typename... Args>
+cudaError_t launch_k(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t s, Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, static_cast<KArgs>(args)...);
+}
+
 // ---------------------------------------------------------------- internal API
 // Every launcher returns cudaSuccess or the launch error; arguments were checked
 // by the C-ABI layer before.
@@ -87,11 +111,18 @@ cudaError_t launch_simt_logits(int dtype, int T, int d, int m, const void* x, co
                                float* logits, cudaStream_t s);
 cudaError_t launch_topk_softmax(int T, int m, int k, int renorm, const float* logits, int32_t* idx, float* w,
                                 cudaStream_t s);
-// mode bit 1: histogram (counts, offsets, lis from idx); bit 2: inv_perm (stable positions from offsets)
+// Stable counting sort of the tasks by expert: route_index (one block: per-range
+// counts, offsets when mode & 1 (plus counts and LIS), range start positions
+// `start` [R][m], R * (m + 1) <= 8192) and rank (one warp per range: perm,
+// inv_perm, w_perm); permute_rows then copies the rows. route_ranges gives R, L.
+void route_ranges(int Tk, int m, int* R, int* L);
 cudaError_t launch_route_index(int mode, int T, int k, int m, const int32_t* idx, int32_t* counts, int32_t* offsets,
-                               moe_lis_t* lis, int32_t* inv_perm, int* status, cudaStream_t s);
-cudaError_t launch_permute_rows(int dtype, int Tk, int k, int d, const void* x, const int32_t* inv_perm,
-                                const float* task_w, int32_t* perm, float* w_perm, void* x_perm, cudaStream_t s);
+                               moe_lis_t* lis, int32_t* start, int* status, cudaStream_t s);
+cudaError_t launch_rank(int T, int k, int m, const int32_t* idx, const int32_t* offsets, const int32_t* start,
+                        const float* task_w, int32_t* perm, int32_t* inv_perm, float* w_perm, int* status,
+                        cudaStream_t s);
+cudaError_t launch_permute_rows(int dtype, int Tk, int k, int d, const void* x, const int32_t* inv_perm, void* x_perm,
+                                cudaStream_t s);
 cudaError_t launch_combine(int dtype, int T, int d, int k, int ksplit, const float* y_perm, long long y_split_stride,
                            const int32_t* inv_perm, int n_shared, const float* y_shared, long long ysh_split_stride,
                            void* out, cudaStream_t s);

@@ -30,6 +30,8 @@ __device__ __forceinline__ float ld_f32<__nv_bfloat16>(const __nv_bfloat16* p, l
 template <typename TIn>
 __global__ void simt_logits_kernel(int T, int d, int m, const TIn* __restrict__ x, const TIn* __restrict__ w,
                                    const float* __restrict__ bias, float* __restrict__ logits) {
+  pdl_launch_dependents();
+  pdl_wait();
   const int lane = threadIdx.x & 31;
   const long long warps = (long long)gridDim.x * (blockDim.x >> 5);
   for (long long item = (long long)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); item < (long long)T * m;
@@ -49,9 +51,9 @@ cudaError_t launch_simt_logits(int dtype, int T, int d, int m, const void* x, co
   const long long items = (long long)T * m;
   const int blocks = (int)std::min<long long>((items + 7) / 8, 4LL * num_sms() * 8);
   if (dtype == MOE_F32)
-    simt_logits_kernel<float><<<blocks, 256, 0, s>>>(T, d, m, (const float*)x, (const float*)w_r, bias, logits);
+    launch_k(simt_logits_kernel<float>, blocks, 256, 0, s, T, d, m, (const float*)x, (const float*)w_r, bias, logits);
   else
-    simt_logits_kernel<__nv_bfloat16><<<blocks, 256, 0, s>>>(T, d, m, (const __nv_bfloat16*)x,
+    launch_k(simt_logits_kernel<__nv_bfloat16>, blocks, 256, 0, s, T, d, m, (const __nv_bfloat16*)x,
                                                              (const __nv_bfloat16*)w_r, bias, logits);
   count_launch();
   return cudaGetLastError();
@@ -66,6 +68,8 @@ __global__ void topk_softmax_kernel(int T, int m, int k, int renorm, const float
                                     int32_t* __restrict__ idx, float* __restrict__ w) {
   __shared__ int s_sel[TOPK_WARPS][32];
   __shared__ float s_val[TOPK_WARPS][32];
+  pdl_launch_dependents();
+  pdl_wait();
   const int lane = threadIdx.x & 31, wib = threadIdx.x >> 5;
   const int t = blockIdx.x * TOPK_WARPS + wib;
   if (t >= T) return;
@@ -115,97 +119,87 @@ __global__ void topk_softmax_kernel(int T, int m, int k, int renorm, const float
 
 cudaError_t launch_topk_softmax(int T, int m, int k, int renorm, const float* logits, int32_t* idx, float* w,
                                 cudaStream_t s) {
-  topk_softmax_kernel<<<(T + TOPK_WARPS - 1) / TOPK_WARPS, TOPK_WARPS * 32, 0, s>>>(T, m, k, renorm, logits, idx, w);
+  launch_k(topk_softmax_kernel, (T + TOPK_WARPS - 1) / TOPK_WARPS, TOPK_WARPS * 32, 0, s, T, m, k, renorm, logits, idx, w);
   count_launch();
   return cudaGetLastError();
 }
 
-// ------------------------------------------------ histogram, offsets, LIS, ranks
-// One block of 1024 threads (the routing tables are tiny: T k ids). Warp w owns
-// the contiguous task range [w L, (w + 1) L), L = ceil(T k / 32), walked 32 tasks
-// at a time in increasing task id.
-//  pass 1: per-warp counts wc[w][e] (peer groups from __match_any_sync; each warp
-//          writes only its own row, so no atomics).
-//  scan:   per expert, exclusive prefix over warps -> wc[w][e] = tasks of e in
-//          warps before w; the total is n_e.
-// mode & 1: offsets = exclusive scan of n_e, max / lowest argmax, and
-//           LIS = m max / (T k) (R&Q Definition 1).
-// mode & 2: pass 2 re-walks each warp's range in the same order:
-//           pos = offsets[e] + wc[w][e] + (rank among the sub-chunk's peers), then
-//           wc[w][e] += peers: the stable counting-sort position, inv_perm[q] = pos
-//           (its inverse perm[pos] = q is scattered by the many-block row copy, so
-//           this one-SM kernel issues only coalesced stores).
-// Any id outside [0, m) (or, with given offsets, a position outside its segment)
-// sets MOE_ERR_DEVICE_INDEX and nothing further is written.
-constexpr int RI_MAX_REG = 16;  // sub-chunks per warp kept in registers between the passes
-
+// ------------------------------------------------ histogram, offsets, LIS, range starts
+// The T k tasks (q = t k + s, in increasing order) are cut into R contiguous
+// ranges of L tasks; range r holds tasks [r L, min(T k, (r + 1) L)). One block of
+// 1024 threads (the routing tables are tiny):
+//  pass 1: c[r][e] = tasks of expert e in range r (warp w counts ranges w, w + 32,
+//          ...; shared-memory atomics on rows no other warp touches).
+//  scan:   per expert (one warp each, a shuffle scan over its R entries),
+//          c[r][e] <- tasks of e in ranges before r; the total is n_e.
+//  mode & 1: offsets = exclusive scan of n_e, max / lowest argmax of n_e and
+//           LIS = m max / (T k) (R&Q Definition 1); otherwise offsets are given.
+//  start[r][e] = offsets[e] + c[r][e]: where range r's first task of expert e
+//  goes in the stable counting sort; rank_kernel finishes it with one warp per
+//  range.
+// Any id outside [0, m) sets MOE_ERR_DEVICE_INDEX and nothing else is written.
 __global__ void __launch_bounds__(RI_THREADS, 1)
-    route_index_kernel(int mode, int T, int k, int m, const int32_t* __restrict__ idx, int32_t* __restrict__ counts,
-                       int32_t* __restrict__ offsets, moe_lis_t* __restrict__ lis, int32_t* __restrict__ inv_perm,
-                       int* status) {
+    route_index_kernel(int mode, int T, int k, int m, int R, int L, const int32_t* __restrict__ idx,
+                       int32_t* __restrict__ counts, int32_t* __restrict__ offsets, moe_lis_t* __restrict__ lis,
+                       int32_t* __restrict__ start, int* status) {
   extern __shared__ int sm[];
-  int* wc = sm;             // [32][m]
-  int* off = wc + 32 * m;   // [m + 1]
+  const int MS = m + 1;     // padded row stride: the per-expert scan reads a column
+  int* c = sm;              // [R][MS]
+  int* off = c + R * MS;    // [m + 1]
   __shared__ int bad;
   __shared__ int wsum[32], wmax[32], warg[32];
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int nw = blockDim.x >> 5;
   const int Tk = T * k;
-  const int L = (Tk + nw - 1) / nw;
-  const int lo = min(Tk, warp * L), hi = min(Tk, lo + L);
-  const unsigned lt = (1u << lane) - 1u;
   if (tid == 0) bad = 0;
-  for (int i = tid; i < nw * m; i += blockDim.x) wc[i] = 0;
+  for (int i = tid; i < R * MS; i += blockDim.x) c[i] = 0;
+  pdl_launch_dependents();
+  pdl_wait();
   __syncthreads();
-  // All of this warp's ids (up to RI_MAX_REG sub-chunks) are loaded up front so the
-  // loads overlap; longer ranges reload the rest in the loops below.
-  int ev[RI_MAX_REG];
-#pragma unroll
-  for (int r = 0; r < RI_MAX_REG; ++r) {
-    const int q = lo + r * 32 + lane;
-    ev[r] = q < hi ? idx[q] : -1;
-  }
-  for (int base = lo, r = 0; base < hi; base += 32, ++r) {
-    const int q = base + lane;
-    int e = -1;
-    if (r < RI_MAX_REG) {
-#pragma unroll
-      for (int rr = 0; rr < RI_MAX_REG; ++rr)
-        if (rr == r) e = ev[rr];
-    } else {
-      e = q < hi ? idx[q] : -1;
+  for (int r = warp; r < R; r += nw) {
+    const int lo = r * L, hi = min(Tk, lo + L);
+    for (int q = lo + lane; q < hi; q += 32) {
+      const int e = idx[q];
+      if (e < 0 || e >= m)
+        bad = 1;
+      else
+        atomicAdd(&c[r * MS + e], 1);
     }
-    if (q < hi && (e < 0 || e >= m)) {
-      bad = 1;
-      e = -2;
-    }
-    const unsigned peers = __match_any_sync(FULL, e);
-    if (e >= 0 && lane == __ffs(peers) - 1) wc[warp * m + e] += __popc(peers);
   }
   __syncthreads();
   if (bad) {
     if (tid == 0) set_status(status, MOE_ERR_DEVICE_INDEX);
     return;
   }
-  for (int e = tid; e < m; e += blockDim.x) {
-    int run = 0;
-    for (int w = 0; w < nw; ++w) {
-      const int t = wc[w * m + e];
-      wc[w * m + e] = run;
-      run += t;
-    }
-    off[e] = run;  // n_e for now
-  }
-  __syncthreads();
-  if (mode & 1) {
-    const int c = tid < m ? off[tid] : 0;
-    int incl = c;
+  for (int e = warp; e < m; e += nw) {
+    const int per = (R + 31) / 32;
+    const int r0 = min(R, lane * per), r1 = min(R, r0 + per);
+    int local = 0;
+    for (int r = r0; r < r1; ++r) local += c[r * MS + e];
+    int incl = local;
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
       const int v = __shfl_up_sync(FULL, incl, o);
       if (lane >= o) incl += v;
     }
-    int mv = tid < m ? c : -1, ma = tid;
+    int run = incl - local;
+    for (int r = r0; r < r1; ++r) {
+      const int t = c[r * MS + e];
+      c[r * MS + e] = run;
+      run += t;
+    }
+    if (lane == 31) off[e] = incl;  // n_e for now
+  }
+  __syncthreads();
+  if (mode & 1) {
+    const int cn = tid < m ? off[tid] : 0;
+    int incl = cn;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int v = __shfl_up_sync(FULL, incl, o);
+      if (lane >= o) incl += v;
+    }
+    int mv = tid < m ? cn : -1, ma = tid;
 #pragma unroll
     for (int o = 16; o; o >>= 1) {
       const int ov = __shfl_xor_sync(FULL, mv, o), oa = __shfl_xor_sync(FULL, ma, o);
@@ -245,13 +239,13 @@ __global__ void __launch_bounds__(RI_THREADS, 1)
     }
     __syncthreads();
     if (tid < m) {
-      const int ex = incl - c + wsum[warp];
+      const int ex = incl - cn + wsum[warp];
       off[tid] = ex;
-      counts[tid] = c;
+      counts[tid] = cn;
       offsets[tid] = ex;
       if (tid == m - 1) {
-        off[m] = ex + c;
-        offsets[m] = ex + c;
+        off[m] = ex + cn;
+        offsets[m] = ex + cn;
       }
     }
     if (tid == 0 && lis) {
@@ -264,79 +258,125 @@ __global__ void __launch_bounds__(RI_THREADS, 1)
     for (int e = tid; e <= m; e += blockDim.x) off[e] = offsets[e];
   }
   __syncthreads();
-  if (!(mode & 2)) return;
-  for (int base = lo, r = 0; base < hi; base += 32, ++r) {
-    const int q = base + lane;
-    int e = -1;
-    if (r < RI_MAX_REG) {
-#pragma unroll
-      for (int rr = 0; rr < RI_MAX_REG; ++rr)
-        if (rr == r) e = ev[rr];
-    } else {
-      e = q < hi ? idx[q] : -1;
-    }
-    const unsigned peers = __match_any_sync(FULL, e);
-    const int leader = __ffs(peers) - 1;
-    const int b = e >= 0 ? wc[warp * m + e] : 0;
-    __syncwarp();
-    if (e >= 0) {
-      const int pos = off[e] + b + __popc(peers & lt);
-      if (pos >= 0 && pos >= off[e] && pos < off[e + 1] && pos < Tk) {
-        inv_perm[q] = pos;  // coalesced; the scattered perm[pos] is written by the row copy
-      } else {
-        set_status(status, MOE_ERR_DEVICE_INDEX);
-      }
-      if (lane == leader) wc[warp * m + e] = b + __popc(peers);
-    }
-    __syncwarp();
+  for (int i = tid; i < R * m; i += blockDim.x) {
+    const int r = i / m, e = i - r * m;
+    start[i] = off[e] + c[r * MS + e];
   }
 }
 
-size_t route_index_smem(int m) { return sizeof(int) * ((size_t)33 * m + 1); }
+size_t route_index_smem(int R, int m) { return sizeof(int) * ((size_t)R * (m + 1) + m + 1); }
+
+// Ranges for the stable sort: short enough that one warp ranks each range in a
+// few shuffle passes, few enough that the [R][m + 1] count table fits 32 KB.
+void route_ranges(int Tk, int m, int* R, int* L) {
+  int r = std::min(8192 / (m + 1), (Tk + 31) / 32);
+  r = std::max(1, r);
+  *L = (Tk + r - 1) / r;
+  *R = (Tk + *L - 1) / *L;
+}
 
 cudaError_t launch_route_index(int mode, int T, int k, int m, const int32_t* idx, int32_t* counts, int32_t* offsets,
-                               moe_lis_t* lis, int32_t* inv_perm, int* status, cudaStream_t s) {
-  const size_t smem = route_index_smem(m);
+                               moe_lis_t* lis, int32_t* start, int* status, cudaStream_t s) {
+  int R, L;
+  route_ranges(T * k, m, &R, &L);
+  const size_t smem = route_index_smem(R, m);
   static size_t attr = 0;
   if (smem > 48 * 1024 && smem > attr) {
     cudaError_t e = cudaFuncSetAttribute(route_index_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     attr = smem;
   }
-  route_index_kernel<<<1, RI_THREADS, smem, s>>>(mode, T, k, m, idx, counts, offsets, lis, inv_perm, status);
+  launch_k(route_index_kernel, 1, RI_THREADS, smem, s, mode, T, k, m, R, L, idx, counts, offsets, lis, start,
+           status);
+  count_launch();
+  return cudaGetLastError();
+}
+
+// ------------------------------------------------ ranks
+// One warp per task range r walks it 32 tasks at a time in increasing task id: a
+// task's rank among the lower lanes with the same expert (a 32-step shuffle scan)
+// plus the expert's cursor (started at start[r][e]) is its position pos in the
+// stable counting sort; the group's last lane advances the cursor. Writes
+// inv_perm[q] = pos, perm[pos] = q and, when given, w_perm[pos] = task_w[q] (the
+// gate weight in segment order). A position outside its expert's segment
+// [offsets[e], offsets[e + 1]) sets MOE_ERR_DEVICE_INDEX and that task is not
+// written; after an earlier device error the kernel does nothing.
+__global__ void rank_kernel(int Tk, int m, int L, const int32_t* __restrict__ idx, const int32_t* __restrict__ offsets,
+                            const int32_t* __restrict__ start, const float* __restrict__ task_w,
+                            int32_t* __restrict__ perm, int32_t* __restrict__ inv_perm, float* __restrict__ w_perm,
+                            int* status) {
+  extern __shared__ int cur[];  // [m]
+  const int lane = threadIdx.x;
+  const int r = blockIdx.x;
+  const int lo = r * L, hi = min(Tk, lo + L);
+  pdl_launch_dependents();
+  pdl_wait();
+  if (status && *reinterpret_cast<volatile int*>(status) != 0) return;  // earlier device error
+  for (int e = lane; e < m; e += 32) cur[e] = start[(long long)r * m + e];
+  __syncwarp();
+  for (int base = lo; base < hi; base += 32) {
+    const int q = base + lane;
+    int e = q < hi ? idx[q] : -1;
+    if (e >= m) e = -1;
+    int rank = 0, cnt = 0;
+#pragma unroll
+    for (int j = 0; j < 32; ++j) {
+      const int ej = __shfl_sync(FULL, e, j);
+      cnt += ej == e;
+      rank += (ej == e) & (j < lane);
+    }
+    const int b = e >= 0 ? cur[e] : 0;
+    __syncwarp();
+    if (q < hi) {
+      const int pos = b + rank;
+      const bool ok = e >= 0 && pos >= 0 && pos < Tk && pos >= offsets[e] && pos < offsets[e + 1];
+      inv_perm[q] = ok ? pos : -1;
+      if (ok) {
+        perm[pos] = q;
+        if (w_perm) w_perm[pos] = task_w[q];
+      } else {
+        set_status(status, MOE_ERR_DEVICE_INDEX);
+      }
+    }
+    if (e >= 0 && rank == cnt - 1) cur[e] = b + cnt;
+    __syncwarp();
+  }
+}
+
+cudaError_t launch_rank(int T, int k, int m, const int32_t* idx, const int32_t* offsets, const int32_t* start,
+                        const float* task_w, int32_t* perm, int32_t* inv_perm, float* w_perm, int* status,
+                        cudaStream_t s) {
+  int R, L;
+  route_ranges(T * k, m, &R, &L);
+  launch_k(rank_kernel, R, 32, sizeof(int) * (size_t)m, s, T * k, m, L, idx, offsets, start, task_w, perm, inv_perm,
+           w_perm, status);
   count_launch();
   return cudaGetLastError();
 }
 
 // ------------------------------------------------------------------ permute rows
-// Walks the tasks q in order (one warp each): pos = inv_perm[q];
-// x_perm[pos, :] = x[q / k, :] with 16-byte vectors; perm[pos] = q; and, when
-// given, w_perm[pos] = task_w[q] (the gate weight in segment order, read by the
-// down-projection epilogue).
+// One thread per 16-byte chunk of x_perm, tasks q in order:
+// x_perm[inv_perm[q], c] = x[q / k, c] (tasks without a valid position are skipped).
 __global__ void permute_rows_kernel(int Tk, int k, int chunks, const int4* __restrict__ x,
-                                    const int32_t* __restrict__ inv_perm, const float* __restrict__ task_w,
-                                    int32_t* __restrict__ perm, float* __restrict__ w_perm, int4* __restrict__ x_perm) {
-  const int lane = threadIdx.x & 31;
-  const long long warps = (long long)gridDim.x * (blockDim.x >> 5);
-  for (long long q = (long long)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); q < Tk; q += warps) {
+                                    const int32_t* __restrict__ inv_perm, int4* __restrict__ x_perm) {
+  pdl_launch_dependents();
+  pdl_wait();
+  const long long n = (long long)Tk * chunks;
+  for (long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += (long long)gridDim.x * blockDim.x) {
+    const long long q = i / chunks;
+    const int c = (int)(i - q * chunks);
     const int pos = inv_perm[q];
     if (pos < 0 || pos >= Tk) continue;
-    if (lane == 0) {
-      perm[pos] = (int32_t)q;
-      if (w_perm) w_perm[pos] = task_w[q];
-    }
-    const int4* src = x + (q / k) * chunks;
-    int4* dst = x_perm + (long long)pos * chunks;
-    for (int c = lane; c < chunks; c += 32) dst[c] = src[c];
+    x_perm[(long long)pos * chunks + c] = x[(q / k) * chunks + c];
   }
 }
 
-cudaError_t launch_permute_rows(int dtype, int Tk, int k, int d, const void* x, const int32_t* inv_perm,
-                                const float* task_w, int32_t* perm, float* w_perm, void* x_perm, cudaStream_t s) {
+cudaError_t launch_permute_rows(int dtype, int Tk, int k, int d, const void* x, const int32_t* inv_perm, void* x_perm,
+                                cudaStream_t s) {
   const int chunks = d * (dtype == MOE_F32 ? 4 : 2) / 16;
-  const int blocks = std::max(1, std::min((Tk + 7) / 8, num_sms() * 8));
-  permute_rows_kernel<<<blocks, 256, 0, s>>>(Tk, k, chunks, (const int4*)x, inv_perm, task_w, perm, w_perm,
-                                             (int4*)x_perm);
+  const long long n = (long long)Tk * chunks;
+  const int blocks = (int)std::max<long long>(1, std::min<long long>((n + 255) / 256, (long long)num_sms() * 16));
+  launch_k(permute_rows_kernel, blocks, 256, 0, s, Tk, k, chunks, (const int4*)x, inv_perm, (int4*)x_perm);
   count_launch();
   return cudaGetLastError();
 }
@@ -364,6 +404,8 @@ template <typename OutT>
 __global__ void combine_kernel(int T, int d4, int k, int ksplit, const float4* __restrict__ y, long long ysplit4,
                                const int32_t* __restrict__ inv_perm, int n_sh, const float4* __restrict__ ysh,
                                long long yshsplit4, OutT* __restrict__ out) {
+  pdl_launch_dependents();
+  pdl_wait();
   const long long n = (long long)T * d4;
   const int Tk = T * k;
   for (long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += (long long)gridDim.x * blockDim.x) {
@@ -394,11 +436,11 @@ cudaError_t launch_combine(int dtype, int T, int d, int k, int ksplit, const flo
   const long long n = (long long)T * d4;
   const int blocks = (int)std::max<long long>(1, std::min<long long>((n + 255) / 256, (long long)num_sms() * 16));
   if (dtype == MOE_F32)
-    combine_kernel<float><<<blocks, 256, 0, s>>>(T, d4, k, ksplit, (const float4*)y_perm, y_split_stride / 4, inv_perm,
+    launch_k(combine_kernel<float>, blocks, 256, 0, s, T, d4, k, ksplit, (const float4*)y_perm, y_split_stride / 4, inv_perm,
                                                  y_shared ? n_shared : 0, (const float4*)y_shared,
                                                  ysh_split_stride / 4, (float*)out);
   else
-    combine_kernel<__nv_bfloat16><<<blocks, 256, 0, s>>>(T, d4, k, ksplit, (const float4*)y_perm, y_split_stride / 4,
+    launch_k(combine_kernel<__nv_bfloat16>, blocks, 256, 0, s, T, d4, k, ksplit, (const float4*)y_perm, y_split_stride / 4,
                                                          inv_perm, y_shared ? n_shared : 0, (const float4*)y_shared,
                                                          ysh_split_stride / 4, (__nv_bfloat16*)out);
   count_launch();
@@ -407,6 +449,8 @@ cudaError_t launch_combine(int dtype, int T, int d, int k, int ksplit, const flo
 
 __global__ void reduce_splits_kernel(long long n4, int ksplit, const float4* __restrict__ in, long long split4,
                                      float4* __restrict__ out) {
+  pdl_launch_dependents();
+  pdl_wait();
   for (long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x; i < n4; i += (long long)gridDim.x * blockDim.x) {
     float4 a = in[i];
     for (int sp = 1; sp < ksplit; ++sp) {
@@ -421,7 +465,7 @@ cudaError_t launch_reduce_splits(long long n, int ksplit, const float* in, long 
                                  cudaStream_t s) {
   const long long n4 = n / 4;
   const int blocks = (int)std::max<long long>(1, std::min<long long>((n4 + 255) / 256, (long long)num_sms() * 16));
-  reduce_splits_kernel<<<blocks, 256, 0, s>>>(n4, ksplit, (const float4*)in, split_stride / 4, (float4*)out);
+  launch_k(reduce_splits_kernel, blocks, 256, 0, s, n4, ksplit, (const float4*)in, split_stride / 4, (float4*)out);
   count_launch();
   return cudaGetLastError();
 }

@@ -34,6 +34,8 @@ template <typename TIn, int EPI>
 __global__ void simt_gemm_kernel(const __grid_constant__ GemmParams p, long long max_rows) {
   const GemmClass& c = p.cls[blockIdx.y];
   const int lane = threadIdx.x & 31;
+  pdl_launch_dependents();
+  pdl_wait();
   if (p.status && *reinterpret_cast<volatile int*>(p.status) != 0) return;  // earlier device error
   const int fblocks = (c.R + 31) / 32;
   const long long nrows = c.seg_off ? max_rows : (long long)c.n_groups * c.const_rows;
@@ -105,9 +107,9 @@ cudaError_t launch_simt_gemm(int epi, int dtype, const GemmParams& p, int max_ro
 #define MOE_SIMT_CASE(EPI_)                                                                          \
   if (epi == EPI_) {                                                                                 \
     if (dtype == MOE_F32)                                                                            \
-      simt_gemm_kernel<float, EPI_><<<grid, 256, 0, s>>>(p, max_rows_per_class);                     \
+      launch_k(simt_gemm_kernel<float, EPI_>, grid, 256, 0, s, p, max_rows_per_class);                     \
     else                                                                                             \
-      simt_gemm_kernel<__nv_bfloat16, EPI_><<<grid, 256, 0, s>>>(p, max_rows_per_class);             \
+      launch_k(simt_gemm_kernel<__nv_bfloat16, EPI_>, grid, 256, 0, s, p, max_rows_per_class);             \
     count_launch();                                                                                  \
     return cudaGetLastError();                                                                       \
   }

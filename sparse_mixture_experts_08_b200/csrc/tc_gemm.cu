@@ -288,6 +288,10 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
     tmem_alloc(&tmem_base_s, S::TMEM_COLS);
     tmem_relinquish();
   }
+  // Everything above overlaps the previous kernel; the segment offsets, the token
+  // rows (TMA) and the row data read below are its outputs.
+  pdl_launch_dependents();
+  pdl_wait();
   // Tile schedule from the device-resident segment sizes.
   if (warp == 0) {
     const int per = (G + 31) / 32;
@@ -551,7 +555,7 @@ static cudaError_t launch_impl(const TcMaps& maps, const GemmParams& p, int num_
     if (e != cudaSuccess) return e;
     attr_set = true;
   }
-  kern<<<num_ctas, TC_THREADS, S::DYN_SMEM, s>>>(m[0], m[1], m[2], m[3], m[4], m[5], p);
+  launch_k(kern, num_ctas, TC_THREADS, S::DYN_SMEM, s, m[0], m[1], m[2], m[3], m[4], m[5], p);
   count_launch();
   return cudaGetLastError();
 }

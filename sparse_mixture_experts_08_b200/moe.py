@@ -220,9 +220,10 @@ def moe_debug_set_wait_limit_ns(ns: int):
 
 def moe_set_stage_events(events):
     """events: list of torch.cuda.Event (enable_timing=True, already recorded once so
-    that the CUDA event exists) or [] to switch the hook off."""
-    handles = [e.cuda_event for e in events]
-    if any(not h for h in handles):
+    that the CUDA event exists) or None entries (boundary not recorded); [] switches
+    the hook off."""
+    handles = [0 if e is None else e.cuda_event for e in events]
+    if any(e is not None and not h for e, h in zip(events, handles)):
         raise ValueError("moe_set_stage_events: record each torch.cuda.Event once before passing it")
     arr = (ctypes.c_void_p * max(1, len(handles)))(*handles)
     _check("moe_set_stage_events", lib().moe_set_stage_events(arr if handles else None, len(handles)))
