@@ -150,6 +150,27 @@ def reference_arm(args):
     return 0
 
 
+# ------------------------------------------------------------------ data-parallel ranks
+
+def rank_inputs(cfg, rank: int):
+    """Inputs of one data-parallel rank: the expert and router weights are the same
+    on every rank (replicate 0); the token batch is the rank's own (replicate = rank)."""
+    inp = W.make_moe_inputs(cfg, replicate=0)
+    if rank:
+        inp["x"] = W.normal(cfg.seed(rank), W.STREAM["x"], (cfg.T, cfg.d), 1.0, cfg.dtype)
+    return inp
+
+
+def max_over_ranks(values, dist=None, device=None):
+    """Element-wise maximum of a list of floats over all ranks (identity on one rank)."""
+    import torch
+
+    t = torch.tensor(values, dtype=torch.float64, device=device)
+    if dist is not None and dist.is_initialized() and dist.get_world_size() > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return [float(v) for v in t.cpu()]
+
+
 # ------------------------------------------------------------------ clocks (NVML, sampled during timing)
 
 REASONS = {0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap", 0x8: "hw_slowdown",
@@ -233,10 +254,11 @@ def stage_costs(cfg, active: int, ksplit: int):
     c["expert_up"] = (2.0 * mats * f * d * Tk + 2.0 * mats * fsh * d * T * nsh,
                       active * mats * f * d * es + nsh * mats * fsh * d * es + Tk * d * es + (T * d * es if nsh else 0)
                       + Tk * f * es + nsh * T * fsh * es)
+    fused_k1 = k == 1 and nsh == 0 and ksplit == 1 and cfg.dtype == W.BF16  # down epilogue writes `out` itself
+    out_bytes = T * d * es if fused_k1 else ksplit * Tk * d * 4 + nsh * T * d * 4
     c["expert_down"] = (2.0 * d * f * Tk + 2.0 * d * fsh * T * nsh,
-                        active * d * f * es + nsh * d * fsh * es + Tk * f * es + nsh * T * fsh * es
-                        + ksplit * Tk * d * 4 + nsh * T * d * 4)
-    c["combine"] = (0.0, ksplit * Tk * d * 4 + nsh * T * d * 4 + Tk * 4 + T * d * es)
+                        active * d * f * es + nsh * d * fsh * es + Tk * f * es + nsh * T * fsh * es + out_bytes)
+    c["combine"] = (0.0, 0.0 if fused_k1 else ksplit * Tk * d * 4 + nsh * T * d * 4 + Tk * 4 + T * d * es)
     layer_flops = 2.0 * T * d * m + c["expert_up"][0] + c["expert_down"][0]
     layer_bytes = (m * d + active * (mats + 1) * f * d + nsh * (mats + 1) * fsh * d) * es + 2 * T * d * es
     return c, layer_flops, layer_bytes
@@ -282,9 +304,7 @@ def ours(args):
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=180), device_id=dev)
 
     cfg = W.CONFIGS[args.config]
-    inp = W.make_moe_inputs(cfg, replicate=0)  # expert weights: identical on every rank
-    if rank:
-        inp["x"] = W.normal(cfg.seed(rank), W.STREAM["x"], (cfg.T, cfg.d), 1.0, cfg.dtype)
+    inp = rank_inputs(cfg, rank)
 
     def to_dev(a):
         if a.dtype == np.uint16:
@@ -408,10 +428,7 @@ def ours(args):
     d2h = out_host.numel() * out_host.element_size()
 
     # ---- max over ranks
-    t = torch.tensor([ms_local, e2e_local], dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    ms, e2e_ms = float(t[0]), float(t[1])
+    ms, e2e_ms = max_over_ranks([ms_local, e2e_local], dist, dev)
 
     pk, pk_src = peaks()
     plan_ksplit = 1
@@ -433,7 +450,7 @@ def ours(args):
     long_step = K * ms > 1000.0
     tensor_peak = pk["bf16_tflops_sustained"] if long_step else pk["bf16_tflops"]
     ridge = tensor_peak * 1e12 / (pk["hbm_gbs"] * 1e9)
-    if fl > 0 and fl / by > ridge and cfg.dtype == W.BF16:
+    if fl > 0 and fl / max(by, 1.0) > ridge and cfg.dtype == W.BF16:
         roof = {"bound": "tensor", "achieved": fl / sec / 1e12, "peak": tensor_peak, "unit": "TFLOP/s"}
         roof["peak_source"] = f"{pk_src} bf16 ({'sustained' if long_step else 'burst'})"
     else:
