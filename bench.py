@@ -51,8 +51,7 @@ def parse():
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=10)
-    ap.add_argument("--config", default="switch", choices=[k for k, v in W.CONFIGS.items()
-                                                           if isinstance(v, W.MoEWorkload)])
+    ap.add_argument("--config", default="switch", choices=list(W.CONFIGS))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--cpu-seconds", type=float, default=12.0, help="CPU-oracle baseline budget (rank 0, N=1)")
     ap.add_argument("--no-cpu-baseline", action="store_true", help="skip the CPU-oracle leg (for profiling runs)")
@@ -148,6 +147,43 @@ def reference_arm(args):
             "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
     return 0
+
+
+# ------------------------------------------------------------------ end-to-end leg
+
+def e2e_pipelined(torch, fwd, x_host, x_devs, out_devs, out_hosts, K, s_comp, dev):
+    """K steps through the C-ABI call with the token batch copied in from pinned host
+    memory and the output copied back every step. Copies run on their own streams and
+    device buffers alternate, so batch i+1's upload and batch i-1's download overlap
+    batch i's forward (a serving loop's arrangement). Returns ms per step."""
+    s_in = torch.cuda.Stream(device=dev)
+    s_out = torch.cuda.Stream(device=dev)
+    ev_in = [torch.cuda.Event() for _ in range(2)]   # upload of the buffer done
+    ev_c = [torch.cuda.Event() for _ in range(2)]    # forward done: input free, output ready
+    ev_o = [torch.cuda.Event() for _ in range(2)]    # download done: output buffer free
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize(dev)
+    start.record(s_in)
+    for i in range(K):
+        b = i % 2
+        with torch.cuda.stream(s_in):
+            if i >= 2:
+                s_in.wait_event(ev_c[b])
+            x_devs[b].copy_(x_host, non_blocking=True)
+            ev_in[b].record(s_in)
+        with torch.cuda.stream(s_comp):
+            s_comp.wait_event(ev_in[b])
+            if i >= 2:
+                s_comp.wait_event(ev_o[b])
+            fwd(x_devs[b], out_devs[b])
+            ev_c[b].record(s_comp)
+        with torch.cuda.stream(s_out):
+            s_out.wait_event(ev_c[b])
+            out_hosts[b].copy_(out_devs[b], non_blocking=True)
+            ev_o[b].record(s_out)
+    end.record(s_out)
+    torch.cuda.synchronize(dev)
+    return start.elapsed_time(end) / K
 
 
 # ------------------------------------------------------------------ data-parallel ranks
@@ -401,31 +437,22 @@ def ours(args):
         raise RuntimeError(f"device status after the timed steps: {moe.moe_status_string(st)}")
 
     # ---- end to end through the C ABI: pinned host batch in, result out, every step
+    raw = (lambda t: t.view(torch.int16)) if tdt == torch.bfloat16 else (lambda t: t)
     x_host = torch.from_numpy(inp["x"].view(np.int16) if inp["x"].dtype == np.uint16 else inp["x"]).pin_memory()
-    out_host = torch.empty(out.shape, dtype=torch.int16 if tdt == torch.bfloat16 else torch.float32).pin_memory()
-    x_dev = torch.empty_like(d_in["x"])
-    xd_raw = x_dev.view(torch.int16) if tdt == torch.bfloat16 else x_dev
-    out_raw = out.view(torch.int16) if tdt == torch.bfloat16 else out
+    out_hosts = [torch.empty(out.shape, dtype=torch.int16 if tdt == torch.bfloat16 else torch.float32).pin_memory()
+                 for _ in range(2)]
+    x_devs = [raw(torch.empty_like(d_in["x"])) for _ in range(2)]
+    out_devs = [torch.empty_like(out) for _ in range(2)]
     Ke = max(3, min(K, 100))
-    e_s = [torch.cuda.Event(enable_timing=True) for _ in range(Ke)]
-    e_e = [torch.cuda.Event(enable_timing=True) for _ in range(Ke)]
     if world > 1:
         dist.barrier()
-    torch.cuda.synchronize(dev)
-    with torch.cuda.stream(s):
-        for i in range(Ke):
-            flush.zero_()
-            e_s[i].record(s)
-            xd_raw.copy_(x_host, non_blocking=True)
-            fwd(x=x_dev)
-            out_host.copy_(out_raw, non_blocking=True)
-            e_e[i].record(s)
-    torch.cuda.synchronize(dev)
+    # the C ABI takes raw device pointers, so bf16 buffers travel as int16 views
+    e2e_local = e2e_pipelined(torch, lambda xd, od: fwd(x=xd, o=od), x_host, x_devs, [raw(o) for o in out_devs],
+                              out_hosts, Ke, s, dev)
     if world > 1:
         dist.barrier()
-    e2e_local = sum(e_s[i].elapsed_time(e_e[i]) for i in range(Ke)) / Ke
     h2d = x_host.numel() * x_host.element_size()
-    d2h = out_host.numel() * out_host.element_size()
+    d2h = out_hosts[0].numel() * out_hosts[0].element_size()
 
     # ---- max over ranks
     ms, e2e_ms = max_over_ranks([ms_local, e2e_local], dist, dev)
@@ -481,7 +508,9 @@ def ours(args):
             "routing": {"lis": lis_v, "max_count": max_count, "heavy_hitter": argmax, "active_experts": active,
                         "reuse_ratio": cfg.T * cfg.k / max(active, 1), "load_entropy": entropy},
             "e2e": {"value": world * cfg.T / (e2e_ms * 1e-3), "unit": UNIT, "h2d_bytes_per_step": h2d,
-                    "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
+                    "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms,
+                    "note": "pinned host -> device batch upload and device -> host output download every step, on "
+                            "their own streams, overlapped with the neighbouring steps' forward (double-buffered)"},
             "gpu_launches": K * launches_per_step, "launches_per_step": launches_per_step,
             "clocks": sampler.report()}
     if world > 1:
@@ -497,11 +526,177 @@ def ours(args):
     return 0
 
 
+# ------------------------------------------------------------------ atomic-expert workload
+
+ATOMIC_STAGES = ["router_projections", "grid_topk", "expert_coefficients", "assembly"]
+
+
+def atomic_config(cfg) -> dict:
+    return {"workload": cfg.name, "tokens": cfg.T, "d_model": cfg.d, "grid": f"{cfg.Nr}x{cfg.Nc}", "experts": cfg.N,
+            "top_k": cfg.K, "activation": "silu" if cfg.act == W.ACT_SILU else "sigmoid", "description": cfg.note}
+
+
+def atomic_stage_costs(cfg, active: int, ksplit: int):
+    T, d, n = cfg.T, cfg.d, cfg.Nr + cfg.Nc
+    c = {"router_projections": (2.0 * T * d * n, n * d * 2 + T * d * 2 + ksplit * T * n * 4),
+         "grid_topk": (0.0, ksplit * T * n * 4 + T * cfg.K * 8),
+         "expert_coefficients": (2.0 * T * cfg.K * d, active * d * 2 + T * d * 2 + T * cfg.K * 8),
+         "assembly": (2.0 * T * cfg.K * d, active * d * 2 + T * d * 2 + T * cfg.K * 8)}
+    layer_flops = 2.0 * T * d * n + 4.0 * T * cfg.K * d
+    layer_bytes = n * d * 2 + 2 * active * d * 2 + 2 * T * d * 2
+    return c, layer_flops, layer_bytes
+
+
+def cpu_oracle_atomic(cfg, inp, budget_s: float):
+    import oracle as O
+
+    def run(n):
+        t0 = time.perf_counter()
+        x = np.ascontiguousarray(inp["x"][:n])
+        lr, lc = O.atomic_logprobs(x, inp["w_row"], inp["w_col"])
+        idx, g = O.atomic_select(lr, lc, cfg.K)
+        O.atomic_output(x, inp["w_in"], inp["w_out"], idx, g, cfg.act)
+        return time.perf_counter() - t0
+
+    n = 1
+    dt = run(n)
+    while dt < budget_s / 4 and n < cfg.T:
+        n = min(cfg.T, n * 2)
+        dt = run(n)
+    return {"value": n / dt, "unit": UNIT, "cores": 1, "kind": "oracle", "seconds": round(dt, 3),
+            "sample": f"first {n} of {cfg.T} tokens of the {cfg.name} workload; Cartesian router, exact grid top-K "
+                      f"(brute-force sort of all {cfg.N} scores per token) and atomic experts, fp64 C, one thread"}
+
+
+def ours_atomic(args):
+    import torch
+
+    import sparse_mixture_experts_08_b200 as moe
+
+    if int(os.environ.get("WORLD_SIZE", "1")) != 1 or args.gpus != 1:
+        raise SystemExit("the atomic-expert workload is benchmarked on one GPU")
+    cfg = W.CONFIGS[args.config]
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    inp = W.make_atomic_inputs(cfg)
+    d_in = {k: torch.from_numpy(v.view(np.int16)).to(dev).view(torch.bfloat16) for k, v in inp.items()}
+    c = moe.make_atomic_config(cfg.T, cfg.d, cfg.Nr, cfg.Nc, cfg.K, cfg.act)
+    ws = moe.workspace(c, device=dev)
+    out = torch.empty((cfg.T, cfg.d), dtype=torch.bfloat16, device=dev)
+    idx = torch.empty((cfg.T, cfg.K), dtype=torch.int32, device=dev)
+    s = torch.cuda.Stream(device=dev)
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+
+    def fwd(x=None):
+        moe.moe_atomic_forward(c, d_in["x"] if x is None else x, d_in["w_row"], d_in["w_col"], d_in["w_in"],
+                               d_in["w_out"], out, ws, idx_out=idx, stream=s)
+
+    with torch.cuda.stream(s):
+        n0 = moe.moe_launch_count()
+        fwd()
+        launches_per_step = moe.moe_launch_count() - n0
+        for _ in range(max(args.warmup, 3)):
+            flush.zero_()
+            fwd()
+    torch.cuda.synchronize(dev)
+    if moe.moe_read_device_status(ws, stream=s) != moe.OK:
+        raise RuntimeError("device status after warm-up is not OK")
+    active = int(np.unique(idx.cpu().numpy()).size)
+    Kp = max(3, min(args.steps, 50))
+    ev_prof = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(Kp)]
+    with torch.cuda.stream(s):
+        for evs in ev_prof:
+            for e in evs:
+                e.record(s)
+        for i in range(Kp):
+            flush.zero_()
+            moe.moe_set_stage_events(ev_prof[i])
+            fwd()
+    torch.cuda.synchronize(dev)
+    moe.moe_set_stage_events([])
+    stage_ms = {name: sum(ev_prof[i][j].elapsed_time(ev_prof[i][j + 1]) for i in range(Kp)) / Kp
+                for j, name in enumerate(ATOMIC_STAGES)}
+    dom = max(ATOMIC_STAGES, key=lambda n: stage_ms[n])
+    jd = ATOMIC_STAGES.index(dom)
+    K = args.steps
+    ev_s = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
+    ev_e = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
+    ev_dom = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(K)]
+    with torch.cuda.stream(s):
+        for evs in ev_dom:
+            for e in evs:
+                e.record(s)
+    sampler = ClockSampler(0)
+    torch.cuda.synchronize(dev)
+    sampler.start()
+    with torch.cuda.stream(s):
+        for i in range(K):
+            flush.zero_()
+            hook = [None] * 5
+            hook[jd], hook[jd + 1] = ev_dom[i][0], ev_dom[i][1]
+            moe.moe_set_stage_events(hook)
+            ev_s[i].record(s)
+            fwd()
+            ev_e[i].record(s)
+    torch.cuda.synchronize(dev)
+    sampler.stop()
+    moe.moe_set_stage_events([])
+    ms = sum(ev_s[i].elapsed_time(ev_e[i]) for i in range(K)) / K
+    dom_ms = sum(ev_dom[i][0].elapsed_time(ev_dom[i][1]) for i in range(K)) / K
+    # end to end: token batch from pinned host memory, output back, every step (pipelined)
+    x_host = torch.from_numpy(inp["x"].view(np.int16)).pin_memory()
+    out_hosts = [torch.empty(out.shape, dtype=torch.int16).pin_memory() for _ in range(2)]
+    x_devs = [torch.empty_like(d_in["x"]).view(torch.int16) for _ in range(2)]
+    out_devs = [torch.empty_like(out) for _ in range(2)]
+
+    def fwd2(xd, od):
+        moe.moe_atomic_forward(c, xd.view(torch.bfloat16), d_in["w_row"], d_in["w_col"], d_in["w_in"], d_in["w_out"],
+                               od, ws, stream=s)
+
+    Ke = max(3, min(K, 100))
+    e2e_ms = e2e_pipelined(torch, lambda xd, od: fwd2(xd, od), x_host, x_devs, [o.view(torch.int16) for o in out_devs],
+                           out_hosts, Ke, s, dev)
+    pk, pk_src = peaks()
+    ksplit = 16
+    costs, layer_flops, layer_bytes = atomic_stage_costs(cfg, active, ksplit)
+    fl, by = costs[dom]
+    roof = {"bound": "hbm", "achieved": by / (dom_ms * 1e-3) / 1e9, "peak": pk["hbm_gbs"], "unit": "GB/s",
+            "peak_source": f"{pk_src} hbm copy"}
+    roof["frac"] = roof["achieved"] / roof["peak"]
+    roof.update(traffic=traffic_for(cfg.name, dom), kernel=dom, algorithmic_bytes=by, algorithmic_flops=fl,
+                duration_us=dom_ms * 1e3)
+    t_layer = max(layer_flops / (pk["bf16_tflops"] * 1e12), layer_bytes / (pk["hbm_gbs"] * 1e9))
+    line = {"metric": METRIC, "value": cfg.T / (ms * 1e-3), "unit": UNIT, "n_gpus": 1, "steps": K,
+            "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic (seeded generator; x ~ N(0,1), router and w_in ~ N(0, 1/sqrt(d)), w_out ~ N(0,1))",
+            "config": dict(atomic_config(cfg), parallelism="single GPU",
+                           l2=f"flushed between steps ({L2_FLUSH_BYTES >> 20} MiB write, outside the timed events)",
+                           launch="eager C-ABI call per step"),
+            "roofline": roof,
+            "layer_roofline": {"time_us": t_layer * 1e6, "frac": t_layer / (ms * 1e-3), "flops": layer_flops,
+                               "bytes": layer_bytes},
+            "stages_us": {k: v * 1e3 for k, v in stage_ms.items()},
+            "routing": {"active_experts": active, "reuse_ratio": cfg.T * cfg.K / max(active, 1)},
+            "e2e": {"value": cfg.T / (e2e_ms * 1e-3), "unit": UNIT, "h2d_bytes_per_step": x_host.numel() * 2,
+                    "d2h_bytes_per_step": out_hosts[0].numel() * 2, "ms_per_step": e2e_ms,
+                    "note": "pinned host -> device batch upload and device -> host output download every step, on "
+                            "their own streams, overlapped with the neighbouring steps' forward (double-buffered)"},
+            "gpu_launches": K * launches_per_step, "launches_per_step": launches_per_step,
+            "clocks": sampler.report()}
+    line["cpu_baseline"] = None if args.no_cpu_baseline else cpu_oracle_atomic(cfg, inp, args.cpu_seconds)
+    print(json.dumps(line), flush=True)
+    return 0
+
+
 def main():
     args = parse()
+    atomic = isinstance(W.CONFIGS[args.config], W.AtomicWorkload)
     if args.impl == "reference":
+        if atomic:
+            raise SystemExit("--impl reference covers the coarse-expert workloads")
         return reference_arm(args)
-    return ours(args)
+    return ours_atomic(args) if atomic else ours(args)
 
 
 if __name__ == "__main__":

@@ -229,7 +229,9 @@ MOE_API moe_status_t moe_debug_set_wait_limit_ns(uint64_t ns);
  * cudaEvent_t handles in `events` (host array, caller-owned events) on its
  * stream at its stage boundaries, in order: 0 start, 1 router logits, 2 top-k,
  * 3 histogram/LIS/ranks, 4 row permutation, 5 up projection, 6 down projection,
- * 7 combine (n <= 8; extra stages are not recorded). A NULL entry skips that
+ * 7 combine (n <= 8; extra stages are not recorded); moe_atomic_forward records
+ * 0 start, 1 router projections, 2 grid top-K, 3 expert coefficients, 4 assembly.
+ * A NULL entry skips that
  * boundary (a recorded event between two kernels stops the second one from
  * starting early, so record only the boundaries you time). n = 0 turns it off.
  * The array is copied. Process-wide and not thread-safe; meant for benchmarks. */

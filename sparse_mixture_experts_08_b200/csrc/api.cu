@@ -30,10 +30,13 @@ static unsigned long long g_wait_limit_ns = 2000ull * 1000 * 1000;
 static cudaEvent_t g_stage_events[8];
 static int g_n_stage_events = 0;
 
+cudaError_t mark_stage_event(int i, cudaStream_t s) {
+  if (i < g_n_stage_events && g_stage_events[i]) return cudaEventRecord(g_stage_events[i], s);
+  return cudaSuccess;
+}
+
 static moe_status_t mark_stage(int i, cudaStream_t s) {
-  if (i < g_n_stage_events && g_stage_events[i])
-    return cudaEventRecord(g_stage_events[i], s) == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
-  return MOE_OK;
+  return mark_stage_event(i, s) == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }
 constexpr int PLAN_SMS = 148;
   // B200 SM count used for static planning (split-K, tile sizes)
@@ -163,7 +166,9 @@ static moe_status_t cuda_status(cudaError_t e) { return e == cudaSuccess ? MOE_O
 
 static moe_status_t run_router(const moe_config_t& c, const void* x, const void* w_r, const float* bias, float* logits,
                                int* status, cudaStream_t s) {
-  // fp32 layers, and batches too small to fill the tensor cores (decode), use CUDA cores.
+  // Batches too small to fill the tensor cores (decode) and fp32 layers use CUDA cores.
+  if (few_expert_logits_ok(c.dtype, c.T, c.m))
+    return cuda_status(launch_few_expert_logits(c.T, c.d, c.m, x, w_r, bias, logits, s));
   if (c.dtype == MOE_F32 || c.T <= 64)
     return cuda_status(launch_simt_logits(c.dtype, c.T, c.d, c.m, x, w_r, bias, logits, s));
   // logits^T = W_r . x^T on the tensor cores: one group, features = experts.
@@ -617,7 +622,7 @@ moe_status_t moe_atomic_workspace_size(const moe_atomic_config_t* cfg, size_t* b
 
 static moe_status_t atomic_route_impl(const moe_atomic_config_t& c, const AtomicPlan& P, const void* x,
                                       const void* w_row, const void* w_col, float* lr_out, float* lc_out,
-                                      int32_t* idx, float* g, void* ws, cudaStream_t s) {
+                                      int32_t* idx, float* g, void* ws, cudaStream_t s, bool stage_marks = false) {
   int* status = at<int>(ws, P.status);
   float* zr = at<float>(ws, P.zr);
   float* zc = at<float>(ws, P.zc);
@@ -645,8 +650,11 @@ static moe_status_t atomic_route_impl(const moe_atomic_config_t& c, const Atomic
   }
   const int bn = c.T <= 16 ? 16 : c.T <= 32 ? 32 : c.T <= 64 ? 64 : 128;
   MOE_CUDA(launch_tc_gemm(EPI_LOGITS, bn, maps, p, num_sms(), s));
-  return cuda_status(launch_atomic_select(c.T, c.Nr, c.Nc, c.K, P.ksplit, zr, (long long)c.T * c.Nr, zc,
-                                          (long long)c.T * c.Nc, lr_out, lc_out, idx, g, status, s));
+  if (stage_marks) MOE_TRY(mark_stage(1, s));
+  MOE_CUDA(launch_atomic_select(c.T, c.Nr, c.Nc, c.K, P.ksplit, zr, (long long)c.T * c.Nr, zc, (long long)c.T * c.Nc,
+                                lr_out, lc_out, idx, g, status, s));
+  if (stage_marks) MOE_TRY(mark_stage(2, s));
+  return MOE_OK;
 }
 
 moe_status_t moe_atomic_route(const moe_atomic_config_t* cfg, const void* x, const void* w_row, const void* w_col,
@@ -697,9 +705,11 @@ moe_status_t moe_atomic_forward(const moe_atomic_config_t* cfg, const void* x, c
   cudaStream_t s = (cudaStream_t)stream;
   int32_t* idx = idx_out ? idx_out : at<int32_t>(ws, P.idx);
   float* g = g_out ? g_out : at<float>(ws, P.g);
-  MOE_TRY(atomic_route_impl(c, P, x, w_row, w_col, nullptr, nullptr, idx, g, ws, s));
-  return cuda_status(launch_atomic_experts(c.T, c.d, c.K, c.act, x, w_in, w_out, idx, g, at<float>(ws, P.coef), out,
-                                           (long long)c.Nr * c.Nc, at<int>(ws, P.status), s));
+  MOE_TRY(mark_stage(0, s));
+  MOE_TRY(atomic_route_impl(c, P, x, w_row, w_col, nullptr, nullptr, idx, g, ws, s, true));
+  MOE_CUDA(launch_atomic_experts(c.T, c.d, c.K, c.act, x, w_in, w_out, idx, g, at<float>(ws, P.coef), out,
+                                 (long long)c.Nr * c.Nc, at<int>(ws, P.status), s, true));
+  return mark_stage(4, s);
 }
 
 // ------------------------------------------------------------------ status helpers

@@ -23,6 +23,53 @@ __device__ __forceinline__ uint64_t globaltimer_ns() {
   return t;
 }
 
+// ---------------------------------------------------------------- mbarriers
+__device__ __forceinline__ uint32_t smem_u32(const void* p) { return (uint32_t)__cvta_generic_to_shared(p); }
+
+__device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count) : "memory");
+}
+__device__ __forceinline__ void fence_mbar_init() { asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory"); }
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes) : "memory");
+}
+__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+__device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}\n"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
+// Bounded wait: true when the phase with `parity` completed; false when the time
+// limit ran out or another role already aborted.
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, unsigned long long limit_ns,
+                                          const volatile int* abort_flag) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = globaltimer_ns();
+  while (true) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if (*abort_flag) return false;
+    if (globaltimer_ns() - t0 > limit_ns) return false;
+  }
+}
+
+
+// Bulk copy global -> shared (the copy engine, no tensor map): bytes % 16 == 0, both
+// addresses 16-byte aligned; completion counted on `bar`.
+__device__ __forceinline__ void bulk_copy_g2s(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
+  asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
+               ::"r"(smem_u32(dst)), "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes), "r"(smem_u32(bar))
+               : "memory");
+}
+
 // ---------------------------------------------------------------- dependent launch
 // Every kernel of the layer is launched with programmatic stream serialization:
 // it tells the hardware at entry that its successor may be scheduled
@@ -109,6 +156,10 @@ cudaError_t launch_simt_gemm(int epi, int dtype, const GemmParams& p, int max_ro
 // Routing
 cudaError_t launch_simt_logits(int dtype, int T, int d, int m, const void* x, const void* w_r, const float* bias,
                                float* logits, cudaStream_t s);
+// logits of a few bf16 tokens (T <= 64) against few experts (m <= 32): one block per token.
+bool few_expert_logits_ok(int dtype, int T, int m);
+cudaError_t launch_few_expert_logits(int T, int d, int m, const void* x, const void* w, const float* bias,
+                                     float* logits, cudaStream_t s);
 cudaError_t launch_topk_softmax(int T, int m, int k, int renorm, const float* logits, int32_t* idx, float* w,
                                 cudaStream_t s);
 // Stable counting sort of the tasks by expert: route_index (one block: per-range
@@ -135,7 +186,9 @@ cudaError_t launch_atomic_select(int T, int Nr, int Nc, int K, int ksplit, const
                                  float* g, int* status, cudaStream_t s);
 cudaError_t launch_atomic_experts(int T, int d, int K, int act, const void* x, const void* w_in, const void* w_out,
                                   const int32_t* idx, const float* g, float* coef, void* out, long long n_experts,
-                                  int* status, cudaStream_t s);
+                                  int* status, cudaStream_t s, bool stage_marks = false);
+// Records the profiling hook's event i (moe_set_stage_events) on `s`, if one is set.
+cudaError_t mark_stage_event(int i, cudaStream_t s);
 
 int num_sms();
 void count_launch(int n = 1);

@@ -98,7 +98,9 @@ extern "C" MOE_API moe_status_t moe_route_static(const moe_config_t* cfg, const 
   if (!lg) {
     float* dst = logits_out ? logits_out : reinterpret_cast<float*>(scratch + STATIC_STATUS_BYTES);
     cudaError_t e;
-    if (c.dtype == MOE_F32 || c.T <= 64) {
+    if (few_expert_logits_ok(c.dtype, c.T, c.m)) {  // the same kernel choice as moe_route
+      e = launch_few_expert_logits(c.T, c.d, c.m, x, w_router, bias, dst, s);
+    } else if (c.dtype == MOE_F32 || c.T <= 64) {
       e = launch_simt_logits(c.dtype, c.T, c.d, c.m, x, w_router, bias, dst, s);
     } else {
       // logits^T = W_r . x^T on the tensor cores, one token tile per CTA in one wave

@@ -59,6 +59,74 @@ cudaError_t launch_simt_logits(int dtype, int T, int d, int m, const void* x, co
   return cudaGetLastError();
 }
 
+// ------------------------------------------------------------------ few-expert logits
+// logits[t, e] = x_t . W_r[e] + bias[e] for routers with few experts (m <= 32,
+// bf16): one block per token, 256 threads; each thread takes d / 8 / 256 16-byte
+// chunks of the token and the same chunks of every expert row (all loads
+// independent), forms m partial dots in fp32 and the block sums them (warp
+// shuffles, then the eight warp results in order).
+constexpr int FE_MAX_M = 32;
+constexpr int FE_THREADS = 256;
+
+__global__ void __launch_bounds__(FE_THREADS) few_expert_logits_kernel(int d, int m, const uint4* __restrict__ x,
+                                                                       const uint4* __restrict__ w,
+                                                                       const float* __restrict__ bias,
+                                                                       float* __restrict__ logits) {
+  __shared__ float part[FE_THREADS / 32][FE_MAX_M];
+  pdl_launch_dependents();
+  pdl_wait();
+  const long long t = blockIdx.x;
+  const int chunks = d / 8;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  float acc[FE_MAX_M];
+#pragma unroll
+  for (int e = 0; e < FE_MAX_M; ++e) acc[e] = 0.f;
+  for (int c = threadIdx.x; c < chunks; c += FE_THREADS) {
+    const uint4 xv = x[t * chunks + c];
+    const __nv_bfloat162* px = reinterpret_cast<const __nv_bfloat162*>(&xv);
+    float2 xf[4];
+#pragma unroll
+    for (int h = 0; h < 4; ++h) xf[h] = __bfloat1622float2(px[h]);
+#pragma unroll
+    for (int e = 0; e < FE_MAX_M; ++e) {
+      if (e < m) {
+        const uint4 wv = w[(long long)e * chunks + c];
+        const __nv_bfloat162* pw = reinterpret_cast<const __nv_bfloat162*>(&wv);
+#pragma unroll
+        for (int h = 0; h < 4; ++h) {
+          const float2 wf = __bfloat1622float2(pw[h]);
+          acc[e] = fmaf(xf[h].x, wf.x, acc[e]);
+          acc[e] = fmaf(xf[h].y, wf.y, acc[e]);
+        }
+      }
+    }
+  }
+#pragma unroll
+  for (int e = 0; e < FE_MAX_M; ++e) {
+    if (e < m) {
+      float v = acc[e];
+#pragma unroll
+      for (int o = 16; o; o >>= 1) v += __shfl_xor_sync(FULL, v, o);
+      if (lane == 0) part[warp][e] = v;
+    }
+  }
+  __syncthreads();
+  if (threadIdx.x < m) {
+    float v = 0.f;
+    for (int w8 = 0; w8 < FE_THREADS / 32; ++w8) v += part[w8][threadIdx.x];
+    logits[t * m + threadIdx.x] = v + (bias ? bias[threadIdx.x] : 0.f);
+  }
+}
+
+bool few_expert_logits_ok(int dtype, int T, int m) { return dtype == MOE_BF16 && T <= 64 && m <= FE_MAX_M; }
+
+cudaError_t launch_few_expert_logits(int T, int d, int m, const void* x, const void* w, const float* bias,
+                                     float* logits, cudaStream_t s) {
+  launch_k(few_expert_logits_kernel, T, FE_THREADS, 0, s, d, m, (const uint4*)x, (const uint4*)w, bias, logits);
+  count_launch();
+  return cudaGetLastError();
+}
+
 // ------------------------------------------------------------------ top-k + softmax
 // One warp per token. k rounds of a warp arg-max over the not-yet-chosen
 // experts, ordered by (logit desc, expert index asc). Gate weights: softmax over

@@ -82,7 +82,7 @@ def test_decode_all_tokens():
     _check_layer(cfg, W.make_moe_inputs(cfg), n_sample=cfg.T)
 
 
-@pytest.mark.parametrize("case", ["one_hot", "T1", "ragged_small", "relu_many_experts"])
+@pytest.mark.parametrize("case", ["one_hot", "T1", "ragged_small", "relu_many_experts", "max_experts_max_k"])
 def test_layer_edge_cases(case):
     if case == "one_hot":  # every token's top-1 is the same expert (huge bias)
         cfg = W.small_moe(T=300, d=256, f=192, m=16, k=2, dtype=W.BF16, zipf_s=0.0, index=72)
@@ -96,8 +96,11 @@ def test_layer_edge_cases(case):
         cfg = W.small_moe(T=77, d=136, f=200, m=12, k=3, dtype=W.BF16, zipf_s=1.5, n_shared=1, f_shared=72,
                           index=74)
         inp = W.make_moe_inputs(cfg)
-    else:
+    elif case == "relu_many_experts":
         cfg = W.small_moe(T=1500, d=128, f=320, m=256, k=2, act=W.RELU, dtype=W.BF16, zipf_s=1.0, index=75)
+        inp = W.make_moe_inputs(cfg)
+    else:  # the largest expert count and top-k the library accepts (m = 1024, k = 32)
+        cfg = W.small_moe(T=700, d=64, f=64, m=1024, k=32, dtype=W.BF16, zipf_s=0.5, index=77)
         inp = W.make_moe_inputs(cfg)
     ref, _ = _check_layer(cfg, inp, n_sample=min(cfg.T, 64))
     if case == "one_hot":  # expert 11 holds every token: LIS reaches its maximum m / k
