@@ -234,6 +234,8 @@ MOE_API moe_status_t moe_debug_set_wait_limit_ns(uint64_t ns);
  * A NULL entry skips that
  * boundary (a recorded event between two kernels stops the second one from
  * starting early, so record only the boundaries you time). n = 0 turns it off.
+ * During a stream capture the records become external event-record nodes of
+ * the graph (each replay records the events again).
  * The array is copied. Process-wide and not thread-safe; meant for benchmarks. */
 MOE_API moe_status_t moe_set_stage_events(void* const* events, int n);
 

@@ -30,9 +30,15 @@ static unsigned long long g_wait_limit_ns = 2000ull * 1000 * 1000;
 static cudaEvent_t g_stage_events[8];
 static int g_n_stage_events = 0;
 
+// Inside a stream capture the record becomes an event-record node of the graph
+// (external), so replays of the graph time their stages too.
 cudaError_t mark_stage_event(int i, cudaStream_t s) {
-  if (i < g_n_stage_events && g_stage_events[i]) return cudaEventRecord(g_stage_events[i], s);
-  return cudaSuccess;
+  if (i >= g_n_stage_events || !g_stage_events[i]) return cudaSuccess;
+  cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+  cudaError_t e = cudaStreamIsCapturing(s, &cs);
+  if (e != cudaSuccess) return e;
+  if (cs == cudaStreamCaptureStatusActive) return cudaEventRecordWithFlags(g_stage_events[i], s, cudaEventRecordExternal);
+  return cudaEventRecord(g_stage_events[i], s);
 }
 
 static moe_status_t mark_stage(int i, cudaStream_t s) {

@@ -2,17 +2,18 @@
 // Dynamic Expert Assembly of atomic experts sigma(x w_in^T) w_out.
 //
 // Exact top-K over the implicit Nr x Nc grid (OmniMoE App. A), scores
-// S(i,j) = fl32(lr_i + lc_j), order (S desc, flat id i*Nc + j asc):
-//  1. R = top-K rows by (lr desc, i asc), C = top-K cols by (lc desc, j asc).
-//  2. tau = K-th best score inside R x C.
-//  3. No pair outside R x C scores ABOVE tau: for i not in R and any j, every
-//     (i', j') in R x C' (C' = the K best columns when j not in C, else j itself)
-//     has lr_i' >= lr_i and lc_j' >= lc_j, so fl(lr_i' + lc_j') >= fl(lr_i + lc_j)
-//     (rounding is monotone); that gives K pairs at least as good, so the pair
-//     can only tie tau. Hence the answer = the pairs of R x C above tau, followed
-//     by the lowest-id pairs of the WHOLE grid that equal tau. (Selecting inside
-//     R x C alone is not exact: rounding can make a pair outside R x C tie tau
-//     with a lower flat id.)
+// S(i,j) = fl32(lr_i + lc_j), order (S desc, flat id i*Nc + j asc).
+// With rows and columns sorted by (value desc, index asc), write (a, b) for the
+// pair of the a-th row and the b-th column. Its (a+1)(b+1) dominators (a' <= a,
+// b' <= b) all score at least as much (fp32 rounding is monotone), so
+//  * tau, the K-th best score of the grid, is also the K-th best over the
+//    staircase set {(a, b) : (a+1)(b+1) <= K} (about K ln K pairs): ordering by
+//    (S desc, a asc, b asc) puts every dominator of a pair ahead of it, so the
+//    first K pairs of that order lie in the staircase;
+//  * every pair scoring ABOVE tau lies in the staircase (fewer than K pairs do);
+//  * the pairs equal to tau may lie anywhere: the lowest flat ids among them are
+//    found row by row (row i first holds flat ids i*Nc .. i*Nc + Nc - 1), each
+//    row's tied columns being one contiguous run of the sorted columns.
 #include <float.h>
 
 #include <algorithm>
@@ -26,7 +27,6 @@ constexpr unsigned FULL = 0xffffffffu;
 constexpr int SEL_THREADS = 1024;
 constexpr int SEL_MAX_SIDE = 1024;
 constexpr int SEL_MAX_K = 64;
-constexpr int SEL_CAND = SEL_MAX_K * SEL_MAX_K;  // 4096
 
 __device__ __forceinline__ uint32_t ordered_bits(float v) {
   if (v == 0.f) v = 0.f;  // -0 and +0 are equal scores
@@ -38,25 +38,18 @@ __device__ __forceinline__ uint64_t make_key(float v, uint32_t id) {
 }
 __device__ __forceinline__ uint32_t key_id(uint64_t key) { return 0xFFFFFFFFu - (uint32_t)(key & 0xFFFFFFFFu); }
 
-__device__ float block_max(float v, float* red) {
-#pragma unroll
-  for (int o = 16; o; o >>= 1) v = fmaxf(v, __shfl_xor_sync(FULL, v, o));
-  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = v;
-  __syncthreads();
-  float r = -FLT_MAX;
-  for (int w = 0; w < (int)(blockDim.x >> 5); ++w) r = fmaxf(r, red[w]);
-  __syncthreads();
-  return r;
+// Log-sum-exp state (m, s): the values seen are s * e^m in total. Merging two
+// states rescales both sums to the larger maximum (fp32 exponentials, fp64 sums).
+struct Lse {
+  float m;
+  double s;
+};
+__device__ __forceinline__ Lse lse_merge(Lse a, Lse b) {
+  const float m = fmaxf(a.m, b.m);
+  return {m, a.s * (double)expf(a.m - m) + b.s * (double)expf(b.m - m)};
 }
-__device__ double block_sum(double v, double* red) {
-#pragma unroll
-  for (int o = 16; o; o >>= 1) v += __shfl_xor_sync(FULL, v, o);
-  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = v;
-  __syncthreads();
-  double r = 0.0;
-  for (int w = 0; w < (int)(blockDim.x >> 5); ++w) r += red[w];
-  __syncthreads();
-  return r;
+__device__ __forceinline__ Lse lse_shfl_xor(Lse a, int o) {
+  return {__shfl_xor_sync(FULL, a.m, o), __shfl_xor_sync(FULL, a.s, o)};
 }
 }  // namespace
 
@@ -64,247 +57,335 @@ __device__ __forceinline__ float ordered_to_float(uint32_t key) {
   return __uint_as_float((key & 0x80000000u) ? (key & 0x7FFFFFFFu) : ~key);
 }
 
-constexpr int TIE_CAP = 512;
+// ---- top 64 of a list of distinct 64-bit keys, descending
+// A warp holds 64 keys: element `lane` in k0, element `lane + 32` in k1.
+__device__ __forceinline__ uint64_t kmax(uint64_t a, uint64_t b) { return a > b ? a : b; }
+__device__ __forceinline__ uint64_t kmin(uint64_t a, uint64_t b) { return a > b ? b : a; }
 
-// One block per token. zr/zc: split-K partial logits [ksplit][T][Nr|Nc].
-//  1. log-softmax of the row and column logits (fp32 values; max and
-//     log-sum-exp in fp64);
-//  2. R, C: top-K rows / columns by (value desc, index asc), each element's rank
-//     counted directly (one comparison pass, no sort);
-//  3. tau = K-th largest S over R x C: radix select over the order-preserving
-//     32-bit image of the fp32 scores (four 8-bit passes);
-//  4. the pairs of R x C above tau (fewer than K), and the pairs of the whole grid
-//     equal to tau (scanned in parallel, kept when at most TIE_CAP; otherwise the
-//     exact flat-id-order block scan runs instead), of which the lowest `need` ids;
-//  5. the K winners ordered by (S desc, id asc) by rank counting; g = softmax.
+// Bitonic sort of the warp's 64 keys, descending. For the pair (e, e ^ j) of
+// stage k the lower index keeps the larger key when (e & k) == 0.
+__device__ __forceinline__ void warp_sort64_desc(uint64_t& k0, uint64_t& k1) {
+  const int lane = threadIdx.x & 31;
+#pragma unroll
+  for (int k = 2; k <= 64; k <<= 1) {
+#pragma unroll
+    for (int j = k >> 1; j > 0; j >>= 1) {
+      if (j == 32) {  // k == 64: elements lane and lane + 32 of one thread
+        const uint64_t hi = kmax(k0, k1), lo = kmin(k0, k1);
+        k0 = hi;
+        k1 = lo;
+      } else {
+        const bool lower = (lane & j) == 0;
+        const bool desc0 = (lane & k) == 0;  // element lane (k <= 64)
+        const bool desc1 = k == 64 ? true : (k == 32 ? false : (lane & k) == 0);  // element lane + 32
+        const uint64_t o0 = __shfl_xor_sync(FULL, k0, j), o1 = __shfl_xor_sync(FULL, k1, j);
+        k0 = (lower == desc0) ? kmax(k0, o0) : kmin(k0, o0);
+        k1 = (lower == desc1) ? kmax(k1, o1) : kmin(k1, o1);
+      }
+    }
+  }
+}
+
+// Sorts a bitonic 64-key sequence descending (the merge half of the sort).
+__device__ __forceinline__ void warp_merge64_desc(uint64_t& k0, uint64_t& k1) {
+  const int lane = threadIdx.x & 31;
+  const uint64_t hi = kmax(k0, k1), lo = kmin(k0, k1);
+  k0 = hi;
+  k1 = lo;
+#pragma unroll
+  for (int j = 16; j > 0; j >>= 1) {
+    const bool lower = (lane & j) == 0;
+    const uint64_t o0 = __shfl_xor_sync(FULL, k0, j), o1 = __shfl_xor_sync(FULL, k1, j);
+    k0 = lower ? kmax(k0, o0) : kmin(k0, o0);
+    k1 = lower ? kmax(k1, o1) : kmin(k1, o1);
+  }
+}
+
+// Top 64 (descending) of `nchunks` chunks of 64 keys, one chunk per warp
+// base_warp .. base_warp + nchunks - 1, each warp's keys already in (k0, k1).
+// buf: nchunks x 64 keys of shared memory owned by these warps; on return
+// buf[0..63] holds the result. Called by every thread of the block (it syncs),
+// with max_chunks >= nchunks the same in every thread.
+__device__ void block_top64(uint64_t k0, uint64_t k1, bool mine, int lw, int nchunks, int max_chunks,
+                            uint64_t* buf) {
+  const int lane = threadIdx.x & 31;
+  if (mine) {
+    warp_sort64_desc(k0, k1);
+    buf[lw * 64 + lane] = k0;
+    buf[lw * 64 + lane + 32] = k1;
+  }
+  for (int stride = 1; stride < max_chunks; stride <<= 1) {  // max_chunks: the same in every thread
+    __syncthreads();
+    if (mine && (lw % (2 * stride)) == 0 && lw + stride < nchunks) {
+      const uint64_t* b = buf + (lw + stride) * 64;  // both lists descending: A[i] vs B[63 - i]
+      k0 = kmax(k0, b[63 - lane]);
+      k1 = kmax(k1, b[31 - lane]);
+      warp_merge64_desc(k0, k1);
+      buf[lw * 64 + lane] = k0;
+      buf[lw * 64 + lane + 32] = k1;
+    }
+  }
+  __syncthreads();
+}
+
+// One block (1024 threads) per token. zr/zc: split-K partial logits [ksplit][T][Nr|Nc].
+//  1. log-softmax of the row and column logits (fp32 values; log-sum-exp with
+//     fp64 sums);
+//  2. the top 64 rows and the top 64 columns by (value desc, index asc): warps
+//     0-15 hold the rows, 16-31 the columns, 64 per warp; warp sorts, then a
+//     merge tree;
+//  3. the staircase pairs (a, b), (a+1)(b+1) <= K, keyed by (score, flat id); their
+//     top 64 give tau (the K-th score) and, in final order, the pairs above tau;
+//  4. the lowest flat ids scoring exactly tau: when three counts show that every
+//     pair scoring >= tau is a staircase pair (the usual case), the first K sorted
+//     candidates; otherwise the rows that can reach tau, in index order, one warp
+//     per row scanning its columns (tied ids come out in ascending order), 32 rows
+//     per wave, until `need` are found;
+//  5. g = softmax of the K scores (one warp).
 __global__ void __launch_bounds__(SEL_THREADS, 1)
     atomic_select_kernel(int T, int Nr, int Nc, int K, int ksplit, const float* __restrict__ zr, long long zr_split,
                          const float* __restrict__ zc, long long zc_split, float* __restrict__ lr_out,
                          float* __restrict__ lc_out, int32_t* __restrict__ idx_out, float* __restrict__ g_out,
                          int* status) {
   __shared__ float lr[SEL_MAX_SIDE], lc[SEL_MAX_SIDE];
-  __shared__ float redf[32];
-  __shared__ double redd[32];
-  __shared__ int rows_sel[SEL_MAX_K], cols_sel[SEL_MAX_K];
-  __shared__ unsigned hist[256];
-  __shared__ unsigned whist[SEL_THREADS / 32][257];  // per-warp histograms (+1 bin for non-matching keys)
-  __shared__ uint32_t prefix_s, mask_s;
-  __shared__ int krem_s;
-  __shared__ int n_gt, n_tie, found_s;
-  __shared__ uint32_t gt_ids[SEL_MAX_K], tie_ids[TIE_CAP], win_ids[SEL_MAX_K];
+  __shared__ uint64_t buf[2][16 * 64];  // merge buffers: rows, columns (candidates reuse rows')
+  __shared__ Lse red_r[32], red_c[32];
+  __shared__ double lse_s[2];
+  __shared__ int stair_off[SEL_MAX_K], top_rows[SEL_MAX_K];
+  __shared__ uint32_t win_ids[SEL_MAX_K];
+  __shared__ int row_list[SEL_MAX_SIDE];
   __shared__ int warp_cnt[32];
+  __shared__ int n_cand, n_rows, found_s;
   const int t = blockIdx.x, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int nthr = blockDim.x;
   pdl_launch_dependents();
   pdl_wait();
 
-  // 1. sum the split-K partials; log-softmax of rows and of columns
-  for (int side = 0; side < 2; ++side) {
-    const int n = side ? Nc : Nr;
-    const float* z = side ? zc : zr;
-    const long long sp = side ? zc_split : zr_split;
-    float* l = side ? lc : lr;
-    float v = -FLT_MAX;
-    if (tid < n) {
-      float a = 0.f;
-      for (int s = 0; s < ksplit; ++s) a += z[s * sp + (long long)t * n + tid];
-      l[tid] = a;
-      v = a;
-    }
-    const float mx = block_max(v, redf);
-    const double se = block_sum(tid < n ? (double)expf(l[tid] - mx) : 0.0, redd);
-    const double lse = (double)mx + log(se);
-    if (tid < n) {
-      l[tid] = (float)((double)l[tid] - lse);
-      float* o = side ? lc_out : lr_out;
-      if (o) o[(long long)t * n + tid] = l[tid];
-    }
-    __syncthreads();
-  }
-  // 2. top rows / columns, ranked directly
-  const int kr = min(K, Nr), kc = min(K, Nc);
-  for (int side = 0; side < 2; ++side) {
-    const int n = side ? Nc : Nr;
-    const float* l = side ? lc : lr;
-    for (int i = tid; i < n; i += nthr) {
-      const float v = l[i];
-      int rank = 0;
-      for (int j = 0; j < n; ++j) {
-        const float u = l[j];
-        rank += (u > v) || (u == v && j < i);
+  // 1. sum the split-K partials (all loads of a thread in flight together, summed
+  //    in split order); log-softmax of rows and of columns
+  const bool hr = tid < Nr, hc = tid < Nc;
+  {
+    float ar = 0.f, ac = 0.f;
+    for (int s0 = 0; s0 < ksplit; s0 += 8) {
+      float vr[8], vc[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        const int s = s0 + u;
+        vr[u] = (s < ksplit && hr) ? zr[s * zr_split + (long long)t * Nr + tid] : 0.f;
+        vc[u] = (s < ksplit && hc) ? zc[s * zc_split + (long long)t * Nc + tid] : 0.f;
       }
-      if (rank < (side ? kc : kr)) (side ? cols_sel : rows_sel)[rank] = i;
-    }
-  }
-  if (tid == 0) {
-    prefix_s = 0;
-    mask_s = 0;
-    krem_s = K;
-    n_gt = 0;
-    n_tie = 0;
-  }
-  __syncthreads();
-  // 3. tau: the K-th largest candidate score (radix select, most significant byte first)
-  const int nc = kr * kc;
-  auto cand_score = [&](int i) { return lr[rows_sel[i / kc]] + lc[cols_sel[i % kc]]; };
-  // (The scores of the candidates share their leading bytes, so one shared histogram
-  // would serialise on a few bins: each warp counts into its own histogram, equal
-  // bins within a warp combined by __match_any_sync, then the warps are summed.)
-  const int nw = nthr >> 5;
-  for (int shift = 24; shift >= 0; shift -= 8) {
-    for (int b = tid; b < nw * 257; b += nthr) (&whist[0][0])[b] = 0;
-    __syncthreads();
-    const uint32_t prefix = prefix_s, mask = mask_s;
-    for (int i0 = 0; i0 < nc; i0 += nthr) {
-      const int i = i0 + tid;
-      int bin = 256;
-      if (i < nc) {
-        const uint32_t key = ordered_bits(cand_score(i));
-        if ((key & mask) == prefix) bin = (int)((key >> shift) & 255u);
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        if (s0 + u < ksplit) {
+          ar += vr[u];
+          ac += vc[u];
+        }
       }
-      const unsigned peers = __match_any_sync(0xffffffffu, bin);
-      if (lane == __ffs(peers) - 1) whist[warp][bin] += __popc(peers);
     }
-    __syncthreads();
-    for (int b = tid; b < 256; b += nthr) {
-      unsigned sum = 0;
-      for (int w = 0; w < nw; ++w) sum += whist[w][b];
-      hist[b] = sum;
+    // block-wide log-sum-exp of rows and of columns: a fixed shuffle tree per
+    // warp, then warp 0 over the warps (the same result on every run)
+    Lse er = {hr ? ar : -FLT_MAX, hr ? 1.0 : 0.0}, ec = {hc ? ac : -FLT_MAX, hc ? 1.0 : 0.0};
+#pragma unroll
+    for (int o = 16; o; o >>= 1) {
+      er = lse_merge(er, lse_shfl_xor(er, o));
+      ec = lse_merge(ec, lse_shfl_xor(ec, o));
+    }
+    if (lane == 0) {
+      red_r[warp] = er;
+      red_c[warp] = ec;
     }
     __syncthreads();
     if (warp == 0) {
-      // lane l holds bins 255 - 8l .. 248 - 8l (descending); find the bin where the
-      // running count from the top reaches krem
-      unsigned c8[8], tot = 0;
+      Lse r = lane < SEL_THREADS / 32 ? red_r[lane] : Lse{-FLT_MAX, 0.0};
+      Lse q = lane < SEL_THREADS / 32 ? red_c[lane] : Lse{-FLT_MAX, 0.0};
 #pragma unroll
-      for (int u = 0; u < 8; ++u) {
-        c8[u] = hist[255 - 8 * lane - u];
-        tot += c8[u];
+      for (int o = 16; o; o >>= 1) {
+        r = lse_merge(r, lse_shfl_xor(r, o));
+        q = lse_merge(q, lse_shfl_xor(q, o));
       }
-      unsigned incl = tot;
+      if (lane == 0) lse_s[0] = (double)r.m + log(r.s);
+      if (lane == 1) lse_s[1] = (double)q.m + log(q.s);
+    }
+    if (warp == 1) {  // staircase row offsets (K <= 64 rows: two per lane)
+      const int kr = min(K, Nr), kc = min(K, Nc);
+      const int c0 = lane < kr ? min(K / (lane + 1), kc) : 0;
+      const int c1 = lane + 32 < kr ? min(K / (lane + 33), kc) : 0;
+      int s0 = c0;  // rows 0 .. 31, then rows 32 .. 63
 #pragma unroll
       for (int o = 1; o < 32; o <<= 1) {
-        const unsigned v = __shfl_up_sync(0xffffffffu, incl, o);
-        if (lane >= o) incl += v;
+        const int u = __shfl_up_sync(FULL, s0, o);
+        if (lane >= o) s0 += u;
       }
-      const int krem = krem_s;
-      unsigned above = incl - tot;  // count in the bins above this lane's
-      const bool here = above < (unsigned)krem && incl >= (unsigned)krem;
-      int digit = 0;
-      if (here) {
-        digit = 255 - 8 * lane;
+      const int tot0 = __shfl_sync(FULL, s0, 31);  // rows 0 .. 31
+      int s1 = c1;
 #pragma unroll
-        for (int u = 0; u < 8; ++u) {
-          if (above + c8[u] >= (unsigned)krem) {
-            digit = 255 - 8 * lane - u;
-            break;
-          }
-          above += c8[u];
-        }
+      for (int o = 1; o < 32; o <<= 1) {
+        const int u = __shfl_up_sync(FULL, s1, o);
+        if (lane >= o) s1 += u;
       }
-      const unsigned who = __ballot_sync(0xffffffffu, here);
-      const int src = who ? __ffs(who) - 1 : 31;
-      digit = __shfl_sync(0xffffffffu, digit, src);
-      above = __shfl_sync(0xffffffffu, above, src);
-      if (lane == 0) {
-        krem_s = krem - (int)above;
-        prefix_s = prefix | ((uint32_t)digit << shift);
-        mask_s = mask | (255u << shift);
-      }
+      stair_off[lane] = s0 - c0;
+      stair_off[lane + 32] = tot0 + s1 - c1;
+      if (lane == 31) n_cand = tot0 + s1;
+    }
+    if (tid == 64) {
+      n_rows = 0;
+      found_s = 0;
+    }
+    __syncthreads();
+    if (hr) {
+      lr[tid] = (float)((double)ar - lse_s[0]);
+      if (lr_out) lr_out[(long long)t * Nr + tid] = lr[tid];
+    }
+    if (hc) {
+      lc[tid] = (float)((double)ac - lse_s[1]);
+      if (lc_out) lc_out[(long long)t * Nc + tid] = lc[tid];
     }
     __syncthreads();
   }
-  const uint32_t tau_key = prefix_s;
+  // 2. top 64 rows and columns
+  {
+    const int side = warp >> 4, lw = warp & 15;
+    const int n = side ? Nc : Nr;
+    const float* l = side ? lc : lr;
+    const int e0 = lw * 64 + lane, e1 = e0 + 32;
+    const uint64_t k0 = e0 < n ? make_key(l[e0], (uint32_t)e0) : 0ull;
+    const uint64_t k1 = e1 < n ? make_key(l[e1], (uint32_t)e1) : 0ull;
+    const int nchunks = (n + 63) / 64, max_chunks = (max(Nr, Nc) + 63) / 64;
+    // both sides merge in the same barrier steps: block_top64 syncs the whole block
+    block_top64(k0, k1, lw < nchunks, lw, nchunks, max_chunks, buf[side]);
+  }
+  // 3. staircase candidates and tau: row a of the staircase holds the pairs
+  //    (a, 0 .. cnt_a - 1), cnt_a = min(K / (a + 1), kc), at slots off_a .. off_a + cnt_a - 1
+  const int kr = min(K, Nr), kc = min(K, Nc);
+  const float lc_max = lc[key_id(buf[1][0])];
+  {
+    const int nc = n_cand, nchunks = (nc + 63) / 64;  // nc <= 280 for K <= 64
+    uint64_t kk[2] = {0ull, 0ull};
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      const int c = warp * 64 + lane + 32 * h;
+      if (warp < nchunks && c < nc) {
+        int lo = 0, hi = kr - 1;  // last a with off_a <= c
+        while (lo < hi) {
+          const int mid = (lo + hi + 1) >> 1;
+          if (stair_off[mid] <= c) lo = mid; else hi = mid - 1;
+        }
+        const uint32_t ri = key_id(buf[0][lo]), cj = key_id(buf[1][c - stair_off[lo]]);
+        kk[h] = make_key(lr[ri] + lc[cj], ri * (uint32_t)Nc + cj);
+      }
+    }
+    if (tid < kr) top_rows[tid] = (int)key_id(buf[0][tid]);
+    __syncthreads();  // every read of the rows' list is done: its buffer is reused below
+    block_top64(kk[0], kk[1], warp < nchunks, warp, nchunks, nchunks, buf[0]);
+  }
+  const uint32_t tau_key = (uint32_t)(buf[0][K - 1] >> 32);
   const float tau = ordered_to_float(tau_key);
-  const int need = krem_s;  // tau-valued pairs to take; K - need candidates score above tau
-  // 4. candidates above tau, and every grid pair equal to tau
-  for (int i = tid; i < nc; i += nthr)
-    if (ordered_bits(cand_score(i)) > tau_key) {
-      const int slot = atomicAdd(&n_gt, 1);
-      if (slot < SEL_MAX_K) gt_ids[slot] = (uint32_t)(rows_sel[i / kc] * Nc + cols_sel[i % kc]);
-    }
-  const float lc_max = lc[cols_sel[0]], lr_max = lr[rows_sel[0]];
-  for (int j = tid; j < Nc; j += nthr) {
-    const float cj = lc[j];
-    if (lr_max + cj < tau) continue;  // no row can bring this column up to tau
-    for (int i = 0; i < Nr; ++i) {
-      const float ri = lr[i];
-      if (ri + lc_max < tau) continue;
-      if (ri + cj == tau) {
-        const int slot = atomicAdd(&n_tie, 1);
-        if (slot < TIE_CAP) tie_ids[slot] = (uint32_t)(i * Nc + j);
-      }
+  int n_above = 0;  // the sorted prefix scoring above tau
+  {
+    const bool a0 = lane < K && (uint32_t)(buf[0][lane] >> 32) > tau_key;
+    const bool a1 = lane + 32 < K && (uint32_t)(buf[0][lane + 32] >> 32) > tau_key;
+    n_above = __popc(__ballot_sync(FULL, a0)) + __popc(__ballot_sync(FULL, a1));
+    if (warp == 0) {
+      if (a0) win_ids[lane] = key_id(buf[0][lane]);
+      if (a1) win_ids[lane + 32] = key_id(buf[0][lane + 32]);
     }
   }
-  __syncthreads();
-  if (n_gt != K - need) {  // cannot happen (every pair above tau lies in R x C)
-    if (tid == 0) set_status(status, MOE_ERR_DEVICE_INDEX);
-    return;
+  const int need = K - n_above;
+  // 4. ties at tau. Every pair scoring >= tau is a staircase pair when (i) at most
+  //    kr rows reach tau with the best column, (ii) at most kc columns reach tau
+  //    with the best row and (iii) the first pair past each staircase row, (a, cnt_a)
+  //    with cnt_a < kc, scores below tau: by (i) and (ii) such a pair has row rank
+  //    a < kr and column rank b < kc, and outside the staircase b >= cnt_a, so
+  //    (a, cnt_a) dominates it. Then the winners are the first K sorted candidates.
+  const float lr_max = lr[top_rows[0]];
+  const int reach_r = __syncthreads_count(tid < Nr && lr[tid] + lc_max >= tau);
+  const int reach_c = __syncthreads_count(tid < Nc && lr_max + lc[tid] >= tau);
+  bool past = false;
+  if (tid < kr) {
+    const int ca = min(K / (tid + 1), kc);
+    past = ca < kc && lr[top_rows[tid]] + lc[key_id(buf[1][ca])] >= tau;
   }
-  if (n_tie <= TIE_CAP) {
-    // lowest `need` tied ids: rank the ids (they are distinct)
-    for (int u = tid; u < n_tie; u += nthr) {
-      const uint32_t id = tie_ids[u];
-      int rank = 0;
-      for (int v = 0; v < n_tie; ++v) rank += tie_ids[v] < id;
-      if (rank < need) win_ids[K - need + rank] = id;
-    }
-  } else {
-    // massive ties: walk the grid rows in flat-id order, block-wide, until `need` found
-    if (tid == 0) found_s = 0;
+  const int any_past = __syncthreads_or(past);
+  const bool fast = reach_r <= kr && reach_c <= kc && !any_past;
+  if (fast) {
+    if (tid >= n_above && tid < K) win_ids[tid] = key_id(buf[0][tid]);
     __syncthreads();
-    for (int i = 0; i < Nr; ++i) {
-      if (found_s >= need) break;
-      if (lr[i] + lc_max < tau) continue;  // uniform across the block
-      bool eq = false;
-      int jj = 0;
-      const int per = (Nc + nthr - 1) / nthr;  // Nc <= 1024 = nthr, so per == 1
-      for (int r = 0; r < per; ++r) {
-        jj = tid * per + r;
-        if (jj < Nc && lr[i] + lc[jj] == tau) {
-          eq = true;
-          break;
-        }
-      }
-      const unsigned bal = __ballot_sync(0xffffffffu, eq);
+  } else {  // rows able to reach tau, in index order, scanned for tied pairs
+    {
+      const bool cand_row = tid < Nr && lr[tid] + lc_max >= tau;
+      const unsigned bal = __ballot_sync(FULL, cand_row);
       if (lane == 0) warp_cnt[warp] = __popc(bal);
       __syncthreads();
-      int before = 0, total = 0;
-      for (int w = 0; w < (int)(nthr >> 5); ++w) {
-        if (w < warp) before += warp_cnt[w];
-        total += warp_cnt[w];
-      }
-      const int base = found_s;
-      if (eq) {
-        const int p = base + before + __popc(bal & ((1u << lane) - 1u));
-        if (p < need) win_ids[K - need + p] = (uint32_t)(i * Nc + jj);
-      }
-      __syncthreads();
-      if (tid == 0) found_s = base + total;
+      int before = 0;
+      for (int w = 0; w < warp; ++w) before += warp_cnt[w];
+      if (cand_row) row_list[before + __popc(bal & ((1u << lane) - 1u))] = tid;
+      if (tid == SEL_THREADS - 1) n_rows = before + __popc(bal);
       __syncthreads();
     }
+    const int nrows = n_rows;
+    uint32_t* tied = reinterpret_cast<uint32_t*>(buf[1]) + warp * SEL_MAX_K;  // first tied columns of this warp's row
+    for (int w0 = 0; w0 < nrows; w0 += SEL_THREADS / 32) {
+      if (found_s >= need) break;  // uniform: read after a barrier
+      const int ri = w0 + warp;
+      const int r = ri < nrows ? row_list[ri] : -1;
+      int cnt = 0;
+      if (r >= 0) {
+        const float lrr = lr[r];
+        for (int j0 = 0; j0 < Nc; j0 += 32) {
+          const int j = j0 + lane;
+          const bool eq = j < Nc && lrr + lc[j] == tau;
+          const unsigned bal = __ballot_sync(FULL, eq);
+          const int q = cnt + __popc(bal & ((1u << lane) - 1u));
+          if (eq && q < SEL_MAX_K) tied[q] = (uint32_t)j;
+          cnt += __popc(bal);
+        }
+      }
+      if (lane == 0) warp_cnt[warp] = cnt;
+      __syncthreads();
+      int before = found_s, wave = 0;
+      for (int w = 0; w < SEL_THREADS / 32; ++w) {
+        const int c = warp_cnt[w];
+        if (w < warp) before += c;
+        wave += c;
+      }
+      if (r >= 0 && cnt > 0 && before < need) {  // this row's lowest tied ids (ascending)
+        const int take = min(cnt, need - before);  // <= need <= SEL_MAX_K
+        for (int q = lane; q < take; q += 32) win_ids[n_above + before + q] = (uint32_t)r * (uint32_t)Nc + tied[q];
+      }
+      __syncthreads();
+      if (tid == 0) found_s += wave;
+      __syncthreads();
+    }
+    if (found_s < need) {  // cannot happen: tau is the score of a grid pair
+      if (tid == 0) set_status(status, MOE_ERR_DEVICE_INDEX);
+      return;
+    }
   }
-  for (int u = tid; u < K - need; u += nthr) win_ids[u] = gt_ids[u];
-  __syncthreads();
-  // 5. order the K winners by (S desc, id asc), then the gate weights
-  auto score_of = [&](uint32_t id) { return lr[id / Nc] + lc[id % Nc]; };
-  uint32_t my_id = 0;
-  int my_rank = 0;
-  if (tid < K) {
-    my_id = win_ids[tid];
-    const uint64_t mk = make_key(score_of(my_id), my_id);
-    for (int v = 0; v < K; ++v) my_rank += make_key(score_of(win_ids[v]), win_ids[v]) > mk;
-  }
-  __syncthreads();
-  if (tid < K) rows_sel[my_rank] = (int)my_id;  // reuse as the ordered output staging area
-  __syncthreads();
-  const float smax = score_of((uint32_t)rows_sel[0]);
-  double z = 0.0;
-  if (tid < K) z = (double)expf(score_of((uint32_t)rows_sel[tid]) - smax);
-  const double zs = block_sum(z, redd);
-  if (tid < K) {
-    idx_out[(long long)t * K + tid] = rows_sel[tid];
-    g_out[(long long)t * K + tid] = (float)(z / zs);
+  // 5. the gate weights (winners are already ordered by (score desc, id asc))
+  if (warp == 0) {
+    float sc0 = 0.f, sc1 = 0.f;
+    uint32_t id0 = 0, id1 = 0;
+    if (lane < K) {
+      id0 = win_ids[lane];
+      sc0 = lr[id0 / Nc] + lc[id0 % Nc];
+    }
+    if (lane + 32 < K) {
+      id1 = win_ids[lane + 32];
+      sc1 = lr[id1 / Nc] + lc[id1 % Nc];
+    }
+    const float smax = __shfl_sync(FULL, sc0, 0);
+    const double z0 = lane < K ? (double)expf(sc0 - smax) : 0.0;
+    const double z1 = lane + 32 < K ? (double)expf(sc1 - smax) : 0.0;
+    double zs = z0 + z1;
+#pragma unroll
+    for (int o = 16; o; o >>= 1) zs += __shfl_xor_sync(FULL, zs, o);
+    if (lane < K) {
+      idx_out[(long long)t * K + lane] = (int32_t)id0;
+      g_out[(long long)t * K + lane] = (float)(z0 / zs);
+    }
+    if (lane + 32 < K) {
+      idx_out[(long long)t * K + lane + 32] = (int32_t)id1;
+      g_out[(long long)t * K + lane + 32] = (float)(z1 / zs);
+    }
   }
 }
 
@@ -318,54 +399,64 @@ cudaError_t launch_atomic_select(int T, int Nr, int Nc, int K, int ksplit, const
 }
 
 // ------------------------------------------------------------------ assembly
-// coef[t, s] = g[t, s] * act(x_t . w_in[idx[t, s]]): one warp per task, 16-byte
-// loads of the 2 d-byte expert row issued eight at a time, fp32 dot, shuffle-tree
-// reduction.
-__global__ void atomic_coef_kernel(int T, int d, int K, int act, const uint4* __restrict__ x,
-                                   const uint4* __restrict__ w_in, const int32_t* __restrict__ idx,
-                                   const float* __restrict__ g, float* __restrict__ coef, long long n_experts,
-                                   int* status) {
+// coef[t, s] = g[t, s] * act(x_t . w_in[idx[t, s]]). Block (task group, token):
+// eight warps, one task each, over the row in windows of 4096 elements. Each lane
+// issues its sixteen 16-byte loads of the expert row before the window of x_t is
+// staged in shared memory, so the gathers of all tasks are in flight together;
+// fp32 dot, shuffle-tree reduction.
+constexpr int COEF_WARPS = 8, COEF_WIN = 512;  // window: 512 chunks of 8 bf16
+__global__ void __launch_bounds__(COEF_WARPS * 32)
+    atomic_coef_kernel(int T, int d, int K, int act, const uint4* __restrict__ x, const uint4* __restrict__ w_in,
+                       const int32_t* __restrict__ idx, const float* __restrict__ g, float* __restrict__ coef,
+                       long long n_experts, int* status) {
+  __shared__ uint4 xs[COEF_WIN];
   pdl_launch_dependents();
   pdl_wait();
-  const int lane = threadIdx.x & 31;
-  const long long task = (long long)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
-  if (task >= (long long)T * K) return;
-  const long long t = task / K;
-  const long long e = idx[task];
-  if (e < 0 || e >= n_experts) {
-    if (lane == 0) {
-      set_status(status, MOE_ERR_DEVICE_INDEX);
-      coef[task] = 0.f;
-    }
-    return;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const long long t = blockIdx.y;
+  const int sl = blockIdx.x * COEF_WARPS + warp;
+  const bool has = sl < K;
+  const long long task = t * K + sl;
+  const long long e = has ? (long long)idx[task] : 0;
+  const bool ok = has && e >= 0 && e < n_experts;
+  if (has && !ok && lane == 0) {
+    set_status(status, MOE_ERR_DEVICE_INDEX);
+    coef[task] = 0.f;
   }
   const int chunks = d / 8;
-  const uint4* xr = x + t * chunks;
-  const uint4* wr = w_in + e * chunks;
+  const uint4* wr = w_in + (ok ? e : 0) * chunks;
   float s = 0.f;
-  for (int c0 = lane; c0 < chunks; c0 += 32 * 8) {
-    uint4 a[8], b[8];
+  for (int w0 = 0; w0 < chunks; w0 += COEF_WIN) {
+    const int wn = min(COEF_WIN, chunks - w0);
+    uint4 b[COEF_WIN / 32];
+    if (ok) {
 #pragma unroll
-    for (int u = 0; u < 8; ++u) {
-      const int c = c0 + 32 * u;
-      if (c < chunks) {
-        a[u] = xr[c];
-        b[u] = wr[c];
+      for (int u = 0; u < COEF_WIN / 32; ++u) {
+        const int c = lane + 32 * u;
+        if (c < wn) b[u] = wr[w0 + c];
       }
     }
+    __syncthreads();  // the previous window is consumed
+    for (int c = threadIdx.x; c < wn; c += COEF_WARPS * 32) xs[c] = x[t * chunks + w0 + c];
+    __syncthreads();
+    if (ok) {
 #pragma unroll
-    for (int u = 0; u < 8; ++u) {
-      if (c0 + 32 * u >= chunks) break;
-      const __nv_bfloat162* pa = reinterpret_cast<const __nv_bfloat162*>(&a[u]);
-      const __nv_bfloat162* pb = reinterpret_cast<const __nv_bfloat162*>(&b[u]);
+      for (int u = 0; u < COEF_WIN / 32; ++u) {
+        const int c = lane + 32 * u;
+        if (c >= wn) break;
+        const uint4 a = xs[c];
+        const __nv_bfloat162* pa = reinterpret_cast<const __nv_bfloat162*>(&a);
+        const __nv_bfloat162* pb = reinterpret_cast<const __nv_bfloat162*>(&b[u]);
 #pragma unroll
-      for (int h = 0; h < 4; ++h) {
-        const float2 fa = __bfloat1622float2(pa[h]), fb = __bfloat1622float2(pb[h]);
-        s = fmaf(fa.x, fb.x, s);
-        s = fmaf(fa.y, fb.y, s);
+        for (int h = 0; h < 4; ++h) {
+          const float2 fa = __bfloat1622float2(pa[h]), fb = __bfloat1622float2(pb[h]);
+          s = fmaf(fa.x, fb.x, s);
+          s = fmaf(fa.y, fb.y, s);
+        }
       }
     }
   }
+  if (!ok) return;
 #pragma unroll
   for (int o = 16; o; o >>= 1) s += __shfl_xor_sync(FULL, s, o);
   if (lane == 0) {
@@ -376,9 +467,9 @@ __global__ void atomic_coef_kernel(int T, int d, int K, int act, const uint4* __
 
 // out[t, c..c+7] = sum_s coef[t, s] w_out[idx[t, s], c..c+7]. A block handles one
 // token and 64 column chunks of 8; its four thread groups take every fourth slot
-// (loads issued eight at a time) and their partial sums are added in group order,
+// (loads issued sixteen at a time) and their partial sums are added in group order,
 // so the result is the same on every run.
-constexpr int ASM_GROUPS = 4, ASM_CHUNKS = 64;
+constexpr int ASM_GROUPS = 4, ASM_CHUNKS = 64, ASM_BATCH = 16;
 __global__ void atomic_assemble_kernel(int T, int d, int K, const uint4* __restrict__ w_out,
                                        const int32_t* __restrict__ idx, const float* __restrict__ coef,
                                        uint4* __restrict__ out, long long n_experts) {
@@ -392,11 +483,11 @@ __global__ void atomic_assemble_kernel(int T, int d, int K, const uint4* __restr
   const int c = (blockIdx.x % cblocks) * ASM_CHUNKS + cl;
   float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
   if (c < chunks) {
-    for (int s0 = grp; s0 < K; s0 += ASM_GROUPS * 8) {
-      uint4 v[8];
-      float cf[8];
+    for (int s0 = grp; s0 < K; s0 += ASM_GROUPS * ASM_BATCH) {
+      uint4 v[ASM_BATCH];
+      float cf[ASM_BATCH];
 #pragma unroll
-      for (int u = 0; u < 8; ++u) {
+      for (int u = 0; u < ASM_BATCH; ++u) {
         const int sl = s0 + ASM_GROUPS * u;
         cf[u] = 0.f;
         if (sl < K) {
@@ -408,7 +499,7 @@ __global__ void atomic_assemble_kernel(int T, int d, int K, const uint4* __restr
         }
       }
 #pragma unroll
-      for (int u = 0; u < 8; ++u) {
+      for (int u = 0; u < ASM_BATCH; ++u) {
         if (cf[u] == 0.f) continue;
         const __nv_bfloat162* pv = reinterpret_cast<const __nv_bfloat162*>(&v[u]);
 #pragma unroll
@@ -437,9 +528,8 @@ __global__ void atomic_assemble_kernel(int T, int d, int K, const uint4* __restr
 cudaError_t launch_atomic_experts(int T, int d, int K, int act, const void* x, const void* w_in, const void* w_out,
                                   const int32_t* idx, const float* g, float* coef, void* out, long long n_experts,
                                   int* status, cudaStream_t s, bool stage_marks) {
-  const long long tasks = (long long)T * K;
-  launch_k(atomic_coef_kernel, (unsigned)((tasks + 7) / 8), 256, 0, s, T, d, K, act, (const uint4*)x, (const uint4*)w_in,
-                                                                 idx, g, coef, n_experts, status);
+  launch_k(atomic_coef_kernel, dim3((K + COEF_WARPS - 1) / COEF_WARPS, T), COEF_WARPS * 32, 0, s, T, d, K, act,
+           (const uint4*)x, (const uint4*)w_in, idx, g, coef, n_experts, status);
   count_launch();
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
@@ -447,7 +537,6 @@ cudaError_t launch_atomic_experts(int T, int d, int K, int act, const void* x, c
   const int cblocks = (d / 8 + ASM_CHUNKS - 1) / ASM_CHUNKS;
   launch_k(atomic_assemble_kernel, (unsigned)(T * cblocks), ASM_GROUPS * ASM_CHUNKS, 0, s, T, d, K,
            (const uint4*)w_out, idx, coef, (uint4*)out, n_experts);
-  
   count_launch();
   return cudaGetLastError();
 }

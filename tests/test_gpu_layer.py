@@ -172,3 +172,50 @@ def test_atomic_select_ties_and_rounding_collapse():
     lr, lc, idx, g, out, _ = _atomic(cfg, inp)
     oidx, og = O.atomic_select(lr, lc, cfg.K)
     np.testing.assert_array_equal(idx, oidx)
+
+
+def _route_only(cfg, inp):
+    c = moe.make_atomic_config(cfg.T, cfg.d, cfg.Nr, cfg.Nc, cfg.K, cfg.act)
+    ws = moe.workspace(c)
+    d_in = device_inputs(inp)
+    lr = torch.empty((cfg.T, cfg.Nr), dtype=torch.float32, device="cuda")
+    lc = torch.empty((cfg.T, cfg.Nc), dtype=torch.float32, device="cuda")
+    idx = torch.empty((cfg.T, cfg.K), dtype=torch.int32, device="cuda")
+    g = torch.empty((cfg.T, cfg.K), dtype=torch.float32, device="cuda")
+    moe.moe_atomic_route(c, d_in["x"], d_in["w_row"], d_in["w_col"], lr, lc, idx, g, ws)
+    assert moe.moe_read_device_status(ws) == moe.OK
+    return host(lr), host(lc), host(idx), host(g)
+
+
+def _level_weights(rows, d, levels, seed):
+    """bf16 weights whose only non-zero column is 0, holding integers in [0, levels)."""
+    vals = np.random.default_rng(seed).integers(0, levels, size=rows).astype(np.float32)
+    w = np.zeros((rows, d), np.uint16)
+    w[:, 0] = (vals.view(np.uint32) >> 16).astype(np.uint16)
+    return w
+
+
+@pytest.mark.parametrize("Nr,Nc,K,kind", [
+    (64, 1024, 7, "random"),      # rectangular grid, K below the row count
+    (1024, 64, 1, "random"),      # K = 1
+    (1024, 1024, 64, "random"),   # largest grid, largest K
+    (1024, 1024, 64, "equal"),    # every pair ties: the K lowest flat ids
+    (128, 128, 64, "levels"),     # few distinct scores: long tied runs per row
+    (1024, 512, 33, "levels"),
+])
+def test_atomic_select_grid_shapes(Nr, Nc, K, kind):
+    cfg = W.AtomicWorkload("atomic_grid", 94, T=3, d=64, Nr=Nr, Nc=Nc, K=K, act=W.ACT_SILU)
+    inp = W.make_atomic_inputs(cfg, experts=False)
+    if kind != "random":
+        x = np.zeros((cfg.T, cfg.d), np.uint16)
+        x[:, 0] = 0x3F80  # bf16 1.0: the logits are column 0 of the weights
+        inp["x"] = x
+        levels = 1 if kind == "equal" else 3
+        inp["w_row"] = _level_weights(Nr, cfg.d, levels, 6)
+        inp["w_col"] = _level_weights(Nc, cfg.d, levels, 7)
+    lr, lc, idx, g = _route_only(cfg, inp)
+    oidx, og = O.atomic_select(lr, lc, cfg.K)
+    np.testing.assert_array_equal(idx, oidx)
+    np.testing.assert_allclose(g, og, rtol=GATE_RTOL * 4, atol=1e-9)
+    if kind == "equal":
+        np.testing.assert_array_equal(idx, np.tile(np.arange(K, dtype=np.int32), (cfg.T, 1)))
