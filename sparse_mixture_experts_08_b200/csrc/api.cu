@@ -99,7 +99,8 @@ static Plan make_plan(const moe_config_t& c) {
 }
 
 struct Layout {
-  size_t status, logits, idx, w, counts, offsets, lis, perm, inv_perm, w_perm, start, x_perm, h, h_sh, y, y_sh, total;
+  size_t status, logits, idx, w, counts, offsets, lis, perm, inv_perm, w_perm, start, x_perm, h, h_sh, y, y_sh;
+  size_t lrank, tile_cnt, total;
 };
 
 static Layout make_layout(const moe_config_t& c, const Plan& p) {
@@ -128,6 +129,8 @@ static Layout make_layout(const moe_config_t& c, const Plan& p) {
   L.h_sh = take((size_t)c.n_shared * T * std::max(c.f_shared, 0) * p.es);
   L.y = take((size_t)p.ksplit * Tk * c.d * 4);
   L.y_sh = take((size_t)p.ksplit * c.n_shared * T * c.d * 4);
+  L.lrank = take(Tk * 4);                          // fused router: task ranks within their tile
+  L.tile_cnt = take((T + 127) / 128 * c.m * 4);    // and tasks per expert per 128-token tile
   L.total = off;
   return L;
 }
@@ -386,6 +389,9 @@ moe_status_t moe_route(const moe_config_t* cfg, const void* x, const void* w_rou
   cudaStream_t s = (cudaStream_t)stream;
   int* status = at<int>(ws, L.status);
   const float* lg = logits_in;
+  if (!lg && fused_route_ok(c))  // logits and top-k in one tensor-core launch
+    return cuda_status(launch_route_topk(c, x, w_router, bias, logits_out, topk_idx, topk_w, nullptr, nullptr, status,
+                                         g_wait_limit_ns, s));
   if (!lg) {
     float* dst = logits_out ? logits_out : at<float>(ws, L.logits);
     MOE_TRY(run_router(c, x, w_router, bias, dst, status, s));
@@ -532,17 +538,30 @@ moe_status_t moe_layer_forward(const moe_config_t* cfg, const void* x, const voi
   int32_t* inv_perm = at<int32_t>(ws, L.inv_perm);
   const long long Tk = (long long)c.T * c.k;
 
-  MOE_TRY(mark_stage(0, s));
-  MOE_TRY(run_router(c, x, w_router, bias, logits, status, s));
-  MOE_TRY(mark_stage(1, s));
-  MOE_CUDA(launch_topk_softmax(c.T, c.m, c.k, c.renormalize, logits, idx, w, s));
-  MOE_TRY(mark_stage(2, s));
   float* w_perm = at<float>(ws, L.w_perm);
-  int32_t* start = at<int32_t>(ws, L.start);
-  MOE_CUDA(launch_route_index(1, c.T, c.k, c.m, idx, counts, offsets, lis, start, status, s));
-  MOE_CUDA(launch_rank(c.T, c.k, c.m, idx, offsets, start, w, perm, inv_perm, w_perm, status, s));
-  MOE_TRY(mark_stage(3, s));
-  MOE_CUDA(launch_permute_rows(c.dtype, (int)Tk, c.k, c.d, x, inv_perm, at<void>(ws, L.x_perm), s));
+  MOE_TRY(mark_stage(0, s));
+  if (fused_route_ok(c)) {
+    // router + top-k + per-tile counts and ranks in the GEMM epilogue, then one
+    // kernel for offsets / LIS / permutation / row copy (stages 1-3 coincide)
+    int32_t* lrank = at<int32_t>(ws, L.lrank);
+    int32_t* tile_cnt = at<int32_t>(ws, L.tile_cnt);
+    MOE_CUDA(launch_route_topk(c, x, w_router, bias, logits_out, idx, w, lrank, tile_cnt, status, g_wait_limit_ns, s));
+    MOE_TRY(mark_stage(1, s));
+    MOE_TRY(mark_stage(2, s));
+    MOE_TRY(mark_stage(3, s));
+    MOE_CUDA(launch_route_scatter(c.dtype, c.T, c.k, c.m, c.d, tile_cnt, idx, lrank, w, x, counts, offsets, lis, perm,
+                                  inv_perm, w_perm, at<void>(ws, L.x_perm), status, s));
+  } else {
+    MOE_TRY(run_router(c, x, w_router, bias, logits, status, s));
+    MOE_TRY(mark_stage(1, s));
+    MOE_CUDA(launch_topk_softmax(c.T, c.m, c.k, c.renormalize, logits, idx, w, s));
+    MOE_TRY(mark_stage(2, s));
+    int32_t* start = at<int32_t>(ws, L.start);
+    MOE_CUDA(launch_route_index(1, c.T, c.k, c.m, idx, counts, offsets, lis, start, status, s));
+    MOE_CUDA(launch_rank(c.T, c.k, c.m, idx, offsets, start, w, perm, inv_perm, w_perm, status, s));
+    MOE_TRY(mark_stage(3, s));
+    MOE_CUDA(launch_permute_rows(c.dtype, (int)Tk, c.k, c.d, x, inv_perm, at<void>(ws, L.x_perm), s));
+  }
   MOE_TRY(mark_stage(4, s));
   FfnIo io;
   std::memset(&io, 0, sizeof(io));

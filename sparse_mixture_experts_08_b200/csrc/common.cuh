@@ -98,7 +98,19 @@ cudaError_t launch_k(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem,
 // Every launcher returns cudaSuccess or the launch error; arguments were checked
 // by the C-ABI layer before.
 
-enum Epi { EPI_LOGITS = 0, EPI_SWIGLU = 1, EPI_RELU = 2, EPI_DOWN = 3 };
+enum Epi { EPI_LOGITS = 0, EPI_SWIGLU = 1, EPI_RELU = 2, EPI_DOWN = 3, EPI_ROUTE = 4 };
+
+// EPI_ROUTE: the router with tokens as the MMA's M rows (A = x) and all experts in
+// one N tile (B = W_r, m <= 256 rows): each epilogue thread owns a token's logits.
+constexpr int ROUTE_MAX_M = 256;
+constexpr int ROUTE_MAX_K = 8;
+// Each CTA streams one 128-token tile through its SM, so the fused router pays off
+// only when the batch has tiles for most SMs; smaller batches keep the separate
+// router, top-k and sort kernels (measured: slower fused at 2048 and 4096 tokens).
+constexpr int ROUTE_MIN_T = 8192;
+inline bool fused_route_ok(const moe_config_t& c) {
+  return c.dtype == MOE_BF16 && c.m <= ROUTE_MAX_M && c.k <= ROUTE_MAX_K && c.T >= ROUTE_MIN_T;
+}
 
 // One class of problems for the grouped GEMM  out = epi(A_g . B_rows^T):
 // A_g = rows [g*R, g*R + R) of a K-major weight matrix, B rows = one segment.
@@ -121,6 +133,12 @@ struct GemmClass {
   const float* task_w;       // DOWN: row weight task_w[perm[row]] (nullable = 1)
   const int* perm;
   int scatter_k1;            // DOWN with top-1 routing: write bf16 out[perm[row]] (combine fused)
+  // ROUTE: top-k selection in the epilogue (out = fp32 logits [T, m], nullable)
+  int k_sel, renorm;
+  int32_t* sel_idx;          // [T, k] experts by (logit desc, expert asc)
+  float* sel_w;              // [T, k] gate weights
+  int32_t* lrank;            // [T, k] rank of task (t, s) among the tile's tasks of its expert (nullable)
+  int32_t* tile_cnt;         // [tiles][m] tasks per expert in each 128-token tile (with lrank)
   // SIMT path only (fp32 / bf16 element pointers, row-major)
   const void* a0;            // [n_groups * R, K]
   const void* a1;            // second matrix (SwiGLU up) or nullptr
@@ -148,6 +166,11 @@ struct TcMaps {
 cudaError_t launch_tc_gemm(int epi, int bn, const TcMaps& maps, const GemmParams& p, int num_ctas,
                            cudaStream_t s);
 int tc_pick_bn(int epi, double avg_rows_per_group);
+// Router logits + top-k softmax (+ per-tile expert counts and task ranks when lrank
+// and tile_cnt are given) in one tensor-core launch (EPI_ROUTE); logits nullable.
+cudaError_t launch_route_topk(const moe_config_t& c, const void* x, const void* w_r, const float* bias, float* logits,
+                              int32_t* idx, float* w, int32_t* lrank, int32_t* tile_cnt, int* status,
+                              unsigned long long wait_limit_ns, cudaStream_t s);
 int tc_max_groups();
 
 // SIMT grouped linear (fp32 or bf16 inputs, fp32 math), same GemmParams.
@@ -169,6 +192,12 @@ cudaError_t launch_topk_softmax(int T, int m, int k, int renorm, const float* lo
 void route_ranges(int Tk, int m, int* R, int* L);
 cudaError_t launch_route_index(int mode, int T, int k, int m, const int32_t* idx, int32_t* counts, int32_t* offsets,
                                moe_lis_t* lis, int32_t* start, int* status, cudaStream_t s);
+// offsets, counts, LIS, perm / inv_perm / w_perm and x_perm from the router's tile
+// counts and ranks (EPI_ROUTE): one block per (128-token tile, column part).
+cudaError_t launch_route_scatter(int dtype, int T, int k, int m, int d, const int32_t* tile_cnt, const int32_t* idx,
+                                 const int32_t* lrank, const float* task_w, const void* x, int32_t* counts,
+                                 int32_t* offsets, moe_lis_t* lis, int32_t* perm, int32_t* inv_perm, float* w_perm,
+                                 void* x_perm, int* status, cudaStream_t s);
 cudaError_t launch_rank(int T, int k, int m, const int32_t* idx, const int32_t* offsets, const int32_t* start,
                         const float* task_w, int32_t* perm, int32_t* inv_perm, float* w_perm, int* status,
                         cudaStream_t s);

@@ -95,6 +95,15 @@ extern "C" MOE_API moe_status_t moe_route_static(const moe_config_t* cfg, const 
   int* status = reinterpret_cast<int*>(scratch);
   if (cudaMemsetAsync(status, 0, sizeof(int), s) != cudaSuccess) return MOE_ERR_CUDA;
   const float* lg = logits_in;
+  if (!lg && fused_route_ok(c)) {  // the same kernel choice as moe_route: logits + top-k in one launch
+    if (launch_route_topk(c, x, w_router, bias, logits_out, topk_idx, topk_w, nullptr, nullptr, status,
+                          2000ull * 1000 * 1000, s) != cudaSuccess)
+      return MOE_ERR_CUDA;
+    if (device_status_out &&
+        cudaMemcpyAsync(device_status_out, status, sizeof(int32_t), cudaMemcpyDeviceToDevice, s) != cudaSuccess)
+      return MOE_ERR_CUDA;
+    return MOE_OK;
+  }
   if (!lg) {
     float* dst = logits_out ? logits_out : reinterpret_cast<float*>(scratch + STATIC_STATUS_BYTES);
     cudaError_t e;

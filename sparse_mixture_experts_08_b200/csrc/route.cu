@@ -449,6 +449,224 @@ cudaError_t launch_permute_rows(int dtype, int Tk, int k, int d, const void* x, 
   return cudaGetLastError();
 }
 
+// ------------------------------------------------ offsets, LIS and the permutation from tile ranks
+// The router's epilogue left, per 128-token tile, the tasks of each expert
+// (tile_cnt[tile][e]) and each task's rank among its tile's tasks of that expert
+// (lrank). In the stable counting sort task q = t k + s of expert e goes to
+//   offsets[e] + (tasks of e in earlier tiles) + lrank[q].
+// Block (tile, part): every block sums the whole count table (the totals give
+// the offsets), places its tile's tasks and copies its share of their rows (the
+// 16-byte columns are split over the parts). Part 0 writes inv_perm, perm and
+// w_perm; block (0, 0) writes counts, offsets and the LIS (R&Q Definition 1).
+// The block's row chunks are loaded in the same batch as the tables, so the copy
+// costs one store pass at the end.
+constexpr int RS_THREADS = 512;
+constexpr int RS_PRE = 8;  // row chunks per thread loaded ahead
+__global__ void __launch_bounds__(RS_THREADS)
+    route_scatter_kernel(int T, int k, int m, int ntiles, int parts, int chunks, const int32_t* __restrict__ tile_cnt,
+                         const int32_t* __restrict__ idx, const int32_t* __restrict__ lrank,
+                         const float* __restrict__ task_w, const int4* __restrict__ x, int32_t* __restrict__ counts,
+                         int32_t* __restrict__ offsets, moe_lis_t* __restrict__ lis, int32_t* __restrict__ perm,
+                         int32_t* __restrict__ inv_perm, float* __restrict__ w_perm, int4* __restrict__ x_perm,
+                         int* status) {
+  __shared__ int part_t[RS_THREADS], part_b[RS_THREADS];
+  __shared__ int tot[ROUTE_MAX_M], base[ROUTE_MAX_M], off[ROUTE_MAX_M + 1];
+  __shared__ int dest[128 * ROUTE_MAX_K];
+  __shared__ int wsum[RS_THREADS / 32], wmax[RS_THREADS / 32], warg[RS_THREADS / 32];
+  __shared__ int prior_s;
+  const int tile = blockIdx.x, part = blockIdx.y, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const long long Tk = (long long)T * k;
+  const long long q0 = (long long)tile * 128 * k;
+  const int nitems = (int)min((long long)128 * k, Tk - q0);
+  const int c_lo = (int)((long long)chunks * part / parts), c_hi = (int)((long long)chunks * (part + 1) / parts);
+  const int pc = c_hi - c_lo, total = nitems * pc;
+  pdl_launch_dependents();
+  // (nothing is read before the wait: a kernel launched early may run beside an
+  // earlier kernel of the stream that is still writing x)
+  pdl_wait();
+  int4 pre[RS_PRE];  // the row chunks, loaded together with the tables below
+#pragma unroll
+  for (int u = 0; u < RS_PRE; ++u) {
+    const int j = tid + u * RS_THREADS;
+    if (j < total) {
+      const int i = j / pc, cc = c_lo + (j - i * pc);
+      pre[u] = x[((q0 + i) / k) * chunks + cc];
+    }
+  }
+  if (tid == 0) prior_s = *reinterpret_cast<volatile int*>(status);
+  // 1. per (group g, expert e): tasks of e in tiles g, g + G, ..., all and before this tile
+  const int G = RS_THREADS / m;  // >= 2 for m <= 256
+  int pt = 0, pb = 0;
+  if (tid < G * m) {
+    const int g = tid / m, e = tid - g * m;
+    for (int tl0 = g; tl0 < ntiles; tl0 += 16 * G) {
+      int v[16];
+#pragma unroll
+      for (int u = 0; u < 16; ++u) {
+        const int tl = tl0 + u * G;
+        v[u] = tl < ntiles ? tile_cnt[(long long)tl * m + e] : 0;
+      }
+#pragma unroll
+      for (int u = 0; u < 16; ++u) {
+        pt += v[u];
+        pb += tl0 + u * G < tile ? v[u] : 0;
+      }
+    }
+  }
+  int ie[2], ir[2];  // this tile's tasks (at most 128 k <= 2 per thread)
+#pragma unroll
+  for (int u = 0; u < 2; ++u) {
+    const int i = tid + u * RS_THREADS;
+    ie[u] = i < nitems ? idx[q0 + i] : -1;
+    ir[u] = i < nitems ? lrank[q0 + i] : 0;
+  }
+  if (tid < G * m) {
+    part_t[tid] = pt;
+    part_b[tid] = pb;
+  }
+  __syncthreads();
+  if (prior_s != 0) return;  // an earlier kernel flagged an error (uniform: read once)
+  // 2. totals, exclusive scan over experts, this tile's bases; LIS in block (0, 0)
+  int n = 0, b = 0;
+  if (tid < m)
+    for (int g = 0; g < G; ++g) {
+      n += part_t[g * m + tid];
+      b += part_b[g * m + tid];
+    }
+  int incl = n;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int v = __shfl_up_sync(FULL, incl, o);
+    if (lane >= o) incl += v;
+  }
+  int mv = tid < m ? n : -1, ma = tid;
+#pragma unroll
+  for (int o = 16; o; o >>= 1) {
+    const int ov = __shfl_xor_sync(FULL, mv, o), oa = __shfl_xor_sync(FULL, ma, o);
+    if (ov > mv || (ov == mv && oa < ma)) {
+      mv = ov;
+      ma = oa;
+    }
+  }
+  if (lane == 31) wsum[warp] = incl;
+  if (lane == 0) {
+    wmax[warp] = mv;
+    warg[warp] = ma;
+  }
+  __syncthreads();
+  if (warp == 0) {
+    const int nw = RS_THREADS / 32;
+    const int ws = lane < nw ? wsum[lane] : 0;
+    int wi = ws;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int v = __shfl_up_sync(FULL, wi, o);
+      if (lane >= o) wi += v;
+    }
+    if (lane < nw) wsum[lane] = wi - ws;
+    int bv = lane < nw ? wmax[lane] : -1, ba = lane < nw ? warg[lane] : 0x7fffffff;
+#pragma unroll
+    for (int o = 16; o; o >>= 1) {
+      const int ov = __shfl_xor_sync(FULL, bv, o), oa = __shfl_xor_sync(FULL, ba, o);
+      if (ov > bv || (ov == bv && oa < ba)) {
+        bv = ov;
+        ba = oa;
+      }
+    }
+    if (lane == 0) {
+      wmax[0] = bv;
+      warg[0] = ba;
+    }
+  }
+  __syncthreads();
+  if (tid < m) {
+    const int ex = incl - n + wsum[warp];
+    tot[tid] = n;
+    off[tid] = ex;
+    base[tid] = ex + b;
+    if (tid == m - 1) off[m] = ex + n;
+    if (tile == 0 && part == 0) {
+      counts[tid] = n;
+      offsets[tid] = ex;
+      if (tid == m - 1) offsets[m] = ex + n;
+    }
+  }
+  if (tile == 0 && part == 0 && tid == 0 && lis) {
+    lis->max_count = wmax[0];
+    lis->argmax_expert = warg[0];
+    lis->lis = (double)((long long)m * wmax[0]) / (double)((long long)T * k);
+  }
+  __syncthreads();
+  // 3. this tile's tasks
+#pragma unroll
+  for (int u = 0; u < 2; ++u) {
+    const int i = tid + u * RS_THREADS;
+    if (i >= nitems) continue;
+    const long long q = q0 + i;
+    const int e = ie[u];
+    int d = -1;
+    if (e >= 0 && e < m) {
+      d = base[e] + ir[u];
+      if (d < off[e] || d >= off[e] + tot[e]) d = -1;
+    }
+    if (d < 0) set_status(status, MOE_ERR_DEVICE_INDEX);
+    dest[i] = d;
+    if (part == 0) {
+      inv_perm[q] = d;
+      if (d >= 0) {
+        perm[d] = (int32_t)q;
+        if (w_perm) w_perm[d] = task_w[q];
+      }
+    }
+  }
+  __syncthreads();
+  // 4. rows: x_perm[dest, c] = x[q / k, c] for this part's columns
+#pragma unroll
+  for (int u = 0; u < RS_PRE; ++u) {
+    const int j = tid + u * RS_THREADS;
+    if (j < total) {
+      const int i = j / pc, cc = c_lo + (j - i * pc);
+      const int d = dest[i];
+      if (d >= 0) x_perm[(long long)d * chunks + cc] = pre[u];
+    }
+  }
+  for (int j0 = tid + RS_PRE * RS_THREADS; j0 < total; j0 += RS_PRE * RS_THREADS) {  // beyond the first batch
+    int4 v[RS_PRE];
+    long long o[RS_PRE];
+#pragma unroll
+    for (int u = 0; u < RS_PRE; ++u) {
+      const int j = j0 + u * RS_THREADS;
+      o[u] = -1;
+      if (j < total) {
+        const int i = j / pc, cc = c_lo + (j - i * pc);
+        const int d = dest[i];
+        if (d >= 0) {
+          v[u] = x[((q0 + i) / k) * chunks + cc];
+          o[u] = (long long)d * chunks + cc;
+        }
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < RS_PRE; ++u)
+      if (o[u] >= 0) x_perm[o[u]] = v[u];
+  }
+}
+
+cudaError_t launch_route_scatter(int dtype, int T, int k, int m, int d, const int32_t* tile_cnt, const int32_t* idx,
+                                 const int32_t* lrank, const float* task_w, const void* x, int32_t* counts,
+                                 int32_t* offsets, moe_lis_t* lis, int32_t* perm, int32_t* inv_perm, float* w_perm,
+                                 void* x_perm, int* status, cudaStream_t s) {
+  const int ntiles = (T + 127) / 128;
+  const int chunks = d * (dtype == MOE_F32 ? 4 : 2) / 16;
+  // about one wave of blocks (one 512-thread block fits an SM's registers); the
+  // rows beyond a block's first batch of loads go through the unrolled loop
+  const int parts = std::max(1, std::min({(num_sms() + ntiles / 2) / ntiles, chunks, 65535}));
+  launch_k(route_scatter_kernel, dim3(ntiles, parts), RS_THREADS, 0, s, T, k, m, ntiles, parts, chunks, tile_cnt, idx,
+           lrank, task_w, (const int4*)x, counts, offsets, lis, perm, inv_perm, w_perm, (int4*)x_perm, status);
+  count_launch();
+  return cudaGetLastError();
+}
+
 // ------------------------------------------------------------------ combine
 // out[t, c] = sum_s sum_split y[split][inv_perm[t k + s], c]
 //           + sum_sh sum_split ysh[split][sh T + t, c], fp32, slot order; 4 columns

@@ -25,6 +25,7 @@
 // records MOE_ERR_TIMEOUT in the status word, the other roles stop, outstanding
 // TMA copies and MMAs are drained (again with a bound) and TMEM is freed.
 #include <algorithm>
+#include <cstring>
 #include <cstdio>
 
 #include "common.cuh"
@@ -124,6 +125,94 @@ __device__ __forceinline__ uint32_t idesc_bf16(int M, int N) {
   return (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
 }
 
+// Barrier of the four epilogue warps only (named barrier 1; 0 is __syncthreads),
+// in its non-aligned form and after reconverging the warp, so lanes that took
+// different branches before it are all counted.
+__device__ __forceinline__ void epi_bar() {
+  __syncwarp();
+  asm volatile("barrier.sync 1, 128;" ::: "memory");
+}
+
+// One pass of the router epilogue over a token's m logits (TMEM columns, 32 per
+// step): the largest logit strictly after (pv, pe) in the order (logit desc,
+// expert asc), by a pairwise tree whose left side always holds the lower experts.
+// With EXP it also writes the logits (lg, when given) and folds the softmax
+// denominator: per 32 columns a pairwise fp32 sum of exp(logit - running max),
+// added to an fp64 sum rescaled whenever the running maximum grows.
+template <bool EXP>
+__device__ __forceinline__ void route_pass(uint32_t t_row, int m, const float* rbias, float pv, int pe, float& bv,
+                                           int& be, float& mrun, double& z, float* lg) {
+  bv = -INFINITY;
+  be = -1;
+#pragma unroll 1
+  for (int c0 = 0; c0 < m; c0 += 32) {
+    uint32_t r[32];
+    tmem_ld_x16(t_row + c0, r);
+    if (c0 + 16 < m) {
+      tmem_ld_x16(t_row + c0 + 16, r + 16);
+    } else {
+#pragma unroll
+      for (int j = 16; j < 32; ++j) r[j] = 0u;
+    }
+    float v[32];
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {  // c0 + 32 <= ROUTE_MAX_M
+      const float4 bb = reinterpret_cast<const float4*>(rbias + c0)[u];
+      v[4 * u] = bb.x;
+      v[4 * u + 1] = bb.y;
+      v[4 * u + 2] = bb.z;
+      v[4 * u + 3] = bb.w;
+    }
+    tmem_ld_wait();
+#pragma unroll
+    for (int j = 0; j < 32; ++j) v[j] = c0 + j < m ? __uint_as_float(r[j]) + v[j] : -INFINITY;
+    if (EXP && lg)
+#pragma unroll
+      for (int j = 0; j < 32; ++j)
+        if (c0 + j < m) lg[c0 + j] = v[j];
+    float cv[32];
+    int ce[32];
+#pragma unroll
+    for (int j = 0; j < 32; ++j) {
+      const bool after = v[j] < pv || (v[j] == pv && c0 + j > pe);
+      cv[j] = after ? v[j] : -INFINITY;
+      ce[j] = c0 + j;
+    }
+#pragma unroll
+    for (int st = 1; st < 32; st <<= 1)
+#pragma unroll
+      for (int j = 0; j < 32; j += 2 * st)
+        if (cv[j + st] > cv[j]) {  // an equal logit keeps the lower expert (left)
+          cv[j] = cv[j + st];
+          ce[j] = ce[j + st];
+        }
+    if (cv[0] > bv) {  // earlier steps hold lower experts
+      bv = cv[0];
+      be = ce[0];
+    }
+    if (EXP) {
+      float mxs[32];
+#pragma unroll
+      for (int j = 0; j < 32; ++j) mxs[j] = v[j];
+#pragma unroll
+      for (int st = 1; st < 32; st <<= 1)
+#pragma unroll
+        for (int j = 0; j < 32; j += 2 * st) mxs[j] = fmaxf(mxs[j], mxs[j + st]);
+      if (mxs[0] > mrun) {
+        z *= (double)expf(mrun - mxs[0]);
+        mrun = mxs[0];
+      }
+#pragma unroll
+      for (int j = 0; j < 32; ++j) mxs[j] = c0 + j < m ? expf(v[j] - mrun) : 0.f;
+#pragma unroll
+      for (int st = 1; st < 32; st <<= 1)
+#pragma unroll
+        for (int j = 0; j < 32; j += 2 * st) mxs[j] += mxs[j + st];
+      z += (double)mxs[0];
+    }
+  }
+}
+
 // ------------------------------------------------------------------ tile schedule
 struct TileInfo {
   int cls, g, mt, ks, nt, rows_in_tile, b_row, out_row, a_row, kb0, kb1;
@@ -220,8 +309,11 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
   __shared__ __align__(8) uint64_t full_bar[STAGES], empty_bar[STAGES], accf_bar[2], acce_bar[2], drain_bar;
   __shared__ float aux_w[4][EPI == EPI_DOWN ? BN : 1];  // per epilogue warp: row weights of the tile
   __shared__ int aux_d[4][EPI == EPI_DOWN ? BN : 1];    // and destination tokens (fused top-1 combine)
+  constexpr int RMASK_M = EPI == EPI_ROUTE ? ROUTE_MAX_M : 1;
+  __shared__ __align__(16) float rbias[RMASK_M];  // ROUTE: router bias (zeros when absent)
+  __shared__ uint32_t rmask[EPI == EPI_ROUTE ? 2 : 1][4][RMASK_M];  // ROUTE: expert -> lanes holding it
   __shared__ uint32_t tmem_base_s;
-  __shared__ int abort_s;
+  __shared__ int abort_s, epi_fail_s;
   __shared__ int total_tiles_s;
   extern __shared__ uint8_t dyn_smem[];
 
@@ -243,6 +335,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
     }
     mbar_init(&drain_bar, 1);
     abort_s = 0;
+    epi_fail_s = 0;
     fence_mbar_init();
     tma_prefetch_desc(&tA0_0);
     tma_prefetch_desc(&tB_0);
@@ -298,6 +391,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
     const int prior = p.status ? *reinterpret_cast<volatile int*>(p.status) : 0;
     if (lane == 31) total_tiles_s = prior ? 0 : incl;
   }
+  __syncwarp();
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -402,6 +496,120 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
     umma_commit(&drain_bar);
     const volatile int never = 0;
     if (!mbar_wait(&drain_bar, 0, TC_DRAIN_LIMIT_NS, &never)) set_status(p.status, MOE_ERR_TIMEOUT);
+  } else if (EPI == EPI_ROUTE && warp >= 2) {
+    // ---------------------------------------------------------------- router epilogue
+    // TMEM lane = token (quarter q of the 128-token tile), column = expert. Every
+    // epilogue warp reaches every epilogue barrier of every tile; a failed wait is
+    // published through epi_fail_s before the barrier, so all four leave together.
+    const int q = warp & 3;
+    const int et = (warp - 2) * 32 + lane;  // 0..127
+    {
+      const GemmClass& c = p.cls[0];
+      for (int e = et; e < ROUTE_MAX_M; e += 128) rbias[e] = (c.bias && e < c.const_rows) ? c.bias[e] : 0.f;
+      epi_bar();
+    }
+    int acc = 0, iter = 0;
+    uint32_t acc_phase = 0;
+    for (int w = blockIdx.x; w < total; w += gridDim.x, ++iter) {
+      TileInfo ti;
+      decode_tile<BN>(p, sched, G, w, ti);
+      const GemmClass& c = p.cls[0];
+      const int t = ti.mt * TC_BM + q * 32 + lane;  // token
+      const bool tv_ok = t < c.R;
+      const int m = ti.rows_in_tile, k = c.k_sel;
+      const bool got = mbar_wait(&accf_bar[acc], acc_phase, lim, abort_flag);
+      if (!got) {
+        set_status(p.status, MOE_ERR_TIMEOUT);
+        abort_s = 1;
+        epi_fail_s = 1;
+      }
+      epi_bar();
+      if (epi_fail_s) break;
+      tc_fence_after();
+      const uint32_t t_row = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * S::ACC_COLS);
+      // Pass s picks the largest logit strictly after pick s - 1 in the order
+      // (logit desc, expert asc), reading the accumulator again from TMEM; pass 0
+      // also writes the logits (when asked) and the softmax denominator. Each pass
+      // stores its expert and, for now, its logit in the outputs.
+      float mrun = -INFINITY, mx = -INFINITY;
+      double z = 0.0;
+      float* lg = c.out && tv_ok ? reinterpret_cast<float*>(c.out) + (long long)t * m : nullptr;
+      int32_t* oi = c.sel_idx + (long long)t * k;
+      float* ow = c.sel_w + (long long)t * k;
+      float pv = INFINITY;
+      int pe = -1;
+      bool bad = false;
+#pragma unroll 1
+      for (int s2 = 0; s2 < k; ++s2) {
+        float bv;
+        int be;
+        if (s2 == 0) {
+          route_pass<true>(t_row, m, rbias, pv, pe, bv, be, mrun, z, lg);
+          mx = bv;
+          z *= (double)expf(mrun - mx);  // the running maximum is the top logit
+        } else {
+          float dm = 0.f;
+          double dz = 0.0;
+          route_pass<false>(t_row, m, rbias, pv, pe, bv, be, dm, dz, nullptr);
+        }
+        if (tv_ok) {
+          oi[s2] = be;
+          ow[s2] = bv;
+        }
+        bad |= be < 0;  // NaN logits
+        pv = bv;
+        pe = be;
+      }
+      // the accumulator is free for the next tile's MMAs
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&acce_bar[acc]);
+      if (++acc == S::NUM_ACC) {
+        acc = 0;
+        acc_phase ^= 1u;
+      }
+      if (tv_ok) {  // gate weights: softmax over all m, renormalised over the k chosen when asked
+        double sel = 0.0;
+#pragma unroll 1
+        for (int s2 = 0; s2 < k; ++s2) sel += (double)expf(ow[s2] - mx) / z;
+#pragma unroll 1
+        for (int s2 = 0; s2 < k; ++s2) {
+          double pr = (double)expf(ow[s2] - mx) / z;
+          if (c.renorm) pr /= sel;
+          ow[s2] = (float)pr;
+        }
+        if (bad) set_status(p.status, MOE_ERR_DEVICE_INDEX);
+      }
+      if (c.lrank) {
+        // rank of each task among the tile's tasks of its expert, in (token, slot)
+        // order: lanes below in this quarter plus all tasks of the quarters before
+        uint32_t(*mk)[RMASK_M] = rmask[EPI == EPI_ROUTE ? (iter & 1) : 0];
+        for (int e = lane; e < m; e += 32) mk[q][e] = 0u;
+        __syncwarp();
+        if (tv_ok)
+#pragma unroll 1
+          for (int s2 = 0; s2 < k; ++s2) {
+            const int e = oi[s2];
+            if (e >= 0) atomicOr(&mk[q][e], 1u << lane);
+          }
+        epi_bar();
+        if (tv_ok)
+#pragma unroll 1
+          for (int s2 = 0; s2 < k; ++s2) {
+            const int e = oi[s2];
+            if (e < 0) continue;
+            int rk = __popc(mk[q][e] & ((1u << lane) - 1u));
+            for (int q2 = 0; q2 < q; ++q2) rk += __popc(mk[q2][e]);
+            c.lrank[(long long)t * k + s2] = rk;
+          }
+        for (int e = et; e < m; e += 128)
+          c.tile_cnt[(long long)ti.mt * m + e] =
+              __popc(mk[0][e]) + __popc(mk[1][e]) + __popc(mk[2][e]) + __popc(mk[3][e]);
+        // (the masks are double-buffered: the next tile writes the other set, and the
+        // one after that passes an epilogue barrier every warp reaches only after
+        // finishing the reads above)
+      }
+    }
   } else if (warp >= 2) {
     // ---------------------------------------------------------------- epilogue
     const int q = warp & 3;  // TMEM lane quarter this warp may access
@@ -459,6 +667,10 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
       }
     }
   }
+  // Warps 0 and 1 ran their roles on lane 0 alone: reconverge each warp before the
+  // block barrier (an aligned barrier reached by part of a warp does not wait for
+  // the rest of the block), so TMEM is freed only after every epilogue read.
+  __syncwarp();
   tc_fence_before();
   __syncthreads();
   if (warp == 1) {
@@ -556,8 +768,48 @@ cudaError_t launch_tc_gemm(int epi, int bn, const TcMaps& maps, const GemmParams
   MOE_TC_CASE(EPI_DOWN, 1, 64)
   MOE_TC_CASE(EPI_DOWN, 1, 128)
   MOE_TC_CASE(EPI_DOWN, 1, 256)
+  MOE_TC_CASE(EPI_ROUTE, 1, 16)
+  MOE_TC_CASE(EPI_ROUTE, 1, 32)
+  MOE_TC_CASE(EPI_ROUTE, 1, 64)
+  MOE_TC_CASE(EPI_ROUTE, 1, 128)
+  MOE_TC_CASE(EPI_ROUTE, 1, 256)
 #undef MOE_TC_CASE
   return cudaErrorInvalidValue;
+}
+
+cudaError_t launch_route_topk(const moe_config_t& c, const void* x, const void* w_r, const float* bias, float* logits,
+                              int32_t* idx, float* w, int32_t* lrank, int32_t* tile_cnt, int* status,
+                              unsigned long long wait_limit_ns, cudaStream_t s) {
+  GemmParams p;
+  std::memset(&p, 0, sizeof(p));
+  GemmClass& g = p.cls[0];
+  g.n_groups = 1;
+  g.R = c.T;  // A = x: tokens are the MMA's rows
+  g.K = c.d;
+  g.ksplit = 1;
+  g.kb_per_split = (c.d + TC_BK - 1) / TC_BK;
+  g.const_rows = c.m;  // B = W_r: every expert in one N tile
+  g.out = logits;
+  g.out_ld = c.m;
+  g.bias = bias;
+  g.k_sel = c.k;
+  g.renorm = c.renormalize;
+  g.sel_idx = idx;
+  g.sel_w = w;
+  g.lrank = lrank;
+  g.tile_cnt = tile_cnt;
+  p.n_classes = 1;
+  p.status = status;
+  p.wait_limit_ns = wait_limit_ns;
+  int bn = 16;
+  while (bn < c.m) bn <<= 1;
+  TcMaps maps;
+  std::memset(&maps, 0, sizeof(maps));
+  maps.a0[0] = {x, c.T, c.d};
+  maps.a1[0] = maps.a0[0];
+  maps.b[0] = {w_r, c.m, c.d};
+  const int tiles = (c.T + TC_BM - 1) / TC_BM;
+  return launch_tc_gemm(EPI_ROUTE, bn, maps, p, std::min(tiles, num_sms()), s);
 }
 
 }  // namespace moe

@@ -41,6 +41,7 @@ ROUTE_CASES = [
     W.small_moe(T=33, d=64, f=64, m=8, k=2, dtype=W.BF16, zipf_s=0.8, renorm=True, index=83),
     W.small_moe(T=5, d=72, f=64, m=200, k=7, dtype=W.BF16, zipf_s=1.0, index=84),
     W.small_moe(T=1, d=4096, f=64, m=8, k=2, dtype=W.BF16, zipf_s=0.0, index=85),
+    W.small_moe(T=600, d=136, f=64, m=200, k=8, dtype=W.BF16, zipf_s=0.7, renorm=True, index=89),
 ]
 
 
@@ -54,6 +55,21 @@ def test_route_topk_bit_exact_on_gpu_logits(cfg):
     oidx, ow = O.topk_softmax(lg, cfg.k, cfg.renorm)  # oracle decides on the GPU's own logits
     np.testing.assert_array_equal(idx, oidx)
     np.testing.assert_allclose(w, ow, rtol=GATE_RTOL, atol=1e-12)
+
+
+def test_route_without_logits_output_selects_the_same():
+    # the tensor-core router writes logits only when asked; the selection must not change
+    cfg = W.small_moe(T=600, d=136, f=64, m=200, k=8, dtype=W.BF16, zipf_s=0.7, renorm=True, index=89)
+    d_in = device_inputs(W.make_moe_inputs(cfg, weights=False))
+    _, idx, w = _route(cfg, d_in)
+    c = config_of(cfg)
+    ws = moe.workspace(c)
+    idx2 = torch.empty((cfg.T, cfg.k), dtype=torch.int32, device="cuda")
+    w2 = torch.empty((cfg.T, cfg.k), dtype=torch.float32, device="cuda")
+    moe.moe_route(c, d_in["x"], d_in["w_router"], d_in["bias"], None, None, idx2, w2, ws)
+    assert moe.moe_read_device_status(ws) == moe.OK
+    np.testing.assert_array_equal(host(idx2), idx)
+    np.testing.assert_array_equal(host(w2), w)
 
 
 def test_route_logits_in_verbatim_with_ties():

@@ -82,7 +82,8 @@ def test_decode_all_tokens():
     _check_layer(cfg, W.make_moe_inputs(cfg), n_sample=cfg.T)
 
 
-@pytest.mark.parametrize("case", ["one_hot", "T1", "ragged_small", "relu_many_experts", "max_experts_max_k"])
+@pytest.mark.parametrize("case", ["one_hot", "T1", "ragged_small", "relu_many_experts", "max_experts_max_k",
+                                  "routed_k8_m200"])
 def test_layer_edge_cases(case):
     if case == "one_hot":  # every token's top-1 is the same expert (huge bias)
         cfg = W.small_moe(T=300, d=256, f=192, m=16, k=2, dtype=W.BF16, zipf_s=0.0, index=72)
@@ -98,6 +99,9 @@ def test_layer_edge_cases(case):
         inp = W.make_moe_inputs(cfg)
     elif case == "relu_many_experts":
         cfg = W.small_moe(T=1500, d=128, f=320, m=256, k=2, act=W.RELU, dtype=W.BF16, zipf_s=1.0, index=75)
+        inp = W.make_moe_inputs(cfg)
+    elif case == "routed_k8_m200":  # largest k of the tensor-core router, m not a power of two, 5 ragged tiles
+        cfg = W.small_moe(T=513, d=136, f=96, m=200, k=8, dtype=W.BF16, zipf_s=0.7, renorm=True, index=78)
         inp = W.make_moe_inputs(cfg)
     else:  # the largest expert count and top-k the library accepts (m = 1024, k = 32)
         cfg = W.small_moe(T=700, d=64, f=64, m=1024, k=32, dtype=W.BF16, zipf_s=0.5, index=77)
