@@ -55,6 +55,9 @@ def parse():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--cpu-seconds", type=float, default=12.0, help="CPU-oracle baseline budget (rank 0, N=1)")
     ap.add_argument("--no-cpu-baseline", action="store_true", help="skip the CPU-oracle leg (for profiling runs)")
+    ap.add_argument("--router-only", action="store_true",
+                    help="time the routing call alone (moe_route / moe_atomic_route) on the workload's inputs; "
+                         "an auxiliary line for profiling, not the layer metric")
     return ap.parse_args()
 
 
@@ -274,6 +277,13 @@ class ClockSampler:
 
 # ------------------------------------------------------------------ algorithmic cost model
 
+def fused_routing(cfg) -> bool:
+    """The library's rule for its one-launch router (logits + top-k + tile ranks in the
+    tensor-core epilogue) followed by the one-kernel scatter: bf16, 8192+ tokens,
+    m <= 256, k <= 8."""
+    return cfg.dtype == W.BF16 and cfg.T >= 8192 and cfg.m <= 256 and cfg.k <= 8
+
+
 def stage_costs(cfg, active: int, ksplit: int):
     """Algorithmic flops and bytes per launch of each stage (operands read once,
     results written once; weights of ACTIVE experts only)."""
@@ -287,6 +297,11 @@ def stage_costs(cfg, active: int, ksplit: int):
     c["topk"] = (0.0, T * m * 4 + Tk * 8)
     c["histogram_lis_ranks"] = (0.0, Tk * 4 + Tk * 8 + (m + 1) * 8)
     c["permute"] = (0.0, Tk * 4 + T * d * es + Tk * d * es)
+    tiles = (T + 127) // 128
+    # fused routing: x and W_r in, ids, weights, tile ranks and tile counts out; then the
+    # scatter reads those back and writes perm / inv_perm / w_perm, counts, offsets and x_perm
+    c["router_topk_ranks"] = (2.0 * T * d * m, T * d * es + m * d * es + Tk * 12 + tiles * m * 4)
+    c["scatter"] = (0.0, tiles * m * 4 + Tk * 12 + Tk * 12 + (2 * m + 1) * 4 + T * d * es + Tk * d * es)
     c["expert_up"] = (2.0 * mats * f * d * Tk + 2.0 * mats * fsh * d * T * nsh,
                       active * mats * f * d * es + nsh * mats * fsh * d * es + Tk * d * es + (T * d * es if nsh else 0)
                       + Tk * f * es + nsh * T * fsh * es)
@@ -400,6 +415,11 @@ def ours(args):
                 for j, name in enumerate(STAGES)}
     dom = max(STAGES, key=lambda n: stage_ms[n])
     jd = STAGES.index(dom)
+    if fused_routing(cfg):
+        # one kernel spans stages 0-1 and one spans 3-4; the two boundaries between them coincide
+        stage_ms = {("router_topk_ranks" if n == "router" else "scatter" if n == "permute" else n): v
+                    for n, v in stage_ms.items() if n not in ("topk", "histogram_lis_ranks")}
+        dom = {"router": "router_topk_ranks", "permute": "scatter"}.get(dom, dom)
 
     # ---- timed region: K steps, CUDA events on the launching stream, L2 flushed between steps
     K = args.steps
@@ -689,9 +709,70 @@ def ours_atomic(args):
     return 0
 
 
+def router_only(args):
+    """The routing call alone: K steps after W warm-ups, L2 flush between steps outside the events."""
+    import torch
+
+    import sparse_mixture_experts_08_b200 as moe
+
+    cfg = W.CONFIGS[args.config]
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    s = torch.cuda.Stream(device=dev)
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    bf = lambda a: torch.from_numpy(a.view(np.int16)).to(dev).view(torch.bfloat16)
+    if isinstance(cfg, W.AtomicWorkload):
+        inp = W.make_atomic_inputs(cfg, experts=False)
+        c = moe.make_atomic_config(cfg.T, cfg.d, cfg.Nr, cfg.Nc, cfg.K, cfg.act)
+        x, wr, wc = bf(inp["x"]), bf(inp["w_row"]), bf(inp["w_col"])
+        idx = torch.empty((cfg.T, cfg.K), dtype=torch.int32, device=dev)
+        g = torch.empty((cfg.T, cfg.K), dtype=torch.float32, device=dev)
+        ws = moe.workspace(c, device=dev)
+
+        def call():
+            moe.moe_atomic_route(c, x, wr, wc, None, None, idx, g, ws, stream=s)
+    else:
+        inp = W.make_moe_inputs(cfg, weights=False)
+        c = moe.make_config(cfg.T, cfg.d, cfg.f, cfg.m, cfg.k, cfg.n_shared, cfg.f_shared, cfg.dtype, cfg.act,
+                            cfg.renorm)
+        conv = bf if cfg.dtype == W.BF16 else (lambda a: torch.from_numpy(a).to(dev))
+        x, wr = conv(inp["x"]), conv(inp["w_router"])
+        bias = None if inp.get("bias") is None else torch.from_numpy(inp["bias"]).to(dev)
+        idx = torch.empty((cfg.T, cfg.k), dtype=torch.int32, device=dev)
+        w = torch.empty((cfg.T, cfg.k), dtype=torch.float32, device=dev)
+        ws = moe.workspace(c, device=dev)
+
+        def call():
+            moe.moe_route(c, x, wr, bias, None, None, idx, w, ws, stream=s)
+    with torch.cuda.stream(s):
+        n0 = moe.moe_launch_count()
+        call()
+        launches = moe.moe_launch_count() - n0
+        for _ in range(max(args.warmup, 3)):
+            flush.zero_()
+            call()
+    torch.cuda.synchronize(dev)
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    with torch.cuda.stream(s):
+        for a, b in ev:
+            flush.zero_()
+            a.record(s)
+            call()
+            b.record(s)
+    torch.cuda.synchronize(dev)
+    if moe.moe_read_device_status(ws, stream=s) != moe.OK:
+        raise RuntimeError("device status after the router runs is not OK")
+    ms = sum(a.elapsed_time(b) for a, b in ev) / len(ev)
+    print(json.dumps({"mode": "router-only", "config": {"workload": cfg.name}, "ms_per_step": ms,
+                      "tokens_per_s": cfg.T / (ms * 1e-3), "gpu_launches_per_step": launches}), flush=True)
+    return 0
+
+
 def main():
     args = parse()
     atomic = isinstance(W.CONFIGS[args.config], W.AtomicWorkload)
+    if args.router_only:
+        return router_only(args)
     if args.impl == "reference":
         if atomic:
             raise SystemExit("--impl reference covers the coarse-expert workloads")

@@ -41,7 +41,8 @@ ROUTE_CASES = [
     W.small_moe(T=33, d=64, f=64, m=8, k=2, dtype=W.BF16, zipf_s=0.8, renorm=True, index=83),
     W.small_moe(T=5, d=72, f=64, m=200, k=7, dtype=W.BF16, zipf_s=1.0, index=84),
     W.small_moe(T=1, d=4096, f=64, m=8, k=2, dtype=W.BF16, zipf_s=0.0, index=85),
-    W.small_moe(T=600, d=136, f=64, m=200, k=8, dtype=W.BF16, zipf_s=0.7, renorm=True, index=89),
+    W.small_moe(T=8269, d=72, f=64, m=200, k=8, dtype=W.BF16, zipf_s=0.7, renorm=True, index=89),
+    W.small_moe(T=8192, d=64, f=64, m=256, k=2, dtype=W.BF16, zipf_s=1.0, index=90),
 ]
 
 
@@ -58,8 +59,9 @@ def test_route_topk_bit_exact_on_gpu_logits(cfg):
 
 
 def test_route_without_logits_output_selects_the_same():
-    # the tensor-core router writes logits only when asked; the selection must not change
-    cfg = W.small_moe(T=600, d=136, f=64, m=200, k=8, dtype=W.BF16, zipf_s=0.7, renorm=True, index=89)
+    # the fused tensor-core router (8192+ tokens) writes logits only when asked; the
+    # selection must not change
+    cfg = W.small_moe(T=8269, d=72, f=64, m=200, k=8, dtype=W.BF16, zipf_s=0.7, renorm=True, index=89)
     d_in = device_inputs(W.make_moe_inputs(cfg, weights=False))
     _, idx, w = _route(cfg, d_in)
     c = config_of(cfg)

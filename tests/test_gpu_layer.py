@@ -82,11 +82,12 @@ def test_decode_all_tokens():
     _check_layer(cfg, W.make_moe_inputs(cfg), n_sample=cfg.T)
 
 
-@pytest.mark.parametrize("case", ["one_hot", "T1", "ragged_small", "relu_many_experts", "max_experts_max_k",
-                                  "routed_k8_m200"])
+@pytest.mark.parametrize("case", ["one_hot", "one_hot_fused", "T1", "ragged_small", "relu_many_experts",
+                                  "max_experts_max_k", "routed_k8_m200"])
 def test_layer_edge_cases(case):
-    if case == "one_hot":  # every token's top-1 is the same expert (huge bias)
-        cfg = W.small_moe(T=300, d=256, f=192, m=16, k=2, dtype=W.BF16, zipf_s=0.0, index=72)
+    if case in ("one_hot", "one_hot_fused"):  # every token's top-1 is the same expert (huge bias)
+        T = 300 if case == "one_hot" else 8192  # 8192: the fused router and scatter
+        cfg = W.small_moe(T=T, d=256, f=192, m=16, k=2, dtype=W.BF16, zipf_s=0.0, index=72)
         inp = W.make_moe_inputs(cfg)
         inp["bias"][:] = 0.0
         inp["bias"][11] = 1000.0
@@ -100,14 +101,14 @@ def test_layer_edge_cases(case):
     elif case == "relu_many_experts":
         cfg = W.small_moe(T=1500, d=128, f=320, m=256, k=2, act=W.RELU, dtype=W.BF16, zipf_s=1.0, index=75)
         inp = W.make_moe_inputs(cfg)
-    elif case == "routed_k8_m200":  # largest k of the tensor-core router, m not a power of two, 5 ragged tiles
-        cfg = W.small_moe(T=513, d=136, f=96, m=200, k=8, dtype=W.BF16, zipf_s=0.7, renorm=True, index=78)
+    elif case == "routed_k8_m200":  # fused router (8192+ tokens): largest k, m not a power of two, ragged tile
+        cfg = W.small_moe(T=8269, d=64, f=64, m=200, k=8, dtype=W.BF16, zipf_s=0.7, renorm=True, index=78)
         inp = W.make_moe_inputs(cfg)
     else:  # the largest expert count and top-k the library accepts (m = 1024, k = 32)
         cfg = W.small_moe(T=700, d=64, f=64, m=1024, k=32, dtype=W.BF16, zipf_s=0.5, index=77)
         inp = W.make_moe_inputs(cfg)
     ref, _ = _check_layer(cfg, inp, n_sample=min(cfg.T, 64))
-    if case == "one_hot":  # expert 11 holds every token: LIS reaches its maximum m / k
+    if case.startswith("one_hot"):  # expert 11 holds every token: LIS reaches its maximum m / k
         assert ref["counts"][11] == cfg.T and ref["lis"] == cfg.m / cfg.k
 
 
