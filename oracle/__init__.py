@@ -54,6 +54,7 @@ def _L():
             "oracle_topk_softmax": [i, i, i, i, _P, _P, _P],
             "oracle_histogram_lis": [i, i, i, _P, _P, _P, _P, _P, _P],
             "oracle_permutation": [i, i, i, _P, _P, _P, _P],
+            "oracle_replica_split": [i, i, i, _P, _P, _P],
             "oracle_expert_ffn": [i, i, i, i, _P, _P, _P, _P, _P],
             "oracle_moe_output": [_P, _P, i, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, i],
             "oracle_layer_forward": [_P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P,
@@ -143,6 +144,27 @@ def permutation(idx: np.ndarray, m: int, offsets: np.ndarray):
     _check(_L().oracle_permutation(T, k, m, _ptr(idx), _ptr(np.ascontiguousarray(offsets, np.int32)),
                                    _ptr(perm), _ptr(inv)), "permutation")
     return perm, inv
+
+
+def replica_split(idx: np.ndarray, m: int):
+    """R&Q replica dispatch: (routing over m + 1 experts, heavy-hitter h). Every
+    second task of h, in task order, goes to the replica expert m."""
+    idx = np.ascontiguousarray(idx, dtype=np.int32)
+    T, k = idx.shape
+    out = np.empty_like(idx)
+    h = np.zeros(1, np.int32)
+    _check(_L().oracle_replica_split(T, k, m, _ptr(idx), _ptr(out), _ptr(h)), "replica_split")
+    return out, int(h[0])
+
+
+def replica_inputs(inp: Dict[str, np.ndarray], heavy: int) -> Dict[str, np.ndarray]:
+    """The layer's inputs with expert m appended as a copy of the heavy-hitter's
+    weights (R&Q Algorithm 3 appends quant(layer[h]); unquantised here)."""
+    out = dict(inp)
+    for key in ("w_gate", "w_up", "w_down"):
+        if inp.get(key) is not None:
+            out[key] = np.ascontiguousarray(np.concatenate([inp[key], inp[key][heavy:heavy + 1]], axis=0))
+    return out
 
 
 # ------------------------------------------------------------------------- experts

@@ -159,6 +159,42 @@ int oracle_permutation(int T, int k, int m, const int32_t* idx, const int32_t* o
   return 0;
 }
 
+/* Replica dispatch (R&Q, "A Replicate-and-Quantize Strategy for Plug-and-Play
+ * Load Balancing of Sparse Mixture-of-Experts LLMs", Sec. 2.5 / Algorithm 3: a
+ * copy of the heavy-hitter is appended to the layer; the page gives no rule that
+ * sends tokens to it, and its review suggests splitting the heavy-hitter's tokens
+ * alternately between the original and the replica). The heavy-hitter h is the
+ * expert with the most tasks, n_j of Definition 1 (lowest index on ties). Its
+ * tasks are taken in increasing task id q = t*k + s, the order of its segment in
+ * the expert-centric permutation: the 1st, 3rd, 5th, ... stay with h, the 2nd,
+ * 4th, ... go to the replica, expert m. Every other task keeps its expert. */
+int oracle_replica_split(int T, int k, int m, const int32_t* idx, int32_t* idx_out, int32_t* heavy) {
+  if (T <= 0 || k <= 0 || m <= 0) return 1;
+  int32_t* counts = (int32_t*)calloc((size_t)m, sizeof(int32_t));
+  for (int64_t q = 0; q < (int64_t)T * k; ++q) {
+    if (idx[q] < 0 || idx[q] >= m) {
+      free(counts);
+      return 2;
+    }
+    counts[idx[q]] += 1;
+  }
+  int h = 0;
+  for (int e = 1; e < m; ++e)
+    if (counts[e] > counts[h]) h = e;
+  int64_t r = 0; /* tasks of h seen so far */
+  for (int64_t q = 0; q < (int64_t)T * k; ++q) {
+    if (idx[q] == h) {
+      idx_out[q] = (r % 2 == 1) ? m : h;
+      ++r;
+    } else {
+      idx_out[q] = idx[q];
+    }
+  }
+  *heavy = h;
+  free(counts);
+  return 0;
+}
+
 /* ------------------------------------------------------------------ experts */
 
 /* One expert applied to one token, fp64 throughout.

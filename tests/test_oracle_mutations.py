@@ -43,6 +43,8 @@ MUTATIONS = {
                                  "return (p->id < q->id) - (p->id > q->id);"),
     "atomic_logprob_unnormalised": ("out[(int64_t)t * n + i] = (float)(z[i] - lse);",
                                     "out[(int64_t)t * n + i] = (float)(z[i] - mx);"),
+    "replica_even_ranks": ("idx_out[q] = (r % 2 == 1) ? m : h;", "idx_out[q] = (r % 2 == 0) ? m : h;"),
+    "replica_heavy_last_tie": ("if (counts[e] > counts[h]) h = e;", "if (counts[e] >= counts[h]) h = e;"),
 }
 
 
@@ -168,7 +170,16 @@ def check_atomic(O):
     np.testing.assert_allclose(out, ref.numpy(), rtol=1e-10, atol=1e-12)
 
 
-CHECKS = [check_lis_golden, check_topk, check_router, check_permutation, check_ffn, check_shared, check_atomic]
+def check_replica(O):
+    for name, m, k, before, heavy, after, counts, lis0, lis1 in _golden_rows("replica_cases.txt"):
+        idx = np.array([[int(e) for e in tok.split(",")] for tok in before.split(";")], dtype=np.int32)
+        got, h = O.replica_split(idx, int(m))
+        assert h == int(heavy)
+        assert got.ravel().tolist() == [int(e) for tok in after.split(";") for e in tok.split(",")]
+
+
+CHECKS = [check_lis_golden, check_topk, check_router, check_permutation, check_ffn, check_shared, check_atomic,
+          check_replica]
 
 
 def _failures(O):

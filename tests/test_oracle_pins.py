@@ -409,3 +409,60 @@ def test_plain_candidate_block_is_not_always_exact():
     assert idx[0].tolist() == [0, 4]
     rows = sorted(range(4), key=lambda i: (-float(lr[i]), i))[:K]
     assert 0 not in rows
+
+
+# ------------------------------------------------------------------ R&Q replica dispatch
+
+def _routing(text):
+    return np.array([[int(e) for e in tok.split(",")] for tok in text.split(";")], dtype=np.int32)
+
+
+def test_replica_split_golden(golden_dir):
+    for name, m, k, before, heavy, after, counts, lis0, lis1 in _golden(os.path.join(golden_dir, "replica_cases.txt")):
+        m, k = int(m), int(k)
+        idx, idx2 = _routing(before), _routing(after)
+        got, h = O.replica_split(idx, m)
+        assert h == int(heavy), name
+        np.testing.assert_array_equal(got, idx2, err_msg=name)
+        assert O.histogram_lis(idx, m)["lis"] == float(Fraction(lis0)), name
+        r = O.histogram_lis(got, m + 1)
+        assert r["counts"].tolist() == [int(c) for c in counts.split(",")], name
+        assert r["lis"] == float(Fraction(lis1)), name
+
+
+@pytest.mark.parametrize("seed,T,m,k", [(0, 200, 8, 2), (1, 333, 16, 1), (2, 64, 4, 4), (3, 1000, 64, 6)])
+def test_replica_split_closed_form(seed, T, m, k):
+    # counts after: the heavy-hitter keeps ceil(n_h / 2), the replica gets floor(n_h / 2),
+    # every other expert and every task of another expert is untouched, and in task
+    # order the heavy-hitter's tasks alternate original, replica, original, ...
+    rng = np.random.default_rng(seed)
+    p = rng.dirichlet(np.full(m, 0.3))
+    idx = np.stack([rng.choice(m, size=k, replace=False, p=p) for _ in range(T)]).astype(np.int32)
+    counts = np.bincount(idx.ravel(), minlength=m)
+    h_ref = int(np.flatnonzero(counts == counts.max())[0])
+    got, h = O.replica_split(idx, m)
+    assert h == h_ref
+    c2 = np.bincount(got.ravel(), minlength=m + 1)
+    assert c2[h] == -(-counts[h] // 2) and c2[m] == counts[h] // 2
+    keep = np.ones(m + 1, bool)
+    keep[[h, m]] = False
+    np.testing.assert_array_equal(c2[keep], counts[np.arange(m) != h])
+    flat, flat2 = idx.ravel(), got.ravel()
+    np.testing.assert_array_equal(flat2[flat != h], flat[flat != h])
+    seq = flat2[flat == h]
+    np.testing.assert_array_equal(seq, np.where(np.arange(len(seq)) % 2 == 0, h, m))
+    assert O.histogram_lis(got, m + 1)["lis"] == (m + 1) * c2.max() / (T * k)
+
+
+@pytest.mark.parametrize("dtype,act", [(W.F32, W.SWIGLU), (W.BF16, W.RELU)])
+def test_replica_leaves_layer_output_unchanged(dtype, act):
+    # the replica carries the heavy-hitter's own weights, so every task computes the
+    # same expert function: the layer output is identical in fp64
+    cfg = W.small_moe(T=24, d=32, f=24, m=5, k=2, act=act, dtype=dtype, zipf_s=1.5, index=95)
+    inp = W.make_moe_inputs(cfg)
+    r = O.layer_forward(cfg, inp)
+    idx2, h = O.replica_split(r["idx"], cfg.m)
+    assert (idx2 == cfg.m).any()
+    cfg2 = W.small_moe(T=24, d=32, f=24, m=6, k=2, act=act, dtype=dtype, zipf_s=1.5, index=95)
+    out2 = O.moe_output(cfg2, O.replica_inputs(inp, h), idx2, r["w"])
+    np.testing.assert_array_equal(out2, r["out"])
