@@ -22,6 +22,7 @@ timed on a bounded sample of the same workload on this host's cores.
 from __future__ import annotations
 
 import argparse
+import dataclasses
 import datetime
 import hashlib
 import json
@@ -55,6 +56,9 @@ def parse():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--cpu-seconds", type=float, default=12.0, help="CPU-oracle baseline budget (rank 0, N=1)")
     ap.add_argument("--no-cpu-baseline", action="store_true", help="skip the CPU-oracle leg (for profiling runs)")
+    ap.add_argument("--replicate", action="store_true",
+                    help="R&Q replica dispatch: time moe_layer_forward_replicated (heavy-hitter split alternately "
+                         "with a replica expert m) instead of moe_layer_forward")
     ap.add_argument("--router-only", action="store_true",
                     help="time the routing call alone (moe_route / moe_atomic_route) on the workload's inputs; "
                          "an auxiliary line for profiling, not the layer metric")
@@ -365,19 +369,27 @@ def ours(args):
     d_in = {k: to_dev(v) for k, v in inp.items()}
     c = moe.make_config(cfg.T, cfg.d, cfg.f, cfg.m, cfg.k, cfg.n_shared, cfg.f_shared, cfg.dtype, cfg.act,
                         cfg.renorm)
-    ws = moe.workspace(c, device=dev)
+    rep = args.replicate
+    if rep and cfg.dtype != W.BF16:
+        raise SystemExit("--replicate runs bf16 layers only")
+    ws = moe.replica_workspace(c, device=dev) if rep else moe.workspace(c, device=dev)
     tdt = torch.float32 if cfg.dtype == W.F32 else torch.bfloat16
     out = torch.empty((cfg.T, cfg.d), dtype=tdt, device=dev)
-    counts = torch.empty(cfg.m, dtype=torch.int32, device=dev)
+    counts = torch.empty(cfg.m + (1 if rep else 0), dtype=torch.int32, device=dev)
     lis = moe.lis_buffer(dev)
+    lis0 = moe.lis_buffer(dev)
     s = torch.cuda.Stream(device=dev)
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
 
     def fwd(x=None, o=None):
-        moe.moe_layer_forward(c, d_in["x"] if x is None else x, d_in["w_router"], d_in["bias"], d_in["w_gate"],
-                              d_in.get("w_up"), d_in["w_down"], d_in.get("ws_gate"), d_in.get("ws_up"),
-                              d_in.get("ws_down"), out if o is None else o, ws, counts_out=counts, lis_out=lis,
-                              stream=s)
+        args_ = (c, d_in["x"] if x is None else x, d_in["w_router"], d_in["bias"], d_in["w_gate"], d_in.get("w_up"),
+                 d_in["w_down"], d_in.get("ws_gate"), d_in.get("ws_up"), d_in.get("ws_down"),
+                 out if o is None else o, ws)
+        if rep:
+            moe.moe_layer_forward_replicated(*args_, counts_out=counts, lis_before_out=lis0, lis_after_out=lis,
+                                             stream=s)
+        else:
+            moe.moe_layer_forward(*args_, counts_out=counts, lis_out=lis, stream=s)
 
     with torch.cuda.stream(s):
         n0 = moe.moe_launch_count()
@@ -415,7 +427,7 @@ def ours(args):
                 for j, name in enumerate(STAGES)}
     dom = max(STAGES, key=lambda n: stage_ms[n])
     jd = STAGES.index(dom)
-    if fused_routing(cfg):
+    if fused_routing(cfg) and not rep:
         # one kernel spans stages 0-1 and one spans 3-4; the two boundaries between them coincide
         stage_ms = {("router_topk_ranks" if n == "router" else "scatter" if n == "permute" else n): v
                     for n, v in stage_ms.items() if n not in ("topk", "histogram_lis_ranks")}
@@ -478,20 +490,21 @@ def ours(args):
     ms, e2e_ms = max_over_ranks([ms_local, e2e_local], dist, dev)
 
     pk, pk_src = peaks()
+    cfg_groups = dataclasses.replace(cfg, m=cfg.m + 1) if rep else cfg  # the replica is one more routed group
     plan_ksplit = 1
     if cfg.dtype == W.BF16 and cfg.n_shared == 0:
         # the library's static down-projection split (mirrors its planner; only affects the byte count)
-        avg = cfg.T * cfg.k / cfg.m
+        avg = cfg.T * cfg.k / cfg_groups.m
         bn = 16
-        while bn < 256 and bn < avg:
+        while bn < 256 and bn < 2.0 * avg:
             bn <<= 1
-        tiles = min(cfg.m, cfg.T * cfg.k) * ((cfg.d + 127) // 128) * max(1, math.ceil(avg / bn))
+        tiles = min(cfg_groups.m, cfg.T * cfg.k) * ((cfg.d + 127) // 128) * max(1, math.ceil(avg / bn))
         if tiles < 4 * 148:
             kb = (cfg.f + 63) // 64
             ks = min(16, -(-4 * 148 // tiles), kb)
             kbps = -(-kb // ks)
             plan_ksplit = -(-kb // kbps)
-    costs, layer_flops, layer_bytes = stage_costs(cfg, active, plan_ksplit)
+    costs, layer_flops, layer_bytes = stage_costs(cfg_groups, active, plan_ksplit)
     fl, by = costs[dom]
     sec = dom_ms * 1e-3
     long_step = K * ms > 1000.0
@@ -527,6 +540,10 @@ def ours(args):
                            "boundaries",
             "routing": {"lis": lis_v, "max_count": max_count, "heavy_hitter": argmax, "active_experts": active,
                         "reuse_ratio": cfg.T * cfg.k / max(active, 1), "load_entropy": entropy},
+            **({"variant": "R&Q replica dispatch: the heavy-hitter's tasks alternate between it and a replica "
+                           "expert m that computes with its bf16 weights; routing.lis is over the m + 1 experts",
+                "lis_before_split": moe.unpack_lis(lis0)[2],
+                "heavy_hitter_before_split": moe.unpack_lis(lis0)[1]} if rep else {}),
             "e2e": {"value": world * cfg.T / (e2e_ms * 1e-3), "unit": UNIT, "h2d_bytes_per_step": h2d,
                     "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms,
                     "note": "pinned host -> device batch upload and device -> host output download every step, on "

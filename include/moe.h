@@ -173,6 +173,41 @@ MOE_API moe_status_t moe_layer_forward(const moe_config_t* cfg, const void* x, c
                                int32_t* topk_idx_out, float* topk_w_out, int32_t* counts_out, moe_lis_t* lis_out,
                                void* ws, size_t ws_bytes, moe_stream_t stream);
 
+/* R&Q replica dispatch ("A Replicate-and-Quantize Strategy for Plug-and-Play Load
+ * Balancing of Sparse Mixture-of-Experts LLMs", Sec. 2.5 and Algorithm 3, which
+ * append a replica of the heavy-hitter but leave the router unchanged and give no
+ * rule that sends tokens to it; the rule here is the one its review suggests:
+ * the heavy-hitter's tokens alternate between the original and the replica).
+ * Inputs are the outputs of moe_histogram_lis / moe_permute for topk_idx (m
+ * experts): the heavy-hitter h = lis->argmax_expert (most tasks, lowest index on
+ * ties); the tasks of h in their segment order (increasing task id t k + s) go
+ * original, replica, original, ...; the replica is expert m.
+ * idx_out [T, k] int32: experts in [0, m] after the split (every other task is
+ * unchanged). Optional: counts_out [m + 1] (h keeps ceil(n_h / 2), the replica
+ * gets floor(n_h / 2)); lis_out = Definition 1 over the m + 1 experts. All device
+ * pointers; ws: moe_workspace_size(cfg) bytes. MOE_ERR_DEVICE_INDEX (device
+ * status) if an id, h or a segment rank is out of range. Needs m + 1 <= 1024. */
+MOE_API moe_status_t moe_replica_split(const moe_config_t* cfg, const int32_t* topk_idx, const int32_t* offsets,
+                                       const int32_t* inv_perm, const moe_lis_t* lis, int32_t* idx_out,
+                                       int32_t* counts_out, moe_lis_t* lis_out, void* ws, size_t ws_bytes,
+                                       moe_stream_t stream);
+
+/* moe_layer_forward with R&Q replica dispatch (bf16 only): route over the m
+ * experts, split the heavy-hitter's tasks as moe_replica_split does, then run
+ * the layer over m + 1 routed groups, the replica computing with the
+ * heavy-hitter's own weights (the pages' replica is a quantised copy; low-precision
+ * weights are not part of this call). The output therefore equals
+ * moe_layer_forward's up to rounding order. Optional device outputs: logits_out
+ * [T, m], topk_idx_out / topk_w_out [T, k] (the router's choice), dispatch_idx_out
+ * [T, k] (after the split), counts_out [m + 1], lis_before_out (m experts),
+ * lis_after_out (m + 1 experts). ws: moe_workspace_size() of the same config with
+ * m + 1 experts. MOE_ERR_UNSUPPORTED for fp32 or m + 1 > 1024. */
+MOE_API moe_status_t moe_layer_forward_replicated(
+    const moe_config_t* cfg, const void* x, const void* w_router, const float* bias, const void* w_gate,
+    const void* w_up, const void* w_down, const void* ws_gate, const void* ws_up, const void* ws_down, void* out,
+    float* logits_out, int32_t* topk_idx_out, float* topk_w_out, int32_t* dispatch_idx_out, int32_t* counts_out,
+    moe_lis_t* lis_before_out, moe_lis_t* lis_after_out, void* ws, size_t ws_bytes, moe_stream_t stream);
+
 /* Cartesian Product Router (OmniMoE Sec. 2.2, Eq. 8; App. A): lr = log_softmax(x
  * w_row^T), lc = log_softmax(x w_col^T) (fp32); expert (i, j) with flat id
  * i Nc + j scores S = fl32(lr_i + lc_j); idx_out [T, K] = the exact top-K of all
@@ -230,7 +265,9 @@ MOE_API moe_status_t moe_debug_set_wait_limit_ns(uint64_t ns);
  * stream at its stage boundaries, in order: 0 start, 1 router logits, 2 top-k,
  * 3 histogram/LIS/ranks, 4 row permutation, 5 up projection, 6 down projection,
  * 7 combine (n <= 8; extra stages are not recorded); moe_atomic_forward records
- * 0 start, 1 router projections, 2 grid top-K, 3 expert coefficients, 4 assembly.
+ * 0 start, 1 router projections, 2 grid top-K, 3 expert coefficients, 4 assembly;
+ * moe_layer_forward_replicated records the stages of moe_layer_forward (3 is
+ * after both sorts and the split).
  * A NULL entry skips that
  * boundary (a recorded event between two kernels stops the second one from
  * starting early, so record only the boundaries you time). n = 0 turns it off.

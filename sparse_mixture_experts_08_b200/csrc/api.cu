@@ -100,7 +100,7 @@ static Plan make_plan(const moe_config_t& c) {
 
 struct Layout {
   size_t status, logits, idx, w, counts, offsets, lis, perm, inv_perm, w_perm, start, x_perm, h, h_sh, y, y_sh;
-  size_t lrank, tile_cnt, total;
+  size_t lrank, tile_cnt, idx2, gmap, lis2, total;
 };
 
 static Layout make_layout(const moe_config_t& c, const Plan& p) {
@@ -131,6 +131,9 @@ static Layout make_layout(const moe_config_t& c, const Plan& p) {
   L.y_sh = take((size_t)p.ksplit * c.n_shared * T * c.d * 4);
   L.lrank = take(Tk * 4);                          // fused router: task ranks within their tile
   L.tile_cnt = take((T + 127) / 128 * c.m * 4);    // and tasks per expert per 128-token tile
+  L.idx2 = take(Tk * 4);                           // replica dispatch: experts after the split
+  L.gmap = take((size_t)(c.m + 1) * 4);            // and the group -> weight matrix map
+  L.lis2 = take(sizeof(moe_lis_t));
   L.total = off;
   return L;
 }
@@ -224,6 +227,8 @@ struct FfnIo {
   const int32_t* perm;
   const float* row_w;     // task_w already gathered into segment order (nullable)
   void* out_k1;           // top-1 layers: the down projection writes the layer output directly
+  const int* group_map;   // device [n_routed]: weight matrix of each routed group (nullable = identity)
+  int n_wgroups;          // routed weight matrices (== n_routed without a map)
   // shared class
   int n_shared;
   const void* x;          // [T, d]
@@ -264,8 +269,10 @@ static moe_status_t run_ffn(const moe_config_t& c, const Plan& pl, const FfnIo& 
     g.b = io.x_perm;
     g.a_ld = c.d;
     g.b_ld = c.d;
-    mu.a0[ncls] = {io.w_gate, (long long)io.n_routed * c.f, c.d};
-    mu.a1[ncls] = {swiglu ? io.w_up : io.w_gate, (long long)io.n_routed * c.f, c.d};
+    g.group_map = io.group_map;
+    g.n_wgroups = io.group_map ? io.n_wgroups : io.n_routed;
+    mu.a0[ncls] = {io.w_gate, (long long)g.n_wgroups * c.f, c.d};
+    mu.a1[ncls] = {swiglu ? io.w_up : io.w_gate, (long long)g.n_wgroups * c.f, c.d};
     mu.b[ncls] = {io.x_perm, io.routed_rows, c.d};
     ++ncls;
   }
@@ -327,7 +334,9 @@ static moe_status_t run_ffn(const moe_config_t& c, const Plan& pl, const FfnIo& 
     g.b = io.h;
     g.a_ld = c.f;
     g.b_ld = c.f;
-    md.a0[ncls] = {io.w_down, (long long)io.n_routed * c.d, c.f};
+    g.group_map = io.group_map;
+    g.n_wgroups = io.group_map ? io.n_wgroups : io.n_routed;
+    md.a0[ncls] = {io.w_down, (long long)g.n_wgroups * c.d, c.f};
     md.a1[ncls] = md.a0[ncls];
     md.b[ncls] = {io.h, io.routed_rows, c.f};
     ++ncls;
@@ -735,6 +744,126 @@ moe_status_t moe_atomic_forward(const moe_atomic_config_t* cfg, const void* x, c
   MOE_CUDA(launch_atomic_experts(c.T, c.d, c.K, c.act, x, w_in, w_out, idx, g, at<float>(ws, P.coef), out,
                                  (long long)c.Nr * c.Nc, at<int>(ws, P.status), s, true));
   return mark_stage(4, s);
+}
+
+// ------------------------------------------------------------------ R&Q replica dispatch
+moe_status_t moe_replica_split(const moe_config_t* cfg, const int32_t* topk_idx, const int32_t* offsets,
+                               const int32_t* inv_perm, const moe_lis_t* lis, int32_t* idx_out, int32_t* counts_out,
+                               moe_lis_t* lis_out, void* ws, size_t ws_bytes, moe_stream_t stream) {
+  MOE_TRY(check_cfg(cfg));
+  const moe_config_t& c = *cfg;
+  if (!topk_idx || !offsets || !inv_perm || !lis || !idx_out) return MOE_ERR_INVALID_ARG;
+  if (c.m + 1 > 1024) return MOE_ERR_UNSUPPORTED;  // the replica is expert m
+  for (const void* p : std::initializer_list<const void*>{(const void*)topk_idx, (const void*)offsets,
+                                                          (const void*)inv_perm, (const void*)lis, (const void*)idx_out,
+                                                          (const void*)counts_out, (const void*)lis_out})
+    if (p && !aligned16(p)) return MOE_ERR_INVALID_ARG;
+  const Layout L = make_layout(c, make_plan(c));
+  MOE_TRY(check_ws(c, ws, ws_bytes, L.total));
+  MOE_TRY(check_device());
+  return cuda_status(launch_replica_split(c.T, c.k, c.m, topk_idx, offsets, inv_perm, lis, idx_out,
+                                          at<int32_t>(ws, L.gmap), counts_out, lis_out, at<int>(ws, L.status),
+                                          (cudaStream_t)stream));
+}
+
+moe_status_t moe_layer_forward_replicated(const moe_config_t* cfg, const void* x, const void* w_router,
+                                          const float* bias, const void* w_gate, const void* w_up, const void* w_down,
+                                          const void* ws_gate, const void* ws_up, const void* ws_down, void* out,
+                                          float* logits_out, int32_t* topk_idx_out, float* topk_w_out,
+                                          int32_t* dispatch_idx_out, int32_t* counts_out, moe_lis_t* lis_before_out,
+                                          moe_lis_t* lis_after_out, void* ws, size_t ws_bytes, moe_stream_t stream) {
+  MOE_TRY(check_cfg(cfg));
+  const moe_config_t& c = *cfg;
+  if (c.dtype != MOE_BF16) return MOE_ERR_UNSUPPORTED;
+  moe_config_t c1 = c;  // the layer after the split: m + 1 routed groups
+  c1.m = c.m + 1;
+  MOE_TRY(check_cfg(&c1));
+  if (!x || !w_router || !w_gate || !w_down || !out) return MOE_ERR_INVALID_ARG;
+  if (c.act == MOE_SWIGLU && !w_up) return MOE_ERR_INVALID_ARG;
+  if (c.n_shared > 0 && (!ws_gate || !ws_down || (c.act == MOE_SWIGLU && !ws_up))) return MOE_ERR_INVALID_ARG;
+  for (const void* p : std::initializer_list<const void*>{
+           x, w_router, (const void*)bias, w_gate, w_up, w_down, ws_gate, ws_up, ws_down, out, (const void*)logits_out,
+           (const void*)topk_idx_out, (const void*)topk_w_out, (const void*)dispatch_idx_out, (const void*)counts_out,
+           (const void*)lis_before_out, (const void*)lis_after_out})
+    if (p && !aligned16(p)) return MOE_ERR_INVALID_ARG;
+  const Plan pl = make_plan(c1);
+  const Layout L = make_layout(c1, pl);
+  MOE_TRY(check_ws(c1, ws, ws_bytes, L.total));
+  MOE_TRY(check_device());
+  cudaStream_t s = (cudaStream_t)stream;
+  int* status = at<int>(ws, L.status);
+  float* logits = logits_out ? logits_out : at<float>(ws, L.logits);
+  int32_t* idx = topk_idx_out ? topk_idx_out : at<int32_t>(ws, L.idx);
+  float* w = topk_w_out ? topk_w_out : at<float>(ws, L.w);
+  int32_t* counts = at<int32_t>(ws, L.counts);
+  int32_t* offsets = at<int32_t>(ws, L.offsets);
+  moe_lis_t* lis0 = lis_before_out ? lis_before_out : at<moe_lis_t>(ws, L.lis);
+  moe_lis_t* lis1 = lis_after_out ? lis_after_out : at<moe_lis_t>(ws, L.lis2);
+  int32_t* perm = at<int32_t>(ws, L.perm);
+  int32_t* inv_perm = at<int32_t>(ws, L.inv_perm);
+  float* w_perm = at<float>(ws, L.w_perm);
+  int32_t* start = at<int32_t>(ws, L.start);
+  int32_t* idx2 = dispatch_idx_out ? dispatch_idx_out : at<int32_t>(ws, L.idx2);
+  int32_t* gmap = at<int32_t>(ws, L.gmap);
+  const long long Tk = (long long)c.T * c.k;
+
+  // 1. router and top-k over the m experts (stage events as in moe_layer_forward)
+  MOE_TRY(mark_stage(0, s));
+  if (fused_route_ok(c)) {
+    MOE_CUDA(launch_route_topk(c, x, w_router, bias, logits_out, idx, w, nullptr, nullptr, status, g_wait_limit_ns,
+                               s));
+    MOE_TRY(mark_stage(1, s));
+  } else {
+    MOE_TRY(run_router(c, x, w_router, bias, logits, status, s));
+    MOE_TRY(mark_stage(1, s));
+    MOE_CUDA(launch_topk_softmax(c.T, c.m, c.k, c.renormalize, logits, idx, w, s));
+  }
+  MOE_TRY(mark_stage(2, s));
+  // 2. histogram / LIS and the stable ranks over the m experts (the heavy-hitter's
+  //    segment order is the split order)
+  MOE_CUDA(launch_route_index(1, c.T, c.k, c.m, idx, counts, offsets, lis0, start, status, s));
+  MOE_CUDA(launch_rank(c.T, c.k, c.m, idx, offsets, start, nullptr, perm, inv_perm, nullptr, status, s));
+  // 3. every second task of the heavy-hitter to the replica, expert m
+  MOE_CUDA(launch_replica_split(c.T, c.k, c.m, idx, offsets, inv_perm, lis0, idx2, gmap, nullptr, nullptr, status, s));
+  // 4. histogram / LIS, ranks and rows over the m + 1 experts
+  int32_t* counts1 = counts_out ? counts_out : counts;
+  MOE_CUDA(launch_route_index(1, c.T, c.k, c1.m, idx2, counts1, offsets, lis1, start, status, s));
+  MOE_CUDA(launch_rank(c.T, c.k, c1.m, idx2, offsets, start, w, perm, inv_perm, w_perm, status, s));
+  MOE_TRY(mark_stage(3, s));
+  MOE_CUDA(launch_permute_rows(c.dtype, (int)Tk, c.k, c.d, x, inv_perm, at<void>(ws, L.x_perm), s));
+  MOE_TRY(mark_stage(4, s));
+  // 5. the grouped FFN over m + 1 groups; group m reads the heavy-hitter's weights
+  FfnIo io;
+  std::memset(&io, 0, sizeof(io));
+  io.n_routed = c1.m;
+  io.offsets = offsets;
+  io.x_perm = at<void>(ws, L.x_perm);
+  io.routed_rows = Tk;
+  io.w_gate = w_gate;
+  io.w_up = w_up;
+  io.w_down = w_down;
+  io.h = at<void>(ws, L.h);
+  io.y = at<float>(ws, L.y);
+  io.task_w = w;
+  io.row_w = w_perm;
+  io.perm = perm;
+  io.group_map = gmap;
+  io.n_wgroups = c.m;
+  io.n_shared = c.n_shared;
+  io.x = x;
+  io.ws_gate = ws_gate;
+  io.ws_up = ws_up;
+  io.ws_down = ws_down;
+  io.h_sh = at<void>(ws, L.h_sh);
+  io.y_sh = at<float>(ws, L.y_sh);
+  const bool fuse_combine = c.k == 1 && c.n_shared == 0 && pl.ksplit == 1;
+  io.out_k1 = fuse_combine ? out : nullptr;
+  MOE_TRY(run_ffn(c1, pl, io, pl.ksplit, pl.kbps, status, s, true));
+  MOE_TRY(mark_stage(6, s));
+  if (!fuse_combine)
+    MOE_CUDA(launch_combine(c.dtype, c.T, c.d, c.k, pl.ksplit, io.y, Tk * c.d, inv_perm, c.n_shared, io.y_sh,
+                            (long long)c.n_shared * c.T * c.d, out, s));
+  return mark_stage(7, s);
 }
 
 // ------------------------------------------------------------------ status helpers

@@ -133,6 +133,8 @@ struct GemmClass {
   const float* task_w;       // DOWN: row weight task_w[perm[row]] (nullable = 1)
   const int* perm;
   int scatter_k1;            // DOWN with top-1 routing: write bf16 out[perm[row]] (combine fused)
+  const int* group_map;      // device [n_groups]: weight matrix of group g (nullable = g); values < n_wgroups
+  int n_wgroups;             // weight matrices behind group_map
   // ROUTE: top-k selection in the epilogue (out = fp32 logits [T, m], nullable)
   int k_sel, renorm;
   int32_t* sel_idx;          // [T, k] experts by (logit desc, expert asc)
@@ -198,6 +200,12 @@ cudaError_t launch_route_scatter(int dtype, int T, int k, int m, int d, const in
                                  const int32_t* lrank, const float* task_w, const void* x, int32_t* counts,
                                  int32_t* offsets, moe_lis_t* lis, int32_t* perm, int32_t* inv_perm, float* w_perm,
                                  void* x_perm, int* status, cudaStream_t s);
+// R&Q replica dispatch: tasks of the heavy-hitter (lis_in->argmax_expert) with an
+// odd rank in its segment go to expert m; writes idx_out, the group -> weight map
+// [m + 1] and, when given, counts [m + 1] and the LIS over m + 1 experts.
+cudaError_t launch_replica_split(int T, int k, int m, const int32_t* idx, const int32_t* offsets,
+                                 const int32_t* inv_perm, const moe_lis_t* lis_in, int32_t* idx_out, int32_t* gmap,
+                                 int32_t* counts_out, moe_lis_t* lis_out, int* status, cudaStream_t s);
 cudaError_t launch_rank(int T, int k, int m, const int32_t* idx, const int32_t* offsets, const int32_t* start,
                         const float* task_w, int32_t* perm, int32_t* inv_perm, float* w_perm, int* status,
                         cudaStream_t s);

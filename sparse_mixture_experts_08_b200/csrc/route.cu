@@ -667,6 +667,88 @@ cudaError_t launch_route_scatter(int dtype, int T, int k, int m, int d, const in
   return cudaGetLastError();
 }
 
+// ------------------------------------------------------------------ R&Q replica dispatch
+// The heavy-hitter h is the device LIS record's argmax (most tasks, lowest index).
+// A task's rank in h's segment of the stable sort is inv_perm[q] - offsets[h]; the
+// odd ranks go to the replica, expert m (every second task of h in task order).
+// Block 0 also writes the group -> weight map (g, and h for the replica) and, when
+// given, the counts and the LIS (R&Q Definition 1) over the m + 1 experts.
+__global__ void replica_split_kernel(int T, int k, int m, const int32_t* __restrict__ idx,
+                                     const int32_t* __restrict__ offsets, const int32_t* __restrict__ inv_perm,
+                                     const moe_lis_t* __restrict__ lis_in, int32_t* __restrict__ idx_out,
+                                     int32_t* __restrict__ gmap, int32_t* __restrict__ counts_out,
+                                     moe_lis_t* __restrict__ lis_out, int* status) {
+  __shared__ int prior_s;
+  pdl_launch_dependents();
+  pdl_wait();
+  if (threadIdx.x == 0) prior_s = *reinterpret_cast<volatile int*>(status);
+  __syncthreads();
+  if (prior_s != 0) return;  // uniform across the block
+  const long long Tk = (long long)T * k;
+  const int h = lis_in->argmax_expert;
+  if (h < 0 || h >= m) {
+    if (threadIdx.x == 0 && blockIdx.x == 0) set_status(status, MOE_ERR_DEVICE_INDEX);
+    return;
+  }
+  const int n_h = offsets[h + 1] - offsets[h];
+  for (long long q = (long long)blockIdx.x * blockDim.x + threadIdx.x; q < Tk; q += (long long)gridDim.x * blockDim.x) {
+    const int e = idx[q];
+    int o = e;
+    if (e < 0 || e >= m) {
+      set_status(status, MOE_ERR_DEVICE_INDEX);
+    } else if (e == h) {
+      const int r = inv_perm[q] - offsets[h];
+      if (r < 0 || r >= n_h) set_status(status, MOE_ERR_DEVICE_INDEX);
+      o = (r & 1) ? m : h;
+    }
+    idx_out[q] = o;
+  }
+  if (blockIdx.x != 0) return;
+  for (int g = threadIdx.x; g <= m; g += blockDim.x) gmap[g] = g < m ? g : h;
+  auto count_after = [&](int j) {
+    if (j == m) return n_h / 2;
+    const int n = offsets[j + 1] - offsets[j];
+    return j == h ? n - n_h / 2 : n;
+  };
+  if (counts_out)
+    for (int j = threadIdx.x; j <= m; j += blockDim.x) counts_out[j] = count_after(j);
+  if (lis_out && threadIdx.x < 32) {
+    const int lane = threadIdx.x;
+    int bv = -1, ba = 0x7fffffff;
+    for (int j = lane; j <= m; j += 32) {
+      const int v = count_after(j);
+      if (v > bv) {  // ascending j per lane: an equal count keeps the lower expert
+        bv = v;
+        ba = j;
+      }
+    }
+#pragma unroll
+    for (int o = 16; o; o >>= 1) {
+      const int ov = __shfl_xor_sync(FULL, bv, o), oa = __shfl_xor_sync(FULL, ba, o);
+      if (ov > bv || (ov == bv && oa < ba)) {
+        bv = ov;
+        ba = oa;
+      }
+    }
+    if (lane == 0) {
+      lis_out->max_count = bv;
+      lis_out->argmax_expert = ba;
+      lis_out->lis = (double)((long long)(m + 1) * bv) / (double)((long long)T * k);
+    }
+  }
+}
+
+cudaError_t launch_replica_split(int T, int k, int m, const int32_t* idx, const int32_t* offsets,
+                                 const int32_t* inv_perm, const moe_lis_t* lis_in, int32_t* idx_out, int32_t* gmap,
+                                 int32_t* counts_out, moe_lis_t* lis_out, int* status, cudaStream_t s) {
+  const long long Tk = (long long)T * k;
+  const int blocks = (int)std::max<long long>(1, std::min<long long>((Tk + 255) / 256, (long long)num_sms() * 4));
+  launch_k(replica_split_kernel, blocks, 256, 0, s, T, k, m, idx, offsets, inv_perm, lis_in, idx_out, gmap, counts_out,
+           lis_out, status);
+  count_launch();
+  return cudaGetLastError();
+}
+
 // ------------------------------------------------------------------ combine
 // out[t, c] = sum_s sum_split y[split][inv_perm[t k + s], c]
 //           + sum_sh sum_split ysh[split][sh T + t, c], fp32, slot order; 4 columns

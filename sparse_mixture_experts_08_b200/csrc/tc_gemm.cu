@@ -246,7 +246,13 @@ __device__ __forceinline__ void decode_tile(const GemmParams& p, const SchedSmem
   ti.rows_in_tile = min(BN, rows - ti.nt * BN);
   ti.b_row = s.brow[gi] + ti.nt * BN;
   ti.out_row = (c.seg_off ? s.brow[gi] : ti.g * c.out_group_stride) + ti.nt * BN;
-  ti.a_row = ti.g * c.R + ti.mt * TC_BM;
+  // the weight matrix of the group (a replica group reads another group's weights)
+  int wg = ti.g;
+  if (c.group_map) {
+    wg = c.group_map[ti.g];
+    if (wg < 0 || wg >= c.n_wgroups) wg = 0;  // (validated where the map is written)
+  }
+  ti.a_row = wg * c.R + ti.mt * TC_BM;
   const int KB = (c.K + TC_BK - 1) / TC_BK;
   ti.kb0 = ti.ks * c.kb_per_split;
   ti.kb1 = min(KB, ti.kb0 + c.kb_per_split);

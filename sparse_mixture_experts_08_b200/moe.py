@@ -30,7 +30,8 @@ STATUS_NAMES = {0: "MOE_OK", 1: "MOE_ERR_INVALID_ARG", 2: "MOE_ERR_UNSUPPORTED",
 EXPORTS = ["moe_workspace_size", "moe_atomic_workspace_size", "moe_route", "moe_histogram_lis", "moe_permute",
            "moe_grouped_ffn", "moe_shared_ffn", "moe_combine", "moe_layer_forward", "moe_atomic_route",
            "moe_atomic_experts", "moe_atomic_forward", "moe_read_device_status", "moe_status_string",
-           "moe_debug_set_wait_limit_ns", "moe_set_stage_events", "moe_launch_count", "moe_route_static"]
+           "moe_debug_set_wait_limit_ns", "moe_set_stage_events", "moe_launch_count", "moe_route_static",
+           "moe_replica_split", "moe_layer_forward_replicated"]
 
 
 class MoEConfig(ctypes.Structure):
@@ -73,6 +74,8 @@ def lib() -> ctypes.CDLL:
             "moe_shared_ffn": [P, P, P, P, P, P, P, S, P],
             "moe_combine": [P, P, P, P, P, P],
             "moe_layer_forward": [P, P, P, P, P, P, P, P, P, P, P, P, P, P, P, P, P, S, P],
+            "moe_replica_split": [P, P, P, P, P, P, P, P, P, S, P],
+            "moe_layer_forward_replicated": [P, P, P, P, P, P, P, P, P, P, P, P, P, P, P, P, P, P, P, S, P],
             "moe_atomic_route": [P, P, P, P, P, P, P, P, P, S, P],
             "moe_atomic_experts": [P, P, P, P, P, P, P, P, S, P],
             "moe_atomic_forward": [P, P, P, P, P, P, P, P, P, P, S, P],
@@ -187,6 +190,23 @@ def moe_layer_forward(cfg, x, w_router, bias, w_gate, w_up, w_down, ws_gate, ws_
         _p(lis_out), _p(ws), ws.numel(), _stream(stream)))
 
 
+def moe_replica_split(cfg, topk_idx, offsets, inv_perm, lis, idx_out, ws, counts_out=None, lis_out=None,
+                      stream=None):
+    _check("moe_replica_split", lib().moe_replica_split(ctypes.byref(cfg), _p(topk_idx), _p(offsets), _p(inv_perm),
+                                                        _p(lis), _p(idx_out), _p(counts_out), _p(lis_out), _p(ws),
+                                                        ws.numel(), _stream(stream)))
+
+
+def moe_layer_forward_replicated(cfg, x, w_router, bias, w_gate, w_up, w_down, ws_gate, ws_up, ws_down, out, ws,
+                                 logits_out=None, topk_idx_out=None, topk_w_out=None, dispatch_idx_out=None,
+                                 counts_out=None, lis_before_out=None, lis_after_out=None, stream=None):
+    """ws: a workspace for the same config with m + 1 experts (replica_workspace)."""
+    _check("moe_layer_forward_replicated", lib().moe_layer_forward_replicated(
+        ctypes.byref(cfg), _p(x), _p(w_router), _p(bias), _p(w_gate), _p(w_up), _p(w_down), _p(ws_gate),
+        _p(ws_up), _p(ws_down), _p(out), _p(logits_out), _p(topk_idx_out), _p(topk_w_out), _p(dispatch_idx_out),
+        _p(counts_out), _p(lis_before_out), _p(lis_after_out), _p(ws), ws.numel(), _stream(stream)))
+
+
 def moe_atomic_route(cfg, x, w_row, w_col, row_logp_out, col_logp_out, idx_out, g_out, ws, stream=None):
     _check("moe_atomic_route", lib().moe_atomic_route(ctypes.byref(cfg), _p(x), _p(w_row), _p(w_col),
                                                       _p(row_logp_out), _p(col_logp_out), _p(idx_out), _p(g_out),
@@ -234,6 +254,13 @@ def moe_launch_count() -> int:
 
 
 # ------------------------------------------------------------------ allocation helpers (torch memory)
+
+def replica_workspace(cfg, device="cuda") -> torch.Tensor:
+    """A zeroed workspace for moe_layer_forward_replicated: the same config with m + 1 experts."""
+    c1 = MoEConfig.from_buffer_copy(cfg)
+    c1.m = cfg.m + 1
+    return workspace(c1, device=device)
+
 
 def workspace(cfg, device="cuda") -> torch.Tensor:
     """A zeroed workspace of the size the config needs (uint8, 256-byte aligned)."""

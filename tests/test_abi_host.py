@@ -134,3 +134,31 @@ def test_debug_wait_limit_hook():
     assert lib.moe_debug_set_wait_limit_ns(5) == moe.OK
     assert lib.moe_debug_set_wait_limit_ns(0) == moe.OK
     assert moe.moe_launch_count() >= 0
+
+
+def test_replica_entry_points_validate_on_the_host():
+    lib = moe.moe.lib()
+    a = _fake(1 << 24)
+    ws = _fake(1 << 20)
+    c = MoEConfig(64, 128, 256, 8, 2, 0, 0, moe.BF16, moe.SWIGLU, 0)
+    # missing inputs
+    assert lib.moe_replica_split(ctypes.byref(c), a, None, a, a, a, None, None, ws, 1 << 30, None) == \
+        moe.ERR_INVALID_ARG
+    # the replica would be expert 1024
+    big = MoEConfig(64, 128, 256, 1024, 2, 0, 0, moe.BF16, moe.SWIGLU, 0)
+    assert lib.moe_replica_split(ctypes.byref(big), a, a, a, a, a, None, None, ws, 1 << 30, None) == \
+        moe.ERR_UNSUPPORTED
+    assert lib.moe_layer_forward_replicated(ctypes.byref(big), a, a, None, a, a, a, None, None, None, a, None, None,
+                                            None, None, None, None, None, ws, 1 << 30, None) == moe.ERR_UNSUPPORTED
+    # bf16 only
+    f32 = MoEConfig(64, 128, 256, 8, 2, 0, 0, moe.F32, moe.SWIGLU, 0)
+    assert lib.moe_layer_forward_replicated(ctypes.byref(f32), a, a, None, a, a, a, None, None, None, a, None, None,
+                                            None, None, None, None, None, ws, 1 << 30, None) == moe.ERR_UNSUPPORTED
+    # the workspace must fit the config with m + 1 experts
+    c1 = MoEConfig(64, 128, 256, 9, 2, 0, 0, moe.BF16, moe.SWIGLU, 0)
+    n0, n1 = ctypes.c_size_t(0), ctypes.c_size_t(0)
+    assert lib.moe_workspace_size(ctypes.byref(c), ctypes.byref(n0)) == moe.OK
+    assert lib.moe_workspace_size(ctypes.byref(c1), ctypes.byref(n1)) == moe.OK
+    assert n1.value > n0.value
+    assert lib.moe_layer_forward_replicated(ctypes.byref(c), a, a, None, a, a, a, None, None, None, a, None, None,
+                                            None, None, None, None, None, ws, n0.value, None) == moe.ERR_WORKSPACE
