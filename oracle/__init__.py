@@ -233,6 +233,43 @@ def dense_masked(cfg, inp: Dict[str, np.ndarray], idx: np.ndarray, w: np.ndarray
     return out
 
 
+# ------------------------------------------------------- FloE contextual sparsity
+
+def floe_threshold(u_abs: np.ndarray, sparsity: float) -> np.float32:
+    """FloE Eq. 6: the threshold from the empirical CDF of |up-projection
+    activations| at target sparsity s: the ceil(s n)-th smallest of the n values
+    (1-based; at least the 1st), so a fraction s of the sample lies at or below it."""
+    v = np.sort(np.asarray(u_abs, dtype=np.float32).ravel())
+    r = max(1, int(np.ceil(sparsity * v.size)))
+    return np.float32(v[min(r, v.size) - 1])
+
+
+def floe_expert(x_row: np.ndarray, wg: np.ndarray, wu: np.ndarray, wd: np.ndarray, thr: float, dtype: int,
+                u_mask: Optional[np.ndarray] = None):
+    """One expert on one token with FloE contextual sparsity (FloE "Core claim",
+    Sec. 3.2): u = x W_up^T; channel j is kept when |u_j| >= thr; for kept channels
+    g_j = x . W_gate[j] and h_j = g_j sigma(g_j) u_j, others contribute nothing;
+    y = sum over kept j of h_j W_down[:, j]. fp64. `u_mask`, when given, is the
+    up-projection output whose magnitudes decide the mask (so both sides of a
+    comparison decide from the same numbers); the arithmetic uses the fp64 u.
+    Returns (y, kept mask)."""
+    as64 = lambda a: np.asarray(_values(a, dtype), dtype=np.float64)
+    x = as64(x_row)
+    u = as64(wu) @ x
+    keep = np.abs(np.asarray(u_mask, np.float32) if u_mask is not None else u) >= thr
+    g = as64(wg)[keep] @ x
+    h = g / (1.0 + np.exp(-g)) * u[keep]
+    y = as64(wd)[:, keep] @ h
+    return y, keep
+
+
+def _values(a, dtype):
+    """bf16 bit patterns (uint16) or fp32 -> fp32 values (input decoding only)."""
+    if dtype == BF16 or a.dtype == np.uint16:
+        return (np.asarray(a, np.uint16).astype(np.uint32) << 16).view(np.float32)
+    return np.asarray(a, np.float32)
+
+
 # -------------------------------------------------------------------- atomic experts
 
 def atomic_logprobs(x: np.ndarray, w_row: np.ndarray, w_col: np.ndarray):

@@ -48,12 +48,24 @@ MUTATIONS = {
 }
 
 
-def _load_oracle(tmpdir, src_text):
+# mistakes planted in the Python part of the oracle (oracle/__init__.py)
+PY_MUTATIONS = {
+    "floe_mask_strict": ("if u_mask is not None else u) >= thr", "if u_mask is not None else u) > thr"),
+    "floe_gate_from_up": ("g = as64(wg)[keep] @ x", "g = as64(wu)[keep] @ x"),
+    "floe_threshold_off_by_one": ("return np.float32(v[min(r, v.size) - 1])", "return np.float32(v[min(r, v.size - 1)])"),
+}
+
+
+def _load_oracle(tmpdir, src_text, py_text=None):
     c_path = os.path.join(tmpdir, "moe_oracle.c")
     with open(c_path, "w") as fh:
         fh.write(src_text)
-    spec = importlib.util.spec_from_file_location(f"oracle_copy_{abs(hash(src_text))}",
-                                                  os.path.join(ROOT, "oracle", "__init__.py"))
+    py_path = os.path.join(ROOT, "oracle", "__init__.py")
+    if py_text is not None:
+        py_path = os.path.join(tmpdir, "oracle_init.py")
+        with open(py_path, "w") as fh:
+            fh.write(py_text)
+    spec = importlib.util.spec_from_file_location(f"oracle_copy_{abs(hash((src_text, py_text)))}", py_path)
     mod = importlib.util.module_from_spec(spec)
     spec.loader.exec_module(mod)
     mod._SRC = c_path
@@ -178,8 +190,24 @@ def check_replica(O):
         assert got.ravel().tolist() == [int(e) for tok in after.split(";") for e in tok.split(",")]
 
 
+def check_floe(O):
+    v = np.array([0.5, 0.1, 0.3, 0.2], np.float32)
+    assert [O.floe_threshold(v, s) for s in (0.0, 0.5, 0.75, 0.9)] == [np.float32(a) for a in (0.1, 0.2, 0.3, 0.5)]
+    cfg = W.small_moe(T=2, d=32, f=24, m=1, k=1, dtype=W.BF16, zipf_s=0.0, index=99)
+    inp = W.make_moe_inputs(cfg)
+    y, _ = O.floe_expert(inp["x"][0], inp["w_gate"][0], inp["w_up"][0], inp["w_down"][0], 0.0, W.BF16)
+    t = lambda key: _t64(inp[key], W.BF16)
+    ref = _torch_ffn(t("x")[0:1], t("w_gate")[0], t("w_up")[0], t("w_down")[0], W.SWIGLU)[0]
+    np.testing.assert_allclose(y, ref.numpy(), rtol=1e-10, atol=1e-12)
+    u32 = (t("w_up")[0] @ t("x")[1]).numpy().astype(np.float32)
+    j = int(np.argsort(np.abs(u32))[12])
+    _, keep = O.floe_expert(inp["x"][1], inp["w_gate"][0], inp["w_up"][0], inp["w_down"][0], float(abs(u32[j])),
+                            W.BF16, u_mask=u32)
+    assert keep[j]
+
+
 CHECKS = [check_lis_golden, check_topk, check_router, check_permutation, check_ffn, check_shared, check_atomic,
-          check_replica]
+          check_replica, check_floe]
 
 
 def _failures(O):
@@ -208,4 +236,18 @@ def test_mutant_is_caught(tmp_path, source, name):
     assert source.count(old) >= 1, f"mutation anchor for {name} not found"
     mutated = source.replace(old, new, 1)
     failed = _failures(_load_oracle(str(tmp_path), mutated))
+    assert failed, f"mutation {name} was not caught by any check"
+
+
+@pytest.fixture(scope="module")
+def py_source():
+    with open(os.path.join(ROOT, "oracle", "__init__.py")) as fh:
+        return fh.read()
+
+
+@pytest.mark.parametrize("name", sorted(PY_MUTATIONS))
+def test_python_mutant_is_caught(tmp_path, source, py_source, name):
+    old, new = PY_MUTATIONS[name]
+    assert py_source.count(old) == 1, f"mutation anchor for {name} not found"
+    failed = _failures(_load_oracle(str(tmp_path), source, py_source.replace(old, new, 1)))
     assert failed, f"mutation {name} was not caught by any check"

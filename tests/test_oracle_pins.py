@@ -466,3 +466,65 @@ def test_replica_leaves_layer_output_unchanged(dtype, act):
     cfg2 = W.small_moe(T=24, d=32, f=24, m=6, k=2, act=act, dtype=dtype, zipf_s=1.5, index=95)
     out2 = O.moe_output(cfg2, O.replica_inputs(inp, h), idx2, r["w"])
     np.testing.assert_array_equal(out2, r["out"])
+
+
+# ------------------------------------------------------------------ FloE contextual sparsity
+
+@pytest.mark.parametrize("s,expect", [(0.0, 0.1), (0.25, 0.1), (0.5, 0.2), (0.75, 0.3), (0.9, 0.5), (1.0, 0.5)])
+def test_floe_threshold_hand_cases(s, expect):
+    # n = 4 values; the ceil(s n)-th smallest (at least the first)
+    assert O.floe_threshold(np.array([0.5, 0.1, 0.3, 0.2], np.float32), s) == np.float32(expect)
+
+
+@pytest.mark.parametrize("s", [0.5, 0.8, 0.9, 0.97])
+def test_floe_threshold_is_the_cdf_quantile(s):
+    # a fraction >= s of the sample lies at or below t, and < s strictly below it
+    v = np.abs(np.random.default_rng(int(100 * s)).standard_normal(5003)).astype(np.float32)
+    t = O.floe_threshold(v, s)
+    assert (v <= t).mean() >= s and (v < t).mean() < s
+
+
+def _expert_case(act_seed=0):
+    cfg = W.small_moe(T=3, d=48, f=40, m=2, k=1, dtype=W.BF16, zipf_s=0.0, index=98 + act_seed)
+    return cfg, W.make_moe_inputs(cfg)
+
+
+def test_floe_expert_threshold_zero_is_the_dense_expert():
+    cfg, inp = _expert_case()
+    for t in range(cfg.T):
+        y, keep = O.floe_expert(inp["x"][t], inp["w_gate"][1], inp["w_up"][1], inp["w_down"][1], 0.0, W.BF16)
+        assert keep.all()
+        ref = O.expert_ffn(inp["x"][t], inp["w_gate"][1], inp["w_up"][1], inp["w_down"][1], W.SWIGLU)
+        np.testing.assert_allclose(y, ref, rtol=1e-12, atol=1e-14)
+
+
+def test_floe_expert_infinite_threshold_is_zero():
+    cfg, inp = _expert_case()
+    y, keep = O.floe_expert(inp["x"][0], inp["w_gate"][0], inp["w_up"][0], inp["w_down"][0], np.inf, W.BF16)
+    assert not keep.any() and not y.any()
+
+
+def test_floe_expert_is_the_dense_expert_with_pruned_channels_zeroed():
+    cfg, inp = _expert_case(1)
+    t64 = lambda a: torch.from_numpy(np.asarray(W.as_f32(a, W.BF16), np.float64))
+    x, wg, wu, wd = t64(inp["x"][2]), t64(inp["w_gate"][0]), t64(inp["w_up"][0]), t64(inp["w_down"][0])
+    u = wu @ x
+    thr = float(np.quantile(np.abs(u.numpy()), 0.7))
+    y, keep = O.floe_expert(inp["x"][2], inp["w_gate"][0], inp["w_up"][0], inp["w_down"][0], thr, W.BF16)
+    h = torch.nn.functional.silu(wg @ x) * u
+    h[torch.from_numpy(~keep)] = 0.0
+    assert 0 < keep.sum() < keep.size
+    np.testing.assert_allclose(y, (wd @ h).numpy(), rtol=1e-12, atol=1e-14)
+
+
+def test_floe_mask_keeps_the_threshold_itself():
+    # Eq. 6 prunes activations strictly below t; one exactly at t is kept
+    cfg, inp = _expert_case(1)
+    u = np.asarray(W.as_f32(inp["w_up"][0], W.BF16), np.float64) @ np.asarray(W.as_f32(inp["x"][1], W.BF16),
+                                                                                 np.float64)
+    j = int(np.argsort(np.abs(u))[len(u) // 2])
+    u32 = u.astype(np.float32)  # the mask compares these; the threshold is one of them exactly
+    thr = float(abs(u32[j]))
+    _, keep = O.floe_expert(inp["x"][1], inp["w_gate"][0], inp["w_up"][0], inp["w_down"][0], thr, W.BF16,
+                            u_mask=u32)
+    assert keep[j] and keep.sum() == (np.abs(u32) >= np.float32(thr)).sum()
