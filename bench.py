@@ -59,6 +59,9 @@ def parse():
     ap.add_argument("--replicate", action="store_true",
                     help="R&Q replica dispatch: time moe_layer_forward_replicated (heavy-hitter split alternately "
                          "with a replica expert m) instead of moe_layer_forward")
+    ap.add_argument("--floe", type=float, default=None, metavar="S",
+                    help="FloE contextual sparsity at target sparsity S: thresholds calibrated on a second "
+                         "synthetic batch (untimed), then moe_layer_forward_floe is timed")
     ap.add_argument("--router-only", action="store_true",
                     help="time the routing call alone (moe_route / moe_atomic_route) on the workload's inputs; "
                          "an auxiliary line for profiling, not the layer metric")
@@ -281,6 +284,11 @@ class ClockSampler:
 
 # ------------------------------------------------------------------ algorithmic cost model
 
+def T_bytes(cfg) -> int:
+    """x in and out of one layer step."""
+    return cfg.T * cfg.d * (4 if cfg.dtype == W.F32 else 2)
+
+
 def fused_routing(cfg) -> bool:
     """The library's rule for its one-launch router (logits + top-k + tile ranks in the
     tensor-core epilogue) followed by the one-kernel scatter: bf16, 8192+ tokens,
@@ -370,9 +378,31 @@ def ours(args):
     c = moe.make_config(cfg.T, cfg.d, cfg.f, cfg.m, cfg.k, cfg.n_shared, cfg.f_shared, cfg.dtype, cfg.act,
                         cfg.renorm)
     rep = args.replicate
+    floe = args.floe
     if rep and cfg.dtype != W.BF16:
         raise SystemExit("--replicate runs bf16 layers only")
-    ws = moe.replica_workspace(c, device=dev) if rep else moe.workspace(c, device=dev)
+    if floe is not None and (cfg.dtype != W.BF16 or cfg.act != W.SWIGLU or cfg.n_shared):
+        raise SystemExit("--floe runs bf16 SwiGLU layers without shared experts")
+    if rep:
+        ws = moe.replica_workspace(c, device=dev)
+    elif floe is not None:
+        ws = moe.floe_workspace(c, device=dev)
+    else:
+        ws = moe.workspace(c, device=dev)
+    if floe is not None:  # one-time weight layout and threshold calibration (untimed)
+        w_down_t = torch.empty((cfg.m, cfg.f, cfg.d), dtype=torch.bfloat16, device=dev)
+        moe.moe_floe_pack_down(c, d_in["w_down"], w_down_t)
+        xc = to_dev(W.make_moe_inputs(cfg, replicate=1, weights=False)["x"])
+        u_cal = torch.empty((cfg.T, cfg.m * cfg.f), dtype=torch.float32, device=dev)
+        thr = torch.empty(cfg.m, dtype=torch.float32, device=dev)
+        ws_cal = moe.workspace(c, device=dev)
+        moe.moe_floe_calibrate(c, xc, d_in["w_up"], floe, u_cal, thr, ws_cal)
+        torch.cuda.synchronize(dev)
+        if moe.moe_read_device_status(ws_cal) != moe.OK:
+            raise RuntimeError("device status after the FloE calibration is not OK")
+        del u_cal
+        kept = torch.zeros(cfg.m, dtype=torch.int32, device=dev)
+        floe_idx = torch.zeros((cfg.T, cfg.k), dtype=torch.int32, device=dev)
     tdt = torch.float32 if cfg.dtype == W.F32 else torch.bfloat16
     out = torch.empty((cfg.T, cfg.d), dtype=tdt, device=dev)
     counts = torch.empty(cfg.m + (1 if rep else 0), dtype=torch.int32, device=dev)
@@ -388,6 +418,9 @@ def ours(args):
         if rep:
             moe.moe_layer_forward_replicated(*args_, counts_out=counts, lis_before_out=lis0, lis_after_out=lis,
                                              stream=s)
+        elif floe is not None:
+            moe.moe_layer_forward_floe(c, args_[1], d_in["w_router"], d_in["bias"], d_in["w_gate"], d_in["w_up"],
+                                       w_down_t, thr, args_[10], ws, topk_idx_out=floe_idx, kept_out=kept, stream=s)
         else:
             moe.moe_layer_forward(*args_, counts_out=counts, lis_out=lis, stream=s)
 
@@ -402,9 +435,14 @@ def ours(args):
     st = moe.moe_read_device_status(ws, stream=s)
     if st != moe.OK:
         raise RuntimeError(f"device status after warm-up: {moe.moe_status_string(st)}")
-    cnt = counts.cpu().numpy()
+    if floe is not None:  # the FloE call returns no histogram: the same statistics from its routing
+        cnt = np.bincount(floe_idx.cpu().numpy().ravel(), minlength=cfg.m).astype(np.int32)
+        argmax = int(np.argmax(cnt))
+        max_count, lis_v = int(cnt[argmax]), cfg.m * int(cnt[argmax]) / (cfg.T * cfg.k)
+    else:
+        cnt = counts.cpu().numpy()
+        max_count, argmax, lis_v = moe.unpack_lis(lis)
     active = int((cnt > 0).sum())
-    max_count, argmax, lis_v = moe.unpack_lis(lis)
     ent = cnt[cnt > 0] / cnt.sum()
     entropy = float(-(ent * np.log(ent)).sum())
 
@@ -505,6 +543,15 @@ def ours(args):
             kbps = -(-kb // ks)
             plan_ksplit = -(-kb // kbps)
     costs, layer_flops, layer_bytes = stage_costs(cfg_groups, active, plan_ksplit)
+    if floe is not None:
+        # dense up projection: W_up only, u written in fp32; sparse part: the gate and
+        # down rows of the kept channels, u and the compact h
+        kc = kept.cpu().numpy().astype(np.int64)
+        Tk = cfg.T * cfg.k
+        costs["expert_up"] = (2.0 * cfg.f * cfg.d * Tk, active * cfg.f * cfg.d * 2 + Tk * cfg.d * 2 + Tk * cfg.f * 4)
+        costs["expert_down"] = (4.0 * cfg.d * float(kc.sum()) * max(1.0, Tk / max(active, 1)),
+                                float(kc.sum()) * 2 * cfg.d * 2 + Tk * cfg.f * 8 + Tk * cfg.d * 4)
+        layer_bytes = (cfg.m * cfg.d + active * cfg.f * cfg.d + float(kc.sum()) * 2 * cfg.d) * 2 + 2 * T_bytes(cfg)
     fl, by = costs[dom]
     sec = dom_ms * 1e-3
     long_step = K * ms > 1000.0
@@ -540,6 +587,10 @@ def ours(args):
                            "boundaries",
             "routing": {"lis": lis_v, "max_count": max_count, "heavy_hitter": argmax, "active_experts": active,
                         "reuse_ratio": cfg.T * cfg.k / max(active, 1), "load_entropy": entropy},
+            **({"variant": f"FloE contextual sparsity at target sparsity {floe}: thresholds from a second batch; "
+                           "expert_up = dense u = x W_up^T, expert_down = kept lists + kept gate rows + kept down rows",
+                "kept_channel_fraction": float(kept.cpu().numpy()[kept.cpu().numpy() > 0].mean() / cfg.f)}
+               if floe is not None else {}),
             **({"variant": "R&Q replica dispatch: the heavy-hitter's tasks alternate between it and a replica "
                            "expert m that computes with its bf16 weights; routing.lis is over the m + 1 experts",
                 "lis_before_split": moe.unpack_lis(lis0)[2],

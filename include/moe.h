@@ -208,6 +208,46 @@ MOE_API moe_status_t moe_layer_forward_replicated(
     float* logits_out, int32_t* topk_idx_out, float* topk_w_out, int32_t* dispatch_idx_out, int32_t* counts_out,
     moe_lis_t* lis_before_out, moe_lis_t* lis_after_out, void* ws, size_t ws_bytes, moe_stream_t stream);
 
+/* FloE contextual sparsity ("FloE: On-the-Fly MoE Inference on Memory-constrained
+ * GPU", "Core claim", Sec. 3.2 and Eq. 6). bf16 SwiGLU layers without shared
+ * experts only (MOE_ERR_UNSUPPORTED otherwise). For a task of expert e:
+ * u = x W_up[e]^T; channel j is kept when |u_j| >= thresholds[e]; kept channels
+ * compute g_j = x . W_gate[e][j] and h_j = g_j sigma(g_j) u_j, the others
+ * contribute nothing; y = w * sum over kept j of h_j W_down[e][:, j]. Only the
+ * gate rows and down columns of channels that some task of e keeps are read.
+ *
+ * moe_floe_pack_down: w_down_t [m, f, d] bf16 = W_down transposed per expert
+ * (channel-major, so a kept channel is one contiguous row); a one-time layout. */
+MOE_API moe_status_t moe_floe_pack_down(const moe_config_t* cfg, const void* w_down, void* w_down_t,
+                                        moe_stream_t stream);
+
+/* Per-expert thresholds from a calibration batch (Eq. 6, the empirical CDF of
+ * |up-projection activations| at target sparsity s in [0, 1]): u_scratch
+ * [T_calib, m f] fp32 receives u[t][e f + j] = x_calib[t] . W_up[e][j] for every
+ * expert (tensor cores, fp32 accumulation); thresholds_out [m] fp32 = the
+ * ceil(s n)-th smallest (at least the 1st) of the n = T_calib f values |u| of
+ * each expert, found exactly. ws: moe_workspace_size(cfg) bytes (status word). */
+MOE_API moe_status_t moe_floe_calibrate(const moe_config_t* cfg, const void* x_calib, int32_t T_calib,
+                                        const void* w_up, double sparsity, float* u_scratch, float* thresholds_out,
+                                        void* ws, size_t ws_bytes, moe_stream_t stream);
+
+/* Workspace of moe_layer_forward_floe (host out-parameter). */
+MOE_API moe_status_t moe_floe_workspace_size(const moe_config_t* cfg, size_t* bytes);
+
+/* The layer with FloE sparse experts: route -> histogram/LIS -> permute -> dense
+ * up projection (fp32 u) -> kept-channel lists -> gate rows and down rows of the
+ * kept channels -> combine. thresholds [m] fp32 (device), w_down_t from
+ * moe_floe_pack_down. Optional device outputs: topk_idx_out / topk_w_out
+ * [T, k]; kept_out [m] int32 = channels read per expert; u_out [T k, f] fp32 =
+ * u of each segment row and perm_out [T k] = the task of each row (for checks).
+ * ws: moe_floe_workspace_size() bytes. */
+MOE_API moe_status_t moe_layer_forward_floe(const moe_config_t* cfg, const void* x, const void* w_router,
+                                            const float* bias, const void* w_gate, const void* w_up,
+                                            const void* w_down_t, const float* thresholds, void* out,
+                                            int32_t* topk_idx_out, float* topk_w_out, int32_t* kept_out,
+                                            float* u_out, int32_t* perm_out, void* ws, size_t ws_bytes,
+                                            moe_stream_t stream);
+
 /* Cartesian Product Router (OmniMoE Sec. 2.2, Eq. 8; App. A): lr = log_softmax(x
  * w_row^T), lc = log_softmax(x w_col^T) (fp32); expert (i, j) with flat id
  * i Nc + j scores S = fl32(lr_i + lc_j); idx_out [T, K] = the exact top-K of all

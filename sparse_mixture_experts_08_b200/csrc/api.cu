@@ -866,6 +866,169 @@ moe_status_t moe_layer_forward_replicated(const moe_config_t* cfg, const void* x
   return mark_stage(7, s);
 }
 
+// ------------------------------------------------------------------ FloE contextual sparsity
+struct FloeLayout {
+  size_t u, list, cnt, hc, y, total;
+};
+
+static FloeLayout make_floe_layout(const moe_config_t& c, size_t base) {
+  FloeLayout F;
+  size_t off = base;
+  auto take = [&](size_t bytes) {
+    const size_t o = off;
+    off += align256(bytes);
+    return o;
+  };
+  const size_t Tk = (size_t)c.T * c.k;
+  const size_t nch = (size_t)floe_chunks(c.f);
+  F.u = take(Tk * c.f * 4);
+  F.list = take((size_t)c.m * nch * floe_chunk_size() * 4);
+  F.cnt = take((size_t)c.m * nch * 4);
+  F.hc = take(Tk * c.f * 4);
+  F.y = take((size_t)floe_splits() * Tk * c.d * 4);  // partial outputs of the kept-channel ranges
+  F.total = off;
+  return F;
+}
+
+static moe_status_t check_floe_cfg(const moe_config_t* cfg) {
+  MOE_TRY(check_cfg(cfg));
+  if (cfg->dtype != MOE_BF16 || cfg->act != MOE_SWIGLU || cfg->n_shared != 0) return MOE_ERR_UNSUPPORTED;
+  if (!floe_shape_ok(cfg->d, cfg->f)) return MOE_ERR_UNSUPPORTED;
+  return MOE_OK;
+}
+
+moe_status_t moe_floe_workspace_size(const moe_config_t* cfg, size_t* bytes) {
+  MOE_TRY(check_floe_cfg(cfg));
+  if (!bytes) return MOE_ERR_INVALID_ARG;
+  const Layout L = make_layout(*cfg, make_plan(*cfg));
+  *bytes = make_floe_layout(*cfg, L.total).total;
+  return MOE_OK;
+}
+
+moe_status_t moe_floe_pack_down(const moe_config_t* cfg, const void* w_down, void* w_down_t, moe_stream_t stream) {
+  MOE_TRY(check_floe_cfg(cfg));
+  if (!w_down || !w_down_t || !aligned16(w_down) || !aligned16(w_down_t)) return MOE_ERR_INVALID_ARG;
+  MOE_TRY(check_device());
+  return cuda_status(launch_floe_pack(cfg->m, cfg->d, cfg->f, w_down, w_down_t, (cudaStream_t)stream));
+}
+
+moe_status_t moe_floe_calibrate(const moe_config_t* cfg, const void* x_calib, int32_t T_calib, const void* w_up,
+                                double sparsity, float* u_scratch, float* thresholds_out, void* ws, size_t ws_bytes,
+                                moe_stream_t stream) {
+  MOE_TRY(check_floe_cfg(cfg));
+  const moe_config_t& c = *cfg;
+  if (!x_calib || !w_up || !u_scratch || !thresholds_out || T_calib < 1) return MOE_ERR_INVALID_ARG;
+  if (!(sparsity >= 0.0 && sparsity <= 1.0)) return MOE_ERR_INVALID_ARG;
+  for (const void* p : std::initializer_list<const void*>{x_calib, w_up, (const void*)u_scratch,
+                                                          (const void*)thresholds_out})
+    if (!aligned16(p)) return MOE_ERR_INVALID_ARG;
+  if ((long long)c.m * c.f > (1LL << 30)) return MOE_ERR_UNSUPPORTED;
+  const Layout L = make_layout(c, make_plan(c));
+  MOE_TRY(check_ws(c, ws, ws_bytes, L.total));
+  MOE_TRY(check_device());
+  cudaStream_t s = (cudaStream_t)stream;
+  // u[t][e f + j] = x_calib[t] . W_up[e][j] for every expert: one tensor-core group
+  GemmParams p;
+  std::memset(&p, 0, sizeof(p));
+  fill_common(p, at<int>(ws, L.status));
+  GemmClass& g = p.cls[0];
+  g.n_groups = 1;
+  g.R = c.m * c.f;
+  g.K = c.d;
+  g.ksplit = 1;
+  g.kb_per_split = kblocks(c.d);
+  g.const_rows = T_calib;
+  g.out = u_scratch;
+  g.out_ld = (long long)c.m * c.f;
+  p.n_classes = 1;
+  TcMaps maps;
+  std::memset(&maps, 0, sizeof(maps));
+  maps.a0[0] = {w_up, (long long)c.m * c.f, c.d};
+  maps.a1[0] = maps.a0[0];
+  maps.b[0] = {x_calib, T_calib, c.d};
+  int bn = 16;
+  while (bn < 128 && bn < T_calib) bn <<= 1;
+  MOE_CUDA(launch_tc_gemm(EPI_LOGITS, bn, maps, p, num_sms(), s));
+  return cuda_status(launch_floe_calib(T_calib, c.m, c.f, u_scratch, sparsity, thresholds_out, s));
+}
+
+moe_status_t moe_layer_forward_floe(const moe_config_t* cfg, const void* x, const void* w_router, const float* bias,
+                                    const void* w_gate, const void* w_up, const void* w_down_t,
+                                    const float* thresholds, void* out, int32_t* topk_idx_out, float* topk_w_out,
+                                    int32_t* kept_out, float* u_out, int32_t* perm_out, void* ws, size_t ws_bytes,
+                                    moe_stream_t stream) {
+  MOE_TRY(check_floe_cfg(cfg));
+  const moe_config_t& c = *cfg;
+  if (!x || !w_router || !w_gate || !w_up || !w_down_t || !thresholds || !out) return MOE_ERR_INVALID_ARG;
+  for (const void* p : std::initializer_list<const void*>{
+           x, w_router, (const void*)bias, w_gate, w_up, w_down_t, (const void*)thresholds, out,
+           (const void*)topk_idx_out, (const void*)topk_w_out, (const void*)kept_out, (const void*)u_out,
+           (const void*)perm_out})
+    if (p && !aligned16(p)) return MOE_ERR_INVALID_ARG;
+  const Plan pl = make_plan(c);
+  const Layout L = make_layout(c, pl);
+  const FloeLayout F = make_floe_layout(c, L.total);
+  MOE_TRY(check_ws(c, ws, ws_bytes, F.total));
+  MOE_TRY(check_device());
+  cudaStream_t s = (cudaStream_t)stream;
+  int* status = at<int>(ws, L.status);
+  float* logits = at<float>(ws, L.logits);
+  int32_t* idx = topk_idx_out ? topk_idx_out : at<int32_t>(ws, L.idx);
+  float* w = topk_w_out ? topk_w_out : at<float>(ws, L.w);
+  int32_t* offsets = at<int32_t>(ws, L.offsets);
+  int32_t* perm = at<int32_t>(ws, L.perm);
+  int32_t* inv_perm = at<int32_t>(ws, L.inv_perm);
+  float* w_perm = at<float>(ws, L.w_perm);
+  int32_t* start = at<int32_t>(ws, L.start);
+  void* x_perm = at<void>(ws, L.x_perm);
+  float* u = at<float>(ws, F.u);
+  float* y = at<float>(ws, F.y);
+  const long long Tk = (long long)c.T * c.k;
+  // route and sort as in moe_layer_forward (stages 0-4)
+  MOE_TRY(mark_stage(0, s));
+  MOE_TRY(run_router(c, x, w_router, bias, logits, status, s));
+  MOE_TRY(mark_stage(1, s));
+  MOE_CUDA(launch_topk_softmax(c.T, c.m, c.k, c.renormalize, logits, idx, w, s));
+  MOE_TRY(mark_stage(2, s));
+  MOE_CUDA(launch_route_index(1, c.T, c.k, c.m, idx, at<int32_t>(ws, L.counts), offsets, at<moe_lis_t>(ws, L.lis),
+                              start, status, s));
+  MOE_CUDA(launch_rank(c.T, c.k, c.m, idx, offsets, start, w, perm, inv_perm, w_perm, status, s));
+  MOE_TRY(mark_stage(3, s));
+  MOE_CUDA(launch_permute_rows(c.dtype, (int)Tk, c.k, c.d, x, inv_perm, x_perm, s));
+  MOE_TRY(mark_stage(4, s));
+  // dense up projection u = x W_up^T per segment (fp32, tensor cores)
+  GemmParams up;
+  std::memset(&up, 0, sizeof(up));
+  fill_common(up, status);
+  GemmClass& g = up.cls[0];
+  g.n_groups = c.m;
+  g.R = c.f;
+  g.K = c.d;
+  g.ksplit = 1;
+  g.kb_per_split = kblocks(c.d);
+  g.seg_off = offsets;
+  g.max_row = (int)Tk;
+  g.out = u;
+  g.out_ld = c.f;
+  up.n_classes = 1;
+  TcMaps mu;
+  std::memset(&mu, 0, sizeof(mu));
+  mu.a0[0] = {w_up, (long long)c.m * c.f, c.d};
+  mu.a1[0] = mu.a0[0];
+  mu.b[0] = {x_perm, Tk, c.d};
+  MOE_CUDA(launch_tc_gemm(EPI_LOGITS, tc_pick_bn(EPI_LOGITS, (double)Tk / c.m), mu, up, num_sms(), s));
+  MOE_TRY(mark_stage(5, s));
+  // kept channels, gate rows and down rows of the kept channels only
+  MOE_CUDA(launch_floe_sparse_ffn(c.m, c.d, c.f, offsets, x_perm, w_gate, w_down_t, u, thresholds,
+                                  at<int32_t>(ws, F.list), at<int32_t>(ws, F.cnt), at<float>(ws, F.hc), w_perm, y,
+                                  Tk * c.d, kept_out, status, s));
+  MOE_TRY(mark_stage(6, s));
+  MOE_CUDA(launch_combine(c.dtype, c.T, c.d, c.k, floe_splits(), y, Tk * c.d, inv_perm, 0, nullptr, 0, out, s));
+  if (u_out) MOE_CUDA(cudaMemcpyAsync(u_out, u, (size_t)Tk * c.f * 4, cudaMemcpyDeviceToDevice, s));
+  if (perm_out) MOE_CUDA(cudaMemcpyAsync(perm_out, perm, (size_t)Tk * 4, cudaMemcpyDeviceToDevice, s));
+  return mark_stage(7, s);
+}
+
 // ------------------------------------------------------------------ status helpers
 moe_status_t moe_read_device_status(void* ws, moe_stream_t stream, moe_status_t* out) {
   if (!ws || !out) return MOE_ERR_INVALID_ARG;

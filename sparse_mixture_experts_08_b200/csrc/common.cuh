@@ -206,6 +206,17 @@ cudaError_t launch_route_scatter(int dtype, int T, int k, int m, int d, const in
 cudaError_t launch_replica_split(int T, int k, int m, const int32_t* idx, const int32_t* offsets,
                                  const int32_t* inv_perm, const moe_lis_t* lis_in, int32_t* idx_out, int32_t* gmap,
                                  int32_t* counts_out, moe_lis_t* lis_out, int* status, cudaStream_t s);
+// FloE contextual sparsity (csrc/floe.cu)
+cudaError_t launch_floe_pack(int m, int d, int f, const void* w, void* w_t, cudaStream_t s);
+cudaError_t launch_floe_calib(int Tc, int m, int f, const float* u, double sparsity, float* thr, cudaStream_t s);
+cudaError_t launch_floe_sparse_ffn(int m, int d, int f, const int32_t* offsets, const void* x_perm,
+                                   const void* w_gate, const void* w_down_t, const float* u, const float* thr,
+                                   int32_t* list, int32_t* cnt, float* hc, const float* row_w, float* y,
+                                   long long y_split, int32_t* kept_out, int* status, cudaStream_t s);
+int floe_chunks(int f);
+int floe_chunk_size();
+int floe_splits();                 // partial outputs of the sparse down projection (summed by the combine)
+bool floe_shape_ok(int d, int f);  // d <= 8192, f <= 65536
 cudaError_t launch_rank(int T, int k, int m, const int32_t* idx, const int32_t* offsets, const int32_t* start,
                         const float* task_w, int32_t* perm, int32_t* inv_perm, float* w_perm, int* status,
                         cudaStream_t s);

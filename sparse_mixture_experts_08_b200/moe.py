@@ -31,7 +31,8 @@ EXPORTS = ["moe_workspace_size", "moe_atomic_workspace_size", "moe_route", "moe_
            "moe_grouped_ffn", "moe_shared_ffn", "moe_combine", "moe_layer_forward", "moe_atomic_route",
            "moe_atomic_experts", "moe_atomic_forward", "moe_read_device_status", "moe_status_string",
            "moe_debug_set_wait_limit_ns", "moe_set_stage_events", "moe_launch_count", "moe_route_static",
-           "moe_replica_split", "moe_layer_forward_replicated"]
+           "moe_replica_split", "moe_layer_forward_replicated", "moe_floe_pack_down", "moe_floe_calibrate",
+           "moe_floe_workspace_size", "moe_layer_forward_floe"]
 
 
 class MoEConfig(ctypes.Structure):
@@ -75,6 +76,10 @@ def lib() -> ctypes.CDLL:
             "moe_combine": [P, P, P, P, P, P],
             "moe_layer_forward": [P, P, P, P, P, P, P, P, P, P, P, P, P, P, P, P, P, S, P],
             "moe_replica_split": [P, P, P, P, P, P, P, P, P, S, P],
+            "moe_floe_pack_down": [P, P, P, P],
+            "moe_floe_calibrate": [P, P, ctypes.c_int32, P, ctypes.c_double, P, P, P, S, P],
+            "moe_floe_workspace_size": [P, P],
+            "moe_layer_forward_floe": [P, P, P, P, P, P, P, P, P, P, P, P, P, P, P, S, P],
             "moe_layer_forward_replicated": [P, P, P, P, P, P, P, P, P, P, P, P, P, P, P, P, P, P, P, S, P],
             "moe_atomic_route": [P, P, P, P, P, P, P, P, P, S, P],
             "moe_atomic_experts": [P, P, P, P, P, P, P, P, S, P],
@@ -205,6 +210,35 @@ def moe_layer_forward_replicated(cfg, x, w_router, bias, w_gate, w_up, w_down, w
         ctypes.byref(cfg), _p(x), _p(w_router), _p(bias), _p(w_gate), _p(w_up), _p(w_down), _p(ws_gate),
         _p(ws_up), _p(ws_down), _p(out), _p(logits_out), _p(topk_idx_out), _p(topk_w_out), _p(dispatch_idx_out),
         _p(counts_out), _p(lis_before_out), _p(lis_after_out), _p(ws), ws.numel(), _stream(stream)))
+
+
+def moe_floe_pack_down(cfg, w_down, w_down_t, stream=None):
+    _check("moe_floe_pack_down", lib().moe_floe_pack_down(ctypes.byref(cfg), _p(w_down), _p(w_down_t),
+                                                          _stream(stream)))
+
+
+def moe_floe_calibrate(cfg, x_calib, w_up, sparsity, u_scratch, thresholds_out, ws, stream=None):
+    _check("moe_floe_calibrate", lib().moe_floe_calibrate(ctypes.byref(cfg), _p(x_calib), int(x_calib.shape[0]),
+                                                          _p(w_up), float(sparsity), _p(u_scratch),
+                                                          _p(thresholds_out), _p(ws), ws.numel(), _stream(stream)))
+
+
+def moe_floe_workspace_size(cfg) -> int:
+    n = ctypes.c_size_t(0)
+    _check("moe_floe_workspace_size", lib().moe_floe_workspace_size(ctypes.byref(cfg), ctypes.byref(n)))
+    return n.value
+
+
+def moe_layer_forward_floe(cfg, x, w_router, bias, w_gate, w_up, w_down_t, thresholds, out, ws, topk_idx_out=None,
+                           topk_w_out=None, kept_out=None, u_out=None, perm_out=None, stream=None):
+    _check("moe_layer_forward_floe", lib().moe_layer_forward_floe(
+        ctypes.byref(cfg), _p(x), _p(w_router), _p(bias), _p(w_gate), _p(w_up), _p(w_down_t), _p(thresholds),
+        _p(out), _p(topk_idx_out), _p(topk_w_out), _p(kept_out), _p(u_out), _p(perm_out), _p(ws), ws.numel(),
+        _stream(stream)))
+
+
+def floe_workspace(cfg, device="cuda") -> torch.Tensor:
+    return torch.zeros(max(moe_floe_workspace_size(cfg), 256), dtype=torch.uint8, device=device)
 
 
 def moe_atomic_route(cfg, x, w_row, w_col, row_logp_out, col_logp_out, idx_out, g_out, ws, stream=None):

@@ -162,3 +162,23 @@ def test_replica_entry_points_validate_on_the_host():
     assert n1.value > n0.value
     assert lib.moe_layer_forward_replicated(ctypes.byref(c), a, a, None, a, a, a, None, None, None, a, None, None,
                                             None, None, None, None, None, ws, n0.value, None) == moe.ERR_WORKSPACE
+
+
+def test_floe_entry_points_validate_on_the_host():
+    lib = moe.moe.lib()
+    a = _fake(1 << 24)
+    ok = MoEConfig(16, 256, 320, 4, 2, 0, 0, moe.BF16, moe.SWIGLU, 0)
+    n = ctypes.c_size_t(0)
+    assert lib.moe_floe_workspace_size(ctypes.byref(ok), ctypes.byref(n)) == moe.OK and n.value > 0
+    for bad in (MoEConfig(16, 256, 320, 4, 2, 0, 0, moe.F32, moe.SWIGLU, 0),   # bf16 only
+                MoEConfig(16, 256, 320, 4, 2, 0, 0, moe.BF16, moe.RELU, 0),    # SwiGLU only
+                MoEConfig(16, 256, 320, 4, 2, 1, 64, moe.BF16, moe.SWIGLU, 0)):  # no shared experts
+        assert lib.moe_floe_workspace_size(ctypes.byref(bad), ctypes.byref(n)) == moe.ERR_UNSUPPORTED
+    assert lib.moe_floe_calibrate(ctypes.byref(ok), a, 8, a, ctypes.c_double(1.5), a, a, a, 1 << 30, None) == \
+        moe.ERR_INVALID_ARG  # sparsity outside [0, 1]
+    assert lib.moe_floe_calibrate(ctypes.byref(ok), a, 0, a, ctypes.c_double(0.9), a, a, a, 1 << 30, None) == \
+        moe.ERR_INVALID_ARG  # no calibration tokens
+    assert lib.moe_layer_forward_floe(ctypes.byref(ok), a, a, None, a, a, a, None, a, None, None, None, None, None,
+                                      a, 1 << 30, None) == moe.ERR_INVALID_ARG  # thresholds missing
+    assert lib.moe_layer_forward_floe(ctypes.byref(ok), a, a, None, a, a, a, a, a, None, None, None, None, None,
+                                      a, n.value - 256, None) == moe.ERR_WORKSPACE
