@@ -305,7 +305,8 @@ MOE_API moe_status_t moe_debug_set_wait_limit_ns(uint64_t ns);
  * stream at its stage boundaries, in order: 0 start, 1 router logits, 2 top-k,
  * 3 histogram/LIS/ranks, 4 row permutation, 5 up projection, 6 down projection,
  * 7 combine (n <= 8; extra stages are not recorded); moe_atomic_forward records
- * 0 start, 1 router projections, 2 grid top-K, 3 expert coefficients, 4 assembly;
+ * 0 start, 1 router projections, 2 grid top-K, 3 and 4 after the atomic-expert FFN (coefficients and
+ * assembly are one launch);
  * moe_layer_forward_replicated records the stages of moe_layer_forward (3 is
  * after both sorts and the split).
  * A NULL entry skips that

@@ -621,7 +621,7 @@ static moe_status_t check_atomic_cfg(const moe_atomic_config_t* c) {
 
 struct AtomicPlan {
   int ksplit, kbps;
-  size_t status, zr, zc, idx, g, coef, total;
+  size_t status, zr, zc, idx, g, coef, bar, total;
 };
 
 static AtomicPlan make_atomic_plan(const moe_atomic_config_t& c) {
@@ -643,6 +643,7 @@ static AtomicPlan make_atomic_plan(const moe_atomic_config_t& c) {
   p.idx = take((size_t)c.T * c.K * 4);
   p.g = take((size_t)c.T * c.K * 4);
   p.coef = take((size_t)c.T * c.K * 4);
+  p.bar = take(256);  // grid-barrier word of the experts kernel
   p.total = off;
   return p;
 }
@@ -686,7 +687,7 @@ static moe_status_t atomic_route_impl(const moe_atomic_config_t& c, const Atomic
   MOE_CUDA(launch_tc_gemm(EPI_LOGITS, bn, maps, p, num_sms(), s));
   if (stage_marks) MOE_TRY(mark_stage(1, s));
   MOE_CUDA(launch_atomic_select(c.T, c.Nr, c.Nc, c.K, P.ksplit, zr, (long long)c.T * c.Nr, zc, (long long)c.T * c.Nc,
-                                lr_out, lc_out, idx, g, status, s));
+                                lr_out, lc_out, idx, g, status, at<unsigned>(ws, P.bar), s));
   if (stage_marks) MOE_TRY(mark_stage(2, s));
   return MOE_OK;
 }
@@ -721,7 +722,8 @@ moe_status_t moe_atomic_experts(const moe_atomic_config_t* cfg, const void* x, c
   if (ws_bytes < P.total) return MOE_ERR_WORKSPACE;
   MOE_TRY(check_device());
   return cuda_status(launch_atomic_experts(c.T, c.d, c.K, c.act, x, w_in, w_out, idx, g, at<float>(ws, P.coef), out,
-                                           (long long)c.Nr * c.Nc, at<int>(ws, P.status), (cudaStream_t)stream));
+                                           (long long)c.Nr * c.Nc, at<unsigned>(ws, P.bar), false, g_wait_limit_ns,
+                                           at<int>(ws, P.status), (cudaStream_t)stream));
 }
 
 moe_status_t moe_atomic_forward(const moe_atomic_config_t* cfg, const void* x, const void* w_row, const void* w_col,
@@ -741,8 +743,11 @@ moe_status_t moe_atomic_forward(const moe_atomic_config_t* cfg, const void* x, c
   float* g = g_out ? g_out : at<float>(ws, P.g);
   MOE_TRY(mark_stage(0, s));
   MOE_TRY(atomic_route_impl(c, P, x, w_row, w_col, nullptr, nullptr, idx, g, ws, s, true));
+  // the select kernel cleared the barrier word; the experts kernel is one launch
   MOE_CUDA(launch_atomic_experts(c.T, c.d, c.K, c.act, x, w_in, w_out, idx, g, at<float>(ws, P.coef), out,
-                                 (long long)c.Nr * c.Nc, at<int>(ws, P.status), s, true));
+                                 (long long)c.Nr * c.Nc, at<unsigned>(ws, P.bar), true, g_wait_limit_ns,
+                                 at<int>(ws, P.status), s));
+  MOE_TRY(mark_stage(3, s));
   return mark_stage(4, s);
 }
 

@@ -146,8 +146,11 @@ __global__ void __launch_bounds__(SEL_THREADS, 1)
     atomic_select_kernel(int T, int Nr, int Nc, int K, int ksplit, const float* __restrict__ zr, long long zr_split,
                          const float* __restrict__ zc, long long zc_split, float* __restrict__ lr_out,
                          float* __restrict__ lc_out, int32_t* __restrict__ idx_out, float* __restrict__ g_out,
-                         int* status) {
+                         int* status, unsigned* bar_reset) {
   __shared__ float lr[SEL_MAX_SIDE], lc[SEL_MAX_SIDE];
+  // the next kernel's grid barrier counts from zero: it passes griddepcontrol.wait
+  // only after this grid has completed, so clearing the word here is enough
+  if (bar_reset && blockIdx.x == 0 && threadIdx.x == 0) *bar_reset = 0u;
   __shared__ uint64_t buf[2][16 * 64];  // merge buffers: rows, columns (candidates reuse rows')
   __shared__ Lse red_r[32], red_c[32];
   __shared__ double lse_s[2];
@@ -391,153 +394,182 @@ __global__ void __launch_bounds__(SEL_THREADS, 1)
 
 cudaError_t launch_atomic_select(int T, int Nr, int Nc, int K, int ksplit, const float* zr, long long zr_split,
                                  const float* zc, long long zc_split, float* lr_out, float* lc_out, int32_t* idx,
-                                 float* g, int* status, cudaStream_t s) {
+                                 float* g, int* status, unsigned* bar_reset, cudaStream_t s) {
   launch_k(atomic_select_kernel, T, SEL_THREADS, 0, s, T, Nr, Nc, K, ksplit, zr, zr_split, zc, zc_split, lr_out,
-           lc_out, idx, g, status);
+           lc_out, idx, g, status, bar_reset);
   count_launch();
   return cudaGetLastError();
 }
 
 // ------------------------------------------------------------------ assembly
-// coef[t, s] = g[t, s] * act(x_t . w_in[idx[t, s]]). Block (task group, token):
-// eight warps, one task each, over the row in windows of 4096 elements. Each lane
-// issues its sixteen 16-byte loads of the expert row before the window of x_t is
-// staged in shared memory, so the gathers of all tasks are in flight together;
-// fp32 dot, shuffle-tree reduction.
-constexpr int COEF_WARPS = 8, COEF_WIN = 512;  // window: 512 chunks of 8 bf16
-__global__ void __launch_bounds__(COEF_WARPS * 32)
-    atomic_coef_kernel(int T, int d, int K, int act, const uint4* __restrict__ x, const uint4* __restrict__ w_in,
-                       const int32_t* __restrict__ idx, const float* __restrict__ g, float* __restrict__ coef,
-                       long long n_experts, int* status) {
-  __shared__ uint4 xs[COEF_WIN];
+constexpr int ASM_GROUPS = 4, ASM_BATCH = 16;  // phase 2: slot groups per 8 columns, loads per batch
+
+// The atomic-expert FFN (OmniMoE Eq. 4) in one cooperative launch, one block per SM:
+//  phase 1, one warp per task (t, s): coef[t, s] = g[t, s] act(x_t . w_in[idx[t, s]]),
+//    fp32 FMAs over each lane's 16-byte chunks in ascending order then a shuffle
+//    tree; the warp also prefetches the task's w_out row into L2 for phase 2;
+//  a grid-wide barrier (bounded: on expiry it records MOE_ERR_TIMEOUT and carries on);
+//  phase 2, four lanes per 8 output columns: lane group j sums slots j, j + 4, ...
+//    in order, and out[t, c..c+7] = ((group 0 + group 1) + group 2) + group 3,
+//    rounded to bf16, so the result is the same on every run.
+constexpr int AX_THREADS = 256;
+__device__ __forceinline__ void prefetch_l2(const void* p) {
+  asm volatile("prefetch.global.L2 [%0];" ::"l"(p));
+}
+
+__global__ void __launch_bounds__(AX_THREADS)
+    atomic_experts_kernel(int T, int d, int K, int act, const uint4* __restrict__ x, const uint4* __restrict__ w_in,
+                          const uint4* __restrict__ w_out, const int32_t* __restrict__ idx,
+                          const float* __restrict__ g, float* __restrict__ coef, uint4* __restrict__ out,
+                          long long n_experts, unsigned* bar, unsigned long long limit_ns, int* status) {
   pdl_launch_dependents();
   pdl_wait();
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  const long long t = blockIdx.y;
-  const int sl = blockIdx.x * COEF_WARPS + warp;
-  const bool has = sl < K;
-  const long long task = t * K + sl;
-  const long long e = has ? (long long)idx[task] : 0;
-  const bool ok = has && e >= 0 && e < n_experts;
-  if (has && !ok && lane == 0) {
-    set_status(status, MOE_ERR_DEVICE_INDEX);
-    coef[task] = 0.f;
-  }
+  const int lane = threadIdx.x & 31;
+  const long long gwarp = ((long long)blockIdx.x * AX_THREADS + threadIdx.x) >> 5;
+  const long long nwarps = (long long)gridDim.x * (AX_THREADS / 32);
   const int chunks = d / 8;
-  const uint4* wr = w_in + (ok ? e : 0) * chunks;
-  float s = 0.f;
-  for (int w0 = 0; w0 < chunks; w0 += COEF_WIN) {
-    const int wn = min(COEF_WIN, chunks - w0);
-    uint4 b[COEF_WIN / 32];
-    if (ok) {
-#pragma unroll
-      for (int u = 0; u < COEF_WIN / 32; ++u) {
-        const int c = lane + 32 * u;
-        if (c < wn) b[u] = wr[w0 + c];
+  const long long tasks = (long long)T * K;
+  // ---- phase 1: coef[t, s] = g[t, s] act(x_t . w_in[idx[t, s]])
+  for (long long task = gwarp; task < tasks; task += nwarps) {
+    const long long t = task / K;
+    const long long e = idx[task];
+    if (e < 0 || e >= n_experts) {
+      if (lane == 0) {
+        set_status(status, MOE_ERR_DEVICE_INDEX);
+        coef[task] = 0.f;
       }
+      continue;
     }
-    __syncthreads();  // the previous window is consumed
-    for (int c = threadIdx.x; c < wn; c += COEF_WARPS * 32) xs[c] = x[t * chunks + w0 + c];
-    __syncthreads();
-    if (ok) {
+    const char* po = reinterpret_cast<const char*>(w_out + e * chunks);
+    for (int b = lane * 128; b < d * 2; b += 32 * 128) prefetch_l2(po + b);
+    const uint4* wr = w_in + e * chunks;
+    const uint4* xr = x + t * chunks;
+    float sacc = 0.f;
+    for (int c0 = lane; c0 < chunks; c0 += 32 * 8) {
+      uint4 av[8], bv[8];
 #pragma unroll
-      for (int u = 0; u < COEF_WIN / 32; ++u) {
-        const int c = lane + 32 * u;
-        if (c >= wn) break;
-        const uint4 a = xs[c];
-        const __nv_bfloat162* pa = reinterpret_cast<const __nv_bfloat162*>(&a);
-        const __nv_bfloat162* pb = reinterpret_cast<const __nv_bfloat162*>(&b[u]);
+      for (int u = 0; u < 8; ++u) {
+        const int c = c0 + 32 * u;
+        if (c < chunks) {
+          av[u] = xr[c];
+          bv[u] = wr[c];
+        }
+      }
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        if (c0 + 32 * u >= chunks) break;
+        const __nv_bfloat162* pa = reinterpret_cast<const __nv_bfloat162*>(&av[u]);
+        const __nv_bfloat162* pb = reinterpret_cast<const __nv_bfloat162*>(&bv[u]);
 #pragma unroll
         for (int h = 0; h < 4; ++h) {
           const float2 fa = __bfloat1622float2(pa[h]), fb = __bfloat1622float2(pb[h]);
-          s = fmaf(fa.x, fb.x, s);
-          s = fmaf(fa.y, fb.y, s);
+          sacc = fmaf(fa.x, fb.x, sacc);
+          sacc = fmaf(fa.y, fb.y, sacc);
         }
       }
     }
-  }
-  if (!ok) return;
 #pragma unroll
-  for (int o = 16; o; o >>= 1) s += __shfl_xor_sync(FULL, s, o);
-  if (lane == 0) {
-    const float sg = 1.f / (1.f + expf(-s));
-    coef[task] = g[task] * (act == MOE_ATOMIC_SILU ? s * sg : sg);
+    for (int o = 16; o; o >>= 1) sacc += __shfl_xor_sync(0xffffffffu, sacc, o);
+    if (lane == 0) {
+      const float sg = 1.f / (1.f + expf(-sacc));
+      coef[task] = g[task] * (act == MOE_ATOMIC_SILU ? sacc * sg : sg);
+    }
   }
-}
-
-// out[t, c..c+7] = sum_s coef[t, s] w_out[idx[t, s], c..c+7]. A block handles one
-// token and 64 column chunks of 8; its four thread groups take every fourth slot
-// (loads issued sixteen at a time) and their partial sums are added in group order,
-// so the result is the same on every run.
-constexpr int ASM_GROUPS = 4, ASM_CHUNKS = 64, ASM_BATCH = 16;
-__global__ void atomic_assemble_kernel(int T, int d, int K, const uint4* __restrict__ w_out,
-                                       const int32_t* __restrict__ idx, const float* __restrict__ coef,
-                                       uint4* __restrict__ out, long long n_experts) {
-  __shared__ float part[ASM_GROUPS][ASM_CHUNKS][8];
-  pdl_launch_dependents();
-  pdl_wait();
-  const int chunks = d / 8;
-  const int cblocks = (chunks + ASM_CHUNKS - 1) / ASM_CHUNKS;
-  const long long t = blockIdx.x / cblocks;
-  const int cl = threadIdx.x % ASM_CHUNKS, grp = threadIdx.x / ASM_CHUNKS;
-  const int c = (blockIdx.x % cblocks) * ASM_CHUNKS + cl;
-  float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-  if (c < chunks) {
-    for (int s0 = grp; s0 < K; s0 += ASM_GROUPS * ASM_BATCH) {
-      uint4 v[ASM_BATCH];
-      float cf[ASM_BATCH];
+  // ---- grid-wide barrier (every block is resident: cooperative launch, one per SM)
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    __threadfence();
+    atomicAdd(bar, 1u);
+    const unsigned long long t0 = globaltimer_ns();
+    while (*reinterpret_cast<volatile unsigned*>(bar) < gridDim.x) {
+      if (globaltimer_ns() - t0 > limit_ns) {
+        set_status(status, MOE_ERR_TIMEOUT);
+        break;
+      }
+    }
+    __threadfence();
+  }
+  __syncthreads();
+  // ---- phase 2: out[t, c..c+7] = sum_s coef[t, s] w_out[idx[t, s], c..c+7]
+  const long long units4 = (long long)T * chunks * ASM_GROUPS;
+  for (long long qb = gwarp * 32; qb < units4; qb += nwarps * 32) {  // warp-aligned: shuffles see all lanes
+    const long long q = qb + lane;
+    const bool valid = q < units4;
+    const int grp = (int)(q & (ASM_GROUPS - 1));
+    const long long unit = q / ASM_GROUPS;
+    const long long t = unit / chunks;
+    const int c = (int)(unit - t * chunks);
+    float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+    if (valid) {
+      for (int s0 = grp; s0 < K; s0 += ASM_GROUPS * ASM_BATCH) {
+        uint4 v[ASM_BATCH];
+        float cf[ASM_BATCH];
 #pragma unroll
-      for (int u = 0; u < ASM_BATCH; ++u) {
-        const int sl = s0 + ASM_GROUPS * u;
-        cf[u] = 0.f;
-        if (sl < K) {
-          const long long e = idx[t * K + sl];
-          if (e >= 0 && e < n_experts) {
-            cf[u] = coef[t * K + sl];
-            v[u] = w_out[e * chunks + c];
+        for (int u = 0; u < ASM_BATCH; ++u) {
+          const int sl = s0 + ASM_GROUPS * u;
+          cf[u] = 0.f;
+          if (sl < K) {
+            const long long e = idx[t * K + sl];
+            if (e >= 0 && e < n_experts) {
+              cf[u] = coef[t * K + sl];
+              v[u] = w_out[e * chunks + c];
+            }
+          }
+        }
+#pragma unroll
+        for (int u = 0; u < ASM_BATCH; ++u) {
+          if (cf[u] == 0.f) continue;
+          const __nv_bfloat162* pv = reinterpret_cast<const __nv_bfloat162*>(&v[u]);
+#pragma unroll
+          for (int h = 0; h < 4; ++h) {
+            const float2 f = __bfloat1622float2(pv[h]);
+            acc[2 * h] = fmaf(cf[u], f.x, acc[2 * h]);
+            acc[2 * h + 1] = fmaf(cf[u], f.y, acc[2 * h + 1]);
           }
         }
       }
-#pragma unroll
-      for (int u = 0; u < ASM_BATCH; ++u) {
-        if (cf[u] == 0.f) continue;
-        const __nv_bfloat162* pv = reinterpret_cast<const __nv_bfloat162*>(&v[u]);
-#pragma unroll
-        for (int h = 0; h < 4; ++h) {
-          const float2 f = __bfloat1622float2(pv[h]);
-          acc[2 * h] = fmaf(cf[u], f.x, acc[2 * h]);
-          acc[2 * h + 1] = fmaf(cf[u], f.y, acc[2 * h + 1]);
-        }
-      }
     }
-  }
+    float r[8];
 #pragma unroll
-  for (int h = 0; h < 8; ++h) part[grp][cl][h] = acc[h];
-  __syncthreads();
-  if (grp == 0 && c < chunks) {
+    for (int h = 0; h < 8; ++h) {  // ((group 0 + group 1) + group 2) + group 3, in lanes 4u .. 4u + 3
+      const float b1 = __shfl_down_sync(0xffffffffu, acc[h], 1);
+      const float b2 = __shfl_down_sync(0xffffffffu, acc[h], 2);
+      const float b3 = __shfl_down_sync(0xffffffffu, acc[h], 3);
+      r[h] = ((acc[h] + b1) + b2) + b3;
+    }
+    if (valid && grp == 0) {
+      uint4 o;
+      __nv_bfloat162* po2 = reinterpret_cast<__nv_bfloat162*>(&o);
 #pragma unroll
-    for (int h = 0; h < 8; ++h) acc[h] = ((part[0][cl][h] + part[1][cl][h]) + part[2][cl][h]) + part[3][cl][h];
-    uint4 o;
-    __nv_bfloat162* po = reinterpret_cast<__nv_bfloat162*>(&o);
-#pragma unroll
-    for (int h = 0; h < 4; ++h) po[h] = __floats2bfloat162_rn(acc[2 * h], acc[2 * h + 1]);
-    out[t * chunks + c] = o;
+      for (int h = 0; h < 4; ++h) po2[h] = __floats2bfloat162_rn(r[2 * h], r[2 * h + 1]);
+      out[t * chunks + c] = o;
+    }
   }
 }
 
 cudaError_t launch_atomic_experts(int T, int d, int K, int act, const void* x, const void* w_in, const void* w_out,
                                   const int32_t* idx, const float* g, float* coef, void* out, long long n_experts,
-                                  int* status, cudaStream_t s, bool stage_marks) {
-  launch_k(atomic_coef_kernel, dim3((K + COEF_WARPS - 1) / COEF_WARPS, T), COEF_WARPS * 32, 0, s, T, d, K, act,
-           (const uint4*)x, (const uint4*)w_in, idx, g, coef, n_experts, status);
+                                  unsigned* bar, bool bar_zeroed, unsigned long long limit_ns, int* status,
+                                  cudaStream_t s) {
+  if (!bar_zeroed) {
+    cudaError_t e = cudaMemsetAsync(bar, 0, sizeof(unsigned), s);
+    if (e != cudaSuccess) return e;
+  }
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(num_sms());  // one block per SM: all resident, as the grid barrier needs
+  cfg.blockDim = dim3(AX_THREADS);
+  cfg.stream = s;
+  cudaLaunchAttribute attr[2];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  attr[1].id = cudaLaunchAttributeCooperative;
+  attr[1].val.cooperative = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 2;
+  cudaError_t e = cudaLaunchKernelEx(&cfg, atomic_experts_kernel, T, d, K, act, (const uint4*)x, (const uint4*)w_in,
+                                     (const uint4*)w_out, idx, g, coef, (uint4*)out, n_experts, bar, limit_ns, status);
   count_launch();
-  cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  if (stage_marks && (e = mark_stage_event(3, s)) != cudaSuccess) return e;
-  const int cblocks = (d / 8 + ASM_CHUNKS - 1) / ASM_CHUNKS;
-  launch_k(atomic_assemble_kernel, (unsigned)(T * cblocks), ASM_GROUPS * ASM_CHUNKS, 0, s, T, d, K,
-           (const uint4*)w_out, idx, coef, (uint4*)out, n_experts);
-  count_launch();
   return cudaGetLastError();
 }
 

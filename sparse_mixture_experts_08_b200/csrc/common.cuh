@@ -231,10 +231,13 @@ cudaError_t launch_reduce_splits(long long n, int ksplit, const float* in, long 
 // Atomic experts
 cudaError_t launch_atomic_select(int T, int Nr, int Nc, int K, int ksplit, const float* zr, long long zr_split,
                                  const float* zc, long long zc_split, float* lr_out, float* lc_out, int32_t* idx,
-                                 float* g, int* status, cudaStream_t s);
+                                 float* g, int* status, unsigned* bar_reset, cudaStream_t s);
+// coef and assembly in one cooperative launch with a grid barrier on `bar` (zeroed
+// by the preceding select kernel when bar_zeroed, else by a memset here)
 cudaError_t launch_atomic_experts(int T, int d, int K, int act, const void* x, const void* w_in, const void* w_out,
                                   const int32_t* idx, const float* g, float* coef, void* out, long long n_experts,
-                                  int* status, cudaStream_t s, bool stage_marks = false);
+                                  unsigned* bar, bool bar_zeroed, unsigned long long limit_ns, int* status,
+                                  cudaStream_t s);
 // Records the profiling hook's event i (moe_set_stage_events) on `s`, if one is set.
 cudaError_t mark_stage_event(int i, cudaStream_t s);
 

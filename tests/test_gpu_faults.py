@@ -108,3 +108,33 @@ def test_layer_forward_after_errors_is_exact_again():
     assert moe.moe_read_device_status(ws) == moe.OK
     r = O.layer_forward(cfg, inp, logits_in=host(lg))
     assert token_rel_err(out_f64(out), r["out"]) <= TOL[W.BF16]
+
+
+def test_atomic_grid_barrier_times_out_and_recovers():
+    # the atomic-expert FFN is one cooperative launch with a grid-wide barrier; with a
+    # 1 ns limit the barrier gives up (MOE_ERR_TIMEOUT) instead of spinning, and the next
+    # call with the default limit is exact again
+    cfg = W.AtomicWorkload("atomic_fault", 93, T=4, d=256, Nr=64, Nc=64, K=16, act=W.ACT_SILU)
+    inp = W.make_atomic_inputs(cfg)
+    c = moe.make_atomic_config(cfg.T, cfg.d, cfg.Nr, cfg.Nc, cfg.K, cfg.act)
+    ws = moe.workspace(c)
+    d = device_inputs(inp)
+    idx = torch.empty((cfg.T, cfg.K), dtype=torch.int32, device="cuda")
+    g = torch.empty((cfg.T, cfg.K), dtype=torch.float32, device="cuda")
+    moe.moe_atomic_route(c, d["x"], d["w_row"], d["w_col"], None, None, idx, g, ws)
+    out = torch.empty((cfg.T, cfg.d), dtype=torch.bfloat16, device="cuda")
+    try:
+        moe.moe_debug_set_wait_limit_ns(1)
+        moe.moe_atomic_experts(c, d["x"], d["w_in"], d["w_out"], idx, g, out, ws)
+        st = moe.moe_read_device_status(ws)
+    finally:
+        moe.moe_debug_set_wait_limit_ns(0)
+    assert st in (moe.ERR_TIMEOUT, moe.OK)  # OK only if every block had arrived before the first check
+    moe.moe_atomic_experts(c, d["x"], d["w_in"], d["w_out"], idx, g, out, ws)
+    assert moe.moe_read_device_status(ws) == moe.OK
+    ref = O.atomic_output(inp["x"], inp["w_in"], inp["w_out"], host(idx), host(g), cfg.act)
+    assert token_rel_err(out_f64(out), ref) <= TOL[W.BF16]
+    out2 = torch.empty_like(out)
+    moe.moe_atomic_forward(c, d["x"], d["w_row"], d["w_col"], d["w_in"], d["w_out"], out2, ws)
+    torch.cuda.synchronize()
+    assert torch.equal(out, out2)
