@@ -533,8 +533,8 @@ def ours(args):
     if cfg.dtype == W.BF16 and cfg.n_shared == 0:
         # the library's static down-projection split (mirrors its planner; only affects the byte count)
         avg = cfg.T * cfg.k / cfg_groups.m
-        bn = 16
-        while bn < 256 and bn < 2.0 * avg:
+        bn, cap = 16, (256 if avg >= 256 else 128)  # the library's down-projection tile rule
+        while bn < cap and bn < 2.0 * avg:
             bn <<= 1
         tiles = min(cfg_groups.m, cfg.T * cfg.k) * ((cfg.d + 127) // 128) * max(1, math.ceil(avg / bn))
         if tiles < 4 * 148:

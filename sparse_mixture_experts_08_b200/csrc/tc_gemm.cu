@@ -744,9 +744,14 @@ static cudaError_t launch_impl(const TcMaps& maps, const GemmParams& p, int num_
 // Token rows per tile: about twice the mean segment, so most experts' segments fit
 // one tile and each weight tile is streamed once (every extra row tile of a segment
 // re-reads the expert's weights), capped by TMEM (two SwiGLU accumulators of BN
-// columns, double-buffered, must fit 512 columns).
+// columns, double-buffered, must fit 512 columns). The down projection takes 256-row
+// tiles only when the mean segment fills them: a 256-row tile leaves room for four
+// pipeline stages, too few to cover the loads of a 1408-deep K loop over short
+// segments (measured: dsv2lite down 283 -> 242 us with 128; mixtral, 1024-row
+// segments, 853 us with 256 against 1228 with 128).
 int tc_pick_bn(int epi, double avg) {
-  const int cap = (epi == EPI_SWIGLU || epi == EPI_LOGITS) ? 128 : 256;
+  int cap = (epi == EPI_SWIGLU || epi == EPI_LOGITS) ? 128 : 256;
+  if (epi == EPI_DOWN && avg < 256.0) cap = 128;
   int bn = 16;
   while (bn < cap && bn < 2.0 * avg) bn <<= 1;
   return bn;
