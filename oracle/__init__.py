@@ -305,3 +305,135 @@ def atomic_output(x: np.ndarray, w_in: np.ndarray, w_out: np.ndarray, idx: np.nd
                                      _ptr(np.ascontiguousarray(g, np.float64)), _ptr(tok), ntok, _ptr(out)),
            "atomic_output")
     return out
+
+
+# ----------------------------------------------------- 8-bit expert weights (e4m3)
+#
+# R&Q ("Free parameters": quantization precision) stores quantized expert copies
+# in 8 bits and names no format or scaling. Reading taken here: OCP E4M3 (1 sign
+# bit, 4 exponent bits with bias 7, 3 mantissa bits, no infinities, largest finite
+# magnitude 448), one fp32 scale per row (per output channel of a weight matrix,
+# per task row of an activation), scale = row max |v| / 448, code = the E4M3 value
+# nearest to v / scale (ties to the even code, saturating at +-448). Both GEMM
+# operands of an 8-bit tensor-core product are 8-bit, so the activations entering
+# each projection are quantized the same way, per row; the hidden activation h is
+# stored in bf16 (round to nearest even) before it is quantized.
+
+E4M3_MAX = 448.0
+
+
+def e4m3_round(v) -> np.ndarray:
+    """float32 values -> E4M3 codes (uint8): round to nearest, ties to even,
+    saturating at +-448; the sign bit follows the sign of v (so -0 -> 0x80)."""
+    v = np.asarray(v, dtype=np.float32)
+    a = np.minimum(np.abs(v).astype(np.float64), E4M3_MAX)
+    # binade of a: quantum 2^(e-3) for a in [2^e, 2^(e+1)), e >= -6; 2^-9 below 2^-6
+    _, ex = np.frexp(np.where(a > 0, a, 1.0))      # a = mant * 2^ex, mant in [0.5, 1)
+    e = np.maximum(ex - 1, -6)
+    quantum = np.ldexp(1.0, e - 3)
+    n = np.rint(a / quantum)                        # exact quotient; rint rounds half to even
+    r = n * quantum                                 # rounded magnitude (may carry into the next binade)
+    # encode r: exponent field E (0 = subnormal), mantissa field M
+    _, rex = np.frexp(np.where(r > 0, r, 1.0))
+    re = rex - 1
+    normal = r >= 2.0 ** -6
+    E = np.where(normal, re + 7, 0)
+    M = np.where(normal, r / np.ldexp(1.0, re) * 8 - 8, r / 2.0 ** -9)
+    M = np.where(r > 0, M, 0)
+    E = np.where(r > 0, E, 0)
+    code = (E.astype(np.int64) << 3) | M.astype(np.int64)
+    code |= np.signbit(v).astype(np.int64) << 7
+    return code.astype(np.uint8)
+
+
+def e4m3_value(codes) -> np.ndarray:
+    """E4M3 codes -> float64 values (NaN for the two NaN codes)."""
+    c = np.asarray(codes, dtype=np.uint8).astype(np.int64)
+    s = np.where(c & 0x80, -1.0, 1.0)
+    E = (c >> 3) & 0xF
+    M = c & 0x7
+    mag = np.where(E == 0, M * 2.0 ** -9, (1.0 + M / 8.0) * np.ldexp(1.0, E - 7))
+    mag = np.where((E == 0xF) & (M == 0x7), np.nan, mag)
+    return s * mag
+
+
+def quantize_rows(a) -> tuple:
+    """Per-row E4M3 quantization of a 2-D float32 array: (codes uint8, scales
+    float32). scale = fl32(max |row| / 448) (1 for an all-zero row); code =
+    e4m3_round(fl32(v / scale)). Both divisions are IEEE fp32."""
+    a = np.asarray(a, dtype=np.float32)
+    amax = np.max(np.abs(a), axis=1) if a.shape[1] else np.zeros(a.shape[0], np.float32)
+    scale = np.where(amax > 0, amax / np.float32(E4M3_MAX), np.float32(1.0)).astype(np.float32)
+    q = (a / scale[:, None]).astype(np.float32)
+    return e4m3_round(q), scale
+
+
+def round_bf16(v) -> np.ndarray:
+    """float64 -> float32 (nearest) -> bf16 (nearest, ties to even), returned as float32."""
+    f = np.asarray(v, dtype=np.float32)
+    u = f.view(np.uint32).astype(np.uint64)
+    u = (u + 0x7FFF + ((u >> 16) & 1)) >> 16 << 16
+    return u.astype(np.uint32).view(np.float32)
+
+
+def quantize_experts(cfg, inp: Dict[str, np.ndarray]) -> Dict[str, np.ndarray]:
+    """Every expert weight matrix of `inp` quantized per output channel: for key
+    K in (w_gate, w_up, w_down, ws_gate, ws_up, ws_down), K -> codes with the
+    same shape and K + "_scale" -> one scale per row of the last axis."""
+    out = {}
+    for key in ("w_gate", "w_up", "w_down", "ws_gate", "ws_up", "ws_down"):
+        w = inp.get(key)
+        if w is None:
+            continue
+        vals = _values(w, cfg.dtype)
+        codes, sc = quantize_rows(vals.reshape(-1, vals.shape[-1]))
+        out[key] = codes.reshape(vals.shape)
+        out[key + "_scale"] = sc.reshape(vals.shape[:-1])
+    return out
+
+
+def _ffn_fp8(xq, sx, gq, gs, uq, us, dq, ds, act):
+    """Expert FFN on quantized rows (fp64 arithmetic on the dequantized values):
+    a = (x . w_gate) [, b = (x . w_up)]; h = silu(a) b or relu(a); h is stored in
+    bf16 and quantized per row; y = h_q . w_down. Rows of xq are tasks."""
+    X = e4m3_value(xq) * sx[:, None].astype(np.float64)
+    a = X @ (e4m3_value(gq) * gs[:, None].astype(np.float64)).T
+    if act == SWIGLU:
+        b = X @ (e4m3_value(uq) * us[:, None].astype(np.float64)).T
+        h = a / (1.0 + np.exp(-a)) * b
+    else:
+        h = np.maximum(a, 0.0)
+    hq, hs = quantize_rows(round_bf16(h))
+    H = e4m3_value(hq) * hs[:, None].astype(np.float64)
+    return H @ (e4m3_value(dq) * ds[:, None].astype(np.float64)).T
+
+
+def layer_forward_fp8(cfg, inp: Dict[str, np.ndarray], qw: Optional[Dict[str, np.ndarray]] = None,
+                      tokens=None) -> Dict[str, object]:
+    """The layer forward with 8-bit expert weights: the router as in the bf16
+    layer (bf16 operands, fp32 logits, top-k softmax); each token row of x is
+    quantized once (its k tasks share codes and scale); every routed task and
+    every shared expert runs _ffn_fp8; out_t = sum_s w[t,s] y_{t,s} + sum of the
+    shared experts' y. Returns out (float64) for `tokens` (all when None), the
+    routing, and the quantized x."""
+    x = inp["x"]
+    T = x.shape[0]
+    qw = qw if qw is not None else quantize_experts(cfg, inp)
+    logits = router_logits(x, inp["w_router"], inp.get("bias"))
+    idx, w = topk_softmax(logits, cfg.k, bool(cfg.renorm))
+    xq, sx = quantize_rows(_values(x, cfg.dtype))
+    tok = np.arange(T) if tokens is None else np.asarray(tokens, dtype=np.int64)
+    out = np.zeros((len(tok), cfg.d), np.float64)
+    swiglu = cfg.act == SWIGLU
+    for e in np.unique(idx[tok]):
+        rows, slots = np.nonzero(idx[tok] == e)
+        t = tok[rows]
+        y = _ffn_fp8(xq[t], sx[t], qw["w_gate"][e], qw["w_gate_scale"][e],
+                     qw["w_up"][e] if swiglu else None, qw["w_up_scale"][e] if swiglu else None,
+                     qw["w_down"][e], qw["w_down_scale"][e], cfg.act)
+        np.add.at(out, rows, w[t, slots][:, None] * y)
+    for sh in range(cfg.n_shared):
+        out += _ffn_fp8(xq[tok], sx[tok], qw["ws_gate"][sh], qw["ws_gate_scale"][sh],
+                        qw["ws_up"][sh] if swiglu else None, qw["ws_up_scale"][sh] if swiglu else None,
+                        qw["ws_down"][sh], qw["ws_down_scale"][sh], cfg.act)
+    return {"out": out, "idx": idx, "w": w, "logits": logits, "xq": xq, "sx": sx}

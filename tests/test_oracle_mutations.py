@@ -53,6 +53,13 @@ PY_MUTATIONS = {
     "floe_mask_strict": ("if u_mask is not None else u) >= thr", "if u_mask is not None else u) > thr"),
     "floe_gate_from_up": ("g = as64(wg)[keep] @ x", "g = as64(wu)[keep] @ x"),
     "floe_threshold_off_by_one": ("return np.float32(v[min(r, v.size) - 1])", "return np.float32(v[min(r, v.size - 1)])"),
+    "e4m3_ties_away": ("n = np.rint(a / quantum)", "n = np.floor(a / quantum + 0.5)"),
+    "e4m3_no_saturation": ("a = np.minimum(np.abs(v).astype(np.float64), E4M3_MAX)", "a = np.abs(v).astype(np.float64)"),
+    "e4m3_bias_8": ("np.ldexp(1.0, E - 7)", "np.ldexp(1.0, E - 8)"),
+    "fp8_scale_240": ("amax / np.float32(E4M3_MAX)", "amax / np.float32(240.0)"),
+    "fp8_h_scale_dropped": ("H = e4m3_value(hq) * hs[:, None].astype(np.float64)", "H = e4m3_value(hq)"),
+    "fp8_x_scale_dropped": ("X = e4m3_value(xq) * sx[:, None].astype(np.float64)", "X = e4m3_value(xq)"),
+    "fp8_column_scales": ("amax = np.max(np.abs(a), axis=1) if", "amax = np.max(np.abs(a), axis=0)[:a.shape[0]] if"),
 }
 
 
@@ -206,8 +213,31 @@ def check_floe(O):
     assert keep[j]
 
 
+def check_fp8(O):
+    for code, val in ((0x01, 2.0 ** -9), (0x08, 2.0 ** -6), (0x38, 1.0), (0x7E, 448.0), (0xFE, -448.0)):
+        assert O.e4m3_value(np.uint8(code)) == val
+    v = np.array([1.0625, 1.1875, 2.0 ** -10, 3 * 2.0 ** -11, 460.0, 1e6, -5.5, 0.3], np.float32)
+    assert O.e4m3_round(v).tolist() == [0x38, 0x3A, 0x00, 0x01, 0x7E, 0x7E, 0xCB, 0x2A]
+    rng = np.random.default_rng(11)
+    a = rng.standard_normal((6, 40)).astype(np.float32)
+    codes, sc = O.quantize_rows(a)
+    assert all(codes[r, int(np.argmax(np.abs(a[r])))] & 0x7F == 0x7E for r in range(6))
+    cfg = W.small_moe(T=16, d=32, f=16, m=3, k=2, act=W.RELU, dtype=W.BF16, zipf_s=0.5, n_shared=1,
+                      f_shared=16, index=93)
+    inp = W.make_moe_inputs(cfg)
+    x = np.zeros((cfg.T, cfg.d), np.uint16)
+    pw = lambda shape, lo, hi: (((rng.integers(lo, hi + 1, shape) + 127) << 7)
+                                | (rng.integers(0, 2, shape) << 15)).astype(np.uint16)
+    x[np.arange(cfg.T), rng.integers(0, cfg.d, cfg.T)] = pw(cfg.T, 0, 2)
+    inp["x"] = x
+    for key in ("w_gate", "w_down", "ws_gate", "ws_down"):
+        inp[key] = pw(inp[key].shape, -3, 0)
+    ref = O.layer_forward(cfg, inp)["out"]
+    np.testing.assert_allclose(O.layer_forward_fp8(cfg, inp)["out"], ref, rtol=1e-5, atol=1e-6 * np.abs(ref).max())
+
+
 CHECKS = [check_lis_golden, check_topk, check_router, check_permutation, check_ffn, check_shared, check_atomic,
-          check_replica, check_floe]
+          check_replica, check_floe, check_fp8]
 
 
 def _failures(O):

@@ -528,3 +528,137 @@ def test_floe_mask_keeps_the_threshold_itself():
     _, keep = O.floe_expert(inp["x"][1], inp["w_gate"][0], inp["w_up"][0], inp["w_down"][0], thr, W.BF16,
                             u_mask=u32)
     assert keep[j] and keep.sum() == (np.abs(u32) >= np.float32(thr)).sum()
+
+
+# ---------------------------------------------------------- 8-bit expert weights
+# Facts of the OCP E4M3 format: bias 7, 3 mantissa bits, no infinities, one NaN
+# pattern per sign (S.1111.111), largest finite 0x7E = 1.75 * 2^8 = 448, smallest
+# subnormal 0x01 = 2^-9, smallest normal 0x08 = 2^-6, 0x38 = 1.
+
+E4M3_FACTS = {0x00: 0.0, 0x01: 2.0 ** -9, 0x07: 7 * 2.0 ** -9, 0x08: 2.0 ** -6, 0x38: 1.0, 0x39: 1.125,
+              0x40: 2.0, 0x7E: 448.0, 0x80: -0.0, 0xB8: -1.0, 0xFE: -448.0}
+
+
+def test_e4m3_decode_format_facts():
+    for code, val in E4M3_FACTS.items():
+        got = O.e4m3_value(np.uint8(code))
+        assert got == val and np.signbit(got) == np.signbit(val), hex(code)
+    assert np.isnan(O.e4m3_value(np.uint8(0x7F))) and np.isnan(O.e4m3_value(np.uint8(0xFF)))
+
+
+def test_e4m3_decode_matches_torch_float8():
+    codes = np.arange(256, dtype=np.uint8)
+    ref = torch.from_numpy(codes).view(torch.float8_e4m3fn).double().numpy()
+    got = O.e4m3_value(codes)
+    assert np.array_equal(np.isnan(ref), np.isnan(got))
+    ok = ~np.isnan(ref)
+    assert np.array_equal(ref[ok], got[ok])
+
+
+def _e4m3_brute(v):
+    """Nearest finite E4M3 value by exhaustive search over the 127 non-negative
+    finite codes; a tie goes to the code with an even mantissa (lowest bit 0);
+    magnitudes past 448 saturate. Sign copied from v."""
+    pos = np.arange(0x7F, dtype=np.uint8)
+    vals = O.e4m3_value(pos)
+    out = []
+    for x in np.asarray(v, np.float32):
+        a = min(abs(float(x)), 448.0)
+        dist = np.abs(vals - a)
+        best = np.flatnonzero(dist == dist.min())
+        code = int(best[0]) if len(best) == 1 else int([b for b in best if b % 2 == 0][0])
+        out.append(code | (0x80 if np.signbit(x) else 0))
+    return np.array(out, np.uint8)
+
+
+def _e4m3_probe_values(rng):
+    vals = O.e4m3_value(np.arange(0x7F, dtype=np.uint8))
+    mids = (vals[:-1] + vals[1:]) / 2                 # every tie between neighbouring codes
+    rnd = rng.standard_normal(3000) * np.exp2(rng.integers(-14, 10, 3000))
+    edge = np.array([447.9, 448, 455.9, 464.0, 470.0, 1e6, 1e30, 2.0 ** -10, 2.0 ** -12, 0.0, -0.0])
+    v = np.concatenate([vals, mids, np.nextafter(mids, 0), np.nextafter(mids, 1e9), rnd, edge]).astype(np.float32)
+    return np.concatenate([v, -v])
+
+
+def test_e4m3_round_is_nearest_even_by_exhaustive_search():
+    v = _e4m3_probe_values(np.random.default_rng(7))
+    np.testing.assert_array_equal(O.e4m3_round(v), _e4m3_brute(v))
+
+
+def test_e4m3_round_matches_torch_cast_in_range():
+    v = _e4m3_probe_values(np.random.default_rng(8))
+    v = v[np.abs(v) < 464]                             # torch's cast gives NaN, not 448, past the last tie
+    ref = torch.from_numpy(v).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+    np.testing.assert_array_equal(O.e4m3_round(v), ref)
+
+
+def test_quantize_rows_invariants():
+    rng = np.random.default_rng(9)
+    a = (rng.standard_normal((40, 96)) * np.exp2(rng.integers(-20, 20, (40, 1)))).astype(np.float32)
+    a[3] = 0.0
+    a[5, :] = 0.0
+    a[5, 17] = -3.0
+    codes, sc = O.quantize_rows(a)
+    assert sc[3] == 1.0 and not codes[3].any()
+    for r in range(40):
+        if r == 3:
+            continue
+        j = int(np.argmax(np.abs(a[r])))
+        assert codes[r, j] & 0x7F == 0x7E                # the row maximum lands on 448
+        assert sc[r] == np.float32(np.abs(a[r]).max() / np.float32(448))
+        dq = O.e4m3_value(codes[r]) * np.float64(sc[r])
+        err = np.abs(dq - a[r])
+        # half a quantum: 2^-4 relative in the normal range, 2^-10 * scale below it
+        bound = np.maximum(np.abs(a[r]).astype(np.float64) * 2.0 ** -4, 2.0 ** -10 * np.float64(sc[r])) * (1 + 1e-6)
+        assert np.all(err <= bound), r
+
+
+def _pow2_bf16(rng, shape, lo, hi, p_zero=0.2):
+    """bf16 bit patterns of +-2^e (e uniform in [lo, hi]) with some exact zeros."""
+    e = rng.integers(lo, hi + 1, shape)
+    bits = ((e + 127) << 7) | (rng.integers(0, 2, shape) << 15)
+    bits = np.where(rng.random(shape) < p_zero, 0, bits)
+    return bits.astype(np.uint16)
+
+
+def test_fp8_layer_is_lossless_on_power_of_two_inputs():
+    """With one-hot token rows and weights that are signed powers of two, every
+    product, every ReLU output and every quantized row is exactly representable
+    (up to the fp32 rounding of the scales), so the 8-bit layer equals the bf16
+    layer to ~1e-6: each scale (x, weight rows, h) must be applied exactly once."""
+    cfg = W.small_moe(T=24, d=32, f=16, m=4, k=2, act=W.RELU, dtype=W.BF16, zipf_s=0.5, n_shared=1,
+                      f_shared=16, index=93)
+    inp = W.make_moe_inputs(cfg)
+    rng = np.random.default_rng(10)
+    x = np.zeros((cfg.T, cfg.d), np.uint16)
+    x[np.arange(cfg.T), rng.integers(0, cfg.d, cfg.T)] = _pow2_bf16(rng, cfg.T, 0, 2, p_zero=0.0)
+    inp["x"] = x
+    for key in ("w_gate", "w_down", "ws_gate", "ws_down"):
+        inp[key] = _pow2_bf16(rng, inp[key].shape, -3, 0)
+    ref = O.layer_forward(cfg, inp)["out"]
+    got = O.layer_forward_fp8(cfg, inp)["out"]
+    assert np.abs(ref).max() > 0.1
+    np.testing.assert_allclose(got, ref, rtol=1e-5, atol=1e-6 * np.abs(ref).max())
+
+
+@pytest.mark.parametrize("act", [W.SWIGLU, W.RELU])
+def test_fp8_layer_is_close_to_bf16_layer(act):
+    """On random bf16 inputs the 8-bit layer differs from the bf16 layer by the
+    quantization error only. Each of the three rounding steps (x, weights, h) has a
+    relative error uniform in +-2^-4, about 3.6 % rms, so the normwise error is a few
+    per cent: never zero, never the size of the output."""
+    cfg = W.small_moe(T=40, d=64, f=48, m=4, k=2, act=act, dtype=W.BF16, zipf_s=0.5, n_shared=1, f_shared=32,
+                      index=94)
+    inp = W.make_moe_inputs(cfg)
+    ref = O.layer_forward(cfg, inp)["out"]
+    got = O.layer_forward_fp8(cfg, inp)["out"]
+    rel = np.linalg.norm(got - ref) / np.linalg.norm(ref)
+    assert 5e-3 < rel < 0.15, rel
+
+
+def test_fp8_sampled_tokens_match_full_output():
+    cfg = W.small_moe(T=30, d=32, f=32, m=5, k=2, act=W.SWIGLU, dtype=W.BF16, zipf_s=1.0, index=95)
+    inp = W.make_moe_inputs(cfg)
+    full = O.layer_forward_fp8(cfg, inp)["out"]
+    tok = [29, 3, 3, 17]
+    np.testing.assert_allclose(O.layer_forward_fp8(cfg, inp, tokens=tok)["out"], full[tok], rtol=1e-12, atol=0)
