@@ -324,37 +324,43 @@ E4M3_MAX = 448.0
 
 def e4m3_round(v) -> np.ndarray:
     """float32 values -> E4M3 codes (uint8): round to nearest, ties to even,
-    saturating at +-448; the sign bit follows the sign of v (so -0 -> 0x80)."""
+    saturating at +-448; the sign bit follows the sign of v (so -0 -> 0x80).
+
+    A magnitude a in the binade [2^e, 2^(e+1)), e >= -6, is a multiple of the
+    quantum 2^(e-3); below 2^-6 the quantum is 2^-9 (subnormals). With n = a /
+    quantum rounded half to even, the non-negative codes count the representable
+    magnitudes in increasing order, 8 per binade from 2^-6 up and 8 subnormal ones
+    (0 .. 7 * 2^-9) below, so the code is 8 (e + 6) + n for e >= -6 and n below
+    2^-6. n = 16 (a rounded up to 2^(e+1)) lands on the first code of the next
+    binade by the same formula."""
     v = np.asarray(v, dtype=np.float32)
     a = np.minimum(np.abs(v).astype(np.float64), E4M3_MAX)
-    # binade of a: quantum 2^(e-3) for a in [2^e, 2^(e+1)), e >= -6; 2^-9 below 2^-6
-    _, ex = np.frexp(np.where(a > 0, a, 1.0))      # a = mant * 2^ex, mant in [0.5, 1)
-    e = np.maximum(ex - 1, -6)
-    quantum = np.ldexp(1.0, e - 3)
-    n = np.rint(a / quantum)                        # exact quotient; rint rounds half to even
-    r = n * quantum                                 # rounded magnitude (may carry into the next binade)
-    # encode r: exponent field E (0 = subnormal), mantissa field M
-    _, rex = np.frexp(np.where(r > 0, r, 1.0))
-    re = rex - 1
-    normal = r >= 2.0 ** -6
-    E = np.where(normal, re + 7, 0)
-    M = np.where(normal, r / np.ldexp(1.0, re) * 8 - 8, r / 2.0 ** -9)
-    M = np.where(r > 0, M, 0)
-    E = np.where(r > 0, E, 0)
-    code = (E.astype(np.int64) << 3) | M.astype(np.int64)
+    _, ex = np.frexp(a)                             # a = mant * 2^ex, mant in [0.5, 1)
+    e = np.where(a >= 2.0 ** -6, ex - 1, -6)        # binade exponent; the subnormal range (and 0) uses -6
+    n = np.rint(np.ldexp(a, 3 - e))                 # exact scaling by a power of two; rint: half to even
+    code = (8 * (e + 6) + n).astype(np.int64)
     code |= np.signbit(v).astype(np.int64) << 7
     return code.astype(np.uint8)
 
 
-def e4m3_value(codes) -> np.ndarray:
-    """E4M3 codes -> float64 values (NaN for the two NaN codes)."""
-    c = np.asarray(codes, dtype=np.uint8).astype(np.int64)
+def _e4m3_table() -> np.ndarray:
+    """Values of the 256 codes from the bit fields: sign, exponent E (bias 7,
+    E = 0 subnormal), mantissa M; S.1111.111 is NaN."""
+    c = np.arange(256, dtype=np.int64)
     s = np.where(c & 0x80, -1.0, 1.0)
     E = (c >> 3) & 0xF
     M = c & 0x7
     mag = np.where(E == 0, M * 2.0 ** -9, (1.0 + M / 8.0) * np.ldexp(1.0, E - 7))
     mag = np.where((E == 0xF) & (M == 0x7), np.nan, mag)
     return s * mag
+
+
+_E4M3_VALUES = _e4m3_table()
+
+
+def e4m3_value(codes) -> np.ndarray:
+    """E4M3 codes -> float64 values (NaN for the two NaN codes)."""
+    return _E4M3_VALUES[np.asarray(codes, dtype=np.uint8)]
 
 
 def quantize_rows(a) -> tuple:
@@ -364,8 +370,11 @@ def quantize_rows(a) -> tuple:
     a = np.asarray(a, dtype=np.float32)
     amax = np.max(np.abs(a), axis=1) if a.shape[1] else np.zeros(a.shape[0], np.float32)
     scale = np.where(amax > 0, amax / np.float32(E4M3_MAX), np.float32(1.0)).astype(np.float32)
-    q = (a / scale[:, None]).astype(np.float32)
-    return e4m3_round(q), scale
+    codes = np.empty(a.shape, np.uint8)
+    for r0 in range(0, a.shape[0], 256):            # row blocks: bounded temporaries
+        r1 = min(a.shape[0], r0 + 256)
+        codes[r0:r1] = e4m3_round((a[r0:r1] / scale[r0:r1, None]).astype(np.float32))
+    return codes, scale
 
 
 def round_bf16(v) -> np.ndarray:
@@ -392,34 +401,67 @@ def quantize_experts(cfg, inp: Dict[str, np.ndarray]) -> Dict[str, np.ndarray]:
     return out
 
 
-def _ffn_fp8(xq, sx, gq, gs, uq, us, dq, ds, act):
-    """Expert FFN on quantized rows (fp64 arithmetic on the dequantized values):
-    a = (x . w_gate) [, b = (x . w_up)]; h = silu(a) b or relu(a); h is stored in
-    bf16 and quantized per row; y = h_q . w_down. Rows of xq are tasks."""
+def fp8_expert_up(xq, sx, gq, gs, uq, us, act) -> np.ndarray:
+    """First half of an 8-bit expert on quantized token rows (fp64 arithmetic on
+    the dequantized values): a = x . w_gate [, b = x . w_up]; h = silu(a) b
+    (SwiGLU) or relu(a). Returns h in fp64, one row per task."""
     X = e4m3_value(xq) * sx[:, None].astype(np.float64)
     a = X @ (e4m3_value(gq) * gs[:, None].astype(np.float64)).T
     if act == SWIGLU:
         b = X @ (e4m3_value(uq) * us[:, None].astype(np.float64)).T
-        h = a / (1.0 + np.exp(-a)) * b
-    else:
-        h = np.maximum(a, 0.0)
-    hq, hs = quantize_rows(round_bf16(h))
+        return a / (1.0 + np.exp(-a)) * b
+    return np.maximum(a, 0.0)
+
+
+def fp8_expert_down(h_stored, dq, ds) -> np.ndarray:
+    """Second half: the stored (bf16-valued, as float32) h rows are quantized per
+    row and multiplied by the quantized W_down: y = h_q . w_down (fp64)."""
+    hq, hs = quantize_rows(h_stored)
     H = e4m3_value(hq) * hs[:, None].astype(np.float64)
     return H @ (e4m3_value(dq) * ds[:, None].astype(np.float64)).T
 
 
+def _ffn_fp8(xq, sx, gq, gs, uq, us, dq, ds, act):
+    """An 8-bit expert: h is stored in bf16 between the two halves."""
+    return fp8_expert_down(round_bf16(fp8_expert_up(xq, sx, gq, gs, uq, us, act)), dq, ds)
+
+
+class QuantizedExperts:
+    """quantize_experts computed on first use, one expert matrix at a time:
+    q["w_gate"][e] -> codes, q["w_gate_scale"][e] -> scales (same values)."""
+
+    def __init__(self, cfg, inp):
+        self.cfg, self.inp, self.cache = cfg, inp, {}
+
+    def _get(self, key, e):
+        if (key, e) not in self.cache:
+            vals = _values(self.inp[key][e], self.cfg.dtype)
+            self.cache[(key, e)] = quantize_rows(vals.reshape(-1, vals.shape[-1]))
+        return self.cache[(key, e)]
+
+    def __getitem__(self, name):
+        key, part = (name[:-6], 1) if name.endswith("_scale") else (name, 0)
+        outer = self
+
+        class _Rows:
+            def __getitem__(self, e):
+                return outer._get(key, int(e))[part]
+        return _Rows()
+
+
 def layer_forward_fp8(cfg, inp: Dict[str, np.ndarray], qw: Optional[Dict[str, np.ndarray]] = None,
-                      tokens=None) -> Dict[str, object]:
+                      tokens=None, logits_in: Optional[np.ndarray] = None) -> Dict[str, object]:
     """The layer forward with 8-bit expert weights: the router as in the bf16
     layer (bf16 operands, fp32 logits, top-k softmax); each token row of x is
     quantized once (its k tasks share codes and scale); every routed task and
     every shared expert runs _ffn_fp8; out_t = sum_s w[t,s] y_{t,s} + sum of the
     shared experts' y. Returns out (float64) for `tokens` (all when None), the
-    routing, and the quantized x."""
+    routing, and the quantized x. With logits_in the top-k is taken on those logits."""
     x = inp["x"]
     T = x.shape[0]
-    qw = qw if qw is not None else quantize_experts(cfg, inp)
-    logits = router_logits(x, inp["w_router"], inp.get("bias"))
+    if qw is None:  # quantize only the experts the tokens reach (per output channel, as quantize_experts)
+        qw = QuantizedExperts(cfg, inp)
+    logits = router_logits(x, inp["w_router"], inp.get("bias")) if logits_in is None else logits_in
     idx, w = topk_softmax(logits, cfg.k, bool(cfg.renorm))
     xq, sx = quantize_rows(_values(x, cfg.dtype))
     tok = np.arange(T) if tokens is None else np.asarray(tokens, dtype=np.int64)

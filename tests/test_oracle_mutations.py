@@ -53,7 +53,7 @@ PY_MUTATIONS = {
     "floe_mask_strict": ("if u_mask is not None else u) >= thr", "if u_mask is not None else u) > thr"),
     "floe_gate_from_up": ("g = as64(wg)[keep] @ x", "g = as64(wu)[keep] @ x"),
     "floe_threshold_off_by_one": ("return np.float32(v[min(r, v.size) - 1])", "return np.float32(v[min(r, v.size - 1)])"),
-    "e4m3_ties_away": ("n = np.rint(a / quantum)", "n = np.floor(a / quantum + 0.5)"),
+    "e4m3_ties_away": ("n = np.rint(np.ldexp(a, 3 - e))", "n = np.floor(np.ldexp(a, 3 - e) + 0.5)"),
     "e4m3_no_saturation": ("a = np.minimum(np.abs(v).astype(np.float64), E4M3_MAX)", "a = np.abs(v).astype(np.float64)"),
     "e4m3_bias_8": ("np.ldexp(1.0, E - 7)", "np.ldexp(1.0, E - 8)"),
     "fp8_scale_240": ("amax / np.float32(E4M3_MAX)", "amax / np.float32(240.0)"),
