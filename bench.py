@@ -62,6 +62,9 @@ def parse():
     ap.add_argument("--floe", type=float, default=None, metavar="S",
                     help="FloE contextual sparsity at target sparsity S: thresholds calibrated on a second "
                          "synthetic batch (untimed), then moe_layer_forward_floe is timed")
+    ap.add_argument("--fp8", action="store_true",
+                    help="8-bit experts: E4M3 weights with per-channel scales (quantized once, untimed), "
+                         "moe_layer_forward_fp8")
     ap.add_argument("--router-only", action="store_true",
                     help="time the routing call alone (moe_route / moe_atomic_route) on the workload's inputs; "
                          "an auxiliary line for profiling, not the layer metric")
@@ -112,6 +115,27 @@ def cpu_oracle_sample(cfg, inp, budget_s: float):
             "sample": f"first {n} of {cfg.T} tokens of the {cfg.name} workload; every step of the layer "
                       f"(router, top-k, histogram/LIS, permutation, expert FFNs, combine) in fp64 C, "
                       f"{threads} threads over tokens"}
+
+
+def cpu_oracle_fp8_sample(cfg, inp, budget_s: float):
+    """Time the oracle's 8-bit layer (oracle.layer_forward_fp8) on the first n tokens,
+    n sized to ~budget_s; each timed call quantizes the experts its tokens reach."""
+    import oracle as O
+
+    def run(n):
+        t0 = time.perf_counter()
+        O.layer_forward_fp8(cfg, inp, tokens=np.arange(n))
+        return time.perf_counter() - t0
+
+    n = 1
+    dt = run(n)
+    while dt < budget_s / 8 and n < cfg.T:
+        n = min(cfg.T, n * 4)
+        dt = run(n)
+    return {"value": n / dt, "unit": UNIT, "cores": 1, "kind": "oracle", "seconds": round(dt, 3),
+            "sample": f"first {n} of {cfg.T} tokens of the {cfg.name} workload; the 8-bit layer (router, E4M3 "
+                      f"quantization of x, of the experts those tokens reach and of h, fp64 expert FFNs, combine) "
+                      f"in numpy, one process"}
 
 
 def reference_arm(args):
@@ -296,10 +320,12 @@ def fused_routing(cfg) -> bool:
     return cfg.dtype == W.BF16 and cfg.T >= 8192 and cfg.m <= 256 and cfg.k <= 8
 
 
-def stage_costs(cfg, active: int, ksplit: int):
+def stage_costs(cfg, active: int, ksplit: int, weight_bytes=None):
     """Algorithmic flops and bytes per launch of each stage (operands read once,
-    results written once; weights of ACTIVE experts only)."""
+    results written once; weights of ACTIVE experts only). weight_bytes = 1 for
+    E4M3 expert weights (activations still enter and leave each stage in bf16)."""
     es = 4 if cfg.dtype == W.F32 else 2
+    ew = es if weight_bytes is None else weight_bytes
     T, d, f, m, k = cfg.T, cfg.d, cfg.f, cfg.m, cfg.k
     Tk = T * k
     mats = 2 if cfg.act == W.SWIGLU else 1
@@ -315,15 +341,15 @@ def stage_costs(cfg, active: int, ksplit: int):
     c["router_topk_ranks"] = (2.0 * T * d * m, T * d * es + m * d * es + Tk * 12 + tiles * m * 4)
     c["scatter"] = (0.0, tiles * m * 4 + Tk * 12 + Tk * 12 + (2 * m + 1) * 4 + T * d * es + Tk * d * es)
     c["expert_up"] = (2.0 * mats * f * d * Tk + 2.0 * mats * fsh * d * T * nsh,
-                      active * mats * f * d * es + nsh * mats * fsh * d * es + Tk * d * es + (T * d * es if nsh else 0)
+                      active * mats * f * d * ew + nsh * mats * fsh * d * ew + Tk * d * es + (T * d * es if nsh else 0)
                       + Tk * f * es + nsh * T * fsh * es)
     fused_k1 = k == 1 and nsh == 0 and ksplit == 1 and cfg.dtype == W.BF16  # down epilogue writes `out` itself
     out_bytes = T * d * es if fused_k1 else ksplit * Tk * d * 4 + nsh * T * d * 4
     c["expert_down"] = (2.0 * d * f * Tk + 2.0 * d * fsh * T * nsh,
-                        active * d * f * es + nsh * d * fsh * es + Tk * f * es + nsh * T * fsh * es + out_bytes)
+                        active * d * f * ew + nsh * d * fsh * ew + Tk * f * es + nsh * T * fsh * es + out_bytes)
     c["combine"] = (0.0, 0.0 if fused_k1 else ksplit * Tk * d * 4 + nsh * T * d * 4 + Tk * 4 + T * d * es)
     layer_flops = 2.0 * T * d * m + c["expert_up"][0] + c["expert_down"][0]
-    layer_bytes = (m * d + active * (mats + 1) * f * d + nsh * (mats + 1) * fsh * d) * es + 2 * T * d * es
+    layer_bytes = m * d * es + (active * (mats + 1) * f * d + nsh * (mats + 1) * fsh * d) * ew + 2 * T * d * es
     return c, layer_flops, layer_bytes
 
 
@@ -379,14 +405,25 @@ def ours(args):
                         cfg.renorm)
     rep = args.replicate
     floe = args.floe
+    fp8 = args.fp8
     if rep and cfg.dtype != W.BF16:
         raise SystemExit("--replicate runs bf16 layers only")
+    if fp8 and (rep or floe is not None or cfg.dtype != W.BF16):
+        raise SystemExit("--fp8 runs plain bf16 layers (no --replicate / --floe)")
     if floe is not None and (cfg.dtype != W.BF16 or cfg.act != W.SWIGLU or cfg.n_shared):
         raise SystemExit("--floe runs bf16 SwiGLU layers without shared experts")
     if rep:
         ws = moe.replica_workspace(c, device=dev)
     elif floe is not None:
         ws = moe.floe_workspace(c, device=dev)
+    elif fp8:
+        ws = moe.fp8_workspace(c, device=dev)
+        # one-time E4M3 weights (untimed), then the bf16 copies are dropped
+        wq = moe.quantize_experts(d_in["w_gate"], d_in.get("w_up"), d_in["w_down"], d_in.get("ws_gate"),
+                                  d_in.get("ws_up"), d_in.get("ws_down"))
+        for key in ("w_gate", "w_up", "w_down", "ws_gate", "ws_up", "ws_down"):
+            d_in.pop(key, None)
+        torch.cuda.synchronize(dev)
     else:
         ws = moe.workspace(c, device=dev)
     if floe is not None:  # one-time weight layout and threshold calibration (untimed)
@@ -412,6 +449,10 @@ def ours(args):
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
 
     def fwd(x=None, o=None):
+        if fp8:
+            moe.moe_layer_forward_fp8(c, d_in["x"] if x is None else x, d_in["w_router"], d_in["bias"], wq,
+                                      out if o is None else o, ws, counts_out=counts, lis_out=lis, stream=s)
+            return
         args_ = (c, d_in["x"] if x is None else x, d_in["w_router"], d_in["bias"], d_in["w_gate"], d_in.get("w_up"),
                  d_in["w_down"], d_in.get("ws_gate"), d_in.get("ws_up"), d_in.get("ws_down"),
                  out if o is None else o, ws)
@@ -542,7 +583,11 @@ def ours(args):
             ks = min(16, -(-4 * 148 // tiles), kb)
             kbps = -(-kb // ks)
             plan_ksplit = -(-kb // kbps)
-    costs, layer_flops, layer_bytes = stage_costs(cfg_groups, active, plan_ksplit)
+            if fp8:  # the same split re-cut into 128-element k-blocks
+                kb8 = (cfg.f + 127) // 128
+                ks8 = min(plan_ksplit, kb8)
+                plan_ksplit = -(-kb8 // -(-kb8 // ks8))
+    costs, layer_flops, layer_bytes = stage_costs(cfg_groups, active, plan_ksplit, weight_bytes=1 if fp8 else None)
     if floe is not None:
         # dense up projection: W_up only, u written in fp32; sparse part: the gate and
         # down rows of the kept channels, u and the compact h
@@ -556,15 +601,18 @@ def ours(args):
     sec = dom_ms * 1e-3
     long_step = K * ms > 1000.0
     tensor_peak = pk["bf16_tflops_sustained"] if long_step else pk["bf16_tflops"]
+    if fp8:  # E4M3 contraction: the measured bf16 peak times the nominal dense fp8 / bf16 ratio (4.5 / 2.25)
+        tensor_peak *= 2.0
     ridge = tensor_peak * 1e12 / (pk["hbm_gbs"] * 1e9)
     if fl > 0 and fl / max(by, 1.0) > ridge and cfg.dtype == W.BF16:
         roof = {"bound": "tensor", "achieved": fl / sec / 1e12, "peak": tensor_peak, "unit": "TFLOP/s"}
-        roof["peak_source"] = f"{pk_src} bf16 ({'sustained' if long_step else 'burst'})"
+        roof["peak_source"] = (f"{pk_src} bf16 ({'sustained' if long_step else 'burst'})"
+                               + (" x 2 (nominal fp8 / bf16 dense ratio)" if fp8 else ""))
     else:
         roof = {"bound": "hbm", "achieved": by / sec / 1e9, "peak": pk["hbm_gbs"], "unit": "GB/s",
                 "peak_source": f"{pk_src} hbm copy"}
     roof["frac"] = roof["achieved"] / roof["peak"]
-    roof["traffic"] = traffic_for(cfg.name, dom)
+    roof["traffic"] = traffic_for(cfg.name + ("_fp8" if fp8 else ""), dom)
     roof["kernel"] = dom
     roof["algorithmic_bytes"] = by
     roof["algorithmic_flops"] = fl
@@ -573,9 +621,10 @@ def ours(args):
 
     line = {"metric": METRIC, "value": world * cfg.T / (ms * 1e-3), "unit": UNIT, "n_gpus": world, "steps": K,
             "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
-            "vs_baseline": None, "dtype": "bf16" if cfg.dtype == W.BF16 else "f32",
+            "vs_baseline": None, "dtype": "e4m3" if fp8 else "bf16" if cfg.dtype == W.BF16 else "f32",
             "data": "synthetic (seeded generator; x ~ N(0,1), weights ~ N(0, 1/sqrt(fan_in)), Zipf router bias)",
-            "config": dict(workload_config(cfg), parallelism=f"data-parallel token batches x{world} (weak scaling)",
+            "config": dict(workload_config(cfg), **({"expert_weights": "e4m3, per-channel fp32 scales"} if fp8 else {}),
+                           parallelism=f"data-parallel token batches x{world} (weak scaling)",
                            l2=f"flushed between steps ({L2_FLUSH_BYTES >> 20} MiB write, outside the timed events)",
                            launch="eager C-ABI call per step"),
             "roofline": roof,
@@ -591,6 +640,9 @@ def ours(args):
                            "expert_up = dense u = x W_up^T, expert_down = kept lists + kept gate rows + kept down rows",
                 "kept_channel_fraction": float(kept.cpu().numpy()[kept.cpu().numpy() > 0].mean() / cfg.f)}
                if floe is not None else {}),
+            **({"variant": "8-bit experts: E4M3 weights with one fp32 scale per output channel (quantized once, "
+                           "outside the timing); x and h rows quantized per row inside each step; router in bf16",
+                "dtype_note": "expert GEMMs e4m3 x e4m3 with fp32 accumulation; router bf16"} if fp8 else {}),
             **({"variant": "R&Q replica dispatch: the heavy-hitter's tasks alternate between it and a replica "
                            "expert m that computes with its bf16 weights; routing.lis is over the m + 1 experts",
                 "lis_before_split": moe.unpack_lis(lis0)[2],
@@ -605,7 +657,8 @@ def ours(args):
         dist.barrier()
     if rank == 0:
         if world == 1 and not args.no_cpu_baseline:
-            line["cpu_baseline"] = cpu_oracle_sample(cfg, inp, args.cpu_seconds)
+            line["cpu_baseline"] = (cpu_oracle_fp8_sample(cfg, inp, args.cpu_seconds) if fp8
+                                    else cpu_oracle_sample(cfg, inp, args.cpu_seconds))
         else:
             line["cpu_baseline"] = None
         print(json.dumps(line), flush=True)

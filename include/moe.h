@@ -248,6 +248,68 @@ MOE_API moe_status_t moe_layer_forward_floe(const moe_config_t* cfg, const void*
                                             float* u_out, int32_t* perm_out, void* ws, size_t ws_bytes,
                                             moe_stream_t stream);
 
+/* 8-bit expert weights (R&Q, "Free parameters": 8-bit expert copies for
+ * LLaMA-MoE and DeepSeek; the format is not named there). Format: OCP E4M3 codes
+ * (uint8: sign, 4 exponent bits with bias 7, 3 mantissa bits; largest finite 448)
+ * with one fp32 scale per row. A row of values v becomes scale = fl32(max |v| /
+ * 448) (1 for an all-zero row) and codes E4M3(fl32(v / scale)), rounded to
+ * nearest even and saturating at +-448; the value of a code is E4M3(code) * scale.
+ *
+ * moe_quantize_e4m3: per-row quantization of a bf16 matrix src [rows, cols]
+ * (device, row-major, 16-byte aligned) into codes [rows, cols] (device, 16-byte
+ * aligned) and scales [rows] (device fp32). cols must be a multiple of 16
+ * (MOE_ERR_UNSUPPORTED otherwise). Used once on the expert weights; outputs are
+ * owned by the caller. Asynchronous on `stream`. */
+MOE_API moe_status_t moe_quantize_e4m3(int64_t rows, int64_t cols, const void* src, uint8_t* codes, float* scales,
+                                       moe_stream_t stream);
+
+/* Quantized expert weights for moe_layer_forward_fp8: the bf16 weights of
+ * moe_layer_forward passed through moe_quantize_e4m3 row by row (each output
+ * channel its own scale). Device pointers; codes 16-byte aligned.
+ *   gate, up  [m, f, d] codes, gate_scale / up_scale [m f]  (up: SwiGLU only)
+ *   down      [m, d, f] codes, down_scale [m d]
+ *   sh_gate, sh_up [n_shared, f_shared, d], scales [n_shared f_shared]
+ *   sh_down   [n_shared, d, f_shared], sh_down_scale [n_shared d]
+ * (sh_*: only with n_shared > 0; unused entries may be NULL). */
+typedef struct {
+  const uint8_t* gate;
+  const float* gate_scale;
+  const uint8_t* up;
+  const float* up_scale;
+  const uint8_t* down;
+  const float* down_scale;
+  const uint8_t* sh_gate;
+  const float* sh_gate_scale;
+  const uint8_t* sh_up;
+  const float* sh_up_scale;
+  const uint8_t* sh_down;
+  const float* sh_down_scale;
+} moe_fp8_experts_t;
+
+/* Workspace of moe_layer_forward_fp8 (host out-parameter): moe_workspace_size()
+ * plus the E4M3 rows of x and h. bf16 layers with d, f and f_shared multiples of
+ * 16 only (MOE_ERR_UNSUPPORTED otherwise). */
+MOE_API moe_status_t moe_fp8_workspace_size(const moe_config_t* cfg, size_t* bytes);
+
+/* moe_layer_forward with 8-bit experts. The router is the bf16 layer's (same
+ * logits, top-k and gate weights, same histogram, LIS and permutation); every
+ * projection of every routed and shared expert multiplies E4M3 operands on the
+ * tensor cores (fp32 accumulation): the permuted token rows and the bf16 h rows
+ * are quantized per row on the way in, and each product is scaled by its weight
+ * row's and its activation row's scales. out [T, d] bf16. Optional outputs as in
+ * moe_layer_forward, plus copies for inspection (all nullable, device): h_out
+ * [T k, f] bf16 = the stored h of each segment row, h_shared_out [n_shared T,
+ * f_shared] bf16, perm_out [T k] int32 = the task (t k + s) of each segment row.
+ * ws: moe_fp8_workspace_size() bytes, 256-byte aligned. Stage events
+ * (moe_set_stage_events) as in moe_layer_forward; the quantization of x rows
+ * falls in stage 4-5 and that of h in 5-6. */
+MOE_API moe_status_t moe_layer_forward_fp8(const moe_config_t* cfg, const void* x, const void* w_router,
+                                           const float* bias, const moe_fp8_experts_t* wq, void* out,
+                                           float* logits_out, int32_t* topk_idx_out, float* topk_w_out,
+                                           int32_t* counts_out, moe_lis_t* lis_out, void* h_out,
+                                           void* h_shared_out, int32_t* perm_out, void* ws, size_t ws_bytes,
+                                           moe_stream_t stream);
+
 /* Cartesian Product Router (OmniMoE Sec. 2.2, Eq. 8; App. A): lr = log_softmax(x
  * w_row^T), lc = log_softmax(x w_col^T) (fp32); expert (i, j) with flat id
  * i Nc + j scores S = fl32(lr_i + lc_j); idx_out [T, K] = the exact top-K of all

@@ -214,6 +214,22 @@ static moe_status_t run_router(const moe_config_t& c, const void* x, const void*
   return cuda_status(launch_tc_gemm(EPI_LOGITS, bn, maps, p, ctas, s));
 }
 
+// 8-bit expert path: the quantized weights and the per-row codes and scales of
+// each projection's input (x_perm rows, h rows, and for shared experts x and h_sh).
+struct Fp8Io {
+  const moe_fp8_experts_t* w;
+  uint8_t* xq;     // [T k, d]
+  float* sx;       // [T k]
+  uint8_t* hq;     // [T k, f]
+  float* sh;       // [T k]
+  uint8_t* xq_sh;  // [T, d]
+  float* sx_sh;    // [T]
+  uint8_t* hq_sh;  // [n_shared T, f_shared]
+  float* sh_sh;    // [n_shared T]
+};
+
+static int kblocks8(int K) { return (K + 127) / 128; }
+
 struct FfnIo {
   // routed class (may be absent: n_routed_groups == 0)
   int n_routed;           // groups (experts) of the routed class
@@ -235,6 +251,7 @@ struct FfnIo {
   const void *ws_gate, *ws_up, *ws_down;
   void* h_sh;             // [n_shared T, f_shared]
   float* y_sh;            // [n_shared T, d]
+  const Fp8Io* q8;        // 8-bit experts (nullable)
 };
 
 static void fill_common(GemmParams& p, int* status) {
@@ -246,6 +263,12 @@ static moe_status_t run_ffn(const moe_config_t& c, const Plan& pl, const FfnIo& 
                             cudaStream_t s, bool stage_marks = false) {
   const bool swiglu = c.act == MOE_SWIGLU;
   const bool tc = c.dtype == MOE_BF16;
+  const Fp8Io* q8 = io.q8;
+  auto kbl = [&](int K) { return q8 ? kblocks8(K) : kblocks(K); };
+  if (q8) {  // E4M3 rows of the up projection's inputs
+    MOE_CUDA(launch_quantize_e4m3(io.routed_rows, c.d, io.x_perm, c.d, q8->xq, c.d, q8->sx, s));
+    if (io.n_shared > 0) MOE_CUDA(launch_quantize_e4m3(c.T, c.d, io.x, c.d, q8->xq_sh, c.d, q8->sx_sh, s));
+  }
   // ---- up projection (+ activation): h = act(x W_gate^T [, x W_up^T])
   GemmParams up;
   std::memset(&up, 0, sizeof(up));
@@ -259,7 +282,7 @@ static moe_status_t run_ffn(const moe_config_t& c, const Plan& pl, const FfnIo& 
     g.R = c.f;
     g.K = c.d;
     g.ksplit = 1;
-    g.kb_per_split = kblocks(c.d);
+    g.kb_per_split = kbl(c.d);
     g.seg_off = io.offsets;
     g.max_row = (int)io.routed_rows;
     g.out = io.h;
@@ -274,6 +297,14 @@ static moe_status_t run_ffn(const moe_config_t& c, const Plan& pl, const FfnIo& 
     mu.a0[ncls] = {io.w_gate, (long long)g.n_wgroups * c.f, c.d};
     mu.a1[ncls] = {swiglu ? io.w_up : io.w_gate, (long long)g.n_wgroups * c.f, c.d};
     mu.b[ncls] = {io.x_perm, io.routed_rows, c.d};
+    if (q8) {
+      mu.a0[ncls].ptr = q8->w->gate;
+      mu.a1[ncls].ptr = swiglu ? q8->w->up : q8->w->gate;
+      mu.b[ncls].ptr = q8->xq;
+      g.a0_scale = q8->w->gate_scale;
+      g.a1_scale = swiglu ? q8->w->up_scale : nullptr;
+      g.b_scale = q8->sx;
+    }
     ++ncls;
   }
   if (io.n_shared > 0) {
@@ -282,7 +313,7 @@ static moe_status_t run_ffn(const moe_config_t& c, const Plan& pl, const FfnIo& 
     g.R = c.f_shared;
     g.K = c.d;
     g.ksplit = 1;
-    g.kb_per_split = kblocks(c.d);
+    g.kb_per_split = kbl(c.d);
     g.const_rows = c.T;
     g.b_group_stride = 0;
     g.out_group_stride = c.T;
@@ -296,16 +327,30 @@ static moe_status_t run_ffn(const moe_config_t& c, const Plan& pl, const FfnIo& 
     mu.a0[ncls] = {io.ws_gate, (long long)io.n_shared * c.f_shared, c.d};
     mu.a1[ncls] = {swiglu ? io.ws_up : io.ws_gate, (long long)io.n_shared * c.f_shared, c.d};
     mu.b[ncls] = {io.x, c.T, c.d};
+    if (q8) {
+      mu.a0[ncls].ptr = q8->w->sh_gate;
+      mu.a1[ncls].ptr = swiglu ? q8->w->sh_up : q8->w->sh_gate;
+      mu.b[ncls].ptr = q8->xq_sh;
+      g.a0_scale = q8->w->sh_gate_scale;
+      g.a1_scale = swiglu ? q8->w->sh_up_scale : nullptr;
+      g.b_scale = q8->sx_sh;
+    }
     ++ncls;
   }
   if (ncls == 0) return MOE_OK;
   up.n_classes = ncls;
   const int epi_up = swiglu ? EPI_SWIGLU : EPI_RELU;
   if (tc)
-    MOE_CUDA(launch_tc_gemm(epi_up, pl.bn_up, mu, up, num_sms(), s));
+    MOE_CUDA(launch_tc_gemm(epi_up, pl.bn_up, mu, up, num_sms(), s, q8 != nullptr));
   else
     MOE_CUDA(launch_simt_gemm(epi_up, c.dtype, up, (int)std::min<long long>(io.routed_rows, 1LL << 30), s));
   if (stage_marks) MOE_TRY(mark_stage(5, s));
+  if (q8) {  // E4M3 rows of the stored bf16 h
+    MOE_CUDA(launch_quantize_e4m3(io.routed_rows, c.f, io.h, c.f, q8->hq, c.f, q8->sh, s));
+    if (io.n_shared > 0)
+      MOE_CUDA(launch_quantize_e4m3((long long)io.n_shared * c.T, c.f_shared, io.h_sh, c.f_shared, q8->hq_sh,
+                                    c.f_shared, q8->sh_sh, s));
+  }
 
   // ---- down projection: y = w * (h W_down^T), K split into `ksplit` partial outputs
   GemmParams dn;
@@ -337,8 +382,14 @@ static moe_status_t run_ffn(const moe_config_t& c, const Plan& pl, const FfnIo& 
     g.group_map = io.group_map;
     g.n_wgroups = io.group_map ? io.n_wgroups : io.n_routed;
     md.a0[ncls] = {io.w_down, (long long)g.n_wgroups * c.d, c.f};
-    md.a1[ncls] = md.a0[ncls];
     md.b[ncls] = {io.h, io.routed_rows, c.f};
+    if (q8) {
+      md.a0[ncls].ptr = q8->w->down;
+      md.b[ncls].ptr = q8->hq;
+      g.a0_scale = q8->w->down_scale;
+      g.b_scale = q8->sh;
+    }
+    md.a1[ncls] = md.a0[ncls];
     ++ncls;
   }
   if (io.n_shared > 0) {
@@ -347,7 +398,7 @@ static moe_status_t run_ffn(const moe_config_t& c, const Plan& pl, const FfnIo& 
     g.R = c.d;
     g.K = c.f_shared;
     g.ksplit = 1;
-    g.kb_per_split = kblocks(c.f_shared);
+    g.kb_per_split = kbl(c.f_shared);
     g.const_rows = c.T;
     g.b_group_stride = c.T;
     g.out_group_stride = c.T;
@@ -358,13 +409,19 @@ static moe_status_t run_ffn(const moe_config_t& c, const Plan& pl, const FfnIo& 
     g.a_ld = c.f_shared;
     g.b_ld = c.f_shared;
     md.a0[ncls] = {io.ws_down, (long long)io.n_shared * c.d, c.f_shared};
-    md.a1[ncls] = md.a0[ncls];
     md.b[ncls] = {io.h_sh, (long long)io.n_shared * c.T, c.f_shared};
+    if (q8) {
+      md.a0[ncls].ptr = q8->w->sh_down;
+      md.b[ncls].ptr = q8->hq_sh;
+      g.a0_scale = q8->w->sh_down_scale;
+      g.b_scale = q8->sh_sh;
+    }
+    md.a1[ncls] = md.a0[ncls];
     ++ncls;
   }
   dn.n_classes = ncls;
   if (tc)
-    return cuda_status(launch_tc_gemm(EPI_DOWN, pl.bn_down, md, dn, num_sms(), s));
+    return cuda_status(launch_tc_gemm(EPI_DOWN, pl.bn_down, md, dn, num_sms(), s, q8 != nullptr));
   return cuda_status(launch_simt_gemm(EPI_DOWN, c.dtype, dn, (int)std::min<long long>(io.routed_rows, 1LL << 30), s));
 }
 
@@ -517,25 +574,45 @@ moe_status_t moe_combine(const moe_config_t* cfg, const float* y_perm, const int
                                     (cudaStream_t)stream));
 }
 
-moe_status_t moe_layer_forward(const moe_config_t* cfg, const void* x, const void* w_router, const float* bias,
-                               const void* w_gate, const void* w_up, const void* w_down, const void* ws_gate,
-                               const void* ws_up, const void* ws_down, void* out, float* logits_out,
-                               int32_t* topk_idx_out, float* topk_w_out, int32_t* counts_out, moe_lis_t* lis_out,
-                               void* ws, size_t ws_bytes, moe_stream_t stream) {
-  MOE_TRY(check_cfg(cfg));
-  const moe_config_t& c = *cfg;
-  if (!x || !w_router || !w_gate || !w_down || !out) return MOE_ERR_INVALID_ARG;
-  if (c.act == MOE_SWIGLU && !w_up) return MOE_ERR_INVALID_ARG;
-  if (c.n_shared > 0 && (!ws_gate || !ws_down || (c.act == MOE_SWIGLU && !ws_up))) return MOE_ERR_INVALID_ARG;
-  for (const void* p : std::initializer_list<const void*>{x, w_router, (const void*)bias, w_gate, w_up, w_down, ws_gate, ws_up, ws_down, out,
-                        (const void*)logits_out, (const void*)topk_idx_out, (const void*)topk_w_out,
-                        (const void*)counts_out, (const void*)lis_out})
-    if (p && !aligned16(p)) return MOE_ERR_INVALID_ARG;
+}  // extern "C"
+
+// The 8-bit path's buffers, after the bf16 layer's workspace.
+struct Fp8Layout {
+  size_t xq, sx, hq, sh, xq_sh, sx_sh, hq_sh, sh_sh, total;
+};
+
+static Fp8Layout make_fp8_layout(const moe_config_t& c, size_t base) {
+  Fp8Layout F;
+  size_t off = base;
+  auto take = [&](size_t bytes) {
+    const size_t o = off;
+    off += align256(bytes);
+    return o;
+  };
+  const size_t Tk = (size_t)c.T * c.k;
+  const size_t nsT = (size_t)c.n_shared * c.T;
+  F.xq = take(Tk * c.d);
+  F.sx = take(Tk * 4);
+  F.hq = take(Tk * c.f);
+  F.sh = take(Tk * 4);
+  F.xq_sh = take(c.n_shared ? (size_t)c.T * c.d : 0);
+  F.sx_sh = take(c.n_shared ? (size_t)c.T * 4 : 0);
+  F.hq_sh = take(nsT * std::max(c.f_shared, 0));
+  F.sh_sh = take(nsT * 4);
+  F.total = off;
+  return F;
+}
+
+// Route -> histogram/LIS -> permute -> expert FFN -> combine; the expert weights
+// are bf16 (w_gate ...) or, with wq, E4M3 codes and scales.
+static moe_status_t layer_forward_impl(const moe_config_t& c, const void* x, const void* w_router, const float* bias,
+                                       const void* w_gate, const void* w_up, const void* w_down, const void* ws_gate,
+                                       const void* ws_up, const void* ws_down, const moe_fp8_experts_t* wq, void* out,
+                                       float* logits_out, int32_t* topk_idx_out, float* topk_w_out,
+                                       int32_t* counts_out, moe_lis_t* lis_out, void* h_out, void* h_shared_out,
+                                       int32_t* perm_out, void* ws, cudaStream_t s) {
   const Plan pl = make_plan(c);
   const Layout L = make_layout(c, pl);
-  MOE_TRY(check_ws(c, ws, ws_bytes, L.total));
-  MOE_TRY(check_device());
-  cudaStream_t s = (cudaStream_t)stream;
   int* status = at<int>(ws, L.status);
   float* logits = logits_out ? logits_out : at<float>(ws, L.logits);
   int32_t* idx = topk_idx_out ? topk_idx_out : at<int32_t>(ws, L.idx);
@@ -593,17 +670,118 @@ moe_status_t moe_layer_forward(const moe_config_t* cfg, const void* x, const voi
   io.ws_down = ws_down;
   io.h_sh = at<void>(ws, L.h_sh);
   io.y_sh = at<float>(ws, L.y_sh);
+  // K split of the down projection: the plan's, re-cut into 128-element k-blocks
+  // for 8-bit operands (never more splits than the plan sized y for)
+  int ksplit = pl.ksplit, kbps = pl.kbps;
+  Fp8Io q8;
+  if (wq) {
+    const Fp8Layout F = make_fp8_layout(c, L.total);
+    q8 = {wq,
+          at<uint8_t>(ws, F.xq), at<float>(ws, F.sx), at<uint8_t>(ws, F.hq), at<float>(ws, F.sh),
+          at<uint8_t>(ws, F.xq_sh), at<float>(ws, F.sx_sh), at<uint8_t>(ws, F.hq_sh), at<float>(ws, F.sh_sh)};
+    io.q8 = &q8;
+    const int kb = kblocks8(c.f);
+    const int ks = std::min(pl.ksplit, kb);
+    kbps = (kb + ks - 1) / ks;
+    ksplit = (kb + kbps - 1) / kbps;
+  }
   // Top-1 routing without shared experts: each token has exactly one weighted
   // expert output, so the down projection's epilogue scatters it straight into
   // `out` and the combine kernel (and the fp32 y_perm round trip) disappears.
-  const bool fuse_combine = c.k == 1 && c.n_shared == 0 && pl.ksplit == 1 && c.dtype == MOE_BF16;
+  const bool fuse_combine = c.k == 1 && c.n_shared == 0 && ksplit == 1 && c.dtype == MOE_BF16;
   io.out_k1 = fuse_combine ? out : nullptr;
-  MOE_TRY(run_ffn(c, pl, io, pl.ksplit, pl.kbps, status, s, true));
+  MOE_TRY(run_ffn(c, pl, io, ksplit, kbps, status, s, true));
   MOE_TRY(mark_stage(6, s));
+  // inspection copies (the stored h rows and the task of each segment row)
+  if (h_out) MOE_CUDA(cudaMemcpyAsync(h_out, io.h, (size_t)Tk * c.f * 2, cudaMemcpyDeviceToDevice, s));
+  if (h_shared_out && c.n_shared > 0)
+    MOE_CUDA(cudaMemcpyAsync(h_shared_out, io.h_sh, (size_t)c.n_shared * c.T * c.f_shared * 2,
+                             cudaMemcpyDeviceToDevice, s));
+  if (perm_out) MOE_CUDA(cudaMemcpyAsync(perm_out, perm, (size_t)Tk * 4, cudaMemcpyDeviceToDevice, s));
   if (!fuse_combine)
-    MOE_CUDA(launch_combine(c.dtype, c.T, c.d, c.k, pl.ksplit, io.y, Tk * c.d, inv_perm, c.n_shared, io.y_sh,
+    MOE_CUDA(launch_combine(c.dtype, c.T, c.d, c.k, ksplit, io.y, Tk * c.d, inv_perm, c.n_shared, io.y_sh,
                             (long long)c.n_shared * c.T * c.d, out, s));
   return mark_stage(7, s);
+}
+
+extern "C" {
+
+moe_status_t moe_layer_forward(const moe_config_t* cfg, const void* x, const void* w_router, const float* bias,
+                               const void* w_gate, const void* w_up, const void* w_down, const void* ws_gate,
+                               const void* ws_up, const void* ws_down, void* out, float* logits_out,
+                               int32_t* topk_idx_out, float* topk_w_out, int32_t* counts_out, moe_lis_t* lis_out,
+                               void* ws, size_t ws_bytes, moe_stream_t stream) {
+  MOE_TRY(check_cfg(cfg));
+  const moe_config_t& c = *cfg;
+  if (!x || !w_router || !w_gate || !w_down || !out) return MOE_ERR_INVALID_ARG;
+  if (c.act == MOE_SWIGLU && !w_up) return MOE_ERR_INVALID_ARG;
+  if (c.n_shared > 0 && (!ws_gate || !ws_down || (c.act == MOE_SWIGLU && !ws_up))) return MOE_ERR_INVALID_ARG;
+  for (const void* p : std::initializer_list<const void*>{x, w_router, (const void*)bias, w_gate, w_up, w_down, ws_gate, ws_up, ws_down, out,
+                        (const void*)logits_out, (const void*)topk_idx_out, (const void*)topk_w_out,
+                        (const void*)counts_out, (const void*)lis_out})
+    if (p && !aligned16(p)) return MOE_ERR_INVALID_ARG;
+  MOE_TRY(check_ws(c, ws, ws_bytes, make_layout(c, make_plan(c)).total));
+  MOE_TRY(check_device());
+  return layer_forward_impl(c, x, w_router, bias, w_gate, w_up, w_down, ws_gate, ws_up, ws_down, nullptr, out,
+                            logits_out, topk_idx_out, topk_w_out, counts_out, lis_out, nullptr, nullptr, nullptr, ws,
+                            (cudaStream_t)stream);
+}
+
+static moe_status_t check_fp8_cfg(const moe_config_t* cfg) {
+  MOE_TRY(check_cfg(cfg));
+  const moe_config_t& c = *cfg;
+  if (c.dtype != MOE_BF16) return MOE_ERR_UNSUPPORTED;
+  if (c.d % 16 || c.f % 16 || (c.n_shared && c.f_shared % 16)) return MOE_ERR_UNSUPPORTED;  // 16-byte code rows
+  return MOE_OK;
+}
+
+moe_status_t moe_fp8_workspace_size(const moe_config_t* cfg, size_t* bytes) {
+  MOE_TRY(check_fp8_cfg(cfg));
+  if (!bytes) return MOE_ERR_INVALID_ARG;
+  *bytes = make_fp8_layout(*cfg, make_layout(*cfg, make_plan(*cfg)).total).total;
+  return MOE_OK;
+}
+
+moe_status_t moe_quantize_e4m3(int64_t rows, int64_t cols, const void* src, uint8_t* codes, float* scales,
+                               moe_stream_t stream) {
+  if (rows < 0 || cols < 8 || cols % 16 || cols > (1LL << 30)) return rows < 0 || cols < 8 ? MOE_ERR_INVALID_ARG
+                                                                                          : MOE_ERR_UNSUPPORTED;
+  if (rows == 0) return MOE_OK;
+  if (!src || !codes || !scales || !aligned16(src) || !aligned16(codes) || ((uintptr_t)scales & 3u))
+    return MOE_ERR_INVALID_ARG;
+  MOE_TRY(check_device());
+  return cuda_status(launch_quantize_e4m3(rows, (int)cols, src, cols, codes, cols, scales, (cudaStream_t)stream));
+}
+
+moe_status_t moe_layer_forward_fp8(const moe_config_t* cfg, const void* x, const void* w_router, const float* bias,
+                                   const moe_fp8_experts_t* wq, void* out, float* logits_out, int32_t* topk_idx_out,
+                                   float* topk_w_out, int32_t* counts_out, moe_lis_t* lis_out, void* h_out,
+                                   void* h_shared_out, int32_t* perm_out, void* ws, size_t ws_bytes,
+                                   moe_stream_t stream) {
+  MOE_TRY(check_fp8_cfg(cfg));
+  const moe_config_t& c = *cfg;
+  const bool swiglu = c.act == MOE_SWIGLU;
+  if (!x || !w_router || !wq || !out) return MOE_ERR_INVALID_ARG;
+  if (!wq->gate || !wq->gate_scale || !wq->down || !wq->down_scale) return MOE_ERR_INVALID_ARG;
+  if (swiglu && (!wq->up || !wq->up_scale)) return MOE_ERR_INVALID_ARG;
+  if (c.n_shared > 0 && (!wq->sh_gate || !wq->sh_gate_scale || !wq->sh_down || !wq->sh_down_scale ||
+                         (swiglu && (!wq->sh_up || !wq->sh_up_scale))))
+    return MOE_ERR_INVALID_ARG;
+  for (const void* p : std::initializer_list<const void*>{x, w_router, (const void*)bias, out, (const void*)logits_out,
+                        (const void*)topk_idx_out, (const void*)topk_w_out, (const void*)counts_out,
+                        (const void*)lis_out, wq->gate, wq->up, wq->down, wq->sh_gate, wq->sh_up, wq->sh_down,
+                        h_out, h_shared_out, (const void*)perm_out})
+    if (p && !aligned16(p)) return MOE_ERR_INVALID_ARG;
+  for (const float* p : {wq->gate_scale, wq->up_scale, wq->down_scale, wq->sh_gate_scale, wq->sh_up_scale,
+                         wq->sh_down_scale})
+    if (p && ((uintptr_t)p & 3u)) return MOE_ERR_INVALID_ARG;
+  size_t need = 0;
+  MOE_TRY(moe_fp8_workspace_size(cfg, &need));
+  MOE_TRY(check_ws(c, ws, ws_bytes, need));
+  MOE_TRY(check_device());
+  return layer_forward_impl(c, x, w_router, bias, nullptr, nullptr, nullptr, nullptr, nullptr, nullptr, wq, out,
+                            logits_out, topk_idx_out, topk_w_out, counts_out, lis_out, h_out, h_shared_out, perm_out,
+                            ws, (cudaStream_t)stream);
 }
 
 // ------------------------------------------------------------------ atomic experts

@@ -119,7 +119,7 @@ struct GemmClass {
   int R;                     // output features per group (rows of A per group)
   int K;                     // reduction length
   int ksplit;                // K is cut into ksplit contiguous ranges (partial outputs)
-  int kb_per_split;          // 64-wide k-blocks per range
+  int kb_per_split;          // k-blocks (64 bf16 or 128 E4M3 elements) per range
   const int* seg_off;        // device [n_groups + 1]: B/out rows of group g (nullable)
   int max_row;               // seg_off entries and perm values must lie in [0, max_row]
   int const_rows;            // rows per group when seg_off == nullptr
@@ -141,6 +141,11 @@ struct GemmClass {
   float* sel_w;              // [T, k] gate weights
   int32_t* lrank;            // [T, k] rank of task (t, s) among the tile's tasks of its expert (nullable)
   int32_t* tile_cnt;         // [tiles][m] tasks per expert in each 128-token tile (with lrank)
+  // 8-bit operands (launch_tc_gemm with f8): fp32 scale of each row of A (weight
+  // rows, indexed like the A operand) and of B (activation rows)
+  const float* a0_scale;
+  const float* a1_scale;
+  const float* b_scale;
   // SIMT path only (fp32 / bf16 element pointers, row-major)
   const void* a0;            // [n_groups * R, K]
   const void* a1;            // second matrix (SwiGLU up) or nullptr
@@ -158,7 +163,7 @@ struct GemmParams {
 // Tensor-core grouped GEMM (bf16 in, fp32 accumulate). Tensor maps are built
 // from the pointers in `maps` (see tc_gemm.cu). mats = 2 for SwiGLU.
 struct TcOperand {
-  const void* ptr;     // bf16 [rows, K] row-major
+  const void* ptr;     // bf16 (or E4M3 codes with f8) [rows, K] row-major
   long long rows;
   long long K;
 };
@@ -166,7 +171,7 @@ struct TcMaps {
   TcOperand a0[2], a1[2], b[2];
 };
 cudaError_t launch_tc_gemm(int epi, int bn, const TcMaps& maps, const GemmParams& p, int num_ctas,
-                           cudaStream_t s);
+                           cudaStream_t s, bool f8 = false);
 int tc_pick_bn(int epi, double avg_rows_per_group);
 // Router logits + top-k softmax (+ per-tile expert counts and task ranks when lrank
 // and tile_cnt are given) in one tensor-core launch (EPI_ROUTE); logits nullable.
@@ -238,6 +243,10 @@ cudaError_t launch_atomic_experts(int T, int d, int K, int act, const void* x, c
                                   const int32_t* idx, const float* g, float* coef, void* out, long long n_experts,
                                   unsigned* bar, bool bar_zeroed, unsigned long long limit_ns, int* status,
                                   cudaStream_t s);
+// Per-row E4M3 codes + fp32 scales of bf16 rows [rows, cols] (row strides in
+// elements, multiples of 8; src 16-byte and dst 8-byte aligned).
+cudaError_t launch_quantize_e4m3(long long rows, int cols, const void* src, long long src_ld, uint8_t* dst,
+                                 long long dst_ld, float* scale, cudaStream_t s);
 // Records the profiling hook's event i (moe_set_stage_events) on `s`, if one is set.
 cudaError_t mark_stage_event(int i, cudaStream_t s);
 

@@ -16,6 +16,12 @@
 // weights [out, in] and row-major activations), staged by TMA with the 128-byte
 // swizzle. One tile = the full K loop (or one of `ksplit` K ranges).
 //
+// 8-bit variant (F8): both operands are E4M3 codes with one fp32 scale per row
+// (weight output channel, activation row); the MMA is kind::f8f6f4 and the
+// epilogue multiplies each accumulator by its two scales. A 128-byte swizzle row
+// then holds 128 elements, so stages, boxes and descriptors keep their byte sizes
+// and only the K elements per k-block double.
+//
 // Warp roles (192 threads): warp 0 = TMA producer, warp 1 = MMA issuer (and TMEM
 // owner), warps 2..5 = epilogue (TMEM -> registers -> activation -> global).
 // The accumulator is double-buffered in TMEM when it fits (2 x mats x BN <= 512
@@ -34,6 +40,7 @@ namespace moe {
 
 constexpr int TC_BM = 128;
 constexpr int TC_BK = 64;  // bf16 elements of one 128-byte swizzle row
+constexpr int TC_BK8 = 128;  // E4M3 elements of one 128-byte swizzle row
 constexpr int TC_THREADS = 192;
 constexpr int TC_MAX_GROUPS = 1040;
 constexpr int TC_SMEM_BUDGET = 200 * 1024;
@@ -93,6 +100,16 @@ __device__ __forceinline__ void umma_bf16(uint32_t d_tmem, uint64_t adesc, uint6
       "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
       : "memory");
 }
+// D(tmem) (+)= A * B^T, kind::f8f6f4 with both operands E4M3 (fp32 accumulator)
+__device__ __forceinline__ void umma_e4m3(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                          uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], %1, %2, %3, p;\n\t}\n" ::"r"(d_tmem),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
 // Arrive on `bar` once every tcgen05.mma issued so far by this thread completed.
 __device__ __forceinline__ void umma_commit(uint64_t* bar) {
   asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(smem_u32(bar))
@@ -123,6 +140,10 @@ __device__ __forceinline__ uint64_t sdesc_sw128(uint32_t saddr) {
 // Instruction descriptor, kind::f16: D fp32, A and B bf16, both K-major.
 __device__ __forceinline__ uint32_t idesc_bf16(int M, int N) {
   return (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
+}
+// Instruction descriptor, kind::f8f6f4: D fp32, A and B E4M3 (format code 0), both K-major.
+__device__ __forceinline__ uint32_t idesc_e4m3(int M, int N) {
+  return (1u << 4) | ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
 }
 
 // Barrier of the four epilogue warps only (named barrier 1; 0 is __syncthreads),
@@ -224,7 +245,7 @@ struct SchedSmem {
   int brow[TC_MAX_GROUPS];
 };
 
-template <int BN>
+template <int BN, int BKE>
 __device__ __forceinline__ void decode_tile(const GemmParams& p, const SchedSmem& s, int G, int w, TileInfo& ti) {
   int lo = 0, hi = G - 1;  // largest gi with tile_start[gi] <= w
   while (lo < hi) {
@@ -253,7 +274,7 @@ __device__ __forceinline__ void decode_tile(const GemmParams& p, const SchedSmem
     if (wg < 0 || wg >= c.n_wgroups) wg = 0;  // (validated where the map is written)
   }
   ti.a_row = wg * c.R + ti.mt * TC_BM;
-  const int KB = (c.K + TC_BK - 1) / TC_BK;
+  const int KB = (c.K + BKE - 1) / BKE;
   ti.kb0 = ti.ks * c.kb_per_split;
   ti.kb1 = min(KB, ti.kb0 + c.kb_per_split);
 }
@@ -302,7 +323,7 @@ __device__ __forceinline__ void store_out(const GemmClass& c, const TileInfo& ti
   }
 }
 
-template <int BN, int MATS, int EPI>
+template <int BN, int MATS, int EPI, bool F8>
 __global__ void __launch_bounds__(TC_THREADS, 1)
     tc_grouped_gemm_kernel(const __grid_constant__ CUtensorMap tA0_0, const __grid_constant__ CUtensorMap tA1_0,
                            const __grid_constant__ CUtensorMap tB_0, const __grid_constant__ CUtensorMap tA0_1,
@@ -310,11 +331,14 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
                            const __grid_constant__ GemmParams p) {
   using S = TcShape<BN, MATS>;
   constexpr int STAGES = S::STAGES;
+  constexpr int BKE = F8 ? TC_BK8 : TC_BK;  // K elements per k-block (one 128-byte row)
+  static_assert(!F8 || EPI == EPI_SWIGLU || EPI == EPI_RELU || EPI == EPI_DOWN, "8-bit operands: expert GEMMs only");
 
   __shared__ SchedSmem sched;
   __shared__ __align__(8) uint64_t full_bar[STAGES], empty_bar[STAGES], accf_bar[2], acce_bar[2], drain_bar;
   __shared__ float aux_w[4][EPI == EPI_DOWN ? BN : 1];  // per epilogue warp: row weights of the tile
   __shared__ int aux_d[4][EPI == EPI_DOWN ? BN : 1];    // and destination tokens (fused top-1 combine)
+  __shared__ float aux_s[4][F8 && EPI != EPI_DOWN ? BN : 1];  // F8: activation-row scales of the tile
   constexpr int RMASK_M = EPI == EPI_ROUTE ? ROUTE_MAX_M : 1;
   __shared__ __align__(16) float rbias[RMASK_M];  // ROUTE: router bias (zeros when absent)
   __shared__ uint32_t rmask[EPI == EPI_ROUTE ? 2 : 1][4][RMASK_M];  // ROUTE: expert -> lanes holding it
@@ -415,7 +439,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
     bool ok = true;
     for (int w = blockIdx.x; w < total && ok; w += gridDim.x) {
       TileInfo ti;
-      decode_tile<BN>(p, sched, G, w, ti);
+      decode_tile<BN, BKE>(p, sched, G, w, ti);
       const CUtensorMap* mA0 = ti.cls ? &tA0_1 : &tA0_0;
       const CUtensorMap* mA1 = ti.cls ? &tA1_1 : &tA1_0;
       const CUtensorMap* mB = ti.cls ? &tB_1 : &tB_0;
@@ -426,9 +450,9 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
         }
         uint8_t* st = smem_gen + stage * S::STAGE_BYTES;
         mbar_arrive_expect_tx(&full_bar[stage], S::STAGE_BYTES);
-        tma_load_2d(mA0, &full_bar[stage], st, kb * TC_BK, ti.a_row);
-        if (MATS == 2) tma_load_2d(mA1, &full_bar[stage], st + S::A_BYTES, kb * TC_BK, ti.a_row);
-        tma_load_2d(mB, &full_bar[stage], st + MATS * S::A_BYTES, kb * TC_BK, ti.b_row);
+        tma_load_2d(mA0, &full_bar[stage], st, kb * BKE, ti.a_row);
+        if (MATS == 2) tma_load_2d(mA1, &full_bar[stage], st + S::A_BYTES, kb * BKE, ti.a_row);
+        tma_load_2d(mB, &full_bar[stage], st + MATS * S::A_BYTES, kb * BKE, ti.b_row);
         last_parity[stage] = (int)phase;
         if (++stage == STAGES) {
           stage = 0;
@@ -456,7 +480,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
     bool ok = true;
     for (int w = blockIdx.x; w < total && ok; w += gridDim.x) {
       TileInfo ti;
-      decode_tile<BN>(p, sched, G, w, ti);
+      decode_tile<BN, BKE>(p, sched, G, w, ti);
       if (!mbar_wait(&acce_bar[acc], acc_phase ^ 1u, lim, abort_flag)) {
         ok = false;
         break;
@@ -464,7 +488,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
       tc_fence_after();
       const uint32_t d_tmem = tmem_base + (uint32_t)(acc * S::ACC_COLS);
       const int n_inst = max(16, (ti.rows_in_tile + 15) & ~15);
-      const uint32_t idesc = idesc_bf16(TC_BM, n_inst);
+      const uint32_t idesc = F8 ? idesc_e4m3(TC_BM, n_inst) : idesc_bf16(TC_BM, n_inst);
       for (int kb = ti.kb0; kb < ti.kb1; ++kb) {
         if (!mbar_wait(&full_bar[stage], phase, lim, abort_flag)) {
           ok = false;
@@ -476,11 +500,16 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
         const uint64_t da1 = sdesc_sw128(st + S::A_BYTES);
         const uint64_t db = sdesc_sw128(st + MATS * S::A_BYTES);
 #pragma unroll
-        for (int kk = 0; kk < TC_BK / 16; ++kk) {
+        for (int kk = 0; kk < 4; ++kk) {
           const uint32_t accum = (kb > ti.kb0 || kk > 0) ? 1u : 0u;
-          // advance 16 bf16 (32 B) along K inside the swizzle atom: +2 in the >>4 address field
-          umma_bf16(d_tmem, da0 + 2 * kk, db + 2 * kk, idesc, accum);
-          if (MATS == 2) umma_bf16(d_tmem + BN, da1 + 2 * kk, db + 2 * kk, idesc, accum);
+          // one MMA takes 32 B of K (16 bf16 or 32 E4M3): +2 in the >>4 address field
+          if (F8) {
+            umma_e4m3(d_tmem, da0 + 2 * kk, db + 2 * kk, idesc, accum);
+            if (MATS == 2) umma_e4m3(d_tmem + BN, da1 + 2 * kk, db + 2 * kk, idesc, accum);
+          } else {
+            umma_bf16(d_tmem, da0 + 2 * kk, db + 2 * kk, idesc, accum);
+            if (MATS == 2) umma_bf16(d_tmem + BN, da1 + 2 * kk, db + 2 * kk, idesc, accum);
+          }
         }
         umma_commit(&empty_bar[stage]);
         if (++stage == STAGES) {
@@ -518,7 +547,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
     uint32_t acc_phase = 0;
     for (int w = blockIdx.x; w < total; w += gridDim.x, ++iter) {
       TileInfo ti;
-      decode_tile<BN>(p, sched, G, w, ti);
+      decode_tile<BN, BKE>(p, sched, G, w, ti);
       const GemmClass& c = p.cls[0];
       const int t = ti.mt * TC_BM + q * 32 + lane;  // token
       const bool tv_ok = t < c.R;
@@ -623,21 +652,28 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
     uint32_t acc_phase = 0;
     for (int w = blockIdx.x; w < total; w += gridDim.x) {
       TileInfo ti;
-      decode_tile<BN>(p, sched, G, w, ti);
+      decode_tile<BN, BKE>(p, sched, G, w, ti);
       const GemmClass& c = p.cls[ti.cls];
       const int feature = ti.mt * TC_BM + q * 32 + lane;
       const bool fvalid = feature < c.R;
       const bool has_k = ti.kb1 > ti.kb0;  // an empty K range leaves the accumulator unwritten
       const float bias = (EPI == EPI_LOGITS && c.bias && fvalid) ? c.bias[feature] : 0.f;
+      // F8: scale of this lane's weight row (index = weight-matrix row of the feature)
+      const float sa0 = (F8 && fvalid) ? c.a0_scale[ti.a_row + q * 32 + lane] : 1.f;
+      const float sa1 = (F8 && MATS == 2 && fvalid) ? c.a1_scale[ti.a_row + q * 32 + lane] : 1.f;
       // Row data of the whole tile (gate weight, destination token), fetched into this
       // warp's shared-memory slice before waiting for the accumulator so the loads
       // overlap the MMAs; the chunk loop below then reads it with broadcasts.
       if (EPI == EPI_DOWN) {
         for (int j = lane; j < BN; j += 32) {
           const RowAux a = load_row_aux<EPI>(c, ti, j);
-          aux_w[q][j] = a.w;
+          // F8: the activation row's scale folds into the row weight
+          aux_w[q][j] = (F8 && j < ti.rows_in_tile) ? a.w * c.b_scale[ti.b_row + j] : a.w;
           aux_d[q][j] = a.dst;
         }
+        __syncwarp();
+      } else if (F8) {
+        for (int j = lane; j < BN; j += 32) aux_s[q][j] = j < ti.rows_in_tile ? c.b_scale[ti.b_row + j] : 0.f;
         __syncwarp();
       }
       const bool got = mbar_wait(&accf_bar[acc], acc_phase, lim, abort_flag);
@@ -658,10 +694,17 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
         if (fvalid) {
 #pragma unroll
           for (int j = 0; j < 16; ++j)
-            if (j < jn)
-              store_out<EPI>(c, ti, feature, c0 + j, has_k ? __uint_as_float(r0[j]) : 0.f,
-                             (MATS == 2 && has_k) ? __uint_as_float(r1[j]) : 0.f, bias,
-                             EPI == EPI_DOWN ? aux_w[q][c0 + j] : 1.f, EPI == EPI_DOWN ? aux_d[q][c0 + j] : -1);
+            if (j < jn) {
+              float v0 = has_k ? __uint_as_float(r0[j]) : 0.f;
+              float v1 = (MATS == 2 && has_k) ? __uint_as_float(r1[j]) : 0.f;
+              if (F8) {
+                const float sb = EPI == EPI_DOWN ? 1.f : aux_s[q][c0 + j];
+                v0 = v0 * sa0 * sb;
+                v1 = v1 * sa1 * sb;
+              }
+              store_out<EPI>(c, ti, feature, c0 + j, v0, v1, bias, EPI == EPI_DOWN ? aux_w[q][c0 + j] : 1.f,
+                             EPI == EPI_DOWN ? aux_d[q][c0 + j] : -1);
+            }
         }
       }
       tc_fence_before();
@@ -702,34 +745,36 @@ static EncodeTiledFn encode_fn() {
   return fn;
 }
 
-// bf16 [rows, K] row-major, box = 64 (K) x box_rows, 128-byte swizzle; out-of-range
-// elements read as zero.
-static bool make_map(CUtensorMap* m, const TcOperand& op, int box_rows) {
+// [rows, K] row-major, bf16 or (u8) E4M3 codes; box = one 128-byte row of K x
+// box_rows, 128-byte swizzle; out-of-range elements read as zero.
+static bool make_map(CUtensorMap* m, const TcOperand& op, int box_rows, bool u8) {
   EncodeTiledFn enc = encode_fn();
   if (!enc || !op.ptr || op.rows <= 0 || op.K <= 0) return false;
+  const int es_bytes = u8 ? 1 : 2;
+  if ((op.K * es_bytes) % 16) return false;  // row pitch must be a multiple of 16 bytes
   cuuint64_t dims[2] = {(cuuint64_t)op.K, (cuuint64_t)op.rows};
-  cuuint64_t strides[1] = {(cuuint64_t)op.K * 2};
-  cuuint32_t box[2] = {(cuuint32_t)TC_BK, (cuuint32_t)box_rows};
+  cuuint64_t strides[1] = {(cuuint64_t)op.K * es_bytes};
+  cuuint32_t box[2] = {(cuuint32_t)(u8 ? TC_BK8 : TC_BK), (cuuint32_t)box_rows};
   cuuint32_t es[2] = {1, 1};
-  CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(op.ptr), dims, strides, box, es,
+  CUresult r = enc(m, u8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(op.ptr), dims, strides, box, es,
                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
 }
 
-template <int BN, int MATS, int EPI>
+template <int BN, int MATS, int EPI, bool F8>
 static cudaError_t launch_impl(const TcMaps& maps, const GemmParams& p, int num_ctas, cudaStream_t s) {
   using S = TcShape<BN, MATS>;
   CUtensorMap m[6];
   const int nc = p.n_classes;
   for (int c = 0; c < 2; ++c) {
     const int src = c < nc ? c : 0;
-    if (!make_map(&m[3 * c + 0], maps.a0[src], TC_BM)) return cudaErrorInvalidValue;
+    if (!make_map(&m[3 * c + 0], maps.a0[src], TC_BM, F8)) return cudaErrorInvalidValue;
     const TcOperand& a1 = MATS == 2 ? maps.a1[src] : maps.a0[src];
-    if (!make_map(&m[3 * c + 1], a1, TC_BM)) return cudaErrorInvalidValue;
-    if (!make_map(&m[3 * c + 2], maps.b[src], BN)) return cudaErrorInvalidValue;
+    if (!make_map(&m[3 * c + 1], a1, TC_BM, F8)) return cudaErrorInvalidValue;
+    if (!make_map(&m[3 * c + 2], maps.b[src], BN, F8)) return cudaErrorInvalidValue;
   }
-  auto kern = tc_grouped_gemm_kernel<BN, MATS, EPI>;
+  auto kern = tc_grouped_gemm_kernel<BN, MATS, EPI, F8>;
   static bool attr_set = false;
   if (!attr_set) {
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, S::DYN_SMEM);
@@ -758,9 +803,17 @@ int tc_pick_bn(int epi, double avg) {
 }
 
 cudaError_t launch_tc_gemm(int epi, int bn, const TcMaps& maps, const GemmParams& p, int num_ctas,
-                           cudaStream_t s) {
+                           cudaStream_t s, bool f8) {
+  if (f8) {
+    if (epi != EPI_SWIGLU && epi != EPI_RELU && epi != EPI_DOWN) return cudaErrorInvalidValue;
+    for (int c = 0; c < p.n_classes; ++c)
+      if (!p.cls[c].a0_scale || !p.cls[c].b_scale || (epi == EPI_SWIGLU && !p.cls[c].a1_scale))
+        return cudaErrorInvalidValue;
+  }
 #define MOE_TC_CASE(EPI_, MATS_, BN_) \
-  if (epi == EPI_ && bn == BN_) return launch_impl<BN_, MATS_, EPI_>(maps, p, num_ctas, s);
+  if (epi == EPI_ && bn == BN_ && !f8) return launch_impl<BN_, MATS_, EPI_, false>(maps, p, num_ctas, s);
+#define MOE_TC_CASE8(EPI_, MATS_, BN_) \
+  if (epi == EPI_ && bn == BN_ && f8) return launch_impl<BN_, MATS_, EPI_, true>(maps, p, num_ctas, s);
   MOE_TC_CASE(EPI_LOGITS, 1, 16)
   MOE_TC_CASE(EPI_LOGITS, 1, 32)
   MOE_TC_CASE(EPI_LOGITS, 1, 64)
@@ -784,7 +837,22 @@ cudaError_t launch_tc_gemm(int epi, int bn, const TcMaps& maps, const GemmParams
   MOE_TC_CASE(EPI_ROUTE, 1, 64)
   MOE_TC_CASE(EPI_ROUTE, 1, 128)
   MOE_TC_CASE(EPI_ROUTE, 1, 256)
+  MOE_TC_CASE8(EPI_SWIGLU, 2, 16)
+  MOE_TC_CASE8(EPI_SWIGLU, 2, 32)
+  MOE_TC_CASE8(EPI_SWIGLU, 2, 64)
+  MOE_TC_CASE8(EPI_SWIGLU, 2, 128)
+  MOE_TC_CASE8(EPI_RELU, 1, 16)
+  MOE_TC_CASE8(EPI_RELU, 1, 32)
+  MOE_TC_CASE8(EPI_RELU, 1, 64)
+  MOE_TC_CASE8(EPI_RELU, 1, 128)
+  MOE_TC_CASE8(EPI_RELU, 1, 256)
+  MOE_TC_CASE8(EPI_DOWN, 1, 16)
+  MOE_TC_CASE8(EPI_DOWN, 1, 32)
+  MOE_TC_CASE8(EPI_DOWN, 1, 64)
+  MOE_TC_CASE8(EPI_DOWN, 1, 128)
+  MOE_TC_CASE8(EPI_DOWN, 1, 256)
 #undef MOE_TC_CASE
+#undef MOE_TC_CASE8
   return cudaErrorInvalidValue;
 }
 

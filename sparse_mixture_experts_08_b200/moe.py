@@ -32,7 +32,8 @@ EXPORTS = ["moe_workspace_size", "moe_atomic_workspace_size", "moe_route", "moe_
            "moe_atomic_experts", "moe_atomic_forward", "moe_read_device_status", "moe_status_string",
            "moe_debug_set_wait_limit_ns", "moe_set_stage_events", "moe_launch_count", "moe_route_static",
            "moe_replica_split", "moe_layer_forward_replicated", "moe_floe_pack_down", "moe_floe_calibrate",
-           "moe_floe_workspace_size", "moe_layer_forward_floe"]
+           "moe_floe_workspace_size", "moe_layer_forward_floe", "moe_quantize_e4m3", "moe_fp8_workspace_size",
+           "moe_layer_forward_fp8"]
 
 
 class MoEConfig(ctypes.Structure):
@@ -47,6 +48,13 @@ class MoEAtomicConfig(ctypes.Structure):
 
 
 LIS_BYTES = 16  # moe_lis_t: int32 max_count, int32 argmax_expert, double lis
+
+
+class MoEFp8Experts(ctypes.Structure):
+    """moe_fp8_experts_t: device pointers to E4M3 codes (uint8) and fp32 row scales."""
+    _fields_ = [(name, ctypes.c_void_p) for name in (
+        "gate", "gate_scale", "up", "up_scale", "down", "down_scale", "sh_gate", "sh_gate_scale", "sh_up",
+        "sh_up_scale", "sh_down", "sh_down_scale")]
 
 
 class MoEError(RuntimeError):
@@ -88,6 +96,9 @@ def lib() -> ctypes.CDLL:
             "moe_debug_set_wait_limit_ns": [ctypes.c_uint64],
             "moe_set_stage_events": [P, ctypes.c_int],
             "moe_route_static": [P, P, P, P, P, P, P, P, P, P],
+            "moe_quantize_e4m3": [ctypes.c_int64, ctypes.c_int64, P, P, P, P],
+            "moe_fp8_workspace_size": [P, P],
+            "moe_layer_forward_fp8": [P, P, P, P, P, P, P, P, P, P, P, P, P, P, P, S, P],
         }
         for name, args in sig.items():
             fn = getattr(L, name)
@@ -235,6 +246,48 @@ def moe_layer_forward_floe(cfg, x, w_router, bias, w_gate, w_up, w_down_t, thres
         ctypes.byref(cfg), _p(x), _p(w_router), _p(bias), _p(w_gate), _p(w_up), _p(w_down_t), _p(thresholds),
         _p(out), _p(topk_idx_out), _p(topk_w_out), _p(kept_out), _p(u_out), _p(perm_out), _p(ws), ws.numel(),
         _stream(stream)))
+
+
+def moe_quantize_e4m3(src, codes, scales, stream=None):
+    """Per-row E4M3 codes [rows, cols] (uint8) and fp32 scales [rows] of a bf16 matrix."""
+    rows = src.numel() // src.shape[-1]
+    _check("moe_quantize_e4m3", lib().moe_quantize_e4m3(rows, int(src.shape[-1]), _p(src), _p(codes), _p(scales),
+                                                        _stream(stream)))
+
+
+def moe_fp8_workspace_size(cfg) -> int:
+    n = ctypes.c_size_t(0)
+    _check("moe_fp8_workspace_size", lib().moe_fp8_workspace_size(ctypes.byref(cfg), ctypes.byref(n)))
+    return n.value
+
+
+def moe_layer_forward_fp8(cfg, x, w_router, bias, wq, out, ws, logits_out=None, topk_idx_out=None, topk_w_out=None,
+                          counts_out=None, lis_out=None, h_out=None, h_shared_out=None, perm_out=None, stream=None):
+    """wq: a dict of device tensors as quantize_experts returns (kept alive by the caller)."""
+    st = MoEFp8Experts(**{k: _p(wq.get(k)) for k, _ in MoEFp8Experts._fields_})
+    _check("moe_layer_forward_fp8", lib().moe_layer_forward_fp8(
+        ctypes.byref(cfg), _p(x), _p(w_router), _p(bias), ctypes.byref(st), _p(out), _p(logits_out),
+        _p(topk_idx_out), _p(topk_w_out), _p(counts_out), _p(lis_out), _p(h_out), _p(h_shared_out), _p(perm_out),
+        _p(ws), ws.numel(), _stream(stream)))
+
+
+def quantize_experts(w_gate, w_up, w_down, ws_gate=None, ws_up=None, ws_down=None, stream=None) -> dict:
+    """E4M3 codes + per-output-channel scales of every expert weight (device bf16
+    tensors in, device tensors out), keyed as moe_fp8_experts_t's fields."""
+    out = {}
+    for key, w in (("gate", w_gate), ("up", w_up), ("down", w_down), ("sh_gate", ws_gate), ("sh_up", ws_up),
+                   ("sh_down", ws_down)):
+        if w is None:
+            continue
+        codes = torch.empty(w.shape, dtype=torch.uint8, device=w.device)
+        scales = torch.empty(w.shape[:-1], dtype=torch.float32, device=w.device)
+        moe_quantize_e4m3(w, codes, scales, stream=stream)
+        out[key], out[key + "_scale"] = codes, scales
+    return out
+
+
+def fp8_workspace(cfg, device="cuda") -> torch.Tensor:
+    return torch.zeros(max(moe_fp8_workspace_size(cfg), 256), dtype=torch.uint8, device=device)
 
 
 def floe_workspace(cfg, device="cuda") -> torch.Tensor:

@@ -182,3 +182,42 @@ def test_floe_entry_points_validate_on_the_host():
                                       a, 1 << 30, None) == moe.ERR_INVALID_ARG  # thresholds missing
     assert lib.moe_layer_forward_floe(ctypes.byref(ok), a, a, None, a, a, a, a, a, None, None, None, None, None,
                                       a, n.value - 256, None) == moe.ERR_WORKSPACE
+
+
+def test_fp8_entry_points_validate_on_the_host():
+    lib = moe.moe.lib()
+    a = _fake(1 << 24)
+    ok = MoEConfig(16, 256, 320, 4, 2, 1, 64, moe.BF16, moe.SWIGLU, 0)
+    n = ctypes.c_size_t(0)
+    base = ctypes.c_size_t(0)
+    assert lib.moe_fp8_workspace_size(ctypes.byref(ok), ctypes.byref(n)) == moe.OK
+    assert lib.moe_workspace_size(ctypes.byref(ok), ctypes.byref(base)) == moe.OK
+    # the bf16 workspace plus codes of x and h (bytes) and their row scales
+    assert n.value >= base.value + 16 * 2 * (256 + 320 + 8) + 16 * (256 + 64 + 4)
+    for bad in (MoEConfig(16, 256, 320, 4, 2, 0, 0, moe.F32, moe.SWIGLU, 0),    # bf16 layers only
+                MoEConfig(16, 264, 320, 4, 2, 0, 0, moe.BF16, moe.SWIGLU, 0),   # d % 16
+                MoEConfig(16, 256, 328, 4, 2, 0, 0, moe.BF16, moe.SWIGLU, 0),   # f % 16
+                MoEConfig(16, 256, 320, 4, 2, 1, 72, moe.BF16, moe.SWIGLU, 0)):  # f_shared % 16
+        assert lib.moe_fp8_workspace_size(ctypes.byref(bad), ctypes.byref(n)) == moe.ERR_UNSUPPORTED
+    assert lib.moe_fp8_workspace_size(ctypes.byref(ok), ctypes.byref(n)) == moe.OK
+    # quantizer: rows of 16-byte multiples only, aligned pointers
+    assert lib.moe_quantize_e4m3(4, 24, a, a, a, None) == moe.ERR_UNSUPPORTED
+    assert lib.moe_quantize_e4m3(-1, 32, a, a, a, None) == moe.ERR_INVALID_ARG
+    assert lib.moe_quantize_e4m3(4, 32, _fake((1 << 24) + 8), a, a, None) == moe.ERR_INVALID_ARG
+    assert lib.moe_quantize_e4m3(0, 32, None, None, None, None) == moe.OK
+    full = {f: 1 << 24 for f, _ in moe.moe.MoEFp8Experts._fields_}
+    wq = moe.moe.MoEFp8Experts(**full)
+    call = lambda cfg, w, ws_bytes: lib.moe_layer_forward_fp8(ctypes.byref(cfg), a, a, None, ctypes.byref(w), a, None,
+                                                              None, None, None, None, None, None, None, a, ws_bytes,
+                                                              None)
+    assert call(ok, wq, n.value - 256) == moe.ERR_WORKSPACE
+    for missing in ("up_scale", "down", "sh_up"):
+        w = moe.moe.MoEFp8Experts(**dict(full, **{missing: None}))
+        assert call(ok, w, 1 << 30) == moe.ERR_INVALID_ARG, missing
+    relu = MoEConfig(16, 256, 320, 4, 2, 0, 0, moe.BF16, moe.RELU, 0)
+    w = moe.moe.MoEFp8Experts(**dict(full, up=None, up_scale=None, sh_gate=None, sh_gate_scale=None, sh_up=None,
+                                     sh_up_scale=None, sh_down=None, sh_down_scale=None))
+    assert lib.moe_fp8_workspace_size(ctypes.byref(relu), ctypes.byref(n)) == moe.OK
+    assert call(relu, w, n.value - 256) == moe.ERR_WORKSPACE   # the pointer set itself is complete for ReLU
+    w = moe.moe.MoEFp8Experts(**dict(full, gate=(1 << 24) + 4))
+    assert call(ok, w, 1 << 30) == moe.ERR_INVALID_ARG         # codes must be 16-byte aligned
