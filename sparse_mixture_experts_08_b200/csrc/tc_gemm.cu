@@ -146,6 +146,12 @@ __device__ __forceinline__ uint32_t idesc_e4m3(int M, int N) {
   return (1u << 4) | ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
 }
 
+// Two floats -> bf16 pair (round to nearest even), the first in the low half.
+__device__ __forceinline__ uint32_t pack_bf16x2(float a, float b) {
+  const __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
+  return *reinterpret_cast<const uint32_t*>(&h);
+}
+
 // Barrier of the four epilogue warps only (named barrier 1; 0 is __syncthreads),
 // in its non-aligned form and after reconverging the warp, so lanes that took
 // different branches before it are all counted.
@@ -339,6 +345,11 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
   __shared__ float aux_w[4][EPI == EPI_DOWN ? BN : 1];  // per epilogue warp: row weights of the tile
   __shared__ int aux_d[4][EPI == EPI_DOWN ? BN : 1];    // and destination tokens (fused top-1 combine)
   __shared__ float aux_s[4][F8 && EPI != EPI_DOWN ? BN : 1];  // F8: activation-row scales of the tile
+  // SWIGLU / RELU / DOWN: per epilogue warp, 16 output rows x its 32 features, so the
+  // global writes leave as 16-byte vectors along the feature axis (rows padded to 36
+  // floats: 16-byte aligned, and the column-wise writes hit 32 distinct banks)
+  constexpr bool VEC = EPI == EPI_SWIGLU || EPI == EPI_RELU || EPI == EPI_DOWN;
+  __shared__ __align__(16) float stg[VEC ? 4 : 1][16][36];
   constexpr int RMASK_M = EPI == EPI_ROUTE ? ROUTE_MAX_M : 1;
   __shared__ __align__(16) float rbias[RMASK_M];  // ROUTE: router bias (zeros when absent)
   __shared__ uint32_t rmask[EPI == EPI_ROUTE ? 2 : 1][4][RMASK_M];  // ROUTE: expert -> lanes holding it
@@ -691,7 +702,50 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
         if (MATS == 2) tmem_ld_x16(t_row + BN + c0, r1);
         tmem_ld_wait();
         const int jn = min(16, ti.rows_in_tile - c0);
-        if (fvalid) {
+        if (VEC) {
+#pragma unroll
+          for (int j = 0; j < 16; ++j) {
+            float v0 = has_k ? __uint_as_float(r0[j]) : 0.f;
+            float v1 = (MATS == 2 && has_k) ? __uint_as_float(r1[j]) : 0.f;
+            if (F8) {
+              const float sb = EPI == EPI_DOWN ? 1.f : aux_s[q][c0 + j];
+              v0 = v0 * sa0 * sb;
+              v1 = v1 * sa1 * sb;
+            }
+            stg[q][j][lane] = EPI == EPI_SWIGLU ? v0 / (1.f + __expf(-v0)) * v1
+                              : EPI == EPI_RELU ? fmaxf(v0, 0.f)
+                                                : v0 * aux_w[q][c0 + j];
+          }
+          __syncwarp();
+          const int fbase = ti.mt * TC_BM + q * 32;  // first feature of this warp (R is a multiple of 8)
+          if (EPI == EPI_DOWN && !c.scatter_k1) {  // fp32 partial rows: 8 float4 per row
+            float* o = reinterpret_cast<float*>(c.out) + (long long)ti.ks * c.out_split_stride + fbase;
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+              const int idx = lane + 32 * i, jj = idx >> 3, part = idx & 7;
+              if (jj < jn && fbase + part * 4 < c.R)
+                *reinterpret_cast<float4*>(o + (long long)(ti.out_row + c0 + jj) * c.out_ld + part * 4) =
+                    *reinterpret_cast<const float4*>(&stg[q][jj][part * 4]);
+            }
+          } else {  // bf16 rows (h, or the layer output with the top-1 combine fused): 4 x 8 per row
+            __nv_bfloat16* o = reinterpret_cast<__nv_bfloat16*>(c.out) + fbase;
+#pragma unroll
+            for (int i = 0; i < 2; ++i) {
+              const int idx = lane + 32 * i, jj = idx >> 2, part = idx & 3;
+              const long long orow = EPI == EPI_DOWN ? (long long)aux_d[q][c0 + jj] : (long long)ti.out_row + c0 + jj;
+              if (jj < jn && fbase + part * 8 < c.R && orow >= 0) {
+                const float* v = &stg[q][jj][part * 8];
+                uint4 pk;
+                pk.x = pack_bf16x2(v[0], v[1]);
+                pk.y = pack_bf16x2(v[2], v[3]);
+                pk.z = pack_bf16x2(v[4], v[5]);
+                pk.w = pack_bf16x2(v[6], v[7]);
+                *reinterpret_cast<uint4*>(o + orow * c.out_ld + part * 8) = pk;
+              }
+            }
+          }
+          __syncwarp();
+        } else if (fvalid) {
 #pragma unroll
           for (int j = 0; j < 16; ++j)
             if (j < jn) {
