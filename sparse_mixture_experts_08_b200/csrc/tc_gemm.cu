@@ -285,9 +285,9 @@ __device__ __forceinline__ void decode_tile(const GemmParams& p, const SchedSmem
   ti.kb1 = min(KB, ti.kb0 + c.kb_per_split);
 }
 
-// Per-row epilogue data for a chunk of 16 output rows, loaded once per warp (lane
-// l < 16 handles row c0 + l) and broadcast with shuffles: the gate weight of the
-// row's task and, for the fused top-1 combine, the destination token.
+// Per-row epilogue data of the down projection, fetched for the whole tile into the
+// warp's shared-memory slice: the gate weight of the row's task and, for the fused
+// top-1 combine, the destination token.
 struct RowAux {
   float w;
   int dst;
@@ -308,25 +308,11 @@ __device__ __forceinline__ RowAux load_row_aux(const GemmClass& c, const TileInf
   return a;
 }
 
-template <int EPI>
-__device__ __forceinline__ void store_out(const GemmClass& c, const TileInfo& ti, int feature, int j, float v0,
-                                          float v1, float bias, float wgt, int dst) {
-  const long long row = (long long)ti.out_row + j;
-  if (EPI == EPI_LOGITS) {
-    float* o = reinterpret_cast<float*>(c.out) + (long long)ti.ks * c.out_split_stride;
-    o[row * c.out_ld + feature] = v0 + bias;
-  } else if (EPI == EPI_SWIGLU) {
-    const float h = v0 / (1.f + __expf(-v0)) * v1;
-    reinterpret_cast<__nv_bfloat16*>(c.out)[row * c.out_ld + feature] = __float2bfloat16_rn(h);
-  } else if (EPI == EPI_RELU) {
-    reinterpret_cast<__nv_bfloat16*>(c.out)[row * c.out_ld + feature] = __float2bfloat16_rn(fmaxf(v0, 0.f));
-  } else if (c.scatter_k1) {  // EPI_DOWN, combine fused: one task per token
-    if (dst >= 0)
-      reinterpret_cast<__nv_bfloat16*>(c.out)[(long long)dst * c.out_ld + feature] = __float2bfloat16_rn(v0 * wgt);
-  } else {  // EPI_DOWN
-    float* o = reinterpret_cast<float*>(c.out) + (long long)ti.ks * c.out_split_stride;
-    o[row * c.out_ld + feature] = v0 * wgt;
-  }
+// LOGITS: one fp32 logit (its row pitch, the expert count, need not keep 16-byte
+// alignment, so these rows stay scalar; the expert epilogues store vectors)
+__device__ __forceinline__ void store_logit(const GemmClass& c, const TileInfo& ti, int feature, int j, float v) {
+  float* o = reinterpret_cast<float*>(c.out) + (long long)ti.ks * c.out_split_stride;
+  o[((long long)ti.out_row + j) * c.out_ld + feature] = v;
 }
 
 template <int BN, int MATS, int EPI, bool F8>
@@ -712,7 +698,8 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
               v0 = v0 * sa0 * sb;
               v1 = v1 * sa1 * sb;
             }
-            stg[q][j][lane] = EPI == EPI_SWIGLU ? v0 / (1.f + __expf(-v0)) * v1
+            // SiLU's quotient by the fast division (2 ulp; h is stored in bf16)
+            stg[q][j][lane] = EPI == EPI_SWIGLU ? __fdividef(v0, 1.f + __expf(-v0)) * v1
                               : EPI == EPI_RELU ? fmaxf(v0, 0.f)
                                                 : v0 * aux_w[q][c0 + j];
           }
@@ -745,20 +732,10 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
             }
           }
           __syncwarp();
-        } else if (fvalid) {
+        } else if (fvalid) {  // LOGITS
 #pragma unroll
           for (int j = 0; j < 16; ++j)
-            if (j < jn) {
-              float v0 = has_k ? __uint_as_float(r0[j]) : 0.f;
-              float v1 = (MATS == 2 && has_k) ? __uint_as_float(r1[j]) : 0.f;
-              if (F8) {
-                const float sb = EPI == EPI_DOWN ? 1.f : aux_s[q][c0 + j];
-                v0 = v0 * sa0 * sb;
-                v1 = v1 * sa1 * sb;
-              }
-              store_out<EPI>(c, ti, feature, c0 + j, v0, v1, bias, EPI == EPI_DOWN ? aux_w[q][c0 + j] : 1.f,
-                             EPI == EPI_DOWN ? aux_d[q][c0 + j] : -1);
-            }
+            if (j < jn) store_logit(c, ti, feature, c0 + j, (has_k ? __uint_as_float(r0[j]) : 0.f) + bias);
         }
       }
       tc_fence_before();
