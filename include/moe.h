@@ -101,7 +101,9 @@ typedef struct {
 } moe_lis_t;
 
 /* Atomic-expert layer: N = Nr * Nc experts on a grid, K selected per token
- * (1..64), Nr and Nc in 64..1024 and multiples of 8; dtype must be MOE_BF16. */
+ * (1..4096, at most N: decode budgets up to 64 use a staircase candidate set,
+ * prefill budgets above 64 a radix selection over the whole grid; both exact),
+ * Nr and Nc in 64..1024 and multiples of 8; dtype must be MOE_BF16. */
 typedef struct {
   int32_t T, d, Nr, Nc, K;
   int32_t act;   /* moe_atomic_act_t */

@@ -791,7 +791,7 @@ static moe_status_t check_atomic_cfg(const moe_atomic_config_t* c) {
   if (c->act != MOE_ATOMIC_SILU && c->act != MOE_ATOMIC_SIGMOID) return MOE_ERR_INVALID_ARG;
   if (c->dtype != MOE_BF16) return MOE_ERR_UNSUPPORTED;
   if ((long long)c->K > (long long)c->Nr * c->Nc) return MOE_ERR_INVALID_ARG;
-  if (c->d % 8 || c->Nr % 8 || c->Nc % 8 || c->Nr < 64 || c->Nc < 64 || c->Nr > 1024 || c->Nc > 1024 || c->K > 64)
+  if (c->d % 8 || c->Nr % 8 || c->Nc % 8 || c->Nr < 64 || c->Nc < 64 || c->Nr > 1024 || c->Nc > 1024 || c->K > 4096)
     return MOE_ERR_UNSUPPORTED;
   if (c->T > 65535) return MOE_ERR_UNSUPPORTED;
   return MOE_OK;

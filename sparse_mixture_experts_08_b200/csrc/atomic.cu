@@ -27,6 +27,7 @@ constexpr unsigned FULL = 0xffffffffu;
 constexpr int SEL_THREADS = 1024;
 constexpr int SEL_MAX_SIDE = 1024;
 constexpr int SEL_MAX_K = 64;
+constexpr int WIDE_MAX_K = 4096;  // the wide selection (K > SEL_MAX_K)
 
 __device__ __forceinline__ uint32_t ordered_bits(float v) {
   if (v == 0.f) v = 0.f;  // -0 and +0 are equal scores
@@ -128,6 +129,70 @@ __device__ void block_top64(uint64_t k0, uint64_t k1, bool mine, int lw, int nch
   __syncthreads();
 }
 
+// Row and column log-probabilities of token t into shared lr[Nr], lc[Nc] (and
+// lr_out / lc_out when given): the split-K partials summed in split order (all
+// loads of a thread in flight together), then log-softmax with a block-wide
+// log-sum-exp (a fixed shuffle tree per warp, then warp 0 over the warps: the same
+// result on every run). One thread per row and per column (blockDim = SEL_THREADS
+// >= Nr, Nc); ends with a block barrier.
+__device__ void block_logprobs(int t, int Nr, int Nc, int ksplit, const float* __restrict__ zr, long long zr_split,
+                               const float* __restrict__ zc, long long zc_split, float* lr, float* lc,
+                               float* __restrict__ lr_out, float* __restrict__ lc_out) {
+  __shared__ Lse red_r[32], red_c[32];
+  __shared__ double lse_s[2];
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const bool hr = tid < Nr, hc = tid < Nc;
+  float ar = 0.f, ac = 0.f;
+  for (int s0 = 0; s0 < ksplit; s0 += 8) {
+    float vr[8], vc[8];
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      const int s = s0 + u;
+      vr[u] = (s < ksplit && hr) ? zr[s * zr_split + (long long)t * Nr + tid] : 0.f;
+      vc[u] = (s < ksplit && hc) ? zc[s * zc_split + (long long)t * Nc + tid] : 0.f;
+    }
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      if (s0 + u < ksplit) {
+        ar += vr[u];
+        ac += vc[u];
+      }
+    }
+  }
+  Lse er = {hr ? ar : -FLT_MAX, hr ? 1.0 : 0.0}, ec = {hc ? ac : -FLT_MAX, hc ? 1.0 : 0.0};
+#pragma unroll
+  for (int o = 16; o; o >>= 1) {
+    er = lse_merge(er, lse_shfl_xor(er, o));
+    ec = lse_merge(ec, lse_shfl_xor(ec, o));
+  }
+  if (lane == 0) {
+    red_r[warp] = er;
+    red_c[warp] = ec;
+  }
+  __syncthreads();
+  if (warp == 0) {
+    Lse r = lane < SEL_THREADS / 32 ? red_r[lane] : Lse{-FLT_MAX, 0.0};
+    Lse q = lane < SEL_THREADS / 32 ? red_c[lane] : Lse{-FLT_MAX, 0.0};
+#pragma unroll
+    for (int o = 16; o; o >>= 1) {
+      r = lse_merge(r, lse_shfl_xor(r, o));
+      q = lse_merge(q, lse_shfl_xor(q, o));
+    }
+    if (lane == 0) lse_s[0] = (double)r.m + log(r.s);
+    if (lane == 1) lse_s[1] = (double)q.m + log(q.s);
+  }
+  __syncthreads();
+  if (hr) {
+    lr[tid] = (float)((double)ar - lse_s[0]);
+    if (lr_out) lr_out[(long long)t * Nr + tid] = lr[tid];
+  }
+  if (hc) {
+    lc[tid] = (float)((double)ac - lse_s[1]);
+    if (lc_out) lc_out[(long long)t * Nc + tid] = lc[tid];
+  }
+  __syncthreads();
+}
+
 // One block (1024 threads) per token. zr/zc: split-K partial logits [ksplit][T][Nr|Nc].
 //  1. log-softmax of the row and column logits (fp32 values; log-sum-exp with
 //     fp64 sums);
@@ -152,8 +217,6 @@ __global__ void __launch_bounds__(SEL_THREADS, 1)
   // only after this grid has completed, so clearing the word here is enough
   if (bar_reset && blockIdx.x == 0 && threadIdx.x == 0) *bar_reset = 0u;
   __shared__ uint64_t buf[2][16 * 64];  // merge buffers: rows, columns (candidates reuse rows')
-  __shared__ Lse red_r[32], red_c[32];
-  __shared__ double lse_s[2];
   __shared__ int stair_off[SEL_MAX_K], top_rows[SEL_MAX_K];
   __shared__ uint32_t win_ids[SEL_MAX_K];
   __shared__ int row_list[SEL_MAX_SIDE];
@@ -163,87 +226,34 @@ __global__ void __launch_bounds__(SEL_THREADS, 1)
   pdl_launch_dependents();
   pdl_wait();
 
-  // 1. sum the split-K partials (all loads of a thread in flight together, summed
-  //    in split order); log-softmax of rows and of columns
-  const bool hr = tid < Nr, hc = tid < Nc;
-  {
-    float ar = 0.f, ac = 0.f;
-    for (int s0 = 0; s0 < ksplit; s0 += 8) {
-      float vr[8], vc[8];
+  // 1. log-softmax of rows and columns (from the split-K partials)
+  block_logprobs(t, Nr, Nc, ksplit, zr, zr_split, zc, zc_split, lr, lc, lr_out, lc_out);
+  if (warp == 1) {  // staircase row offsets (K <= 64 rows: two per lane)
+    const int kr = min(K, Nr), kc = min(K, Nc);
+    const int c0 = lane < kr ? min(K / (lane + 1), kc) : 0;
+    const int c1 = lane + 32 < kr ? min(K / (lane + 33), kc) : 0;
+    int s0 = c0;  // rows 0 .. 31, then rows 32 .. 63
 #pragma unroll
-      for (int u = 0; u < 8; ++u) {
-        const int s = s0 + u;
-        vr[u] = (s < ksplit && hr) ? zr[s * zr_split + (long long)t * Nr + tid] : 0.f;
-        vc[u] = (s < ksplit && hc) ? zc[s * zc_split + (long long)t * Nc + tid] : 0.f;
-      }
+    for (int o = 1; o < 32; o <<= 1) {
+      const int u = __shfl_up_sync(FULL, s0, o);
+      if (lane >= o) s0 += u;
+    }
+    const int tot0 = __shfl_sync(FULL, s0, 31);  // rows 0 .. 31
+    int s1 = c1;
 #pragma unroll
-      for (int u = 0; u < 8; ++u) {
-        if (s0 + u < ksplit) {
-          ar += vr[u];
-          ac += vc[u];
-        }
-      }
+    for (int o = 1; o < 32; o <<= 1) {
+      const int u = __shfl_up_sync(FULL, s1, o);
+      if (lane >= o) s1 += u;
     }
-    // block-wide log-sum-exp of rows and of columns: a fixed shuffle tree per
-    // warp, then warp 0 over the warps (the same result on every run)
-    Lse er = {hr ? ar : -FLT_MAX, hr ? 1.0 : 0.0}, ec = {hc ? ac : -FLT_MAX, hc ? 1.0 : 0.0};
-#pragma unroll
-    for (int o = 16; o; o >>= 1) {
-      er = lse_merge(er, lse_shfl_xor(er, o));
-      ec = lse_merge(ec, lse_shfl_xor(ec, o));
-    }
-    if (lane == 0) {
-      red_r[warp] = er;
-      red_c[warp] = ec;
-    }
-    __syncthreads();
-    if (warp == 0) {
-      Lse r = lane < SEL_THREADS / 32 ? red_r[lane] : Lse{-FLT_MAX, 0.0};
-      Lse q = lane < SEL_THREADS / 32 ? red_c[lane] : Lse{-FLT_MAX, 0.0};
-#pragma unroll
-      for (int o = 16; o; o >>= 1) {
-        r = lse_merge(r, lse_shfl_xor(r, o));
-        q = lse_merge(q, lse_shfl_xor(q, o));
-      }
-      if (lane == 0) lse_s[0] = (double)r.m + log(r.s);
-      if (lane == 1) lse_s[1] = (double)q.m + log(q.s);
-    }
-    if (warp == 1) {  // staircase row offsets (K <= 64 rows: two per lane)
-      const int kr = min(K, Nr), kc = min(K, Nc);
-      const int c0 = lane < kr ? min(K / (lane + 1), kc) : 0;
-      const int c1 = lane + 32 < kr ? min(K / (lane + 33), kc) : 0;
-      int s0 = c0;  // rows 0 .. 31, then rows 32 .. 63
-#pragma unroll
-      for (int o = 1; o < 32; o <<= 1) {
-        const int u = __shfl_up_sync(FULL, s0, o);
-        if (lane >= o) s0 += u;
-      }
-      const int tot0 = __shfl_sync(FULL, s0, 31);  // rows 0 .. 31
-      int s1 = c1;
-#pragma unroll
-      for (int o = 1; o < 32; o <<= 1) {
-        const int u = __shfl_up_sync(FULL, s1, o);
-        if (lane >= o) s1 += u;
-      }
-      stair_off[lane] = s0 - c0;
-      stair_off[lane + 32] = tot0 + s1 - c1;
-      if (lane == 31) n_cand = tot0 + s1;
-    }
-    if (tid == 64) {
-      n_rows = 0;
-      found_s = 0;
-    }
-    __syncthreads();
-    if (hr) {
-      lr[tid] = (float)((double)ar - lse_s[0]);
-      if (lr_out) lr_out[(long long)t * Nr + tid] = lr[tid];
-    }
-    if (hc) {
-      lc[tid] = (float)((double)ac - lse_s[1]);
-      if (lc_out) lc_out[(long long)t * Nc + tid] = lc[tid];
-    }
-    __syncthreads();
+    stair_off[lane] = s0 - c0;
+    stair_off[lane + 32] = tot0 + s1 - c1;
+    if (lane == 31) n_cand = tot0 + s1;
   }
+  if (tid == 64) {
+    n_rows = 0;
+    found_s = 0;
+  }
+  __syncthreads();
   // 2. top 64 rows and columns
   {
     const int side = warp >> 4, lw = warp & 15;
@@ -392,11 +402,219 @@ __global__ void __launch_bounds__(SEL_THREADS, 1)
   }
 }
 
+// Exact top-K for K > 64 (prefill budgets, OmniMoE "Top-K budget K = 512-4096"),
+// one block (1024 threads) per token:
+//  1. log-softmax of rows and columns (block_logprobs);
+//  2. tau, the K-th best score, by a radix select over all Nr Nc grid scores
+//     (fl32(lr_i + lc_j), recomputed from shared memory in each pass) on their
+//     order-preserving 32-bit codes: digits of 11, 11 and 10 bits from the top,
+//     each pass a histogram (warp-aggregated shared atomics) of the pairs that
+//     match the digits fixed so far; it also gives n_gt (pairs above tau) and
+//     n_eq (pairs equal to tau);
+//  3. the winners: every pair above tau, and the need = K - n_gt tied pairs of
+//     lowest flat id. When need == n_eq (no real tie at the threshold, the usual
+//     case) every tied pair is taken; otherwise the grid is walked in flat-id
+//     order, 1024 ids per step, a block-wide count ranking the tied ones, until
+//     need are found;
+//  4. a bitonic sort of the K keys (score desc, flat id asc);
+//  5. g = softmax of the K scores (fp32 exponentials, fp64 sum in a fixed tree).
+__global__ void __launch_bounds__(SEL_THREADS, 1)
+    atomic_select_wide_kernel(int T, int Nr, int Nc, int K, int ksplit, const float* __restrict__ zr,
+                              long long zr_split, const float* __restrict__ zc, long long zc_split,
+                              float* __restrict__ lr_out, float* __restrict__ lc_out, int32_t* __restrict__ idx_out,
+                              float* __restrict__ g_out, int* status, unsigned* bar_reset) {
+  __shared__ float lr[SEL_MAX_SIDE], lc[SEL_MAX_SIDE];
+  __shared__ uint64_t sel[WIDE_MAX_K];  // winners' keys; the radix histograms live here before them
+  __shared__ int warp_cnt[32];
+  __shared__ double warp_z[32];
+  __shared__ uint32_t digit_s;
+  __shared__ int above_s, n_sel, found_s, stop_s;
+  if (bar_reset && blockIdx.x == 0 && threadIdx.x == 0) *bar_reset = 0u;  // as atomic_select_kernel
+  const int t = blockIdx.x, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  pdl_launch_dependents();
+  pdl_wait();
+  block_logprobs(t, Nr, Nc, ksplit, zr, zr_split, zc, zc_split, lr, lc, lr_out, lc_out);
+
+  const int N = Nr * Nc;
+  const int di = SEL_THREADS / Nc, dj = SEL_THREADS % Nc;  // (i, j) step of a thread's walk
+  uint32_t* hist = reinterpret_cast<uint32_t*>(sel);       // 2048 bins = 8 KB of the 32 KB
+  // 2. radix select of the K-th largest code
+  uint32_t prefix = 0, pmask = 0;
+  int krem = K, n_gt = 0, n_eq = 0;
+  const int bits[3] = {11, 11, 10};
+  int shift = 32;
+#pragma unroll 1
+  for (int pass = 0; pass < 3; ++pass) {
+    const int nb = 1 << bits[pass];
+    shift -= bits[pass];
+    for (int b = tid; b < nb; b += SEL_THREADS) hist[b] = 0u;
+    __syncthreads();
+    int i = tid / Nc, j = tid % Nc;
+    for (int p = tid; p < N; p += SEL_THREADS) {
+      const uint32_t u = ordered_bits(lr[i] + lc[j]);
+      if ((u & pmask) == prefix) {
+        const uint32_t dg = (u >> shift) & (uint32_t)(nb - 1);
+        const unsigned same = __match_any_sync(__activemask(), dg);
+        if (lane == __ffs(same) - 1) atomicAdd(&hist[dg], (uint32_t)__popc(same));
+      }
+      i += di;
+      j += dj;
+      if (j >= Nc) {
+        j -= Nc;
+        ++i;
+      }
+    }
+    __syncthreads();
+    if (warp == 0) {  // the bin holding the krem-th largest: scan bins from the top
+      const int per = nb / 32;  // bins per lane, lane 0 holding the highest
+      int sum = 0;
+      for (int b = 0; b < per; ++b) sum += (int)hist[nb - 1 - (lane * per + b)];
+      int incl = sum;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int v = __shfl_up_sync(FULL, incl, o);
+        if (lane >= o) incl += v;
+      }
+      const int excl = incl - sum;  // pairs in the bins above this lane's
+      const unsigned hit = __ballot_sync(FULL, excl < krem && incl >= krem);
+      const int src = __ffs(hit) - 1;  // exactly one lane holds the crossing
+      if (lane == src) {
+        int above = excl;
+        for (int b = 0; b < per; ++b) {
+          const int bin = nb - 1 - (lane * per + b);
+          const int c = (int)hist[bin];
+          if (above + c >= krem) {
+            digit_s = (uint32_t)bin;
+            above_s = above;
+            found_s = c;
+            break;
+          }
+          above += c;
+        }
+      }
+    }
+    __syncthreads();
+    prefix |= digit_s << shift;
+    pmask |= (uint32_t)(nb - 1) << shift;
+    krem -= above_s;
+    n_gt += above_s;
+    n_eq = found_s;  // after the last pass: the pairs whose code equals tau's
+    __syncthreads();
+  }
+  const uint32_t tau = prefix;
+  const int need = krem;  // 1 <= need <= n_eq
+  if (need < 1 || need > n_eq || n_gt + need != K) {  // cannot happen: tau is the code of a grid pair
+    if (tid == 0) set_status(status, MOE_ERR_DEVICE_INDEX);
+    return;
+  }
+  // 3. the winners, appended in any order (sorted next)
+  if (tid == 0) {
+    n_sel = 0;
+    found_s = 0;
+    stop_s = 0;
+  }
+  __syncthreads();
+  const bool all_ties = need == n_eq;
+  {
+    int i = tid / Nc, j = tid % Nc;
+    for (int p = tid; p < N; p += SEL_THREADS) {
+      const float sc = lr[i] + lc[j];
+      const uint32_t u = ordered_bits(sc);
+      if (u > tau || (all_ties && u == tau)) {
+        const unsigned grp = __activemask();
+        const int leader = __ffs(grp) - 1;
+        int base = 0;
+        if (lane == leader) base = atomicAdd(&n_sel, __popc(grp));
+        base = __shfl_sync(grp, base, leader);
+        const int pos = base + __popc(grp & ((1u << lane) - 1u));
+        if (pos < K) sel[pos] = make_key(sc, (uint32_t)p);  // (the counts above keep pos < K)
+        else set_status(status, MOE_ERR_DEVICE_INDEX);
+      }
+      i += di;
+      j += dj;
+      if (j >= Nc) {
+        j -= Nc;
+        ++i;
+      }
+    }
+  }
+  __syncthreads();
+  if (!all_ties) {  // the lowest flat ids among the pairs scoring tau, 1024 ids at a time
+    for (int p0 = 0; p0 < N; p0 += SEL_THREADS) {
+      const int p = p0 + tid;
+      const bool eq = p < N && ordered_bits(lr[p / Nc] + lc[p % Nc]) == tau;
+      const unsigned bal = __ballot_sync(FULL, eq);
+      if (lane == 0) warp_cnt[warp] = __popc(bal);
+      __syncthreads();
+      int before = found_s;
+      for (int w = 0; w < warp; ++w) before += warp_cnt[w];
+      const int rank = before + __popc(bal & ((1u << lane) - 1u));
+      if (eq && rank < need) sel[n_gt + rank] = make_key(lr[p / Nc] + lc[p % Nc], (uint32_t)p);
+      __syncthreads();
+      if (tid == 0) {
+        int tot = 0;
+        for (int w = 0; w < SEL_THREADS / 32; ++w) tot += warp_cnt[w];
+        found_s += tot;
+        stop_s = found_s >= need;
+      }
+      __syncthreads();
+      if (stop_s) break;
+    }
+  }
+  // 4. bitonic sort, descending, over the next power of two (padding keys are 0)
+  int n2 = 1;
+  while (n2 < K) n2 <<= 1;
+  for (int q = K + tid; q < n2; q += SEL_THREADS) sel[q] = 0ull;
+  __syncthreads();
+  for (int k = 2; k <= n2; k <<= 1) {
+    for (int jj = k >> 1; jj > 0; jj >>= 1) {
+      for (int q = tid; q < n2; q += SEL_THREADS) {
+        const int r = q ^ jj;
+        if (r > q) {
+          const uint64_t a = sel[q], b = sel[r];
+          const bool desc = (q & k) == 0;
+          if (desc ? a < b : a > b) {
+            sel[q] = b;
+            sel[r] = a;
+          }
+        }
+      }
+      __syncthreads();
+    }
+  }
+  // 5. gate weights
+  const float smax = ordered_to_float((uint32_t)(sel[0] >> 32));
+  double z = 0.0;
+  for (int q = tid; q < K; q += SEL_THREADS) z += (double)expf(ordered_to_float((uint32_t)(sel[q] >> 32)) - smax);
+#pragma unroll
+  for (int o = 16; o; o >>= 1) z += __shfl_xor_sync(FULL, z, o);
+  if (lane == 0) warp_z[warp] = z;
+  __syncthreads();
+  if (warp == 0) {
+    double zz = warp_z[lane];
+#pragma unroll
+    for (int o = 16; o; o >>= 1) zz += __shfl_xor_sync(FULL, zz, o);
+    if (lane == 0) warp_z[0] = zz;
+  }
+  __syncthreads();
+  const double zs = warp_z[0];
+  for (int q = tid; q < K; q += SEL_THREADS) {
+    const uint64_t key = sel[q];
+    idx_out[(long long)t * K + q] = (int32_t)key_id(key);
+    g_out[(long long)t * K + q] = (float)((double)expf(ordered_to_float((uint32_t)(key >> 32)) - smax) / zs);
+  }
+}
+
 cudaError_t launch_atomic_select(int T, int Nr, int Nc, int K, int ksplit, const float* zr, long long zr_split,
                                  const float* zc, long long zc_split, float* lr_out, float* lc_out, int32_t* idx,
                                  float* g, int* status, unsigned* bar_reset, cudaStream_t s) {
-  launch_k(atomic_select_kernel, T, SEL_THREADS, 0, s, T, Nr, Nc, K, ksplit, zr, zr_split, zc, zc_split, lr_out,
-           lc_out, idx, g, status, bar_reset);
+  if (K > WIDE_MAX_K) return cudaErrorInvalidValue;
+  if (K > SEL_MAX_K)
+    launch_k(atomic_select_wide_kernel, T, SEL_THREADS, 0, s, T, Nr, Nc, K, ksplit, zr, zr_split, zc, zc_split,
+             lr_out, lc_out, idx, g, status, bar_reset);
+  else
+    launch_k(atomic_select_kernel, T, SEL_THREADS, 0, s, T, Nr, Nc, K, ksplit, zr, zr_split, zc, zc_split, lr_out,
+             lc_out, idx, g, status, bar_reset);
   count_launch();
   return cudaGetLastError();
 }
@@ -407,7 +625,8 @@ constexpr int ASM_GROUPS = 4, ASM_BATCH = 16;  // phase 2: slot groups per 8 col
 // The atomic-expert FFN (OmniMoE Eq. 4) in one cooperative launch, one block per SM:
 //  phase 1, one warp per task (t, s): coef[t, s] = g[t, s] act(x_t . w_in[idx[t, s]]),
 //    fp32 FMAs over each lane's 16-byte chunks in ascending order then a shuffle
-//    tree; the warp also prefetches the task's w_out row into L2 for phase 2;
+//    tree; when all gathered w_out rows fit comfortably in L2 (decode budgets) the
+//    warp also prefetches the task's w_out row for phase 2;
 //  a grid-wide barrier (bounded: on expiry it records MOE_ERR_TIMEOUT and carries on);
 //  phase 2, four lanes per 8 output columns: lane group j sums slots j, j + 4, ...
 //    in order, and out[t, c..c+7] = ((group 0 + group 1) + group 2) + group 3,
@@ -421,7 +640,8 @@ __global__ void __launch_bounds__(AX_THREADS)
     atomic_experts_kernel(int T, int d, int K, int act, const uint4* __restrict__ x, const uint4* __restrict__ w_in,
                           const uint4* __restrict__ w_out, const int32_t* __restrict__ idx,
                           const float* __restrict__ g, float* __restrict__ coef, uint4* __restrict__ out,
-                          long long n_experts, unsigned* bar, unsigned long long limit_ns, int* status) {
+                          long long n_experts, int prefetch_out, unsigned* bar, unsigned long long limit_ns,
+                          int* status) {
   pdl_launch_dependents();
   pdl_wait();
   const int lane = threadIdx.x & 31;
@@ -440,8 +660,10 @@ __global__ void __launch_bounds__(AX_THREADS)
       }
       continue;
     }
-    const char* po = reinterpret_cast<const char*>(w_out + e * chunks);
-    for (int b = lane * 128; b < d * 2; b += 32 * 128) prefetch_l2(po + b);
+    if (prefetch_out) {
+      const char* po = reinterpret_cast<const char*>(w_out + e * chunks);
+      for (int b = lane * 128; b < d * 2; b += 32 * 128) prefetch_l2(po + b);
+    }
     const uint4* wr = w_in + e * chunks;
     const uint4* xr = x + t * chunks;
     float sacc = 0.f;
@@ -566,8 +788,11 @@ cudaError_t launch_atomic_experts(int T, int d, int K, int act, const void* x, c
   attr[1].val.cooperative = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 2;
+  // rows gathered for phase 2 prefetched in phase 1 only while they stay well inside L2
+  const int prefetch_out = (double)T * K * d * 2 <= 32.0 * (1 << 20) ? 1 : 0;
   cudaError_t e = cudaLaunchKernelEx(&cfg, atomic_experts_kernel, T, d, K, act, (const uint4*)x, (const uint4*)w_in,
-                                     (const uint4*)w_out, idx, g, coef, (uint4*)out, n_experts, bar, limit_ns, status);
+                                     (const uint4*)w_out, idx, g, coef, (uint4*)out, n_experts, prefetch_out, bar,
+                                     limit_ns, status);
   count_launch();
   if (e != cudaSuccess) return e;
   return cudaGetLastError();

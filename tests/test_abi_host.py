@@ -109,7 +109,10 @@ def test_calls_reject_bad_pointers_and_small_workspace_before_launch():
 
 
 @pytest.mark.parametrize("kw,code", [
-    (dict(K=65), moe.ERR_UNSUPPORTED),
+    (dict(K=4097), moe.ERR_UNSUPPORTED),
+    (dict(Nr=64, Nc=64, K=4097), moe.ERR_INVALID_ARG),   # more than the grid holds
+    (dict(K=65), moe.OK),
+    (dict(K=4096), moe.OK),
     (dict(Nr=32), moe.ERR_UNSUPPORTED),
     (dict(Nc=2048), moe.ERR_UNSUPPORTED),
     (dict(dtype=moe.F32), moe.ERR_UNSUPPORTED),

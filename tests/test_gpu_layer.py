@@ -140,10 +140,12 @@ def _atomic(cfg, inp):
     return host(lr), host(lc), host(idx), host(g), out, out2
 
 
-@pytest.mark.parametrize("full", [False, True])
-def test_atomic_layer(full):
-    if full:
+@pytest.mark.parametrize("case", ["small", "full", "wide_k"])
+def test_atomic_layer(case):
+    if case == "full":
         cfg = W.CONFIGS["atomic"]
+    elif case == "wide_k":  # a prefill budget: K = 512 (the radix selection), every slot through the experts
+        cfg = W.AtomicWorkload("atomic_wide", 95, T=6, d=256, Nr=64, Nc=128, K=512, act=W.ACT_SILU)
     else:
         cfg = W.AtomicWorkload("atomic_small", 92, T=5, d=256, Nr=64, Nc=128, K=16, act=W.ACT_SIGMOID)
     inp = W.make_atomic_inputs(cfg)
@@ -207,6 +209,14 @@ def _level_weights(rows, d, levels, seed):
     (1024, 1024, 64, "equal"),    # every pair ties: the K lowest flat ids
     (128, 128, 64, "levels"),     # few distinct scores: long tied runs per row
     (1024, 512, 33, "levels"),
+    # K > 64: the radix selection over the whole grid
+    (128, 128, 65, "random"),
+    (64, 64, 4096, "random"),      # K = N: the whole grid in order
+    (512, 512, 512, "random"),
+    (1024, 1024, 4096, "random"),  # largest grid, largest K
+    (512, 512, 1000, "levels"),    # ties at the threshold: lowest flat ids among them
+    (1024, 64, 2000, "levels"),
+    (256, 256, 4096, "equal"),     # every pair ties
 ])
 def test_atomic_select_grid_shapes(Nr, Nc, K, kind):
     cfg = W.AtomicWorkload("atomic_grid", 94, T=3, d=64, Nr=Nr, Nc=Nc, K=K, act=W.ACT_SILU)
@@ -224,3 +234,27 @@ def test_atomic_select_grid_shapes(Nr, Nc, K, kind):
     np.testing.assert_allclose(g, og, rtol=GATE_RTOL * 4, atol=1e-9)
     if kind == "equal":
         np.testing.assert_array_equal(idx, np.tile(np.arange(K, dtype=np.int32), (cfg.T, 1)))
+
+
+def test_atomic_prefill_full_size():
+    """4096 tokens, K = 512 of a 512 x 512 grid: routing of every token bit-exact on the
+    GPU's log-probabilities; the output of a token sample within the bf16 tolerance."""
+    cfg = W.CONFIGS["atomic_prefill"]
+    inp = W.make_atomic_inputs(cfg)
+    lr, lc, idx, g, out, out2 = _atomic(cfg, inp)
+    olr, olc = O.atomic_logprobs(inp["x"][:8], inp["w_row"], inp["w_col"])
+    np.testing.assert_allclose(lr[:8], olr, rtol=0, atol=2e-4)
+    np.testing.assert_allclose(lc[:8], olc, rtol=0, atol=2e-4)
+    toks = np.r_[0:6, 2047, cfg.T - 6:cfg.T]
+    oidx, og = O.atomic_select(lr[toks], lc[toks], cfg.K)
+    np.testing.assert_array_equal(idx[toks], oidx)
+    np.testing.assert_allclose(g[toks], og, rtol=GATE_RTOL * 4, atol=1e-9)
+    assert np.all((idx >= 0) & (idx < cfg.N))
+    assert np.all(np.sort(idx, axis=1)[:, 1:] != np.sort(idx, axis=1)[:, :-1])  # K distinct experts per token
+    idx_s = np.zeros((cfg.T, cfg.K), np.int32)  # the oracle's routing at the sampled tokens
+    g_s = np.zeros((cfg.T, cfg.K), np.float64)
+    idx_s[toks], g_s[toks] = oidx, og
+    exp = O.atomic_output(inp["x"], inp["w_in"], inp["w_out"], idx_s, g_s, cfg.act, tokens=toks)
+    assert token_rel_err(out_f64(out)[toks], exp) <= TOL[W.BF16]
+    torch.cuda.synchronize()
+    assert torch.equal(out, out2)

@@ -113,6 +113,9 @@ CONFIGS: Dict[str, object] = {
                           note="decode regime: 16 tokens, d_model 4096, d_ff 14336, 8 experts, top-2"),
     "atomic": AtomicWorkload("atomic", 6, T=16, d=4096, Nr=512, Nc=512, K=64, act=ACT_SILU,
                              note="atomic experts: 16 tokens, d_model 4096, 512x512 Cartesian router, top-64 of 262144"),
+    "atomic_prefill": AtomicWorkload("atomic_prefill", 7, T=4096, d=4096, Nr=512, Nc=512, K=512, act=ACT_SILU,
+                                     note="atomic experts at prefill scale: 4096 tokens, d_model 4096, 512x512 "
+                                          "Cartesian router, top-512 of 262144"),
 }
 
 _ALPHA_FILE = os.path.join(_HERE, "zipf_alpha.json")
