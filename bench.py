@@ -353,23 +353,26 @@ def stage_costs(cfg, active: int, ksplit: int, weight_bytes=None):
     return c, layer_flops, layer_bytes
 
 
-def source_hash() -> str:
+def source_hash(files=None) -> str:
+    """Hash of the library sources: the named files of csrc/ (all of them when None)."""
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "sparse_mixture_experts_08_b200", "csrc")
-    for name in sorted(os.listdir(csrc)):
+    for name in sorted(files if files else os.listdir(csrc)):
         with open(os.path.join(csrc, name), "rb") as fh:
             h.update(name.encode() + fh.read())
     return h.hexdigest()[:16]
 
 
 def traffic_for(workload: str, stage: str):
-    """dram bytes per launch from a committed ncu capture, if it matches the current source."""
+    """dram bytes per launch from a committed ncu capture, if the sources that define the
+    captured kernel (its entry's source_files) are unchanged since the capture."""
     path = os.path.join(ROOT, "profiles", "traffic.json")
     try:
         with open(path) as fh:
             t = json.load(fh)
         e = t[workload][stage]
-        return e["dram_bytes_per_launch"] if e.get("source_hash") == source_hash() else None
+        ok = e.get("source_hash") == source_hash(e.get("source_files"))
+        return e["dram_bytes_per_launch"] if ok else None
     except Exception:
         return None
 

@@ -405,42 +405,70 @@ __global__ void __launch_bounds__(SEL_THREADS, 1)
 // Exact top-K for K > 64 (prefill budgets, OmniMoE "Top-K budget K = 512-4096"),
 // one block (1024 threads) per token:
 //  1. log-softmax of rows and columns (block_logprobs);
-//  2. tau, the K-th best score, by a radix select over all Nr Nc grid scores
-//     (fl32(lr_i + lc_j), recomputed from shared memory in each pass) on their
-//     order-preserving 32-bit codes: digits of 11, 11 and 10 bits from the top,
-//     each pass a histogram (warp-aggregated shared atomics) of the pairs that
-//     match the digits fixed so far; it also gives n_gt (pairs above tau) and
-//     n_eq (pairs equal to tau);
-//  3. the winners: every pair above tau, and the need = K - n_gt tied pairs of
-//     lowest flat id. When need == n_eq (no real tie at the threshold, the usual
-//     case) every tied pair is taken; otherwise the grid is walked in flat-id
-//     order, 1024 ids per step, a block-wide count ranking the tied ones, until
-//     need are found;
-//  4. a bitonic sort of the K keys (score desc, flat id asc);
-//  5. g = softmax of the K scores (fp32 exponentials, fp64 sum in a fixed tree).
+//  2. rows and columns sorted by (value desc, index asc) (bitonic, in shared memory);
+//  3. tau, the K-th best score, by a radix select over the staircase pairs
+//     {(a, b) : (a+1)(b+1) <= K} of sorted row a and sorted column b (about K ln K
+//     of them; the file header shows tau and every pair above it lie there), on
+//     the scores' order-preserving 32-bit codes: digits of 11, 11 and 10 bits from
+//     the top, each pass a histogram (warp-aggregated shared atomics) of the pairs
+//     that match the digits fixed so far; it also gives n_gt, the pairs above tau;
+//  4. the winners. When the first pair past the staircase in every staircase row,
+//     and the best pair of the first row left out, all score below tau (the usual
+//     case), no pair outside the staircase reaches tau: the staircase pairs scoring
+//     >= tau (above tau, plus every tied pair) are sorted and the first K kept.
+//     Otherwise one pass over the whole grid takes the pairs above tau and those
+//     scoring exactly tau; when these number more than need = K - n_gt, the grid is
+//     walked in flat-id order, 1024 ids per step, a block-wide count ranking the
+//     tied pairs, until the need lowest ids are found;
+//  5. a bitonic sort of the winners' keys (score desc, flat id asc);
+//  6. g = softmax of the K scores (fp32 exponentials, fp64 sum in a fixed tree).
 __global__ void __launch_bounds__(SEL_THREADS, 1)
     atomic_select_wide_kernel(int T, int Nr, int Nc, int K, int ksplit, const float* __restrict__ zr,
                               long long zr_split, const float* __restrict__ zc, long long zc_split,
                               float* __restrict__ lr_out, float* __restrict__ lc_out, int32_t* __restrict__ idx_out,
                               float* __restrict__ g_out, int* status, unsigned* bar_reset) {
   __shared__ float lr[SEL_MAX_SIDE], lc[SEL_MAX_SIDE];
-  __shared__ uint64_t sel[WIDE_MAX_K];  // winners' keys; the radix histograms live here before them
+  __shared__ uint16_t row_ord[SEL_MAX_SIDE], col_ord[SEL_MAX_SIDE];
+  // winners' keys; before them the row / column sort and the radix histograms
+  __shared__ uint64_t sel[WIDE_MAX_K];
   __shared__ int warp_cnt[32];
   __shared__ double warp_z[32];
   __shared__ uint32_t digit_s;
-  __shared__ int above_s, n_sel, found_s, stop_s;
+  __shared__ int above_s, bin_s, n_sel, n_tie, found_s, stop_s, outside_s;
   if (bar_reset && blockIdx.x == 0 && threadIdx.x == 0) *bar_reset = 0u;  // as atomic_select_kernel
   const int t = blockIdx.x, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   pdl_launch_dependents();
   pdl_wait();
   block_logprobs(t, Nr, Nc, ksplit, zr, zr_split, zc, zc_split, lr, lc, lr_out, lc_out);
 
-  const int N = Nr * Nc;
-  const int di = SEL_THREADS / Nc, dj = SEL_THREADS % Nc;  // (i, j) step of a thread's walk
-  uint32_t* hist = reinterpret_cast<uint32_t*>(sel);       // 2048 bins = 8 KB of the 32 KB
-  // 2. radix select of the K-th largest code
+  // 2. sorted rows (sel[0, 1024)) and columns (sel[1024, 2048)); padding keys 0 sink
+  sel[tid] = tid < Nr ? make_key(lr[tid], (uint32_t)tid) : 0ull;
+  sel[SEL_MAX_SIDE + tid] = tid < Nc ? make_key(lc[tid], (uint32_t)tid) : 0ull;
+  __syncthreads();
+  for (int k = 2; k <= SEL_MAX_SIDE; k <<= 1) {
+    for (int jj = k >> 1; jj > 0; jj >>= 1) {
+      for (int q = tid; q < 2 * SEL_MAX_SIDE; q += SEL_THREADS) {  // both lists in the same steps
+        const int e = q & (SEL_MAX_SIDE - 1), base = q - e, r = e ^ jj;
+        if (r > e) {
+          const uint64_t va = sel[base + e], vb = sel[base + r];
+          if ((e & k) == 0 ? va < vb : va > vb) {
+            sel[base + e] = vb;
+            sel[base + r] = va;
+          }
+        }
+      }
+      __syncthreads();
+    }
+  }
+  if (tid < Nr) row_ord[tid] = (uint16_t)key_id(sel[tid]);
+  if (tid < Nc) col_ord[tid] = (uint16_t)key_id(sel[SEL_MAX_SIDE + tid]);
+  __syncthreads();
+
+  // 3. radix select of the K-th largest code over the staircase
+  uint32_t* hist = reinterpret_cast<uint32_t*>(sel);  // 2048 bins = 8 KB of the 32 KB
+  const int kr = min(Nr, K);
   uint32_t prefix = 0, pmask = 0;
-  int krem = K, n_gt = 0, n_eq = 0;
+  int krem = K, n_gt = 0;
   const int bits[3] = {11, 11, 10};
   int shift = 32;
 #pragma unroll 1
@@ -449,19 +477,16 @@ __global__ void __launch_bounds__(SEL_THREADS, 1)
     shift -= bits[pass];
     for (int b = tid; b < nb; b += SEL_THREADS) hist[b] = 0u;
     __syncthreads();
-    int i = tid / Nc, j = tid % Nc;
-    for (int p = tid; p < N; p += SEL_THREADS) {
-      const uint32_t u = ordered_bits(lr[i] + lc[j]);
-      if ((u & pmask) == prefix) {
-        const uint32_t dg = (u >> shift) & (uint32_t)(nb - 1);
-        const unsigned same = __match_any_sync(__activemask(), dg);
-        if (lane == __ffs(same) - 1) atomicAdd(&hist[dg], (uint32_t)__popc(same));
-      }
-      i += di;
-      j += dj;
-      if (j >= Nc) {
-        j -= Nc;
-        ++i;
+    for (int a = warp; a < kr; a += SEL_THREADS / 32) {  // one sorted row per warp
+      const int cnt = min(Nc, K / (a + 1));
+      const float la = lr[row_ord[a]];
+      for (int b = lane; b < cnt; b += 32) {
+        const uint32_t u = ordered_bits(la + lc[col_ord[b]]);
+        if ((u & pmask) == prefix) {
+          const uint32_t dg = (u >> shift) & (uint32_t)(nb - 1);
+          const unsigned same = __match_any_sync(__activemask(), dg);
+          if (lane == __ffs(same) - 1) atomicAdd(&hist[dg], (uint32_t)__popc(same));
+        }
       }
     }
     __syncthreads();
@@ -477,8 +502,8 @@ __global__ void __launch_bounds__(SEL_THREADS, 1)
       }
       const int excl = incl - sum;  // pairs in the bins above this lane's
       const unsigned hit = __ballot_sync(FULL, excl < krem && incl >= krem);
-      const int src = __ffs(hit) - 1;  // exactly one lane holds the crossing
-      if (lane == src) {
+      if (lane == 0 && !hit) digit_s = 0xFFFFFFFFu;  // (cannot happen: the staircase holds K pairs)
+      if (hit && lane == __ffs(hit) - 1) {
         int above = excl;
         for (int b = 0; b < per; ++b) {
           const int bin = nb - 1 - (lane * per + b);
@@ -486,7 +511,7 @@ __global__ void __launch_bounds__(SEL_THREADS, 1)
           if (above + c >= krem) {
             digit_s = (uint32_t)bin;
             above_s = above;
-            found_s = c;
+            bin_s = c;
             break;
           }
           above += c;
@@ -494,41 +519,81 @@ __global__ void __launch_bounds__(SEL_THREADS, 1)
       }
     }
     __syncthreads();
+    if (digit_s == 0xFFFFFFFFu) {
+      if (tid == 0) set_status(status, MOE_ERR_DEVICE_INDEX);
+      return;
+    }
     prefix |= digit_s << shift;
     pmask |= (uint32_t)(nb - 1) << shift;
     krem -= above_s;
     n_gt += above_s;
-    n_eq = found_s;  // after the last pass: the pairs whose code equals tau's
     __syncthreads();
   }
   const uint32_t tau = prefix;
-  const int need = krem;  // 1 <= need <= n_eq
-  if (need < 1 || need > n_eq || n_gt + need != K) {  // cannot happen: tau is the code of a grid pair
-    if (tid == 0) set_status(status, MOE_ERR_DEVICE_INDEX);
-    return;
-  }
-  // 3. the winners, appended in any order (sorted next)
+  const int need = krem;         // >= 1: tau is the code of the K-th pair
+  const int n_stair = n_gt + bin_s;  // staircase pairs scoring >= tau
+  // 4. the winners
   if (tid == 0) {
     n_sel = 0;
+    n_tie = 0;
     found_s = 0;
     stop_s = 0;
+    outside_s = 0;
   }
   __syncthreads();
-  const bool all_ties = need == n_eq;
-  {
+  // can a pair outside the staircase reach tau? (columns and rows are sorted, so
+  // each row's first pair past the staircase, and the first row left out, bound them)
+  for (int a = tid; a <= kr; a += SEL_THREADS) {
+    if (a < kr) {
+      const int cnt = min(Nc, K / (a + 1));
+      if (cnt < Nc && ordered_bits(lr[row_ord[a]] + lc[col_ord[cnt]]) >= tau) outside_s = 1;
+    } else if (kr < Nr && ordered_bits(lr[row_ord[kr]] + lc[col_ord[0]]) >= tau) {
+      outside_s = 1;
+    }
+  }
+  __syncthreads();
+  int n_win = K;
+  if (!outside_s && n_stair <= WIDE_MAX_K) {
+    // every pair >= tau is a staircase pair: all of them, sorted below, the first K kept
+    for (int a = warp; a < kr; a += SEL_THREADS / 32) {
+      const int cnt = min(Nc, K / (a + 1));
+      const int ri = row_ord[a];
+      const float la = lr[ri];
+      for (int b = lane; b < cnt; b += 32) {
+        const int cj = col_ord[b];
+        const float sc = la + lc[cj];
+        if (ordered_bits(sc) >= tau) {
+          const unsigned grp = __activemask();
+          const int leader = __ffs(grp) - 1;
+          int base = 0;
+          if (lane == leader) base = atomicAdd(&n_sel, __popc(grp));
+          base = __shfl_sync(grp, base, leader);
+          const int pos = base + __popc(grp & ((1u << lane) - 1u));
+          if (pos < n_stair) sel[pos] = make_key(sc, (uint32_t)(ri * Nc + cj));
+        }
+      }
+    }
+    __syncthreads();
+    if (n_sel != n_stair) {  // cannot happen: the same codes were counted in the radix passes
+      if (tid == 0) set_status(status, MOE_ERR_DEVICE_INDEX);
+      return;
+    }
+    n_win = n_stair;
+  } else {
+    const int N = Nr * Nc;
+    const int di = SEL_THREADS / Nc, dj = SEL_THREADS % Nc;  // (i, j) step of a thread's walk
     int i = tid / Nc, j = tid % Nc;
     for (int p = tid; p < N; p += SEL_THREADS) {
       const float sc = lr[i] + lc[j];
       const uint32_t u = ordered_bits(sc);
-      if (u > tau || (all_ties && u == tau)) {
-        const unsigned grp = __activemask();
+      if (u >= tau) {
+        const unsigned grp = __match_any_sync(__activemask(), u > tau ? 1u : 0u);
         const int leader = __ffs(grp) - 1;
         int base = 0;
-        if (lane == leader) base = atomicAdd(&n_sel, __popc(grp));
+        if (lane == leader) base = atomicAdd(u > tau ? &n_sel : &n_tie, __popc(grp));
         base = __shfl_sync(grp, base, leader);
-        const int pos = base + __popc(grp & ((1u << lane) - 1u));
-        if (pos < K) sel[pos] = make_key(sc, (uint32_t)p);  // (the counts above keep pos < K)
-        else set_status(status, MOE_ERR_DEVICE_INDEX);
+        const int pos = (u > tau ? 0 : n_gt) + base + __popc(grp & ((1u << lane) - 1u));
+        if (pos < (u > tau ? n_gt : K)) sel[pos] = make_key(sc, (uint32_t)p);
       }
       i += di;
       j += dj;
@@ -537,52 +602,56 @@ __global__ void __launch_bounds__(SEL_THREADS, 1)
         ++i;
       }
     }
-  }
-  __syncthreads();
-  if (!all_ties) {  // the lowest flat ids among the pairs scoring tau, 1024 ids at a time
-    for (int p0 = 0; p0 < N; p0 += SEL_THREADS) {
-      const int p = p0 + tid;
-      const bool eq = p < N && ordered_bits(lr[p / Nc] + lc[p % Nc]) == tau;
-      const unsigned bal = __ballot_sync(FULL, eq);
-      if (lane == 0) warp_cnt[warp] = __popc(bal);
-      __syncthreads();
-      int before = found_s;
-      for (int w = 0; w < warp; ++w) before += warp_cnt[w];
-      const int rank = before + __popc(bal & ((1u << lane) - 1u));
-      if (eq && rank < need) sel[n_gt + rank] = make_key(lr[p / Nc] + lc[p % Nc], (uint32_t)p);
-      __syncthreads();
-      if (tid == 0) {
-        int tot = 0;
-        for (int w = 0; w < SEL_THREADS / 32; ++w) tot += warp_cnt[w];
-        found_s += tot;
-        stop_s = found_s >= need;
+    __syncthreads();
+    if (n_sel != n_gt || n_tie < need) {  // cannot happen: the counts come from the same codes
+      if (tid == 0) set_status(status, MOE_ERR_DEVICE_INDEX);
+      return;
+    }
+    if (n_tie > need) {  // a real tie at the threshold: the lowest flat ids, 1024 ids at a time
+      const int N = Nr * Nc;
+      for (int p0 = 0; p0 < N; p0 += SEL_THREADS) {
+        const int p = p0 + tid;
+        const bool eq = p < N && ordered_bits(lr[p / Nc] + lc[p % Nc]) == tau;
+        const unsigned bal = __ballot_sync(FULL, eq);
+        if (lane == 0) warp_cnt[warp] = __popc(bal);
+        __syncthreads();
+        int before = found_s;
+        for (int w = 0; w < warp; ++w) before += warp_cnt[w];
+        const int rank = before + __popc(bal & ((1u << lane) - 1u));
+        if (eq && rank < need) sel[n_gt + rank] = make_key(lr[p / Nc] + lc[p % Nc], (uint32_t)p);
+        __syncthreads();
+        if (tid == 0) {
+          int tot = 0;
+          for (int w = 0; w < SEL_THREADS / 32; ++w) tot += warp_cnt[w];
+          found_s += tot;
+          stop_s = found_s >= need;
+        }
+        __syncthreads();
+        if (stop_s) break;
       }
-      __syncthreads();
-      if (stop_s) break;
     }
   }
-  // 4. bitonic sort, descending, over the next power of two (padding keys are 0)
+  // 5. bitonic sort, descending, over the next power of two (padding keys are 0)
   int n2 = 1;
-  while (n2 < K) n2 <<= 1;
-  for (int q = K + tid; q < n2; q += SEL_THREADS) sel[q] = 0ull;
+  while (n2 < n_win) n2 <<= 1;
+  for (int q = n_win + tid; q < n2; q += SEL_THREADS) sel[q] = 0ull;
   __syncthreads();
   for (int k = 2; k <= n2; k <<= 1) {
     for (int jj = k >> 1; jj > 0; jj >>= 1) {
       for (int q = tid; q < n2; q += SEL_THREADS) {
         const int r = q ^ jj;
         if (r > q) {
-          const uint64_t a = sel[q], b = sel[r];
-          const bool desc = (q & k) == 0;
-          if (desc ? a < b : a > b) {
-            sel[q] = b;
-            sel[r] = a;
+          const uint64_t va = sel[q], vb = sel[r];
+          if ((q & k) == 0 ? va < vb : va > vb) {
+            sel[q] = vb;
+            sel[r] = va;
           }
         }
       }
       __syncthreads();
     }
   }
-  // 5. gate weights
+  // 6. gate weights
   const float smax = ordered_to_float((uint32_t)(sel[0] >> 32));
   double z = 0.0;
   for (int q = tid; q < K; q += SEL_THREADS) z += (double)expf(ordered_to_float((uint32_t)(sel[q] >> 32)) - smax);
@@ -636,6 +705,45 @@ __device__ __forceinline__ void prefetch_l2(const void* p) {
   asm volatile("prefetch.global.L2 [%0];" ::"l"(p));
 }
 
+// x . w over `chunks` 16-byte chunks of bf16 by one warp: fp32 FMAs over each
+// lane's chunks in ascending order (8 chunks of each operand in flight), then a
+// shuffle tree; every lane returns the sum.
+__device__ __forceinline__ float warp_dot_bf16(const uint4* __restrict__ xr, const uint4* __restrict__ wr, int chunks,
+                                               int lane) {
+  float sacc = 0.f;
+  for (int c0 = lane; c0 < chunks; c0 += 32 * 8) {
+    uint4 av[8], bv[8];
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      const int c = c0 + 32 * u;
+      if (c < chunks) {
+        av[u] = xr[c];
+        bv[u] = wr[c];
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      if (c0 + 32 * u >= chunks) break;
+      const __nv_bfloat162* pa = reinterpret_cast<const __nv_bfloat162*>(&av[u]);
+      const __nv_bfloat162* pb = reinterpret_cast<const __nv_bfloat162*>(&bv[u]);
+#pragma unroll
+      for (int h = 0; h < 4; ++h) {
+        const float2 fa = __bfloat1622float2(pa[h]), fb = __bfloat1622float2(pb[h]);
+        sacc = fmaf(fa.x, fb.x, sacc);
+        sacc = fmaf(fa.y, fb.y, sacc);
+      }
+    }
+  }
+#pragma unroll
+  for (int o = 16; o; o >>= 1) sacc += __shfl_xor_sync(0xffffffffu, sacc, o);
+  return sacc;
+}
+
+__device__ __forceinline__ float atomic_act(float z, int act) {
+  const float sg = 1.f / (1.f + expf(-z));
+  return act == MOE_ATOMIC_SILU ? z * sg : sg;
+}
+
 __global__ void __launch_bounds__(AX_THREADS)
     atomic_experts_kernel(int T, int d, int K, int act, const uint4* __restrict__ x, const uint4* __restrict__ w_in,
                           const uint4* __restrict__ w_out, const int32_t* __restrict__ idx,
@@ -664,38 +772,8 @@ __global__ void __launch_bounds__(AX_THREADS)
       const char* po = reinterpret_cast<const char*>(w_out + e * chunks);
       for (int b = lane * 128; b < d * 2; b += 32 * 128) prefetch_l2(po + b);
     }
-    const uint4* wr = w_in + e * chunks;
-    const uint4* xr = x + t * chunks;
-    float sacc = 0.f;
-    for (int c0 = lane; c0 < chunks; c0 += 32 * 8) {
-      uint4 av[8], bv[8];
-#pragma unroll
-      for (int u = 0; u < 8; ++u) {
-        const int c = c0 + 32 * u;
-        if (c < chunks) {
-          av[u] = xr[c];
-          bv[u] = wr[c];
-        }
-      }
-#pragma unroll
-      for (int u = 0; u < 8; ++u) {
-        if (c0 + 32 * u >= chunks) break;
-        const __nv_bfloat162* pa = reinterpret_cast<const __nv_bfloat162*>(&av[u]);
-        const __nv_bfloat162* pb = reinterpret_cast<const __nv_bfloat162*>(&bv[u]);
-#pragma unroll
-        for (int h = 0; h < 4; ++h) {
-          const float2 fa = __bfloat1622float2(pa[h]), fb = __bfloat1622float2(pb[h]);
-          sacc = fmaf(fa.x, fb.x, sacc);
-          sacc = fmaf(fa.y, fb.y, sacc);
-        }
-      }
-    }
-#pragma unroll
-    for (int o = 16; o; o >>= 1) sacc += __shfl_xor_sync(0xffffffffu, sacc, o);
-    if (lane == 0) {
-      const float sg = 1.f / (1.f + expf(-sacc));
-      coef[task] = g[task] * (act == MOE_ATOMIC_SILU ? sacc * sg : sg);
-    }
+    const float z = warp_dot_bf16(x + t * chunks, w_in + e * chunks, chunks, lane);
+    if (lane == 0) coef[task] = g[task] * atomic_act(z, act);
   }
   // ---- grid-wide barrier (every block is resident: cooperative launch, one per SM)
   __syncthreads();
@@ -769,10 +847,115 @@ __global__ void __launch_bounds__(AX_THREADS)
   }
 }
 
+// Prefill budgets (many tasks): the two phases as separate, fully occupied kernels.
+// Coefficients: one warp per task, as phase 1 above.
+constexpr int AW_THREADS = 256;
+constexpr long long AW_MIN_TASKS = 16384;  // below this the single cooperative launch wins
+
+__global__ void __launch_bounds__(AW_THREADS)
+    atomic_coef_kernel(int T, int d, int K, int act, const uint4* __restrict__ x, const uint4* __restrict__ w_in,
+                       const int32_t* __restrict__ idx, const float* __restrict__ g, float* __restrict__ coef,
+                       long long n_experts, int* status) {
+  pdl_launch_dependents();
+  pdl_wait();
+  const int lane = threadIdx.x & 31;
+  const long long gwarp = ((long long)blockIdx.x * AW_THREADS + threadIdx.x) >> 5;
+  const long long nwarps = (long long)gridDim.x * (AW_THREADS / 32);
+  const int chunks = d / 8;
+  const long long tasks = (long long)T * K;
+  for (long long task = gwarp; task < tasks; task += nwarps) {
+    const long long e = idx[task];
+    if (e < 0 || e >= n_experts) {
+      if (lane == 0) {
+        set_status(status, MOE_ERR_DEVICE_INDEX);
+        coef[task] = 0.f;
+      }
+      continue;
+    }
+    const float z = warp_dot_bf16(x + (task / K) * chunks, w_in + e * chunks, chunks, lane);
+    if (lane == 0) coef[task] = g[task] * atomic_act(z, act);
+  }
+}
+
+// Assembly: out[t, cols] = sum over s (ascending) of coef[t, s] w_out[idx[t, s], cols].
+// A half-warp owns one token and 128 columns (8 per lane, one 16-byte load per
+// slot); units run column block by column block over all tokens, so the slice of
+// W_out being gathered (N rows x 256 B) stays in L2 while every token reads it.
+__global__ void __launch_bounds__(AW_THREADS)
+    atomic_assemble_kernel(int T, int d, int K, const uint4* __restrict__ w_out, const int32_t* __restrict__ idx,
+                           const float* __restrict__ coef, uint4* __restrict__ out, long long n_experts) {
+  pdl_launch_dependents();
+  pdl_wait();
+  const int lane = threadIdx.x & 31, hl = lane & 15;
+  const long long gwarp = ((long long)blockIdx.x * AW_THREADS + threadIdx.x) >> 5;
+  const long long nwarps = (long long)gridDim.x * (AW_THREADS / 32);
+  const int chunks = d / 8;
+  const int blocks = (chunks + 15) / 16;
+  const long long pairs = ((long long)T + 1) / 2;
+  const long long units = (long long)blocks * pairs;
+  for (long long u = gwarp; u < units; u += nwarps) {
+    const int cb = (int)(u / pairs);
+    const long long t = (u - (long long)cb * pairs) * 2 + (lane >> 4);
+    const int c = cb * 16 + hl;
+    if (t >= T || c >= chunks) continue;
+    const int32_t* ir = idx + t * K;
+    const float* cr = coef + t * K;
+    float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+    for (int s0 = 0; s0 < K; s0 += 8) {
+      uint4 v[8];
+      float cf[8];
+#pragma unroll
+      for (int q = 0; q < 8; ++q) {
+        const int sl = s0 + q;
+        cf[q] = 0.f;
+        if (sl < K) {
+          const long long e = ir[sl];
+          if (e >= 0 && e < n_experts) {  // (phase 1 flagged any bad index)
+            cf[q] = cr[sl];
+            v[q] = w_out[e * chunks + c];
+          }
+        }
+      }
+#pragma unroll
+      for (int q = 0; q < 8; ++q) {
+        if (cf[q] == 0.f) continue;
+        const __nv_bfloat162* pv = reinterpret_cast<const __nv_bfloat162*>(&v[q]);
+#pragma unroll
+        for (int h = 0; h < 4; ++h) {
+          const float2 f = __bfloat1622float2(pv[h]);
+          acc[2 * h] = fmaf(cf[q], f.x, acc[2 * h]);
+          acc[2 * h + 1] = fmaf(cf[q], f.y, acc[2 * h + 1]);
+        }
+      }
+    }
+    uint4 o;
+    __nv_bfloat162* po2 = reinterpret_cast<__nv_bfloat162*>(&o);
+#pragma unroll
+    for (int h = 0; h < 4; ++h) po2[h] = __floats2bfloat162_rn(acc[2 * h], acc[2 * h + 1]);
+    out[t * chunks + c] = o;
+  }
+}
+
 cudaError_t launch_atomic_experts(int T, int d, int K, int act, const void* x, const void* w_in, const void* w_out,
                                   const int32_t* idx, const float* g, float* coef, void* out, long long n_experts,
                                   unsigned* bar, bool bar_zeroed, unsigned long long limit_ns, int* status,
                                   cudaStream_t s) {
+  if ((long long)T * K >= AW_MIN_TASKS) {
+    const long long tasks = (long long)T * K;
+    const long long cap = (long long)num_sms() * 8;  // 8 blocks of 8 warps per SM
+    const int gc = (int)std::min<long long>(cap, (tasks + AW_THREADS / 32 - 1) / (AW_THREADS / 32));
+    cudaError_t e = launch_k(atomic_coef_kernel, gc, AW_THREADS, 0, s, T, d, K, act, (const uint4*)x,
+                             (const uint4*)w_in, idx, g, coef, n_experts, status);
+    count_launch();
+    if (e != cudaSuccess) return e;
+    const long long units = (long long)((d / 8 + 15) / 16) * (((long long)T + 1) / 2);
+    const int ga = (int)std::min<long long>(cap, (units + AW_THREADS / 32 - 1) / (AW_THREADS / 32));
+    e = launch_k(atomic_assemble_kernel, ga, AW_THREADS, 0, s, T, d, K, (const uint4*)w_out, idx, coef, (uint4*)out,
+                 n_experts);
+    count_launch();
+    if (e != cudaSuccess) return e;
+    return cudaGetLastError();
+  }
   if (!bar_zeroed) {
     cudaError_t e = cudaMemsetAsync(bar, 0, sizeof(unsigned), s);
     if (e != cudaSuccess) return e;
