@@ -17,7 +17,7 @@ CSRC = os.path.join(PKG, "csrc")
 BUILD = os.path.join(ROOT, "_build")
 LIB = os.path.join(PKG, "libmoe.so")
 SOURCES = ["tc_gemm.cu", "route.cu", "simt_gemm.cu", "atomic.cu", "floe.cu", "quant.cu", "api.cu", "noalloc.cu"]
-HEADERS = [os.path.join(CSRC, "common.cuh"), os.path.join(ROOT, "include", "moe.h")]
+HEADERS = [os.path.join(CSRC, "common.cuh"), os.path.join(CSRC, "atomic.cuh"), os.path.join(ROOT, "include", "moe.h")]
 
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 FLAGS = ["-O3", "-std=c++17", "-lineinfo", "-Xcompiler", "-fPIC", "-Xcompiler", "-fvisibility=hidden",

@@ -7,7 +7,7 @@
 #include <cstring>
 #include <initializer_list>
 
-#include "common.cuh"
+#include "atomic.cuh"
 
 namespace moe {
 
@@ -799,7 +799,7 @@ static moe_status_t check_atomic_cfg(const moe_atomic_config_t* c) {
 
 struct AtomicPlan {
   int ksplit, kbps;
-  size_t status, zr, zc, idx, g, coef, bar, total;
+  size_t status, zr, zc, idx, g, coef, bar, sort, total;
 };
 
 static AtomicPlan make_atomic_plan(const moe_atomic_config_t& c) {
@@ -822,6 +822,9 @@ static AtomicPlan make_atomic_plan(const moe_atomic_config_t& c) {
   p.g = take((size_t)c.T * c.K * 4);
   p.coef = take((size_t)c.T * c.K * 4);
   p.bar = take(256);  // grid-barrier word of the experts kernel
+  const long long tasks = (long long)c.T * c.K;
+  // prefill budgets: the counting sort of the tasks by expert (run ends, then the order)
+  p.sort = tasks >= ATOMIC_WIDE_MIN_TASKS ? take(((size_t)c.Nr * c.Nc + (size_t)tasks) * 4) : 0;
   p.total = off;
   return p;
 }
@@ -899,9 +902,10 @@ moe_status_t moe_atomic_experts(const moe_atomic_config_t* cfg, const void* x, c
   if (!ws || ((uintptr_t)ws & 255u)) return MOE_ERR_INVALID_ARG;
   if (ws_bytes < P.total) return MOE_ERR_WORKSPACE;
   MOE_TRY(check_device());
-  return cuda_status(launch_atomic_experts(c.T, c.d, c.K, c.act, x, w_in, w_out, idx, g, at<float>(ws, P.coef), out,
+  return cuda_status(launch_atomic_experts_sorted(c.T, c.d, c.K, c.act, x, w_in, w_out, idx, g, at<float>(ws, P.coef), out,
                                            (long long)c.Nr * c.Nc, at<unsigned>(ws, P.bar), false, g_wait_limit_ns,
-                                           at<int>(ws, P.status), (cudaStream_t)stream));
+                                           at<int>(ws, P.status), P.sort ? at<int32_t>(ws, P.sort) : nullptr,
+                                           (cudaStream_t)stream));
 }
 
 moe_status_t moe_atomic_forward(const moe_atomic_config_t* cfg, const void* x, const void* w_row, const void* w_col,
@@ -922,9 +926,9 @@ moe_status_t moe_atomic_forward(const moe_atomic_config_t* cfg, const void* x, c
   MOE_TRY(mark_stage(0, s));
   MOE_TRY(atomic_route_impl(c, P, x, w_row, w_col, nullptr, nullptr, idx, g, ws, s, true));
   // the select kernel cleared the barrier word; the experts kernel is one launch
-  MOE_CUDA(launch_atomic_experts(c.T, c.d, c.K, c.act, x, w_in, w_out, idx, g, at<float>(ws, P.coef), out,
+  MOE_CUDA(launch_atomic_experts_sorted(c.T, c.d, c.K, c.act, x, w_in, w_out, idx, g, at<float>(ws, P.coef), out,
                                  (long long)c.Nr * c.Nc, at<unsigned>(ws, P.bar), true, g_wait_limit_ns,
-                                 at<int>(ws, P.status), s));
+                                 at<int>(ws, P.status), P.sort ? at<int32_t>(ws, P.sort) : nullptr, s));
   MOE_TRY(mark_stage(3, s));
   return mark_stage(4, s);
 }

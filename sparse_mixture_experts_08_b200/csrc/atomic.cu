@@ -18,7 +18,7 @@
 
 #include <algorithm>
 
-#include "common.cuh"
+#include "atomic.cuh"
 
 namespace moe {
 
@@ -848,14 +848,84 @@ __global__ void __launch_bounds__(AX_THREADS)
 }
 
 // Prefill budgets (many tasks): the two phases as separate, fully occupied kernels.
-// Coefficients: one warp per task, as phase 1 above.
+// Coefficients: one warp per task, as phase 1 above, with the tasks taken in
+// expert order (OmniMoE's expert-centric scheduling: a counting sort of the tasks
+// by expert), so each w_in row is read from HBM once and its other tasks hit L2
+// while the token rows (T x d) stay in L2 too.
 constexpr int AW_THREADS = 256;
-constexpr long long AW_MIN_TASKS = 16384;  // below this the single cooperative launch wins
+constexpr long long AW_MIN_TASKS = ATOMIC_WIDE_MIN_TASKS;  // below this the single cooperative launch wins
+
+// counts[e] = tasks of expert e (counts zeroed by the caller); a task whose expert
+// index is out of range is counted nowhere and flagged
+__global__ void __launch_bounds__(AW_THREADS)
+    atomic_count_kernel(long long tasks, const int32_t* __restrict__ idx, int32_t* __restrict__ counts,
+                        long long n_experts, int* status) {
+  pdl_launch_dependents();
+  pdl_wait();
+  for (long long q = (long long)blockIdx.x * AW_THREADS + threadIdx.x; q < tasks; q += (long long)gridDim.x * AW_THREADS) {
+    const long long e = idx[q];
+    if (e >= 0 && e < n_experts) atomicAdd(&counts[e], 1);
+    else set_status(status, MOE_ERR_DEVICE_INDEX);
+  }
+}
+
+// counts -> exclusive prefix sums in place (one block): thread i scans a contiguous
+// run of n / 1024 entries, the runs' totals are scanned across the block.
+__global__ void __launch_bounds__(1024) atomic_scan_kernel(long long n, int32_t* __restrict__ counts) {
+  __shared__ int warp_tot[32];
+  pdl_launch_dependents();
+  pdl_wait();
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const long long per = (n + 1023) / 1024, lo = (long long)tid * per, hi = min(n, lo + per);
+  int sum = 0;
+  for (long long i = lo; i < hi; ++i) sum += counts[i];
+  int incl = sum;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int v = __shfl_up_sync(FULL, incl, o);
+    if (lane >= o) incl += v;
+  }
+  if (lane == 31) warp_tot[warp] = incl;
+  __syncthreads();
+  if (warp == 0) {
+    int w = warp_tot[lane];
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int v = __shfl_up_sync(FULL, w, o);
+      if (lane >= o) w += v;
+    }
+    warp_tot[lane] = w;  // inclusive over warps
+  }
+  __syncthreads();
+  int run = incl - sum + (warp ? warp_tot[warp - 1] : 0);
+  for (long long i = lo; i < hi; ++i) {
+    const int c = counts[i];
+    counts[i] = run;
+    run += c;
+  }
+}
+
+// order[cursor[e]++] = task: afterwards cursor[e] is the end of expert e's run (the
+// order inside a run is arbitrary; every coefficient is computed on its own)
+__global__ void __launch_bounds__(AW_THREADS)
+    atomic_scatter_kernel(long long tasks, const int32_t* __restrict__ idx, int32_t* __restrict__ cursor,
+                          int32_t* __restrict__ order, long long n_experts) {
+  pdl_launch_dependents();
+  pdl_wait();
+  for (long long q = (long long)blockIdx.x * AW_THREADS + threadIdx.x; q < tasks; q += (long long)gridDim.x * AW_THREADS) {
+    const long long e = idx[q];
+    if (e >= 0 && e < n_experts) {
+      const int pos = atomicAdd(&cursor[e], 1);
+      if (pos >= 0 && pos < tasks) order[pos] = (int32_t)q;
+    }
+  }
+}
 
 __global__ void __launch_bounds__(AW_THREADS)
     atomic_coef_kernel(int T, int d, int K, int act, const uint4* __restrict__ x, const uint4* __restrict__ w_in,
                        const int32_t* __restrict__ idx, const float* __restrict__ g, float* __restrict__ coef,
-                       long long n_experts, int* status) {
+                       const int32_t* __restrict__ order, const int32_t* __restrict__ n_ordered, long long n_experts,
+                       int* status) {
   pdl_launch_dependents();
   pdl_wait();
   const int lane = threadIdx.x & 31;
@@ -863,6 +933,17 @@ __global__ void __launch_bounds__(AW_THREADS)
   const long long nwarps = (long long)gridDim.x * (AW_THREADS / 32);
   const int chunks = d / 8;
   const long long tasks = (long long)T * K;
+  if (order) {  // expert order: valid tasks only (a task with a bad index never entered it)
+    const long long n_valid = min((long long)*n_ordered, tasks);  // end of the last expert's run
+    for (long long pos = gwarp; pos < n_valid; pos += nwarps) {
+      const long long task = order[pos];
+      if (task < 0 || task >= tasks) continue;
+      const long long e = idx[task];
+      const float z = warp_dot_bf16(x + (task / K) * chunks, w_in + e * chunks, chunks, lane);
+      if (lane == 0) coef[task] = g[task] * atomic_act(z, act);
+    }
+    return;
+  }
   for (long long task = gwarp; task < tasks; task += nwarps) {
     const long long e = idx[task];
     if (e < 0 || e >= n_experts) {
@@ -940,12 +1021,42 @@ cudaError_t launch_atomic_experts(int T, int d, int K, int act, const void* x, c
                                   const int32_t* idx, const float* g, float* coef, void* out, long long n_experts,
                                   unsigned* bar, bool bar_zeroed, unsigned long long limit_ns, int* status,
                                   cudaStream_t s) {
+  return launch_atomic_experts_sorted(T, d, K, act, x, w_in, w_out, idx, g, coef, out, n_experts, bar, bar_zeroed,
+                                      limit_ns, status, nullptr, s);
+}
+
+cudaError_t launch_atomic_experts_sorted(int T, int d, int K, int act, const void* x, const void* w_in,
+                                         const void* w_out, const int32_t* idx, const float* g, float* coef, void* out,
+                                         long long n_experts, unsigned* bar, bool bar_zeroed,
+                                         unsigned long long limit_ns, int* status, int32_t* sort_ws, cudaStream_t s) {
   if ((long long)T * K >= AW_MIN_TASKS) {
     const long long tasks = (long long)T * K;
     const long long cap = (long long)num_sms() * 8;  // 8 blocks of 8 warps per SM
     const int gc = (int)std::min<long long>(cap, (tasks + AW_THREADS / 32 - 1) / (AW_THREADS / 32));
-    cudaError_t e = launch_k(atomic_coef_kernel, gc, AW_THREADS, 0, s, T, d, K, act, (const uint4*)x,
-                             (const uint4*)w_in, idx, g, coef, n_experts, status);
+    cudaError_t e = cudaSuccess;
+    const int32_t* order = nullptr;
+    const int32_t* n_ordered = nullptr;
+    if (sort_ws) {  // counting sort of the tasks by expert
+      int32_t* cursor = sort_ws;
+      int32_t* ord = sort_ws + n_experts;
+      // tasks with a bad index are left out of the order: zero their coefficients first
+      if ((e = cudaMemsetAsync(coef, 0, (size_t)tasks * sizeof(float), s)) != cudaSuccess) return e;
+      if ((e = cudaMemsetAsync(cursor, 0, (size_t)n_experts * sizeof(int32_t), s)) != cudaSuccess) return e;
+      const int gs = (int)std::min<long long>((long long)num_sms() * 8, (tasks + AW_THREADS - 1) / AW_THREADS);
+      e = launch_k(atomic_count_kernel, gs, AW_THREADS, 0, s, tasks, idx, cursor, n_experts, status);
+      count_launch();
+      if (e != cudaSuccess) return e;
+      e = launch_k(atomic_scan_kernel, 1, 1024, 0, s, n_experts, cursor);
+      count_launch();
+      if (e != cudaSuccess) return e;
+      e = launch_k(atomic_scatter_kernel, gs, AW_THREADS, 0, s, tasks, idx, cursor, ord, n_experts);
+      count_launch();
+      if (e != cudaSuccess) return e;
+      order = ord;
+      n_ordered = cursor + (n_experts - 1);  // after the scatter: the end of the last run
+    }
+    e = launch_k(atomic_coef_kernel, gc, AW_THREADS, 0, s, T, d, K, act, (const uint4*)x, (const uint4*)w_in, idx,
+                 g, coef, order, n_ordered, n_experts, status);
     count_launch();
     if (e != cudaSuccess) return e;
     const long long units = (long long)((d / 8 + 15) / 16) * (((long long)T + 1) / 2);
