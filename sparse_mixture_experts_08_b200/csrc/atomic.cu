@@ -870,15 +870,23 @@ __global__ void __launch_bounds__(AW_THREADS)
 }
 
 // counts -> exclusive prefix sums in place (one block): thread i scans a contiguous
-// run of n / 1024 entries, the runs' totals are scanned across the block.
+// run of counters (a multiple of 4, read and written as int4: the array is 16-byte
+// aligned), the runs' totals are scanned across the block.
 __global__ void __launch_bounds__(1024) atomic_scan_kernel(long long n, int32_t* __restrict__ counts) {
   __shared__ int warp_tot[32];
   pdl_launch_dependents();
   pdl_wait();
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const long long per = (n + 1023) / 1024, lo = (long long)tid * per, hi = min(n, lo + per);
+  const long long per = (((n + 1023) / 1024) + 3) & ~3LL;
+  const long long lo = min(n, (long long)tid * per), hi = min(n, lo + per);
+  const long long hi4 = lo + ((hi - lo) & ~3LL);  // end of the whole int4s of the run
   int sum = 0;
-  for (long long i = lo; i < hi; ++i) sum += counts[i];
+#pragma unroll 8
+  for (long long i = lo; i < hi4; i += 4) {
+    const int4 v = *reinterpret_cast<const int4*>(counts + i);
+    sum += (v.x + v.y) + (v.z + v.w);
+  }
+  for (long long i = hi4; i < hi; ++i) sum += counts[i];
   int incl = sum;
 #pragma unroll
   for (int o = 1; o < 32; o <<= 1) {
@@ -898,7 +906,18 @@ __global__ void __launch_bounds__(1024) atomic_scan_kernel(long long n, int32_t*
   }
   __syncthreads();
   int run = incl - sum + (warp ? warp_tot[warp - 1] : 0);
-  for (long long i = lo; i < hi; ++i) {
+#pragma unroll 8
+  for (long long i = lo; i < hi4; i += 4) {
+    int4 v = *reinterpret_cast<const int4*>(counts + i);
+    const int4 c = v;
+    v.x = run;
+    v.y = run + c.x;
+    v.z = v.y + c.y;
+    v.w = v.z + c.z;
+    run = v.w + c.w;
+    *reinterpret_cast<int4*>(counts + i) = v;
+  }
+  for (long long i = hi4; i < hi; ++i) {
     const int c = counts[i];
     counts[i] = run;
     run += c;
