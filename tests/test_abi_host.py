@@ -224,3 +224,20 @@ def test_fp8_entry_points_validate_on_the_host():
     assert call(relu, w, n.value - 256) == moe.ERR_WORKSPACE   # the pointer set itself is complete for ReLU
     w = moe.moe.MoEFp8Experts(**dict(full, gate=(1 << 24) + 4))
     assert call(ok, w, 1 << 30) == moe.ERR_INVALID_ARG         # codes must be 16-byte aligned
+
+
+def test_atomic_workspace_holds_the_expert_sort_at_prefill_budgets():
+    """From 16384 (token, slot) tasks on, the workspace adds the counting sort of the
+    tasks by expert: one int32 run end per expert and one int32 per task."""
+    lib = moe.moe.lib()
+    n = ctypes.c_size_t(0)
+
+    def size(T, K):
+        c = MoEAtomicConfig(T=T, d=4096, Nr=512, Nc=512, K=K, act=moe.ATOMIC_SILU, dtype=moe.BF16)
+        assert lib.moe_atomic_workspace_size(ctypes.byref(c), ctypes.byref(n)) == moe.OK
+        return n.value
+
+    small = size(16, 64)        # 1024 tasks: the single cooperative launch, no sort
+    wide = size(4096, 512)      # 2M tasks
+    per_task_no_sort = 3 * 4    # idx, g, coef
+    assert wide - small >= (4096 * 512 - 16 * 64) * (per_task_no_sort + 4) + 512 * 512 * 4
