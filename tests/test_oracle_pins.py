@@ -400,6 +400,53 @@ def test_grid_topk_method_exact_on_adversarial_grids():
             assert grid_topk_threshold_method(lr, lc, K) == idx[0].tolist()
 
 
+def grid_topk_staircase_method(lr, lc, K):
+    """The prefill-budget selection method (K > 64) of the GPU kernel, restated in plain
+    Python: with rows and columns sorted by (value desc, index asc), the candidates are
+    the staircase pairs (a, b) with (a+1)(b+1) <= K; tau = the K-th best candidate score.
+    If every staircase row's first pair past the staircase, and the first row left out,
+    score below tau, the answer is the first K of the staircase pairs scoring >= tau in
+    (score desc, id asc) order; otherwise the pairs above tau plus the lowest-id pairs of
+    the whole grid scoring exactly tau. Returns (flat ids, whether the bound held)."""
+    Nr, Nc = len(lr), len(lc)
+    rows = sorted(range(Nr), key=lambda i: (-float(lr[i]), i))
+    cols = sorted(range(Nc), key=lambda j: (-float(lc[j]), j))
+    S = lambda i, j: np.float32(np.float32(lr[i]) + np.float32(lc[j]))
+    kr = min(Nr, K)
+    stair = [(S(rows[a], cols[b]), rows[a] * Nc + cols[b]) for a in range(kr) for b in range(min(Nc, K // (a + 1)))]
+    tau = sorted((p[0] for p in stair), key=lambda v: -float(v))[K - 1]
+    outside = any(min(Nc, K // (a + 1)) < Nc and S(rows[a], cols[min(Nc, K // (a + 1))]) >= tau for a in range(kr))
+    outside = outside or (kr < Nr and S(rows[kr], cols[0]) >= tau)
+    if not outside:
+        win = sorted((p for p in stair if p[0] >= tau), key=lambda p: (-float(p[0]), p[1]))[:K]
+        return [q for _, q in win], True
+    above = [p for p in stair if p[0] > tau]
+    need = K - len(above)
+    tied = [(S(q // Nc, q % Nc), q) for q in range(Nr * Nc) if S(q // Nc, q % Nc) == tau][:need]
+    return [q for _, q in sorted(above + tied, key=lambda p: (-float(p[0]), p[1]))], False
+
+
+def test_grid_topk_staircase_method_exact():
+    """Both branches of the prefill-budget method against the oracle's brute-force sort:
+    random grids (the bound holds), level grids and all-equal grids (ties reach past
+    the staircase), and the rounding-collapse case, for K up to the whole grid."""
+    rng = np.random.default_rng(12)
+    cases = [_collapse_case(), (np.zeros(9, np.float32), np.zeros(7, np.float32))]
+    for _ in range(12):
+        Nr, Nc = int(rng.integers(2, 40)), int(rng.integers(2, 40))
+        cases.append(((rng.standard_normal(Nr) - 6).astype(np.float32), (rng.standard_normal(Nc) - 6).astype(np.float32)))
+        cases.append(((rng.integers(0, 3, Nr) - 5).astype(np.float32), (rng.integers(0, 3, Nc) - 5).astype(np.float32)))
+    branches = set()
+    for lr, lc in cases:
+        N = lr.size * lc.size
+        for K in sorted({1, 2, min(65, N), min(100, N), N // 2 or 1, N}):
+            idx, _ = O.atomic_select(lr[None], lc[None], K)
+            got, fast = grid_topk_staircase_method(lr, lc, K)
+            assert got == idx[0].tolist(), (lr.size, lc.size, K)
+            branches.add(fast)
+    assert branches == {True, False}  # both branches were exercised
+
+
 def test_plain_candidate_block_is_not_always_exact():
     # Selecting only inside top-K rows x top-K cols misses (0, 0) here: the
     # rounding of the fp32 sums ties it with rows 1 and 2, and it has the lowest id.
