@@ -1,0 +1,60 @@
+"""Host-side logic of bench.py (no GPU): the algorithmic byte counts behind the
+roofline fractions and the rule that ties an ncu traffic figure to the sources of
+its kernel."""
+import json
+import os
+import sys
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+sys.path.insert(0, ROOT)
+
+import bench  # noqa: E402
+import workloads as W  # noqa: E402
+
+
+def test_fp8_weights_count_one_byte_each():
+    cfg = W.CONFIGS["decode"]
+    active = 8
+    bf16, _, bf16_layer = bench.stage_costs(cfg, active, 1)
+    fp8, _, fp8_layer = bench.stage_costs(cfg, active, 1, weight_bytes=1)
+    mats = 2  # SwiGLU: gate and up
+    assert bf16["expert_up"][1] - fp8["expert_up"][1] == active * mats * cfg.f * cfg.d
+    assert bf16["expert_down"][1] - fp8["expert_down"][1] == active * cfg.d * cfg.f
+    assert bf16["expert_up"][0] == fp8["expert_up"][0]  # the same flops
+    assert bf16_layer - fp8_layer == active * (mats + 1) * cfg.f * cfg.d
+
+
+def test_stage_bytes_match_the_layer_definition():
+    cfg = W.CONFIGS["switch"]  # top-1 ReLU, no shared experts: the down projection writes out itself
+    c, flops, layer_bytes = bench.stage_costs(cfg, cfg.m, 1)
+    Tk = cfg.T * cfg.k
+    assert c["expert_up"][0] == 2.0 * cfg.f * cfg.d * Tk
+    assert c["expert_down"][1] == cfg.m * cfg.d * cfg.f * 2 + Tk * cfg.f * 2 + cfg.T * cfg.d * 2
+    assert c["combine"][1] == 0.0
+    assert layer_bytes == cfg.m * cfg.d * 2 + cfg.m * 2 * cfg.f * cfg.d * 2 + 2 * cfg.T * cfg.d * 2
+
+
+def test_committed_traffic_matches_the_current_gemm_sources():
+    with open(os.path.join(ROOT, "profiles", "traffic.json")) as fh:
+        t = json.load(fh)
+    e = t["switch"]["expert_up"]
+    assert e["source_files"] == ["tc_gemm.cu", "common.cuh"]
+    assert bench.traffic_for("switch", "expert_up") == e["dram_bytes_per_launch"]
+
+
+def test_traffic_goes_null_when_its_kernel_sources_change(tmp_path, monkeypatch):
+    csrc = tmp_path / "sparse_mixture_experts_08_b200" / "csrc"
+    csrc.mkdir(parents=True)
+    (csrc / "k.cu").write_text("kernel v1")
+    (csrc / "other.cu").write_text("unrelated")
+    (tmp_path / "profiles").mkdir()
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    h = bench.source_hash(["k.cu"])
+    (tmp_path / "profiles" / "traffic.json").write_text(json.dumps(
+        {"w": {"s": {"dram_bytes_per_launch": 123.0, "source_hash": h, "source_files": ["k.cu"]}}}))
+    assert bench.traffic_for("w", "s") == 123.0
+    (csrc / "other.cu").write_text("unrelated, edited")  # another kernel's file: still valid
+    assert bench.traffic_for("w", "s") == 123.0
+    (csrc / "k.cu").write_text("kernel v2")              # the captured kernel changed: no figure
+    assert bench.traffic_for("w", "s") is None
+    assert bench.traffic_for("w", "missing") is None
