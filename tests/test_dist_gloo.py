@@ -44,8 +44,9 @@ def _worker(rank, world, port, q):
         hashes = [None] * world
         dist.all_gather_object(hashes, (wh, xh))
         out = O.layer_forward(cfg, inp)["out"]
+        out8 = O.layer_forward_fp8(cfg, inp)["out"]  # the 8-bit layer: per-row scales, so also per token
         outs = [None] * world
-        dist.all_gather_object(outs, (inp["x"], out))
+        dist.all_gather_object(outs, (inp["x"], out, out8))
         mx = bench.max_over_ranks([float(rank + 1), 10.0 - rank], dist)
         q.put((rank, hashes, outs, mx))
     finally:
@@ -91,3 +92,20 @@ def test_token_sharding_leaves_outputs_unchanged(two_ranks):
     inp["x"] = np.concatenate([outs[0][0], outs[1][0]])
     whole = O.layer_forward(cfg, inp)["out"]
     np.testing.assert_array_equal(whole, np.concatenate([outs[0][1], outs[1][1]]))
+
+
+def test_token_sharding_leaves_8bit_outputs_unchanged(two_ranks):
+    """x and h are quantized per row (token, task), never across the batch, so the 8-bit
+    layer shards by tokens with no exchange either."""
+    import sys
+
+    sys.path.insert(0, ROOT)
+    import oracle as O
+    import workloads as W
+
+    cfg = W.small_moe(T=48, d=64, f=96, m=6, k=2, dtype=W.BF16, zipf_s=1.0, index=41, name="dp_small")
+    outs = two_ranks[0][2]
+    inp = W.make_moe_inputs(cfg, replicate=0)
+    inp["x"] = np.concatenate([outs[0][0], outs[1][0]])
+    whole = O.layer_forward_fp8(cfg, inp)["out"]
+    np.testing.assert_allclose(whole, np.concatenate([outs[0][2], outs[1][2]]), rtol=1e-12, atol=0)
