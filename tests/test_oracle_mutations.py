@@ -60,6 +60,11 @@ PY_MUTATIONS = {
     "fp8_h_scale_dropped": ("H = e4m3_value(hq) * hs[:, None].astype(np.float64)", "H = e4m3_value(hq)"),
     "fp8_x_scale_dropped": ("X = e4m3_value(xq) * sx[:, None].astype(np.float64)", "X = e4m3_value(xq)"),
     "fp8_column_scales": ("amax = np.max(np.abs(a), axis=1) if", "amax = np.max(np.abs(a), axis=0)[:a.shape[0]] if"),
+    "fp8_up_scale_from_gate": ("b = X @ (e4m3_value(uq) * us[:, None].astype(np.float64)).T",
+                               "b = X @ (e4m3_value(uq) * gs[:, None].astype(np.float64)).T"),
+    "fp8_silu_dropped": ("return a / (1.0 + np.exp(-a)) * b", "return a * b"),
+    "bf16_truncates": ("u = (u + 0x7FFF + ((u >> 16) & 1)) >> 16 << 16", "u = u >> 16 << 16"),
+    "bf16_ties_away": ("u = (u + 0x7FFF + ((u >> 16) & 1)) >> 16 << 16", "u = (u + 0x8000) >> 16 << 16"),
 }
 
 
@@ -234,10 +239,32 @@ def check_fp8(O):
         inp[key] = pw(inp[key].shape, -3, 0)
     ref = O.layer_forward(cfg, inp)["out"]
     np.testing.assert_allclose(O.layer_forward_fp8(cfg, inp)["out"], ref, rtol=1e-5, atol=1e-6 * np.abs(ref).max())
+    # SwiGLU on exact inputs: one-hot rows of 2^9..2^10 make every gate pre-activation
+    # 0 or at least 2^6 in size, where SiLU(g) = g (or ~0); see test_oracle_pins
+    cfg = W.small_moe(T=20, d=32, f=16, m=4, k=2, act=W.SWIGLU, dtype=W.BF16, zipf_s=0.5, n_shared=1,
+                      f_shared=16, index=96)
+    inp = W.make_moe_inputs(cfg)
+    x = np.zeros((cfg.T, cfg.d), np.uint16)
+    x[np.arange(cfg.T), rng.integers(0, cfg.d, cfg.T)] = (((rng.integers(9, 11, cfg.T) + 127) << 7)
+                                                          | (rng.integers(0, 2, cfg.T) << 15)).astype(np.uint16)
+    inp["x"] = x
+    for key in ("w_gate", "w_up", "w_down", "ws_gate", "ws_up", "ws_down"):
+        inp[key] = pw(inp[key].shape, -6, -3) if key.endswith("up") else pw(inp[key].shape, -3, 0)
+    ref = O.layer_forward(cfg, inp)["out"]
+    np.testing.assert_allclose(O.layer_forward_fp8(cfg, inp)["out"], ref, rtol=1e-5, atol=1e-6 * np.abs(ref).max())
+
+
+def check_round_bf16(O):
+    # hand-worked ties (bf16 spacing 2^-7 next to 1): 1 + 2^-8 -> 1, 1 + 3 2^-8 -> 1 + 2^-6
+    v = np.array([1 + 2.0 ** -8, 1 + 3 * 2.0 ** -8, 1 + 2.0 ** -8 + 2.0 ** -20, -(1 + 3 * 2.0 ** -8), 255.5])
+    assert O.round_bf16(v).tolist() == [1.0, 1 + 2.0 ** -6, 1 + 2.0 ** -7, -(1 + 2.0 ** -6), 256.0]
+    f = np.random.default_rng(3).standard_normal(5000).astype(np.float32)
+    ref = torch.from_numpy(f).to(torch.bfloat16).float().numpy()
+    np.testing.assert_array_equal(O.round_bf16(f.astype(np.float64)), ref)
 
 
 CHECKS = [check_lis_golden, check_topk, check_router, check_permutation, check_ffn, check_shared, check_atomic,
-          check_replica, check_floe, check_fp8]
+          check_replica, check_floe, check_fp8, check_round_bf16]
 
 
 def _failures(O):

@@ -688,6 +688,81 @@ def test_fp8_layer_is_lossless_on_power_of_two_inputs():
     np.testing.assert_allclose(got, ref, rtol=1e-5, atol=1e-6 * np.abs(ref).max())
 
 
+def _swiglu_pow2_case(seed):
+    """A SwiGLU layer whose 8-bit run is exact: one-hot token rows of +-2^9 or 2^10,
+    gate and down weights +-2^-3 .. 2^0, up weights +-2^-6 .. 2^-3 (some zero). Every
+    gate pre-activation is then 0 or +-2^6 .. 2^10: at +2^6 and above the logistic
+    function is 1 in fp64 (exp(-64) is below half an ulp of 1), so SiLU(g) = g and
+    h = g u is a power of two; at -2^6 and below h is ~1e-26 u. A row's non-negligible
+    h values (2^9 .. 2^17) span at most 2^8, so each lands on an E4M3 code after its row scale;
+    the negligible ones quantize to 0."""
+    cfg = W.small_moe(T=20, d=32, f=16, m=4, k=2, act=W.SWIGLU, dtype=W.BF16, zipf_s=0.5, n_shared=1,
+                      f_shared=16, index=96)
+    inp = W.make_moe_inputs(cfg)
+    rng = np.random.default_rng(seed)
+    x = np.zeros((cfg.T, cfg.d), np.uint16)
+    x[np.arange(cfg.T), rng.integers(0, cfg.d, cfg.T)] = _pow2_bf16(rng, cfg.T, 9, 10, p_zero=0.0)
+    inp["x"] = x
+    for key in ("w_gate", "w_up", "w_down", "ws_gate", "ws_up", "ws_down"):
+        lo, hi = (-6, -3) if key.endswith("up") else (-3, 0)  # up rows on another scale than gate rows
+        inp[key] = _pow2_bf16(rng, inp[key].shape, lo, hi)
+    return cfg, inp
+
+
+def test_fp8_swiglu_layer_is_lossless_on_power_of_two_inputs():
+    """The SwiGLU branch of the 8-bit oracle (gate and up scales, SiLU, h's row
+    scale) against the bf16 oracle on inputs where every quantization is exact:
+    equal up to the fp32 rounding of the scales. A swapped scale, a dropped SiLU or
+    a dropped up factor changes the output by a power of two or more."""
+    cfg, inp = _swiglu_pow2_case(12)
+    ref = O.layer_forward(cfg, inp)["out"]
+    got = O.layer_forward_fp8(cfg, inp)["out"]
+    assert np.abs(ref).max() > 1.0
+    np.testing.assert_allclose(got, ref, rtol=1e-5, atol=1e-6 * np.abs(ref).max())
+
+
+# --------------------------------------------- bf16 rounding of stored activations
+# bf16 keeps 8 significand bits (7 stored): next to 1 its spacing is 2^-7. A value
+# exactly half way between two bf16 numbers goes to the one with an even last
+# significand bit (IEEE 754 round to nearest, ties to even); the oracle rounds
+# float64 to float32 first, then float32 to bf16.
+BF16_CASES = [
+    (1.0 + 2.0 ** -8, 1.0),                       # tie between 1 (even) and 1 + 2^-7 (odd): down
+    (1.0 + 3 * 2.0 ** -8, 1.0 + 2.0 ** -6),       # tie between 1 + 2^-7 (odd) and 1 + 2^-6 (even): up
+    (1.0 + 2.0 ** -8 + 2.0 ** -20, 1.0 + 2.0 ** -7),  # just above the tie: up
+    (1.0 + 2.0 ** -8 - 2.0 ** -20, 1.0),          # just below: down
+    (-(1.0 + 2.0 ** -8), -1.0),                   # the sign does not change the tie rule
+    (-(1.0 + 3 * 2.0 ** -8), -(1.0 + 2.0 ** -6)),
+    (1.0 + 2.0 ** -8 + 2.0 ** -30, 1.0),          # 2^-30 is lost in the float32 step; then a tie
+    (255.5, 256.0),                               # 255 and 256 are neighbours near 2^8: the tie goes to 256
+    (3.0, 3.0),                                   # representable values are unchanged
+    (2.0 ** -133, 2.0 ** -133),                   # a float32 subnormal that bf16 holds exactly
+    (0.0, 0.0),
+]
+
+
+def test_round_bf16_hand_worked_ties_to_even():
+    v = np.array([a for a, _ in BF16_CASES], np.float64)
+    got = O.round_bf16(v)
+    assert got.dtype == np.float32
+    assert got.tolist() == [b for _, b in BF16_CASES]
+    assert np.signbit(O.round_bf16(np.array([-0.0])))[0]
+    big = O.round_bf16(np.array([np.finfo(np.float32).max], np.float64))  # past the largest bf16: infinity
+    assert np.isinf(big[0])
+
+
+def test_round_bf16_matches_torch_bfloat16_cast():
+    rng = np.random.default_rng(31)
+    bits = rng.integers(0, 2 ** 32, 200000, dtype=np.uint64).astype(np.uint32)
+    bits = bits[(bits & 0x7F800000) != 0x7F800000]   # no inf / NaN patterns
+    ties = ((rng.integers(0, 2 ** 16, 20000, dtype=np.uint64) << 16) | 0x8000).astype(np.uint32)
+    ties = ties[(ties & 0x7F800000) != 0x7F800000]   # exact ties, both parities of the kept part
+    f = np.concatenate([bits, ties]).view(np.float32)
+    ref = torch.from_numpy(f.copy()).to(torch.bfloat16).float().numpy()
+    got = O.round_bf16(f.astype(np.float64))
+    np.testing.assert_array_equal(got.view(np.uint32), ref.view(np.uint32))
+
+
 @pytest.mark.parametrize("act", [W.SWIGLU, W.RELU])
 def test_fp8_layer_is_close_to_bf16_layer(act):
     """On random bf16 inputs the 8-bit layer differs from the bf16 layer by the
