@@ -167,12 +167,17 @@ MOE_API moe_status_t moe_combine(const moe_config_t* cfg, const float* y_perm, c
 /* The whole layer in one call, on one stream with no host synchronisation:
  * route -> histogram/LIS -> permute -> grouped FFN (+ shared experts) -> combine.
  * Optional device outputs (each may be NULL): logits_out [T, m], topk_idx_out,
- * topk_w_out [T, k], counts_out [m], lis_out. w_up / ws_up are NULL for ReLU;
- * ws_* are NULL when n_shared == 0. */
+ * topk_w_out [T, k], counts_out [m], lis_out; and copies of the expert-centric
+ * permutation the layer computed, as moe_histogram_lis / moe_permute define it
+ * (OmniMoE Fig. 3): offsets_out [m + 1], perm_out [T k] (segment row -> task
+ * t k + s), inv_perm_out [T k] (task -> segment row) and x_perm_out [T k, d]
+ * (the permuted token rows, cfg->dtype). w_up / ws_up are NULL for ReLU; ws_* are
+ * NULL when n_shared == 0. */
 MOE_API moe_status_t moe_layer_forward(const moe_config_t* cfg, const void* x, const void* w_router, const float* bias,
                                const void* w_gate, const void* w_up, const void* w_down, const void* ws_gate,
                                const void* ws_up, const void* ws_down, void* out, float* logits_out,
                                int32_t* topk_idx_out, float* topk_w_out, int32_t* counts_out, moe_lis_t* lis_out,
+                               int32_t* offsets_out, int32_t* perm_out, int32_t* inv_perm_out, void* x_perm_out,
                                void* ws, size_t ws_bytes, moe_stream_t stream);
 
 /* R&Q replica dispatch ("A Replicate-and-Quantize Strategy for Plug-and-Play Load

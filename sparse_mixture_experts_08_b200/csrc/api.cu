@@ -610,7 +610,8 @@ static moe_status_t layer_forward_impl(const moe_config_t& c, const void* x, con
                                        const void* ws_up, const void* ws_down, const moe_fp8_experts_t* wq, void* out,
                                        float* logits_out, int32_t* topk_idx_out, float* topk_w_out,
                                        int32_t* counts_out, moe_lis_t* lis_out, void* h_out, void* h_shared_out,
-                                       int32_t* perm_out, void* ws, cudaStream_t s) {
+                                       int32_t* perm_out, int32_t* offsets_out, int32_t* inv_perm_out,
+                                       void* x_perm_out, void* ws, cudaStream_t s) {
   const Plan pl = make_plan(c);
   const Layout L = make_layout(c, pl);
   int* status = at<int>(ws, L.status);
@@ -698,6 +699,11 @@ static moe_status_t layer_forward_impl(const moe_config_t& c, const void* x, con
     MOE_CUDA(cudaMemcpyAsync(h_shared_out, io.h_sh, (size_t)c.n_shared * c.T * c.f_shared * 2,
                              cudaMemcpyDeviceToDevice, s));
   if (perm_out) MOE_CUDA(cudaMemcpyAsync(perm_out, perm, (size_t)Tk * 4, cudaMemcpyDeviceToDevice, s));
+  if (inv_perm_out) MOE_CUDA(cudaMemcpyAsync(inv_perm_out, inv_perm, (size_t)Tk * 4, cudaMemcpyDeviceToDevice, s));
+  if (offsets_out)
+    MOE_CUDA(cudaMemcpyAsync(offsets_out, offsets, (size_t)(c.m + 1) * 4, cudaMemcpyDeviceToDevice, s));
+  if (x_perm_out)
+    MOE_CUDA(cudaMemcpyAsync(x_perm_out, io.x_perm, (size_t)Tk * c.d * pl.es, cudaMemcpyDeviceToDevice, s));
   if (!fuse_combine)
     MOE_CUDA(launch_combine(c.dtype, c.T, c.d, c.k, ksplit, io.y, Tk * c.d, inv_perm, c.n_shared, io.y_sh,
                             (long long)c.n_shared * c.T * c.d, out, s));
@@ -710,6 +716,7 @@ moe_status_t moe_layer_forward(const moe_config_t* cfg, const void* x, const voi
                                const void* w_gate, const void* w_up, const void* w_down, const void* ws_gate,
                                const void* ws_up, const void* ws_down, void* out, float* logits_out,
                                int32_t* topk_idx_out, float* topk_w_out, int32_t* counts_out, moe_lis_t* lis_out,
+                               int32_t* offsets_out, int32_t* perm_out, int32_t* inv_perm_out, void* x_perm_out,
                                void* ws, size_t ws_bytes, moe_stream_t stream) {
   MOE_TRY(check_cfg(cfg));
   const moe_config_t& c = *cfg;
@@ -718,13 +725,14 @@ moe_status_t moe_layer_forward(const moe_config_t* cfg, const void* x, const voi
   if (c.n_shared > 0 && (!ws_gate || !ws_down || (c.act == MOE_SWIGLU && !ws_up))) return MOE_ERR_INVALID_ARG;
   for (const void* p : std::initializer_list<const void*>{x, w_router, (const void*)bias, w_gate, w_up, w_down, ws_gate, ws_up, ws_down, out,
                         (const void*)logits_out, (const void*)topk_idx_out, (const void*)topk_w_out,
-                        (const void*)counts_out, (const void*)lis_out})
+                        (const void*)counts_out, (const void*)lis_out, (const void*)offsets_out,
+                        (const void*)perm_out, (const void*)inv_perm_out, x_perm_out})
     if (p && !aligned16(p)) return MOE_ERR_INVALID_ARG;
   MOE_TRY(check_ws(c, ws, ws_bytes, make_layout(c, make_plan(c)).total));
   MOE_TRY(check_device());
   return layer_forward_impl(c, x, w_router, bias, w_gate, w_up, w_down, ws_gate, ws_up, ws_down, nullptr, out,
-                            logits_out, topk_idx_out, topk_w_out, counts_out, lis_out, nullptr, nullptr, nullptr, ws,
-                            (cudaStream_t)stream);
+                            logits_out, topk_idx_out, topk_w_out, counts_out, lis_out, nullptr, nullptr, perm_out,
+                            offsets_out, inv_perm_out, x_perm_out, ws, (cudaStream_t)stream);
 }
 
 static moe_status_t check_fp8_cfg(const moe_config_t* cfg) {
@@ -781,7 +789,7 @@ moe_status_t moe_layer_forward_fp8(const moe_config_t* cfg, const void* x, const
   MOE_TRY(check_device());
   return layer_forward_impl(c, x, w_router, bias, nullptr, nullptr, nullptr, nullptr, nullptr, nullptr, wq, out,
                             logits_out, topk_idx_out, topk_w_out, counts_out, lis_out, h_out, h_shared_out, perm_out,
-                            ws, (cudaStream_t)stream);
+                            nullptr, nullptr, nullptr, ws, (cudaStream_t)stream);
 }
 
 // ------------------------------------------------------------------ atomic experts

@@ -82,7 +82,7 @@ def lib() -> ctypes.CDLL:
             "moe_grouped_ffn": [P, P, P, P, P, P, P, P, P, P, S, P],
             "moe_shared_ffn": [P, P, P, P, P, P, P, S, P],
             "moe_combine": [P, P, P, P, P, P],
-            "moe_layer_forward": [P, P, P, P, P, P, P, P, P, P, P, P, P, P, P, P, P, S, P],
+            "moe_layer_forward": [P, P, P, P, P, P, P, P, P, P, P, P, P, P, P, P, P, P, P, P, P, S, P],
             "moe_replica_split": [P, P, P, P, P, P, P, P, P, S, P],
             "moe_floe_pack_down": [P, P, P, P],
             "moe_floe_calibrate": [P, P, ctypes.c_int32, P, ctypes.c_double, P, P, P, S, P],
@@ -199,11 +199,12 @@ def moe_combine(cfg, y_perm, inv_perm, y_shared, out, stream=None):
 
 def moe_layer_forward(cfg, x, w_router, bias, w_gate, w_up, w_down, ws_gate, ws_up, ws_down, out, ws,
                       logits_out=None, topk_idx_out=None, topk_w_out=None, counts_out=None, lis_out=None,
-                      stream=None):
+                      offsets_out=None, perm_out=None, inv_perm_out=None, x_perm_out=None, stream=None):
     _check("moe_layer_forward", lib().moe_layer_forward(
         ctypes.byref(cfg), _p(x), _p(w_router), _p(bias), _p(w_gate), _p(w_up), _p(w_down), _p(ws_gate),
         _p(ws_up), _p(ws_down), _p(out), _p(logits_out), _p(topk_idx_out), _p(topk_w_out), _p(counts_out),
-        _p(lis_out), _p(ws), ws.numel(), _stream(stream)))
+        _p(lis_out), _p(offsets_out), _p(perm_out), _p(inv_perm_out), _p(x_perm_out), _p(ws), ws.numel(),
+        _stream(stream)))
 
 
 def moe_replica_split(cfg, topk_idx, offsets, inv_perm, lis, idx_out, ws, counts_out=None, lis_out=None,

@@ -53,6 +53,44 @@ def token_rel_err(got: np.ndarray, ref: np.ndarray) -> float:
     return float((num / np.maximum(den, 1e-300)).max())
 
 
+def elem_rel_err(got: np.ndarray, ref: np.ndarray) -> float:
+    """Elementwise companion figure (reported, not asserted): max |got - ref| /
+    (|ref| + 1e-3 rms(ref)) over all elements."""
+    rms = float(np.sqrt(np.mean(np.square(ref)))) if ref.size else 0.0
+    return float((np.abs(got - ref) / (np.abs(ref) + 1e-3 * rms + 1e-300)).max()) if ref.size else 0.0
+
+
+def err_report(got: np.ndarray, ref: np.ndarray) -> str:
+    return (f"max per-token relative error {token_rel_err(got, ref):.3e}, "
+            f"elementwise max |d|/(|ref| + 1e-3 rms) {elem_rel_err(got, ref):.3e}")
+
+
+def tile_cover_tokens(perm: np.ndarray, offsets: np.ndarray, k: int, tile: int = 128) -> np.ndarray:
+    """Tokens whose tasks reach every `tile`-row token tile of every expert segment
+    (the first and last row of each tile, counted from the segment start). A token
+    tile of any multiple of `tile` rows, in either projection, then holds at least
+    one checked task."""
+    pick = set()
+    for e in range(len(offsets) - 1):
+        a, b = int(offsets[e]), int(offsets[e + 1])
+        for r0 in range(a, b, tile):
+            pick.add(int(perm[r0]) // k)
+            pick.add(int(perm[min(b, r0 + tile) - 1]) // k)
+    return np.array(sorted(pick), dtype=np.int32)
+
+
+def covered_tiles(tokens: np.ndarray, perm: np.ndarray, offsets: np.ndarray, k: int, tile: int) -> bool:
+    """True when every `tile`-row tile of every segment holds a task of `tokens`."""
+    chosen = np.zeros(len(perm), bool)
+    chosen[np.isin(perm // k, tokens)] = True
+    for e in range(len(offsets) - 1):
+        a, b = int(offsets[e]), int(offsets[e + 1])
+        for r0 in range(a, b, tile):
+            if not chosen[r0:min(b, r0 + tile)].any():
+                return False
+    return True
+
+
 def device_inputs(inp):
     return {k: dev(v) for k, v in inp.items()}
 
@@ -69,11 +107,17 @@ def layer_forward(cfg: W.MoEWorkload, d_in, ws=None, stream=None):
     w = torch.empty((T, k), dtype=torch.float32, device="cuda")
     counts = torch.empty((m,), dtype=torch.int32, device="cuda")
     lis = moe.lis_buffer()
+    offsets = torch.full((m + 1,), -7, dtype=torch.int32, device="cuda")
+    perm = torch.full((T * k,), -7, dtype=torch.int32, device="cuda")
+    inv_perm = torch.full((T * k,), -7, dtype=torch.int32, device="cuda")
+    x_perm = torch.empty((T * k, cfg.d), dtype=torch_dtype(cfg.dtype), device="cuda")
     moe.moe_layer_forward(c, d_in["x"], d_in["w_router"], d_in["bias"], d_in["w_gate"], d_in.get("w_up"),
                           d_in["w_down"], d_in.get("ws_gate"), d_in.get("ws_up"), d_in.get("ws_down"), out, ws,
                           logits_out=logits, topk_idx_out=idx, topk_w_out=w, counts_out=counts, lis_out=lis,
+                          offsets_out=offsets, perm_out=perm, inv_perm_out=inv_perm, x_perm_out=x_perm,
                           stream=stream)
-    return {"out": out, "logits": logits, "idx": idx, "w": w, "counts": counts, "lis": lis, "ws": ws}
+    return {"out": out, "logits": logits, "idx": idx, "w": w, "counts": counts, "lis": lis, "ws": ws,
+            "offsets": offsets, "perm": perm, "inv_perm": inv_perm, "x_perm": x_perm}
 
 
 def sample_tokens(idx: np.ndarray, counts: np.ndarray, T: int, n: int, seed: int = 0) -> np.ndarray:

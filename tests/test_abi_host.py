@@ -94,9 +94,14 @@ def test_calls_reject_bad_pointers_and_small_workspace_before_launch():
     # workspace too small / misaligned
     assert lib.moe_route(ctypes.byref(c), a, a, None, None, None, a, a, ok_ws, 16, None) == moe.ERR_WORKSPACE
     assert lib.moe_layer_forward(ctypes.byref(c), a, a, None, a, a, a, None, None, None, a, None, None, None, None,
-                                 None, _fake((1 << 20) + 16), 1 << 30, None) == moe.ERR_INVALID_ARG
+                                 None, None, None, None, None, _fake((1 << 20) + 16), 1 << 30, None) == \
+        moe.ERR_INVALID_ARG
     assert lib.moe_layer_forward(ctypes.byref(c), a, a, None, a, a, a, None, None, None, a, None, None, None, None,
-                                 None, ok_ws, 1024, None) == moe.ERR_WORKSPACE
+                                 None, None, None, None, None, ok_ws, 1024, None) == moe.ERR_WORKSPACE
+    # a misaligned inspection output (the permutation copies) is rejected too
+    assert lib.moe_layer_forward(ctypes.byref(c), a, a, None, a, a, a, None, None, None, a, None, None, None, None,
+                                 None, None, _fake((1 << 24) + 8), None, None, ok_ws, 1 << 30, None) == \
+        moe.ERR_INVALID_ARG
     # SwiGLU needs w_up
     assert lib.moe_grouped_ffn(ctypes.byref(c), a, a, a, None, a, None, None, a, ok_ws, 1 << 30, None) == \
         moe.ERR_INVALID_ARG

@@ -107,8 +107,10 @@ def _check_fp8(cfg, inp, tokens=None):
     toks = np.arange(cfg.T) if tokens is None else np.asarray(tokens)
     got = out_f64(r["out"])
     assert np.all(np.isfinite(got))
-    # -- stored h of every task of the checked tokens, and the output from it
+    # -- the permutation it ran on (bit-exact), then the stored h of every task of the
+    # checked tokens, and the output from it
     perm = host(r["perm"])
+    np.testing.assert_array_equal(perm, O.permutation(oidx, cfg.m, ref["offsets"])[0])
     row_of_task = np.empty(cfg.T * cfg.k, np.int64)
     row_of_task[perm] = np.arange(cfg.T * cfg.k)
     h_gpu = W.bf16_to_f32(host(r["h"]))

@@ -1,11 +1,13 @@
 """End-to-end parity of moe_layer_forward (the call the benchmark times) on every
 workload at full size, plus the atomic-expert variant.
 
-All tokens: top-k ids, counts, max/argmax and LIS bit-exact against the oracle
-deciding on the GPU's own fp32 logits. Outputs: every token for the small
-workloads; for the large ones a sample the oracle can evaluate token by token
-(always the first and last token and tokens of the most and least loaded
-experts), within the per-token relative tolerance.
+All tokens: top-k ids, counts, max/argmax, LIS, segment offsets, perm and
+inv_perm bit-exact against the oracle deciding on the GPU's own fp32 logits, and
+every permuted token row a bit copy of its token's row. Outputs: every token for
+the small workloads; for the large ones a sample the oracle can evaluate token by
+token that reaches every 128-row token tile of every expert segment (plus the
+first and last token and tokens of the most and least loaded experts), within the
+per-token relative tolerance; the elementwise figure is reported beside it.
 """
 import numpy as np
 import pytest
@@ -14,8 +16,8 @@ import torch
 import oracle as O
 import sparse_mixture_experts_08_b200 as moe
 import workloads as W
-from gpu_helpers import (GATE_RTOL, TOL, device_inputs, host, layer_forward, out_f64, require_gpu, sample_tokens,
-                         token_rel_err)
+from gpu_helpers import (GATE_RTOL, TOL, covered_tiles, device_inputs, err_report, host, layer_forward, out_f64,
+                         require_gpu, sample_tokens, tile_cover_tokens, token_rel_err)
 
 pytestmark = pytest.mark.gpu
 
@@ -38,13 +40,26 @@ def _check_layer(cfg, inp, n_sample):
     np.testing.assert_array_equal(counts, ref["counts"])
     mx, am, lis = moe.unpack_lis(r["lis"])
     assert (mx, am, lis) == (ref["max_count"], ref["argmax"], ref["lis"])
+    # the expert-centric permutation (OmniMoE Fig. 3), whichever routing path ran
+    np.testing.assert_array_equal(host(r["offsets"]), ref["offsets"])
+    operm, oinv = O.permutation(oidx, cfg.m, ref["offsets"])
+    perm = host(r["perm"])
+    np.testing.assert_array_equal(perm, operm)
+    np.testing.assert_array_equal(host(r["inv_perm"]), oinv)
+    x_perm = host(r["x_perm"])
+    assert np.array_equal(x_perm.view(np.uint32 if x_perm.dtype == np.float32 else np.uint16),
+                          inp["x"][operm // cfg.k].view(np.uint32 if x_perm.dtype == np.float32 else np.uint16))
     # float parity
-    toks = np.arange(cfg.T, dtype=np.int32) if n_sample >= cfg.T else sample_tokens(oidx, ref["counts"], cfg.T,
-                                                                                    n_sample)
+    if n_sample >= cfg.T:
+        toks = np.arange(cfg.T, dtype=np.int32)
+    else:
+        toks = np.union1d(sample_tokens(oidx, ref["counts"], cfg.T, n_sample),
+                          tile_cover_tokens(operm, ref["offsets"], cfg.k)).astype(np.int32)
+        assert covered_tiles(toks, operm, ref["offsets"], cfg.k, 128)
     exp = O.moe_output(cfg, inp, oidx, ow, tokens=toks)
     got = out_f64(r["out"])[toks]
     err = token_rel_err(got, exp)
-    assert err <= TOL[cfg.dtype], f"max per-token relative error {err:.3e}"
+    assert err <= TOL[cfg.dtype], err_report(got, exp)
     assert np.all(np.isfinite(out_f64(r["out"])))
     return ref, err
 
