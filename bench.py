@@ -10,6 +10,11 @@ parallel: every rank holds the same expert weights and its own token batch, no
 collective touches the data path (weak scaling); the timing barrier and the
 max-over-ranks reduction are the only collectives.
 
+The headline workload is the Mixtral-8x7B-shaped prefill layer (--config picks
+another). On one GPU without a variant flag the line also carries the decode and
+Switch-style layers under "workloads" (each timed for over a second) and the
+headline layer timed again for over a second under "sustained".
+
 Prints ONE JSON line on rank 0. `value` = tokens/s of the whole job from CUDA
 events on the launching stream (L2 flushed between steps, outside the timed
 events); `e2e` = the same metric through the C-ABI call with the batch copied
@@ -44,7 +49,14 @@ METRIC = "MoE-layer tokens/sec at 1 B200; grouped-GEMM TFLOPS and HBM GB/s as % 
 UNIT = "tokens/s"
 STAGES = ["router", "topk", "histogram_lis_ranks", "permute", "expert_up", "expert_down", "combine"]
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+NOMINAL_BF16_TFLOPS = 2250.0  # B200 dense bf16 tensor-core rate from the spec sheet (context beside the measured peak)
 L2_FLUSH_BYTES = 256 << 20
+# Workloads timed beside the headline one (single-GPU runs without a variant flag), each
+# for at least EXTRA_MIN_MS of device time; the headline workload is timed again for
+# SUSTAINED_MS when its K steps are shorter than that.
+EXTRA_WORKLOADS = ["decode", "switch"]
+EXTRA_MIN_MS = 1200.0
+SUSTAINED_MS = 1500.0
 
 
 def parse():
@@ -52,10 +64,14 @@ def parse():
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=10)
-    ap.add_argument("--config", default="switch", choices=list(W.CONFIGS))
+    ap.add_argument("--config", default="mixtral", choices=list(W.CONFIGS),
+                    help="workload of the headline line (default: the Mixtral-shaped prefill, the largest "
+                         "single-GPU configuration)")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--cpu-seconds", type=float, default=12.0, help="CPU-oracle baseline budget (rank 0, N=1)")
     ap.add_argument("--no-cpu-baseline", action="store_true", help="skip the CPU-oracle leg (for profiling runs)")
+    ap.add_argument("--no-extra", action="store_true",
+                    help="time only the selected workload (no decode / switch keys, no sustained run)")
     ap.add_argument("--replicate", action="store_true",
                     help="R&Q replica dispatch: time moe_layer_forward_replicated (heavy-hitter split alternately "
                          "with a replica expert m) instead of moe_layer_forward")
@@ -379,23 +395,68 @@ def traffic_for(workload: str, stage: str):
 
 # ------------------------------------------------------------------ our arm
 
-def ours(args):
+def _down_ksplit(cfg, cfg_groups, fp8: bool) -> int:
+    """The library's static down-projection K split (mirrors its planner; it only
+    enters the byte count of the fp32 partial outputs)."""
+    plan_ksplit = 1
+    if cfg.dtype == W.BF16 and cfg.n_shared == 0:
+        avg = cfg.T * cfg.k / cfg_groups.m
+        bn, cap = 16, (256 if avg >= 256 else 128)  # the library's down-projection tile rule
+        while bn < cap and bn < 2.0 * avg:
+            bn <<= 1
+        tiles = min(cfg_groups.m, cfg.T * cfg.k) * ((cfg.d + 127) // 128) * max(1, math.ceil(avg / bn))
+        if tiles < 4 * 148:
+            kb = (cfg.f + 63) // 64
+            ks = min(16, -(-4 * 148 // tiles), kb)
+            kbps = -(-kb // ks)
+            plan_ksplit = -(-kb // kbps)
+            if fp8:  # the same split re-cut into 128-element k-blocks
+                kb8 = (cfg.f + 127) // 128
+                ks8 = min(plan_ksplit, kb8)
+                plan_ksplit = -(-kb8 // -(-kb8 // ks8))
+    return plan_ksplit
+
+
+def roofline_for(cfg, stage: str, fl: float, by: float, dom_ms: float, pk: dict, pk_src: str, long_step: bool,
+                 fp8: bool, traffic_key: str) -> dict:
+    """Roofline object of one kernel: algorithmic flops / bytes per launch over its
+    event-timed duration, against the measured peaks; a contraction also states its
+    fraction of the nominal dense tensor-core rate (2.25 PFLOP/s bf16, 4.5 E4M3)."""
+    sec = dom_ms * 1e-3
+    tensor_peak = pk["bf16_tflops_sustained"] if long_step else pk["bf16_tflops"]
+    nominal = NOMINAL_BF16_TFLOPS
+    if fp8:  # E4M3 contraction: the measured bf16 peak times the nominal dense fp8 / bf16 ratio (4.5 / 2.25)
+        tensor_peak *= 2.0
+        nominal *= 2.0
+    ridge = tensor_peak * 1e12 / (pk["hbm_gbs"] * 1e9)
+    if fl > 0 and fl / max(by, 1.0) > ridge and cfg.dtype == W.BF16:
+        roof = {"bound": "tensor", "achieved": fl / sec / 1e12, "peak": tensor_peak, "unit": "TFLOP/s"}
+        roof["peak_source"] = (f"{pk_src} bf16 ({'sustained' if long_step else 'burst'})"
+                               + (" x 2 (nominal fp8 / bf16 dense ratio)" if fp8 else ""))
+        roof["frac_of_nominal_dense"] = roof["achieved"] / nominal
+        roof["nominal_dense_tflops"] = nominal
+    else:
+        roof = {"bound": "hbm", "achieved": by / sec / 1e9, "peak": pk["hbm_gbs"], "unit": "GB/s",
+                "peak_source": f"{pk_src} hbm copy"}
+    roof["frac"] = roof["achieved"] / roof["peak"]
+    roof["traffic"] = traffic_for(traffic_key, stage)
+    roof["kernel"] = stage
+    roof["algorithmic_bytes"] = by
+    roof["algorithmic_flops"] = fl
+    roof["duration_us"] = dom_ms * 1e3
+    return roof
+
+
+def layer_run(cfg, args, dev, rank: int, world: int, dist, steps, warmup: int, with_e2e: bool,
+              min_timed_ms: float = 0.0, sustained_ms: float = 0.0):
+    """Everything measured for one coarse-expert workload: warm-up, the per-stage
+    pass, `steps` timed steps (None: enough steps for min_timed_ms of device time),
+    optionally a second, longer timed run (sustained_ms) and the end-to-end leg.
+    Returns a dict of results; rank 0's line is built from it by the caller."""
     import torch
-    import torch.distributed as dist
 
     import sparse_mixture_experts_08_b200 as moe
 
-    rank = int(os.environ.get("RANK", "0"))
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    local = int(os.environ.get("LOCAL_RANK", "0"))
-    if world != args.gpus:
-        raise SystemExit(f"--gpus {args.gpus} needs {args.gpus} ranks (torchrun), found WORLD_SIZE={world}")
-    torch.cuda.set_device(local)
-    dev = torch.device("cuda", local)
-    if world > 1:
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=180), device_id=dev)
-
-    cfg = W.CONFIGS[args.config]
     inp = rank_inputs(cfg, rank)
 
     def to_dev(a):
@@ -472,7 +533,7 @@ def ours(args):
         n0 = moe.moe_launch_count()
         fwd()
         launches_per_step = moe.moe_launch_count() - n0
-        for _ in range(max(args.warmup, 3)):
+        for _ in range(max(warmup, 3)):
             flush.zero_()
             fwd()
     torch.cuda.synchronize(dev)
@@ -493,7 +554,7 @@ def ours(args):
     # ---- profiling pass (untimed): every stage boundary gets an event, which
     # serialises the kernels; it gives the per-kernel breakdown and picks the
     # dominant kernel, whose boundaries alone are then recorded in the timed region.
-    Kp = max(3, min(args.steps, 50))
+    Kp = max(3, min(steps if steps else 50, 50))
     ev_prof = [[torch.cuda.Event(enable_timing=True) for _ in range(8)] for _ in range(Kp)]
     with torch.cuda.stream(s):  # torch creates the CUDA events on first record
         for evs in ev_prof:
@@ -507,6 +568,7 @@ def ours(args):
     moe.moe_set_stage_events([])
     stage_ms = {name: sum(ev_prof[i][j].elapsed_time(ev_prof[i][j + 1]) for i in range(Kp)) / Kp
                 for j, name in enumerate(STAGES)}
+    prof_step_ms = sum(ev_prof[i][0].elapsed_time(ev_prof[i][7]) for i in range(Kp)) / Kp
     dom = max(STAGES, key=lambda n: stage_ms[n])
     jd = STAGES.index(dom)
     if fused_routing(cfg) and not rep:
@@ -514,83 +576,75 @@ def ours(args):
         stage_ms = {("router_topk_ranks" if n == "router" else "scatter" if n == "permute" else n): v
                     for n, v in stage_ms.items() if n not in ("topk", "histogram_lis_ranks")}
         dom = {"router": "router_topk_ranks", "permute": "scatter"}.get(dom, dom)
+    K = steps if steps else max(3, int(math.ceil(min_timed_ms / max(prof_step_ms, 1e-3))))
 
-    # ---- timed region: K steps, CUDA events on the launching stream, L2 flushed between steps
-    K = args.steps
-    ev_s = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
-    ev_e = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
-    ev_dom = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(K)]
-    with torch.cuda.stream(s):
-        for evs in ev_dom:
-            for e in evs:
-                e.record(s)
-    sampler = ClockSampler(local)
-    if world > 1:
-        dist.barrier()
-    torch.cuda.synchronize(dev)
-    sampler.start()
-    with torch.cuda.stream(s):
-        for i in range(K):
-            flush.zero_()
-            hook = [None] * 8
-            hook[jd], hook[jd + 1] = ev_dom[i][0], ev_dom[i][1]
-            moe.moe_set_stage_events(hook)
-            ev_s[i].record(s)
-            fwd()
-            ev_e[i].record(s)
-    torch.cuda.synchronize(dev)
-    if world > 1:
-        dist.barrier()
-    sampler.stop()
-    moe.moe_set_stage_events([])
-    step_ms = [ev_s[i].elapsed_time(ev_e[i]) for i in range(K)]
-    dom_ms = sum(ev_dom[i][0].elapsed_time(ev_dom[i][1]) for i in range(K)) / K
-    ms_local = sum(step_ms) / K
-    st = moe.moe_read_device_status(ws, stream=s)
-    if st != moe.OK:
-        raise RuntimeError(f"device status after the timed steps: {moe.moe_status_string(st)}")
+    def timed(nsteps):
+        """nsteps steps, CUDA events on the launching stream, L2 flushed between steps;
+        returns (mean step ms, mean dominant-kernel ms, clock report)."""
+        ev_s = [torch.cuda.Event(enable_timing=True) for _ in range(nsteps)]
+        ev_e = [torch.cuda.Event(enable_timing=True) for _ in range(nsteps)]
+        ev_dom = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(nsteps)]
+        with torch.cuda.stream(s):
+            for evs in ev_dom:
+                for e in evs:
+                    e.record(s)
+        sampler = ClockSampler(dev.index)
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize(dev)
+        sampler.start()
+        with torch.cuda.stream(s):
+            for i in range(nsteps):
+                flush.zero_()
+                hook = [None] * 8
+                hook[jd], hook[jd + 1] = ev_dom[i][0], ev_dom[i][1]
+                moe.moe_set_stage_events(hook)
+                ev_s[i].record(s)
+                fwd()
+                ev_e[i].record(s)
+        torch.cuda.synchronize(dev)
+        if world > 1:
+            dist.barrier()
+        sampler.stop()
+        moe.moe_set_stage_events([])
+        ms_ = sum(ev_s[i].elapsed_time(ev_e[i]) for i in range(nsteps)) / nsteps
+        dom_ = sum(ev_dom[i][0].elapsed_time(ev_dom[i][1]) for i in range(nsteps)) / nsteps
+        st_ = moe.moe_read_device_status(ws, stream=s)
+        if st_ != moe.OK:
+            raise RuntimeError(f"device status after the timed steps: {moe.moe_status_string(st_)}")
+        return ms_, dom_, sampler.report()
 
-    # ---- end to end through the C ABI: pinned host batch in, result out, every step
-    raw = (lambda t: t.view(torch.int16)) if tdt == torch.bfloat16 else (lambda t: t)
-    x_host = torch.from_numpy(inp["x"].view(np.int16) if inp["x"].dtype == np.uint16 else inp["x"]).pin_memory()
-    out_hosts = [torch.empty(out.shape, dtype=torch.int16 if tdt == torch.bfloat16 else torch.float32).pin_memory()
-                 for _ in range(2)]
-    x_devs = [raw(torch.empty_like(d_in["x"])) for _ in range(2)]
-    out_devs = [torch.empty_like(out) for _ in range(2)]
-    Ke = max(3, min(K, 100))
-    if world > 1:
-        dist.barrier()
-    # the C ABI takes raw device pointers, so bf16 buffers travel as int16 views
-    e2e_local = e2e_pipelined(torch, lambda xd, od: fwd(x=xd, o=od), x_host, x_devs, [raw(o) for o in out_devs],
-                              out_hosts, Ke, s, dev)
-    if world > 1:
-        dist.barrier()
-    h2d = x_host.numel() * x_host.element_size()
-    d2h = out_hosts[0].numel() * out_hosts[0].element_size()
+    ms_local, dom_ms, clocks = timed(K)
+    sustained = None
+    if sustained_ms > 0 and K * ms_local < sustained_ms:
+        Ks = int(math.ceil(sustained_ms / max(ms_local, 1e-3)))
+        s_ms, s_dom, s_clocks = timed(Ks)
+        sustained = {"steps": Ks, "ms_per_step": s_ms, "dom_ms": s_dom, "clocks": s_clocks}
 
-    # ---- max over ranks
-    ms, e2e_ms = max_over_ranks([ms_local, e2e_local], dist, dev)
+    e2e = None
+    if with_e2e:
+        # ---- end to end through the C ABI: pinned host batch in, result out, every step
+        raw = (lambda t: t.view(torch.int16)) if tdt == torch.bfloat16 else (lambda t: t)
+        x_host = torch.from_numpy(inp["x"].view(np.int16) if inp["x"].dtype == np.uint16 else inp["x"]).pin_memory()
+        out_hosts = [torch.empty(out.shape, dtype=torch.int16 if tdt == torch.bfloat16 else torch.float32)
+                     .pin_memory() for _ in range(2)]
+        x_devs = [raw(torch.empty_like(d_in["x"])) for _ in range(2)]
+        out_devs = [torch.empty_like(out) for _ in range(2)]
+        Ke = max(3, min(K, 100))
+        if world > 1:
+            dist.barrier()
+        # the C ABI takes raw device pointers, so bf16 buffers travel as int16 views
+        e2e_local = e2e_pipelined(torch, lambda xd, od: fwd(x=xd, o=od), x_host, x_devs, [raw(o) for o in out_devs],
+                                  out_hosts, Ke, s, dev)
+        if world > 1:
+            dist.barrier()
+        e2e = {"ms_local": e2e_local, "h2d": x_host.numel() * x_host.element_size(),
+               "d2h": out_hosts[0].numel() * out_hosts[0].element_size()}
 
-    pk, pk_src = peaks()
     cfg_groups = dataclasses.replace(cfg, m=cfg.m + 1) if rep else cfg  # the replica is one more routed group
-    plan_ksplit = 1
-    if cfg.dtype == W.BF16 and cfg.n_shared == 0:
-        # the library's static down-projection split (mirrors its planner; only affects the byte count)
-        avg = cfg.T * cfg.k / cfg_groups.m
-        bn, cap = 16, (256 if avg >= 256 else 128)  # the library's down-projection tile rule
-        while bn < cap and bn < 2.0 * avg:
-            bn <<= 1
-        tiles = min(cfg_groups.m, cfg.T * cfg.k) * ((cfg.d + 127) // 128) * max(1, math.ceil(avg / bn))
-        if tiles < 4 * 148:
-            kb = (cfg.f + 63) // 64
-            ks = min(16, -(-4 * 148 // tiles), kb)
-            kbps = -(-kb // ks)
-            plan_ksplit = -(-kb // kbps)
-            if fp8:  # the same split re-cut into 128-element k-blocks
-                kb8 = (cfg.f + 127) // 128
-                ks8 = min(plan_ksplit, kb8)
-                plan_ksplit = -(-kb8 // -(-kb8 // ks8))
+    plan_ksplit = _down_ksplit(cfg, cfg_groups, fp8)
     costs, layer_flops, layer_bytes = stage_costs(cfg_groups, active, plan_ksplit, weight_bytes=1 if fp8 else None)
+    extra = {}
     if floe is not None:
         # dense up projection: W_up only, u written in fp32; sparse part: the gate and
         # down rows of the kept channels, u and the compact h
@@ -600,28 +654,80 @@ def ours(args):
         costs["expert_down"] = (4.0 * cfg.d * float(kc.sum()) * max(1.0, Tk / max(active, 1)),
                                 float(kc.sum()) * 2 * cfg.d * 2 + Tk * cfg.f * 8 + Tk * cfg.d * 4)
         layer_bytes = (cfg.m * cfg.d + active * cfg.f * cfg.d + float(kc.sum()) * 2 * cfg.d) * 2 + 2 * T_bytes(cfg)
-    fl, by = costs[dom]
-    sec = dom_ms * 1e-3
-    long_step = K * ms > 1000.0
-    tensor_peak = pk["bf16_tflops_sustained"] if long_step else pk["bf16_tflops"]
-    if fp8:  # E4M3 contraction: the measured bf16 peak times the nominal dense fp8 / bf16 ratio (4.5 / 2.25)
-        tensor_peak *= 2.0
-    ridge = tensor_peak * 1e12 / (pk["hbm_gbs"] * 1e9)
-    if fl > 0 and fl / max(by, 1.0) > ridge and cfg.dtype == W.BF16:
-        roof = {"bound": "tensor", "achieved": fl / sec / 1e12, "peak": tensor_peak, "unit": "TFLOP/s"}
-        roof["peak_source"] = (f"{pk_src} bf16 ({'sustained' if long_step else 'burst'})"
-                               + (" x 2 (nominal fp8 / bf16 dense ratio)" if fp8 else ""))
-    else:
-        roof = {"bound": "hbm", "achieved": by / sec / 1e9, "peak": pk["hbm_gbs"], "unit": "GB/s",
-                "peak_source": f"{pk_src} hbm copy"}
-    roof["frac"] = roof["achieved"] / roof["peak"]
-    roof["traffic"] = traffic_for(cfg.name + ("_fp8" if fp8 else ""), dom)
-    roof["kernel"] = dom
-    roof["algorithmic_bytes"] = by
-    roof["algorithmic_flops"] = fl
-    roof["duration_us"] = dom_ms * 1e3
-    t_layer = max(layer_flops / (tensor_peak * 1e12), layer_bytes / (pk["hbm_gbs"] * 1e9))
+        extra["kept_channel_fraction"] = float(kc[kc > 0].mean() / cfg.f)
+    if rep:
+        extra["lis_before_split"] = moe.unpack_lis(lis0)[2]
+        extra["heavy_hitter_before_split"] = moe.unpack_lis(lis0)[1]
+    return {"K": K, "Kp": Kp, "ms_local": ms_local, "dom": dom, "dom_ms": dom_ms, "clocks": clocks,
+            "sustained": sustained, "e2e": e2e, "stage_ms": stage_ms, "costs": costs, "layer_flops": layer_flops,
+            "layer_bytes": layer_bytes, "launches_per_step": launches_per_step, "inp": inp, "fp8": fp8,
+            "routing": {"lis": lis_v, "max_count": max_count, "heavy_hitter": argmax, "active_experts": active,
+                        "reuse_ratio": cfg.T * cfg.k / max(active, 1), "load_entropy": entropy},
+            "extra": extra}
 
+
+def workload_summary(cfg, r: dict, world: int) -> dict:
+    """A workload measured beside the headline one: its own step time, tokens/s,
+    dominant-kernel roofline (against the peak its timed length calls for), layer
+    roofline, stage breakdown, routing statistics and clocks."""
+    pk, pk_src = peaks()
+    ms = r["ms_local"]
+    long_step = r["K"] * ms > 1000.0
+    fl, by = r["costs"][r["dom"]]
+    roof = roofline_for(cfg, r["dom"], fl, by, r["dom_ms"], pk, pk_src, long_step, r["fp8"],
+                        cfg.name + ("_fp8" if r["fp8"] else ""))
+    tensor_peak = (pk["bf16_tflops_sustained"] if long_step else pk["bf16_tflops"]) * (2.0 if r["fp8"] else 1.0)
+    t_layer = max(r["layer_flops"] / (tensor_peak * 1e12), r["layer_bytes"] / (pk["hbm_gbs"] * 1e9))
+    return {"config": workload_config(cfg), "value": world * cfg.T / (ms * 1e-3), "unit": UNIT, "steps": r["K"],
+            "ms_per_step": ms, "timed_region_ms": r["K"] * ms, "roofline": roof,
+            "layer_roofline": {"time_us": t_layer * 1e6, "frac": t_layer / (ms * 1e-3), "flops": r["layer_flops"],
+                               "bytes": r["layer_bytes"]},
+            "stages_us": {k: v * 1e3 for k, v in r["stage_ms"].items()}, "routing": r["routing"],
+            "gpu_launches": r["K"] * r["launches_per_step"], "clocks": r["clocks"]}
+
+
+def ours(args):
+    import torch
+    import torch.distributed as dist
+
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world != args.gpus:
+        raise SystemExit(f"--gpus {args.gpus} needs {args.gpus} ranks (torchrun), found WORLD_SIZE={world}")
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=180), device_id=dev)
+
+    cfg = W.CONFIGS[args.config]
+    rep, floe, fp8 = args.replicate, args.floe, args.fp8
+    variant = rep or floe is not None or fp8
+    r = layer_run(cfg, args, dev, rank, world, dist, args.steps, args.warmup, with_e2e=True,
+                  sustained_ms=SUSTAINED_MS if (world == 1 and not variant and not args.no_extra) else 0.0)
+    # ---- max over ranks
+    ms, e2e_ms = max_over_ranks([r["ms_local"], r["e2e"]["ms_local"]], dist, dev)
+    K = r["K"]
+    pk, pk_src = peaks()
+    long_step = K * ms > 1000.0
+    fl, by = r["costs"][r["dom"]]
+    roof = roofline_for(cfg, r["dom"], fl, by, r["dom_ms"], pk, pk_src, long_step, fp8,
+                        cfg.name + ("_fp8" if fp8 else ""))
+    tensor_peak = (pk["bf16_tflops_sustained"] if long_step else pk["bf16_tflops"]) * (2.0 if fp8 else 1.0)
+    t_layer = max(r["layer_flops"] / (tensor_peak * 1e12), r["layer_bytes"] / (pk["hbm_gbs"] * 1e9))
+    variant_note = {}
+    if floe is not None:
+        variant_note = {"variant": f"FloE contextual sparsity at target sparsity {floe}: thresholds from a second "
+                                   "batch; expert_up = dense u = x W_up^T, expert_down = kept lists + kept gate rows + "
+                                   "kept down rows"}
+    elif fp8:
+        variant_note = {"variant": "8-bit experts: E4M3 weights with one fp32 scale per output channel (quantized "
+                                   "once, outside the timing); x and h rows quantized per row inside each step; router "
+                                   "in bf16",
+                        "dtype_note": "expert GEMMs e4m3 x e4m3 with fp32 accumulation; router bf16"}
+    elif rep:
+        variant_note = {"variant": "R&Q replica dispatch: the heavy-hitter's tasks alternate between it and a replica "
+                                   "expert m that computes with its bf16 weights; routing.lis is over the m + 1 experts"}
     line = {"metric": METRIC, "value": world * cfg.T / (ms * 1e-3), "unit": UNIT, "n_gpus": world, "steps": K,
             "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "e4m3" if fp8 else "bf16" if cfg.dtype == W.BF16 else "f32",
@@ -632,30 +738,44 @@ def ours(args):
                            launch="eager C-ABI call per step"),
             "roofline": roof,
             "layer_roofline": {"time_us": t_layer * 1e6, "frac": t_layer / (ms * 1e-3),
-                               "flops": layer_flops, "bytes": layer_bytes},
-            "stages_us": {k: v * 1e3 for k, v in stage_ms.items()},
-            "stages_note": f"per-kernel breakdown from a separate {Kp}-step pass with an event at every stage "
+                               "flops": r["layer_flops"], "bytes": r["layer_bytes"]},
+            "stages_us": {k: v * 1e3 for k, v in r["stage_ms"].items()},
+            "stages_note": f"per-kernel breakdown from a separate {r['Kp']}-step pass with an event at every stage "
                            "boundary (serialised launches); the timed region records only the dominant kernel's "
                            "boundaries",
-            "routing": {"lis": lis_v, "max_count": max_count, "heavy_hitter": argmax, "active_experts": active,
-                        "reuse_ratio": cfg.T * cfg.k / max(active, 1), "load_entropy": entropy},
-            **({"variant": f"FloE contextual sparsity at target sparsity {floe}: thresholds from a second batch; "
-                           "expert_up = dense u = x W_up^T, expert_down = kept lists + kept gate rows + kept down rows",
-                "kept_channel_fraction": float(kept.cpu().numpy()[kept.cpu().numpy() > 0].mean() / cfg.f)}
-               if floe is not None else {}),
-            **({"variant": "8-bit experts: E4M3 weights with one fp32 scale per output channel (quantized once, "
-                           "outside the timing); x and h rows quantized per row inside each step; router in bf16",
-                "dtype_note": "expert GEMMs e4m3 x e4m3 with fp32 accumulation; router bf16"} if fp8 else {}),
-            **({"variant": "R&Q replica dispatch: the heavy-hitter's tasks alternate between it and a replica "
-                           "expert m that computes with its bf16 weights; routing.lis is over the m + 1 experts",
-                "lis_before_split": moe.unpack_lis(lis0)[2],
-                "heavy_hitter_before_split": moe.unpack_lis(lis0)[1]} if rep else {}),
-            "e2e": {"value": world * cfg.T / (e2e_ms * 1e-3), "unit": UNIT, "h2d_bytes_per_step": h2d,
-                    "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms,
+            "routing": r["routing"], **variant_note, **r["extra"],
+            "e2e": {"value": world * cfg.T / (e2e_ms * 1e-3), "unit": UNIT, "h2d_bytes_per_step": r["e2e"]["h2d"],
+                    "d2h_bytes_per_step": r["e2e"]["d2h"], "ms_per_step": e2e_ms,
                     "note": "pinned host -> device batch upload and device -> host output download every step, on "
                             "their own streams, overlapped with the neighbouring steps' forward (double-buffered)"},
-            "gpu_launches": K * launches_per_step, "launches_per_step": launches_per_step,
-            "clocks": sampler.report()}
+            "gpu_launches": K * r["launches_per_step"], "launches_per_step": r["launches_per_step"],
+            "clocks": r["clocks"]}
+    if r["sustained"] is not None:
+        su = r["sustained"]
+        roof_s = roofline_for(cfg, r["dom"], fl, by, su["dom_ms"], pk, pk_src, True, fp8, cfg.name)
+        line["sustained"] = {"steps": su["steps"], "ms_per_step": su["ms_per_step"],
+                             "value": cfg.T / (su["ms_per_step"] * 1e-3), "unit": UNIT,
+                             "timed_region_ms": su["steps"] * su["ms_per_step"], "roofline": roof_s,
+                             "clocks": su["clocks"],
+                             "note": "the same workload timed again for over a second after the headline steps, so "
+                                     "the clocks settle under the power cap; its roofline uses the sustained peak"}
+    inp = r["inp"]
+    del r
+    if world == 1 and not variant and not args.no_extra:
+        # the other single-GPU workloads the targets name, each timed long enough for
+        # the clock sampler to see a steady state
+        torch.cuda.empty_cache()
+        extras = {}
+        for name in EXTRA_WORKLOADS:
+            if name == cfg.name:
+                continue
+            xc = W.CONFIGS[name]
+            rx = layer_run(xc, args, dev, rank, world, dist, None, args.warmup, with_e2e=False,
+                           min_timed_ms=EXTRA_MIN_MS)
+            extras[name] = workload_summary(xc, rx, world)
+            del rx
+            torch.cuda.empty_cache()
+        line["workloads"] = extras
     if world > 1:
         dist.barrier()
     if rank == 0:
