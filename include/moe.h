@@ -339,10 +339,10 @@ MOE_API moe_status_t moe_atomic_forward(const moe_atomic_config_t* cfg, const vo
                                 void* ws, size_t ws_bytes, moe_stream_t stream);
 
 /* moe_route without a workspace, for callers that cannot allocate device memory:
- * code running while a CUDA graph is captured (cudaMalloc is not allowed then),
- * plugins that only see the tensors a host framework hands them, or request paths
- * that must not allocate. (The reviewed pages have no counterpart: this is a
- * deployment convenience, not part of the method.) Same arguments and results as
+ * plugins that only see the tensors a host framework hands them (the framework
+ * owns the allocator), or request paths that must not allocate (an allocation can
+ * block or fail under memory pressure). (The reviewed pages have no counterpart:
+ * this is a deployment convenience, not part of the method.) Same arguments and results as
  * moe_route, except that the status word and - when neither logits_in nor
  * logits_out is given - the router logits live in an 8 MiB array compiled into
  * the library, held on every GPU that loads it until the process exits. It
@@ -368,6 +368,14 @@ MOE_API const char* moe_status_string(moe_status_t status);
  * tensor-core kernels launched after this call (0 restores the default of 2 s).
  * Not thread-safe; meant for fault-injection tests. */
 MOE_API moe_status_t moe_debug_set_wait_limit_ns(uint64_t ns);
+
+/* Test hook: the grid-wide barrier of the decode-budget atomic-expert kernel
+ * (moe_atomic_experts / moe_atomic_forward with T K < 16384) waits for n arrivals
+ * more than its grid has, so with n > 0 it can only end at the bounded wait's
+ * time limit: the kernel then records MOE_ERR_TIMEOUT and its blocks return
+ * without the assembly phase. 0 (the default) restores the normal barrier. Not
+ * thread-safe; meant for fault-injection tests. */
+MOE_API moe_status_t moe_debug_set_barrier_extra(uint32_t n);
 
 /* Profiling hook: when n > 0, every later moe_layer_forward records the n
  * cudaEvent_t handles in `events` (host array, caller-owned events) on its

@@ -176,13 +176,15 @@ static moe_status_t cuda_status(cudaError_t e) { return e == cudaSuccess ? MOE_O
 
 // ------------------------------------------------------------------ building blocks
 
-static moe_status_t run_router(const moe_config_t& c, const void* x, const void* w_r, const float* bias, float* logits,
-                               int* status, cudaStream_t s) {
+unsigned long long wait_limit_ns() { return g_wait_limit_ns; }
+
+// Router logits (x W_r^T + bias, fp32) into `logits`, by the kernel that suits the
+// batch; shared by the workspace entry points and moe_route_static.
+cudaError_t launch_router_logits(const moe_config_t& c, const void* x, const void* w_r, const float* bias,
+                                 float* logits, int* status, cudaStream_t s) {
   // Batches too small to fill the tensor cores (decode) and fp32 layers use CUDA cores.
-  if (few_expert_logits_ok(c.dtype, c.T, c.m))
-    return cuda_status(launch_few_expert_logits(c.T, c.d, c.m, x, w_r, bias, logits, s));
-  if (c.dtype == MOE_F32 || c.T <= 64)
-    return cuda_status(launch_simt_logits(c.dtype, c.T, c.d, c.m, x, w_r, bias, logits, s));
+  if (few_expert_logits_ok(c.dtype, c.T, c.m)) return launch_few_expert_logits(c.T, c.d, c.m, x, w_r, bias, logits, s);
+  if (c.dtype == MOE_F32 || c.T <= 64) return launch_simt_logits(c.dtype, c.T, c.d, c.m, x, w_r, bias, logits, s);
   // logits^T = W_r . x^T on the tensor cores: one group, features = experts.
   GemmParams p;
   std::memset(&p, 0, sizeof(p));
@@ -211,7 +213,12 @@ static moe_status_t run_router(const moe_config_t& c, const void* x, const void*
   maps.b[0] = {x, c.T, c.d};
   const long long tiles = mt * ((c.T + bn - 1) / bn);
   const int ctas = (int)std::min<long long>(tiles, num_sms());
-  return cuda_status(launch_tc_gemm(EPI_LOGITS, bn, maps, p, ctas, s));
+  return launch_tc_gemm(EPI_LOGITS, bn, maps, p, ctas, s);
+}
+
+static moe_status_t run_router(const moe_config_t& c, const void* x, const void* w_r, const float* bias, float* logits,
+                               int* status, cudaStream_t s) {
+  return cuda_status(launch_router_logits(c, x, w_r, bias, logits, status, s));
 }
 
 // 8-bit expert path: the quantized weights and the per-row codes and scales of
@@ -1250,6 +1257,11 @@ const char* moe_status_string(moe_status_t s) {
 
 moe_status_t moe_debug_set_wait_limit_ns(uint64_t ns) {
   g_wait_limit_ns = ns ? (unsigned long long)ns : 2000ull * 1000 * 1000;
+  return MOE_OK;
+}
+
+moe_status_t moe_debug_set_barrier_extra(uint32_t n) {
+  set_grid_barrier_extra(n);
   return MOE_OK;
 }
 

@@ -696,7 +696,8 @@ constexpr int ASM_GROUPS = 4, ASM_BATCH = 16;  // phase 2: slot groups per 8 col
 //    fp32 FMAs over each lane's 16-byte chunks in ascending order then a shuffle
 //    tree; when all gathered w_out rows fit comfortably in L2 (decode budgets) the
 //    warp also prefetches the task's w_out row for phase 2;
-//  a grid-wide barrier (bounded: on expiry it records MOE_ERR_TIMEOUT and carries on);
+//  a grid-wide barrier (bounded: on expiry the block records MOE_ERR_TIMEOUT and
+//    returns without phase 2, whose coefficients other blocks may not have written);
 //  phase 2, four lanes per 8 output columns: lane group j sums slots j, j + 4, ...
 //    in order, and out[t, c..c+7] = ((group 0 + group 1) + group 2) + group 3,
 //    rounded to bf16, so the result is the same on every run.
@@ -748,8 +749,8 @@ __global__ void __launch_bounds__(AX_THREADS)
     atomic_experts_kernel(int T, int d, int K, int act, const uint4* __restrict__ x, const uint4* __restrict__ w_in,
                           const uint4* __restrict__ w_out, const int32_t* __restrict__ idx,
                           const float* __restrict__ g, float* __restrict__ coef, uint4* __restrict__ out,
-                          long long n_experts, int prefetch_out, unsigned* bar, unsigned long long limit_ns,
-                          int* status) {
+                          long long n_experts, int prefetch_out, unsigned* bar, unsigned bar_extra,
+                          unsigned long long limit_ns, int* status) {
   pdl_launch_dependents();
   pdl_wait();
   const int lane = threadIdx.x & 31;
@@ -775,21 +776,28 @@ __global__ void __launch_bounds__(AX_THREADS)
     const float z = warp_dot_bf16(x + t * chunks, w_in + e * chunks, chunks, lane);
     if (lane == 0) coef[task] = g[task] * atomic_act(z, act);
   }
-  // ---- grid-wide barrier (every block is resident: cooperative launch, one per SM)
+  // ---- grid-wide barrier (every block is resident: cooperative launch, one per SM).
+  // It waits for gridDim.x + bar_extra arrivals; bar_extra is 0 except under the
+  // fault-injection hook, where the wait can only end at its time limit.
+  __shared__ int bar_failed;
   __syncthreads();
   if (threadIdx.x == 0) {
+    bar_failed = 0;
     __threadfence();
     atomicAdd(bar, 1u);
+    const unsigned target = gridDim.x + bar_extra;
     const unsigned long long t0 = globaltimer_ns();
-    while (*reinterpret_cast<volatile unsigned*>(bar) < gridDim.x) {
+    while (*reinterpret_cast<volatile unsigned*>(bar) < target) {
       if (globaltimer_ns() - t0 > limit_ns) {
         set_status(status, MOE_ERR_TIMEOUT);
+        bar_failed = 1;
         break;
       }
     }
     __threadfence();
   }
   __syncthreads();
+  if (bar_failed) return;
   // ---- phase 2: out[t, c..c+7] = sum_s coef[t, s] w_out[idx[t, s], c..c+7]
   const long long units4 = (long long)T * chunks * ASM_GROUPS;
   for (long long qb = gwarp * 32; qb < units4; qb += nwarps * 32) {  // warp-aligned: shuffles see all lanes
@@ -1036,6 +1044,9 @@ __global__ void __launch_bounds__(AW_THREADS)
   }
 }
 
+static unsigned g_barrier_extra = 0;
+void set_grid_barrier_extra(unsigned n) { g_barrier_extra = n; }
+
 cudaError_t launch_atomic_experts(int T, int d, int K, int act, const void* x, const void* w_in, const void* w_out,
                                   const int32_t* idx, const float* g, float* coef, void* out, long long n_experts,
                                   unsigned* bar, bool bar_zeroed, unsigned long long limit_ns, int* status,
@@ -1105,7 +1116,7 @@ cudaError_t launch_atomic_experts_sorted(int T, int d, int K, int act, const voi
   const int prefetch_out = (double)T * K * d * 2 <= 32.0 * (1 << 20) ? 1 : 0;
   cudaError_t e = cudaLaunchKernelEx(&cfg, atomic_experts_kernel, T, d, K, act, (const uint4*)x, (const uint4*)w_in,
                                      (const uint4*)w_out, idx, g, coef, (uint4*)out, n_experts, prefetch_out, bar,
-                                     limit_ns, status);
+                                     g_barrier_extra, limit_ns, status);
   count_launch();
   if (e != cudaSuccess) return e;
   return cudaGetLastError();

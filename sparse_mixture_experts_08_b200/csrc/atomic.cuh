@@ -16,4 +16,8 @@ cudaError_t launch_atomic_experts_sorted(int T, int d, int K, int act, const voi
                                          long long n_experts, unsigned* bar, bool bar_zeroed,
                                          unsigned long long limit_ns, int* status, int32_t* sort_ws, cudaStream_t s);
 
+// Fault-injection hook: the decode-budget atomic-expert kernel's grid barrier waits
+// for n arrivals more than its grid has, so it ends only at its time limit.
+void set_grid_barrier_extra(unsigned n);
+
 }  // namespace moe

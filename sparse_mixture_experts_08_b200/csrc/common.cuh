@@ -179,6 +179,12 @@ cudaError_t launch_route_topk(const moe_config_t& c, const void* x, const void* 
                               int32_t* idx, float* w, int32_t* lrank, int32_t* tile_cnt, int* status,
                               unsigned long long wait_limit_ns, cudaStream_t s);
 int tc_max_groups();
+// Router logits by the kernel that suits the batch (CUDA cores for fp32 or small
+// batches, the tensor cores otherwise); the bounded waits use wait_limit_ns().
+cudaError_t launch_router_logits(const moe_config_t& c, const void* x, const void* w_r, const float* bias,
+                                 float* logits, int* status, cudaStream_t s);
+// The current time limit of the bounded waits (moe_debug_set_wait_limit_ns).
+unsigned long long wait_limit_ns();
 
 // SIMT grouped linear (fp32 or bf16 inputs, fp32 math), same GemmParams.
 cudaError_t launch_simt_gemm(int epi, int dtype, const GemmParams& p, int max_rows_per_group, cudaStream_t s);

@@ -1,10 +1,11 @@
 // moe_route_static: the router (logits -> top-k -> gate weights) for callers that
 // cannot hand the library a workspace.
 //
-// Some callers have no way to obtain device memory for scratch: code that runs
-// while a CUDA graph is being captured (cudaMalloc is not allowed then), plugins
-// that only ever see the tensors a host framework gives them, or serving loops
-// that forbid allocation on the request path. moe_route needs scratch for the
+// Some callers have no way to obtain device memory for scratch: plugins that only
+// ever see the tensors a host framework gives them (the framework owns the
+// allocator and hands out no extra buffers), and serving loops that forbid
+// allocation on the request path (an allocation can block, fragment the pool or
+// fail under memory pressure at the worst moment). moe_route needs scratch for the
 // intermediate router logits (when the caller does not want them) and for the
 // device status word; this entry point keeps both in a fixed array compiled into
 // the library instead, and allocates nothing.
@@ -22,8 +23,8 @@
 //  - The first call on each device looks up the array's device address with
 //    cudaGetSymbolAddress (with that device current); make that first call
 //    before starting any stream capture.
-#include <algorithm>
-#include <cstring>
+//  - The kernels are the ones moe_route launches (the same choice of router
+//    kernel, the same bounded-wait limit), so both give identical results.
 #include <initializer_list>
 
 #include "common.cuh"
@@ -97,7 +98,7 @@ extern "C" MOE_API moe_status_t moe_route_static(const moe_config_t* cfg, const 
   const float* lg = logits_in;
   if (!lg && fused_route_ok(c)) {  // the same kernel choice as moe_route: logits + top-k in one launch
     if (launch_route_topk(c, x, w_router, bias, logits_out, topk_idx, topk_w, nullptr, nullptr, status,
-                          2000ull * 1000 * 1000, s) != cudaSuccess)
+                          wait_limit_ns(), s) != cudaSuccess)
       return MOE_ERR_CUDA;
     if (device_status_out &&
         cudaMemcpyAsync(device_status_out, status, sizeof(int32_t), cudaMemcpyDeviceToDevice, s) != cudaSuccess)
@@ -106,40 +107,7 @@ extern "C" MOE_API moe_status_t moe_route_static(const moe_config_t* cfg, const 
   }
   if (!lg) {
     float* dst = logits_out ? logits_out : reinterpret_cast<float*>(scratch + STATIC_STATUS_BYTES);
-    cudaError_t e;
-    if (few_expert_logits_ok(c.dtype, c.T, c.m)) {  // the same kernel choice as moe_route
-      e = launch_few_expert_logits(c.T, c.d, c.m, x, w_router, bias, dst, s);
-    } else if (c.dtype == MOE_F32 || c.T <= 64) {
-      e = launch_simt_logits(c.dtype, c.T, c.d, c.m, x, w_router, bias, dst, s);
-    } else {
-      // logits^T = W_r . x^T on the tensor cores, one token tile per CTA in one wave
-      GemmParams p;
-      std::memset(&p, 0, sizeof(p));
-      GemmClass& g = p.cls[0];
-      g.n_groups = 1;
-      g.R = c.m;
-      g.K = c.d;
-      g.ksplit = 1;
-      g.kb_per_split = (c.d + 63) / 64;
-      g.const_rows = c.T;
-      g.out = dst;
-      g.out_ld = c.m;
-      g.bias = bias;
-      p.n_classes = 1;
-      p.status = status;
-      p.wait_limit_ns = 2000ull * 1000 * 1000;
-      const long long mt = (c.m + 127) / 128;
-      int bn = 16;
-      while (bn < 128 && mt * ((c.T + bn - 1) / bn) > 148) bn <<= 1;
-      TcMaps maps;
-      std::memset(&maps, 0, sizeof(maps));
-      maps.a0[0] = {w_router, c.m, c.d};
-      maps.a1[0] = maps.a0[0];
-      maps.b[0] = {x, c.T, c.d};
-      const long long tiles = mt * ((c.T + bn - 1) / bn);
-      e = launch_tc_gemm(EPI_LOGITS, bn, maps, p, (int)std::min<long long>(tiles, num_sms()), s);
-    }
-    if (e != cudaSuccess) return MOE_ERR_CUDA;
+    if (launch_router_logits(c, x, w_router, bias, dst, status, s) != cudaSuccess) return MOE_ERR_CUDA;
     lg = dst;
   } else if (logits_out && logits_out != logits_in) {
     if (cudaMemcpyAsync(logits_out, logits_in, logits_bytes, cudaMemcpyDeviceToDevice, s) != cudaSuccess)

@@ -30,7 +30,7 @@ STATUS_NAMES = {0: "MOE_OK", 1: "MOE_ERR_INVALID_ARG", 2: "MOE_ERR_UNSUPPORTED",
 EXPORTS = ["moe_workspace_size", "moe_atomic_workspace_size", "moe_route", "moe_histogram_lis", "moe_permute",
            "moe_grouped_ffn", "moe_shared_ffn", "moe_combine", "moe_layer_forward", "moe_atomic_route",
            "moe_atomic_experts", "moe_atomic_forward", "moe_read_device_status", "moe_status_string",
-           "moe_debug_set_wait_limit_ns", "moe_set_stage_events", "moe_launch_count", "moe_route_static",
+           "moe_debug_set_wait_limit_ns", "moe_debug_set_barrier_extra", "moe_set_stage_events", "moe_launch_count", "moe_route_static",
            "moe_replica_split", "moe_layer_forward_replicated", "moe_floe_pack_down", "moe_floe_calibrate",
            "moe_floe_workspace_size", "moe_layer_forward_floe", "moe_quantize_e4m3", "moe_fp8_workspace_size",
            "moe_layer_forward_fp8"]
@@ -94,6 +94,7 @@ def lib() -> ctypes.CDLL:
             "moe_atomic_forward": [P, P, P, P, P, P, P, P, P, P, S, P],
             "moe_read_device_status": [P, P, P],
             "moe_debug_set_wait_limit_ns": [ctypes.c_uint64],
+            "moe_debug_set_barrier_extra": [ctypes.c_uint32],
             "moe_set_stage_events": [P, ctypes.c_int],
             "moe_route_static": [P, P, P, P, P, P, P, P, P, P],
             "moe_quantize_e4m3": [ctypes.c_int64, ctypes.c_int64, P, P, P, P],
@@ -324,6 +325,10 @@ def moe_status_string(status: int) -> str:
 
 def moe_debug_set_wait_limit_ns(ns: int):
     _check("moe_debug_set_wait_limit_ns", lib().moe_debug_set_wait_limit_ns(ns))
+
+
+def moe_debug_set_barrier_extra(n: int):
+    _check("moe_debug_set_barrier_extra", lib().moe_debug_set_barrier_extra(n))
 
 
 def moe_set_stage_events(events):

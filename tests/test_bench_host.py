@@ -34,12 +34,15 @@ def test_stage_bytes_match_the_layer_definition():
     assert layer_bytes == cfg.m * cfg.d * 2 + cfg.m * 2 * cfg.f * cfg.d * 2 + 2 * cfg.T * cfg.d * 2
 
 
-def test_committed_traffic_matches_the_current_gemm_sources():
+def test_committed_traffic_is_reported_only_for_unchanged_sources():
     with open(os.path.join(ROOT, "profiles", "traffic.json")) as fh:
         t = json.load(fh)
-    e = t["switch"]["expert_up"]
-    assert e["source_files"] == ["tc_gemm.cu", "common.cuh"]
-    assert bench.traffic_for("switch", "expert_up") == e["dram_bytes_per_launch"]
+    for workload, stages in t.items():
+        for stage, e in stages.items():
+            assert e["dram_bytes_per_launch"] > 0 and e["source_files"], (workload, stage)
+            current = e["source_hash"] == bench.source_hash(e["source_files"])
+            got = bench.traffic_for(workload, stage)
+            assert got == (e["dram_bytes_per_launch"] if current else None), (workload, stage)
 
 
 def test_traffic_goes_null_when_its_kernel_sources_change(tmp_path, monkeypatch):

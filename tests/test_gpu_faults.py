@@ -7,6 +7,9 @@
   call (default limit) is correct again.
 * Corrupted routing tables: expert ids outside [0, m) and inconsistent segment
   offsets become MOE_ERR_DEVICE_INDEX with no out-of-range write.
+* The atomic-expert kernel's grid barrier: a test hook makes it wait for one
+  arrival more than the grid has, so it ends only at its (1 ms) limit; the kernel
+  records MOE_ERR_TIMEOUT and its blocks return.
 """
 import numpy as np
 import pytest
@@ -96,6 +99,8 @@ def test_permute_rejects_bad_expert_id_without_writing():
 
 
 def test_layer_forward_after_errors_is_exact_again():
+    # a layer call whose tensor-core waits run out (1 ns limit) records TIMEOUT; the
+    # next call on the same workspace, with the default limit, is exact again
     cfg = W.small_moe(T=64, d=128, f=256, m=8, k=2, dtype=W.BF16, zipf_s=1.2, index=53)
     inp = W.make_moe_inputs(cfg)
     d = device_inputs(inp)
@@ -103,6 +108,15 @@ def test_layer_forward_after_errors_is_exact_again():
     ws = moe.workspace(c)
     out = torch.empty((cfg.T, cfg.d), dtype=torch.bfloat16, device="cuda")
     lg = torch.empty((cfg.T, cfg.m), dtype=torch.float32, device="cuda")
+    try:
+        moe.moe_debug_set_wait_limit_ns(1)
+        moe.moe_layer_forward(c, d["x"], d["w_router"], d["bias"], d["w_gate"], d["w_up"], d["w_down"], None, None,
+                              None, out, ws, logits_out=lg)
+        st = moe.moe_read_device_status(ws)
+    finally:
+        moe.moe_debug_set_wait_limit_ns(0)
+    assert st == moe.ERR_TIMEOUT
+    out.fill_(float("nan"))
     moe.moe_layer_forward(c, d["x"], d["w_router"], d["bias"], d["w_gate"], d["w_up"], d["w_down"], None, None, None,
                           out, ws, logits_out=lg)
     assert moe.moe_read_device_status(ws) == moe.OK
@@ -111,9 +125,10 @@ def test_layer_forward_after_errors_is_exact_again():
 
 
 def test_atomic_grid_barrier_times_out_and_recovers():
-    # the atomic-expert FFN is one cooperative launch with a grid-wide barrier; with a
-    # 1 ns limit the barrier gives up (MOE_ERR_TIMEOUT) instead of spinning, and the next
-    # call with the default limit is exact again
+    # the atomic-expert FFN is one cooperative launch with a grid-wide barrier. The
+    # test hook makes the barrier wait for one arrival more than the grid has, so it
+    # can only end at its time limit (1 ms here): the kernel must record
+    # MOE_ERR_TIMEOUT and return, and the next call with the normal barrier is exact.
     cfg = W.AtomicWorkload("atomic_fault", 93, T=4, d=256, Nr=64, Nc=64, K=16, act=W.ACT_SILU)
     inp = W.make_atomic_inputs(cfg)
     c = moe.make_atomic_config(cfg.T, cfg.d, cfg.Nr, cfg.Nc, cfg.K, cfg.act)
@@ -122,19 +137,27 @@ def test_atomic_grid_barrier_times_out_and_recovers():
     idx = torch.empty((cfg.T, cfg.K), dtype=torch.int32, device="cuda")
     g = torch.empty((cfg.T, cfg.K), dtype=torch.float32, device="cuda")
     moe.moe_atomic_route(c, d["x"], d["w_row"], d["w_col"], None, None, idx, g, ws)
+    assert moe.moe_read_device_status(ws) == moe.OK
     out = torch.empty((cfg.T, cfg.d), dtype=torch.bfloat16, device="cuda")
-    try:
-        moe.moe_debug_set_wait_limit_ns(1)
-        moe.moe_atomic_experts(c, d["x"], d["w_in"], d["w_out"], idx, g, out, ws)
-        st = moe.moe_read_device_status(ws)
-    finally:
-        moe.moe_debug_set_wait_limit_ns(0)
-    assert st in (moe.ERR_TIMEOUT, moe.OK)  # OK only if every block had arrived before the first check
+    for forward in (False, True):  # the experts call alone, and the whole layer (select zeroes the barrier)
+        try:
+            moe.moe_debug_set_wait_limit_ns(1_000_000)
+            moe.moe_debug_set_barrier_extra(1)
+            if forward:
+                moe.moe_atomic_forward(c, d["x"], d["w_row"], d["w_col"], d["w_in"], d["w_out"], out, ws)
+            else:
+                moe.moe_atomic_experts(c, d["x"], d["w_in"], d["w_out"], idx, g, out, ws)
+            st = moe.moe_read_device_status(ws)
+        finally:
+            moe.moe_debug_set_barrier_extra(0)
+            moe.moe_debug_set_wait_limit_ns(0)
+        assert st == moe.ERR_TIMEOUT
     moe.moe_atomic_experts(c, d["x"], d["w_in"], d["w_out"], idx, g, out, ws)
     assert moe.moe_read_device_status(ws) == moe.OK
     ref = O.atomic_output(inp["x"], inp["w_in"], inp["w_out"], host(idx), host(g), cfg.act)
     assert token_rel_err(out_f64(out), ref) <= TOL[W.BF16]
     out2 = torch.empty_like(out)
     moe.moe_atomic_forward(c, d["x"], d["w_row"], d["w_col"], d["w_in"], d["w_out"], out2, ws)
+    assert moe.moe_read_device_status(ws) == moe.OK
     torch.cuda.synchronize()
     assert torch.equal(out, out2)
