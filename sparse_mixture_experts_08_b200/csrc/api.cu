@@ -70,6 +70,7 @@ struct Plan {
   int bn_up, bn_down;
   int ksplit;      // down-projection K split (1 when shared experts are present)
   int kbps;        // k-blocks per split of the routed down projection
+  bool pair;       // bf16 expert GEMMs as two-CTA tiles (256 token rows, no K split)
 };
 
 static int kblocks(int K) { return (K + 63) / 64; }
@@ -82,7 +83,8 @@ static Plan make_plan(const moe_config_t& c) {
   p.bn_down = tc_pick_bn(EPI_DOWN, avg);
   p.ksplit = 1;
   p.kbps = kblocks(c.f);
-  if (c.dtype == MOE_BF16 && c.n_shared == 0) {
+  p.pair = c.dtype == MOE_BF16 && tc_pick_pair(avg);
+  if (c.dtype == MOE_BF16 && c.n_shared == 0 && !p.pair) {
     const long long active = std::min<long long>(c.m, (long long)c.T * c.k);
     const long long nt = std::max<long long>(1, (long long)((avg + p.bn_down - 1) / p.bn_down));
     const long long tiles = active * ((c.d + 127) / 128) * nt;
@@ -347,8 +349,9 @@ static moe_status_t run_ffn(const moe_config_t& c, const Plan& pl, const FfnIo& 
   if (ncls == 0) return MOE_OK;
   up.n_classes = ncls;
   const int epi_up = swiglu ? EPI_SWIGLU : EPI_RELU;
+  const bool pair = tc && pl.pair && !q8 && ksplit == 1;  // two-CTA tiles: bf16 operands only
   if (tc)
-    MOE_CUDA(launch_tc_gemm(epi_up, pl.bn_up, mu, up, num_sms(), s, q8 != nullptr));
+    MOE_CUDA(launch_tc_gemm(epi_up, pair ? 256 : pl.bn_up, mu, up, num_sms(), s, q8 != nullptr, pair));
   else
     MOE_CUDA(launch_simt_gemm(epi_up, c.dtype, up, (int)std::min<long long>(io.routed_rows, 1LL << 30), s));
   if (stage_marks) MOE_TRY(mark_stage(5, s));
@@ -428,7 +431,7 @@ static moe_status_t run_ffn(const moe_config_t& c, const Plan& pl, const FfnIo& 
   }
   dn.n_classes = ncls;
   if (tc)
-    return cuda_status(launch_tc_gemm(EPI_DOWN, pl.bn_down, md, dn, num_sms(), s, q8 != nullptr));
+    return cuda_status(launch_tc_gemm(EPI_DOWN, pair ? 256 : pl.bn_down, md, dn, num_sms(), s, q8 != nullptr, pair));
   return cuda_status(launch_simt_gemm(EPI_DOWN, c.dtype, dn, (int)std::min<long long>(io.routed_rows, 1LL << 30), s));
 }
 

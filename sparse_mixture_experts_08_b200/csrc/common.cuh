@@ -170,9 +170,13 @@ struct TcOperand {
 struct TcMaps {
   TcOperand a0[2], a1[2], b[2];
 };
+// pair = two-CTA tiles (tcgen05.mma.cta_group::2, 256 weight rows x up to 256 token
+// rows per tile; bf16 SwiGLU / ReLU / down projections with bn = 256 and no K split).
 cudaError_t launch_tc_gemm(int epi, int bn, const TcMaps& maps, const GemmParams& p, int num_ctas,
-                           cudaStream_t s, bool f8 = false);
+                           cudaStream_t s, bool f8 = false, bool pair = false);
 int tc_pick_bn(int epi, double avg_rows_per_group);
+// Whether the expert GEMMs of a layer with this mean segment length run as pair tiles.
+bool tc_pick_pair(double avg_rows_per_group);
 // Router logits + top-k softmax (+ per-tile expert counts and task ranks when lrank
 // and tile_cnt are given) in one tensor-core launch (EPI_ROUTE); logits nullable.
 cudaError_t launch_route_topk(const moe_config_t& c, const void* x, const void* w_r, const float* bias, float* logits,

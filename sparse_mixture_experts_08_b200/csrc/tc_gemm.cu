@@ -30,6 +30,17 @@
 // Every wait on an mbarrier is bounded in time (globaltimer); on expiry the kernel
 // records MOE_ERR_TIMEOUT in the status word, the other roles stop, outstanding
 // TMA copies and MMAs are drained (again with a bound) and TMEM is freed.
+//
+// Pair variant (PAIR, large segments): a cluster of two CTAs on two SMs runs one
+// tcgen05.mma.cta_group::2 per K step with M = 256 weight rows, 128 in each CTA's
+// shared memory, and N = up to 256 token rows, half of them in each CTA; each CTA's
+// TMEM holds its own 128 features x N tokens, so the epilogue stays local. Per SM
+// the MMA then reads half the operand bytes from shared memory that a one-SM tile
+// of the same N reads, which is what bounds the one-SM kernel on the prefill
+// shapes. The leader CTA (rank 0) issues the MMAs; both CTAs' TMA copies complete
+// on the leader's stage barrier; the leader's commits arrive on both CTAs' barriers;
+// both CTAs' epilogues release the accumulator on the leader's barrier. Both CTAs
+// meet at a cluster barrier before TMEM is freed and the CTAs exit.
 #include <algorithm>
 #include <cstring>
 #include <cstdio>
@@ -48,10 +59,12 @@ constexpr unsigned long long TC_DRAIN_LIMIT_NS = 200ull * 1000 * 1000;
 
 int tc_max_groups() { return TC_MAX_GROUPS; }
 
-template <int BN, int MATS>
+template <int BN, int MATS, bool PAIR = false>
 struct TcShape {
+  static constexpr int TILE_M = PAIR ? 2 * TC_BM : TC_BM;  // weight rows per tile (both CTAs)
+  static constexpr int B_ROWS = PAIR ? BN / 2 : BN;        // token rows per CTA
   static constexpr int A_BYTES = TC_BM * TC_BK * 2;    // 16 KB
-  static constexpr int B_BYTES = BN * TC_BK * 2;       // BN * 128 B
+  static constexpr int B_BYTES = B_ROWS * TC_BK * 2;   // B_ROWS * 128 B
   static constexpr int STAGE_BYTES = MATS * A_BYTES + B_BYTES;
   static constexpr int STAGES_RAW = TC_SMEM_BUDGET / STAGE_BYTES;
   static constexpr int STAGES = STAGES_RAW > 8 ? 8 : STAGES_RAW;
@@ -75,6 +88,87 @@ __device__ __forceinline__ void tma_load_2d(const CUtensorMap* map, uint64_t* ba
 }
 __device__ __forceinline__ void tma_prefetch_desc(const CUtensorMap* map) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
+}
+
+// ---- two-CTA (cluster pair) forms
+__device__ __forceinline__ uint32_t cluster_ctarank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+__device__ __forceinline__ uint32_t cluster_id_x() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%clusterid.x;" : "=r"(r));
+  return r;
+}
+__device__ __forceinline__ uint32_t nclusters_x() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%nclusterid.x;" : "=r"(r));
+  return r;
+}
+// shared::cluster address of the variable at shared::cta address `addr` in CTA `rank`
+__device__ __forceinline__ uint32_t mapa_shared(uint32_t addr, uint32_t rank) {
+  uint32_t r;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(addr), "r"(rank));
+  return r;
+}
+// Every thread of both CTAs arrives, then waits (release / acquire at cluster scope).
+__device__ __forceinline__ void cluster_sync_all() {
+  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+// TMA tile load into this CTA's shared memory whose completion is counted on an
+// mbarrier that may sit in the peer CTA of the pair (a shared::cluster address).
+__device__ __forceinline__ void tma_load_2d_pair(const CUtensorMap* map, uint32_t bar_cluster, void* dst, int x,
+                                                 int y) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4}], "
+      "[%2];" ::"r"(smem_u32(dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(bar_cluster), "r"(x), "r"(y)
+      : "memory");
+}
+__device__ __forceinline__ void mbar_arrive_cluster(uint32_t bar_cluster) {
+  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(bar_cluster) : "memory");
+}
+
+template <bool PAIR>
+__device__ __forceinline__ void tmem_alloc_g(uint32_t* dst, uint32_t ncols) {
+  if (PAIR)
+    asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(dst)), "r"(ncols)
+                 : "memory");
+  else
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(dst)), "r"(ncols)
+                 : "memory");
+}
+template <bool PAIR>
+__device__ __forceinline__ void tmem_relinquish_g() {
+  if (PAIR)
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
+  else
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+}
+template <bool PAIR>
+__device__ __forceinline__ void tmem_dealloc_g(uint32_t taddr, uint32_t ncols) {
+  if (PAIR)
+    asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols) : "memory");
+  else
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols) : "memory");
+}
+// D (+)= A * B^T over the pair: M = 256 (128 rows of A in each CTA), N token rows
+// (N / 2 in each CTA), kind::f16 (bf16 operands, fp32 accumulator)
+__device__ __forceinline__ void umma_bf16_pair(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                               uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n\t}\n" ::"r"(d_tmem),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+// Arrive on the mbarrier at shared::cluster address `bar_cluster` (this CTA's or the
+// peer's) once every pair MMA this thread issued so far completed.
+__device__ __forceinline__ void umma_commit_pair(uint32_t bar_cluster) {
+  asm volatile("tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar_cluster)
+               : "memory");
 }
 
 __device__ __forceinline__ void tmem_alloc(uint32_t* dst, uint32_t ncols) {
@@ -251,7 +345,7 @@ struct SchedSmem {
   int brow[TC_MAX_GROUPS];
 };
 
-template <int BN, int BKE>
+template <int BN, int BKE, int TILE_M = TC_BM>
 __device__ __forceinline__ void decode_tile(const GemmParams& p, const SchedSmem& s, int G, int w, TileInfo& ti) {
   int lo = 0, hi = G - 1;  // largest gi with tile_start[gi] <= w
   while (lo < hi) {
@@ -279,7 +373,7 @@ __device__ __forceinline__ void decode_tile(const GemmParams& p, const SchedSmem
     wg = c.group_map[ti.g];
     if (wg < 0 || wg >= c.n_wgroups) wg = 0;  // (validated where the map is written)
   }
-  ti.a_row = wg * c.R + ti.mt * TC_BM;
+  ti.a_row = wg * c.R + ti.mt * TILE_M;
   const int KB = (c.K + BKE - 1) / BKE;
   ti.kb0 = ti.ks * c.kb_per_split;
   ti.kb1 = min(KB, ti.kb0 + c.kb_per_split);
@@ -315,16 +409,19 @@ __device__ __forceinline__ void store_logit(const GemmClass& c, const TileInfo& 
   o[((long long)ti.out_row + j) * c.out_ld + feature] = v;
 }
 
-template <int BN, int MATS, int EPI, bool F8>
+template <int BN, int MATS, int EPI, bool F8, bool PAIR>
 __global__ void __launch_bounds__(TC_THREADS, 1)
     tc_grouped_gemm_kernel(const __grid_constant__ CUtensorMap tA0_0, const __grid_constant__ CUtensorMap tA1_0,
                            const __grid_constant__ CUtensorMap tB_0, const __grid_constant__ CUtensorMap tA0_1,
                            const __grid_constant__ CUtensorMap tA1_1, const __grid_constant__ CUtensorMap tB_1,
                            const __grid_constant__ GemmParams p) {
-  using S = TcShape<BN, MATS>;
+  using S = TcShape<BN, MATS, PAIR>;
   constexpr int STAGES = S::STAGES;
   constexpr int BKE = F8 ? TC_BK8 : TC_BK;  // K elements per k-block (one 128-byte row)
+  constexpr int TILE_M = S::TILE_M;
   static_assert(!F8 || EPI == EPI_SWIGLU || EPI == EPI_RELU || EPI == EPI_DOWN, "8-bit operands: expert GEMMs only");
+  static_assert(!PAIR || (!F8 && (EPI == EPI_SWIGLU || EPI == EPI_RELU || EPI == EPI_DOWN)),
+                "pair tiles: bf16 expert GEMMs only");
 
   __shared__ SchedSmem sched;
   __shared__ __align__(8) uint64_t full_bar[STAGES], empty_bar[STAGES], accf_bar[2], acce_bar[2], drain_bar;
@@ -345,6 +442,12 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
   extern __shared__ uint8_t dyn_smem[];
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  // PAIR: rank 0 of the cluster pair is the leader (it issues the MMAs); both CTAs
+  // walk the same tiles, indexed by cluster. Otherwise one CTA is one walker.
+  const uint32_t rank = PAIR ? cluster_ctarank() : 0u;
+  const bool leader = rank == 0;
+  const int walker = PAIR ? (int)cluster_id_x() : (int)blockIdx.x;
+  const int walkers = PAIR ? (int)nclusters_x() : (int)gridDim.x;
   const uint32_t smem_base = (smem_u32(dyn_smem) + 1023u) & ~1023u;
   uint8_t* smem_gen = dyn_smem + (smem_base - smem_u32(dyn_smem));
   const int G0 = p.cls[0].n_groups;
@@ -358,7 +461,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&accf_bar[i], 1);
-      mbar_init(&acce_bar[i], 4);
+      mbar_init(&acce_bar[i], PAIR ? 8 : 4);  // PAIR: the epilogue warps of both CTAs release the leader's
     }
     mbar_init(&drain_bar, 1);
     abort_s = 0;
@@ -368,9 +471,12 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
     tma_prefetch_desc(&tB_0);
   }
   if (warp == 1) {
-    tmem_alloc(&tmem_base_s, S::TMEM_COLS);
-    tmem_relinquish();
+    tmem_alloc_g<PAIR>(&tmem_base_s, S::TMEM_COLS);
+    tmem_relinquish_g<PAIR>();
   }
+  // PAIR: the peer's barriers must be initialised before either CTA signals them
+  __syncwarp();
+  if (PAIR) cluster_sync_all();
   // Everything above overlaps the previous kernel; the segment offsets, the token
   // rows (TMA) and the row data read below are its outputs.
   pdl_launch_dependents();
@@ -400,7 +506,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
       }
       sched.rows[gi] = rows;
       sched.brow[gi] = brow;
-      const int MT = (c.R + TC_BM - 1) / TC_BM;
+      const int MT = (c.R + TILE_M - 1) / TILE_M;
       local += MT * c.ksplit * ((rows + BN - 1) / BN);
       sched.tile_start[gi + 1] = local;
     }
@@ -434,23 +540,37 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
 #pragma unroll
     for (int i = 0; i < STAGES; ++i) last_parity[i] = -1;
     bool ok = true;
-    for (int w = blockIdx.x; w < total && ok; w += gridDim.x) {
+    for (int w = walker; w < total && ok; w += walkers) {
       TileInfo ti;
-      decode_tile<BN, BKE>(p, sched, G, w, ti);
+      decode_tile<BN, BKE, TILE_M>(p, sched, G, w, ti);
       const CUtensorMap* mA0 = ti.cls ? &tA0_1 : &tA0_0;
       const CUtensorMap* mA1 = ti.cls ? &tA1_1 : &tA1_0;
       const CUtensorMap* mB = ti.cls ? &tB_1 : &tB_0;
+      // PAIR: this CTA's 128 weight rows and its half of the tile's token rows
+      const int n_inst = max(16, (ti.rows_in_tile + 15) & ~15);
+      const int a_row = ti.a_row + (int)rank * TC_BM;
+      const int b_row = ti.b_row + (int)rank * (n_inst / 2);
       for (int kb = ti.kb0; kb < ti.kb1; ++kb) {
         if (!mbar_wait(&empty_bar[stage], phase ^ 1u, lim, abort_flag)) {
           ok = false;
           break;
         }
         uint8_t* st = smem_gen + stage * S::STAGE_BYTES;
-        mbar_arrive_expect_tx(&full_bar[stage], S::STAGE_BYTES);
-        tma_load_2d(mA0, &full_bar[stage], st, kb * BKE, ti.a_row);
-        if (MATS == 2) tma_load_2d(mA1, &full_bar[stage], st + S::A_BYTES, kb * BKE, ti.a_row);
-        tma_load_2d(mB, &full_bar[stage], st + MATS * S::A_BYTES, kb * BKE, ti.b_row);
-        last_parity[stage] = (int)phase;
+        if (PAIR) {
+          // both CTAs' copies complete on the leader's barrier, which expects them all
+          const uint32_t fb = mapa_shared(smem_u32(&full_bar[stage]), 0);
+          if (leader) mbar_arrive_expect_tx(&full_bar[stage], 2 * S::STAGE_BYTES);
+          tma_load_2d_pair(mA0, fb, st, kb * BKE, a_row);
+          if (MATS == 2) tma_load_2d_pair(mA1, fb, st + S::A_BYTES, kb * BKE, a_row);
+          tma_load_2d_pair(mB, fb, st + MATS * S::A_BYTES, kb * BKE, b_row);
+          if (leader) last_parity[stage] = (int)phase;
+        } else {
+          mbar_arrive_expect_tx(&full_bar[stage], S::STAGE_BYTES);
+          tma_load_2d(mA0, &full_bar[stage], st, kb * BKE, ti.a_row);
+          if (MATS == 2) tma_load_2d(mA1, &full_bar[stage], st + S::A_BYTES, kb * BKE, ti.a_row);
+          tma_load_2d(mB, &full_bar[stage], st + MATS * S::A_BYTES, kb * BKE, ti.b_row);
+          last_parity[stage] = (int)phase;
+        }
         if (++stage == STAGES) {
           stage = 0;
           phase ^= 1u;
@@ -461,23 +581,25 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
       set_status(p.status, MOE_ERR_TIMEOUT);
       abort_s = 1;
     }
-    // Drain: every issued copy must land before the CTA may exit.
+    // Drain: every issued copy must land before the CTA may exit. (PAIR: the leader's
+    // barriers count both CTAs' copies, and the peer waits for the leader at the
+    // final cluster barrier.)
     for (int i = 0; i < STAGES; ++i)
       if (last_parity[i] >= 0) {
         const volatile int never = 0;
         if (!mbar_wait(&full_bar[i], (uint32_t)last_parity[i], TC_DRAIN_LIMIT_NS, &never))
           set_status(p.status, MOE_ERR_TIMEOUT);
       }
-  } else if (warp == 1 && lane == 0) {
+  } else if (warp == 1 && lane == 0 && leader) {
     // ---------------------------------------------------------------- MMA issuer
     int stage = 0;
     uint32_t phase = 0;
     int acc = 0;
     uint32_t acc_phase = 0;
     bool ok = true;
-    for (int w = blockIdx.x; w < total && ok; w += gridDim.x) {
+    for (int w = walker; w < total && ok; w += walkers) {
       TileInfo ti;
-      decode_tile<BN, BKE>(p, sched, G, w, ti);
+      decode_tile<BN, BKE, TILE_M>(p, sched, G, w, ti);
       if (!mbar_wait(&acce_bar[acc], acc_phase ^ 1u, lim, abort_flag)) {
         ok = false;
         break;
@@ -485,7 +607,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
       tc_fence_after();
       const uint32_t d_tmem = tmem_base + (uint32_t)(acc * S::ACC_COLS);
       const int n_inst = max(16, (ti.rows_in_tile + 15) & ~15);
-      const uint32_t idesc = F8 ? idesc_e4m3(TC_BM, n_inst) : idesc_bf16(TC_BM, n_inst);
+      const uint32_t idesc = F8 ? idesc_e4m3(TILE_M, n_inst) : idesc_bf16(TILE_M, n_inst);
       for (int kb = ti.kb0; kb < ti.kb1; ++kb) {
         if (!mbar_wait(&full_bar[stage], phase, lim, abort_flag)) {
           ok = false;
@@ -500,7 +622,10 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
         for (int kk = 0; kk < 4; ++kk) {
           const uint32_t accum = (kb > ti.kb0 || kk > 0) ? 1u : 0u;
           // one MMA takes 32 B of K (16 bf16 or 32 E4M3): +2 in the >>4 address field
-          if (F8) {
+          if (PAIR) {
+            umma_bf16_pair(d_tmem, da0 + 2 * kk, db + 2 * kk, idesc, accum);
+            if (MATS == 2) umma_bf16_pair(d_tmem + BN, da1 + 2 * kk, db + 2 * kk, idesc, accum);
+          } else if (F8) {
             umma_e4m3(d_tmem, da0 + 2 * kk, db + 2 * kk, idesc, accum);
             if (MATS == 2) umma_e4m3(d_tmem + BN, da1 + 2 * kk, db + 2 * kk, idesc, accum);
           } else {
@@ -508,14 +633,24 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
             if (MATS == 2) umma_bf16(d_tmem + BN, da1 + 2 * kk, db + 2 * kk, idesc, accum);
           }
         }
-        umma_commit(&empty_bar[stage]);
+        if (PAIR) {  // the stage is free in both CTAs
+          umma_commit_pair(smem_u32(&empty_bar[stage]));
+          umma_commit_pair(mapa_shared(smem_u32(&empty_bar[stage]), 1));
+        } else {
+          umma_commit(&empty_bar[stage]);
+        }
         if (++stage == STAGES) {
           stage = 0;
           phase ^= 1u;
         }
       }
       if (!ok) break;
-      umma_commit(&accf_bar[acc]);
+      if (PAIR) {  // both CTAs' accumulators are ready
+        umma_commit_pair(smem_u32(&accf_bar[acc]));
+        umma_commit_pair(mapa_shared(smem_u32(&accf_bar[acc]), 1));
+      } else {
+        umma_commit(&accf_bar[acc]);
+      }
       if (++acc == S::NUM_ACC) {
         acc = 0;
         acc_phase ^= 1u;
@@ -525,7 +660,10 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
       set_status(p.status, MOE_ERR_TIMEOUT);
       abort_s = 1;
     }
-    umma_commit(&drain_bar);
+    if (PAIR)
+      umma_commit_pair(smem_u32(&drain_bar));
+    else
+      umma_commit(&drain_bar);
     const volatile int never = 0;
     if (!mbar_wait(&drain_bar, 0, TC_DRAIN_LIMIT_NS, &never)) set_status(p.status, MOE_ERR_TIMEOUT);
   } else if (EPI == EPI_ROUTE && warp >= 2) {
@@ -542,7 +680,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
     }
     int acc = 0, iter = 0;
     uint32_t acc_phase = 0;
-    for (int w = blockIdx.x; w < total; w += gridDim.x, ++iter) {
+    for (int w = walker; w < total; w += walkers, ++iter) {
       TileInfo ti;
       decode_tile<BN, BKE>(p, sched, G, w, ti);
       const GemmClass& c = p.cls[0];
@@ -647,17 +785,18 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
     const int q = warp & 3;  // TMEM lane quarter this warp may access
     int acc = 0;
     uint32_t acc_phase = 0;
-    for (int w = blockIdx.x; w < total; w += gridDim.x) {
+    for (int w = walker; w < total; w += walkers) {
       TileInfo ti;
-      decode_tile<BN, BKE>(p, sched, G, w, ti);
+      decode_tile<BN, BKE, TILE_M>(p, sched, G, w, ti);
       const GemmClass& c = p.cls[ti.cls];
-      const int feature = ti.mt * TC_BM + q * 32 + lane;
+      const int fcta = ti.mt * TILE_M + (int)rank * TC_BM;  // first feature of this CTA's TMEM lanes
+      const int feature = fcta + q * 32 + lane;
       const bool fvalid = feature < c.R;
       const bool has_k = ti.kb1 > ti.kb0;  // an empty K range leaves the accumulator unwritten
       const float bias = (EPI == EPI_LOGITS && c.bias && fvalid) ? c.bias[feature] : 0.f;
       // F8: scale of this lane's weight row (index = weight-matrix row of the feature)
-      const float sa0 = (F8 && fvalid) ? c.a0_scale[ti.a_row + q * 32 + lane] : 1.f;
-      const float sa1 = (F8 && MATS == 2 && fvalid) ? c.a1_scale[ti.a_row + q * 32 + lane] : 1.f;
+      const float sa0 = (F8 && fvalid) ? c.a0_scale[ti.a_row + (int)rank * TC_BM + q * 32 + lane] : 1.f;
+      const float sa1 = (F8 && MATS == 2 && fvalid) ? c.a1_scale[ti.a_row + (int)rank * TC_BM + q * 32 + lane] : 1.f;
       // Row data of the whole tile (gate weight, destination token), fetched into this
       // warp's shared-memory slice before waiting for the accumulator so the loads
       // overlap the MMAs; the chunk loop below then reads it with broadcasts.
@@ -704,7 +843,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
                                                 : v0 * aux_w[q][c0 + j];
           }
           __syncwarp();
-          const int fbase = ti.mt * TC_BM + q * 32;  // first feature of this warp (R is a multiple of 8)
+          const int fbase = fcta + q * 32;  // first feature of this warp (R is a multiple of 8)
           if (EPI == EPI_DOWN && !c.scatter_k1) {  // fp32 partial rows: 8 float4 per row
             float* o = reinterpret_cast<float*>(c.out) + (long long)ti.ks * c.out_split_stride + fbase;
 #pragma unroll
@@ -740,7 +879,12 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
       }
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&acce_bar[acc]);
+      if (lane == 0) {
+        if (PAIR && !leader)  // the leader's MMA waits for both CTAs' epilogues
+          mbar_arrive_cluster(mapa_shared(smem_u32(&acce_bar[acc]), 0));
+        else
+          mbar_arrive(&acce_bar[acc]);
+      }
       if (++acc == S::NUM_ACC) {
         acc = 0;
         acc_phase ^= 1u;
@@ -753,9 +897,12 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
   __syncwarp();
   tc_fence_before();
   __syncthreads();
+  // PAIR: neither CTA frees TMEM or exits while the other may still signal its
+  // barriers or (leader) have MMAs writing the peer's accumulators
+  if (PAIR) cluster_sync_all();
   if (warp == 1) {
     tc_fence_after();
-    tmem_dealloc(tmem_base, S::TMEM_COLS);
+    tmem_dealloc_g<PAIR>(tmem_base, S::TMEM_COLS);
   }
 }
 
@@ -793,9 +940,9 @@ static bool make_map(CUtensorMap* m, const TcOperand& op, int box_rows, bool u8)
   return r == CUDA_SUCCESS;
 }
 
-template <int BN, int MATS, int EPI, bool F8>
+template <int BN, int MATS, int EPI, bool F8, bool PAIR = false>
 static cudaError_t launch_impl(const TcMaps& maps, const GemmParams& p, int num_ctas, cudaStream_t s) {
-  using S = TcShape<BN, MATS>;
+  using S = TcShape<BN, MATS, PAIR>;
   CUtensorMap m[6];
   const int nc = p.n_classes;
   for (int c = 0; c < 2; ++c) {
@@ -803,14 +950,47 @@ static cudaError_t launch_impl(const TcMaps& maps, const GemmParams& p, int num_
     if (!make_map(&m[3 * c + 0], maps.a0[src], TC_BM, F8)) return cudaErrorInvalidValue;
     const TcOperand& a1 = MATS == 2 ? maps.a1[src] : maps.a0[src];
     if (!make_map(&m[3 * c + 1], a1, TC_BM, F8)) return cudaErrorInvalidValue;
-    if (!make_map(&m[3 * c + 2], maps.b[src], BN, F8)) return cudaErrorInvalidValue;
+    if (!make_map(&m[3 * c + 2], maps.b[src], S::B_ROWS, F8)) return cudaErrorInvalidValue;
   }
-  auto kern = tc_grouped_gemm_kernel<BN, MATS, EPI, F8>;
+  auto kern = tc_grouped_gemm_kernel<BN, MATS, EPI, F8, PAIR>;
   static bool attr_set = false;
   if (!attr_set) {
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, S::DYN_SMEM);
     if (e != cudaSuccess) return e;
     attr_set = true;
+  }
+  if (PAIR) {
+    // clusters of two CTAs on two SMs (persistent): as many pairs as can be resident
+    // at once, so no pair waits for another to finish (a GPC with an odd number of
+    // free SMs leaves one SM out)
+    static int max_pairs = 0;
+    cudaLaunchConfig_t cfg = {};
+    cfg.blockDim = dim3(TC_THREADS);
+    cfg.dynamicSmemBytes = S::DYN_SMEM;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[2];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[1].val.programmaticStreamSerializationAllowed = 1;
+    if (!max_pairs) {  // the occupancy query takes the cluster shape alone
+      cfg.gridDim = dim3(std::max(2, num_ctas & ~1));
+      cfg.attrs = attr;
+      cfg.numAttrs = 1;
+      int n = 0;
+      const cudaError_t eo = cudaOccupancyMaxActiveClusters(&n, kern, &cfg);
+      if (eo != cudaSuccess) return eo;
+      max_pairs = std::max(1, n);
+    }
+    cfg.gridDim = dim3(2 * std::min(max_pairs, std::max(1, num_ctas / 2)));
+    cfg.attrs = attr;
+    cfg.numAttrs = 2;
+    cudaError_t e = cudaLaunchKernelEx(&cfg, kern, m[0], m[1], m[2], m[3], m[4], m[5], p);
+    count_launch();
+    if (e != cudaSuccess) return e;
+    return cudaGetLastError();
   }
   launch_k(kern, num_ctas, TC_THREADS, S::DYN_SMEM, s, m[0], m[1], m[2], m[3], m[4], m[5], p);
   count_launch();
@@ -833,8 +1013,23 @@ int tc_pick_bn(int epi, double avg) {
   return bn;
 }
 
+// Pair tiles (256 weight rows over two SMs, up to 256 token rows) when the mean
+// segment fills a 256-row token tile: then each SM reads half the operand bytes per
+// MMA that a one-SM 128-row tile reads, and shared-memory bandwidth stops bounding
+// the tensor pipe (Mixtral-shaped prefill: 1024 rows per expert on average).
+bool tc_pick_pair(double avg) { return avg >= 256.0; }
+
 cudaError_t launch_tc_gemm(int epi, int bn, const TcMaps& maps, const GemmParams& p, int num_ctas,
-                           cudaStream_t s, bool f8) {
+                           cudaStream_t s, bool f8, bool pair) {
+  if (pair) {  // two-CTA tiles: bf16 expert GEMMs with 256-row token tiles, no K split
+    if (f8 || bn != 256) return cudaErrorInvalidValue;
+    for (int c = 0; c < p.n_classes; ++c)
+      if (p.cls[c].ksplit != 1) return cudaErrorInvalidValue;
+    if (epi == EPI_SWIGLU) return launch_impl<256, 2, EPI_SWIGLU, false, true>(maps, p, num_ctas, s);
+    if (epi == EPI_RELU) return launch_impl<256, 1, EPI_RELU, false, true>(maps, p, num_ctas, s);
+    if (epi == EPI_DOWN) return launch_impl<256, 1, EPI_DOWN, false, true>(maps, p, num_ctas, s);
+    return cudaErrorInvalidValue;
+  }
   if (f8) {
     if (epi != EPI_SWIGLU && epi != EPI_RELU && epi != EPI_DOWN) return cudaErrorInvalidValue;
     for (int c = 0; c < p.n_classes; ++c)

@@ -172,6 +172,12 @@ FFN_CASES = [
     (1, 512, 1024, 8, 2, W.SWIGLU, W.BF16, 0.0),
     (700, 64, 64, 4, 1, W.RELU, W.BF16, 3.0),
     (130, 96, 160, 3, 2, W.RELU, W.F32, 0.5),
+    # 256+ rows per expert on average: two-CTA pair tiles (256 weight rows over two SMs,
+    # up to 256 token rows); f and K not multiples of the tile, ragged and skewed segments
+    (1000, 256, 384, 4, 2, W.SWIGLU, W.BF16, 1.0),
+    (2048, 136, 200, 4, 1, W.RELU, W.BF16, 2.0),
+    (600, 512, 256, 2, 1, W.SWIGLU, W.BF16, 0.0),
+    (1300, 64, 520, 3, 2, W.SWIGLU, W.BF16, 3.0),
 ]
 
 

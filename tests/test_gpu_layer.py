@@ -98,7 +98,8 @@ def test_decode_all_tokens():
 
 
 @pytest.mark.parametrize("case", ["one_hot", "one_hot_fused", "T1", "ragged_small", "relu_many_experts",
-                                  "max_experts_max_k", "routed_k8_m200"])
+                                  "max_experts_max_k", "routed_k8_m200", "pair_shared", "pair_empty_and_single",
+                                  "pair_relu_top1"])
 def test_layer_edge_cases(case):
     if case in ("one_hot", "one_hot_fused"):  # every token's top-1 is the same expert (huge bias)
         T = 300 if case == "one_hot" else 8192  # 8192: the fused router and scatter
@@ -119,12 +120,31 @@ def test_layer_edge_cases(case):
     elif case == "routed_k8_m200":  # fused router (8192+ tokens): largest k, m not a power of two, ragged tile
         cfg = W.small_moe(T=8269, d=64, f=64, m=200, k=8, dtype=W.BF16, zipf_s=0.7, renorm=True, index=78)
         inp = W.make_moe_inputs(cfg)
+    elif case == "pair_shared":  # pair tiles (256+ rows per expert) with a shared expert as a second class
+        cfg = W.small_moe(T=1024, d=256, f=256, m=4, k=1, dtype=W.BF16, zipf_s=1.0, n_shared=1, f_shared=136,
+                          index=79)
+        inp = W.make_moe_inputs(cfg)
+    elif case == "pair_empty_and_single":  # pair tiles; one expert gets no task, one exactly one
+        cfg = W.small_moe(T=1200, d=192, f=320, m=4, k=1, dtype=W.BF16, zipf_s=0.0, index=80)
+        inp = W.make_moe_inputs(cfg)
+        inp["bias"][:] = 0.0
+        inp["bias"][2] = -1000.0                          # expert 2: no task
+        inp["bias"][3] = -100.0                           # expert 3: only token 0, through input column 5
+        inp["x"][:, 5] = 0
+        inp["x"][0, 5] = 0x4180                           # bf16 16.0
+        inp["w_router"][3, :] = 0
+        inp["w_router"][3, 5] = 0x4280                    # bf16 64.0: logit 1024 - 100 for token 0, -100 for the rest
+    elif case == "pair_relu_top1":  # pair tiles, top-1 ReLU: the down epilogue writes the layer output
+        cfg = W.small_moe(T=2048, d=384, f=512, m=4, k=1, act=W.RELU, dtype=W.BF16, zipf_s=1.5, index=81)
+        inp = W.make_moe_inputs(cfg)
     else:  # the largest expert count and top-k the library accepts (m = 1024, k = 32)
         cfg = W.small_moe(T=700, d=64, f=64, m=1024, k=32, dtype=W.BF16, zipf_s=0.5, index=77)
         inp = W.make_moe_inputs(cfg)
     ref, _ = _check_layer(cfg, inp, n_sample=min(cfg.T, 64))
     if case.startswith("one_hot"):  # expert 11 holds every token: LIS reaches its maximum m / k
         assert ref["counts"][11] == cfg.T and ref["lis"] == cfg.m / cfg.k
+    if case == "pair_empty_and_single":
+        assert ref["counts"][2] == 0 and ref["counts"][3] == 1
 
 
 def test_workspace_reuse_is_stable():
