@@ -81,6 +81,10 @@ def parse():
     ap.add_argument("--fp8", action="store_true",
                     help="8-bit experts: E4M3 weights with per-channel scales (quantized once, untimed), "
                          "moe_layer_forward_fp8")
+    ap.add_argument("--global-lis", action="store_true",
+                    help="every step also sums the per-expert counts over all ranks (NCCL all-reduce of m int32) "
+                         "and takes the Load Imbalance Score of the whole job's batch (moe_lis_from_counts); "
+                         "routing.global_lis reports it")
     ap.add_argument("--router-only", action="store_true",
                     help="time the routing call alone (moe_route / moe_atomic_route) on the workload's inputs; "
                          "an auxiliary line for profiling, not the layer metric")
@@ -245,6 +249,15 @@ def rank_inputs(cfg, rank: int):
     if rank:
         inp["x"] = W.normal(cfg.seed(rank), W.STREAM["x"], (cfg.T, cfg.d), 1.0, cfg.dtype)
     return inp
+
+
+def global_histogram(counts, dist=None):
+    """Sum a rank's per-expert counts over all ranks, in place (identity on one rank):
+    the histogram of the whole job's batch, whose LIS is R&Q Definition 1 over every
+    rank's tokens together."""
+    if dist is not None and dist.is_initialized() and dist.get_world_size() > 1:
+        dist.all_reduce(counts, op=dist.ReduceOp.SUM)
+    return counts
 
 
 def max_over_ranks(values, dist=None, device=None):
@@ -509,6 +522,11 @@ def layer_run(cfg, args, dev, rank: int, world: int, dist, steps, warmup: int, w
     counts = torch.empty(cfg.m + (1 if rep else 0), dtype=torch.int32, device=dev)
     lis = moe.lis_buffer(dev)
     lis0 = moe.lis_buffer(dev)
+    glob = args.global_lis
+    if glob and (rep or floe is not None or fp8):
+        raise SystemExit("--global-lis runs the plain layer")
+    gcounts = torch.empty(cfg.m, dtype=torch.int32, device=dev)
+    glis = moe.lis_buffer(dev)
     s = torch.cuda.Stream(device=dev)
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
 
@@ -528,6 +546,10 @@ def layer_run(cfg, args, dev, rank: int, world: int, dist, steps, warmup: int, w
                                        w_down_t, thr, args_[10], ws, topk_idx_out=floe_idx, kept_out=kept, stream=s)
         else:
             moe.moe_layer_forward(*args_, counts_out=counts, lis_out=lis, stream=s)
+            if glob:  # the whole job's histogram and its LIS (an exchange of m int32 per step)
+                gcounts.copy_(counts)
+                global_histogram(gcounts, dist)
+                moe.moe_lis_from_counts(cfg.m, world * cfg.T * cfg.k, gcounts, glis, stream=s)
 
     with torch.cuda.stream(s):
         n0 = moe.moe_launch_count()
@@ -655,6 +677,11 @@ def layer_run(cfg, args, dev, rank: int, world: int, dist, steps, warmup: int, w
                                 float(kc.sum()) * 2 * cfg.d * 2 + Tk * cfg.f * 8 + Tk * cfg.d * 4)
         layer_bytes = (cfg.m * cfg.d + active * cfg.f * cfg.d + float(kc.sum()) * 2 * cfg.d) * 2 + 2 * T_bytes(cfg)
         extra["kept_channel_fraction"] = float(kc[kc > 0].mean() / cfg.f)
+    if glob:
+        gmx, gam, glv = moe.unpack_lis(glis)
+        extra["global_lis"] = {"lis": glv, "max_count": gmx, "heavy_hitter": gam, "ranks": world,
+                               "note": "per-expert counts summed over all ranks every step (all-reduce of m int32) "
+                                       "and the LIS of the whole job's batch; routing.lis is the rank's own"}
     if rep:
         extra["lis_before_split"] = moe.unpack_lis(lis0)[2]
         extra["heavy_hitter_before_split"] = moe.unpack_lis(lis0)[1]

@@ -131,6 +131,16 @@ MOE_API moe_status_t moe_route(const moe_config_t* cfg, const void* x, const voi
 MOE_API moe_status_t moe_histogram_lis(const moe_config_t* cfg, const int32_t* topk_idx, int32_t* counts, int32_t* offsets,
                                moe_lis_t* lis, void* ws, size_t ws_bytes, moe_stream_t stream);
 
+/* Load Imbalance Score of a given histogram (R&Q Definition 1): lis->max_count =
+ * max_j counts[j], lis->argmax_expert = the lowest j attaining it, lis->lis =
+ * m * max / tasks (one fp64 division). For a histogram that spans more than one
+ * call, e.g. the per-expert counts of every data-parallel rank's batch summed
+ * across ranks, where tasks = the summed T k. counts [m] int32 and lis are device
+ * pointers (counts 4-byte, lis 16-byte aligned); m in 1..1024 (MOE_ERR_UNSUPPORTED
+ * above), tasks >= 1; no workspace. */
+MOE_API moe_status_t moe_lis_from_counts(int32_t m, int64_t tasks, const int32_t* counts, moe_lis_t* lis,
+                                         moe_stream_t stream);
+
 /* Expert-centric permutation (OmniMoE Fig. 3). Task q = t k + s goes to
  * position pos = offsets[e] + (number of earlier tasks q' < q with the same
  * expert e): segments are contiguous and ordered by task id. Writes

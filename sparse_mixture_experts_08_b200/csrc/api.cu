@@ -492,6 +492,15 @@ moe_status_t moe_histogram_lis(const moe_config_t* cfg, const int32_t* topk_idx,
                                         at<int>(ws, L.status), (cudaStream_t)stream));
 }
 
+moe_status_t moe_lis_from_counts(int32_t m, int64_t tasks, const int32_t* counts, moe_lis_t* lis,
+                                 moe_stream_t stream) {
+  if (m < 1 || tasks < 1 || !counts || !lis) return MOE_ERR_INVALID_ARG;
+  if (m > 1024) return MOE_ERR_UNSUPPORTED;
+  if (((uintptr_t)counts & 3u) || !aligned16(lis)) return MOE_ERR_INVALID_ARG;
+  MOE_TRY(check_device());
+  return cuda_status(launch_lis_from_counts(m, (long long)tasks, counts, lis, (cudaStream_t)stream));
+}
+
 moe_status_t moe_permute(const moe_config_t* cfg, const void* x, const int32_t* topk_idx, const int32_t* offsets,
                          void* x_perm, int32_t* perm, int32_t* inv_perm, void* ws, size_t ws_bytes,
                          moe_stream_t stream) {

@@ -215,6 +215,8 @@ cudaError_t launch_route_scatter(int dtype, int T, int k, int m, int d, const in
                                  const int32_t* lrank, const float* task_w, const void* x, int32_t* counts,
                                  int32_t* offsets, moe_lis_t* lis, int32_t* perm, int32_t* inv_perm, float* w_perm,
                                  void* x_perm, int* status, cudaStream_t s);
+// max / argmax / LIS (R&Q Definition 1) of a given histogram counts[m] over `tasks` tasks.
+cudaError_t launch_lis_from_counts(int m, long long tasks, const int32_t* counts, moe_lis_t* lis, cudaStream_t s);
 // R&Q replica dispatch: tasks of the heavy-hitter (lis_in->argmax_expert) with an
 // odd rank in its segment go to expert m; writes idx_out, the group -> weight map
 // [m + 1] and, when given, counts [m + 1] and the LIS over m + 1 experts.

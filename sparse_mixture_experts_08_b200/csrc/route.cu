@@ -343,6 +343,62 @@ void route_ranges(int Tk, int m, int* R, int* L) {
   *R = (Tk + *L - 1) / *L;
 }
 
+// ------------------------------------------------ LIS of a given histogram
+// R&Q Definition 1 over counts that another step produced (e.g. the histogram of
+// every rank's batch, summed across ranks): max_j n_j, the lowest j attaining it,
+// and LIS = m max / tasks as one fp64 division. One block; counts are read once.
+__global__ void lis_from_counts_kernel(int m, long long tasks, const int32_t* __restrict__ counts,
+                                       moe_lis_t* __restrict__ lis) {
+  __shared__ int wmax[32], warg[32];
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  pdl_launch_dependents();
+  pdl_wait();
+  int mv = -1, ma = 0x7fffffff;
+  for (int e = tid; e < m; e += blockDim.x) {  // ascending e per thread: a strict > keeps the lowest
+    const int c = counts[e];
+    if (c > mv) {
+      mv = c;
+      ma = e;
+    }
+  }
+#pragma unroll
+  for (int o = 16; o; o >>= 1) {
+    const int ov = __shfl_xor_sync(FULL, mv, o), oa = __shfl_xor_sync(FULL, ma, o);
+    if (ov > mv || (ov == mv && oa < ma)) {
+      mv = ov;
+      ma = oa;
+    }
+  }
+  if (lane == 0) {
+    wmax[warp] = mv;
+    warg[warp] = ma;
+  }
+  __syncthreads();
+  if (warp == 0) {
+    const int nw = blockDim.x >> 5;
+    int bv = lane < nw ? wmax[lane] : -1, ba = lane < nw ? warg[lane] : 0x7fffffff;
+#pragma unroll
+    for (int o = 16; o; o >>= 1) {
+      const int ov = __shfl_xor_sync(FULL, bv, o), oa = __shfl_xor_sync(FULL, ba, o);
+      if (ov > bv || (ov == bv && oa < ba)) {
+        bv = ov;
+        ba = oa;
+      }
+    }
+    if (lane == 0) {
+      lis->max_count = bv;
+      lis->argmax_expert = ba;
+      lis->lis = (double)((long long)m * bv) / (double)tasks;
+    }
+  }
+}
+
+cudaError_t launch_lis_from_counts(int m, long long tasks, const int32_t* counts, moe_lis_t* lis, cudaStream_t s) {
+  launch_k(lis_from_counts_kernel, 1, 1024, 0, s, m, tasks, counts, lis);
+  count_launch();
+  return cudaGetLastError();
+}
+
 cudaError_t launch_route_index(int mode, int T, int k, int m, const int32_t* idx, int32_t* counts, int32_t* offsets,
                                moe_lis_t* lis, int32_t* start, int* status, cudaStream_t s) {
   int R, L;

@@ -29,7 +29,7 @@ STATUS_NAMES = {0: "MOE_OK", 1: "MOE_ERR_INVALID_ARG", 2: "MOE_ERR_UNSUPPORTED",
 # every symbol include/moe.h declares
 EXPORTS = ["moe_workspace_size", "moe_atomic_workspace_size", "moe_route", "moe_histogram_lis", "moe_permute",
            "moe_grouped_ffn", "moe_shared_ffn", "moe_combine", "moe_layer_forward", "moe_atomic_route",
-           "moe_atomic_experts", "moe_atomic_forward", "moe_read_device_status", "moe_status_string",
+           "moe_atomic_experts", "moe_atomic_forward", "moe_lis_from_counts", "moe_read_device_status", "moe_status_string",
            "moe_debug_set_wait_limit_ns", "moe_debug_set_barrier_extra", "moe_set_stage_events", "moe_launch_count", "moe_route_static",
            "moe_replica_split", "moe_layer_forward_replicated", "moe_floe_pack_down", "moe_floe_calibrate",
            "moe_floe_workspace_size", "moe_layer_forward_floe", "moe_quantize_e4m3", "moe_fp8_workspace_size",
@@ -79,6 +79,7 @@ def lib() -> ctypes.CDLL:
             "moe_route": [P, P, P, P, P, P, P, P, P, S, P],
             "moe_histogram_lis": [P, P, P, P, P, P, S, P],
             "moe_permute": [P, P, P, P, P, P, P, P, S, P],
+            "moe_lis_from_counts": [ctypes.c_int32, ctypes.c_int64, P, P, P],
             "moe_grouped_ffn": [P, P, P, P, P, P, P, P, P, P, S, P],
             "moe_shared_ffn": [P, P, P, P, P, P, P, S, P],
             "moe_combine": [P, P, P, P, P, P],
@@ -175,6 +176,11 @@ def moe_route_static(cfg, x, w_router, bias, logits_in, logits_out, topk_idx, to
 def moe_histogram_lis(cfg, topk_idx, counts, offsets, lis, ws, stream=None):
     _check("moe_histogram_lis", lib().moe_histogram_lis(ctypes.byref(cfg), _p(topk_idx), _p(counts), _p(offsets),
                                                         _p(lis), _p(ws), ws.numel(), _stream(stream)))
+
+
+def moe_lis_from_counts(m, tasks, counts, lis, stream=None):
+    _check("moe_lis_from_counts", lib().moe_lis_from_counts(int(m), int(tasks), _p(counts), _p(lis),
+                                                            _stream(stream)))
 
 
 def moe_permute(cfg, x, topk_idx, offsets, x_perm, perm, inv_perm, ws, stream=None):

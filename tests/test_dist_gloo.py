@@ -48,7 +48,10 @@ def _worker(rank, world, port, q):
         outs = [None] * world
         dist.all_gather_object(outs, (inp["x"], out, out8))
         mx = bench.max_over_ranks([float(rank + 1), 10.0 - rank], dist)
-        q.put((rank, hashes, outs, mx))
+        # the whole job's histogram (bench --global-lis): each rank's counts summed
+        routed = O.layer_forward(cfg, inp)
+        summed = bench.global_histogram(torch.from_numpy(routed["counts"].copy()), dist).numpy()
+        q.put((rank, hashes, outs, mx, summed))
     finally:
         dist.destroy_process_group()
 
@@ -75,7 +78,7 @@ def test_ranks_share_weights_and_own_their_batch(two_ranks):
 
 
 def test_max_over_ranks(two_ranks):
-    for _, _, _, mx in two_ranks:
+    for _, _, _, mx, _ in two_ranks:
         assert mx == [2.0, 10.0]
 
 
@@ -109,3 +112,26 @@ def test_token_sharding_leaves_8bit_outputs_unchanged(two_ranks):
     inp["x"] = np.concatenate([outs[0][0], outs[1][0]])
     whole = O.layer_forward_fp8(cfg, inp)["out"]
     np.testing.assert_allclose(whole, np.concatenate([outs[0][2], outs[1][2]]), rtol=1e-12, atol=0)
+
+
+def test_global_histogram_is_the_whole_batch_histogram(two_ranks):
+    """R&Q Definition 1 over the whole job's batch: the per-expert counts summed over
+    the two ranks equal the oracle's histogram of the two batches together, and the
+    LIS of that histogram (what moe_lis_from_counts computes from it on the GPU) is
+    the oracle's LIS of the concatenated routing."""
+    import sys
+
+    sys.path.insert(0, ROOT)
+    import oracle as O
+    import workloads as W
+
+    cfg = W.small_moe(T=48, d=64, f=96, m=6, k=2, dtype=W.BF16, zipf_s=1.0, index=41, name="dp_small")
+    outs = two_ranks[0][2]
+    inp = W.make_moe_inputs(cfg, replicate=0)
+    inp["x"] = np.concatenate([outs[0][0], outs[1][0]])
+    whole = O.layer_forward(cfg, inp)
+    for r in range(2):
+        np.testing.assert_array_equal(two_ranks[r][4], whole["counts"])
+    c = two_ranks[0][4]
+    assert whole["max_count"] == int(c.max()) and whole["argmax"] == int(np.argmax(c))
+    assert whole["lis"] == cfg.m * int(c.max()) / (cfg.T * cfg.k)

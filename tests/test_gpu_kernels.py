@@ -126,6 +126,32 @@ def test_histogram_lis_bit_exact(T, m, k, pattern):
     assert lis == ref["lis"]  # one correctly rounded fp64 division on both sides
 
 
+def test_lis_from_counts_of_two_batches_is_the_whole_batch_lis():
+    """The job-wide LIS (bench --global-lis): two batches' histograms from the GPU,
+    summed as the all-reduce across ranks sums them, then moe_lis_from_counts; equal
+    to the oracle's max, argmax and LIS of the two routings taken together."""
+    m, k = 64, 6
+    rng = np.random.default_rng(12)
+    p = 1.0 / np.arange(1, m + 1) ** 1.2
+    batches = [np.stack([rng.choice(m, size=k, replace=False, p=p / p.sum()) for _ in range(T)]).astype(np.int32)
+               for T in (300, 517)]
+    total = torch.zeros(m, dtype=torch.int32, device="cuda")
+    for idx in batches:
+        cfg = W.small_moe(T=idx.shape[0], d=64, f=64, m=m, k=k)
+        st, counts, _, _ = _hist(cfg, idx)
+        assert st == moe.OK
+        total += dev(counts)
+    lis = moe.lis_buffer()
+    moe.moe_lis_from_counts(m, sum(b.shape[0] for b in batches) * k, total, lis)
+    ref = O.histogram_lis(np.concatenate(batches), m)
+    assert moe.unpack_lis(lis) == (ref["max_count"], ref["argmax"], ref["lis"])
+    # equal maxima: the lowest expert index, as in moe_histogram_lis
+    tied = torch.zeros(m, dtype=torch.int32, device="cuda")
+    tied[[5, 40, 63]] = 9
+    moe.moe_lis_from_counts(m, 27, tied, lis)
+    assert moe.unpack_lis(lis) == (9, 5, m * 9 / 27)
+
+
 def test_histogram_rejects_bad_expert_id_without_writing():
     cfg = W.small_moe(T=10, d=64, f=64, m=8, k=2)
     idx = np.tile(np.array([1, 2], np.int32), (10, 1))
