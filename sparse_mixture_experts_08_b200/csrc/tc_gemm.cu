@@ -336,9 +336,10 @@ __device__ __forceinline__ void route_pass(uint32_t t_row, int m, const float* r
 
 // The router epilogue for m <= 128 experts: a token's m logits are read from TMEM
 // once (eight loads, one wait) and kept in registers for all k passes. Pass s takes
-// the largest logit strictly after pick s - 1 in (logit desc, expert asc): four
-// compare chains over interleaved columns (each keeps its first maximum, columns
-// ascending), merged with ties to the lower expert. The softmax denominator is the
+// the largest logit strictly after pick s - 1 in (logit desc, expert asc), by 32-wide
+// pairwise trees whose left side holds the lower experts, merged in column order
+// (trees keep the dependency chains short: one warp per SM sub-partition runs
+// this epilogue, so latency, not issue, bounds it). The softmax denominator is the
 // fp64 sum, per 32 columns, of fp32 partial sums of exp(logit - max), the max being
 // pick 0. Picks stay in registers (k <= 8).
 constexpr int ROUTE_REG_M = 128;
@@ -353,25 +354,34 @@ __device__ __forceinline__ void tmem_ld_x16f(uint32_t taddr, float* r) {
 
 template <int RM>
 __device__ __forceinline__ void route_best_after(const float (&v)[RM], int m, float pv, int pe, float& bv, int& be) {
-  float cb[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
-  int ci[4] = {-1, -1, -1, -1};
+  bv = -INFINITY;
+  be = -1;
 #pragma unroll
-  for (int j = 0; j < RM; ++j) {
-    const float x = v[j];
-    const bool after = x < pv || (x == pv && j > pe);
-    if (j < m && after && x > cb[j & 3]) {  // strict: the chain keeps its lowest column among equals
-      cb[j & 3] = x;
-      ci[j & 3] = j;
+  for (int c0 = 0; c0 < RM; c0 += 32) {
+    if (c0 >= m) break;
+    constexpr int W = RM < 32 ? RM : 32;
+    float cv[W];
+    int ce[W];
+#pragma unroll
+    for (int j = 0; j < W; ++j) {
+      const float x = v[c0 + j];
+      const bool after = x < pv || (x == pv && c0 + j > pe);
+      cv[j] = (c0 + j < m && after) ? x : -INFINITY;
+      ce[j] = c0 + j;
+    }
+#pragma unroll
+    for (int st = 1; st < W; st <<= 1)
+#pragma unroll
+      for (int j = 0; j < W; j += 2 * st)
+        if (cv[j + st] > cv[j]) {  // an equal logit keeps the lower expert (left)
+          cv[j] = cv[j + st];
+          ce[j] = ce[j + st];
+        }
+    if (cv[0] > bv) {  // earlier chunks hold lower experts
+      bv = cv[0];
+      be = ce[0];
     }
   }
-  bv = cb[0];
-  be = ci[0];
-#pragma unroll
-  for (int i = 1; i < 4; ++i)
-    if (cb[i] > bv || (cb[i] == bv && ci[i] >= 0 && (be < 0 || ci[i] < be))) {
-      bv = cb[i];
-      be = ci[i];
-    }
 }
 
 // ------------------------------------------------------------------ tile schedule
