@@ -218,6 +218,27 @@ __device__ __forceinline__ void tmem_ld_x16(uint32_t taddr, uint32_t* r) {
       : "r"(taddr));
 }
 __device__ __forceinline__ void tmem_ld_wait() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
+// Waits for this thread's TMEM loads, naming the registers they fill as read-write
+// operands: the compiler then reads them only after the wait, even when other loads
+// were issued in between (the epilogue keeps the next chunk's load in flight).
+__device__ __forceinline__ void tmem_ld_wait_keep(uint32_t (&r)[16]) {
+  asm volatile("tcgen05.wait::ld.sync.aligned;"
+               : "+r"(r[0]), "+r"(r[1]), "+r"(r[2]), "+r"(r[3]), "+r"(r[4]), "+r"(r[5]), "+r"(r[6]), "+r"(r[7]),
+                 "+r"(r[8]), "+r"(r[9]), "+r"(r[10]), "+r"(r[11]), "+r"(r[12]), "+r"(r[13]), "+r"(r[14]),
+                 "+r"(r[15])
+               :
+               : "memory");
+}
+__device__ __forceinline__ void tmem_ld_wait_keep(uint32_t (&r)[16], uint32_t (&u)[16]) {
+  asm volatile("tcgen05.wait::ld.sync.aligned;"
+               : "+r"(r[0]), "+r"(r[1]), "+r"(r[2]), "+r"(r[3]), "+r"(r[4]), "+r"(r[5]), "+r"(r[6]), "+r"(r[7]),
+                 "+r"(r[8]), "+r"(r[9]), "+r"(r[10]), "+r"(r[11]), "+r"(r[12]), "+r"(r[13]), "+r"(r[14]),
+                 "+r"(r[15]), "+r"(u[0]), "+r"(u[1]), "+r"(u[2]), "+r"(u[3]), "+r"(u[4]), "+r"(u[5]), "+r"(u[6]),
+                 "+r"(u[7]), "+r"(u[8]), "+r"(u[9]), "+r"(u[10]), "+r"(u[11]), "+r"(u[12]), "+r"(u[13]),
+                 "+r"(u[14]), "+r"(u[15])
+               :
+               : "memory");
+}
 
 // Shared-memory matrix descriptor: K-major operand, 128-byte swizzle, rows of
 // 128 B, 8-row core groups 1024 B apart (SBO), descriptor version 1 (sm_100).
@@ -928,12 +949,8 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
       }
       tc_fence_after();
       const uint32_t t_row = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * S::ACC_COLS);
-#pragma unroll 1
-      for (int c0 = 0; c0 < ti.rows_in_tile; c0 += 16) {
-        uint32_t r0[16], r1[16];
-        tmem_ld_x16(t_row + c0, r0);
-        if (MATS == 2) tmem_ld_x16(t_row + BN + c0, r1);
-        tmem_ld_wait();
+      // One 16-row chunk of accumulator columns (r0: gate or the single matrix, r1: up).
+      auto chunk = [&](const int c0, const uint32_t (&r0)[16], const uint32_t (&r1)[16]) {
         const int jn = min(16, ti.rows_in_tile - c0);
         if (VEC) {
 #pragma unroll
@@ -984,6 +1001,33 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
           for (int j = 0; j < 16; ++j)
             if (j < jn) store_logit(c, ti, feature, c0 + j, (has_k ? __uint_as_float(r0[j]) : 0.f) + bias);
         }
+        __syncwarp();
+      };
+      // The loads of chunk i + 1 are in flight while chunk i is computed and stored
+      // (two register buffers; the loop body takes the even chunk, then the odd one).
+      const int rows = ti.rows_in_tile;
+      uint32_t ra0[16], ra1[16], rb0[16], rb1[16];
+#pragma unroll
+      for (int j = 0; j < 16; ++j) ra1[j] = rb1[j] = 0u;
+      if (rows > 0) {
+        tmem_ld_x16(t_row, ra0);
+        if (MATS == 2) tmem_ld_x16(t_row + BN, ra1);
+      }
+#pragma unroll 1
+      for (int c0 = 0; c0 < rows; c0 += 32) {
+        if (MATS == 2) tmem_ld_wait_keep(ra0, ra1); else tmem_ld_wait_keep(ra0);
+        if (c0 + 16 < rows) {
+          tmem_ld_x16(t_row + c0 + 16, rb0);
+          if (MATS == 2) tmem_ld_x16(t_row + BN + c0 + 16, rb1);
+        }
+        chunk(c0, ra0, ra1);
+        if (c0 + 16 >= rows) break;
+        if (MATS == 2) tmem_ld_wait_keep(rb0, rb1); else tmem_ld_wait_keep(rb0);
+        if (c0 + 32 < rows) {
+          tmem_ld_x16(t_row + c0 + 32, ra0);
+          if (MATS == 2) tmem_ld_x16(t_row + BN + c0 + 32, ra1);
+        }
+        chunk(c0 + 16, rb0, rb1);
       }
       tc_fence_before();
       __syncwarp();
