@@ -223,6 +223,43 @@ static moe_status_t run_router(const moe_config_t& c, const void* x, const void*
   return cuda_status(launch_router_logits(c, x, w_r, bias, logits, status, s));
 }
 
+// Everything moe_route computes on the device: logits (from x, or logits_in
+// verbatim), top-k ids and gate weights, by the kernels that suit the batch.
+// logits_out receives the logits when given; otherwise logits_scratch holds them
+// where a kernel needs them in memory. With stage_marks, stage events 1 (logits)
+// and 2 (top-k) are recorded (together when one kernel does both).
+cudaError_t launch_route(const moe_config_t& c, const void* x, const void* w_r, const float* bias,
+                         const float* logits_in, float* logits_out, float* logits_scratch, int32_t* idx, float* w,
+                         int* status, cudaStream_t s, bool stage_marks) {
+  cudaError_t e = cudaSuccess;
+  const float* lg = logits_in;
+  if (!lg && fused_route_ok(c)) {  // logits and top-k in one tensor-core launch
+    e = launch_route_topk(c, x, w_r, bias, logits_out, idx, w, nullptr, nullptr, status, g_wait_limit_ns, s);
+    if (e == cudaSuccess && stage_marks) e = mark_stage_event(1, s);
+    if (e == cudaSuccess && stage_marks) e = mark_stage_event(2, s);
+    return e;
+  }
+  if (!lg && small_route_ok(c.dtype, c.m)) {  // few experts: logits and top-k in one CUDA-core launch
+    e = launch_small_route(c.T, c.d, c.m, c.k, c.renormalize, x, w_r, bias, logits_out, idx, w, s);
+    if (e == cudaSuccess && stage_marks) e = mark_stage_event(1, s);
+    if (e == cudaSuccess && stage_marks) e = mark_stage_event(2, s);
+    return e;
+  }
+  if (!lg) {
+    float* dst = logits_out ? logits_out : logits_scratch;
+    if ((e = launch_router_logits(c, x, w_r, bias, dst, status, s)) != cudaSuccess) return e;
+    lg = dst;
+  } else if (logits_out && logits_out != logits_in) {
+    if ((e = cudaMemcpyAsync(logits_out, logits_in, (size_t)c.T * c.m * 4, cudaMemcpyDeviceToDevice, s)) !=
+        cudaSuccess)
+      return e;
+  }
+  if (stage_marks && (e = mark_stage_event(1, s)) != cudaSuccess) return e;
+  if ((e = launch_topk_softmax(c.T, c.m, c.k, c.renormalize, lg, idx, w, s)) != cudaSuccess) return e;
+  if (stage_marks) e = mark_stage_event(2, s);
+  return e;
+}
+
 // 8-bit expert path: the quantized weights and the per-row codes and scales of
 // each projection's input (x_perm rows, h rows, and for shared experts x and h_sh).
 struct Fp8Io {
@@ -462,20 +499,8 @@ moe_status_t moe_route(const moe_config_t* cfg, const void* x, const void* w_rou
     if (p && !aligned16(p)) return MOE_ERR_INVALID_ARG;
   MOE_TRY(check_ws(c, ws, ws_bytes, L.logits + align256((size_t)c.T * c.m * 4)));
   MOE_TRY(check_device());
-  cudaStream_t s = (cudaStream_t)stream;
-  int* status = at<int>(ws, L.status);
-  const float* lg = logits_in;
-  if (!lg && fused_route_ok(c))  // logits and top-k in one tensor-core launch
-    return cuda_status(launch_route_topk(c, x, w_router, bias, logits_out, topk_idx, topk_w, nullptr, nullptr, status,
-                                         g_wait_limit_ns, s));
-  if (!lg) {
-    float* dst = logits_out ? logits_out : at<float>(ws, L.logits);
-    MOE_TRY(run_router(c, x, w_router, bias, dst, status, s));
-    lg = dst;
-  } else if (logits_out && logits_out != logits_in) {
-    MOE_CUDA(cudaMemcpyAsync(logits_out, logits_in, (size_t)c.T * c.m * 4, cudaMemcpyDeviceToDevice, s));
-  }
-  return cuda_status(launch_topk_softmax(c.T, c.m, c.k, c.renormalize, lg, topk_idx, topk_w, s));
+  return cuda_status(launch_route(c, x, w_router, bias, logits_in, logits_out, at<float>(ws, L.logits), topk_idx,
+                                  topk_w, at<int>(ws, L.status), (cudaStream_t)stream, false));
 }
 
 moe_status_t moe_histogram_lis(const moe_config_t* cfg, const int32_t* topk_idx, int32_t* counts, int32_t* offsets,
@@ -658,10 +683,7 @@ static moe_status_t layer_forward_impl(const moe_config_t& c, const void* x, con
     MOE_CUDA(launch_route_scatter(c.dtype, c.T, c.k, c.m, c.d, tile_cnt, idx, lrank, w, x, counts, offsets, lis, perm,
                                   inv_perm, w_perm, at<void>(ws, L.x_perm), status, s));
   } else {
-    MOE_TRY(run_router(c, x, w_router, bias, logits, status, s));
-    MOE_TRY(mark_stage(1, s));
-    MOE_CUDA(launch_topk_softmax(c.T, c.m, c.k, c.renormalize, logits, idx, w, s));
-    MOE_TRY(mark_stage(2, s));
+    MOE_CUDA(launch_route(c, x, w_router, bias, nullptr, logits_out, logits, idx, w, status, s, true));
     int32_t* start = at<int32_t>(ws, L.start);
     MOE_CUDA(launch_route_index(1, c.T, c.k, c.m, idx, counts, offsets, lis, start, status, s));
     MOE_CUDA(launch_rank(c.T, c.k, c.m, idx, offsets, start, w, perm, inv_perm, w_perm, status, s));
@@ -869,6 +891,16 @@ static moe_status_t atomic_route_impl(const moe_atomic_config_t& c, const Atomic
   int* status = at<int>(ws, P.status);
   float* zr = at<float>(ws, P.zr);
   float* zc = at<float>(ws, P.zc);
+  if (atomic_proj_ok(c.T, c.d)) {
+    // decode budgets: one CUDA-core pass writes the final logits (the tensor-core
+    // tile would hold at most 16 of its 128 token rows and need split-K partials)
+    MOE_CUDA(launch_atomic_proj(c.T, c.d, c.Nr, c.Nc, x, w_row, w_col, zr, zc, s));
+    if (stage_marks) MOE_TRY(mark_stage(1, s));
+    MOE_CUDA(launch_atomic_select(c.T, c.Nr, c.Nc, c.K, 1, zr, (long long)c.T * c.Nr, zc, (long long)c.T * c.Nc,
+                                  lr_out, lc_out, idx, g, status, at<unsigned>(ws, P.bar), s));
+    if (stage_marks) MOE_TRY(mark_stage(2, s));
+    return MOE_OK;
+  }
   GemmParams p;
   std::memset(&p, 0, sizeof(p));
   fill_common(p, status);
@@ -1023,16 +1055,7 @@ moe_status_t moe_layer_forward_replicated(const moe_config_t* cfg, const void* x
 
   // 1. router and top-k over the m experts (stage events as in moe_layer_forward)
   MOE_TRY(mark_stage(0, s));
-  if (fused_route_ok(c)) {
-    MOE_CUDA(launch_route_topk(c, x, w_router, bias, logits_out, idx, w, nullptr, nullptr, status, g_wait_limit_ns,
-                               s));
-    MOE_TRY(mark_stage(1, s));
-  } else {
-    MOE_TRY(run_router(c, x, w_router, bias, logits, status, s));
-    MOE_TRY(mark_stage(1, s));
-    MOE_CUDA(launch_topk_softmax(c.T, c.m, c.k, c.renormalize, logits, idx, w, s));
-  }
-  MOE_TRY(mark_stage(2, s));
+  MOE_CUDA(launch_route(c, x, w_router, bias, nullptr, logits_out, logits, idx, w, status, s, true));
   // 2. histogram / LIS and the stable ranks over the m experts (the heavy-hitter's
   //    segment order is the split order)
   MOE_CUDA(launch_route_index(1, c.T, c.k, c.m, idx, counts, offsets, lis0, start, status, s));
@@ -1200,10 +1223,7 @@ moe_status_t moe_layer_forward_floe(const moe_config_t* cfg, const void* x, cons
   const long long Tk = (long long)c.T * c.k;
   // route and sort as in moe_layer_forward (stages 0-4)
   MOE_TRY(mark_stage(0, s));
-  MOE_TRY(run_router(c, x, w_router, bias, logits, status, s));
-  MOE_TRY(mark_stage(1, s));
-  MOE_CUDA(launch_topk_softmax(c.T, c.m, c.k, c.renormalize, logits, idx, w, s));
-  MOE_TRY(mark_stage(2, s));
+  MOE_CUDA(launch_route(c, x, w_router, bias, nullptr, nullptr, logits, idx, w, status, s, true));
   MOE_CUDA(launch_route_index(1, c.T, c.k, c.m, idx, at<int32_t>(ws, L.counts), offsets, at<moe_lis_t>(ws, L.lis),
                               start, status, s));
   MOE_CUDA(launch_rank(c.T, c.k, c.m, idx, offsets, start, w, perm, inv_perm, w_perm, status, s));

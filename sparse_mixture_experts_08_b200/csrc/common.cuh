@@ -189,6 +189,12 @@ cudaError_t launch_router_logits(const moe_config_t& c, const void* x, const voi
                                  float* logits, int* status, cudaStream_t s);
 // The current time limit of the bounded waits (moe_debug_set_wait_limit_ns).
 unsigned long long wait_limit_ns();
+// moe_route's device work (logits, top-k, gate weights) by the kernels that suit the
+// batch; logits_scratch (T m floats) serves when logits_out is NULL and a kernel
+// needs the logits in memory.
+cudaError_t launch_route(const moe_config_t& c, const void* x, const void* w_r, const float* bias,
+                         const float* logits_in, float* logits_out, float* logits_scratch, int32_t* idx, float* w,
+                         int* status, cudaStream_t s, bool stage_marks);
 
 // SIMT grouped linear (fp32 or bf16 inputs, fp32 math), same GemmParams.
 cudaError_t launch_simt_gemm(int epi, int dtype, const GemmParams& p, int max_rows_per_group, cudaStream_t s);
@@ -202,6 +208,10 @@ cudaError_t launch_few_expert_logits(int T, int d, int m, const void* x, const v
                                      float* logits, cudaStream_t s);
 cudaError_t launch_topk_softmax(int T, int m, int k, int renorm, const float* logits, int32_t* idx, float* w,
                                 cudaStream_t s);
+// logits (nullable), top-k ids and gate weights in one launch: bf16 layers with m <= 16.
+bool small_route_ok(int dtype, int m);
+cudaError_t launch_small_route(int T, int d, int m, int k, int renorm, const void* x, const void* w, const float* bias,
+                               float* logits, int32_t* idx, float* wout, cudaStream_t s);
 // Stable counting sort of the tasks by expert: route_index (one block: per-range
 // counts, offsets when mode & 1 (plus counts and LIS), range start positions
 // `start` [R][m], R * (m + 1) <= 8192) and rank (one warp per range: perm,

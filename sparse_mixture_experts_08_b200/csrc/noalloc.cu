@@ -23,8 +23,8 @@
 //  - The first call on each device looks up the array's device address with
 //    cudaGetSymbolAddress (with that device current); make that first call
 //    before starting any stream capture.
-//  - The kernels are the ones moe_route launches (the same choice of router
-//    kernel, the same bounded-wait limit), so both give identical results.
+//  - The device work is moe_route's (one shared launcher: the same choice of
+//    router kernels, the same bounded-wait limit), so both give identical results.
 #include <initializer_list>
 
 #include "common.cuh"
@@ -95,25 +95,10 @@ extern "C" MOE_API moe_status_t moe_route_static(const moe_config_t* cfg, const 
   cudaStream_t s = (cudaStream_t)stream;
   int* status = reinterpret_cast<int*>(scratch);
   if (cudaMemsetAsync(status, 0, sizeof(int), s) != cudaSuccess) return MOE_ERR_CUDA;
-  const float* lg = logits_in;
-  if (!lg && fused_route_ok(c)) {  // the same kernel choice as moe_route: logits + top-k in one launch
-    if (launch_route_topk(c, x, w_router, bias, logits_out, topk_idx, topk_w, nullptr, nullptr, status,
-                          wait_limit_ns(), s) != cudaSuccess)
-      return MOE_ERR_CUDA;
-    if (device_status_out &&
-        cudaMemcpyAsync(device_status_out, status, sizeof(int32_t), cudaMemcpyDeviceToDevice, s) != cudaSuccess)
-      return MOE_ERR_CUDA;
-    return MOE_OK;
-  }
-  if (!lg) {
-    float* dst = logits_out ? logits_out : reinterpret_cast<float*>(scratch + STATIC_STATUS_BYTES);
-    if (launch_router_logits(c, x, w_router, bias, dst, status, s) != cudaSuccess) return MOE_ERR_CUDA;
-    lg = dst;
-  } else if (logits_out && logits_out != logits_in) {
-    if (cudaMemcpyAsync(logits_out, logits_in, logits_bytes, cudaMemcpyDeviceToDevice, s) != cudaSuccess)
-      return MOE_ERR_CUDA;
-  }
-  if (launch_topk_softmax(c.T, c.m, c.k, c.renormalize, lg, topk_idx, topk_w, s) != cudaSuccess) return MOE_ERR_CUDA;
+  if (launch_route(c, x, w_router, bias, logits_in, logits_out,
+                   reinterpret_cast<float*>(scratch + STATIC_STATUS_BYTES), topk_idx, topk_w, status, s,
+                   false) != cudaSuccess)
+    return MOE_ERR_CUDA;
   if (device_status_out &&
       cudaMemcpyAsync(device_status_out, status, sizeof(int32_t), cudaMemcpyDeviceToDevice, s) != cudaSuccess)
     return MOE_ERR_CUDA;

@@ -127,6 +127,150 @@ cudaError_t launch_few_expert_logits(int T, int d, int m, const void* x, const v
   return cudaGetLastError();
 }
 
+// ------------------------------------------------------------------ router for few experts, any batch
+// Logits, top-k and gate weights in one launch for bf16 layers with m <= 16 experts
+// (R&Q's token-choice routing over a Mixtral-like expert count). One block of
+// SR_THREADS per SR_VALUES / M tokens: thread i owns the 16-byte chunks i, i +
+// SR_THREADS, ... of the model dimension, loads those chunks of every expert's
+// router row once and applies them to each of the block's tokens (fp32 FMAs, chunks
+// in ascending order). The SR_VALUES partial sums per thread are reduced by a
+// shuffle reduce-scatter in each warp (lane L ends with values 2L and 2L + 1) and
+// then over the warps in warp order; the logit gets its bias. Then one thread per
+// token takes the top-k by (logit desc, expert asc) and the gate weights as
+// topk_softmax_kernel does: exp in fp32 of l - max, sums in fp64, renormalised over
+// the k chosen when asked. Every sum has a fixed order: the result does not depend
+// on timing.
+constexpr int SR_THREADS = 256, SR_VALUES = 64;
+
+template <int M>
+__global__ void __launch_bounds__(SR_THREADS)
+    small_route_kernel(int T, int d, int m, int k, int renorm, const uint4* __restrict__ x,
+                       const uint4* __restrict__ w, const float* __restrict__ bias, float* __restrict__ logits,
+                       int32_t* __restrict__ idx, float* __restrict__ wout) {
+  constexpr int TB = SR_VALUES / M;  // tokens per block
+  __shared__ float red[SR_THREADS / 32][SR_VALUES];
+  __shared__ float lg[TB][M];
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int chunks = d / 8;
+  const long long t0 = (long long)blockIdx.x * TB;
+  pdl_launch_dependents();
+  pdl_wait();
+  float acc[TB][M];
+#pragma unroll
+  for (int t = 0; t < TB; ++t)
+#pragma unroll
+    for (int e = 0; e < M; ++e) acc[t][e] = 0.f;
+  for (int c = tid; c < chunks; c += SR_THREADS) {
+    uint4 wv[M];
+#pragma unroll
+    for (int e = 0; e < M; ++e) wv[e] = e < m ? w[(long long)e * chunks + c] : make_uint4(0u, 0u, 0u, 0u);
+#pragma unroll
+    for (int t = 0; t < TB; ++t) {
+      if (t0 + t >= T) break;
+      const uint4 xv = x[(t0 + t) * chunks + c];
+      const __nv_bfloat162* xh = reinterpret_cast<const __nv_bfloat162*>(&xv);
+#pragma unroll
+      for (int e = 0; e < M; ++e) {
+        const __nv_bfloat162* wh = reinterpret_cast<const __nv_bfloat162*>(&wv[e]);
+        float a = acc[t][e];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const float2 xf = __bfloat1622float2(xh[u]), wf = __bfloat1622float2(wh[u]);
+          a = fmaf(xf.x, wf.x, a);
+          a = fmaf(xf.y, wf.y, a);
+        }
+        acc[t][e] = a;
+      }
+    }
+  }
+  // reduce-scatter over the warp: value index v = t M + e; lane L keeps 2L, 2L + 1
+  float* v = &acc[0][0];
+#pragma unroll
+  for (int half = SR_VALUES / 2, bit = 16; half >= 2; half >>= 1, bit >>= 1) {
+    const bool upper = (lane & bit) != 0;
+#pragma unroll
+    for (int i = 0; i < half; ++i) {
+      const float keep = upper ? v[half + i] : v[i];
+      const float send = upper ? v[i] : v[half + i];
+      v[i] = keep + __shfl_xor_sync(FULL, send, bit);
+    }
+  }
+  red[warp][2 * lane] = v[0];
+  red[warp][2 * lane + 1] = v[1];
+  __syncthreads();
+  if (tid < SR_VALUES) {
+    const int t = tid / M, e = tid % M;
+    float sum = 0.f;
+#pragma unroll
+    for (int w8 = 0; w8 < SR_THREADS / 32; ++w8) sum += red[w8][tid];
+    if (e < m) {
+      sum += bias ? bias[e] : 0.f;
+      lg[t][e] = sum;
+      if (logits && t0 + t < T) logits[(t0 + t) * m + e] = sum;
+    }
+  }
+  __syncthreads();
+  if (tid < TB && t0 + tid < T) {
+    const float* L = lg[tid];
+    int sel_e[M];
+    float sel_v[M];
+#pragma unroll
+    for (int s2 = 0; s2 < M; ++s2) {
+      if (s2 >= k) break;
+      float bv = 0.f;
+      int be = -1;
+#pragma unroll
+      for (int e = 0; e < M; ++e) {
+        if (e >= m) break;
+        bool taken = false;
+#pragma unroll
+        for (int j = 0; j < M; ++j)
+          if (j < s2) taken |= sel_e[j] == e;
+        if (!taken && (be < 0 || L[e] > bv)) {  // ascending e: a tie keeps the lower expert
+          bv = L[e];
+          be = e;
+        }
+      }
+      sel_e[s2] = be;
+      sel_v[s2] = bv;
+    }
+    const float mx = sel_v[0];
+    double z = 0.0;
+#pragma unroll
+    for (int e = 0; e < M; ++e)
+      if (e < m) z += (double)expf(L[e] - mx);
+    double sel = 0.0;
+#pragma unroll
+    for (int s2 = 0; s2 < M; ++s2)
+      if (s2 < k) sel += (double)expf(sel_v[s2] - mx) / z;
+#pragma unroll
+    for (int s2 = 0; s2 < M; ++s2) {
+      if (s2 >= k) break;
+      double pr = (double)expf(sel_v[s2] - mx) / z;
+      if (renorm) pr /= sel;
+      idx[(t0 + tid) * k + s2] = sel_e[s2];
+      wout[(t0 + tid) * k + s2] = (float)pr;
+    }
+  }
+}
+
+bool small_route_ok(int dtype, int m) { return dtype == MOE_BF16 && m <= 16; }
+
+cudaError_t launch_small_route(int T, int d, int m, int k, int renorm, const void* x, const void* w, const float* bias,
+                               float* logits, int32_t* idx, float* wout, cudaStream_t s) {
+  if (m <= 8) {
+    const int tb = SR_VALUES / 8;
+    launch_k(small_route_kernel<8>, (T + tb - 1) / tb, SR_THREADS, 0, s, T, d, m, k, renorm, (const uint4*)x,
+             (const uint4*)w, bias, logits, idx, wout);
+  } else {
+    const int tb = SR_VALUES / 16;
+    launch_k(small_route_kernel<16>, (T + tb - 1) / tb, SR_THREADS, 0, s, T, d, m, k, renorm, (const uint4*)x,
+             (const uint4*)w, bias, logits, idx, wout);
+  }
+  count_launch();
+  return cudaGetLastError();
+}
+
 // ------------------------------------------------------------------ top-k + softmax
 // One warp per token. k rounds of a warp arg-max over the not-yet-chosen
 // experts, ordered by (logit desc, expert index asc). Gate weights: softmax over

@@ -355,56 +355,6 @@ __device__ __forceinline__ void route_pass(uint32_t t_row, int m, const float* r
   }
 }
 
-// The router epilogue for m <= 128 experts: a token's m logits are read from TMEM
-// once (eight loads, one wait) and kept in registers for all k passes. Pass s takes
-// the largest logit strictly after pick s - 1 in (logit desc, expert asc), by 32-wide
-// pairwise trees whose left side holds the lower experts, merged in column order
-// (trees keep the dependency chains short: one warp per SM sub-partition runs
-// this epilogue, so latency, not issue, bounds it). The softmax denominator is the
-// fp64 sum, per 32 columns, of fp32 partial sums of exp(logit - max), the max being
-// pick 0. Picks stay in registers (k <= 8).
-constexpr int ROUTE_REG_M = 128;
-
-__device__ __forceinline__ void tmem_ld_x16f(uint32_t taddr, float* r) {
-  asm volatile(
-      "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
-      : "=f"(r[0]), "=f"(r[1]), "=f"(r[2]), "=f"(r[3]), "=f"(r[4]), "=f"(r[5]), "=f"(r[6]), "=f"(r[7]),
-        "=f"(r[8]), "=f"(r[9]), "=f"(r[10]), "=f"(r[11]), "=f"(r[12]), "=f"(r[13]), "=f"(r[14]), "=f"(r[15])
-      : "r"(taddr));
-}
-
-template <int RM>
-__device__ __forceinline__ void route_best_after(const float (&v)[RM], int m, float pv, int pe, float& bv, int& be) {
-  bv = -INFINITY;
-  be = -1;
-#pragma unroll
-  for (int c0 = 0; c0 < RM; c0 += 32) {
-    if (c0 >= m) break;
-    constexpr int W = RM < 32 ? RM : 32;
-    float cv[W];
-    int ce[W];
-#pragma unroll
-    for (int j = 0; j < W; ++j) {
-      const float x = v[c0 + j];
-      const bool after = x < pv || (x == pv && c0 + j > pe);
-      cv[j] = (c0 + j < m && after) ? x : -INFINITY;
-      ce[j] = c0 + j;
-    }
-#pragma unroll
-    for (int st = 1; st < W; st <<= 1)
-#pragma unroll
-      for (int j = 0; j < W; j += 2 * st)
-        if (cv[j + st] > cv[j]) {  // an equal logit keeps the lower expert (left)
-          cv[j] = cv[j + st];
-          ce[j] = ce[j + st];
-        }
-    if (cv[0] > bv) {  // earlier chunks hold lower experts
-      bv = cv[0];
-      be = ce[0];
-    }
-  }
-}
-
 // ------------------------------------------------------------------ tile schedule
 struct TileInfo {
   int cls, g, mt, ks, nt, rows_in_tile, b_row, out_row, a_row, kb0, kb1;
@@ -507,9 +457,6 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
   constexpr int RMASK_M = EPI == EPI_ROUTE ? ROUTE_MAX_M : 1;
   __shared__ __align__(16) float rbias[RMASK_M];  // ROUTE: router bias (zeros when absent)
   __shared__ uint32_t rmask[EPI == EPI_ROUTE ? 2 : 1][4][RMASK_M];  // ROUTE: expert -> lanes holding it
-  // ROUTE: each epilogue thread's k picks (value, expert), in pick order
-  __shared__ float rpick_v[EPI == EPI_ROUTE ? 128 : 1][ROUTE_MAX_K];
-  __shared__ int rpick_e[EPI == EPI_ROUTE ? 128 : 1][ROUTE_MAX_K];
   __shared__ uint32_t tmem_base_s;
   __shared__ int abort_s, epi_fail_s;
   __shared__ int total_tiles_s;
@@ -780,88 +727,34 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
       float* lg = c.out && tv_ok ? reinterpret_cast<float*>(c.out) + (long long)t * m : nullptr;
       int32_t* oi = c.sel_idx + (long long)t * k;
       float* ow = c.sel_w + (long long)t * k;
-      float* pick_v = rpick_v[EPI == EPI_ROUTE ? et : 0];
-      int* pick_e = rpick_e[EPI == EPI_ROUTE ? et : 0];
+      float pv = INFINITY;
+      int pe = -1;
       bool bad = false;
-      // the expert tile is BN = the smallest power of two >= m (at least 16), so tiles
-      // of up to 128 experts keep the logits in registers and larger ones re-read TMEM
-      constexpr int RM = BN < ROUTE_REG_M ? BN : ROUTE_REG_M;
-      if (BN <= ROUTE_REG_M) {
-        // all m logits in registers: one round of TMEM loads, then k passes
-        float v[RM];
-#pragma unroll
-        for (int c0 = 0; c0 < RM; c0 += 16) {
-          if (c0 < m) {  // m is the same for the whole warp
-            tmem_ld_x16f(t_row + c0, v + c0);
-          } else {
-#pragma unroll
-            for (int j = 0; j < 16; ++j) v[c0 + j] = 0.f;
-          }
-        }
-        tmem_ld_wait();
-#pragma unroll
-        for (int j = 0; j < RM; ++j) v[j] = j < m ? v[j] + rbias[j] : -INFINITY;
-        // the accumulator is free for the next tile's MMAs
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&acce_bar[acc]);
-        if (lg)
-#pragma unroll
-          for (int j = 0; j < RM; ++j)
-            if (j < m) lg[j] = v[j];
-        float pv = INFINITY;
-        int pe = -1;
 #pragma unroll 1
-        for (int s2 = 0; s2 < k; ++s2) {
-          float bv;
-          int be;
-          route_best_after<RM>(v, m, pv, pe, bv, be);
-          if (s2 == 0) mx = bv;
-          pick_v[s2] = bv;
-          pick_e[s2] = be;
-          bad |= be < 0;  // NaN logits
-          pv = bv;
-          pe = be;
+      for (int s2 = 0; s2 < k; ++s2) {
+        float bv;
+        int be;
+        if (s2 == 0) {
+          route_pass<true>(t_row, m, rbias, pv, pe, bv, be, mrun, z, lg);
+          mx = bv;
+          z *= (double)expf(mrun - mx);  // the running maximum is the top logit
+        } else {
+          float dm = 0.f;
+          double dz = 0.0;
+          route_pass<false>(t_row, m, rbias, pv, pe, bv, be, dm, dz, nullptr);
         }
-#pragma unroll
-        for (int c0 = 0; c0 < RM; c0 += 32) {
-          if (c0 >= m) break;
-          float ex[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-          for (int j = 0; j < 32; ++j)
-            if (c0 + j < m && c0 + j < RM) ex[j & 3] += expf(v[(c0 + j) % RM] - mx);
-          z += (double)((ex[0] + ex[1]) + (ex[2] + ex[3]));
+        if (tv_ok) {
+          oi[s2] = be;
+          ow[s2] = bv;
         }
-      } else {
-        // Pass s picks the largest logit strictly after pick s - 1 in the order
-        // (logit desc, expert asc), reading the accumulator again from TMEM; pass 0
-        // also writes the logits (when asked) and the softmax denominator.
-        float pv = INFINITY;
-        int pe = -1;
-#pragma unroll 1
-        for (int s2 = 0; s2 < k; ++s2) {
-          float bv;
-          int be;
-          if (s2 == 0) {
-            route_pass<true>(t_row, m, rbias, pv, pe, bv, be, mrun, z, lg);
-            mx = bv;
-            z *= (double)expf(mrun - mx);  // the running maximum is the top logit
-          } else {
-            float dm = 0.f;
-            double dz = 0.0;
-            route_pass<false>(t_row, m, rbias, pv, pe, bv, be, dm, dz, nullptr);
-          }
-          pick_v[s2] = bv;
-          pick_e[s2] = be;
-          bad |= be < 0;  // NaN logits
-          pv = bv;
-          pe = be;
-        }
-        // the accumulator is free for the next tile's MMAs
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&acce_bar[acc]);
+        bad |= be < 0;  // NaN logits
+        pv = bv;
+        pe = be;
       }
+      // the accumulator is free for the next tile's MMAs
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&acce_bar[acc]);
       if (++acc == S::NUM_ACC) {
         acc = 0;
         acc_phase ^= 1u;
@@ -869,12 +762,11 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
       if (tv_ok) {  // gate weights: softmax over all m, renormalised over the k chosen when asked
         double sel = 0.0;
 #pragma unroll 1
-        for (int s2 = 0; s2 < k; ++s2) sel += (double)expf(pick_v[s2] - mx) / z;
+        for (int s2 = 0; s2 < k; ++s2) sel += (double)expf(ow[s2] - mx) / z;
 #pragma unroll 1
         for (int s2 = 0; s2 < k; ++s2) {
-          double pr = (double)expf(pick_v[s2] - mx) / z;
+          double pr = (double)expf(ow[s2] - mx) / z;
           if (c.renorm) pr /= sel;
-          oi[s2] = pick_e[s2];
           ow[s2] = (float)pr;
         }
         if (bad) set_status(p.status, MOE_ERR_DEVICE_INDEX);
@@ -888,14 +780,14 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
         if (tv_ok)
 #pragma unroll 1
           for (int s2 = 0; s2 < k; ++s2) {
-            const int e = pick_e[s2];
+            const int e = oi[s2];
             if (e >= 0) atomicOr(&mk[q][e], 1u << lane);
           }
         epi_bar();
         if (tv_ok)
 #pragma unroll 1
           for (int s2 = 0; s2 < k; ++s2) {
-            const int e = pick_e[s2];
+            const int e = oi[s2];
             if (e < 0) continue;
             int rk = __popc(mk[q][e] & ((1u << lane) - 1u));
             for (int q2 = 0; q2 < q; ++q2) rk += __popc(mk[q2][e]);

@@ -43,6 +43,12 @@ ROUTE_CASES = [
     W.small_moe(T=1, d=4096, f=64, m=8, k=2, dtype=W.BF16, zipf_s=0.0, index=85),
     W.small_moe(T=8269, d=72, f=64, m=200, k=8, dtype=W.BF16, zipf_s=0.7, renorm=True, index=89),
     W.small_moe(T=8192, d=64, f=64, m=256, k=2, dtype=W.BF16, zipf_s=1.0, index=90),
+    # few experts (m <= 16): logits, top-k and gate weights in one CUDA-core launch;
+    # ragged last block (T not a multiple of the tokens per block), m not a power of two
+    W.small_moe(T=4099, d=4096, f=64, m=8, k=2, dtype=W.BF16, zipf_s=0.8, renorm=True, index=96),
+    W.small_moe(T=777, d=264, f=64, m=12, k=3, dtype=W.BF16, zipf_s=1.0, index=97),
+    W.small_moe(T=130, d=2048, f=64, m=16, k=16, dtype=W.BF16, zipf_s=0.5, index=98),
+    W.small_moe(T=3, d=8, f=64, m=1, k=1, dtype=W.BF16, zipf_s=0.0, index=99),
 ]
 
 
