@@ -98,7 +98,10 @@ cudaError_t launch_k(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem,
 // Every launcher returns cudaSuccess or the launch error; arguments were checked
 // by the C-ABI layer before.
 
-enum Epi { EPI_LOGITS = 0, EPI_SWIGLU = 1, EPI_RELU = 2, EPI_DOWN = 3, EPI_ROUTE = 4 };
+enum Epi { EPI_LOGITS = 0, EPI_SWIGLU = 1, EPI_RELU = 2, EPI_DOWN = 3, EPI_ROUTE = 4,
+           // the down projection with two consecutive feature blocks per tile sharing the
+           // token rows (pair tiles only: 512 output features x up to 256 token rows)
+           EPI_DOWN_DUAL = 5 };
 
 // EPI_ROUTE: the router with tokens as the MMA's M rows (A = x) and all experts in
 // one N tile (B = W_r, m <= 256 rows): each epilogue thread owns a token's logits.

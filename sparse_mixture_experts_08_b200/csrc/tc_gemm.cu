@@ -439,8 +439,13 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
   using S = TcShape<BN, MATS, PAIR>;
   constexpr int STAGES = S::STAGES;
   constexpr int BKE = F8 ? TC_BK8 : TC_BK;  // K elements per k-block (one 128-byte row)
-  constexpr int TILE_M = S::TILE_M;
+  // DUAL (the down projection with MATS = 2): two consecutive blocks of S::TILE_M
+  // output features of the same weight matrix share each token tile, so the token
+  // rows are staged once for twice the MMA work (less shared-memory traffic per flop)
+  constexpr bool DUAL = EPI == EPI_DOWN && MATS == 2;
+  constexpr int TILE_M = S::TILE_M * (DUAL ? 2 : 1);
   static_assert(!F8 || EPI == EPI_SWIGLU || EPI == EPI_RELU || EPI == EPI_DOWN, "8-bit operands: expert GEMMs only");
+  static_assert(!DUAL || !F8, "two feature blocks: bf16 only");
   static_assert(!PAIR || (!F8 && (EPI == EPI_SWIGLU || EPI == EPI_RELU || EPI == EPI_DOWN)),
                 "pair tiles: bf16 expert GEMMs only");
 
@@ -582,13 +587,16 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
           const uint32_t fb = mapa_shared(smem_u32(&full_bar[stage]), 0);
           if (leader) mbar_arrive_expect_tx(&full_bar[stage], 2 * S::STAGE_BYTES);
           tma_load_2d_pair(mA0, fb, st, kb * BKE, a_row);
-          if (MATS == 2) tma_load_2d_pair(mA1, fb, st + S::A_BYTES, kb * BKE, a_row);
+          if (MATS == 2)
+            tma_load_2d_pair(DUAL ? mA0 : mA1, fb, st + S::A_BYTES, kb * BKE, a_row + (DUAL ? S::TILE_M : 0));
           tma_load_2d_pair(mB, fb, st + MATS * S::A_BYTES, kb * BKE, b_row);
           if (leader) last_parity[stage] = (int)phase;
         } else {
           mbar_arrive_expect_tx(&full_bar[stage], S::STAGE_BYTES);
           tma_load_2d(mA0, &full_bar[stage], st, kb * BKE, ti.a_row);
-          if (MATS == 2) tma_load_2d(mA1, &full_bar[stage], st + S::A_BYTES, kb * BKE, ti.a_row);
+          if (MATS == 2)
+            tma_load_2d(DUAL ? mA0 : mA1, &full_bar[stage], st + S::A_BYTES, kb * BKE,
+                        ti.a_row + (DUAL ? S::TILE_M : 0));
           tma_load_2d(mB, &full_bar[stage], st + MATS * S::A_BYTES, kb * BKE, ti.b_row);
           last_parity[stage] = (int)phase;
         }
@@ -844,11 +852,13 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
       // One 16-row chunk of accumulator columns (r0: gate or the single matrix, r1: up).
       auto chunk = [&](const int c0, const uint32_t (&r0)[16], const uint32_t (&r1)[16]) {
         const int jn = min(16, ti.rows_in_tile - c0);
-        if (VEC) {
+        // activation of 16 rows x this warp's 32 features, staged, then stored as
+        // 16-byte vectors along the feature axis from feature fbase on
+        auto emit = [&](const uint32_t (&ra)[16], const uint32_t (&rb)[16], const int fbase) {
 #pragma unroll
           for (int j = 0; j < 16; ++j) {
-            float v0 = has_k ? __uint_as_float(r0[j]) : 0.f;
-            float v1 = (MATS == 2 && has_k) ? __uint_as_float(r1[j]) : 0.f;
+            float v0 = has_k ? __uint_as_float(ra[j]) : 0.f;
+            float v1 = (MATS == 2 && !DUAL && has_k) ? __uint_as_float(rb[j]) : 0.f;
             if (F8) {
               const float sb = EPI == EPI_DOWN ? 1.f : aux_s[q][c0 + j];
               v0 = v0 * sa0 * sb;
@@ -860,7 +870,6 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
                                                 : v0 * aux_w[q][c0 + j];
           }
           __syncwarp();
-          const int fbase = fcta + q * 32;  // first feature of this warp (R is a multiple of 8)
           if (EPI == EPI_DOWN && !c.scatter_k1) {  // fp32 partial rows: 8 float4 per row
             float* o = reinterpret_cast<float*>(c.out) + (long long)ti.ks * c.out_split_stride + fbase;
 #pragma unroll
@@ -888,6 +897,11 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
             }
           }
           __syncwarp();
+        };
+        if (VEC) {
+          const int fbase = fcta + q * 32;  // first feature of this warp (R is a multiple of 8)
+          emit(r0, r1, fbase);
+          if (DUAL) emit(r1, r1, fbase + S::TILE_M);  // the second feature block
         } else if (fvalid) {  // LOGITS
 #pragma unroll
           for (int j = 0; j < 16; ++j)
@@ -1072,6 +1086,7 @@ cudaError_t launch_tc_gemm(int epi, int bn, const TcMaps& maps, const GemmParams
     if (epi == EPI_SWIGLU) return launch_impl<256, 2, EPI_SWIGLU, false, true>(maps, p, num_ctas, s);
     if (epi == EPI_RELU) return launch_impl<256, 1, EPI_RELU, false, true>(maps, p, num_ctas, s);
     if (epi == EPI_DOWN) return launch_impl<256, 1, EPI_DOWN, false, true>(maps, p, num_ctas, s);
+    if (epi == EPI_DOWN_DUAL) return launch_impl<256, 2, EPI_DOWN, false, true>(maps, p, num_ctas, s);
     return cudaErrorInvalidValue;
   }
   if (f8) {

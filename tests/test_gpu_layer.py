@@ -99,7 +99,7 @@ def test_decode_all_tokens():
 
 @pytest.mark.parametrize("case", ["one_hot", "one_hot_fused", "T1", "ragged_small", "relu_many_experts",
                                   "max_experts_max_k", "routed_k8_m200", "pair_shared", "pair_empty_and_single",
-                                  "pair_relu_top1"])
+                                  "pair_relu_top1", "pair_dual_shared"])
 def test_layer_edge_cases(case):
     if case in ("one_hot", "one_hot_fused"):  # every token's top-1 is the same expert (huge bias)
         T = 300 if case == "one_hot" else 8192  # 8192: the fused router and scatter
@@ -134,8 +134,13 @@ def test_layer_edge_cases(case):
         inp["x"][0, 5] = 0x4180                           # bf16 16.0
         inp["w_router"][3, :] = 0
         inp["w_router"][3, 5] = 0x4280                    # bf16 64.0: logit 1024 - 100 for token 0, -100 for the rest
-    elif case == "pair_relu_top1":  # pair tiles, top-1 ReLU: the down epilogue writes the layer output
-        cfg = W.small_moe(T=2048, d=384, f=512, m=4, k=1, act=W.RELU, dtype=W.BF16, zipf_s=1.5, index=81)
+    elif case == "pair_relu_top1":  # pair tiles, top-1 ReLU: the down epilogue writes the layer output;
+        # d = 640: the down projection's two 256-row feature blocks, the second one ragged
+        cfg = W.small_moe(T=2048, d=640, f=512, m=4, k=1, act=W.RELU, dtype=W.BF16, zipf_s=1.5, index=81)
+        inp = W.make_moe_inputs(cfg)
+    elif case == "pair_dual_shared":  # two feature blocks per down tile (d = 768) beside a shared expert
+        cfg = W.small_moe(T=1024, d=768, f=256, m=4, k=2, dtype=W.BF16, zipf_s=1.0, n_shared=1, f_shared=128,
+                          index=82)
         inp = W.make_moe_inputs(cfg)
     else:  # the largest expert count and top-k the library accepts (m = 1024, k = 32)
         cfg = W.small_moe(T=700, d=64, f=64, m=1024, k=32, dtype=W.BF16, zipf_s=0.5, index=77)
