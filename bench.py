@@ -949,9 +949,7 @@ def ours_atomic(args):
     e2e_ms = e2e_pipelined(torch, lambda xd, od: fwd2(xd, od), x_host, x_devs, [o.view(torch.int16) for o in out_devs],
                            out_hosts, Ke, s, dev)
     pk, pk_src = peaks()
-    # the library's projection choice: one pass of final logits for 16 tokens or fewer,
-    # else tensor-core tiles with 16 split-K partials per logit
-    ksplit = 1 if cfg.T <= 16 else 16
+    ksplit = 16  # the router projections' split-K partials per logit (tensor-core tiles)
     costs, layer_flops, layer_bytes = atomic_stage_costs(cfg, active, ksplit)
     fl, by = costs[dom]
     roof = {"bound": "hbm", "achieved": by / (dom_ms * 1e-3) / 1e9, "peak": pk["hbm_gbs"], "unit": "GB/s",

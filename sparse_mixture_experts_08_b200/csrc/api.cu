@@ -894,16 +894,6 @@ static moe_status_t atomic_route_impl(const moe_atomic_config_t& c, const Atomic
   int* status = at<int>(ws, P.status);
   float* zr = at<float>(ws, P.zr);
   float* zc = at<float>(ws, P.zc);
-  if (atomic_proj_ok(c.T, c.d)) {
-    // decode budgets: one CUDA-core pass writes the final logits (the tensor-core
-    // tile would hold at most 16 of its 128 token rows and need split-K partials)
-    MOE_CUDA(launch_atomic_proj(c.T, c.d, c.Nr, c.Nc, x, w_row, w_col, zr, zc, s));
-    if (stage_marks) MOE_TRY(mark_stage(1, s));
-    MOE_CUDA(launch_atomic_select(c.T, c.Nr, c.Nc, c.K, 1, zr, (long long)c.T * c.Nr, zc, (long long)c.T * c.Nc,
-                                  lr_out, lc_out, idx, g, status, at<unsigned>(ws, P.bar), s));
-    if (stage_marks) MOE_TRY(mark_stage(2, s));
-    return MOE_OK;
-  }
   GemmParams p;
   std::memset(&p, 0, sizeof(p));
   fill_common(p, status);

@@ -674,106 +674,6 @@ __global__ void __launch_bounds__(SEL_THREADS, 1)
   }
 }
 
-// ------------------------------------------------------------------ router projections, decode budgets
-// z[t][r] = x_t . w[r] for the Nr + Nc rows of W_row and W_col (Cartesian Product
-// Router, OmniMoE Sec. 2.2: both projections are d -> Nr and d -> Nc linear maps),
-// for batches of at most AP_MAX_T tokens and d <= 8 AP_THREADS. One CTA per AP_ROWS
-// rows; thread i owns the 16-byte chunk i of the model dimension, keeps that chunk
-// of every token's x in registers and, per row, forms its partial dot products in
-// fp32 (the chunk's 8 elements in order); the partials are summed by a
-// fixed shuffle reduce-scatter in each warp and then over the warps in warp order,
-// so the result does not depend on timing. The final logits leave in one pass: no
-// split-K partials for the selection kernel to add up.
-constexpr int AP_THREADS = 512, AP_ROWS = 8, AP_MAX_T = 16;
-
-__global__ void __launch_bounds__(AP_THREADS, 1)
-    atomic_proj_kernel(int T, int d, int Nr, int Nc, const uint4* __restrict__ x, const uint4* __restrict__ w_row,
-                       const uint4* __restrict__ w_col, float* __restrict__ zr, float* __restrict__ zc) {
-  __shared__ float red[2][AP_THREADS / 32][AP_MAX_T];
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int chunks = d / 8;  // <= AP_THREADS: one chunk per thread
-  const int c = tid;
-  const int r0 = blockIdx.x * AP_ROWS;
-  const int nrows = Nr + Nc;
-  pdl_launch_dependents();
-  // the weights are not written by an earlier kernel of the stream: the first row's
-  // chunk is requested before waiting for the predecessor; each row's load is issued
-  // one row ahead of its use
-  auto wload = [&](int rr) {
-    const int r = r0 + rr;
-    const uint4* wr = r < Nr ? w_row + (long long)r * chunks : w_col + (long long)(r - Nr) * chunks;
-    return (rr < AP_ROWS && r < nrows && c < chunks) ? wr[c] : make_uint4(0u, 0u, 0u, 0u);
-  };
-  uint4 wnext = wload(0);
-  pdl_wait();
-  // this thread's chunk of every token's x, kept as bf16 pairs (zero past T or d)
-  uint4 xp[AP_MAX_T];
-#pragma unroll
-  for (int t = 0; t < AP_MAX_T; ++t)
-    xp[t] = (t < T && c < chunks) ? x[(long long)t * chunks + c] : make_uint4(0u, 0u, 0u, 0u);
-#pragma unroll 1
-  for (int rr = 0; rr < AP_ROWS; ++rr) {
-    const uint4 wcur = wnext;
-    wnext = wload(rr + 1);
-    // keep x packed: without this the compiler hoists the bf16 -> fp32 conversions
-    // out of the row loop and runs out of registers
-#pragma unroll
-    for (int t = 0; t < AP_MAX_T; ++t)
-      asm volatile("" : "+r"(xp[t].x), "+r"(xp[t].y), "+r"(xp[t].z), "+r"(xp[t].w));
-    float acc[AP_MAX_T];
-    const __nv_bfloat162* wh = reinterpret_cast<const __nv_bfloat162*>(&wcur);
-#pragma unroll
-    for (int t = 0; t < AP_MAX_T; ++t) {
-      const __nv_bfloat162* xh = reinterpret_cast<const __nv_bfloat162*>(&xp[t]);
-      float a = 0.f;
-#pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        const float2 w2 = __bfloat1622float2(wh[u]), x2 = __bfloat1622float2(xh[u]);
-        a = fmaf(x2.x, w2.x, a);
-        a = fmaf(x2.y, w2.y, a);
-      }
-      acc[t] = a;
-    }
-    // reduce-scatter over the warp: lane bits 4..1 pick the token, bit 0 pairs up
-#pragma unroll
-    for (int half = AP_MAX_T / 2, bit = 16; half >= 1; half >>= 1, bit >>= 1) {
-      const bool upper = (lane & bit) != 0;
-#pragma unroll
-      for (int i = 0; i < half; ++i) {
-        const float keep = upper ? acc[half + i] : acc[i];
-        const float send = upper ? acc[i] : acc[half + i];
-        acc[i] = keep + __shfl_xor_sync(FULL, send, bit);
-      }
-    }
-    acc[0] += __shfl_xor_sync(FULL, acc[0], 1);
-    float(*rb)[AP_MAX_T] = red[rr & 1];
-    if ((lane & 1) == 0) rb[warp][lane >> 1] = acc[0];
-    __syncthreads();
-    const int r = r0 + rr;
-    if (tid < T && r < nrows) {
-      float sum = 0.f;
-#pragma unroll
-      for (int w = 0; w < AP_THREADS / 32; ++w) sum += rb[w][tid];
-      if (r < Nr)
-        zr[(long long)tid * Nr + r] = sum;
-      else
-        zc[(long long)tid * Nc + (r - Nr)] = sum;
-    }
-    // (the next row writes the other buffer; the one after passes another barrier first)
-  }
-}
-
-bool atomic_proj_ok(int T, int d) { return T <= AP_MAX_T && d % 8 == 0 && d / 8 <= AP_THREADS; }
-
-cudaError_t launch_atomic_proj(int T, int d, int Nr, int Nc, const void* x, const void* w_row, const void* w_col,
-                               float* zr, float* zc, cudaStream_t s) {
-  const int ctas = (Nr + Nc + AP_ROWS - 1) / AP_ROWS;
-  launch_k(atomic_proj_kernel, ctas, AP_THREADS, 0, s, T, d, Nr, Nc, (const uint4*)x, (const uint4*)w_row,
-           (const uint4*)w_col, zr, zc);
-  count_launch();
-  return cudaGetLastError();
-}
-
 cudaError_t launch_atomic_select(int T, int Nr, int Nc, int K, int ksplit, const float* zr, long long zr_split,
                                  const float* zc, long long zc_split, float* lr_out, float* lc_out, int32_t* idx,
                                  float* g, int* status, unsigned* bar_reset, cudaStream_t s) {

@@ -16,12 +16,6 @@ cudaError_t launch_atomic_experts_sorted(int T, int d, int K, int act, const voi
                                          long long n_experts, unsigned* bar, bool bar_zeroed,
                                          unsigned long long limit_ns, int* status, int32_t* sort_ws, cudaStream_t s);
 
-// Router projections (final fp32 logits, no split-K partials) for batches of at most
-// 16 tokens with d <= 4096: z_row [T, Nr] and z_col [T, Nc].
-bool atomic_proj_ok(int T, int d);
-cudaError_t launch_atomic_proj(int T, int d, int Nr, int Nc, const void* x, const void* w_row, const void* w_col,
-                               float* zr, float* zc, cudaStream_t s);
-
 // Fault-injection hook: the decode-budget atomic-expert kernel's grid barrier waits
 // for n arrivals more than its grid has, so it ends only at its time limit.
 void set_grid_barrier_extra(unsigned n);

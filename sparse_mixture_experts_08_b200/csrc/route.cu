@@ -134,13 +134,13 @@ cudaError_t launch_few_expert_logits(int T, int d, int m, const void* x, const v
 // SR_THREADS, ... of the model dimension, loads those chunks of every expert's
 // router row once and applies them to each of the block's tokens (fp32 FMAs, chunks
 // in ascending order). The SR_VALUES partial sums per thread are reduced by a
-// shuffle reduce-scatter in each warp (lane L ends with values 2L and 2L + 1) and
+// shuffle reduce-scatter in each warp (lane L ends with value L) and
 // then over the warps in warp order; the logit gets its bias. Then one thread per
 // token takes the top-k by (logit desc, expert asc) and the gate weights as
 // topk_softmax_kernel does: exp in fp32 of l - max, sums in fp64, renormalised over
 // the k chosen when asked. Every sum has a fixed order: the result does not depend
 // on timing.
-constexpr int SR_THREADS = 256, SR_VALUES = 64;
+constexpr int SR_THREADS = 256, SR_VALUES = 32;
 
 template <int M>
 __global__ void __launch_bounds__(SR_THREADS)
@@ -161,14 +161,16 @@ __global__ void __launch_bounds__(SR_THREADS)
 #pragma unroll
     for (int e = 0; e < M; ++e) acc[t][e] = 0.f;
   for (int c = tid; c < chunks; c += SR_THREADS) {
-    uint4 wv[M];
+    // every load of a chunk is independent: all of them (M router rows, TB tokens)
+    // are issued before the chunk's FMAs
+    uint4 wv[M], xv[TB];
 #pragma unroll
     for (int e = 0; e < M; ++e) wv[e] = e < m ? w[(long long)e * chunks + c] : make_uint4(0u, 0u, 0u, 0u);
 #pragma unroll
+    for (int t = 0; t < TB; ++t) xv[t] = t0 + t < T ? x[(t0 + t) * chunks + c] : make_uint4(0u, 0u, 0u, 0u);
+#pragma unroll
     for (int t = 0; t < TB; ++t) {
-      if (t0 + t >= T) break;
-      const uint4 xv = x[(t0 + t) * chunks + c];
-      const __nv_bfloat162* xh = reinterpret_cast<const __nv_bfloat162*>(&xv);
+      const __nv_bfloat162* xh = reinterpret_cast<const __nv_bfloat162*>(&xv[t]);
 #pragma unroll
       for (int e = 0; e < M; ++e) {
         const __nv_bfloat162* wh = reinterpret_cast<const __nv_bfloat162*>(&wv[e]);
@@ -183,10 +185,10 @@ __global__ void __launch_bounds__(SR_THREADS)
       }
     }
   }
-  // reduce-scatter over the warp: value index v = t M + e; lane L keeps 2L, 2L + 1
+  // reduce-scatter over the warp: value index v = t M + e; lane L keeps value L
   float* v = &acc[0][0];
 #pragma unroll
-  for (int half = SR_VALUES / 2, bit = 16; half >= 2; half >>= 1, bit >>= 1) {
+  for (int half = SR_VALUES / 2, bit = 16; half >= 1; half >>= 1, bit >>= 1) {
     const bool upper = (lane & bit) != 0;
 #pragma unroll
     for (int i = 0; i < half; ++i) {
@@ -195,8 +197,7 @@ __global__ void __launch_bounds__(SR_THREADS)
       v[i] = keep + __shfl_xor_sync(FULL, send, bit);
     }
   }
-  red[warp][2 * lane] = v[0];
-  red[warp][2 * lane + 1] = v[1];
+  red[warp][lane] = v[0];
   __syncthreads();
   if (tid < SR_VALUES) {
     const int t = tid / M, e = tid % M;
