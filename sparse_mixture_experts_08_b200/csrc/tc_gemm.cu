@@ -636,7 +636,8 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
       tc_fence_after();
       const uint32_t d_tmem = tmem_base + (uint32_t)(acc * S::ACC_COLS);
       const int n_inst = max(16, (ti.rows_in_tile + 15) & ~15);
-      const uint32_t idesc = F8 ? idesc_e4m3(TILE_M, n_inst) : idesc_bf16(TILE_M, n_inst);
+      // one MMA covers S::TILE_M weight rows (DUAL tiles issue two of them per K step)
+      const uint32_t idesc = F8 ? idesc_e4m3(S::TILE_M, n_inst) : idesc_bf16(S::TILE_M, n_inst);
       for (int kb = ti.kb0; kb < ti.kb1; ++kb) {
         if (!mbar_wait(&full_bar[stage], phase, lim, abort_flag)) {
           ok = false;
