@@ -23,7 +23,8 @@
 // and only the K elements per k-block double.
 //
 // Warp roles (192 threads): warp 0 = TMA producer, warp 1 = MMA issuer (and TMEM
-// owner), warps 2..5 = epilogue (TMEM -> registers -> activation -> global).
+// owner), warps 2..5 = epilogue (TMEM -> registers -> activation -> global); pair
+// SwiGLU tiles use 320 threads, warps 2..9 = epilogue, two per TMEM lane quarter.
 // The accumulator is double-buffered in TMEM when it fits (2 x mats x BN <= 512
 // columns) so the epilogue of tile i overlaps the MMAs of tile i + 1.
 //
@@ -52,7 +53,13 @@ namespace moe {
 constexpr int TC_BM = 128;
 constexpr int TC_BK = 64;  // bf16 elements of one 128-byte swizzle row
 constexpr int TC_BK8 = 128;  // E4M3 elements of one 128-byte swizzle row
-constexpr int TC_THREADS = 192;
+// Epilogue warps of a kernel instance: pair SwiGLU tiles hold one accumulator (2 x 256
+// TMEM columns), so the MMAs of the next tile wait for the whole epilogue; there two
+// warps per TMEM lane quarter share the chunks (8 warps). Elsewhere 4.
+template <int EPI, bool PAIR, bool F8>
+constexpr int tc_epi_warps() { return (PAIR && EPI == EPI_SWIGLU && !F8) ? 8 : 4; }
+template <int EPI, bool PAIR, bool F8>
+constexpr int tc_threads() { return 64 + 32 * tc_epi_warps<EPI, PAIR, F8>(); }
 constexpr int TC_MAX_GROUPS = 1040;
 constexpr int TC_SMEM_BUDGET = 200 * 1024;
 constexpr unsigned long long TC_DRAIN_LIMIT_NS = 200ull * 1000 * 1000;
@@ -431,7 +438,7 @@ __device__ __forceinline__ void store_logit(const GemmClass& c, const TileInfo& 
 }
 
 template <int BN, int MATS, int EPI, bool F8, bool PAIR>
-__global__ void __launch_bounds__(TC_THREADS, 1)
+__global__ void __launch_bounds__(tc_threads<EPI, PAIR, F8>(), 1)
     tc_grouped_gemm_kernel(const __grid_constant__ CUtensorMap tA0_0, const __grid_constant__ CUtensorMap tA1_0,
                            const __grid_constant__ CUtensorMap tB_0, const __grid_constant__ CUtensorMap tA0_1,
                            const __grid_constant__ CUtensorMap tA1_1, const __grid_constant__ CUtensorMap tB_1,
@@ -458,7 +465,8 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
   // global writes leave as 16-byte vectors along the feature axis (rows padded to 36
   // floats: 16-byte aligned, and the column-wise writes hit 32 distinct banks)
   constexpr bool VEC = EPI == EPI_SWIGLU || EPI == EPI_RELU || EPI == EPI_DOWN;
-  __shared__ __align__(16) float stg[VEC ? 4 : 1][16][36];
+  constexpr int NEPI = tc_epi_warps<EPI, PAIR, F8>();
+  __shared__ __align__(16) float stg[VEC ? NEPI : 1][16][36];
   constexpr int RMASK_M = EPI == EPI_ROUTE ? ROUTE_MAX_M : 1;
   __shared__ __align__(16) float rbias[RMASK_M];  // ROUTE: router bias (zeros when absent)
   __shared__ uint32_t rmask[EPI == EPI_ROUTE ? 2 : 1][4][RMASK_M];  // ROUTE: expert -> lanes holding it
@@ -487,7 +495,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&accf_bar[i], 1);
-      mbar_init(&acce_bar[i], PAIR ? 8 : 4);  // PAIR: the epilogue warps of both CTAs release the leader's
+      mbar_init(&acce_bar[i], (PAIR ? 2 : 1) * NEPI);  // PAIR: the epilogue warps of both CTAs release the leader's
     }
     mbar_init(&drain_bar, 1);
     abort_s = 0;
@@ -813,6 +821,9 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
   } else if (warp >= 2) {
     // ---------------------------------------------------------------- epilogue
     const int q = warp & 3;  // TMEM lane quarter this warp may access
+    const int ew = warp - 2;  // epilogue warp index (its staging tile)
+    // with 8 epilogue warps the two warps of a quarter take alternate 16-row chunks
+    const int cfirst = 16 * (ew >> 2), cstep = 16 * (NEPI / 4);
     int acc = 0;
     uint32_t acc_phase = 0;
     for (int w = walker; w < total; w += walkers) {
@@ -866,7 +877,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
               v1 = v1 * sa1 * sb;
             }
             // SiLU's quotient by the fast division (2 ulp; h is stored in bf16)
-            stg[q][j][lane] = EPI == EPI_SWIGLU ? __fdividef(v0, 1.f + __expf(-v0)) * v1
+            stg[ew][j][lane] = EPI == EPI_SWIGLU ? __fdividef(v0, 1.f + __expf(-v0)) * v1
                               : EPI == EPI_RELU ? fmaxf(v0, 0.f)
                                                 : v0 * aux_w[q][c0 + j];
           }
@@ -878,7 +889,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
               const int idx = lane + 32 * i, jj = idx >> 3, part = idx & 7;
               if (jj < jn && fbase + part * 4 < c.R)
                 *reinterpret_cast<float4*>(o + (long long)(ti.out_row + c0 + jj) * c.out_ld + part * 4) =
-                    *reinterpret_cast<const float4*>(&stg[q][jj][part * 4]);
+                    *reinterpret_cast<const float4*>(&stg[ew][jj][part * 4]);
             }
           } else {  // bf16 rows (h, or the layer output with the top-1 combine fused): 4 x 8 per row
             __nv_bfloat16* o = reinterpret_cast<__nv_bfloat16*>(c.out) + fbase;
@@ -887,7 +898,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
               const int idx = lane + 32 * i, jj = idx >> 2, part = idx & 3;
               const long long orow = EPI == EPI_DOWN ? (long long)aux_d[q][c0 + jj] : (long long)ti.out_row + c0 + jj;
               if (jj < jn && fbase + part * 8 < c.R && orow >= 0) {
-                const float* v = &stg[q][jj][part * 8];
+                const float* v = &stg[ew][jj][part * 8];
                 uint4 pk;
                 pk.x = pack_bf16x2(v[0], v[1]);
                 pk.y = pack_bf16x2(v[2], v[3]);
@@ -916,25 +927,25 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
       uint32_t ra0[16], ra1[16], rb0[16], rb1[16];
 #pragma unroll
       for (int j = 0; j < 16; ++j) ra1[j] = rb1[j] = 0u;
-      if (rows > 0) {
-        tmem_ld_x16(t_row, ra0);
-        if (MATS == 2) tmem_ld_x16(t_row + BN, ra1);
+      if (cfirst < rows) {
+        tmem_ld_x16(t_row + cfirst, ra0);
+        if (MATS == 2) tmem_ld_x16(t_row + BN + cfirst, ra1);
       }
 #pragma unroll 1
-      for (int c0 = 0; c0 < rows; c0 += 32) {
+      for (int c0 = cfirst; c0 < rows; c0 += 2 * cstep) {
         if (MATS == 2) tmem_ld_wait_keep(ra0, ra1); else tmem_ld_wait_keep(ra0);
-        if (c0 + 16 < rows) {
-          tmem_ld_x16(t_row + c0 + 16, rb0);
-          if (MATS == 2) tmem_ld_x16(t_row + BN + c0 + 16, rb1);
+        if (c0 + cstep < rows) {
+          tmem_ld_x16(t_row + c0 + cstep, rb0);
+          if (MATS == 2) tmem_ld_x16(t_row + BN + c0 + cstep, rb1);
         }
         chunk(c0, ra0, ra1);
-        if (c0 + 16 >= rows) break;
+        if (c0 + cstep >= rows) break;
         if (MATS == 2) tmem_ld_wait_keep(rb0, rb1); else tmem_ld_wait_keep(rb0);
-        if (c0 + 32 < rows) {
-          tmem_ld_x16(t_row + c0 + 32, ra0);
-          if (MATS == 2) tmem_ld_x16(t_row + BN + c0 + 32, ra1);
+        if (c0 + 2 * cstep < rows) {
+          tmem_ld_x16(t_row + c0 + 2 * cstep, ra0);
+          if (MATS == 2) tmem_ld_x16(t_row + BN + c0 + 2 * cstep, ra1);
         }
-        chunk(c0 + 16, rb0, rb1);
+        chunk(c0 + cstep, rb0, rb1);
       }
       tc_fence_before();
       __syncwarp();
@@ -1024,7 +1035,7 @@ static cudaError_t launch_impl(const TcMaps& maps, const GemmParams& p, int num_
     // free SMs leaves one SM out)
     static int max_pairs = 0;
     cudaLaunchConfig_t cfg = {};
-    cfg.blockDim = dim3(TC_THREADS);
+    cfg.blockDim = dim3(tc_threads<EPI, PAIR, F8>());
     cfg.dynamicSmemBytes = S::DYN_SMEM;
     cfg.stream = s;
     cudaLaunchAttribute attr[2];
@@ -1051,7 +1062,7 @@ static cudaError_t launch_impl(const TcMaps& maps, const GemmParams& p, int num_
     if (e != cudaSuccess) return e;
     return cudaGetLastError();
   }
-  launch_k(kern, num_ctas, TC_THREADS, S::DYN_SMEM, s, m[0], m[1], m[2], m[3], m[4], m[5], p);
+  launch_k(kern, num_ctas, tc_threads<EPI, PAIR, F8>(), S::DYN_SMEM, s, m[0], m[1], m[2], m[3], m[4], m[5], p);
   count_launch();
   return cudaGetLastError();
 }
