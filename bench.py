@@ -343,9 +343,9 @@ def T_bytes(cfg) -> int:
 
 
 def fused_routing(cfg) -> bool:
-    """The library's rule for its tile-rank routing (tensor-core logits, then top-k and
-    128-token tile ranks in one kernel) followed by the one-kernel scatter: bf16, 8192+
-    tokens, m <= 256, k <= 8."""
+    """The library's rule for its one-launch router (logits + top-k + tile ranks in the
+    tensor-core epilogue) followed by the one-kernel scatter: bf16, 8192+ tokens,
+    m <= 256, k <= 8."""
     return cfg.dtype == W.BF16 and cfg.T >= 8192 and cfg.m <= 256 and cfg.k <= 8
 
 
@@ -365,10 +365,9 @@ def stage_costs(cfg, active: int, ksplit: int, weight_bytes=None):
     c["histogram_lis_ranks"] = (0.0, Tk * 4 + Tk * 8 + (m + 1) * 8)
     c["permute"] = (0.0, Tk * 4 + T * d * es + Tk * d * es)
     tiles = (T + 127) // 128
-    # tile-rank routing: the logits, then top-k + ranks (logits in; ids, weights, tile
-    # ranks and tile counts out); the scatter reads those back and writes perm / inv_perm
-    # / w_perm, counts, offsets and x_perm
-    c["topk_ranks"] = (0.0, T * m * 4 + Tk * 12 + tiles * m * 4)
+    # fused routing: x and W_r in, ids, weights, tile ranks and tile counts out; then the
+    # scatter reads those back and writes perm / inv_perm / w_perm, counts, offsets and x_perm
+    c["router_topk_ranks"] = (2.0 * T * d * m, T * d * es + m * d * es + Tk * 12 + tiles * m * 4)
     c["scatter"] = (0.0, tiles * m * 4 + Tk * 12 + Tk * 12 + (2 * m + 1) * 4 + T * d * es + Tk * d * es)
     c["expert_up"] = (2.0 * mats * f * d * Tk + 2.0 * mats * fsh * d * T * nsh,
                       active * mats * f * d * ew + nsh * mats * fsh * d * ew + Tk * d * es + (T * d * es if nsh else 0)
@@ -595,10 +594,10 @@ def layer_run(cfg, args, dev, rank: int, world: int, dist, steps, warmup: int, w
     dom = max(STAGES, key=lambda n: stage_ms[n])
     jd = STAGES.index(dom)
     if fused_routing(cfg) and not rep:
-        # stages 1-2 are top-k + tile ranks, 3-4 the scatter; stages 2-3 coincide
-        stage_ms = {("topk_ranks" if n == "topk" else "scatter" if n == "permute" else n): v
-                    for n, v in stage_ms.items() if n != "histogram_lis_ranks"}
-        dom = {"topk": "topk_ranks", "permute": "scatter"}.get(dom, dom)
+        # one kernel spans stages 0-1 and one spans 3-4; the two boundaries between them coincide
+        stage_ms = {("router_topk_ranks" if n == "router" else "scatter" if n == "permute" else n): v
+                    for n, v in stage_ms.items() if n not in ("topk", "histogram_lis_ranks")}
+        dom = {"router": "router_topk_ranks", "permute": "scatter"}.get(dom, dom)
     K = steps if steps else max(3, int(math.ceil(min_timed_ms / max(prof_step_ms, 1e-3))))
 
     def timed(nsteps):

@@ -233,11 +233,9 @@ cudaError_t launch_route(const moe_config_t& c, const void* x, const void* w_r, 
                          int* status, cudaStream_t s, bool stage_marks) {
   cudaError_t e = cudaSuccess;
   const float* lg = logits_in;
-  if (!lg && fused_route_ok(c)) {  // large batches: tensor-core logits, then one block per 128-token tile
-    float* dst = logits_out ? logits_out : logits_scratch;
-    if ((e = launch_router_logits(c, x, w_r, bias, dst, status, s)) != cudaSuccess) return e;
-    if (stage_marks && (e = mark_stage_event(1, s)) != cudaSuccess) return e;
-    e = launch_route_topk_rank(c.T, c.m, c.k, c.renormalize, dst, idx, w, nullptr, nullptr, status, s);
+  if (!lg && fused_route_ok(c)) {  // logits and top-k in one tensor-core launch
+    e = launch_route_topk(c, x, w_r, bias, logits_out, idx, w, nullptr, nullptr, status, g_wait_limit_ns, s);
+    if (e == cudaSuccess && stage_marks) e = mark_stage_event(1, s);
     if (e == cudaSuccess && stage_marks) e = mark_stage_event(2, s);
     return e;
   }
@@ -677,14 +675,12 @@ static moe_status_t layer_forward_impl(const moe_config_t& c, const void* x, con
   float* w_perm = at<float>(ws, L.w_perm);
   MOE_TRY(mark_stage(0, s));
   if (fused_route_ok(c)) {
-    // large batches: tensor-core logits; top-k, gate weights and each 128-token
-    // tile's per-expert counts and ranks in one block per tile; then one kernel for
-    // offsets / LIS / permutation / row copy (stages 2 and 3 coincide)
+    // router + top-k + per-tile counts and ranks in the GEMM epilogue, then one
+    // kernel for offsets / LIS / permutation / row copy (stages 1-3 coincide)
     int32_t* lrank = at<int32_t>(ws, L.lrank);
     int32_t* tile_cnt = at<int32_t>(ws, L.tile_cnt);
-    MOE_TRY(run_router(c, x, w_router, bias, logits, status, s));
+    MOE_CUDA(launch_route_topk(c, x, w_router, bias, logits_out, idx, w, lrank, tile_cnt, status, g_wait_limit_ns, s));
     MOE_TRY(mark_stage(1, s));
-    MOE_CUDA(launch_route_topk_rank(c.T, c.m, c.k, c.renormalize, logits, idx, w, lrank, tile_cnt, status, s));
     MOE_TRY(mark_stage(2, s));
     MOE_TRY(mark_stage(3, s));
     MOE_CUDA(launch_route_scatter(c.dtype, c.T, c.k, c.m, c.d, tile_cnt, idx, lrank, w, x, counts, offsets, lis, perm,

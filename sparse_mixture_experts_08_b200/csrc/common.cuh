@@ -211,10 +211,6 @@ cudaError_t launch_few_expert_logits(int T, int d, int m, const void* x, const v
                                      float* logits, cudaStream_t s);
 cudaError_t launch_topk_softmax(int T, int m, int k, int renorm, const float* logits, int32_t* idx, float* w,
                                 cudaStream_t s);
-// top-k ids and gate weights from logits [T, m] (m <= 256, k <= 8), and when lrank and
-// tile_cnt are given the per-128-token-tile ranks and counts route_scatter takes.
-cudaError_t launch_route_topk_rank(int T, int m, int k, int renorm, const float* logits, int32_t* idx, float* w,
-                                   int32_t* lrank, int32_t* tile_cnt, int* status, cudaStream_t s);
 // logits (nullable), top-k ids and gate weights in one launch: bf16 layers with m <= 16.
 bool small_route_ok(int dtype, int m);
 cudaError_t launch_small_route(int T, int d, int m, int k, int renorm, const void* x, const void* w, const float* bias,

@@ -337,128 +337,6 @@ cudaError_t launch_topk_softmax(int T, int m, int k, int renorm, const float* lo
   return cudaGetLastError();
 }
 
-// ------------------------------------------------ top-k, gate weights and tile ranks, large batches
-// One block of RT_THREADS per 128-token tile of the router logits (written by the
-// tensor-core logits kernel, bias included). Each warp takes 4 tokens, its lanes the
-// experts e = lane + 32 u: k rounds of a warp arg-max by (logit desc, expert asc)
-// over the experts not yet picked, then the gate weights with the arithmetic of
-// topk_softmax_kernel (exp in fp32 of l - max, sums in fp64, renormalised over the
-// k chosen when asked). When lrank and tile_cnt are given, the tile's picks then
-// go into per-expert 128-bit token masks (shared memory): a task's rank among the
-// tile's tasks of its expert, in (token, slot) order, is the popcount of its
-// expert's mask below its token (a token picks an expert at most once), and the
-// tile's count of an expert is its mask's popcount. These are the tables
-// route_scatter_kernel turns into offsets, LIS and the permutation.
-constexpr int RT_THREADS = 1024;
-
-__global__ void __launch_bounds__(RT_THREADS)
-    route_topk_rank_kernel(int T, int m, int k, int renorm, const float* __restrict__ logits,
-                           int32_t* __restrict__ idx, float* __restrict__ w, int32_t* __restrict__ lrank,
-                           int32_t* __restrict__ tile_cnt, int* status) {
-  __shared__ int pick[128][ROUTE_MAX_K];
-  __shared__ uint32_t mask[ROUTE_MAX_M][4];
-  __shared__ int bad_s;
-  const int tile = blockIdx.x, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const long long t0 = (long long)tile * 128;
-  const int nu = (m + 31) / 32;  // experts per lane (<= 8)
-  for (int i = tid; i < ROUTE_MAX_M * 4; i += RT_THREADS) mask[i >> 2][i & 3] = 0u;
-  if (tid == 0) bad_s = 0;
-  pdl_launch_dependents();
-  pdl_wait();
-  __syncthreads();
-  for (int j = warp; j < 128; j += RT_THREADS / 32) {
-    const long long t = t0 + j;
-    if (t >= T) break;  // the same for the whole warp
-    const float* L = logits + t * m;
-    float v[8];
-#pragma unroll
-    for (int u = 0; u < 8; ++u) v[u] = (u < nu && lane + 32 * u < m) ? L[lane + 32 * u] : -INFINITY;
-    uint32_t taken = 0u;  // bit u: this lane's expert lane + 32 u is picked
-    float pv[ROUTE_MAX_K];
-    int pe[ROUTE_MAX_K];
-#pragma unroll
-    for (int s2 = 0; s2 < ROUTE_MAX_K; ++s2) {
-      if (s2 >= k) break;
-      float bv = -INFINITY;
-      int be = 0x7fffffff;
-#pragma unroll
-      for (int u = 0; u < 8; ++u) {
-        const int e = lane + 32 * u;
-        if (u < nu && e < m && !(taken >> u & 1u) && (be == 0x7fffffff || v[u] > bv)) {  // ascending e
-          bv = v[u];
-          be = e;
-        }
-      }
-#pragma unroll
-      for (int o = 16; o; o >>= 1) {
-        const float ov = __shfl_xor_sync(FULL, bv, o);
-        const int oe = __shfl_xor_sync(FULL, be, o);
-        if (oe != 0x7fffffff && (be == 0x7fffffff || ov > bv || (ov == bv && oe < be))) {
-          bv = ov;
-          be = oe;
-        }
-      }
-      if (be != 0x7fffffff && (be & 31) == lane) taken |= 1u << (be >> 5);
-      pv[s2] = bv;
-      pe[s2] = be == 0x7fffffff ? -1 : be;
-    }
-    const float mx = pv[0];
-    double z = 0.0;
-#pragma unroll
-    for (int u = 0; u < 8; ++u)
-      if (u < nu && lane + 32 * u < m) z += (double)expf(v[u] - mx);
-#pragma unroll
-    for (int o = 16; o; o >>= 1) z += __shfl_xor_sync(FULL, z, o);
-    double sel = 0.0;
-#pragma unroll
-    for (int s2 = 0; s2 < ROUTE_MAX_K; ++s2)
-      if (s2 < k) sel += (double)expf(pv[s2] - mx) / z;
-#pragma unroll
-    for (int s2 = 0; s2 < ROUTE_MAX_K; ++s2) {
-      if (s2 >= k) break;
-      if (lane == s2) {
-        double pr = (double)expf(pv[s2] - mx) / z;
-        if (renorm) pr /= sel;
-        idx[t * k + s2] = pe[s2];
-        w[t * k + s2] = (float)pr;
-        pick[j][s2] = pe[s2];
-        if (pe[s2] < 0) bad_s = 1;  // NaN logits
-      }
-    }
-  }
-  if (!lrank) {
-    __syncthreads();
-    if (tid == 0 && bad_s) set_status(status, MOE_ERR_DEVICE_INDEX);
-    return;
-  }
-  __syncthreads();
-  const int ntok = (int)(T - t0 < 128 ? T - t0 : 128);
-  for (int i = tid; i < ntok * k; i += RT_THREADS) {
-    const int j = i / k, e = pick[j][i - j * k];
-    if (e >= 0 && e < m) atomicOr(&mask[e][j >> 5], 1u << (j & 31));
-  }
-  __syncthreads();
-  for (int i = tid; i < ntok * k; i += RT_THREADS) {
-    const int j = i / k, e = pick[j][i - j * k];
-    if (e < 0 || e >= m) continue;
-    int rk = __popc(mask[e][j >> 5] & ((1u << (j & 31)) - 1u));
-    for (int q = 0; q < (j >> 5); ++q) rk += __popc(mask[e][q]);
-    lrank[(t0 + j) * k + (i - j * k)] = rk;
-  }
-  for (int e = tid; e < m; e += RT_THREADS)
-    tile_cnt[(long long)tile * m + e] =
-        __popc(mask[e][0]) + __popc(mask[e][1]) + __popc(mask[e][2]) + __popc(mask[e][3]);
-  if (tid == 0 && bad_s) set_status(status, MOE_ERR_DEVICE_INDEX);
-}
-
-cudaError_t launch_route_topk_rank(int T, int m, int k, int renorm, const float* logits, int32_t* idx, float* w,
-                                   int32_t* lrank, int32_t* tile_cnt, int* status, cudaStream_t s) {
-  launch_k(route_topk_rank_kernel, (T + 127) / 128, RT_THREADS, 0, s, T, m, k, renorm, logits, idx, w, lrank,
-           tile_cnt, status);
-  count_launch();
-  return cudaGetLastError();
-}
-
 // ------------------------------------------------ histogram, offsets, LIS, range starts
 // The T k tasks (q = t k + s, in increasing order) are cut into R contiguous
 // ranges of L tasks; range r holds tasks [r L, min(T k, (r + 1) L)). One block of
