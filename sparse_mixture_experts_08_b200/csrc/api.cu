@@ -1098,7 +1098,8 @@ moe_status_t moe_layer_forward_replicated(const moe_config_t* cfg, const void* x
 
 // ------------------------------------------------------------------ FloE contextual sparsity
 struct FloeLayout {
-  size_t u, list, cnt, hc, y, total;
+  size_t u, list, cnt, rsplit, y, total;
+  int slots;
 };
 
 static FloeLayout make_floe_layout(const moe_config_t& c, size_t base) {
@@ -1114,8 +1115,9 @@ static FloeLayout make_floe_layout(const moe_config_t& c, size_t base) {
   F.u = take(Tk * c.f * 4);
   F.list = take((size_t)c.m * nch * floe_chunk_size() * 4);
   F.cnt = take((size_t)c.m * nch * 4);
-  F.hc = take(Tk * c.f * 4);
-  F.y = take((size_t)floe_splits() * Tk * c.d * 4);  // partial outputs of the kept-channel ranges
+  F.rsplit = take(Tk * 4);
+  F.slots = floe_max_slots((long long)Tk, c.d);
+  F.y = take((size_t)F.slots * Tk * c.d * 4);  // partial outputs of the kept-channel ranges
   F.total = off;
   return F;
 }
@@ -1246,11 +1248,12 @@ moe_status_t moe_layer_forward_floe(const moe_config_t* cfg, const void* x, cons
   MOE_CUDA(launch_tc_gemm(EPI_LOGITS, tc_pick_bn(EPI_LOGITS, (double)Tk / c.m), mu, up, num_sms(), s));
   MOE_TRY(mark_stage(5, s));
   // kept channels, gate rows and down rows of the kept channels only
+  int32_t* rsplit = at<int32_t>(ws, F.rsplit);
   MOE_CUDA(launch_floe_sparse_ffn(c.m, c.d, c.f, offsets, x_perm, w_gate, w_down_t, u, thresholds,
-                                  at<int32_t>(ws, F.list), at<int32_t>(ws, F.cnt), at<float>(ws, F.hc), w_perm, y,
-                                  Tk * c.d, kept_out, status, s));
+                                  at<int32_t>(ws, F.list), at<int32_t>(ws, F.cnt), w_perm, y, Tk * c.d, F.slots,
+                                  rsplit, kept_out, status, g_wait_limit_ns, s));
   MOE_TRY(mark_stage(6, s));
-  MOE_CUDA(launch_combine(c.dtype, c.T, c.d, c.k, floe_splits(), y, Tk * c.d, inv_perm, 0, nullptr, 0, out, s));
+  MOE_CUDA(launch_combine(c.dtype, c.T, c.d, c.k, F.slots, y, Tk * c.d, inv_perm, 0, nullptr, 0, out, s, rsplit));
   if (u_out) MOE_CUDA(cudaMemcpyAsync(u_out, u, (size_t)Tk * c.f * 4, cudaMemcpyDeviceToDevice, s));
   if (perm_out) MOE_CUDA(cudaMemcpyAsync(perm_out, perm, (size_t)Tk * 4, cudaMemcpyDeviceToDevice, s));
   return mark_stage(7, s);

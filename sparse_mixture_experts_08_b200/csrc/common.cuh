@@ -239,14 +239,17 @@ cudaError_t launch_replica_split(int T, int k, int m, const int32_t* idx, const 
 // FloE contextual sparsity (csrc/floe.cu)
 cudaError_t launch_floe_pack(int m, int d, int f, const void* w, void* w_t, cudaStream_t s);
 cudaError_t launch_floe_calib(int Tc, int m, int f, const float* u, double sparsity, float* thr, cudaStream_t s);
+// keep lists, then the gate + down stream writing partial outputs y[slot][row][:]
+// (row_splits[row] slots per row, at most max_slots)
 cudaError_t launch_floe_sparse_ffn(int m, int d, int f, const int32_t* offsets, const void* x_perm,
                                    const void* w_gate, const void* w_down_t, const float* u, const float* thr,
-                                   int32_t* list, int32_t* cnt, float* hc, const float* row_w, float* y,
-                                   long long y_split, int32_t* kept_out, int* status, cudaStream_t s);
+                                   int32_t* list, int32_t* cnt, const float* row_w, float* y, long long y_split,
+                                   int max_slots, int32_t* row_splits, int32_t* kept_out, int* status,
+                                   unsigned long long lim, cudaStream_t s);
 int floe_chunks(int f);
 int floe_chunk_size();
-int floe_splits();                 // partial outputs of the sparse down projection (summed by the combine)
-bool floe_shape_ok(int d, int f);  // d <= 8192, f <= 65536
+int floe_max_slots(long long rows, int d);  // partial-output slots the workspace holds per row
+bool floe_shape_ok(int d, int f);           // d <= 8192, f <= 65536
 cudaError_t launch_rank(int T, int k, int m, const int32_t* idx, const int32_t* offsets, const int32_t* start,
                         const float* task_w, int32_t* perm, int32_t* inv_perm, float* w_perm, int* status,
                         cudaStream_t s);
@@ -254,7 +257,7 @@ cudaError_t launch_permute_rows(int dtype, int Tk, int k, int d, const void* x, 
                                 cudaStream_t s);
 cudaError_t launch_combine(int dtype, int T, int d, int k, int ksplit, const float* y_perm, long long y_split_stride,
                            const int32_t* inv_perm, int n_shared, const float* y_shared, long long ysh_split_stride,
-                           void* out, cudaStream_t s);
+                           void* out, cudaStream_t s, const int32_t* row_splits = nullptr);
 cudaError_t launch_reduce_splits(long long n, int ksplit, const float* in, long long split_stride, float* out,
                                  cudaStream_t s);
 

@@ -953,7 +953,8 @@ cudaError_t launch_replica_split(int T, int k, int m, const int32_t* idx, const 
 // ------------------------------------------------------------------ combine
 // out[t, c] = sum_s sum_split y[split][inv_perm[t k + s], c]
 //           + sum_sh sum_split ysh[split][sh T + t, c], fp32, slot order; 4 columns
-// per thread (16-byte loads).
+// per thread (16-byte loads). With row_splits the routed rows have their own split
+// counts (row_splits[pos] <= ksplit partials for permuted row pos).
 template <typename OutT>
 __device__ __forceinline__ void store4(OutT* out, long long i4, float4 v);
 template <>
@@ -972,7 +973,7 @@ __device__ __forceinline__ void store4<__nv_bfloat16>(__nv_bfloat16* out, long l
 template <typename OutT>
 __global__ void combine_kernel(int T, int d4, int k, int ksplit, const float4* __restrict__ y, long long ysplit4,
                                const int32_t* __restrict__ inv_perm, int n_sh, const float4* __restrict__ ysh,
-                               long long yshsplit4, OutT* __restrict__ out) {
+                               long long yshsplit4, OutT* __restrict__ out, const int32_t* __restrict__ row_splits) {
   pdl_launch_dependents();
   pdl_wait();
   const long long n = (long long)T * d4;
@@ -984,7 +985,8 @@ __global__ void combine_kernel(int T, int d4, int k, int ksplit, const float4* _
     for (int s = 0; s < k; ++s) {
       const int pos = inv_perm[t * k + s];
       if (pos < 0 || pos >= Tk) continue;
-      for (int sp = 0; sp < ksplit; ++sp) {
+      const int ns = row_splits ? min(ksplit, row_splits[pos]) : ksplit;
+      for (int sp = 0; sp < ns; ++sp) {
         const float4 v = y[sp * ysplit4 + (long long)pos * d4 + c];
         a.x += v.x; a.y += v.y; a.z += v.z; a.w += v.w;
       }
@@ -1000,18 +1002,18 @@ __global__ void combine_kernel(int T, int d4, int k, int ksplit, const float4* _
 
 cudaError_t launch_combine(int dtype, int T, int d, int k, int ksplit, const float* y_perm, long long y_split_stride,
                            const int32_t* inv_perm, int n_shared, const float* y_shared, long long ysh_split_stride,
-                           void* out, cudaStream_t s) {
+                           void* out, cudaStream_t s, const int32_t* row_splits) {
   const int d4 = d / 4;
   const long long n = (long long)T * d4;
   const int blocks = (int)std::max<long long>(1, std::min<long long>((n + 255) / 256, (long long)num_sms() * 16));
   if (dtype == MOE_F32)
     launch_k(combine_kernel<float>, blocks, 256, 0, s, T, d4, k, ksplit, (const float4*)y_perm, y_split_stride / 4, inv_perm,
                                                  y_shared ? n_shared : 0, (const float4*)y_shared,
-                                                 ysh_split_stride / 4, (float*)out);
+                                                 ysh_split_stride / 4, (float*)out, row_splits);
   else
     launch_k(combine_kernel<__nv_bfloat16>, blocks, 256, 0, s, T, d4, k, ksplit, (const float4*)y_perm, y_split_stride / 4,
                                                          inv_perm, y_shared ? n_shared : 0, (const float4*)y_shared,
-                                                         ysh_split_stride / 4, (__nv_bfloat16*)out);
+                                                         ysh_split_stride / 4, (__nv_bfloat16*)out, row_splits);
   count_launch();
   return cudaGetLastError();
 }

@@ -75,6 +75,23 @@ def _floe_layer(cfg, inp, thr):
 CASES = [
     (W.small_moe(T=16, d=256, f=320, m=4, k=2, dtype=W.BF16, zipf_s=0.5, index=112, name="small"), 0.8),
     (W.CONFIGS["decode"], 0.9),
+    # d > 4096: four 16-byte column chunks per thread, two channels per stage, a
+    # ragged last column slice; ~27 rows per expert = several 4-row passes (sparsity
+    # high enough that the union over an expert's rows still skips channels)
+    (W.small_moe(T=40, d=4352, f=200, m=3, k=2, dtype=W.BF16, zipf_s=0.3, index=114, name="wide"), 0.97),
+    # 3 keep-list chunks (the last ragged) and a hot expert with many passes
+    (W.small_moe(T=300, d=512, f=2056, m=6, k=2, dtype=W.BF16, zipf_s=1.2, index=115, name="chunks"), 0.995),
+    # f = 16 caps the channel ranges per expert, so its blocks also split the passes
+    (W.small_moe(T=300, d=256, f=16, m=2, k=1, dtype=W.BF16, zipf_s=0.0, index=116, name="row_split"), 0.995),
+    # more experts than blocks to share out, most of them without tokens
+    (W.small_moe(T=64, d=64, f=48, m=160, k=2, dtype=W.BF16, zipf_s=0.8, index=117, name="many_experts"), 0.5),
+    # the tensor-core variants: 4 and 8 column units per warp (d = 2048 without column
+    # checks), and token rows staged in shared memory with a ragged last unit (d = 3000)
+    # and without (d = 4096), several 8-row passes each
+    (W.small_moe(T=48, d=768, f=264, m=4, k=2, dtype=W.BF16, zipf_s=0.4, index=118, name="d768"), 0.95),
+    (W.small_moe(T=40, d=2048, f=200, m=4, k=2, dtype=W.BF16, zipf_s=0.4, index=119, name="d2048"), 0.95),
+    (W.small_moe(T=40, d=3000, f=136, m=3, k=2, dtype=W.BF16, zipf_s=0.4, index=120, name="d3000"), 0.97),
+    (W.small_moe(T=64, d=4096, f=256, m=4, k=2, dtype=W.BF16, zipf_s=0.4, index=121, name="d4096_passes"), 0.97),
 ]
 
 
