@@ -632,10 +632,11 @@ __global__ void __launch_bounds__(FS_THREADS, 1)
 // [w KT, (w + 1) KT) of d, for the gate's reduction dimension and the down's output
 // columns alike. Lane (g = lane / 4, t = lane % 4) holds, per unit u:
 //   gate  (M = 16 token rows, 8 real; N = 8 channels, CB real; K = the unit):
-//         A = x[g][16u + 2t, +1] and x[g][16u + 8 + 2t, +1], from registers loaded once
-//         per pass, or (XS) through ldmatrix from the pass's token rows staged in
-//         shared memory; B = the staged gate rows through ldmatrix (a channel's row
-//         is a tile row); D = this warp's partial g[g][2t, 2t + 1];
+//         A = x[g][16u + 2t, +1] and x[g][16u + 8 + 2t, +1], built once per pass and
+//         kept in registers, or (XS, from 8 units per warp on, so that the registers
+//         can hold the accumulators) as the pass's token rows staged in shared memory
+//         and read through ldmatrix; B = the staged gate rows through ldmatrix (a
+//         channel's row is a tile row); D = this warp's partial g[g][2t, 2t + 1];
 //   down  (M = the unit's 16 columns; N = 8 token rows; K = 8 channels, CB real):
 //         A = the staged down rows through ldmatrix.trans (channel = tile row, its 8
 //         columns transposed into the fragment); B = h[g][2t, 2t + 1] as bf16;
@@ -896,7 +897,7 @@ cudaError_t launch_floe_sparse_ffn(int m, int d, int f, const int32_t* offsets, 
   if (err != cudaSuccess) return err;
   const int nblk = num_sms();
   const dim3 grid(nblk + m);
-#define MOE_FLOE_RING(KERN_, CB_, XS_BYTES_, THREADS_, XT_)                                                     \
+#define MOE_FLOE_RING(KERN_, CB_, XS_BYTES_, THREADS_, XTYPE_)                                                  \
   do {                                                                                                          \
     const size_t stage = (size_t)(CB_) * 2 * fs_pitch(d), xs_bytes = (XS_BYTES_);                              \
     const int nst = (int)std::min<size_t>(FS_MAX_STAGES, (FS_DYN_BYTES - xs_bytes) / stage);                   \
@@ -909,12 +910,14 @@ cudaError_t launch_floe_sparse_ffn(int m, int d, int f, const int32_t* offsets, 
       attr = true;                                                                                              \
     }                                                                                                           \
     err = launch_k(KERN_, grid, THREADS_, dyn, s, m, d, f, nchunks, nst, nblk, max_slots, offsets,             \
-                   (const XT_*)x_perm, (const __nv_bfloat16*)w_gate, (const __nv_bfloat16*)w_down_t, u, thr,    \
+                   (const XTYPE_*)x_perm, (const __nv_bfloat16*)w_gate, (const __nv_bfloat16*)w_down_t, u, thr, \
                    (const int32_t*)list, (const int32_t*)cnt, row_w, y, y_split, row_splits, kept_out, status,  \
                    lim);                                                                                        \
   } while (0)
   const int n16 = (d + 15) / 16;
-  if (d == 4096)  // token rows staged in shared memory (registers hold the accumulators), 3 channels per stage
+  // token-row fragments in registers up to 4 units per warp (and at d = 2048), else
+  // staged in shared memory so the registers can hold the accumulators
+  if (d == 4096)
     MOE_FLOE_RING((floe_mma_kernel<16, true, 3, true>), 3, (size_t)FM_ROWS * fs_pitch(d), FM_THREADS, uint32_t);
   else if (d == 2048)
     MOE_FLOE_RING((floe_mma_kernel<8, true, FM_CB, false>), FM_CB, 0, FM_THREADS, uint32_t);
@@ -924,7 +927,7 @@ cudaError_t launch_floe_sparse_ffn(int m, int d, int f, const int32_t* offsets, 
     MOE_FLOE_RING((floe_mma_kernel<2, false, FM_CB, false>), FM_CB, 0, FM_THREADS, uint32_t);
   else if (n16 <= 4 * FM_WARPS)
     MOE_FLOE_RING((floe_mma_kernel<4, false, FM_CB, false>), FM_CB, 0, FM_THREADS, uint32_t);
-  else if (n16 <= 8 * FM_WARPS)  // token rows staged in shared memory (registers hold the accumulators)
+  else if (n16 <= 8 * FM_WARPS)
     MOE_FLOE_RING((floe_mma_kernel<8, false, FM_CB, true>), FM_CB, (size_t)FM_ROWS * fs_pitch(d), FM_THREADS,
                   uint32_t);
   else if (d <= FM_MAX_D)  // 2048 < d < 4096: as at 4096, with column checks

@@ -986,8 +986,18 @@ __global__ void combine_kernel(int T, int d4, int k, int ksplit, const float4* _
       const int pos = inv_perm[t * k + s];
       if (pos < 0 || pos >= Tk) continue;
       const int ns = row_splits ? min(ksplit, row_splits[pos]) : ksplit;
-      for (int sp = 0; sp < ns; ++sp) {
-        const float4 v = y[sp * ysplit4 + (long long)pos * d4 + c];
+      const float4* yp = y + (long long)pos * d4 + c;
+      int sp = 0;
+      for (; sp + 4 <= ns; sp += 4) {  // four partials' loads in flight together, added in order
+        const float4 v0 = yp[sp * ysplit4], v1 = yp[(sp + 1) * ysplit4], v2 = yp[(sp + 2) * ysplit4],
+                     v3 = yp[(sp + 3) * ysplit4];
+        a.x += v0.x; a.y += v0.y; a.z += v0.z; a.w += v0.w;
+        a.x += v1.x; a.y += v1.y; a.z += v1.z; a.w += v1.w;
+        a.x += v2.x; a.y += v2.y; a.z += v2.z; a.w += v2.w;
+        a.x += v3.x; a.y += v3.y; a.z += v3.z; a.w += v3.w;
+      }
+      for (; sp < ns; ++sp) {
+        const float4 v = yp[sp * ysplit4];
         a.x += v.x; a.y += v.y; a.z += v.z; a.w += v.w;
       }
     }
