@@ -739,7 +739,8 @@ def ours(args):
     long_step = K * ms > 1000.0
     fl, by = r["costs"][r["dom"]]
     roof = roofline_for(cfg, r["dom"], fl, by, r["dom_ms"], pk, pk_src, long_step, fp8,
-                        cfg.name + ("_fp8" if fp8 else ""))
+                        cfg.name + ("_fp8" if fp8 else "") + ("_floe" if floe is not None else "")
+                        + ("_replicated" if rep else ""))
     tensor_peak = (pk["bf16_tflops_sustained"] if long_step else pk["bf16_tflops"]) * (2.0 if fp8 else 1.0)
     t_layer = max(r["layer_flops"] / (tensor_peak * 1e12), r["layer_bytes"] / (pk["hbm_gbs"] * 1e9))
     variant_note = {}
