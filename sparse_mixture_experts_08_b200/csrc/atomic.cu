@@ -130,8 +130,8 @@ __device__ void block_top64(uint64_t k0, uint64_t k1, bool mine, int lw, int nch
 }
 
 // Row and column log-probabilities of token t into shared lr[Nr], lc[Nc] (and
-// lr_out / lc_out when given): the split-K partials summed in split order (all
-// loads of a thread in flight together), then log-softmax with a block-wide
+// lr_out / lc_out when given): the split-K partials summed in split order (up to 16
+// loads of each side in flight together), then log-softmax with a block-wide
 // log-sum-exp (a fixed shuffle tree per warp, then warp 0 over the warps: the same
 // result on every run). One thread per row and per column (blockDim = SEL_THREADS
 // >= Nr, Nc); ends with a block barrier.
@@ -143,16 +143,16 @@ __device__ void block_logprobs(int t, int Nr, int Nc, int ksplit, const float* _
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const bool hr = tid < Nr, hc = tid < Nc;
   float ar = 0.f, ac = 0.f;
-  for (int s0 = 0; s0 < ksplit; s0 += 8) {
-    float vr[8], vc[8];
+  for (int s0 = 0; s0 < ksplit; s0 += 16) {
+    float vr[16], vc[16];
 #pragma unroll
-    for (int u = 0; u < 8; ++u) {
+    for (int u = 0; u < 16; ++u) {
       const int s = s0 + u;
       vr[u] = (s < ksplit && hr) ? zr[s * zr_split + (long long)t * Nr + tid] : 0.f;
       vc[u] = (s < ksplit && hc) ? zc[s * zc_split + (long long)t * Nc + tid] : 0.f;
     }
 #pragma unroll
-    for (int u = 0; u < 8; ++u) {
+    for (int u = 0; u < 16; ++u) {
       if (s0 + u < ksplit) {
         ar += vr[u];
         ac += vc[u];
@@ -689,42 +689,49 @@ cudaError_t launch_atomic_select(int T, int Nr, int Nc, int K, int ksplit, const
 }
 
 // ------------------------------------------------------------------ assembly
-constexpr int ASM_GROUPS = 4, ASM_BATCH = 16;  // phase 2: slot groups per 8 columns, loads per batch
+constexpr int ASM_GROUPS = 16, ASM_BATCH = 4;  // phase 2: slot groups per 8 columns, loads per batch
 
-// The atomic-expert FFN (OmniMoE Eq. 4) in one cooperative launch, one block per SM:
-//  phase 1, one warp per task (t, s): coef[t, s] = g[t, s] act(x_t . w_in[idx[t, s]]),
-//    fp32 FMAs over each lane's 16-byte chunks in ascending order then a shuffle
-//    tree; when all gathered w_out rows fit comfortably in L2 (decode budgets) the
-//    warp also prefetches the task's w_out row for phase 2;
+// The atomic-expert FFN (OmniMoE Eq. 4) in one cooperative launch, one 1024-thread
+// block per SM (all of them resident, as the grid barrier needs):
+//  phase 1, AX_PARTS warps per task (t, s), each over its quarter of d:
+//    coef[t, s] = g[t, s] act(x_t . w_in[idx[t, s]]), fp32 FMAs over each lane's
+//    16-byte chunks in ascending order, a shuffle tree per warp, and the parts added
+//    in part order; when all gathered w_out rows fit comfortably in L2 (decode
+//    budgets) each warp also prefetches its part of the task's w_out row for phase 2;
 //  a grid-wide barrier (bounded: on expiry the block records MOE_ERR_TIMEOUT and
 //    returns without phase 2, whose coefficients other blocks may not have written);
-//  phase 2, four lanes per 8 output columns: lane group j sums slots j, j + 4, ...
-//    in order, and out[t, c..c+7] = ((group 0 + group 1) + group 2) + group 3,
+//  phase 2, sixteen lanes per 8 output columns: lane group j sums slots j, j + 16,
+//    ... in order, the groups are added by a fixed xor tree, and out[t, c..c+7] is
 //    rounded to bf16, so the result is the same on every run.
-constexpr int AX_THREADS = 256;
+// Splitting each dot product over four warps and each output chunk over sixteen
+// lanes keeps every SM's 32 warps busy at decode budgets (16 tokens x 64 slots).
+constexpr int AX_THREADS = 1024;
+constexpr int AX_WARPS = AX_THREADS / 32;
+constexpr int AX_PARTS = 4;                   // warps per task in phase 1
+constexpr int AX_TPB = AX_WARPS / AX_PARTS;   // tasks per block per round
 __device__ __forceinline__ void prefetch_l2(const void* p) {
   asm volatile("prefetch.global.L2 [%0];" ::"l"(p));
 }
 
-// x . w over `chunks` 16-byte chunks of bf16 by one warp: fp32 FMAs over each
-// lane's chunks in ascending order (8 chunks of each operand in flight), then a
+// x . w over the 16-byte chunks [c_lo, c_hi) of bf16 by one warp: fp32 FMAs over
+// each lane's chunks in ascending order (4 chunks of each operand in flight), then a
 // shuffle tree; every lane returns the sum.
-__device__ __forceinline__ float warp_dot_bf16(const uint4* __restrict__ xr, const uint4* __restrict__ wr, int chunks,
-                                               int lane) {
+__device__ __forceinline__ float warp_dot_bf16(const uint4* __restrict__ xr, const uint4* __restrict__ wr, int c_lo,
+                                               int c_hi, int lane) {
   float sacc = 0.f;
-  for (int c0 = lane; c0 < chunks; c0 += 32 * 8) {
-    uint4 av[8], bv[8];
+  for (int c0 = c_lo + lane; c0 < c_hi; c0 += 32 * 4) {
+    uint4 av[4], bv[4];
 #pragma unroll
-    for (int u = 0; u < 8; ++u) {
+    for (int u = 0; u < 4; ++u) {
       const int c = c0 + 32 * u;
-      if (c < chunks) {
+      if (c < c_hi) {
         av[u] = xr[c];
         bv[u] = wr[c];
       }
     }
 #pragma unroll
-    for (int u = 0; u < 8; ++u) {
-      if (c0 + 32 * u >= chunks) break;
+    for (int u = 0; u < 4; ++u) {
+      if (c0 + 32 * u >= c_hi) break;
       const __nv_bfloat162* pa = reinterpret_cast<const __nv_bfloat162*>(&av[u]);
       const __nv_bfloat162* pb = reinterpret_cast<const __nv_bfloat162*>(&bv[u]);
 #pragma unroll
@@ -751,30 +758,52 @@ __global__ void __launch_bounds__(AX_THREADS)
                           const float* __restrict__ g, float* __restrict__ coef, uint4* __restrict__ out,
                           long long n_experts, int prefetch_out, unsigned* bar, unsigned bar_extra,
                           unsigned long long limit_ns, int* status) {
+  __shared__ float part_s[AX_TPB][AX_PARTS];
   pdl_launch_dependents();
   pdl_wait();
-  const int lane = threadIdx.x & 31;
+  const int lane = threadIdx.x & 31, wib = threadIdx.x >> 5;
   const long long gwarp = ((long long)blockIdx.x * AX_THREADS + threadIdx.x) >> 5;
-  const long long nwarps = (long long)gridDim.x * (AX_THREADS / 32);
+  const long long nwarps = (long long)gridDim.x * AX_WARPS;
   const int chunks = d / 8;
   const long long tasks = (long long)T * K;
-  // ---- phase 1: coef[t, s] = g[t, s] act(x_t . w_in[idx[t, s]])
-  for (long long task = gwarp; task < tasks; task += nwarps) {
-    const long long t = task / K;
-    const long long e = idx[task];
-    if (e < 0 || e >= n_experts) {
-      if (lane == 0) {
-        set_status(status, MOE_ERR_DEVICE_INDEX);
-        coef[task] = 0.f;
+  // ---- phase 1: coef[t, s] = g[t, s] act(x_t . w_in[idx[t, s]]); warp wib takes part
+  // wib % AX_PARTS of task slot wib / AX_PARTS (rounds are uniform per block)
+  {
+    const int tslot = wib / AX_PARTS, part = wib % AX_PARTS;
+    const int pc = (chunks + AX_PARTS - 1) / AX_PARTS;
+    const int c_lo = min(chunks, part * pc), c_hi = min(chunks, c_lo + pc);
+    for (long long base = (long long)blockIdx.x * AX_TPB; base < tasks; base += (long long)gridDim.x * AX_TPB) {
+      const long long task = base + tslot;
+      float z = 0.f;
+      if (task < tasks) {
+        const long long e = idx[task];
+        if (e >= 0 && e < n_experts) {
+          if (prefetch_out) {  // this part's bytes of the task's w_out row, one 128-byte line per lane
+            const char* po = reinterpret_cast<const char*>(w_out + e * chunks);
+            for (int b = c_lo * 16 + lane * 128; b < c_hi * 16; b += 32 * 128) prefetch_l2(po + b);
+          }
+          z = warp_dot_bf16(x + (task / K) * chunks, w_in + e * chunks, c_lo, c_hi, lane);
+        }
       }
-      continue;
+      if (lane == 0) part_s[tslot][part] = z;
+      __syncthreads();
+      if (threadIdx.x < AX_TPB) {
+        const long long tk = base + threadIdx.x;
+        if (tk < tasks) {
+          const long long e = idx[tk];
+          if (e < 0 || e >= n_experts) {
+            set_status(status, MOE_ERR_DEVICE_INDEX);
+            coef[tk] = 0.f;
+          } else {
+            float zz = part_s[threadIdx.x][0];
+#pragma unroll
+            for (int q = 1; q < AX_PARTS; ++q) zz += part_s[threadIdx.x][q];
+            coef[tk] = g[tk] * atomic_act(zz, act);
+          }
+        }
+      }
+      __syncthreads();
     }
-    if (prefetch_out) {
-      const char* po = reinterpret_cast<const char*>(w_out + e * chunks);
-      for (int b = lane * 128; b < d * 2; b += 32 * 128) prefetch_l2(po + b);
-    }
-    const float z = warp_dot_bf16(x + t * chunks, w_in + e * chunks, chunks, lane);
-    if (lane == 0) coef[task] = g[task] * atomic_act(z, act);
   }
   // ---- grid-wide barrier (every block is resident: cooperative launch, one per SM).
   // It waits for gridDim.x + bar_extra arrivals; bar_extra is 0 except under the
@@ -798,11 +827,12 @@ __global__ void __launch_bounds__(AX_THREADS)
   }
   __syncthreads();
   if (bar_failed) return;
-  // ---- phase 2: out[t, c..c+7] = sum_s coef[t, s] w_out[idx[t, s], c..c+7]
-  const long long units4 = (long long)T * chunks * ASM_GROUPS;
-  for (long long qb = gwarp * 32; qb < units4; qb += nwarps * 32) {  // warp-aligned: shuffles see all lanes
+  // ---- phase 2: out[t, c..c+7] = sum_s coef[t, s] w_out[idx[t, s], c..c+7]; a warp
+  // covers two output chunks, sixteen lanes (slot groups) each
+  const long long unitsG = (long long)T * chunks * ASM_GROUPS;
+  for (long long qb = gwarp * 32; qb < unitsG; qb += nwarps * 32) {  // warp-aligned: shuffles see all lanes
     const long long q = qb + lane;
-    const bool valid = q < units4;
+    const bool valid = q < unitsG;
     const int grp = (int)(q & (ASM_GROUPS - 1));
     const long long unit = q / ASM_GROUPS;
     const long long t = unit / chunks;
@@ -837,19 +867,15 @@ __global__ void __launch_bounds__(AX_THREADS)
         }
       }
     }
-    float r[8];
 #pragma unroll
-    for (int h = 0; h < 8; ++h) {  // ((group 0 + group 1) + group 2) + group 3, in lanes 4u .. 4u + 3
-      const float b1 = __shfl_down_sync(0xffffffffu, acc[h], 1);
-      const float b2 = __shfl_down_sync(0xffffffffu, acc[h], 2);
-      const float b3 = __shfl_down_sync(0xffffffffu, acc[h], 3);
-      r[h] = ((acc[h] + b1) + b2) + b3;
-    }
+    for (int o = 1; o < ASM_GROUPS; o <<= 1)  // the sixteen groups by a fixed xor tree (a + b = b + a)
+#pragma unroll
+      for (int h = 0; h < 8; ++h) acc[h] += __shfl_xor_sync(0xffffffffu, acc[h], o);
     if (valid && grp == 0) {
       uint4 o;
       __nv_bfloat162* po2 = reinterpret_cast<__nv_bfloat162*>(&o);
 #pragma unroll
-      for (int h = 0; h < 4; ++h) po2[h] = __floats2bfloat162_rn(r[2 * h], r[2 * h + 1]);
+      for (int h = 0; h < 4; ++h) po2[h] = __floats2bfloat162_rn(acc[2 * h], acc[2 * h + 1]);
       out[t * chunks + c] = o;
     }
   }
@@ -966,7 +992,7 @@ __global__ void __launch_bounds__(AW_THREADS)
       const long long task = order[pos];
       if (task < 0 || task >= tasks) continue;
       const long long e = idx[task];
-      const float z = warp_dot_bf16(x + (task / K) * chunks, w_in + e * chunks, chunks, lane);
+      const float z = warp_dot_bf16(x + (task / K) * chunks, w_in + e * chunks, 0, chunks, lane);
       if (lane == 0) coef[task] = g[task] * atomic_act(z, act);
     }
     return;
@@ -980,7 +1006,7 @@ __global__ void __launch_bounds__(AW_THREADS)
       }
       continue;
     }
-    const float z = warp_dot_bf16(x + (task / K) * chunks, w_in + e * chunks, chunks, lane);
+    const float z = warp_dot_bf16(x + (task / K) * chunks, w_in + e * chunks, 0, chunks, lane);
     if (lane == 0) coef[task] = g[task] * atomic_act(z, act);
   }
 }
