@@ -341,8 +341,8 @@ cudaError_t launch_topk_softmax(int T, int m, int k, int renorm, const float* lo
 // The T k tasks (q = t k + s, in increasing order) are cut into R contiguous
 // ranges of L tasks; range r holds tasks [r L, min(T k, (r + 1) L)). One block of
 // 1024 threads (the routing tables are tiny):
-//  pass 1: c[r][e] = tasks of expert e in range r (warp w counts ranges w, w + 32,
-//          ...; shared-memory atomics on rows no other warp touches).
+//  pass 1: c[r][e] = tasks of expert e in range r (thread i takes tasks i, i + 1024,
+//          ..., eight of its ids loaded together, then shared-memory atomics).
 //  scan:   per expert (one warp each, a shuffle scan over its R entries),
 //          c[r][e] <- tasks of e in ranges before r; the total is n_e.
 //  mode & 1: offsets = exclusive scan of n_e, max / lowest argmax of n_e and
@@ -369,14 +369,23 @@ __global__ void __launch_bounds__(RI_THREADS, 1)
   pdl_launch_dependents();
   pdl_wait();
   __syncthreads();
-  for (int r = warp; r < R; r += nw) {
-    const int lo = r * L, hi = min(Tk, lo + L);
-    for (int q = lo + lane; q < hi; q += 32) {
-      const int e = idx[q];
+  const int nth = blockDim.x;
+  for (int q0 = tid; q0 < Tk; q0 += 8 * nth) {
+    int ev[8];
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      const int q = q0 + u * nth;
+      ev[u] = q < Tk ? idx[q] : 0;
+    }
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      const int q = q0 + u * nth;
+      if (q >= Tk) break;
+      const int e = ev[u];
       if (e < 0 || e >= m)
         bad = 1;
       else
-        atomicAdd(&c[r * MS + e], 1);
+        atomicAdd(&c[(q / L) * MS + e], 1);
     }
   }
   __syncthreads();
@@ -562,10 +571,11 @@ cudaError_t launch_route_index(int mode, int T, int k, int m, const int32_t* idx
 }
 
 // ------------------------------------------------ ranks
-// One warp per task range r walks it 32 tasks at a time in increasing task id: a
-// task's rank among the lower lanes with the same expert (a 32-step shuffle scan)
-// plus the expert's cursor (started at start[r][e]) is its position pos in the
-// stable counting sort; the group's last lane advances the cursor. Writes
+// One warp per task range r walks it 32 tasks at a time in increasing task id (the
+// ids of eight such steps loaded together): a task's rank among the lower lanes with
+// the same expert (a 32-step shuffle scan) plus the expert's cursor (started at
+// start[r][e]) is its position pos in the stable counting sort; the group's last
+// lane advances the cursor. Writes
 // inv_perm[q] = pos, perm[pos] = q and, when given, w_perm[pos] = task_w[q] (the
 // gate weight in segment order). A position outside its expert's segment
 // [offsets[e], offsets[e + 1]) sets MOE_ERR_DEVICE_INDEX and that task is not
@@ -583,9 +593,21 @@ __global__ void rank_kernel(int Tk, int m, int L, const int32_t* __restrict__ id
   if (status && *reinterpret_cast<volatile int*>(status) != 0) return;  // earlier device error
   for (int e = lane; e < m; e += 32) cur[e] = start[(long long)r * m + e];
   __syncwarp();
+  int ev[8];
   for (int base = lo; base < hi; base += 32) {
+    const int step = ((base - lo) >> 5) & 7;
+    if (step == 0) {  // the ids of the next eight steps
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        const int qq = base + 32 * u + lane;
+        ev[u] = qq < hi ? idx[qq] : -1;
+      }
+    }
     const int q = base + lane;
-    int e = q < hi ? idx[q] : -1;
+    int e = -1;
+#pragma unroll
+    for (int u = 0; u < 8; ++u)
+      if (u == step) e = ev[u];
     if (e >= m) e = -1;
     int rank = 0, cnt = 0;
 #pragma unroll
@@ -624,28 +646,51 @@ cudaError_t launch_rank(int T, int k, int m, const int32_t* idx, const int32_t* 
 }
 
 // ------------------------------------------------------------------ permute rows
-// One thread per 16-byte chunk of x_perm, tasks q in order:
-// x_perm[inv_perm[q], c] = x[q / k, c] (tasks without a valid position are skipped).
-__global__ void permute_rows_kernel(int Tk, int k, int chunks, const int4* __restrict__ x,
-                                    const int32_t* __restrict__ inv_perm, int4* __restrict__ x_perm) {
+// One warp per token t: its row x[t] is read once, 8 of each lane's 16-byte chunks in
+// flight, and written to the permuted position of each of its k tasks:
+// x_perm[inv_perm[t k + s], c] = x[t, c] (tasks without a valid position are skipped).
+constexpr int PR_THREADS = 256, PR_BATCH = 8;
+__global__ void __launch_bounds__(PR_THREADS)
+    permute_rows_kernel(int T, int k, int chunks, const int4* __restrict__ x, const int32_t* __restrict__ inv_perm,
+                        int4* __restrict__ x_perm) {
+  __shared__ int dst_s[PR_THREADS / 32][32];  // the warp's token: position of each task (or -1)
   pdl_launch_dependents();
   pdl_wait();
-  const long long n = (long long)Tk * chunks;
-  for (long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += (long long)gridDim.x * blockDim.x) {
-    const long long q = i / chunks;
-    const int c = (int)(i - q * chunks);
-    const int pos = inv_perm[q];
-    if (pos < 0 || pos >= Tk) continue;
-    x_perm[(long long)pos * chunks + c] = x[(q / k) * chunks + c];
+  const int lane = threadIdx.x & 31, wib = threadIdx.x >> 5;
+  const int Tk = T * k;
+  const long long nw = (long long)gridDim.x * (PR_THREADS / 32);
+  for (long long t = (long long)blockIdx.x * (PR_THREADS / 32) + wib; t < T; t += nw) {
+    __syncwarp();  // the previous token's readers of dst_s are done
+    if (lane < k) {
+      const int pos = inv_perm[t * k + lane];
+      dst_s[wib][lane] = (pos >= 0 && pos < Tk) ? pos : -1;
+    }
+    __syncwarp();
+    const int4* src = x + t * chunks;
+    for (int c0 = lane; c0 < chunks; c0 += 32 * PR_BATCH) {  // lanes past the row's chunks skip it
+      int4 v[PR_BATCH];
+#pragma unroll
+      for (int u = 0; u < PR_BATCH; ++u)
+        if (c0 + 32 * u < chunks) v[u] = src[c0 + 32 * u];
+      for (int sl = 0; sl < k; ++sl) {
+        const int dp = dst_s[wib][sl];
+        if (dp < 0) continue;
+        int4* o = x_perm + (long long)dp * chunks;
+#pragma unroll
+        for (int u = 0; u < PR_BATCH; ++u)
+          if (c0 + 32 * u < chunks) o[c0 + 32 * u] = v[u];
+      }
+    }
   }
 }
 
 cudaError_t launch_permute_rows(int dtype, int Tk, int k, int d, const void* x, const int32_t* inv_perm, void* x_perm,
                                 cudaStream_t s) {
   const int chunks = d * (dtype == MOE_F32 ? 4 : 2) / 16;
-  const long long n = (long long)Tk * chunks;
-  const int blocks = (int)std::max<long long>(1, std::min<long long>((n + 255) / 256, (long long)num_sms() * 16));
-  launch_k(permute_rows_kernel, blocks, 256, 0, s, Tk, k, chunks, (const int4*)x, inv_perm, (int4*)x_perm);
+  const int T = Tk / k;
+  const int wpb = PR_THREADS / 32;
+  const int blocks = (int)std::max<long long>(1, std::min<long long>((T + wpb - 1) / wpb, (long long)num_sms() * 16));
+  launch_k(permute_rows_kernel, blocks, PR_THREADS, 0, s, T, k, chunks, (const int4*)x, inv_perm, (int4*)x_perm);
   count_launch();
   return cudaGetLastError();
 }
@@ -952,9 +997,9 @@ cudaError_t launch_replica_split(int T, int k, int m, const int32_t* idx, const 
 
 // ------------------------------------------------------------------ combine
 // out[t, c] = sum_s sum_split y[split][inv_perm[t k + s], c]
-//           + sum_sh sum_split ysh[split][sh T + t, c], fp32, slot order; 4 columns
-// per thread (16-byte loads). With row_splits the routed rows have their own split
-// counts (row_splits[pos] <= ksplit partials for permuted row pos).
+//           + sum_sh sum_split ysh[split][sh T + t, c], fp32, in that order. With
+// row_splits the routed rows have their own split counts (row_splits[pos] <= ksplit
+// partials for permuted row pos).
 template <typename OutT>
 __device__ __forceinline__ void store4(OutT* out, long long i4, float4 v);
 template <>
@@ -970,43 +1015,88 @@ __device__ __forceinline__ void store4<__nv_bfloat16>(__nv_bfloat16* out, long l
   reinterpret_cast<uint2*>(out)[i4] = u;
 }
 
-template <typename OutT>
-__global__ void combine_kernel(int T, int d4, int k, int ksplit, const float4* __restrict__ y, long long ysplit4,
-                               const int32_t* __restrict__ inv_perm, int n_sh, const float4* __restrict__ ysh,
-                               long long yshsplit4, OutT* __restrict__ out, const int32_t* __restrict__ row_splits) {
+// Block (token t, column block): the token's partial rows are listed first — the
+// (slot, split) rows of its routed tasks, then the (shared expert, split) rows — as
+// float4 offsets in shared memory, built in parallel (one thread per slot); then
+// each thread owns CPT 16-byte column chunks and loads U listed rows' chunks at once
+// (U CPT = 8 float4 in flight), adding them in list order, so every output is the
+// same sum in the same order as one thread walking the list. Few tokens (decode)
+// take narrow column blocks so the grid still covers the SMs.
+constexpr int CB_THREADS = 256;
+constexpr int CB_MAX_ROWS = 32 * 64 + 8 * 64;  // k <= 32 slots, n_shared <= 8, <= 64 splits each
+template <typename OutT, int CPT>
+__global__ void __launch_bounds__(CB_THREADS, 4)
+    combine_kernel(int T, int d4, int k, int ksplit, const float4* __restrict__ y, long long ysplit4,
+                   const int32_t* __restrict__ inv_perm, int n_sh, const float4* __restrict__ ysh,
+                   long long yshsplit4, OutT* __restrict__ out, const int32_t* __restrict__ row_splits, int ncb) {
+  constexpr int U = 8 / CPT > 1 ? 8 / CPT : 2;
+  __shared__ long long rows_s[CB_MAX_ROWS];
+  __shared__ int cnt_s[33];
   pdl_launch_dependents();
   pdl_wait();
-  const long long n = (long long)T * d4;
   const int Tk = T * k;
-  for (long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += (long long)gridDim.x * blockDim.x) {
-    const long long t = i / d4;
-    const int c = (int)(i - t * d4);
-    float4 a = make_float4(0.f, 0.f, 0.f, 0.f);
-    for (int s = 0; s < k; ++s) {
-      const int pos = inv_perm[t * k + s];
-      if (pos < 0 || pos >= Tk) continue;
-      const int ns = row_splits ? min(ksplit, row_splits[pos]) : ksplit;
-      const float4* yp = y + (long long)pos * d4 + c;
-      int sp = 0;
-      for (; sp + 4 <= ns; sp += 4) {  // four partials' loads in flight together, added in order
-        const float4 v0 = yp[sp * ysplit4], v1 = yp[(sp + 1) * ysplit4], v2 = yp[(sp + 2) * ysplit4],
-                     v3 = yp[(sp + 3) * ysplit4];
-        a.x += v0.x; a.y += v0.y; a.z += v0.z; a.w += v0.w;
-        a.x += v1.x; a.y += v1.y; a.z += v1.z; a.w += v1.w;
-        a.x += v2.x; a.y += v2.y; a.z += v2.z; a.w += v2.w;
-        a.x += v3.x; a.y += v3.y; a.z += v3.z; a.w += v3.w;
+  const int tid = threadIdx.x, lane = tid & 31;
+  for (long long tb = blockIdx.x; tb < (long long)T * ncb; tb += gridDim.x) {
+    const long long t = tb / ncb;
+    const int cb = (int)(tb - t * ncb) * CB_THREADS * CPT;
+    __syncthreads();  // the previous token's readers of rows_s are done
+    if (tid < 32) {  // warp 0: rows per slot, their prefix, then each slot's rows
+      long long base = -1;
+      int ns = 0;
+      if (lane < k) {
+        const int pos = inv_perm[t * k + lane];
+        if (pos >= 0 && pos < Tk) {
+          base = (long long)pos * d4;
+          ns = row_splits ? min(ksplit, row_splits[pos]) : ksplit;
+        }
       }
-      for (; sp < ns; ++sp) {
-        const float4 v = yp[sp * ysplit4];
-        a.x += v.x; a.y += v.y; a.z += v.z; a.w += v.w;
+      int incl = ns;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int v = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += v;
       }
+      for (int sp = 0; sp < ns; ++sp) rows_s[incl - ns + sp] = base + sp * ysplit4;
+      if (lane == 31) cnt_s[0] = incl;
     }
-    for (int sh = 0; sh < n_sh; ++sh)
-      for (int sp = 0; sp < ksplit; ++sp) {
-        const float4 v = ysh[sp * yshsplit4 + ((long long)sh * T + t) * d4 + c];
-        a.x += v.x; a.y += v.y; a.z += v.z; a.w += v.w;
+    __syncthreads();
+    const int nr = cnt_s[0];
+    for (int i = tid; i < n_sh * ksplit; i += CB_THREADS) {  // shared-expert rows after the routed ones
+      const int sh = i / ksplit, sp = i - sh * ksplit;
+      rows_s[nr + i] = -1 - (sp * yshsplit4 + ((long long)sh * T + t) * d4);  // tagged: from ysh
+    }
+    __syncthreads();
+    const int P = nr + n_sh * ksplit;
+    float4 a[CPT];
+#pragma unroll
+    for (int j = 0; j < CPT; ++j) a[j] = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int i0 = 0; i0 < P; i0 += U) {
+      float4 v[U][CPT];
+#pragma unroll
+      for (int u = 0; u < U; ++u) {
+        if (i0 + u < P) {
+          const long long r = rows_s[i0 + u];
+          const float4* src = r >= 0 ? y + r : ysh + (-1 - r);
+#pragma unroll
+          for (int j = 0; j < CPT; ++j) {
+            const int c = cb + tid + CB_THREADS * j;
+            if (c < d4) v[u][j] = src[c];
+          }
+        }
       }
-    store4<OutT>(out, i, a);
+#pragma unroll
+      for (int u = 0; u < U; ++u)
+        if (i0 + u < P)
+#pragma unroll
+          for (int j = 0; j < CPT; ++j) {
+            a[j].x += v[u][j].x; a[j].y += v[u][j].y; a[j].z += v[u][j].z; a[j].w += v[u][j].w;
+          }
+    }
+#pragma unroll
+    for (int j = 0; j < CPT; ++j) {
+      const int c = cb + tid + CB_THREADS * j;
+      if (c < d4) store4<OutT>(out, t * d4 + c, a[j]);
+    }
   }
 }
 
@@ -1014,16 +1104,31 @@ cudaError_t launch_combine(int dtype, int T, int d, int k, int ksplit, const flo
                            const int32_t* inv_perm, int n_shared, const float* y_shared, long long ysh_split_stride,
                            void* out, cudaStream_t s, const int32_t* row_splits) {
   const int d4 = d / 4;
-  const long long n = (long long)T * d4;
-  const int blocks = (int)std::max<long long>(1, std::min<long long>((n + 255) / 256, (long long)num_sms() * 16));
-  if (dtype == MOE_F32)
-    launch_k(combine_kernel<float>, blocks, 256, 0, s, T, d4, k, ksplit, (const float4*)y_perm, y_split_stride / 4, inv_perm,
-                                                 y_shared ? n_shared : 0, (const float4*)y_shared,
-                                                 ysh_split_stride / 4, (float*)out, row_splits);
+  const int nsh = y_shared ? n_shared : 0;
+  if (k > 32 || nsh > 8 || ksplit > 64) return cudaErrorInvalidValue;
+  // widest column blocks that still give the grid two blocks per SM
+  int cpt = 4;
+  while (cpt > 1 && (long long)T * ((d4 + CB_THREADS * cpt - 1) / (CB_THREADS * cpt)) < 2LL * num_sms()) cpt >>= 1;
+  const int ncb = (d4 + CB_THREADS * cpt - 1) / (CB_THREADS * cpt);
+  const int blocks = (int)std::max<long long>(1, std::min<long long>((long long)T * ncb, (long long)num_sms() * 8));
+#define MOE_COMBINE(CPT_)                                                                                          \
+  do {                                                                                                           \
+    if (dtype == MOE_F32)                                                                                        \
+      launch_k(combine_kernel<float, CPT_>, blocks, CB_THREADS, 0, s, T, d4, k, ksplit, (const float4*)y_perm,   \
+               y_split_stride / 4, inv_perm, nsh, (const float4*)y_shared, ysh_split_stride / 4, (float*)out,      \
+               row_splits, ncb);                                                                                 \
+    else                                                                                                         \
+      launch_k(combine_kernel<__nv_bfloat16, CPT_>, blocks, CB_THREADS, 0, s, T, d4, k, ksplit,                  \
+               (const float4*)y_perm, y_split_stride / 4, inv_perm, nsh, (const float4*)y_shared,                  \
+               ysh_split_stride / 4, (__nv_bfloat16*)out, row_splits, ncb);                                      \
+  } while (0)
+  if (cpt == 1)
+    MOE_COMBINE(1);
+  else if (cpt == 2)
+    MOE_COMBINE(2);
   else
-    launch_k(combine_kernel<__nv_bfloat16>, blocks, 256, 0, s, T, d4, k, ksplit, (const float4*)y_perm, y_split_stride / 4,
-                                                         inv_perm, y_shared ? n_shared : 0, (const float4*)y_shared,
-                                                         ysh_split_stride / 4, (__nv_bfloat16*)out, row_splits);
+    MOE_COMBINE(4);
+#undef MOE_COMBINE
   count_launch();
   return cudaGetLastError();
 }
