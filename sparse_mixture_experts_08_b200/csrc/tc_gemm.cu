@@ -57,7 +57,7 @@ constexpr int TC_BK8 = 128;  // E4M3 elements of one 128-byte swizzle row
 // TMEM columns), so the MMAs of the next tile wait for the whole epilogue; there two
 // warps per TMEM lane quarter share the chunks (8 warps). Elsewhere 4.
 template <int EPI, bool PAIR, bool F8>
-constexpr int tc_epi_warps() { return (PAIR && EPI == EPI_SWIGLU && !F8) ? 8 : 4; }
+constexpr int tc_epi_warps() { return ((PAIR && EPI == EPI_SWIGLU && !F8) || EPI == EPI_ROUTE) ? 8 : 4; }
 template <int EPI, bool PAIR, bool F8>
 constexpr int tc_threads() { return 64 + 32 * tc_epi_warps<EPI, PAIR, F8>(); }
 constexpr int TC_MAX_GROUPS = 1040;
@@ -274,12 +274,12 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float a, float b) {
   return *reinterpret_cast<const uint32_t*>(&h);
 }
 
-// Barrier of the four epilogue warps only (named barrier 1; 0 is __syncthreads),
-// in its non-aligned form and after reconverging the warp, so lanes that took
-// different branches before it are all counted.
+// Barrier of the router's eight epilogue warps only (named barrier 1; 0 is
+// __syncthreads), in its non-aligned form and after reconverging the warp, so lanes
+// that took different branches before it are all counted.
 __device__ __forceinline__ void epi_bar() {
   __syncwarp();
-  asm volatile("barrier.sync 1, 128;" ::: "memory");
+  asm volatile("barrier.sync 1, 256;" ::: "memory");
 }
 
 // One pass of the router epilogue over a token's m logits (TMEM columns, 32 per
@@ -287,14 +287,16 @@ __device__ __forceinline__ void epi_bar() {
 // expert asc), by a pairwise tree whose left side always holds the lower experts.
 // With EXP it also writes the logits (lg, when given) and folds the softmax
 // denominator: per 32 columns a pairwise fp32 sum of exp(logit - running max),
-// added to an fp64 sum rescaled whenever the running maximum grows.
+// added to an fp64 sum rescaled whenever the running maximum grows. A pass covers
+// the columns [c_lo, c_hi) (multiples of 32); the two threads of a token take the
+// lower and the upper half of the experts.
 template <bool EXP>
-__device__ __forceinline__ void route_pass(uint32_t t_row, int m, const float* rbias, float pv, int pe, float& bv,
-                                           int& be, float& mrun, double& z, float* lg) {
+__device__ __forceinline__ void route_pass(uint32_t t_row, int c_lo, int c_hi, int m, const float* rbias, float pv,
+                                           int pe, float& bv, int& be, float& mrun, double& z, float* lg) {
   bv = -INFINITY;
   be = -1;
 #pragma unroll 1
-  for (int c0 = 0; c0 < m; c0 += 32) {
+  for (int c0 = c_lo; c0 < c_hi; c0 += 32) {
     uint32_t r[32];
     tmem_ld_x16(t_row + c0, r);
     if (c0 + 16 < m) {
@@ -470,6 +472,10 @@ __global__ void __launch_bounds__(tc_threads<EPI, PAIR, F8>(), 1)
   constexpr int RMASK_M = EPI == EPI_ROUTE ? ROUTE_MAX_M : 1;
   __shared__ __align__(16) float rbias[RMASK_M];  // ROUTE: router bias (zeros when absent)
   __shared__ uint32_t rmask[EPI == EPI_ROUTE ? 2 : 1][4][RMASK_M];  // ROUTE: expert -> lanes holding it
+  constexpr int RX = EPI == EPI_ROUTE ? 4 : 1;  // ROUTE: the upper-half thread's pick and sums, per token
+  __shared__ float rx_v[RX][32], rx_m[RX][32];
+  __shared__ int rx_e[RX][32];
+  __shared__ double rx_z[RX][32];
   __shared__ uint32_t tmem_base_s;
   __shared__ int abort_s, epi_fail_s;
   __shared__ int total_tiles_s;
@@ -706,14 +712,18 @@ __global__ void __launch_bounds__(tc_threads<EPI, PAIR, F8>(), 1)
     if (!mbar_wait(&drain_bar, 0, TC_DRAIN_LIMIT_NS, &never)) set_status(p.status, MOE_ERR_TIMEOUT);
   } else if (EPI == EPI_ROUTE && warp >= 2) {
     // ---------------------------------------------------------------- router epilogue
-    // TMEM lane = token (quarter q of the 128-token tile), column = expert. Every
-    // epilogue warp reaches every epilogue barrier of every tile; a failed wait is
-    // published through epi_fail_s before the barrier, so all four leave together.
-    const int q = warp & 3;
-    const int et = (warp - 2) * 32 + lane;  // 0..127
+    // TMEM lane = token (quarter q of the 128-token tile), column = expert. Two warps
+    // per lane quarter: half 0 takes the lower half of the expert columns, half 1 the
+    // upper, and each pass merges them through shared memory (half 1's pick wins only
+    // when strictly larger, as a walk over all columns in order would have it; the
+    // softmax sums are rescaled to the larger maximum). Every epilogue warp reaches
+    // every epilogue barrier of every tile; a failed wait is published through
+    // epi_fail_s before the barrier, so all eight leave together.
+    const int q = warp & 3, half = (warp - 2) >> 2;
+    const int et = (warp - 2) * 32 + lane;  // 0..255
     {
       const GemmClass& c = p.cls[0];
-      for (int e = et; e < ROUTE_MAX_M; e += 128) rbias[e] = (c.bias && e < c.const_rows) ? c.bias[e] : 0.f;
+      for (int e = et; e < ROUTE_MAX_M; e += 256) rbias[e] = (c.bias && e < c.const_rows) ? c.bias[e] : 0.f;
       epi_bar();
     }
     int acc = 0, iter = 0;
@@ -725,6 +735,8 @@ __global__ void __launch_bounds__(tc_threads<EPI, PAIR, F8>(), 1)
       const int t = ti.mt * TC_BM + q * 32 + lane;  // token
       const bool tv_ok = t < c.R;
       const int m = ti.rows_in_tile, k = c.k_sel;
+      const int nch = (m + 31) / 32, hch = (nch + 1) / 2;
+      const int c_lo = half ? 32 * hch : 0, c_hi = half ? 32 * nch : 32 * hch;
       const bool got = mbar_wait(&accf_bar[acc], acc_phase, lim, abort_flag);
       if (!got) {
         set_status(p.status, MOE_ERR_TIMEOUT);
@@ -738,7 +750,7 @@ __global__ void __launch_bounds__(tc_threads<EPI, PAIR, F8>(), 1)
       // Pass s picks the largest logit strictly after pick s - 1 in the order
       // (logit desc, expert asc), reading the accumulator again from TMEM; pass 0
       // also writes the logits (when asked) and the softmax denominator. Each pass
-      // stores its expert and, for now, its logit in the outputs.
+      // stores its expert and, for now, its logit in the outputs (half 0).
       float mrun = -INFINITY, mx = -INFINITY;
       double z = 0.0;
       float* lg = c.out && tv_ok ? reinterpret_cast<float*>(c.out) + (long long)t * m : nullptr;
@@ -752,19 +764,48 @@ __global__ void __launch_bounds__(tc_threads<EPI, PAIR, F8>(), 1)
         float bv;
         int be;
         if (s2 == 0) {
-          route_pass<true>(t_row, m, rbias, pv, pe, bv, be, mrun, z, lg);
-          mx = bv;
-          z *= (double)expf(mrun - mx);  // the running maximum is the top logit
+          route_pass<true>(t_row, c_lo, c_hi, m, rbias, pv, pe, bv, be, mrun, z, lg);
         } else {
           float dm = 0.f;
           double dz = 0.0;
-          route_pass<false>(t_row, m, rbias, pv, pe, bv, be, dm, dz, nullptr);
+          route_pass<false>(t_row, c_lo, c_hi, m, rbias, pv, pe, bv, be, dm, dz, nullptr);
         }
-        if (tv_ok) {
-          oi[s2] = be;
-          ow[s2] = bv;
+        if (half) {
+          rx_v[q][lane] = bv;
+          rx_e[q][lane] = be;
+          if (s2 == 0) {
+            rx_m[q][lane] = mrun;
+            rx_z[q][lane] = z;
+          }
         }
-        bad |= be < 0;  // NaN logits
+        epi_bar();
+        if (!half) {
+          const float ov = rx_v[q][lane];
+          const int oe = rx_e[q][lane];
+          if (ov > bv) {  // the upper half holds higher experts: it wins only when strictly larger
+            bv = ov;
+            be = oe;
+          }
+          if (s2 == 0) {
+            const float om = rx_m[q][lane], mm = fmaxf(mrun, om);
+            z = z * (double)expf(mrun - mm) + rx_z[q][lane] * (double)expf(om - mm);
+            mrun = mm;
+            mx = bv;
+            z *= (double)expf(mrun - mx);  // the running maximum is the top logit
+          }
+          rx_v[q][lane] = bv;  // the merged pick, for the upper half's next pass
+          rx_e[q][lane] = be;
+          if (tv_ok) {
+            oi[s2] = be;
+            ow[s2] = bv;
+          }
+          bad |= be < 0;  // NaN logits
+        }
+        epi_bar();
+        if (half) {
+          bv = rx_v[q][lane];
+          be = rx_e[q][lane];
+        }
         pv = bv;
         pe = be;
       }
@@ -776,7 +817,7 @@ __global__ void __launch_bounds__(tc_threads<EPI, PAIR, F8>(), 1)
         acc = 0;
         acc_phase ^= 1u;
       }
-      if (tv_ok) {  // gate weights: softmax over all m, renormalised over the k chosen when asked
+      if (tv_ok && !half) {  // gate weights: softmax over all m, renormalised over the k chosen when asked
         double sel = 0.0;
 #pragma unroll 1
         for (int s2 = 0; s2 < k; ++s2) sel += (double)expf(ow[s2] - mx) / z;
@@ -791,17 +832,20 @@ __global__ void __launch_bounds__(tc_threads<EPI, PAIR, F8>(), 1)
       if (c.lrank) {
         // rank of each task among the tile's tasks of its expert, in (token, slot)
         // order: lanes below in this quarter plus all tasks of the quarters before
+        // (the lower-half warps build the masks; every epilogue warp passes the barrier)
         uint32_t(*mk)[RMASK_M] = rmask[EPI == EPI_ROUTE ? (iter & 1) : 0];
-        for (int e = lane; e < m; e += 32) mk[q][e] = 0u;
-        __syncwarp();
-        if (tv_ok)
+        if (!half) {
+          for (int e = lane; e < m; e += 32) mk[q][e] = 0u;
+          __syncwarp();
+          if (tv_ok)
 #pragma unroll 1
-          for (int s2 = 0; s2 < k; ++s2) {
-            const int e = oi[s2];
-            if (e >= 0) atomicOr(&mk[q][e], 1u << lane);
-          }
+            for (int s2 = 0; s2 < k; ++s2) {
+              const int e = oi[s2];
+              if (e >= 0) atomicOr(&mk[q][e], 1u << lane);
+            }
+        }
         epi_bar();
-        if (tv_ok)
+        if (tv_ok && !half)
 #pragma unroll 1
           for (int s2 = 0; s2 < k; ++s2) {
             const int e = oi[s2];
@@ -810,7 +854,7 @@ __global__ void __launch_bounds__(tc_threads<EPI, PAIR, F8>(), 1)
             for (int q2 = 0; q2 < q; ++q2) rk += __popc(mk[q2][e]);
             c.lrank[(long long)t * k + s2] = rk;
           }
-        for (int e = et; e < m; e += 128)
+        for (int e = et; e < m; e += 256)
           c.tile_cnt[(long long)ti.mt * m + e] =
               __popc(mk[0][e]) + __popc(mk[1][e]) + __popc(mk[2][e]) + __popc(mk[3][e]);
         // (the masks are double-buffered: the next tile writes the other set, and the
