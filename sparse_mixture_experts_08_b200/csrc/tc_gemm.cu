@@ -53,13 +53,17 @@ namespace moe {
 constexpr int TC_BM = 128;
 constexpr int TC_BK = 64;  // bf16 elements of one 128-byte swizzle row
 constexpr int TC_BK8 = 128;  // E4M3 elements of one 128-byte swizzle row
-// Epilogue warps of a kernel instance: pair SwiGLU tiles hold one accumulator (2 x 256
-// TMEM columns), so the MMAs of the next tile wait for the whole epilogue; there two
-// warps per TMEM lane quarter share the chunks (8 warps). Elsewhere 4.
-template <int EPI, bool PAIR, bool F8>
-constexpr int tc_epi_warps() { return ((PAIR && EPI == EPI_SWIGLU && !F8) || EPI == EPI_ROUTE) ? 8 : 4; }
-template <int EPI, bool PAIR, bool F8>
-constexpr int tc_threads() { return 64 + 32 * tc_epi_warps<EPI, PAIR, F8>(); }
+// Epilogue warps of a kernel instance. Pair SwiGLU tiles and pair down tiles with two
+// feature blocks hold one accumulator (2 x 256 TMEM columns), so the MMAs of the next
+// tile wait for the epilogue: SwiGLU gives each TMEM lane quarter three warps that
+// share its chunks (12 warps), the down tiles two warps that take one feature block
+// each (8). The router uses 8, the rest 4.
+template <int EPI, bool PAIR, bool F8, int MATS>
+constexpr int tc_epi_warps() {
+  return (PAIR && EPI == EPI_SWIGLU && !F8) ? 12 : (PAIR && EPI == EPI_DOWN && MATS == 2) || EPI == EPI_ROUTE ? 8 : 4;
+}
+template <int EPI, bool PAIR, bool F8, int MATS>
+constexpr int tc_threads() { return 64 + 32 * tc_epi_warps<EPI, PAIR, F8, MATS>(); }
 constexpr int TC_MAX_GROUPS = 1040;
 constexpr int TC_SMEM_BUDGET = 200 * 1024;
 constexpr unsigned long long TC_DRAIN_LIMIT_NS = 200ull * 1000 * 1000;
@@ -135,6 +139,29 @@ __device__ __forceinline__ void tma_load_2d_pair(const CUtensorMap* map, uint32_
 }
 __device__ __forceinline__ void mbar_arrive_cluster(uint32_t bar_cluster) {
   asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(bar_cluster) : "memory");
+}
+// Relaxed arrivals: they order no memory operation of the arriving thread, so they do
+// not wait for its global stores to be performed. Used where the waiter only reuses
+// TMEM whose reads (tcgen05.wait::ld) the arriving warp has already completed.
+__device__ __forceinline__ void mbar_arrive_relaxed(uint64_t* bar) {
+  asm volatile("mbarrier.arrive.relaxed.cta.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+__device__ __forceinline__ void mbar_arrive_cluster_relaxed(uint32_t bar_cluster) {
+  asm volatile("mbarrier.arrive.relaxed.cluster.shared::cluster.b64 _, [%0];" ::"r"(bar_cluster) : "memory");
+}
+
+// SiLU(g) * u for the gated epilogue with one special-function op per element (e^-g):
+// 1 / (1 + e^-g) comes from an integer seed (relative error at most 5.1% over any
+// binade; the constant minimises that maximum) and two Newton steps r += r (1 - d r)
+// on the FMA pipe (relative error below 7e-6, far under the bf16 rounding of h). The
+// exponent is clamped at 44 so that d stays below 2^64 and the seed stays normal;
+// for g < -44 the sigmoid below e^-44 is then taken as e^-44.
+__device__ __forceinline__ float silu_mul(float g, float u) {
+  const float d = 1.f + __expf(fminf(-g, 44.f));
+  float r = __int_as_float(0x7EF311C2 - __float_as_int(d));
+  r = fmaf(r, fmaf(-d, r, 1.f), r);
+  r = fmaf(r, fmaf(-d, r, 1.f), r);
+  return g * r * u;
 }
 
 template <bool PAIR>
@@ -274,6 +301,13 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float a, float b) {
   return *reinterpret_cast<const uint32_t*>(&h);
 }
 
+// Barrier of the two epilogue warps of TMEM lane quarter q (named barriers 2..5),
+// reached by both with the warp converged.
+__device__ __forceinline__ void quarter_bar(int q) {
+  __syncwarp();
+  asm volatile("barrier.sync %0, 64;" ::"r"(2 + q) : "memory");
+}
+
 // Barrier of the router's eight epilogue warps only (named barrier 1; 0 is
 // __syncthreads), in its non-aligned form and after reconverging the warp, so lanes
 // that took different branches before it are all counted.
@@ -369,34 +403,57 @@ struct TileInfo {
   int cls, g, mt, ks, nt, rows_in_tile, b_row, out_row, a_row, kb0, kb1;
 };
 
+// Groups in walk order: gid[pos] is the group at position pos and tile_start[pos] its
+// first tile (tile_start[G] = all tiles); rows and brow are indexed by group.
 struct SchedSmem {
   int tile_start[TC_MAX_GROUPS + 1];
+  int gid[TC_MAX_GROUPS];
   int rows[TC_MAX_GROUPS];
   int brow[TC_MAX_GROUPS];
 };
 
+// Height of the tiles a group of `rows` rows splits into: NT = ceil(rows / BN) tiles of
+// equal height (a multiple of 16, at most BN) rather than full tiles and a ragged last
+// one: a tile streams the whole weight panel whatever its height, so a short last tile
+// costs nearly a full one, while NT tiles of height rows / NT keep every tile near the
+// MMA-bound rate. (NT - 1) * height < rows, as height <= BN and (NT - 1) * BN < rows.
+template <int BN>
+__device__ __forceinline__ int tile_height(int rows) {
+  const int NT = (rows + BN - 1) / BN;
+  return NT > 0 ? min(BN, (((rows + NT - 1) / NT) + 15) & ~15) : 0;
+}
+
+// The r-th tile of walker `walker`: rounds of `walkers` consecutive tiles, taken in
+// alternating direction, so that with the groups ordered tallest tiles first every
+// walker draws from each height band.
+__device__ __forceinline__ int walk_tile(int r, int walker, int walkers) {
+  return r * walkers + ((r & 1) ? walkers - 1 - walker : walker);
+}
+
 template <int BN, int BKE, int TILE_M = TC_BM>
 __device__ __forceinline__ void decode_tile(const GemmParams& p, const SchedSmem& s, int G, int w, TileInfo& ti) {
-  int lo = 0, hi = G - 1;  // largest gi with tile_start[gi] <= w
+  int lo = 0, hi = G - 1;  // largest position with tile_start[pos] <= w
   while (lo < hi) {
     int mid = (lo + hi + 1) >> 1;
     if (s.tile_start[mid] <= w) lo = mid; else hi = mid - 1;
   }
-  const int gi = lo;
+  const int pos = lo;
+  const int gi = s.gid[pos];
   const int G0 = p.cls[0].n_groups;
   ti.cls = gi < G0 ? 0 : 1;
   ti.g = gi - (ti.cls ? G0 : 0);
   const GemmClass& c = p.cls[ti.cls];
   const int rows = s.rows[gi];
   const int NT = (rows + BN - 1) / BN;
-  const int local = w - s.tile_start[gi];
+  const int tsz = tile_height<BN>(rows);
+  const int local = w - s.tile_start[pos];
   ti.nt = local % NT;
   const int rest = local / NT;
   ti.ks = rest % c.ksplit;
   ti.mt = rest / c.ksplit;
-  ti.rows_in_tile = min(BN, rows - ti.nt * BN);
-  ti.b_row = s.brow[gi] + ti.nt * BN;
-  ti.out_row = (c.seg_off ? s.brow[gi] : ti.g * c.out_group_stride) + ti.nt * BN;
+  ti.rows_in_tile = min(tsz, rows - ti.nt * tsz);
+  ti.b_row = s.brow[gi] + ti.nt * tsz;
+  ti.out_row = (c.seg_off ? s.brow[gi] : ti.g * c.out_group_stride) + ti.nt * tsz;
   // the weight matrix of the group (a replica group reads another group's weights)
   int wg = ti.g;
   if (c.group_map) {
@@ -440,7 +497,7 @@ __device__ __forceinline__ void store_logit(const GemmClass& c, const TileInfo& 
 }
 
 template <int BN, int MATS, int EPI, bool F8, bool PAIR>
-__global__ void __launch_bounds__(tc_threads<EPI, PAIR, F8>(), 1)
+__global__ void __launch_bounds__(tc_threads<EPI, PAIR, F8, MATS>(), 1)
     tc_grouped_gemm_kernel(const __grid_constant__ CUtensorMap tA0_0, const __grid_constant__ CUtensorMap tA1_0,
                            const __grid_constant__ CUtensorMap tB_0, const __grid_constant__ CUtensorMap tA0_1,
                            const __grid_constant__ CUtensorMap tA1_1, const __grid_constant__ CUtensorMap tB_1,
@@ -463,12 +520,18 @@ __global__ void __launch_bounds__(tc_threads<EPI, PAIR, F8>(), 1)
   __shared__ float aux_w[4][EPI == EPI_DOWN ? BN : 1];  // per epilogue warp: row weights of the tile
   __shared__ int aux_d[4][EPI == EPI_DOWN ? BN : 1];    // and destination tokens (fused top-1 combine)
   __shared__ float aux_s[4][F8 && EPI != EPI_DOWN ? BN : 1];  // F8: activation-row scales of the tile
-  // SWIGLU / RELU / DOWN: per epilogue warp, 16 output rows x its 32 features, so the
-  // global writes leave as 16-byte vectors along the feature axis (rows padded to 36
-  // floats: 16-byte aligned, and the column-wise writes hit 32 distinct banks)
+  // SWIGLU / RELU / DOWN into bf16 rows: per epilogue warp, 16 output rows x its 32
+  // features, so the global writes leave as 16-byte vectors along the feature axis.
+  // DOWN stages fp32, 8 rows at a time (rows padded to 36 floats: 16-byte aligned, and
+  // the column-wise writes hit 32 distinct banks); SWIGLU and RELU stage the rounded
+  // bf16 values of all 16 rows (rows of 64 bytes: a row's column-wise writes fill 16
+  // distinct banks, and the two rows a quarter-warp reads back as 16-byte vectors
+  // cover all 32).
   constexpr bool VEC = EPI == EPI_SWIGLU || EPI == EPI_RELU || EPI == EPI_DOWN;
-  constexpr int NEPI = tc_epi_warps<EPI, PAIR, F8>();
-  __shared__ __align__(16) float stg[VEC ? NEPI : 1][16][36];
+  constexpr bool STG16 = EPI == EPI_SWIGLU || EPI == EPI_RELU;
+  constexpr int NEPI = tc_epi_warps<EPI, PAIR, F8, MATS>();
+  __shared__ __align__(16) float stg[VEC && !STG16 ? NEPI : 1][8][36];  // 8 rows per pass
+  __shared__ __align__(16) __nv_bfloat16 stg16[STG16 ? NEPI : 1][16][32];
   constexpr int RMASK_M = EPI == EPI_ROUTE ? ROUTE_MAX_M : 1;
   __shared__ __align__(16) float rbias[RMASK_M];  // ROUTE: router bias (zeros when absent)
   __shared__ uint32_t rmask[EPI == EPI_ROUTE ? 2 : 1][4][RMASK_M];  // ROUTE: expert -> lanes holding it
@@ -477,7 +540,7 @@ __global__ void __launch_bounds__(tc_threads<EPI, PAIR, F8>(), 1)
   __shared__ int rx_e[RX][32];
   __shared__ double rx_z[RX][32];
   __shared__ uint32_t tmem_base_s;
-  __shared__ int abort_s, epi_fail_s;
+  __shared__ int abort_s, epi_fail_s, qfail_s[4];
   __shared__ int total_tiles_s;
   extern __shared__ uint8_t dyn_smem[];
 
@@ -506,6 +569,7 @@ __global__ void __launch_bounds__(tc_threads<EPI, PAIR, F8>(), 1)
     mbar_init(&drain_bar, 1);
     abort_s = 0;
     epi_fail_s = 0;
+    for (int i = 0; i < 4; ++i) qfail_s[i] = 0;
     fence_mbar_init();
     tma_prefetch_desc(&tA0_0);
     tma_prefetch_desc(&tB_0);
@@ -521,11 +585,20 @@ __global__ void __launch_bounds__(tc_threads<EPI, PAIR, F8>(), 1)
   // rows (TMA) and the row data read below are its outputs.
   pdl_launch_dependents();
   pdl_wait();
-  // Tile schedule from the device-resident segment sizes.
+  // Tile schedule from the device-resident segment sizes. Groups are walked tallest
+  // tiles first (a tile's height sets its MMA work and so its time): a counting sort
+  // over the heights 16, 32, ..., BN, stable in group order.
   if (warp == 0) {
+    constexpr int NB = BN / 16 + 1;  // bucket = tile height / 16 (0: a group without rows)
     const int per = (G + 31) / 32;
     const int lo = lane * per, hi = min(G, lo + per);
-    int local = 0;
+    auto group_tiles = [&](const int gi, const int rows) {
+      const GemmClass& c = p.cls[gi < G0 ? 0 : 1];
+      return ((c.R + TILE_M - 1) / TILE_M) * c.ksplit * ((rows + BN - 1) / BN);
+    };
+    int cnt[NB], tl[NB];
+#pragma unroll
+    for (int b = 0; b < NB; ++b) cnt[b] = tl[b] = 0;
     for (int gi = lo; gi < hi; ++gi) {
       const int cl = gi < G0 ? 0 : 1;
       const int g = gi - (cl ? G0 : 0);
@@ -546,19 +619,48 @@ __global__ void __launch_bounds__(tc_threads<EPI, PAIR, F8>(), 1)
       }
       sched.rows[gi] = rows;
       sched.brow[gi] = brow;
-      const int MT = (c.R + TILE_M - 1) / TILE_M;
-      local += MT * c.ksplit * ((rows + BN - 1) / BN);
-      sched.tile_start[gi + 1] = local;
-    }
-    int incl = local;
+      const int key = tile_height<BN>(rows) / 16, tiles = group_tiles(gi, rows);
 #pragma unroll
-    for (int off = 1; off < 32; off <<= 1) {
-      const int v = __shfl_up_sync(0xffffffffu, incl, off);
-      if (lane >= off) incl += v;
+      for (int b = 0; b < NB; ++b)
+        if (b == key) {
+          ++cnt[b];
+          tl[b] += tiles;
+        }
     }
-    const int excl = incl - local;
-    for (int gi = lo; gi < hi; ++gi) sched.tile_start[gi + 1] += excl;
-    if (lane == 0) sched.tile_start[0] = 0;
+    // first position and first tile of this lane's groups in each bucket: the buckets
+    // above it, then the lanes below in this bucket
+    int base_c = 0, base_t = 0;
+#pragma unroll
+    for (int b = NB - 1; b >= 0; --b) {
+      int ic = cnt[b], it = tl[b];
+#pragma unroll
+      for (int off = 1; off < 32; off <<= 1) {
+        const int vc = __shfl_up_sync(0xffffffffu, ic, off), vt = __shfl_up_sync(0xffffffffu, it, off);
+        if (lane >= off) {
+          ic += vc;
+          it += vt;
+        }
+      }
+      const int sum_c = __shfl_sync(0xffffffffu, ic, 31), sum_t = __shfl_sync(0xffffffffu, it, 31);
+      cnt[b] = base_c + ic - cnt[b];
+      tl[b] = base_t + it - tl[b];
+      base_c += sum_c;
+      base_t += sum_t;
+    }
+    for (int gi = lo; gi < hi; ++gi) {
+      const int rows = sched.rows[gi];
+      const int key = tile_height<BN>(rows) / 16, tiles = group_tiles(gi, rows);
+#pragma unroll
+      for (int b = 0; b < NB; ++b)
+        if (b == key) {
+          sched.gid[cnt[b]] = gi;
+          sched.tile_start[cnt[b]] = tl[b];
+          ++cnt[b];
+          tl[b] += tiles;
+        }
+    }
+    const int incl = base_t;  // every tile
+    if (lane == 0) sched.tile_start[G] = incl;
     // An earlier kernel of this layer flagged a device error: its index tables
     // cannot be trusted, so this launch does no work.
     const int prior = p.status ? *reinterpret_cast<volatile int*>(p.status) : 0;
@@ -580,7 +682,7 @@ __global__ void __launch_bounds__(tc_threads<EPI, PAIR, F8>(), 1)
 #pragma unroll
     for (int i = 0; i < STAGES; ++i) last_parity[i] = -1;
     bool ok = true;
-    for (int w = walker; w < total && ok; w += walkers) {
+    for (int r = 0, w = walker; w < total && ok; ++r, w = walk_tile(r, walker, walkers)) {
       TileInfo ti;
       decode_tile<BN, BKE, TILE_M>(p, sched, G, w, ti);
       const CUtensorMap* mA0 = ti.cls ? &tA0_1 : &tA0_0;
@@ -640,7 +742,7 @@ __global__ void __launch_bounds__(tc_threads<EPI, PAIR, F8>(), 1)
     int acc = 0;
     uint32_t acc_phase = 0;
     bool ok = true;
-    for (int w = walker; w < total && ok; w += walkers) {
+    for (int r = 0, w = walker; w < total && ok; ++r, w = walk_tile(r, walker, walkers)) {
       TileInfo ti;
       decode_tile<BN, BKE, TILE_M>(p, sched, G, w, ti);
       if (!mbar_wait(&acce_bar[acc], acc_phase ^ 1u, lim, abort_flag)) {
@@ -728,7 +830,7 @@ __global__ void __launch_bounds__(tc_threads<EPI, PAIR, F8>(), 1)
     }
     int acc = 0, iter = 0;
     uint32_t acc_phase = 0;
-    for (int w = walker; w < total; w += walkers, ++iter) {
+    for (int r = 0, w = walker; w < total; ++r, w = walk_tile(r, walker, walkers), ++iter) {
       TileInfo ti;
       decode_tile<BN, BKE>(p, sched, G, w, ti);
       const GemmClass& c = p.cls[0];
@@ -866,11 +968,15 @@ __global__ void __launch_bounds__(tc_threads<EPI, PAIR, F8>(), 1)
     // ---------------------------------------------------------------- epilogue
     const int q = warp & 3;  // TMEM lane quarter this warp may access
     const int ew = warp - 2;  // epilogue warp index (its staging tile)
-    // with 8 epilogue warps the two warps of a quarter take alternate 16-row chunks
-    const int cfirst = 16 * (ew >> 2), cstep = 16 * (NEPI / 4);
+    // SPLITB (down tiles with two feature blocks, 8 warps): the two warps of a quarter
+    // take one feature block each over all chunks, and share the quarter's row data.
+    // Otherwise the NEPI / 4 warps of a quarter take alternate 16-row chunks.
+    constexpr bool SPLITB = DUAL && NEPI == 8;
+    const int blk = SPLITB ? (ew >> 2) : 0;
+    const int cfirst = SPLITB ? 0 : 16 * (ew >> 2), cstep = SPLITB ? 16 : 16 * (NEPI / 4);
     int acc = 0;
     uint32_t acc_phase = 0;
-    for (int w = walker; w < total; w += walkers) {
+    for (int r = 0, w = walker; w < total; ++r, w = walk_tile(r, walker, walkers)) {
       TileInfo ti;
       decode_tile<BN, BKE, TILE_M>(p, sched, G, w, ti);
       const GemmClass& c = p.cls[ti.cls];
@@ -883,8 +989,11 @@ __global__ void __launch_bounds__(tc_threads<EPI, PAIR, F8>(), 1)
       const float sa0 = (F8 && fvalid) ? c.a0_scale[ti.a_row + (int)rank * TC_BM + q * 32 + lane] : 1.f;
       const float sa1 = (F8 && MATS == 2 && fvalid) ? c.a1_scale[ti.a_row + (int)rank * TC_BM + q * 32 + lane] : 1.f;
       // Row data of the whole tile (gate weight, destination token), fetched into this
-      // warp's shared-memory slice before waiting for the accumulator so the loads
-      // overlap the MMAs; the chunk loop below then reads it with broadcasts.
+      // quarter's shared-memory slice before waiting for the accumulator so the loads
+      // overlap the MMAs; the chunk loop below then reads it with broadcasts. SPLITB:
+      // both warps of the quarter write the same values, after both finished reading
+      // the previous tile's.
+      if (SPLITB) quarter_bar(q);
       if (EPI == EPI_DOWN) {
         for (int j = lane; j < BN; j += 32) {
           const RowAux a = load_row_aux<EPI>(c, ti, j);
@@ -901,63 +1010,96 @@ __global__ void __launch_bounds__(tc_threads<EPI, PAIR, F8>(), 1)
       if (!got) {
         set_status(p.status, MOE_ERR_TIMEOUT);
         abort_s = 1;
-        break;
+        if (!SPLITB) break;
+        qfail_s[q] = 1;
+      }
+      if (SPLITB) {  // both warps of the quarter leave together or go on together
+        quarter_bar(q);
+        if (qfail_s[q]) break;
       }
       tc_fence_after();
-      const uint32_t t_row = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * S::ACC_COLS);
+      // (SPLITB: the columns of this warp's feature block)
+      const uint32_t t_row =
+          tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * S::ACC_COLS + (SPLITB ? blk * BN : 0));
       // One 16-row chunk of accumulator columns (r0: gate or the single matrix, r1: up).
       auto chunk = [&](const int c0, const uint32_t (&r0)[16], const uint32_t (&r1)[16]) {
         const int jn = min(16, ti.rows_in_tile - c0);
+        // DOWN: the chunk's 16 row weights, read once for both feature blocks
+        float wrow[16];
+        if constexpr (EPI == EPI_DOWN) {
+#pragma unroll
+          for (int j = 0; j < 16; ++j) wrow[j] = aux_w[q][c0 + j];
+        }
         // activation of 16 rows x this warp's 32 features, staged, then stored as
         // 16-byte vectors along the feature axis from feature fbase on
         auto emit = [&](const uint32_t (&ra)[16], const uint32_t (&rb)[16], const int fbase) {
+          if constexpr (STG16) {
 #pragma unroll
-          for (int j = 0; j < 16; ++j) {
-            float v0 = has_k ? __uint_as_float(ra[j]) : 0.f;
-            float v1 = (MATS == 2 && !DUAL && has_k) ? __uint_as_float(rb[j]) : 0.f;
-            if (F8) {
-              const float sb = EPI == EPI_DOWN ? 1.f : aux_s[q][c0 + j];
-              v0 = v0 * sa0 * sb;
-              v1 = v1 * sa1 * sb;
+            for (int j = 0; j < 16; ++j) {
+              float v0 = has_k ? __uint_as_float(ra[j]) : 0.f;
+              float v1 = (MATS == 2 && has_k) ? __uint_as_float(rb[j]) : 0.f;
+              if (F8) {
+                const float sb = aux_s[q][c0 + j];
+                v0 = v0 * sa0 * sb;
+                v1 = v1 * sa1 * sb;
+              }
+              stg16[ew][j][lane] = __float2bfloat16_rn(EPI == EPI_SWIGLU ? silu_mul(v0, v1) : fmaxf(v0, 0.f));
             }
-            // SiLU's quotient by the fast division (2 ulp; h is stored in bf16)
-            stg[ew][j][lane] = EPI == EPI_SWIGLU ? __fdividef(v0, 1.f + __expf(-v0)) * v1
-                              : EPI == EPI_RELU ? fmaxf(v0, 0.f)
-                                                : v0 * aux_w[q][c0 + j];
-          }
-          __syncwarp();
-          if (EPI == EPI_DOWN && !c.scatter_k1) {  // fp32 partial rows: 8 float4 per row
-            float* o = reinterpret_cast<float*>(c.out) + (long long)ti.ks * c.out_split_stride + fbase;
-#pragma unroll
-            for (int i = 0; i < 4; ++i) {
-              const int idx = lane + 32 * i, jj = idx >> 3, part = idx & 7;
-              if (jj < jn && fbase + part * 4 < c.R)
-                *reinterpret_cast<float4*>(o + (long long)(ti.out_row + c0 + jj) * c.out_ld + part * 4) =
-                    *reinterpret_cast<const float4*>(&stg[ew][jj][part * 4]);
-            }
-          } else {  // bf16 rows (h, or the layer output with the top-1 combine fused): 4 x 8 per row
-            __nv_bfloat16* o = reinterpret_cast<__nv_bfloat16*>(c.out) + fbase;
+            __syncwarp();
+            __nv_bfloat16* o = reinterpret_cast<__nv_bfloat16*>(c.out) + fbase;  // bf16 rows of h: 4 x 8 per row
 #pragma unroll
             for (int i = 0; i < 2; ++i) {
               const int idx = lane + 32 * i, jj = idx >> 2, part = idx & 3;
-              const long long orow = EPI == EPI_DOWN ? (long long)aux_d[q][c0 + jj] : (long long)ti.out_row + c0 + jj;
-              if (jj < jn && fbase + part * 8 < c.R && orow >= 0) {
-                const float* v = &stg[ew][jj][part * 8];
-                uint4 pk;
-                pk.x = pack_bf16x2(v[0], v[1]);
-                pk.y = pack_bf16x2(v[2], v[3]);
-                pk.z = pack_bf16x2(v[4], v[5]);
-                pk.w = pack_bf16x2(v[6], v[7]);
-                *reinterpret_cast<uint4*>(o + orow * c.out_ld + part * 8) = pk;
+              if (jj < jn && fbase + part * 8 < c.R)
+                *reinterpret_cast<uint4*>(o + ((long long)ti.out_row + c0 + jj) * c.out_ld + part * 8) =
+                    *reinterpret_cast<const uint4*>(&stg16[ew][jj][part * 8]);
+            }
+            __syncwarp();
+          } else if constexpr (EPI == EPI_DOWN) {
+            // rows weighted by their task's gate weight, in two passes of 8 rows
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+#pragma unroll
+              for (int j = 0; j < 8; ++j) {
+                const float v0 = has_k ? __uint_as_float(ra[8 * h + j]) * (F8 ? sa0 : 1.f) : 0.f;
+                stg[ew][j][lane] = v0 * wrow[8 * h + j];
               }
+              __syncwarp();
+              if (!c.scatter_k1) {  // fp32 partial rows: 8 float4 per row
+                float* o = reinterpret_cast<float*>(c.out) + (long long)ti.ks * c.out_split_stride + fbase;
+#pragma unroll
+                for (int i = 0; i < 2; ++i) {
+                  const int idx = lane + 32 * i, jj = idx >> 3, part = idx & 7;
+                  if (8 * h + jj < jn && fbase + part * 4 < c.R)
+                    *reinterpret_cast<float4*>(o + (long long)(ti.out_row + c0 + 8 * h + jj) * c.out_ld + part * 4) =
+                        *reinterpret_cast<const float4*>(&stg[ew][jj][part * 4]);
+                }
+              } else {  // bf16 rows of the layer output with the top-1 combine fused: 4 x 8 per row
+                __nv_bfloat16* o = reinterpret_cast<__nv_bfloat16*>(c.out) + fbase;
+                const int jj = lane >> 2, part = lane & 3;
+                const long long orow = (long long)aux_d[q][c0 + 8 * h + jj];
+                if (8 * h + jj < jn && fbase + part * 8 < c.R && orow >= 0) {
+                  const float* v = &stg[ew][jj][part * 8];
+                  uint4 pk;
+                  pk.x = pack_bf16x2(v[0], v[1]);
+                  pk.y = pack_bf16x2(v[2], v[3]);
+                  pk.z = pack_bf16x2(v[4], v[5]);
+                  pk.w = pack_bf16x2(v[6], v[7]);
+                  *reinterpret_cast<uint4*>(o + orow * c.out_ld + part * 8) = pk;
+                }
+              }
+              __syncwarp();
             }
           }
-          __syncwarp();
         };
         if (VEC) {
           const int fbase = fcta + q * 32;  // first feature of this warp (R is a multiple of 8)
-          emit(r0, r1, fbase);
-          if (DUAL) emit(r1, r1, fbase + S::TILE_M);  // the second feature block
+          if (SPLITB) {
+            emit(r0, r0, fbase + blk * S::TILE_M);  // this warp's feature block
+          } else {
+            emit(r0, r1, fbase);
+            if (DUAL) emit(r1, r1, fbase + S::TILE_M);  // the second feature block
+          }
         } else if (fvalid) {  // LOGITS
 #pragma unroll
           for (int j = 0; j < 16; ++j)
@@ -965,39 +1107,53 @@ __global__ void __launch_bounds__(tc_threads<EPI, PAIR, F8>(), 1)
         }
         __syncwarp();
       };
+      // The accumulator goes back to the MMA issuer as soon as this warp's last TMEM
+      // load has landed in registers: its last chunk is computed and stored while the
+      // next tile's MMAs already run (with one accumulator, as for the SwiGLU pair
+      // tiles, this is the only overlap of epilogue and MMAs). Called exactly once per
+      // tile by every epilogue warp.
+      auto release_acc = [&]() {
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) {
+          if (PAIR && !leader)  // the leader's MMA waits for both CTAs' epilogues
+            mbar_arrive_cluster_relaxed(mapa_shared(smem_u32(&acce_bar[acc]), 0));
+          else
+            mbar_arrive_relaxed(&acce_bar[acc]);
+        }
+      };
       // The loads of chunk i + 1 are in flight while chunk i is computed and stored
       // (two register buffers; the loop body takes the even chunk, then the odd one).
       const int rows = ti.rows_in_tile;
+      constexpr bool LD2 = MATS == 2 && !SPLITB;  // both matrices' (or blocks') columns
       uint32_t ra0[16], ra1[16], rb0[16], rb1[16];
 #pragma unroll
       for (int j = 0; j < 16; ++j) ra1[j] = rb1[j] = 0u;
       if (cfirst < rows) {
         tmem_ld_x16(t_row + cfirst, ra0);
-        if (MATS == 2) tmem_ld_x16(t_row + BN + cfirst, ra1);
+        if (LD2) tmem_ld_x16(t_row + BN + cfirst, ra1);
+      } else {
+        release_acc();
       }
 #pragma unroll 1
       for (int c0 = cfirst; c0 < rows; c0 += 2 * cstep) {
-        if (MATS == 2) tmem_ld_wait_keep(ra0, ra1); else tmem_ld_wait_keep(ra0);
+        if (LD2) tmem_ld_wait_keep(ra0, ra1); else tmem_ld_wait_keep(ra0);
         if (c0 + cstep < rows) {
           tmem_ld_x16(t_row + c0 + cstep, rb0);
-          if (MATS == 2) tmem_ld_x16(t_row + BN + c0 + cstep, rb1);
+          if (LD2) tmem_ld_x16(t_row + BN + c0 + cstep, rb1);
+        } else {
+          release_acc();
         }
         chunk(c0, ra0, ra1);
         if (c0 + cstep >= rows) break;
-        if (MATS == 2) tmem_ld_wait_keep(rb0, rb1); else tmem_ld_wait_keep(rb0);
+        if (LD2) tmem_ld_wait_keep(rb0, rb1); else tmem_ld_wait_keep(rb0);
         if (c0 + 2 * cstep < rows) {
           tmem_ld_x16(t_row + c0 + 2 * cstep, ra0);
-          if (MATS == 2) tmem_ld_x16(t_row + BN + c0 + 2 * cstep, ra1);
+          if (LD2) tmem_ld_x16(t_row + BN + c0 + 2 * cstep, ra1);
+        } else {
+          release_acc();
         }
         chunk(c0 + cstep, rb0, rb1);
-      }
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) {
-        if (PAIR && !leader)  // the leader's MMA waits for both CTAs' epilogues
-          mbar_arrive_cluster(mapa_shared(smem_u32(&acce_bar[acc]), 0));
-        else
-          mbar_arrive(&acce_bar[acc]);
       }
       if (++acc == S::NUM_ACC) {
         acc = 0;
@@ -1079,7 +1235,7 @@ static cudaError_t launch_impl(const TcMaps& maps, const GemmParams& p, int num_
     // free SMs leaves one SM out)
     static int max_pairs = 0;
     cudaLaunchConfig_t cfg = {};
-    cfg.blockDim = dim3(tc_threads<EPI, PAIR, F8>());
+    cfg.blockDim = dim3(tc_threads<EPI, PAIR, F8, MATS>());
     cfg.dynamicSmemBytes = S::DYN_SMEM;
     cfg.stream = s;
     cudaLaunchAttribute attr[2];
@@ -1106,7 +1262,7 @@ static cudaError_t launch_impl(const TcMaps& maps, const GemmParams& p, int num_
     if (e != cudaSuccess) return e;
     return cudaGetLastError();
   }
-  launch_k(kern, num_ctas, tc_threads<EPI, PAIR, F8>(), S::DYN_SMEM, s, m[0], m[1], m[2], m[3], m[4], m[5], p);
+  launch_k(kern, num_ctas, tc_threads<EPI, PAIR, F8, MATS>(), S::DYN_SMEM, s, m[0], m[1], m[2], m[3], m[4], m[5], p);
   count_launch();
   return cudaGetLastError();
 }
