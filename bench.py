@@ -412,8 +412,9 @@ def _down_ksplit(cfg, cfg_groups, fp8: bool) -> int:
     """The library's static down-projection K split (mirrors its planner; it only
     enters the byte count of the fp32 partial outputs)."""
     plan_ksplit = 1
-    if cfg.dtype == W.BF16 and cfg.n_shared == 0:
-        avg = cfg.T * cfg.k / cfg_groups.m
+    avg = cfg.T * cfg.k / cfg_groups.m
+    pair = cfg.dtype == W.BF16 and avg > 128  # the library's pair-tile rule (no K split)
+    if cfg.dtype == W.BF16 and cfg.n_shared == 0 and not pair:
         bn, cap = 16, (256 if avg >= 256 else 128)  # the library's down-projection tile rule
         while bn < cap and bn < 2.0 * avg:
             bn <<= 1

@@ -468,8 +468,12 @@ static moe_status_t run_ffn(const moe_config_t& c, const Plan& pl, const FfnIo& 
   }
   dn.n_classes = ncls;
   // pair tiles of the down projection take two 256-row feature blocks per token tile
-  // when d covers them
-  const int epi_dn = pair && c.d >= 512 ? EPI_DOWN_DUAL : EPI_DOWN;
+  // when d covers them and segments average 256+ rows (long K loops per tile, where
+  // staging the token rows once for twice the MMA work keeps shared memory below its
+  // limit); shorter segments keep one block per tile: twice the tiles to spread over
+  // the pairs, and two accumulators, so the epilogue overlaps the next tile
+  const bool long_segments = (double)c.T * c.k / c.m >= 256.0;
+  const int epi_dn = pair && c.d >= 512 && long_segments ? EPI_DOWN_DUAL : EPI_DOWN;
   if (tc)
     return cuda_status(launch_tc_gemm(epi_dn, pair ? 256 : pl.bn_down, md, dn, num_sms(), s, q8 != nullptr, pair));
   return cuda_status(launch_simt_gemm(EPI_DOWN, c.dtype, dn, (int)std::min<long long>(io.routed_rows, 1LL << 30), s));

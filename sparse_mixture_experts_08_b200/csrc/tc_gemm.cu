@@ -1284,10 +1284,13 @@ int tc_pick_bn(int epi, double avg) {
 }
 
 // Pair tiles (256 weight rows over two SMs, up to 256 token rows) when the mean
-// segment fills a 256-row token tile: then each SM reads half the operand bytes per
-// MMA that a one-SM 128-row tile reads, and shared-memory bandwidth stops bounding
-// the tensor pipe (Mixtral-shaped prefill: 1024 rows per expert on average).
-bool tc_pick_pair(double avg) { return avg >= 256.0; }
+// segment is longer than the 128 token rows a one-SM tile takes. A one-SM tile then
+// needs two or more token tiles per expert, each streaming the expert's weights again,
+// where a pair tile covers up to 256 rows with one pass; and for long segments each
+// SM reads half the operand bytes per MMA, so shared-memory bandwidth stops bounding
+// the tensor pipe (Mixtral-shaped prefill: 1024 rows per expert on average;
+// DeepSeek-V2-Lite-shaped: 192).
+bool tc_pick_pair(double avg) { return avg > 128.0; }
 
 cudaError_t launch_tc_gemm(int epi, int bn, const TcMaps& maps, const GemmParams& p, int num_ctas,
                            cudaStream_t s, bool f8, bool pair) {
