@@ -318,12 +318,16 @@ __device__ __forceinline__ void epi_bar() {
 
 // One pass of the router epilogue over a token's m logits (TMEM columns, 32 per
 // step): the largest logit strictly after (pv, pe) in the order (logit desc,
-// expert asc), by a pairwise tree whose left side always holds the lower experts.
-// With EXP it also writes the logits (lg, when given) and folds the softmax
-// denominator: per 32 columns a pairwise fp32 sum of exp(logit - running max),
-// added to an fp64 sum rescaled whenever the running maximum grows. A pass covers
-// the columns [c_lo, c_hi) (multiples of 32); the two threads of a token take the
-// lower and the upper half of the experts.
+// expert asc). Per 32 columns a pairwise max tree gives the largest remaining
+// logit and a bitmask of the columns equal to it gives the lowest expert holding
+// it (a tree carrying (logit, expert) pairs through conditional swaps cost about
+// three times as much). With EXP (the first pass: nothing picked yet, so "after"
+// means "not NaN") it also writes the logits (lg, when given) and folds the
+// softmax denominator: per 32 columns a pairwise fp32 sum of exp(logit - running
+// max), added to an fp64 sum rescaled whenever the running maximum grows; that
+// maximum is the pick's (the max tree ignores NaN just as fmaxf does). A pass
+// covers the columns [c_lo, c_hi) (multiples of 32); the two threads of a token
+// take the lower and the upper half of the experts.
 template <bool EXP>
 __device__ __forceinline__ void route_pass(uint32_t t_row, int c_lo, int c_hi, int m, const float* rbias, float pv,
                                            int pe, float& bv, int& be, float& mrun, double& z, float* lg) {
@@ -355,37 +359,30 @@ __device__ __forceinline__ void route_pass(uint32_t t_row, int c_lo, int c_hi, i
 #pragma unroll
       for (int j = 0; j < 32; ++j)
         if (c0 + j < m) lg[c0 + j] = v[j];
-    float cv[32];
-    int ce[32];
+    float cv[32], mt[32];
 #pragma unroll
     for (int j = 0; j < 32; ++j) {
-      const bool after = v[j] < pv || (v[j] == pv && c0 + j > pe);
+      const bool after = EXP ? v[j] == v[j] : (v[j] < pv || (v[j] == pv && c0 + j > pe));
       cv[j] = after ? v[j] : -INFINITY;
-      ce[j] = c0 + j;
+      mt[j] = cv[j];
     }
 #pragma unroll
     for (int st = 1; st < 32; st <<= 1)
 #pragma unroll
-      for (int j = 0; j < 32; j += 2 * st)
-        if (cv[j + st] > cv[j]) {  // an equal logit keeps the lower expert (left)
-          cv[j] = cv[j + st];
-          ce[j] = ce[j + st];
-        }
-    if (cv[0] > bv) {  // earlier steps hold lower experts
-      bv = cv[0];
-      be = ce[0];
+      for (int j = 0; j < 32; j += 2 * st) mt[j] = fmaxf(mt[j], mt[j + st]);
+    const float mx = mt[0];
+    uint32_t tie = 0u;
+#pragma unroll
+    for (int j = 0; j < 32; ++j) tie |= (cv[j] == mx ? 1u : 0u) << j;
+    if (mx > bv) {  // earlier steps hold lower experts; an all -inf step changes nothing
+      bv = mx;
+      be = c0 + __ffs(tie) - 1;
     }
     if (EXP) {
       float mxs[32];
-#pragma unroll
-      for (int j = 0; j < 32; ++j) mxs[j] = v[j];
-#pragma unroll
-      for (int st = 1; st < 32; st <<= 1)
-#pragma unroll
-        for (int j = 0; j < 32; j += 2 * st) mxs[j] = fmaxf(mxs[j], mxs[j + st]);
-      if (mxs[0] > mrun) {
-        z *= (double)expf(mrun - mxs[0]);
-        mrun = mxs[0];
+      if (mx > mrun) {
+        z *= (double)expf(mrun - mx);
+        mrun = mx;
       }
 #pragma unroll
       for (int j = 0; j < 32; ++j) mxs[j] = c0 + j < m ? expf(v[j] - mrun) : 0.f;
