@@ -431,6 +431,18 @@ def _down_ksplit(cfg, cfg_groups, fp8: bool) -> int:
     return plan_ksplit
 
 
+def sustained_applies(K: int, ms: float, clocks) -> bool:
+    """The sustained tensor peak (a seconds-long GEMM loop under the power cap) is the
+    denominator when the timed region is itself seconds long, or when the GPU sat under
+    its power cap for it (median SM clock below 90% of max with sw_power_cap active):
+    the burst peak was measured at full clock."""
+    if K * ms > 1000.0:
+        return True
+    c = clocks or {}
+    med, mx = c.get("sm_mhz"), c.get("sm_max_mhz")
+    return bool(med and mx and "sw_power_cap" in (c.get("reasons") or []) and med < 0.9 * mx)
+
+
 def roofline_for(cfg, stage: str, fl: float, by: float, dom_ms: float, pk: dict, pk_src: str, long_step: bool,
                  fp8: bool, traffic_key: str) -> dict:
     """Roofline object of one kernel: algorithmic flops / bytes per launch over its
@@ -449,6 +461,8 @@ def roofline_for(cfg, stage: str, fl: float, by: float, dom_ms: float, pk: dict,
                                + (" x 2 (nominal fp8 / bf16 dense ratio)" if fp8 else ""))
         roof["frac_of_nominal_dense"] = roof["achieved"] / nominal
         roof["nominal_dense_tflops"] = nominal
+        if long_step:  # the burst figure beside it
+            roof["frac_of_burst"] = roof["achieved"] / (pk["bf16_tflops"] * (2.0 if fp8 else 1.0))
     else:
         roof = {"bound": "hbm", "achieved": by / sec / 1e9, "peak": pk["hbm_gbs"], "unit": "GB/s",
                 "peak_source": f"{pk_src} hbm copy"}
@@ -700,7 +714,7 @@ def workload_summary(cfg, r: dict, world: int) -> dict:
     roofline, stage breakdown, routing statistics and clocks."""
     pk, pk_src = peaks()
     ms = r["ms_local"]
-    long_step = r["K"] * ms > 1000.0
+    long_step = sustained_applies(r["K"], ms, r.get("clocks"))
     fl, by = r["costs"][r["dom"]]
     roof = roofline_for(cfg, r["dom"], fl, by, r["dom_ms"], pk, pk_src, long_step, r["fp8"],
                         cfg.name + ("_fp8" if r["fp8"] else ""))
@@ -737,7 +751,7 @@ def ours(args):
     ms, e2e_ms = max_over_ranks([r["ms_local"], r["e2e"]["ms_local"]], dist, dev)
     K = r["K"]
     pk, pk_src = peaks()
-    long_step = K * ms > 1000.0
+    long_step = sustained_applies(K, ms, r.get("clocks"))
     fl, by = r["costs"][r["dom"]]
     roof = roofline_for(cfg, r["dom"], fl, by, r["dom_ms"], pk, pk_src, long_step, fp8,
                         cfg.name + ("_fp8" if fp8 else "") + ("_floe" if floe is not None else "")
