@@ -218,11 +218,6 @@ cudaError_t launch_router_logits(const moe_config_t& c, const void* x, const voi
   return launch_tc_gemm(EPI_LOGITS, bn, maps, p, ctas, s);
 }
 
-static moe_status_t run_router(const moe_config_t& c, const void* x, const void* w_r, const float* bias, float* logits,
-                               int* status, cudaStream_t s) {
-  return cuda_status(launch_router_logits(c, x, w_r, bias, logits, status, s));
-}
-
 // Everything moe_route computes on the device: logits (from x, or logits_in
 // verbatim), top-k ids and gate weights, by the kernels that suit the batch.
 // logits_out receives the logits when given; otherwise logits_scratch holds them
