@@ -273,66 +273,90 @@ cudaError_t launch_small_route(int T, int d, int m, int k, int renorm, const voi
 }
 
 // ------------------------------------------------------------------ top-k + softmax
-// One warp per token. k rounds of a warp arg-max over the not-yet-chosen
-// experts, ordered by (logit desc, expert index asc). Gate weights: softmax over
-// all m logits (exp in fp32 of l - max, sum in fp64), renormalised over the k
-// chosen when requested.
+// One warp per token; lane l holds the logits of experts l, l + 32, ... (NI of
+// them, in registers). k rounds of a warp arg-max over the not-yet-chosen experts,
+// ordered by (logit desc, expert index asc): each lane's best candidate, then the
+// warp's largest logit by one redux on an order-preserving 32-bit code of it, then
+// the lowest expert holding that logit by a second redux; the winner's lane marks
+// it taken. (A NaN logit codes below -inf, so it is picked only when nothing else
+// is left.) Gate weights: softmax over all m logits (exp in fp32 of l - max, the
+// per-lane fp64 sums in expert order, then a fixed xor tree), renormalised over the
+// k chosen when requested, their sum taken in pick order.
+__device__ __forceinline__ uint32_t order_code(float v) {
+  const uint32_t b = __float_as_uint(v == 0.f ? 0.f : v);  // -0 and +0 compare equal: one code
+  if (v != v) return 0u;
+  return (b & 0x80000000u) ? ~b : (b | 0x80000000u);
+}
+
+template <int NI>
 __global__ void topk_softmax_kernel(int T, int m, int k, int renorm, const float* __restrict__ logits,
                                     int32_t* __restrict__ idx, float* __restrict__ w) {
-  __shared__ int s_sel[TOPK_WARPS][32];
-  __shared__ float s_val[TOPK_WARPS][32];
   pdl_launch_dependents();
   pdl_wait();
   const int lane = threadIdx.x & 31, wib = threadIdx.x >> 5;
   const int t = blockIdx.x * TOPK_WARPS + wib;
-  if (t >= T) return;
+  if (t >= T) return;  // uniform across the warp
   const float* L = logits + (long long)t * m;
-  for (int s = 0; s < k; ++s) {
-    float bv = -FLT_MAX;
+  float v[NI];
+#pragma unroll
+  for (int i = 0; i < NI; ++i) v[i] = lane + 32 * i < m ? L[lane + 32 * i] : 0.f;
+  uint32_t taken = 0u;  // bit i: expert lane + 32 i chosen already
+  int my_e = -1;        // lane s < k: the s-th pick
+  float my_v = 0.f;
+  float mx = 0.f;
+  for (int s2 = 0; s2 < k; ++s2) {
+    uint32_t bc = 0u;
     int be = 0x7fffffff;
-    for (int e = lane; e < m; e += 32) {
-      bool taken = false;
-      for (int j = 0; j < s; ++j) taken |= (s_sel[wib][j] == e);
-      if (taken) continue;
-      const float v = L[e];
-      if (be == 0x7fffffff || v > bv || (v == bv && e < be)) {
-        bv = v;
+#pragma unroll
+    for (int i = 0; i < NI; ++i) {
+      const int e = lane + 32 * i;
+      const uint32_t cd = order_code(v[i]);
+      if (e < m && !((taken >> i) & 1u) && (be == 0x7fffffff || cd > bc)) {  // ascending e: ties keep the lower
+        bc = cd;
         be = e;
       }
     }
+    const uint32_t wc = __reduce_max_sync(FULL, be == 0x7fffffff ? 0u : bc);
+    const int we = (int)__reduce_min_sync(FULL, (be != 0x7fffffff && bc == wc) ? (uint32_t)be : 0x7fffffffu);
+    // the winner's logit, from the lane that holds it
+    float mine = 0.f;
 #pragma unroll
-    for (int o = 16; o; o >>= 1) {
-      const float ov = __shfl_xor_sync(FULL, bv, o);
-      const int oe = __shfl_xor_sync(FULL, be, o);
-      if (oe != 0x7fffffff && (be == 0x7fffffff || ov > bv || (ov == bv && oe < be))) {
-        bv = ov;
-        be = oe;
-      }
+    for (int i = 0; i < NI; ++i)
+      if (lane + 32 * i == we) mine = v[i];
+    const float pick = __shfl_sync(FULL, mine, we & 31);
+    if ((we & 31) == lane) taken |= 1u << (we >> 5);
+    if (lane == s2) {
+      my_e = we;
+      my_v = pick;
     }
-    if (lane == 0) {
-      s_sel[wib][s] = be;
-      s_val[wib][s] = bv;
-    }
-    __syncwarp();
+    if (s2 == 0) mx = pick;
   }
-  const float mx = s_val[wib][0];
   double z = 0.0;
-  for (int e = lane; e < m; e += 32) z += (double)expf(L[e] - mx);
+#pragma unroll
+  for (int i = 0; i < NI; ++i)
+    if (lane + 32 * i < m) z += (double)expf(v[i] - mx);
 #pragma unroll
   for (int o = 16; o; o >>= 1) z += __shfl_xor_sync(FULL, z, o);
+  double p = lane < k ? (double)expf(my_v - mx) / z : 0.0;
   double sel = 0.0;
-  for (int s = 0; s < k; ++s) sel += (double)expf(s_val[wib][s] - mx) / z;
+  for (int s2 = 0; s2 < k; ++s2) sel += __shfl_sync(FULL, p, s2);
   if (lane < k) {
-    double p = (double)expf(s_val[wib][lane] - mx) / z;
     if (renorm) p /= sel;
-    idx[(long long)t * k + lane] = s_sel[wib][lane];
+    idx[(long long)t * k + lane] = my_e;
     w[(long long)t * k + lane] = (float)p;
   }
 }
 
 cudaError_t launch_topk_softmax(int T, int m, int k, int renorm, const float* logits, int32_t* idx, float* w,
                                 cudaStream_t s) {
-  launch_k(topk_softmax_kernel, (T + TOPK_WARPS - 1) / TOPK_WARPS, TOPK_WARPS * 32, 0, s, T, m, k, renorm, logits, idx, w);
+  const int blocks = (T + TOPK_WARPS - 1) / TOPK_WARPS, threads = TOPK_WARPS * 32;
+  if (m > 1024 || k > 32 || k > m) return cudaErrorInvalidValue;
+  if (m <= 64)
+    launch_k(topk_softmax_kernel<2>, blocks, threads, 0, s, T, m, k, renorm, logits, idx, w);
+  else if (m <= 256)
+    launch_k(topk_softmax_kernel<8>, blocks, threads, 0, s, T, m, k, renorm, logits, idx, w);
+  else
+    launch_k(topk_softmax_kernel<32>, blocks, threads, 0, s, T, m, k, renorm, logits, idx, w);
   count_launch();
   return cudaGetLastError();
 }

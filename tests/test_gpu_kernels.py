@@ -93,6 +93,31 @@ def test_route_logits_in_verbatim_with_ties():
     np.testing.assert_allclose(w, ow, rtol=GATE_RTOL)
 
 
+@pytest.mark.parametrize("m,k", [(64, 6), (300, 17), (1024, 32)])
+def test_route_logits_in_wide_rows_ties_signed_zeros_and_infinities(m, k):
+    # the top-k kernel's register layouts (2, 8 and 32 logits per lane), heavy ties,
+    # -0 against +0 (equal: the lower expert first), -inf logits and whole rows of them
+    T = 67
+    cfg = W.small_moe(T=T, d=64, f=64, m=m, k=k, dtype=W.BF16)
+    rng = np.random.default_rng(m + k)
+    lg_in = (rng.integers(-3, 4, size=(T, m)) * 0.25).astype(np.float32)
+    lg_in[rng.random((T, m)) < 0.2] = -np.inf
+    zeros = rng.random((T, m)) < 0.3
+    lg_in[zeros] = np.where(rng.random(int(zeros.sum())) < 0.5, -0.0, 0.0).astype(np.float32)
+    lg_in[1] = -0.0
+    lg_in[2, : m // 2] = 0.0
+    lg_in[2, m // 2:] = -0.0
+    lg_in[3] = -np.inf
+    lg_in[3, m - 1] = 1.0
+    lg, idx, w = _route(cfg, {}, logits_in=dev(lg_in))
+    np.testing.assert_array_equal(lg.view(np.uint32), lg_in.view(np.uint32))
+    oidx, ow = O.topk_softmax(lg_in, k, False)
+    np.testing.assert_array_equal(idx, oidx)
+    assert idx[1].tolist() == list(range(k)) and idx[2].tolist() == list(range(k))
+    assert idx[3, 0] == m - 1 and idx[3, 1:].tolist() == list(range(k - 1))
+    np.testing.assert_allclose(w, ow, rtol=GATE_RTOL, atol=1e-12)
+
+
 def _hist(cfg, idx_np):
     c = config_of(cfg)
     ws = moe.workspace(c)
