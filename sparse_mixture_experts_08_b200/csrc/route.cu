@@ -706,7 +706,7 @@ cudaError_t launch_route_index(int mode, int T, int k, int m, const int32_t* idx
 // ------------------------------------------------ ranks
 // One warp per task range r walks it 32 tasks at a time in increasing task id (the
 // ids of eight such steps loaded together): a task's rank among the lower lanes with
-// the same expert (a 32-step shuffle scan) plus the expert's cursor (started at
+// the same expert (one match over the warp) plus the expert's cursor (started at
 // start[r][e]) is its position pos in the stable counting sort; the group's last
 // lane advances the cursor. Writes
 // inv_perm[q] = pos, perm[pos] = q and, when given, w_perm[pos] = task_w[q] (the
@@ -742,13 +742,9 @@ __global__ void rank_kernel(int Tk, int m, int L, const int32_t* __restrict__ id
     for (int u = 0; u < 8; ++u)
       if (u == step) e = ev[u];
     if (e >= m) e = -1;
-    int rank = 0, cnt = 0;
-#pragma unroll
-    for (int j = 0; j < 32; ++j) {
-      const int ej = __shfl_sync(FULL, e, j);
-      cnt += ej == e;
-      rank += (ej == e) & (j < lane);
-    }
+    // lanes holding the same expert (tasks past the range hold -1 and match only each other)
+    const unsigned same = __match_any_sync(FULL, e);
+    const int rank = __popc(same & ((1u << lane) - 1u)), cnt = __popc(same);
     const int b = e >= 0 ? cur[e] : 0;
     __syncwarp();
     if (q < hi) {
