@@ -717,7 +717,8 @@ __global__ void rank_kernel(int Tk, int m, int L, const int32_t* __restrict__ id
                             const int32_t* __restrict__ start, const float* __restrict__ task_w,
                             int32_t* __restrict__ perm, int32_t* __restrict__ inv_perm, float* __restrict__ w_perm,
                             int* status) {
-  extern __shared__ int cur[];  // [m]
+  extern __shared__ int cur[];  // [m] cursors, then [m + 1] offsets
+  int* off_s = cur + m;
   const int lane = threadIdx.x;
   const int r = blockIdx.x;
   const int lo = r * L, hi = min(Tk, lo + L);
@@ -725,6 +726,7 @@ __global__ void rank_kernel(int Tk, int m, int L, const int32_t* __restrict__ id
   pdl_wait();
   if (status && *reinterpret_cast<volatile int*>(status) != 0) return;  // earlier device error
   for (int e = lane; e < m; e += 32) cur[e] = start[(long long)r * m + e];
+  for (int e = lane; e <= m; e += 32) off_s[e] = offsets[e];  // each step validates against them
   __syncwarp();
   int ev[8];
   for (int base = lo; base < hi; base += 32) {
@@ -749,7 +751,7 @@ __global__ void rank_kernel(int Tk, int m, int L, const int32_t* __restrict__ id
     __syncwarp();
     if (q < hi) {
       const int pos = b + rank;
-      const bool ok = e >= 0 && pos >= 0 && pos < Tk && pos >= offsets[e] && pos < offsets[e + 1];
+      const bool ok = e >= 0 && pos >= 0 && pos < Tk && pos >= off_s[e] && pos < off_s[e + 1];
       inv_perm[q] = ok ? pos : -1;
       if (ok) {
         perm[pos] = q;
@@ -768,8 +770,8 @@ cudaError_t launch_rank(int T, int k, int m, const int32_t* idx, const int32_t* 
                         cudaStream_t s) {
   int R, L;
   route_ranges(T * k, m, &R, &L);
-  launch_k(rank_kernel, R, 32, sizeof(int) * (size_t)m, s, T * k, m, L, idx, offsets, start, task_w, perm, inv_perm,
-           w_perm, status);
+  launch_k(rank_kernel, R, 32, sizeof(int) * (2 * (size_t)m + 1), s, T * k, m, L, idx, offsets, start, task_w, perm,
+           inv_perm, w_perm, status);
   count_launch();
   return cudaGetLastError();
 }
