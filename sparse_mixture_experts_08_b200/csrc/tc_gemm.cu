@@ -689,6 +689,19 @@ __global__ void __launch_bounds__(tc_threads<EPI, PAIR, F8, MATS>(), 1)
       const int n_inst = max(16, (ti.rows_in_tile + 15) & ~15);
       const int a_row = ti.a_row + (int)rank * TC_BM;
       const int b_row = ti.b_row + (int)rank * (n_inst / 2);
+      // PAIR: a CTA's 128 weight rows of a block that lie wholly past the group's rows
+      // (the last feature tile when R is not a multiple of 256) are not loaded: they
+      // belong to the next group, and the stale stage bytes left in their place feed
+      // only accumulator rows that the epilogue skips (feature >= R). The leader arms
+      // the stage barrier with the bytes both CTAs do load.
+      const int a_loc = ti.mt * TILE_M;  // the tile's first weight row within its group
+      const int a_rows = p.cls[ti.cls].R;
+      auto a_live = [&](int cta, int blk) { return a_loc + blk * S::TILE_M + cta * TC_BM < a_rows; };
+      const bool live0 = a_live((int)rank, 0), live1 = a_live((int)rank, DUAL ? 1 : 0);
+      uint32_t pair_bytes = 2 * S::B_BYTES;
+      if (PAIR)
+        for (int cta = 0; cta < 2; ++cta)
+          pair_bytes += (a_live(cta, 0) ? S::A_BYTES : 0) + (MATS == 2 && a_live(cta, DUAL ? 1 : 0) ? S::A_BYTES : 0);
       for (int kb = ti.kb0; kb < ti.kb1; ++kb) {
         if (!mbar_wait(&empty_bar[stage], phase ^ 1u, lim, abort_flag)) {
           ok = false;
@@ -698,9 +711,9 @@ __global__ void __launch_bounds__(tc_threads<EPI, PAIR, F8, MATS>(), 1)
         if (PAIR) {
           // both CTAs' copies complete on the leader's barrier, which expects them all
           const uint32_t fb = mapa_shared(smem_u32(&full_bar[stage]), 0);
-          if (leader) mbar_arrive_expect_tx(&full_bar[stage], 2 * S::STAGE_BYTES);
-          tma_load_2d_pair(mA0, fb, st, kb * BKE, a_row);
-          if (MATS == 2)
+          if (leader) mbar_arrive_expect_tx(&full_bar[stage], pair_bytes);
+          if (live0) tma_load_2d_pair(mA0, fb, st, kb * BKE, a_row);
+          if (MATS == 2 && live1)
             tma_load_2d_pair(DUAL ? mA0 : mA1, fb, st + S::A_BYTES, kb * BKE, a_row + (DUAL ? S::TILE_M : 0));
           tma_load_2d_pair(mB, fb, st + MATS * S::A_BYTES, kb * BKE, b_row);
           if (leader) last_parity[stage] = (int)phase;
