@@ -49,6 +49,9 @@ ROUTE_CASES = [
     W.small_moe(T=777, d=264, f=64, m=12, k=3, dtype=W.BF16, zipf_s=1.0, index=97),
     W.small_moe(T=130, d=2048, f=64, m=16, k=16, dtype=W.BF16, zipf_s=0.5, index=98),
     W.small_moe(T=3, d=8, f=64, m=1, k=1, dtype=W.BF16, zipf_s=0.0, index=99),
+    # 17 to 64 experts: the logits GEMM then the warp top-k (one and two logits per lane)
+    W.small_moe(T=300, d=256, f=64, m=24, k=3, dtype=W.BF16, zipf_s=1.0, renorm=True, index=100),
+    W.small_moe(T=2053, d=2048, f=64, m=64, k=6, dtype=W.BF16, zipf_s=1.0, index=101),
 ]
 
 
