@@ -503,6 +503,10 @@ __global__ void __launch_bounds__(RI_THREADS, 1)
   pdl_wait();
   __syncthreads();
   const int nth = blockDim.x;
+  // a thread's tasks are q = tid + n nth; their range q / L is walked by adding
+  // (nth / L, nth % L) with one carry instead of a division per task
+  const int dq = nth / L, dl = nth - dq * L;
+  int rq = tid / L, rl = tid - rq * L;
   for (int q0 = tid; q0 < Tk; q0 += 8 * nth) {
     int ev[8];
 #pragma unroll
@@ -518,7 +522,13 @@ __global__ void __launch_bounds__(RI_THREADS, 1)
       if (e < 0 || e >= m)
         bad = 1;
       else
-        atomicAdd(&c[(q / L) * MS + e], 1);
+        atomicAdd(&c[rq * MS + e], 1);
+      rq += dq;
+      rl += dl;
+      if (rl >= L) {
+        rl -= L;
+        ++rq;
+      }
     }
   }
   __syncthreads();
@@ -613,10 +623,8 @@ __global__ void __launch_bounds__(RI_THREADS, 1)
     for (int e = tid; e <= m; e += blockDim.x) off[e] = offsets[e];
   }
   __syncthreads();
-  for (int i = tid; i < R * m; i += blockDim.x) {
-    const int r = i / m, e = i - r * m;
-    start[i] = off[e] + c[r * MS + e];
-  }
+  for (int r = warp; r < R; r += nw)  // a warp per range row, lanes along the experts
+    for (int e = lane; e < m; e += 32) start[(long long)r * m + e] = off[e] + c[r * MS + e];
 }
 
 size_t route_index_smem(int R, int m) { return sizeof(int) * ((size_t)R * (m + 1) + m + 1); }
@@ -724,25 +732,38 @@ __global__ void rank_kernel(int Tk, int m, int L, const int32_t* __restrict__ id
   const int lo = r * L, hi = min(Tk, lo + L);
   pdl_launch_dependents();
   pdl_wait();
-  if (status && *reinterpret_cast<volatile int*>(status) != 0) return;  // earlier device error
+  // an earlier device error stops the kernel; its status word is read in the same batch
+  // of loads as the first eight steps' ids and gate weights, the cursors and the
+  // offsets (one round trip before the first step, none inside it; nothing is stored
+  // to global memory before the check)
+  const int prior = status ? *reinterpret_cast<volatile int*>(status) : 0;
+  int ev[8];
+  float wv[8];
+  auto load_steps = [&](int base) {
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      const int qq = base + 32 * u + lane;
+      ev[u] = qq < hi ? idx[qq] : -1;
+      wv[u] = (w_perm && qq < hi) ? task_w[qq] : 0.f;
+    }
+  };
+  load_steps(lo);
   for (int e = lane; e < m; e += 32) cur[e] = start[(long long)r * m + e];
   for (int e = lane; e <= m; e += 32) off_s[e] = offsets[e];  // each step validates against them
   __syncwarp();
-  int ev[8];
+  if (prior != 0) return;
   for (int base = lo; base < hi; base += 32) {
     const int step = ((base - lo) >> 5) & 7;
-    if (step == 0) {  // the ids of the next eight steps
-#pragma unroll
-      for (int u = 0; u < 8; ++u) {
-        const int qq = base + 32 * u + lane;
-        ev[u] = qq < hi ? idx[qq] : -1;
-      }
-    }
+    if (step == 0 && base != lo) load_steps(base);  // the ids of the next eight steps
     const int q = base + lane;
     int e = -1;
+    float tw = 0.f;
 #pragma unroll
     for (int u = 0; u < 8; ++u)
-      if (u == step) e = ev[u];
+      if (u == step) {
+        e = ev[u];
+        tw = wv[u];
+      }
     if (e >= m) e = -1;
     // lanes holding the same expert (tasks past the range hold -1 and match only each other)
     const unsigned same = __match_any_sync(FULL, e);
@@ -755,7 +776,7 @@ __global__ void rank_kernel(int Tk, int m, int L, const int32_t* __restrict__ id
       inv_perm[q] = ok ? pos : -1;
       if (ok) {
         perm[pos] = q;
-        if (w_perm) w_perm[pos] = task_w[q];
+        if (w_perm) w_perm[pos] = tw;
       } else {
         set_status(status, MOE_ERR_DEVICE_INDEX);
       }
@@ -874,14 +895,29 @@ __global__ void __launch_bounds__(RS_THREADS)
   // (nothing is read before the wait: a kernel launched early may run beside an
   // earlier kernel of the stream that is still writing x)
   pdl_wait();
+  // Item j of the block's copy is task i = j / pc of the tile (token tile * 128 + i / k)
+  // and column chunk c_lo + j % pc. A thread's items are j = tid + n * RS_THREADS, so
+  // (i, j % pc) is walked by adding (RS_THREADS / pc, RS_THREADS % pc) with one carry:
+  // no division per item (divisions were most of the kernel's instructions).
+  const unsigned upc = (unsigned)pc, uk = (unsigned)k;  // pc >= 1: parts <= chunks
+  const unsigned di = RS_THREADS / upc, dr = RS_THREADS - di * upc;
+  const unsigned wi0 = (unsigned)tid / upc, wr0 = (unsigned)tid - wi0 * upc;
+  const long long tok0 = (long long)tile * 128;
+  auto advance = [&](unsigned& i, unsigned& r) {
+    i += di;
+    r += dr;
+    if (r >= upc) {
+      r -= upc;
+      ++i;
+    }
+  };
+  auto src_row = [&](unsigned i) { return (tok0 + (uk == 1u ? i : i / uk)) * chunks; };
   int4 pre[RS_PRE];  // the row chunks, loaded together with the tables below
+  unsigned wi = wi0, wr = wr0;
 #pragma unroll
   for (int u = 0; u < RS_PRE; ++u) {
-    const int j = tid + u * RS_THREADS;
-    if (j < total) {
-      const int i = j / pc, cc = c_lo + (j - i * pc);
-      pre[u] = x[((q0 + i) / k) * chunks + cc];
-    }
+    if (tid + u * RS_THREADS < total) pre[u] = x[src_row(wi) + c_lo + wr];
+    advance(wi, wr);
   }
   if (tid == 0) prior_s = *reinterpret_cast<volatile int*>(status);
   // 1. per (group g, expert e): tasks of e in tiles g, g + G, ..., all and before this tile
@@ -1011,13 +1047,15 @@ __global__ void __launch_bounds__(RS_THREADS)
   }
   __syncthreads();
   // 4. rows: x_perm[dest, c] = x[q / k, c] for this part's columns
+  {
+    unsigned si = wi0, sr = wr0;
 #pragma unroll
-  for (int u = 0; u < RS_PRE; ++u) {
-    const int j = tid + u * RS_THREADS;
-    if (j < total) {
-      const int i = j / pc, cc = c_lo + (j - i * pc);
-      const int d = dest[i];
-      if (d >= 0) x_perm[(long long)d * chunks + cc] = pre[u];
+    for (int u = 0; u < RS_PRE; ++u) {
+      if (tid + u * RS_THREADS < total) {
+        const int d = dest[si];
+        if (d >= 0) x_perm[(long long)d * chunks + c_lo + sr] = pre[u];
+      }
+      advance(si, sr);
     }
   }
   for (int j0 = tid + RS_PRE * RS_THREADS; j0 < total; j0 += RS_PRE * RS_THREADS) {  // beyond the first batch
@@ -1025,16 +1063,15 @@ __global__ void __launch_bounds__(RS_THREADS)
     long long o[RS_PRE];
 #pragma unroll
     for (int u = 0; u < RS_PRE; ++u) {
-      const int j = j0 + u * RS_THREADS;
       o[u] = -1;
-      if (j < total) {
-        const int i = j / pc, cc = c_lo + (j - i * pc);
-        const int d = dest[i];
+      if (j0 + u * RS_THREADS < total) {
+        const int d = dest[wi];
         if (d >= 0) {
-          v[u] = x[((q0 + i) / k) * chunks + cc];
-          o[u] = (long long)d * chunks + cc;
+          v[u] = x[src_row(wi) + c_lo + wr];
+          o[u] = (long long)d * chunks + c_lo + wr;
         }
       }
+      advance(wi, wr);
     }
 #pragma unroll
     for (int u = 0; u < RS_PRE; ++u)
