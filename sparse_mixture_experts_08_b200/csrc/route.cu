@@ -272,7 +272,7 @@ __global__ void __launch_bounds__(SR_THREADS)
 // map for A and B, so every product pairs matching elements. The warps' partial
 // logits are added in warp order, then the bias; one thread per token takes the
 // top-k and gate weights as small_route_kernel does. The sums have a fixed order.
-constexpr int SRT_WARPS = 8, SRT_UNROLL = 4;
+constexpr int SRT_WARPS = 16, SRT_UNROLL = 4;
 __device__ __forceinline__ void mma_bf16_16816(float (&c)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
   asm volatile(
       "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
