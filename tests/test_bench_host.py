@@ -61,3 +61,45 @@ def test_traffic_goes_null_when_its_kernel_sources_change(tmp_path, monkeypatch)
     (csrc / "k.cu").write_text("kernel v2")              # the captured kernel changed: no figure
     assert bench.traffic_for("w", "s") is None
     assert bench.traffic_for("w", "missing") is None
+
+
+PEAKS = {"hbm_gbs": 6500.0, "bf16_tflops": 1600.0, "bf16_tflops_sustained": 1400.0}
+
+
+def test_sustained_peak_applies_to_long_or_power_capped_regions():
+    full = {"sm_mhz": 1965.0, "sm_max_mhz": 1965.0, "reasons": []}
+    capped = {"sm_mhz": 1330.0, "sm_max_mhz": 1965.0, "reasons": ["sw_power_cap"]}
+    brief_cap = {"sm_mhz": 1900.0, "sm_max_mhz": 1965.0, "reasons": ["sw_power_cap"]}
+    slow_no_reason = {"sm_mhz": 1330.0, "sm_max_mhz": 1965.0, "reasons": []}
+    assert not bench.sustained_applies(200, 2.0, full)  # 0.4 s at full clock: the burst peak
+    assert bench.sustained_applies(600, 2.0, full)  # over a second of timed steps
+    assert bench.sustained_applies(200, 2.4, capped)  # the cap held the clock down
+    assert not bench.sustained_applies(200, 2.1, brief_cap)  # capped for a moment, clock near max
+    assert not bench.sustained_applies(200, 2.1, slow_no_reason)  # no cap reason: not the cap's regime
+    assert not bench.sustained_applies(10, 2.0, None)
+
+
+def test_contraction_roofline_uses_the_peak_of_its_regime_and_dtype():
+    cfg = W.CONFIGS["mixtral"]
+    fl, by, ms = 1.924e12, 2.181e9, 1.3  # Mixtral-shaped up projection, 1.3 ms per launch
+    burst = bench.roofline_for(cfg, "expert_up", fl, by, ms, PEAKS, "measured", False, False, "none")
+    assert burst["bound"] == "tensor" and burst["peak"] == PEAKS["bf16_tflops"]
+    assert abs(burst["achieved"] - fl / 1.3e-3 / 1e12) < 1e-9
+    assert abs(burst["frac"] - burst["achieved"] / 1600.0) < 1e-12
+    assert "frac_of_burst" not in burst
+    assert abs(burst["frac_of_nominal_dense"] - burst["achieved"] / 2250.0) < 1e-12
+    sus = bench.roofline_for(cfg, "expert_up", fl, by, ms, PEAKS, "measured", True, False, "none")
+    assert sus["peak"] == PEAKS["bf16_tflops_sustained"]
+    assert abs(sus["frac_of_burst"] - burst["frac"]) < 1e-12  # the same time against the burst figure
+    f8 = bench.roofline_for(cfg, "expert_up", fl, by / 2, ms, PEAKS, "measured", False, True, "none")
+    assert f8["peak"] == 2 * PEAKS["bf16_tflops"] and f8["nominal_dense_tflops"] == 4500.0
+    assert abs(f8["frac"] - burst["frac"] / 2) < 1e-12
+
+
+def test_weight_streaming_roofline_is_bound_by_hbm():
+    cfg = W.CONFIGS["decode"]  # 16 tokens: a few flops per weight byte, far below the ridge point
+    fl, by, ms = 7.5e9, 1.88e9, 0.31
+    r = bench.roofline_for(cfg, "expert_up", fl, by, ms, PEAKS, "measured", False, False, "none")
+    assert r["bound"] == "hbm" and r["unit"] == "GB/s" and r["peak"] == PEAKS["hbm_gbs"]
+    assert abs(r["achieved"] - by / 0.31e-3 / 1e9) < 1e-6
+    assert r["traffic"] is None  # no committed capture under this key
