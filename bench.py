@@ -158,6 +158,16 @@ def cpu_oracle_fp8_sample(cfg, inp, budget_s: float):
                       f"in numpy, one process"}
 
 
+def run_config(cfg, world: int) -> dict:
+    """The `config` object both arms print for a workload: what is computed, how the job
+    is split and how the steps are timed, so the two lines describe the same run; an
+    arm's own execution details go in its other keys."""
+    return dict(workload_config(cfg), parallelism=f"data-parallel token batches x{world} (weak scaling)",
+                l2=f"GPU arm: flushed between steps ({L2_FLUSH_BYTES >> 20} MiB write, outside the timed events); "
+                   "CPU oracle arm: not applicable",
+                launch="GPU arm: eager C-ABI call per step")
+
+
 def reference_arm(args):
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
@@ -196,7 +206,8 @@ def reference_arm(args):
     line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": sec * 1e3, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "f64", "data": "synthetic (seeded generator)", "impl": "reference",
-            "config": dict(workload_config(cfg), parallelism="host threads", l2="n/a (CPU)"),
+            "config": run_config(cfg, args.gpus),
+            "execution": {"parallelism": f"one process, {threads} host threads over tokens", "l2": "n/a (CPU)"},
             "cpu_baseline": {"value": value, "unit": UNIT, "cores": threads, "kind": "oracle", "sample": sample},
             "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
@@ -775,10 +786,8 @@ def ours(args):
             "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "e4m3" if fp8 else "bf16" if cfg.dtype == W.BF16 else "f32",
             "data": "synthetic (seeded generator; x ~ N(0,1), weights ~ N(0, 1/sqrt(fan_in)), Zipf router bias)",
-            "config": dict(workload_config(cfg), **({"expert_weights": "e4m3, per-channel fp32 scales"} if fp8 else {}),
-                           parallelism=f"data-parallel token batches x{world} (weak scaling)",
-                           l2=f"flushed between steps ({L2_FLUSH_BYTES >> 20} MiB write, outside the timed events)",
-                           launch="eager C-ABI call per step"),
+            "config": dict(run_config(cfg, world),
+                           **({"expert_weights": "e4m3, per-channel fp32 scales"} if fp8 else {})),
             "roofline": roof,
             "layer_roofline": {"time_us": t_layer * 1e6, "frac": t_layer / (ms * 1e-3),
                                "flops": r["layer_flops"], "bytes": r["layer_bytes"]},

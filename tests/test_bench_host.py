@@ -103,3 +103,17 @@ def test_weight_streaming_roofline_is_bound_by_hbm():
     assert r["bound"] == "hbm" and r["unit"] == "GB/s" and r["peak"] == PEAKS["hbm_gbs"]
     assert abs(r["achieved"] - by / 0.31e-3 / 1e9) < 1e-6
     assert r["traffic"] is None  # no committed capture under this key
+
+
+def test_reference_arm_prints_the_config_of_the_gpu_arm(capsys):
+    """Both arms describe the same run in `config`, so a comparison of the two lines
+    compares like with like; the oracle's own execution goes under `execution`."""
+    import argparse
+
+    args = argparse.Namespace(config="tiny", steps=1, warmup=3, gpus=1)
+    assert bench.reference_arm(args) == 0
+    line = json.loads(capsys.readouterr().out.strip().splitlines()[-1])
+    assert line["impl"] == "reference" and line["steps"] == 1 and line["warmup"] == 3
+    assert line["config"] == bench.run_config(W.CONFIGS["tiny"], 1)
+    assert line["e2e"]["value"] == line["value"] == line["cpu_baseline"]["value"]
+    assert line["execution"]["l2"] == "n/a (CPU)"
