@@ -65,17 +65,19 @@ def err_report(got: np.ndarray, ref: np.ndarray) -> str:
             f"elementwise max |d|/(|ref| + 1e-3 rms) {elem_rel_err(got, ref):.3e}")
 
 
-def tile_cover_tokens(perm: np.ndarray, offsets: np.ndarray, k: int, tile: int = 128) -> np.ndarray:
-    """Tokens whose tasks reach every `tile`-row token tile of every expert segment
-    (the first and last row of each tile, counted from the segment start). A token
-    tile of any multiple of `tile` rows, in either projection, then holds at least
-    one checked task."""
+def tile_cover_tokens(perm: np.ndarray, offsets: np.ndarray, k: int, step: int = 16) -> np.ndarray:
+    """Tokens whose tasks sit at every `step`-th row of every expert segment (counted
+    from the segment start), and at its last row. The grouped GEMM cuts a segment into
+    token tiles whose height is a multiple of 16, so every tile of either projection
+    starts at a segment row that is a multiple of 16 and holds a checked task, whatever
+    tile height the library picked."""
     pick = set()
     for e in range(len(offsets) - 1):
         a, b = int(offsets[e]), int(offsets[e + 1])
-        for r0 in range(a, b, tile):
+        for r0 in range(a, b, step):
             pick.add(int(perm[r0]) // k)
-            pick.add(int(perm[min(b, r0 + tile) - 1]) // k)
+        if b > a:
+            pick.add(int(perm[b - 1]) // k)
     return np.array(sorted(pick), dtype=np.int32)
 
 

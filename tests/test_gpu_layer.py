@@ -55,7 +55,7 @@ def _check_layer(cfg, inp, n_sample):
     else:
         toks = np.union1d(sample_tokens(oidx, ref["counts"], cfg.T, n_sample),
                           tile_cover_tokens(operm, ref["offsets"], cfg.k)).astype(np.int32)
-        assert covered_tiles(toks, operm, ref["offsets"], cfg.k, 128)
+        assert covered_tiles(toks, operm, ref["offsets"], cfg.k, 16)
     exp = O.moe_output(cfg, inp, oidx, ow, tokens=toks)
     got = out_f64(r["out"])[toks]
     err = token_rel_err(got, exp)
