@@ -117,3 +117,18 @@ def test_reference_arm_prints_the_config_of_the_gpu_arm(capsys):
     assert line["config"] == bench.run_config(W.CONFIGS["tiny"], 1)
     assert line["e2e"]["value"] == line["value"] == line["cpu_baseline"]["value"]
     assert line["execution"]["l2"] == "n/a (CPU)"
+
+
+def test_profiles_index_lists_every_summary_and_each_gives_its_command():
+    pdir = os.path.join(ROOT, "profiles")
+    with open(os.path.join(pdir, "README.md")) as fh:
+        index = fh.read()
+    summaries = sorted(f for f in os.listdir(pdir) if f.endswith(".md") and f != "README.md")
+    for f in summaries:
+        assert f"`{f}`" in index, f"{f} is not in profiles/README.md"
+        with open(os.path.join(pdir, f)) as fh:
+            text = fh.read()
+        assert "ncu " in text and "--clock-control none" in text, f"{f} gives no ncu command"
+        assert "python bench.py" in text, f"{f} does not name the committed command it profiled"
+    for f in os.listdir(pdir):  # summaries only: no raw reports or scripts
+        assert f.endswith((".md", ".txt", ".json")), f
